@@ -1,0 +1,416 @@
+"""Benchmark of one LSA layer (indexer + sparse attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (default): Flat LSA prefill at T = 131072 -- 64-dim index keys and
+queries from the run-of-8 mixture generator (1024 components), k = 2048,
+sink 4, window 512, attention with 32 query heads over 8 KV heads,
+head_dim 128, bf16.  One step is the whole hot path over that batch:
+bucket-cache build (normalise + pool + Ward for all 256 blocks), Flat index
+of all 131072 queries, and sparse attention for all of them.
+value = prefill tokens (queries) per second, whole job.
+
+Also reported: decode us/token at T = 1,048,576 (index_decode + attention
+for 64 new tokens, batch 1), the roofline of the dominant kernel, the
+oracle's CPU time on a bounded sample, and an end-to-end number through the
+same C-ABI calls with inputs copied from pinned host memory every step and
+the output copied back.
+
+Multi-GPU: the layer does not shard here (each rank runs its own replica,
+"replicas only"); value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hierarchical_key_clustering_b200 import inputs as I  # noqa: E402
+from hierarchical_key_clustering_b200 import lsa  # noqa: E402
+from hierarchical_key_clustering_b200.layer import SparseLayer  # noqa: E402
+
+METRIC = "indexer+sparse-attn prefill tokens/s & decode us/token per layer; % roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes per listed (query, KV head, key) measured by ncu for k_attn at the
+# 128K workload (profiles/k_attn_flat_128k.md); None until captured.
+ATTN_DRAM_BYTES_PER_ROW = None
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = f"/tmp/lsa_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        med = float(np.median(sm)) if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": smax, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                             timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- workload
+
+def make_prefill_inputs(wl: dict, seed: int = 0):
+    T = wl["T"]
+    keys = I.index_keys(seed, T, wl["n_components"])
+    nq = wl["n_prefill"]
+    pos = np.arange(T - nq, T, dtype=np.int64)
+    q = I.index_queries(seed, keys, pos)
+    return keys, q, pos
+
+
+def device_qkv(nq, n_kv, hq, hkv, seed=0, dev="cuda"):
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed * 1000 + 5)
+    Q = torch.randn((nq, hq, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    K = torch.randn((n_kv, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    V = torch.randn((n_kv, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    return Q, K, V
+
+
+def attn_algorithmic_bytes(lens: np.ndarray, hq: int, hkv: int) -> int:
+    """K and V rows of every listed (query, KV head, key) + Q read + O write +
+    the lists themselves."""
+    rows = int(lens.astype(np.int64).sum())
+    return rows * hkv * 2 * 256 + len(lens) * hq * 128 * 2 * 2 + rows * 4
+
+
+def run_ours(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = I.WORKLOADS[args.workload]
+    T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
+    keys_np, q_np, pos_np = make_prefill_inputs(wl)
+    layer = SparseLayer(T, k=wl["k"], mode=wl["mode"], beam=wl.get("beam", 32), max_queries=nq, Hq=hq)
+    keys = torch.from_numpy(keys_np).to(dev)
+    qidx = torch.from_numpy(q_np).to(dev)
+    pos = torch.from_numpy(pos_np).to(dev)
+    Q, K, V = device_qkv(nq, T, hq, hkv)
+    O = torch.empty_like(Q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(times=None):
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        e0.record(st)
+        layer.build(keys)
+        e1.record(st)
+        layer.index(qidx, pos)
+        e2.record(st)
+        layer.attend(Q, K, V, O)
+        e3.record(st)
+        if times is not None:
+            times.append((e0, e1, e2, e3))
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    lens_np = layer.lens[:nq].cpu().numpy()
+
+    launches0 = lsa.lsa_launch_count()
+    clk = Clocks(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        step(times)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    barrier(world)
+    launches = lsa.lsa_launch_count() - launches0
+    per = np.array([[a.elapsed_time(b), b.elapsed_time(c), c.elapsed_time(d), a.elapsed_time(d)]
+                    for a, b, c, d in times])
+    total_ms = float(per[:, 3].sum())
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    value = world * nq * args.steps / (total_ms / 1e3)
+
+    # roofline of the dominant kernel (attention: one k_attn launch per step)
+    pk = peaks()
+    attn_ms = float(per[:, 2].mean())
+    abytes = attn_algorithmic_bytes(lens_np, hq, hkv)
+    achieved = abytes / (attn_ms / 1e3) / 1e9
+    traffic = None
+    if ATTN_DRAM_BYTES_PER_ROW is not None:
+        traffic = int(ATTN_DRAM_BYTES_PER_ROW * int(lens_np.sum()) * hkv)
+    roofline = {"kernel": "k_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
+                "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
+                "peak_source": pk["src"], "algorithmic_bytes": abytes}
+
+    # end to end: same calls, inputs from pinned host memory, output back to host
+    e2e = run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
+
+    decode = None
+    if not args.no_decode:
+        del Q, K, V, O, flush
+        torch.cuda.empty_cache()
+        decode = run_decode(args, dev)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "T": T, "queries": nq, "k": wl["k"], "sink": 4, "window": 512,
+                   "mode": wl["mode"], "Hq": hq, "Hkv": hkv, "head_dim": 128, "index_dim": 64,
+                   "mixture_components": wl["n_components"], "parallelism": "replicas",
+                   "l2": "256 MiB buffer written between timed steps; Q/K/V (1.6 GB) exceed L2"},
+        "breakdown_ms": {"build": round(float(per[:, 0].mean()), 3), "index": round(float(per[:, 1].mean()), 3),
+                         "attention": round(attn_ms, 3)},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "decode": decode,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, dev, world):
+    st = torch.cuda.current_stream()
+    pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+    h_keys, h_q, h_pos = pin(keys_np), pin(q_np), pin(pos_np)
+    h_Q, h_K, h_V = Qd.cpu().pin_memory(), Kd.cpu().pin_memory(), Vd.cpu().pin_memory()
+    h_O = torch.empty(Qd.shape, dtype=Qd.dtype).pin_memory()
+    d_keys, d_q, d_pos = torch.empty_like(h_keys, device=dev), torch.empty_like(h_q, device=dev), \
+        torch.empty_like(h_pos, device=dev)
+    d_Q, d_K, d_V = torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd)
+    d_O = torch.empty_like(Qd)
+    h2d = sum(t.numel() * t.element_size() for t in (h_keys, h_q, h_pos, h_Q, h_K, h_V))
+    d2h = h_O.numel() * h_O.element_size()
+
+    def step():
+        for d, h in ((d_keys, h_keys), (d_q, h_q), (d_pos, h_pos), (d_Q, h_Q), (d_K, h_K), (d_V, h_V)):
+            d.copy_(h, non_blocking=True)
+        layer.build(d_keys)
+        layer.index(d_q, d_pos)
+        layer.attend(d_Q, d_K, d_V, d_O)
+        h_O.copy_(d_O, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    nq = q_np.shape[0]
+    return {"value": round(world * nq * args.steps / (ms / 1e3), 1), "unit": UNIT,
+            "ms_per_step": round(ms / args.steps, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def run_decode(args, dev):
+    """Decode at T = 1M (Flat, k = 4096): batch-1 index_decode + attention per
+    new token, 64 tokens; mean us/token over the timed tokens."""
+    wl = I.WORKLOADS["flat_1m"]
+    T, nd, hq, hkv = wl["T"], wl["n_decode"], wl["hq"], wl["hkv"]
+    keys_all = I.index_keys(0, T + nd, wl["n_components"])
+    pos_np = np.arange(T, T + nd, dtype=np.int64)
+    q_np = I.index_queries(0, keys_all, pos_np)
+    layer = SparseLayer(T, k=wl["k"], mode="flat", max_queries=1, Hq=hq)
+    layer.build(torch.from_numpy(keys_all[:T]).to(dev))
+    g = torch.Generator(device=dev)
+    g.manual_seed(77)
+    K = torch.randn((T + nd, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    V = torch.randn((T + nd, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    Qd = torch.randn((nd, 1, hq, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    qd = torch.from_numpy(q_np).to(dev)
+    pd = torch.from_numpy(pos_np).to(dev)
+    O = torch.empty((1, hq, 128), dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.current_stream()
+    for i in range(4):
+        layer.index(qd[i:i + 1], pd[i:i + 1], decode=True)
+        layer.attend(Qd[i], K, V, O)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for i in range(nd):
+        layer.index(qd[i:i + 1], pd[i:i + 1], decode=True)
+        layer.attend(Qd[i], K, V, O)
+    e1.record(st)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / nd
+    lens = layer.lens[:1].item()
+    return {"workload": "flat_1m", "T": T, "tokens": nd, "us_per_token": round(us, 2), "list_len": int(lens),
+            "note": "batch 1; index_decode + sparse attention per token, launched eagerly"}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=20.0, sample=None):
+    """The oracle as it stands on this host's cores: full cache build + index and
+    attention of evenly spaced sample queries, extrapolated to all queries."""
+    import oracle as O
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    O.build()
+    nq = len(pos_np)
+    t0 = time.perf_counter()
+    oc = O.build_cache(keys_np)
+    t_build = time.perf_counter() - t0
+    Kb = K.view(torch.int16).cpu().numpy().view(np.uint16)
+    Vb = V.view(torch.int16).cpu().numpy().view(np.uint16)
+    hkv = Kb.shape[1]
+    S = sample or 64
+    done, t_q = 0, 0.0
+    rng_idx = np.linspace(0, nq - 1, 4096).astype(np.int64)
+    while True:
+        sel = rng_idx[(np.arange(S) * 4096 // S)]
+        Qb = I.normal_bf16_bits(1, I.STREAM_Q, (S, hq, 128))
+        t0 = time.perf_counter()
+        lists, lens = O.index(q_np[sel], pos_np[sel], oc, k=wl["k"])
+        O.attention(Qb, Kb, Vb, lists, lens)
+        t_q = time.perf_counter() - t0
+        done = S
+        if t_q * 2 > budget_s or S >= 1024:
+            break
+        S *= 2
+    per_q = t_q / done
+    total = t_build + per_q * nq
+    return {"value": round(nq / total, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"full cache build ({t_build:.2f} s) + index and attention of {done} evenly spaced of "
+                      f"{nq} queries ({t_q:.2f} s), extrapolated to all queries",
+            "hkv": hkv}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle on this host, same metric and workload."""
+    if rank != 0:
+        return
+    wl = I.WORKLOADS[args.workload]
+    keys_np, q_np, pos_np = make_prefill_inputs(wl)
+    T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
+    Kb = torch.from_numpy(I.normal_bf16_bits(0, I.STREAM_K, (T, hkv, 128)).view(np.int16)).view(torch.bfloat16)
+    Vb = torch.from_numpy(I.normal_bf16_bits(0, I.STREAM_V, (T, hkv, 128)).view(np.int16)).view(torch.bfloat16)
+    vals = []
+    for _ in range(args.warmup + args.steps):
+        vals.append(cpu_baseline(wl, keys_np, q_np, pos_np, Kb, Vb, hq, budget_s=args.cpu_budget, sample=32))
+    vals = vals[args.warmup:]
+    v = float(np.mean([x["value"] for x in vals]))
+    line = {"metric": METRIC, "value": round(v, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(nq / v * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "T": T, "queries": nq, "k": wl["k"], "mode": wl["mode"],
+                       "Hq": hq, "Hkv": hkv, "head_dim": 128, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": vals[-1]["cores"], "kind": "oracle",
+                             "sample": vals[-1]["sample"]},
+            "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="flat_128k", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    world, rank, local = init_dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

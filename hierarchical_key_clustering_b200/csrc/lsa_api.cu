@@ -1,0 +1,488 @@
+// C ABI of the LSA hot path (see include/lsa.h for the contract of every
+// entry point).  This file only checks arguments, carves caller buffers and
+// enqueues the kernels of lsa_build.cu, lsa_index.cu and lsa_attn.cu on the
+// caller's stream.  It never allocates device memory and never synchronises.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "lsa.h"
+#include "lsa_common.cuh"
+#include "lsa_kernels.h"
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+thread_local char g_err[512] = "no error";
+
+int fail(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(LSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p)
+{
+    return ((uintptr_t)p & 15u) == 0;
+}
+
+int64_t align256(int64_t x)
+{
+    return (x + 255) & ~(int64_t)255;
+}
+
+int sm_count()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+int check_params(const lsa_params *p)
+{
+    if (!p) return fail(LSA_ERR_ARG, "params is NULL");
+    if (p->n_pool != LSA_N_POOL || p->block != LSA_BLOCK || p->n_buckets != LSA_BUCKETS ||
+        p->cap_items != LSA_N_POOL)
+        return fail(LSA_ERR_ARG,
+                    "only n_pool=4, block=512, n_buckets=64, cap_items=4 are built (got %d, %d, %d, %d)",
+                    p->n_pool, p->block, p->n_buckets, p->cap_items);
+    if (p->sink < 0 || p->window < 0 || p->k < 0) return fail(LSA_ERR_ARG, "sink, window and k must be >= 0");
+    if (p->k > (1 << 20)) return fail(LSA_ERR_ARG, "k = %d is above the supported 1048576", p->k);
+    if (p->mode != LSA_MODE_FLAT && p->mode != LSA_MODE_TREE) return fail(LSA_ERR_ARG, "mode must be 0 or 1");
+    if (p->mode == LSA_MODE_TREE && p->beam < 1) return fail(LSA_ERR_ARG, "beam must be >= 1");
+    return LSA_OK;
+}
+
+int64_t top_buckets(const lsa_params *p)
+{
+    return ((int64_t)p->k + p->sink + p->window + LSA_N_POOL - 1) / LSA_N_POOL;
+}
+
+int64_t cand_cap(const lsa_params *p)
+{
+    const int64_t P = top_buckets(p);
+    int64_t cap = p->cand_cap > 0 ? p->cand_cap : lsa::pow2_ceil64(2 * P);
+    if (p->mode == LSA_MODE_TREE) {
+        int64_t need = p->beam > P ? p->beam : P;
+        if (cap < need) cap = need;
+    }
+    return cap;
+}
+
+struct CacheLayout {
+    int64_t off[6];
+    int64_t bytes;
+};
+
+CacheLayout cache_layout(int64_t capacity)
+{
+    const int64_t items = capacity / LSA_N_POOL, nblk = capacity / LSA_BLOCK, nb = nblk * LSA_BUCKETS;
+    const int64_t sz[6] = {items * LSA_DIM * 4, nblk * LSA_ITEMS, nb * LSA_SLOTS * 4, nb * 4, nb * LSA_DIM * 4,
+                           nb * LSA_DIM * 2};
+    CacheLayout L;
+    int64_t o = 0;
+    for (int i = 0; i < 6; ++i) {
+        L.off[i] = o;
+        o += align256(sz[i]);
+    }
+    L.bytes = o;
+    return L;
+}
+
+int tree_levels(int64_t nb, int64_t *size, int64_t *offset)
+{
+    int L = 0;
+    int64_t n = nb, o = 0;
+    while (L < LSA_MAX_LEVELS) {
+        size[L] = n;
+        offset[L] = o;
+        o += n;
+        ++L;
+        if (n <= 1) break;
+        n = (n + 1) / 2;
+    }
+    offset[L] = o;
+    return L;
+}
+
+struct TreeLayout {
+    int64_t off[8];
+    int64_t bytes;
+    int64_t nodes;
+};
+
+TreeLayout tree_layout(int64_t nblk)
+{
+    int64_t size[LSA_MAX_LEVELS + 1], offset[LSA_MAX_LEVELS + 2];
+    int L = tree_levels(nblk * LSA_BUCKETS, size, offset);
+    const int64_t n = offset[L];
+    const int64_t sz[8] = {n * 2 * 4, n * 4, n * 4, n * 4, n * 4, n * LSA_DIM * 4, n * LSA_DIM * 4, n * LSA_DIM * 2};
+    TreeLayout T;
+    int64_t o = 0;
+    for (int i = 0; i < 8; ++i) {
+        T.off[i] = o;
+        o += align256(sz[i]);
+    }
+    T.bytes = o;
+    T.nodes = n;
+    return T;
+}
+
+struct IndexLayout {
+    int64_t off[7];
+    int64_t bytes;
+    int64_t gstride;
+    int64_t cap;
+};
+
+IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
+{
+    const int64_t P = top_buckets(p);
+    const int64_t N = nblk * LSA_BUCKETS;
+    int64_t G = lsa::n_groups(N, P);
+    if (G < 8 * P) G = 8 * P;  // groups of any smaller visible range never exceed this
+    if (p->mode == LSA_MODE_TREE) G = 1;
+    IndexLayout L;
+    L.gstride = G;
+    L.cap = cand_cap(p);
+    const int64_t sz[7] = {nq * LSA_DIM * 2, nq * 4, nq * 4, nq * 4, nq * G * 4, nq * L.cap * 4, nq * L.cap * 4};
+    int64_t o = 0;
+    for (int i = 0; i < 7; ++i) {
+        L.off[i] = o;
+        o += align256(sz[i]);
+    }
+    L.bytes = o;
+    return L;
+}
+
+int attention_nsplit(int64_t nq, int32_t Hkv, int32_t Lmax)
+{
+    const int64_t units = nq * (int64_t)Hkv;
+    if (units >= 2048) return 1;
+    int64_t s = (2048 + units - 1) / units;
+    const int64_t chunks = (Lmax + 15) / 16;
+    if (s > chunks) s = chunks;
+    return (int)(s < 1 ? 1 : s);
+}
+
+int64_t attention_ws_bytes(int64_t nq, int32_t Hq, int32_t nsplit)
+{
+    if (nsplit <= 1) return 0;
+    return align256(nq * Hq * (int64_t)nsplit * LSA_HEAD_DIM * 4) + align256(nq * Hq * (int64_t)nsplit * 2 * 4);
+}
+
+int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache, const lsa_tree *tree,
+               int32_t *lists, int32_t *lens, int32_t Lmax, const lsa_params *p, void *ws, int64_t ws_bytes,
+               void *stream)
+{
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (nq < 0) return fail(LSA_ERR_SHAPE, "nq < 0");
+    if (!cache) return fail(LSA_ERR_ARG, "cache is NULL");
+    if (nq == 0) return LSA_OK;
+    if (!qidx || !pos || !lists || !lens) return fail(LSA_ERR_ARG, "qidx, pos, lists and lens must be non-NULL");
+    if (!aligned16(qidx) || !aligned16(lists)) return fail(LSA_ERR_ARG, "qidx and lists must be 16-byte aligned");
+    if (Lmax < lsa_list_budget(p)) return fail(LSA_ERR_SHAPE, "Lmax %d < list budget %d", Lmax, lsa_list_budget(p));
+    if (cache->n_blocks < 0 || cache->n_blocks * LSA_BLOCK > cache->capacity)
+        return fail(LSA_ERR_SHAPE, "cache n_blocks %lld out of range", (long long)cache->n_blocks);
+    if (cache->n_blocks > 0 && (!cache->members || !cache->count || !cache->centroid_bf16))
+        return fail(LSA_ERR_ARG, "cache arrays are NULL");
+    if (p->mode == LSA_MODE_TREE) {
+        if (!tree) return fail(LSA_ERR_ARG, "Tree mode needs a tree");
+        if (cache->n_blocks > 0 && tree->n_blocks != cache->n_blocks)
+            return fail(LSA_ERR_SHAPE, "tree covers %lld blocks, cache has %lld", (long long)tree->n_blocks,
+                        (long long)cache->n_blocks);
+        const int64_t P = top_buckets(p);
+        const int64_t B1 = ((P + 1) / 2) > p->beam ? (P + 1) / 2 : p->beam;
+        if (2 * B1 + LSA_ITEMS + 2 > 8192)
+            return fail(LSA_ERR_ARG, "beam %d / k %d too large for the beam kernel", p->beam, p->k);
+    }
+    const int64_t P = top_buckets(p);
+    IndexLayout L = index_layout(nq, cache->n_blocks, p);
+    if (L.cap < P) return fail(LSA_ERR_ARG, "cand_cap %lld < top buckets %lld", (long long)L.cap, (long long)P);
+    if (L.cap > 8192) return fail(LSA_ERR_ARG, "cand_cap %lld above 8192", (long long)L.cap);
+    if ((int64_t)lsa::pow2_ceil64(p->k > 0 ? p->k : 1) * 4 + lsa::pow2_ceil64(L.cap) * 8 + P * 4 > 200 * 1024)
+        return fail(LSA_ERR_ARG, "k %d too large for the expansion kernel", p->k);
+    if (!ws || ws_bytes < L.bytes)
+        return fail(LSA_ERR_WORKSPACE, "index workspace %lld bytes < %lld", (long long)ws_bytes, (long long)L.bytes);
+    if (((uintptr_t)ws & 255u) != 0) return fail(LSA_ERR_ARG, "workspace must be 256-byte aligned");
+    char *w = (char *)ws;
+    lsa::IndexWs iw;
+    iw.qhat = (uint16_t *)(w + L.off[0]);
+    iw.horizon = (int32_t *)(w + L.off[1]);
+    iw.tau = (float *)(w + L.off[2]);
+    iw.cnt = (int32_t *)(w + L.off[3]);
+    iw.gmax = (float *)(w + L.off[4]);
+    iw.cand_s = (float *)(w + L.off[5]);
+    iw.cand_id = (int32_t *)(w + L.off[6]);
+    iw.gmax_stride = L.gstride;
+    iw.cap = (int32_t)L.cap;
+    lsa::IndexArgs a;
+    a.qidx = qidx;
+    a.pos = pos;
+    a.nq = nq;
+    a.n_blocks = cache->n_blocks;
+    a.members = cache->members;
+    a.count = cache->count;
+    a.centroid_bf16 = cache->centroid_bf16;
+    a.lists = lists;
+    a.lens = lens;
+    a.Lmax = Lmax;
+    a.k = p->k;
+    a.sink = p->sink;
+    a.window = p->window;
+    a.beam = p->beam;
+    a.mode = p->mode;
+    a.P = (int32_t)P;
+    lsa::TreeView tv;
+    const lsa::TreeView *tvp = nullptr;
+    if (p->mode == LSA_MODE_TREE && cache->n_blocks > 0) {
+        tv.child = tree->child;
+        tv.parent = tree->parent;
+        tv.max_block = tree->max_block;
+        tv.centroid_bf16 = tree->centroid_bf16;
+        tv.n_levels = tree->n_levels;
+        for (int l = 0; l < 40; ++l) tv.level_size[l] = tree->level_size[l];
+        for (int l = 0; l < 41; ++l) tv.level_offset[l] = tree->level_offset[l];
+        tvp = &tv;
+    }
+    cudaError_t e = lsa::launch_index(a, iw, tvp, (cudaStream_t)stream, sm_count());
+    if (e != cudaSuccess) return cuda_fail(e, "index launch");
+    return LSA_OK;
+}
+
+}  // namespace
+
+namespace lsa {
+void count_launches(int n)
+{
+    g_launches.fetch_add(n, std::memory_order_relaxed);
+}
+}  // namespace lsa
+
+extern "C" {
+
+int64_t lsa_launch_count(void)
+{
+    return g_launches.load(std::memory_order_relaxed);
+}
+
+void lsa_default_params(lsa_params *p)
+{
+    if (!p) return;
+    p->n_pool = LSA_N_POOL;
+    p->block = LSA_BLOCK;
+    p->n_buckets = LSA_BUCKETS;
+    p->cap_items = LSA_N_POOL;
+    p->sink = 4;
+    p->window = 512;
+    p->k = 4096;
+    p->beam = 32;
+    p->mode = LSA_MODE_FLAT;
+    p->cand_cap = 0;
+}
+
+const char *lsa_last_error_string(void)
+{
+    return g_err;
+}
+
+int32_t lsa_list_budget(const lsa_params *p)
+{
+    return p ? p->k + p->sink + p->window + 1 : -1;
+}
+
+int32_t lsa_top_buckets(const lsa_params *p)
+{
+    return p ? (int32_t)top_buckets(p) : -1;
+}
+
+int64_t lsa_cache_bytes(int64_t capacity)
+{
+    if (capacity < 0) return -1;
+    return cache_layout(capacity).bytes;
+}
+
+int lsa_cache_bind(void *base, int64_t bytes, int64_t capacity, lsa_cache *out)
+{
+    if (!out) return fail(LSA_ERR_ARG, "out is NULL");
+    if (capacity < 0) return fail(LSA_ERR_SHAPE, "capacity < 0");
+    CacheLayout L = cache_layout(capacity);
+    if (!base || ((uintptr_t)base & 255u)) return fail(LSA_ERR_ARG, "cache buffer must be non-NULL and 256-byte aligned");
+    if (bytes < L.bytes) return fail(LSA_ERR_SHAPE, "cache buffer %lld bytes < %lld", (long long)bytes, (long long)L.bytes);
+    char *b = (char *)base;
+    out->capacity = capacity;
+    out->n_blocks = 0;
+    out->pooled = (float *)(b + L.off[0]);
+    out->item_bucket = (uint8_t *)(b + L.off[1]);
+    out->members = (int32_t *)(b + L.off[2]);
+    out->count = (int32_t *)(b + L.off[3]);
+    out->centroid = (float *)(b + L.off[4]);
+    out->centroid_bf16 = (uint16_t *)(b + L.off[5]);
+    return LSA_OK;
+}
+
+int64_t lsa_tree_bytes(int64_t n_blocks)
+{
+    if (n_blocks < 0) return -1;
+    return tree_layout(n_blocks).bytes;
+}
+
+int lsa_tree_bind(void *base, int64_t bytes, int64_t n_blocks, lsa_tree *out)
+{
+    if (!out) return fail(LSA_ERR_ARG, "out is NULL");
+    if (n_blocks < 1) return fail(LSA_ERR_SHAPE, "a tree needs at least one block");
+    TreeLayout T = tree_layout(n_blocks);
+    if (!base || ((uintptr_t)base & 255u)) return fail(LSA_ERR_ARG, "tree buffer must be non-NULL and 256-byte aligned");
+    if (bytes < T.bytes) return fail(LSA_ERR_SHAPE, "tree buffer %lld bytes < %lld", (long long)bytes, (long long)T.bytes);
+    memset(out, 0, sizeof(*out));
+    int64_t size[LSA_MAX_LEVELS + 1], offset[LSA_MAX_LEVELS + 2];
+    int L = tree_levels(n_blocks * LSA_BUCKETS, size, offset);
+    out->n_blocks = 0;
+    out->n_levels = L;
+    for (int l = 0; l < L; ++l) {
+        out->level_size[l] = size[l];
+        out->level_offset[l] = offset[l];
+    }
+    out->level_offset[L] = offset[L];
+    char *b = (char *)base;
+    out->child = (int32_t *)(b + T.off[0]);
+    out->parent = (int32_t *)(b + T.off[1]);
+    out->weight = (int32_t *)(b + T.off[2]);
+    out->min_block = (int32_t *)(b + T.off[3]);
+    out->max_block = (int32_t *)(b + T.off[4]);
+    out->sum = (float *)(b + T.off[5]);
+    out->centroid = (float *)(b + T.off[6]);
+    out->centroid_bf16 = (uint16_t *)(b + T.off[7]);
+    return LSA_OK;
+}
+
+int64_t lsa_index_workspace_bytes(int64_t nq, int64_t n_blocks, const lsa_params *p)
+{
+    if (!p || nq < 0 || n_blocks < 0) return -1;
+    return index_layout(nq, n_blocks, p).bytes;
+}
+
+int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, int32_t Lmax)
+{
+    if (nq < 0 || Hq < 1 || head_dim != LSA_HEAD_DIM || Lmax < 1) return -1;
+    return attention_ws_bytes(nq, Hq, attention_nsplit(nq, 1, Lmax));
+}
+
+int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache *cache, const lsa_params *p,
+                    void *stream)
+{
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (!cache) return fail(LSA_ERR_ARG, "cache is NULL");
+    if (t_begin < 0 || t_end < t_begin) return fail(LSA_ERR_SHAPE, "need 0 <= t_begin <= t_end");
+    if (t_end > cache->capacity)
+        return fail(LSA_ERR_SHAPE, "t_end %lld > cache capacity %lld", (long long)t_end, (long long)cache->capacity);
+    const int64_t i0 = t_begin / LSA_N_POOL, i1 = t_end / LSA_N_POOL;
+    const int64_t b0 = t_begin / LSA_BLOCK, b1 = t_end / LSA_BLOCK;
+    if (i1 > i0 || b1 > b0) {
+        if (!keys || !aligned16(keys)) return fail(LSA_ERR_ARG, "keys must be non-NULL and 16-byte aligned");
+        if (!cache->pooled || !cache->item_bucket || !cache->members || !cache->count || !cache->centroid ||
+            !cache->centroid_bf16)
+            return fail(LSA_ERR_ARG, "cache arrays are NULL (bind the cache first)");
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = lsa::launch_pool_norm(keys, i0, i1, cache->pooled, st, sm_count());
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    e = lsa::launch_ward(cache->pooled, b0, b1, p->cap_items, cache->item_bucket, cache->members, cache->count,
+                         cache->centroid, cache->centroid_bf16, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ward launch");
+    if (b1 > cache->n_blocks) cache->n_blocks = b1;
+    return LSA_OK;
+}
+
+int lsa_build_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream)
+{
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (!cache || !tree) return fail(LSA_ERR_ARG, "cache and tree must be non-NULL");
+    if (cache->n_blocks < 1) return fail(LSA_ERR_SHAPE, "the cache has no complete block");
+    int64_t size[LSA_MAX_LEVELS + 1], offset[LSA_MAX_LEVELS + 2];
+    int L = tree_levels(cache->n_blocks * LSA_BUCKETS, size, offset);
+    if (tree->n_levels < L || tree->level_offset[tree->n_levels] < offset[L] || !tree->child || !tree->sum)
+        return fail(LSA_ERR_SHAPE, "tree buffer bound for fewer blocks than the cache holds");
+    tree->n_levels = L;
+    for (int l = 0; l < LSA_MAX_LEVELS; ++l) tree->level_size[l] = l < L ? size[l] : 0;
+    for (int l = 0; l <= LSA_MAX_LEVELS; ++l) tree->level_offset[l] = l <= L ? offset[l] : offset[L];
+    lsa::TreeDev td{tree->child, tree->parent, tree->weight, tree->min_block, tree->max_block,
+                    tree->sum, tree->centroid, tree->centroid_bf16};
+    cudaError_t e = lsa::launch_tree(cache->pooled, cache->members, cache->count, size[0], td, size, offset, L,
+                                     (cudaStream_t)stream, sm_count());
+    if (e != cudaSuccess) return cuda_fail(e, "tree launch");
+    tree->n_blocks = cache->n_blocks;
+    return LSA_OK;
+}
+
+int lsa_index_prefill(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache,
+                      const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax, const lsa_params *p,
+                      void *ws, int64_t ws_bytes, void *stream)
+{
+    return index_impl(qidx, pos, nq, cache, tree, lists, lens, Lmax, p, ws, ws_bytes, stream);
+}
+
+int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache,
+                     const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax, const lsa_params *p,
+                     void *ws, int64_t ws_bytes, void *stream)
+{
+    return index_impl(qidx, pos, nq, cache, tree, lists, lens, Lmax, p, ws, ws_bytes, stream);
+}
+
+int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t nq, int32_t Hq,
+                         int32_t Hkv, int32_t head_dim, int64_t Tk, const int32_t *lists, const int32_t *lens,
+                         int32_t Lmax, float scale, uint16_t *O, float *lse, void *ws, int64_t ws_bytes,
+                         void *stream)
+{
+    if (nq < 0) return fail(LSA_ERR_SHAPE, "nq < 0");
+    if (nq == 0) return LSA_OK;
+    if (head_dim != LSA_HEAD_DIM) return fail(LSA_ERR_ARG, "head_dim must be %d", LSA_HEAD_DIM);
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 16)
+        return fail(LSA_ERR_ARG, "need Hq a multiple of Hkv with Hq/Hkv <= 16 (Hq=%d Hkv=%d)", Hq, Hkv);
+    if (Tk < 1 || Lmax < 1) return fail(LSA_ERR_SHAPE, "Tk and Lmax must be >= 1");
+    if (!Q || !K || !V || !lists || !lens || !O) return fail(LSA_ERR_ARG, "tensor pointers must be non-NULL");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return fail(LSA_ERR_ARG, "Q, K, V and O must be 16-byte aligned");
+    if (!(scale > 0.0f)) return fail(LSA_ERR_ARG, "scale must be > 0");
+    int nsplit = attention_nsplit(nq, Hkv, Lmax);
+    while (nsplit > 1 && (!ws || ws_bytes < attention_ws_bytes(nq, Hq, nsplit))) nsplit >>= 1;
+    lsa::AttnArgs a;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.nq = nq;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Tk = Tk;
+    a.lists = lists;
+    a.lens = lens;
+    a.Lmax = Lmax;
+    a.scale = scale;
+    a.O = O;
+    a.lse = lse;
+    a.nsplit = nsplit;
+    a.part_o = nullptr;
+    a.part_ml = nullptr;
+    if (nsplit > 1) {
+        if (((uintptr_t)ws & 255u) != 0) return fail(LSA_ERR_ARG, "workspace must be 256-byte aligned");
+        a.part_o = (float *)ws;
+        a.part_ml = (float *)((char *)ws + align256(nq * Hq * (int64_t)nsplit * LSA_HEAD_DIM * 4));
+    }
+    cudaError_t e = lsa::launch_attention(a, (cudaStream_t)stream, sm_count());
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return LSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,328 @@
+// Exact sparse attention over LSA index lists on sm_100a.
+//
+// Method: Latent Sparse Attention pages -- learnaivisually explainer, "What
+// one query actually does": one index list per query, shared by all of its
+// attention heads, then ordinary (softmax) attention over sink, selected keys
+// and window.
+//
+// Each list is private to one query, so the work is a gather: per (query,
+// KV head) the listed K and V rows (256 B each) stream in once and are used
+// by the Hq/Hkv query heads of that group.  One warp owns one (query, KV
+// head[, key split]) unit: its G = Hq/Hkv heads form the rows of a 16-row
+// mma.sync tile (rows >= G are zero), 16 gathered keys form a chunk, and an
+// fp32 online softmax carries the running max and sum.  K/V rows are
+// gathered with cp.async into a 3-stage ring in shared memory.  A decode
+// query (few queries, long list) splits its list over many warps and a
+// second kernel merges the partial results by log-sum-exp.
+#include <cuda_bf16.h>
+
+#include "lsa_common.cuh"
+#include "lsa_kernels.h"
+
+namespace lsa {
+
+constexpr int KCH = 16;                          // keys per chunk
+constexpr int ROWB = 136;                        // bf16 per smem row (128 + 8 pad)
+constexpr int NST = 3;                           // pipeline stages
+constexpr int STAGE_BYTES = 2 * KCH * ROWB * 2;  // K + V
+constexpr int WARP_BYTES = NST * STAGE_BYTES;
+constexpr int AWARPS = 4;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes));
+}
+
+__device__ __forceinline__ void cp_commit()
+{
+    asm volatile("cp.async.commit_group;\n" ::);
+}
+
+template <int N>
+__device__ __forceinline__ void cp_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t ld_u32(const uint16_t *p)
+{
+    return *reinterpret_cast<const uint32_t *>(p);
+}
+
+__global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_split)
+{
+    extern __shared__ __align__(128) uint8_t asmem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * AWARPS + warp;
+    const int64_t total = a.nq * a.Hkv * a.nsplit;
+    if (unit >= total) return;
+    const int split = (int)(unit % a.nsplit);
+    const int64_t qg = unit / a.nsplit;
+    const int g = (int)(qg % a.Hkv);
+    const int64_t q = qg / a.Hkv;
+    const int G = a.Hq / a.Hkv;
+    const int len = a.lens[q];
+    const int begin = split * keys_per_split;
+    const int end = min(len, begin + keys_per_split);
+    const int nch = end > begin ? (end - begin + KCH - 1) / KCH : 0;
+    const uint32_t sbase = smem_u32(asmem + warp * WARP_BYTES);
+    const int32_t *lst = a.lists + q * (int64_t)a.Lmax;
+
+    const int r0 = lane >> 2, c = lane & 3;
+    const uint16_t *Qb = a.Q + ((q * a.Hq) + (int64_t)g * G) * LSA_HEAD;
+    uint32_t qa[8][4];
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        qa[kk][0] = r0 < G ? ld_u32(Qb + r0 * LSA_HEAD + kk * 16 + 2 * c) : 0u;
+        qa[kk][1] = r0 + 8 < G ? ld_u32(Qb + (r0 + 8) * LSA_HEAD + kk * 16 + 2 * c) : 0u;
+        qa[kk][2] = r0 < G ? ld_u32(Qb + r0 * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
+        qa[kk][3] = r0 + 8 < G ? ld_u32(Qb + (r0 + 8) * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
+    }
+
+    auto load = [&](int ch, int st) {
+        const int base = begin + ch * KCH;
+        int my = -1;
+        if (lane < KCH && base + lane < end) my = lst[base + lane];
+        if (my >= a.Tk) my = -1;  // out-of-range entries are read as zeros, never fetched
+        const uint32_t sK = sbase + st * STAGE_BYTES;
+        const uint32_t sV = sK + KCH * ROWB * 2;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int lin = it * 32 + lane;
+            const int row = lin >> 4, seg = lin & 15;
+            const int idx = __shfl_sync(LSA_FULL, my, row);
+            const int64_t off = ((int64_t)(idx < 0 ? 0 : idx) * a.Hkv + g) * LSA_HEAD + seg * 8;
+            const int bytes = idx < 0 ? 0 : 16;
+            const uint32_t so = (uint32_t)((row * ROWB + seg * 8) * 2);
+            cp_async16(sK + so, a.K + off, bytes);
+            cp_async16(sV + so, a.V + off, bytes);
+        }
+        cp_commit();
+    };
+
+    float o[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[nt][j] = 0.0f;
+    const float NEG = __int_as_float(0xff800000);
+    float m0 = NEG, m1 = NEG, l0 = 0.0f, l1 = 0.0f;
+    const float sl2 = a.scale * LOG2E;
+
+#pragma unroll
+    for (int s = 0; s < NST - 1; ++s) {
+        if (s < nch) load(s, s);
+        else cp_commit();
+    }
+    for (int ch = 0; ch < nch; ++ch) {
+        const int nxt = ch + NST - 1;
+        if (nxt < nch) load(nxt, nxt % NST);
+        else cp_commit();
+        cp_wait<NST - 1>();
+        __syncwarp();
+        const uint32_t sK = sbase + (ch % NST) * STAGE_BYTES;
+        const uint32_t sV = sK + KCH * ROWB * 2;
+        float s[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s[nt][j] = 0.0f;
+        {
+            const int mat = lane >> 3, rr = lane & 7;
+            const int key = rr + ((mat >> 1) << 3);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t b[4];
+                const int dim = kk * 16 + ((mat & 1) << 3);
+                ldsm_x4(b, sK + (uint32_t)((key * ROWB + dim) * 2));
+                mma16816(s[0], qa[kk], b[0], b[1]);
+                mma16816(s[1], qa[kk], b[2], b[3]);
+            }
+        }
+        const int base = begin + ch * KCH;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int kidx = nt * 8 + 2 * c + (j & 1);
+                s[nt][j] = (base + kidx < end) ? s[nt][j] * sl2 : NEG;
+            }
+        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(LSA_FULL, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(LSA_FULL, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(LSA_FULL, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(LSA_FULL, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+        float rs0 = 0.0f, rs1 = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            s[nt][0] = exp2f(s[nt][0] - mn0);
+            s[nt][1] = exp2f(s[nt][1] - mn0);
+            s[nt][2] = exp2f(s[nt][2] - mn1);
+            s[nt][3] = exp2f(s[nt][3] - mn1);
+            rs0 += s[nt][0] + s[nt][1];
+            rs1 += s[nt][2] + s[nt][3];
+        }
+        rs0 += __shfl_xor_sync(LSA_FULL, rs0, 1);
+        rs0 += __shfl_xor_sync(LSA_FULL, rs0, 2);
+        rs1 += __shfl_xor_sync(LSA_FULL, rs1, 1);
+        rs1 += __shfl_xor_sync(LSA_FULL, rs1, 2);
+        l0 = l0 * al0 + rs0;
+        l1 = l1 * al1 + rs1;
+        m0 = mn0;
+        m1 = mn1;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            o[nt][0] *= al0;
+            o[nt][1] *= al0;
+            o[nt][2] *= al1;
+            o[nt][3] *= al1;
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf16(s[0][0], s[0][1]);
+        pa[1] = pack_bf16(s[0][2], s[0][3]);
+        pa[2] = pack_bf16(s[1][0], s[1][1]);
+        pa[3] = pack_bf16(s[1][2], s[1][3]);
+        {
+            const int mat = lane >> 3, rr = lane & 7;
+            const int key = rr + ((mat & 1) << 3);
+#pragma unroll
+            for (int nt2 = 0; nt2 < 8; ++nt2) {
+                uint32_t b[4];
+                const int dim = nt2 * 16 + ((mat >> 1) << 3);
+                ldsm_x4_t(b, sV + (uint32_t)((key * ROWB + dim) * 2));
+                mma16816(o[2 * nt2], pa, b[0], b[1]);
+                mma16816(o[2 * nt2 + 1], pa, b[2], b[3]);
+            }
+        }
+        __syncwarp();
+    }
+    cp_wait<0>();
+
+    if (a.nsplit == 1) {
+        const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
+        uint16_t *Ob = a.O + ((q * a.Hq) + (int64_t)g * G) * LSA_HEAD;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int dim = nt * 8 + 2 * c;
+            if (r0 < G)
+                *reinterpret_cast<uint32_t *>(Ob + r0 * LSA_HEAD + dim) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
+            if (r0 + 8 < G)
+                *reinterpret_cast<uint32_t *>(Ob + (r0 + 8) * LSA_HEAD + dim) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
+        }
+        if (c == 0 && a.lse) {
+            if (r0 < G) a.lse[q * a.Hq + g * G + r0] = m0 * LN2 + logf(l0);
+            if (r0 + 8 < G) a.lse[q * a.Hq + g * G + r0 + 8] = m1 * LN2 + logf(l1);
+        }
+    } else {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int r = r0 + 8 * half;
+            if (r >= G) continue;
+            const int64_t pidx = ((q * a.Hq) + (int64_t)g * G + r) * a.nsplit + split;
+            float *po = a.part_o + pidx * LSA_HEAD;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                const int dim = nt * 8 + 2 * c;
+                *reinterpret_cast<float2 *>(po + dim) = make_float2(o[nt][2 * half], o[nt][2 * half + 1]);
+            }
+            if (c == 0) {
+                a.part_ml[pidx * 2] = half ? m1 : m0;
+                a.part_ml[pidx * 2 + 1] = half ? l1 : l0;
+            }
+        }
+    }
+}
+
+// Merge the partial results of the key splits of one (query, head): one warp.
+__global__ void __launch_bounds__(256) k_attn_combine(AttnArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t unit = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (unit >= a.nq * a.Hq) return;
+    const float *ml = a.part_ml + unit * a.nsplit * 2;
+    float M = __int_as_float(0xff800000);
+    for (int s = 0; s < a.nsplit; ++s)
+        if (ml[2 * s + 1] > 0.0f) M = fmaxf(M, ml[2 * s]);
+    float L = 0.0f;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int s = 0; s < a.nsplit; ++s) {
+        const float l = ml[2 * s + 1];
+        if (!(l > 0.0f)) continue;
+        const float w = exp2f(ml[2 * s] - M);
+        L += l * w;
+        const float4 v = *reinterpret_cast<const float4 *>(a.part_o + (unit * a.nsplit + s) * LSA_HEAD + lane * 4);
+        acc[0] += v.x * w;
+        acc[1] += v.y * w;
+        acc[2] += v.z * w;
+        acc[3] += v.w * w;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    uint16_t *Ob = a.O + unit * LSA_HEAD + lane * 4;
+    *reinterpret_cast<uint32_t *>(Ob) = pack_bf16(acc[0] * inv, acc[1] * inv);
+    *reinterpret_cast<uint32_t *>(Ob + 2) = pack_bf16(acc[2] * inv, acc[3] * inv);
+    if (lane == 0 && a.lse) a.lse[unit] = M * LN2 + logf(L);
+}
+
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
+{
+    (void)n_sm;
+    if (a.nq <= 0) return cudaSuccess;
+    const int smem = AWARPS * WARP_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(k_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int kps = (a.Lmax + a.nsplit - 1) / a.nsplit;
+    kps = ((kps + KCH - 1) / KCH) * KCH;
+    const int64_t units = a.nq * a.Hkv * a.nsplit;
+    const int64_t blocks = (units + AWARPS - 1) / AWARPS;
+    k_attn<<<(unsigned)blocks, AWARPS * 32, smem, st>>>(a, kps);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.nsplit > 1) {
+        const int64_t warps = a.nq * a.Hq;
+        k_attn_combine<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(a);
+        count_launches(1);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace lsa

@@ -1,0 +1,165 @@
+// Device helpers shared by the LSA kernels (sm_100a).
+//
+// Build-path arithmetic (normalise, pool, Ward costs, tree costs, centroids)
+// uses the IEEE-rounded intrinsics __fadd_rn / __fmul_rn / __fsub_rn /
+// __fdiv_rn / __fsqrt_rn so that nvcc never contracts a multiply and an add
+// into an FMA: every value is reproducible bit for bit.  64-term sums of
+// squares follow one fixed order: lane l holds terms l and l+32, adds them,
+// then an xor butterfly over offsets 16, 8, 4, 2, 1 (IEEE addition is
+// commutative, so all lanes end with the same bits).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define LSA_D 64
+#define LSA_BLK 512
+#define LSA_NP 4
+#define LSA_NITEMS 128
+#define LSA_NBKT 64
+#define LSA_NSLOT 16
+#define LSA_RUN 128
+#define LSA_HEAD 128
+#define LSA_FULL 0xffffffffu
+
+namespace lsa {
+
+__device__ __forceinline__ float warp_sum_pairs(float t)
+{
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) t = __fadd_rn(t, __shfl_xor_sync(LSA_FULL, t, s));
+    return t;
+}
+
+// Sum of squares of a 64-vector held as (a = x[lane], b = x[lane + 32]).
+__device__ __forceinline__ float warp_sumsq(float a, float b)
+{
+    return warp_sum_pairs(__fadd_rn(__fmul_rn(a, a), __fmul_rn(b, b)));
+}
+
+// Squared distance of two 64-vectors held lane-wise.
+__device__ __forceinline__ float warp_sqdist(float a0, float a1, float b0, float b1)
+{
+    float e0 = __fsub_rn(a0, b0), e1 = __fsub_rn(a1, b1);
+    return warp_sum_pairs(__fadd_rn(__fmul_rn(e0, e0), __fmul_rn(e1, e1)));
+}
+
+// The same fixed-order reduction done by one thread over 32 partial terms.
+__device__ __forceinline__ float thread_tree32(float *t)
+{
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1)
+#pragma unroll
+        for (int l = 0; l < s; ++l) t[l] = __fadd_rn(t[l], t[l + s]);
+    return t[0];
+}
+
+// Normalise one lane-wise 64-vector: x / sqrt(sum x^2); zero stays zero.
+__device__ __forceinline__ void warp_normalize(float &a, float &b)
+{
+    float n = __fsqrt_rn(warp_sumsq(a, b));
+    if (n > 0.0f) {
+        a = __fdiv_rn(a, n);
+        b = __fdiv_rn(b, n);
+    } else {
+        a = 0.0f;
+        b = 0.0f;
+    }
+}
+
+__device__ __forceinline__ uint16_t f2bf_bits(float f)
+{
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t *>(&h);
+}
+
+__device__ __forceinline__ float bf_bits2f(uint16_t b)
+{
+    return __uint_as_float(((uint32_t)b) << 16);
+}
+
+// Monotone map float -> uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t f2ord(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float ord2f(uint32_t k)
+{
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+// Rank key for buckets: ascending order = (score desc, id asc).
+__device__ __forceinline__ uint64_t rank_key(float s, int32_t id)
+{
+    s = __fadd_rn(s, 0.0f);  // -0 ranks as +0 (they compare equal)
+    return ((uint64_t)(~f2ord(s)) << 32) | (uint32_t)id;
+}
+
+__device__ __forceinline__ float rank_key_score(uint64_t k)
+{
+    return ord2f(~(uint32_t)(k >> 32));
+}
+
+__device__ __forceinline__ int32_t rank_key_id(uint64_t k)
+{
+    return (int32_t)(uint32_t)(k & 0xffffffffu);
+}
+
+// Block-wide bitonic sort (ascending) of n = power of two keys in shared
+// memory.  All threads of the block must call it.
+template <typename T>
+__device__ void block_bitonic_sort(T *a, int n)
+{
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                int ixj = i ^ j;
+                if (ixj > i) {
+                    T x = a[i], y = a[ixj];
+                    bool up = ((i & k) == 0);
+                    if ((x > y) == up) {
+                        a[i] = y;
+                        a[ixj] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+__host__ __device__ __forceinline__ int64_t pow2_ceil64(int64_t x)
+{
+    int64_t p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+__host__ __device__ __forceinline__ int64_t pow2_floor64(int64_t x)
+{
+    int64_t p = 1;
+    while ((p << 1) <= x) p <<= 1;
+    return p;
+}
+
+// Group width of the Flat threshold pass for a query that sees N buckets:
+// the largest power of two <= N / (4P), clamped to [1, 128], so a query has
+// between 4P and 8P group maxima (or N of them when N is small).
+__host__ __device__ __forceinline__ int group_width(int64_t N, int64_t P)
+{
+    int64_t g = (N >= 4 * P) ? pow2_floor64(N / (4 * P)) : 1;
+    if (g > 128) g = 128;
+    return (int)g;
+}
+
+__host__ __device__ __forceinline__ int64_t n_groups(int64_t N, int64_t P)
+{
+    int g = group_width(N, P);
+    return (N + g - 1) / g;
+}
+
+}  // namespace lsa

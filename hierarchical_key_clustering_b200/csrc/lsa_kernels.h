@@ -1,0 +1,90 @@
+// Internal launch interface between the C ABI (lsa_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lsa {
+
+// Kernels enqueued since load (see lsa_launch_count in lsa.h).
+void count_launches(int n);
+
+struct TreeDev {
+    int32_t *child;
+    int32_t *parent;
+    int32_t *weight;
+    int32_t *min_block;
+    int32_t *max_block;
+    float *sum;
+    float *centroid;
+    uint16_t *centroid_bf16;
+};
+
+// Read-only view of the tree used by the beam search.
+struct TreeView {
+    const int32_t *child;
+    const int32_t *parent;
+    const int32_t *max_block;
+    const uint16_t *centroid_bf16;
+    int32_t n_levels;
+    int64_t level_size[40];
+    int64_t level_offset[41];
+};
+
+// Per-call index workspace (device pointers carved by the C ABI).
+struct IndexWs {
+    uint16_t *qhat;     // [nq, 64] bf16 normalised queries
+    int32_t *horizon;   // [nq] visible blocks
+    float *tau;         // [nq] Flat threshold
+    int32_t *cnt;       // [nq] candidates written
+    float *gmax;        // [nq, gmax_stride] group maxima
+    float *cand_s;      // [nq, cap] candidate scores
+    int32_t *cand_id;   // [nq, cap] candidate bucket ids
+    int64_t gmax_stride;
+    int32_t cap;
+};
+
+cudaError_t launch_pool_norm(const float *keys, int64_t item_begin, int64_t item_end, float *pooled,
+                             cudaStream_t st, int n_sm);
+cudaError_t launch_ward(const float *pooled, int64_t blk_begin, int64_t blk_end, int cap, uint8_t *item_bucket,
+                        int32_t *members, int32_t *count, float *centroid, uint16_t *centroid_bf16,
+                        cudaStream_t st);
+cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32_t *count, int64_t nb,
+                        const TreeDev &tr, const int64_t *level_size, const int64_t *level_offset, int n_levels,
+                        cudaStream_t st, int n_sm);
+
+struct IndexArgs {
+    const float *qidx;
+    const int64_t *pos;
+    int64_t nq;
+    int64_t n_blocks;
+    const int32_t *members;
+    const int32_t *count;
+    const uint16_t *centroid_bf16;
+    int32_t *lists;
+    int32_t *lens;
+    int32_t Lmax;
+    int32_t k, sink, window, beam, mode;
+    int32_t P;  // top buckets kept
+};
+
+cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *tree, cudaStream_t st, int n_sm);
+
+struct AttnArgs {
+    const uint16_t *Q, *K, *V;
+    int64_t nq;
+    int32_t Hq, Hkv;
+    int64_t Tk;
+    const int32_t *lists, *lens;
+    int32_t Lmax;
+    float scale;
+    uint16_t *O;
+    float *lse;
+    float *part_o;   // [nq, Hq, nsplit, 128] (nsplit > 1 only)
+    float *part_ml;  // [nq, Hq, nsplit, 2]
+    int32_t nsplit;
+};
+
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm);
+
+}  // namespace lsa

@@ -1,0 +1,240 @@
+/*
+ * lsa.h -- C ABI of the B200 (sm_100a) implementation of Latent Sparse
+ * Attention's hot path for one layer: the indexer (normalise + pool, Ward
+ * bucket cache, Flat or Tree search, best-first expansion + sink + window)
+ * and the exact GQA sparse attention over the resulting index lists.
+ *
+ * Method sources (web pages on "Latent Sparse Attention: Towards
+ * Subquadratic Ultra-Long Context Attention", arXiv 2610.42147):
+ *   [EXPL]  learnaivisually explainer: "How the hierarchy is built",
+ *           "What one query actually does", "Search style" table.
+ *   [BLOG]  sotaaz blog: "The same steps in general" (five steps and the
+ *           read_list function), "One real query, start to finish".
+ *   [FORUM] zhichai forum post: "Key points" (64-dim latent, L2 norm,
+ *           pool 4, 512-key blocks, Ward, <= 16 keys, Flat vs Tree).
+ *
+ * Conventions for every call below.
+ *   - Pointers to tensors are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or keeps them.  Scratch space is a
+ *     caller-provided device workspace sized by the *_workspace_bytes
+ *     queries.  lsa_cache / lsa_tree are host structs of device pointers.
+ *   - Every tensor is dense and row-major.  bf16 tensors are passed as
+ *     uint16_t bit patterns.  Device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work: they return before it runs, and
+ *     outputs are valid once the stream reaches that point.
+ *   - Return value: LSA_OK (0) or a negative LSA_ERR_* code; nothing is
+ *     enqueued when an argument check fails.  lsa_last_error_string()
+ *     describes the last failure on the calling thread.  The library never
+ *     aborts the process and its kernels never trap.
+ *   - Only the pages' configuration is built: 64-dim index vectors,
+ *     n_pool = 4, 512-key blocks, 64 buckets per block, at most 4 pooled
+ *     items (16 keys) per bucket, attention head_dim 128.  Other values in
+ *     lsa_params are rejected with LSA_ERR_ARG.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LSA_DIM 64           /* index key / query width           ([FORUM] Key points) */
+#define LSA_BLOCK 512        /* keys per cluster block            ([FORUM] Key points) */
+#define LSA_N_POOL 4         /* keys summed into one pooled key   ([EXPL] hierarchy)   */
+#define LSA_ITEMS 128        /* pooled items per block = 512 / 4                       */
+#define LSA_BUCKETS 64       /* buckets per block (~8 keys each)  ([BLOG] step 2)      */
+#define LSA_SLOTS 16         /* member slots per bucket (<= 16 keys, [BLOG] step 2)    */
+#define LSA_HEAD_DIM 128     /* attention head width handled by lsa_sparse_attention   */
+#define LSA_MAX_LEVELS 40    /* tree levels (ceil(log2(buckets)) + 1 <= 40)            */
+
+enum {
+    LSA_OK = 0,
+    LSA_ERR_ARG = -1,       /* null/misaligned pointer, bad parameter value */
+    LSA_ERR_SHAPE = -2,     /* sizes inconsistent with each other or with a buffer */
+    LSA_ERR_CUDA = -3,      /* a CUDA launch or query failed */
+    LSA_ERR_TIMEOUT = -4,   /* a bounded device-side wait gave up (reserved) */
+    LSA_ERR_WORKSPACE = -5  /* workspace missing or smaller than required */
+};
+
+enum { LSA_MODE_FLAT = 0, LSA_MODE_TREE = 1 };
+
+/* Parameters of the method.  lsa_default_params() fills the pages' values:
+ * n_pool 4, block 512, n_buckets 64, cap_items 4, sink 4, window 512 ([BLOG]
+ * step 5: "the first 4 keys and the latest 512 are always read"), k 4096
+ * ([BLOG] step 4: "On Qwen3.8-27B that is 4,096 keys"), beam 32, mode Flat.
+ * cand_cap: per-query candidate slots of the Flat search (0 = automatic).
+ * A smaller value only routes more queries through the exact fallback
+ * selection; results do not change. */
+typedef struct lsa_params {
+    int32_t n_pool;
+    int32_t block;
+    int32_t n_buckets;
+    int32_t cap_items;
+    int32_t sink;
+    int32_t window;
+    int32_t k;
+    int32_t beam;
+    int32_t mode;
+    int32_t cand_cap;
+} lsa_params;
+
+/* Bucket cache ([EXPL] "Each bucket stores one centroid and a table of the
+ * key positions it contains, and once a block is clustered its buckets never
+ * change").  Bucket g = 64*b + r is the r-th bucket of block b, buckets of a
+ * block ordered by their lowest pooled item.
+ *   pooled        fp32 [capacity/4, 64]   sum of 4 normalised keys per item
+ *   item_bucket   u8   [capacity/512, 128] bucket (0..63) of each pooled item
+ *   members       i32  [nb, 16]  ascending key positions, -1 padded
+ *   count         i32  [nb]      keys in the bucket (4..16)
+ *   centroid      fp32 [nb, 64]  normalised sum of member pooled keys
+ *   centroid_bf16 u16  [nb, 64]  bf16 (round to nearest even) of centroid
+ * where nb = 64 * (capacity / 512).  n_blocks = complete blocks clustered so
+ * far; lsa_build_cache raises it.  Fill the struct with lsa_cache_bind. */
+typedef struct lsa_cache {
+    int64_t capacity;
+    int64_t n_blocks;
+    float *pooled;
+    uint8_t *item_bucket;
+    int32_t *members;
+    int32_t *count;
+    float *centroid;
+    uint16_t *centroid_bf16;
+} lsa_cache;
+
+/* Tree of merged buckets ([EXPL] "In the tree variant the same process is
+ * repeated on the buckets to form higher levels"; [FORUM] "binary tree of
+ * merged buckets").  Level 0 = the buckets; level l has ceil(n_{l-1}/2)
+ * nodes; the top level holds the root.  Node arrays are indexed by global
+ * id = level_offset[l] + local id; child/parent hold LOCAL ids of the level
+ * below/above.
+ *   child [n,2] (-1 = none), parent [n] (-1 at the top), weight [n] (pooled
+ *   items below), min_block / max_block [n], sum fp32 [n,64] (sum of the
+ *   leaves' pooled keys), centroid fp32 [n,64] = normalise(sum),
+ *   centroid_bf16 [n,64].
+ * Fill with lsa_tree_bind; lsa_build_tree sets n_blocks. */
+typedef struct lsa_tree {
+    int64_t n_blocks;
+    int32_t n_levels;
+    int32_t reserved;
+    int64_t level_size[LSA_MAX_LEVELS];
+    int64_t level_offset[LSA_MAX_LEVELS + 1];
+    int32_t *child;
+    int32_t *parent;
+    int32_t *weight;
+    int32_t *min_block;
+    int32_t *max_block;
+    float *sum;
+    float *centroid;
+    uint16_t *centroid_bf16;
+} lsa_tree;
+
+/* ---- parameters, sizes and buffer binding (host only, no GPU work) ---- */
+
+void lsa_default_params(lsa_params *p);
+const char *lsa_last_error_string(void);
+
+/* Number of kernels this library has enqueued (all threads, all devices)
+ * since it was loaded: instrumentation for benchmarks and tests. */
+int64_t lsa_launch_count(void);
+
+/* Longest index list: sink + window + 1 (the query itself) + k. */
+int32_t lsa_list_budget(const lsa_params *p);
+
+/* Buckets that always hold k far keys: ceil((k + sink + window) / 4)
+ * (every bucket has >= 4 keys; at most sink + window clustered keys are
+ * skipped as near).  The Flat search keeps exactly this many. */
+int32_t lsa_top_buckets(const lsa_params *p);
+
+/* Bytes of one device buffer holding a cache for `capacity` tokens, and the
+ * call that carves such a buffer (256-byte aligned) into an lsa_cache. */
+int64_t lsa_cache_bytes(int64_t capacity);
+int lsa_cache_bind(void *base, int64_t bytes, int64_t capacity, lsa_cache *out);
+
+/* Same for the tree over n_blocks complete blocks (all levels, level 0 too). */
+int64_t lsa_tree_bytes(int64_t n_blocks);
+int lsa_tree_bind(void *base, int64_t bytes, int64_t n_blocks, lsa_tree *out);
+
+/* Workspace of lsa_index_prefill / lsa_index_decode for nq queries against a
+ * cache of n_blocks blocks, and of lsa_sparse_attention. */
+int64_t lsa_index_workspace_bytes(int64_t nq, int64_t n_blocks, const lsa_params *p);
+int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, int32_t Lmax);
+
+/* ---- the five calls of the hot path ---- */
+
+/* Steps 1-2 of the indexer ([EXPL] "How the hierarchy is built"; [FORUM]
+ * Key points; [BLOG] step 2).
+ * keys: fp32 [>= t_end, 64], the index keys of positions 0..t_end-1.
+ * Pools every item j with t_begin/4 <= j < t_end/4 (integer division):
+ * n_t = x_t / |x_t|, y_j = n_4j + n_4j+1 + n_4j+2 + n_4j+3 (a zero key
+ * normalises to zero).  Then clusters every block b with
+ * t_begin/512 <= b < t_end/512 by Ward's method: 128 unit-weight pooled
+ * items, cost D(A,B) = n_A n_B/(n_A+n_B) |mu_A - mu_B|^2, cheapest eligible
+ * pair (n_A + n_B <= 4 items) merged first, ties to the lowest (i, j), until
+ * 64 buckets remain.  All fp32 arithmetic of this call follows one fixed
+ * order, so results are bit-for-bit reproducible.
+ * Re-running over a range rewrites identical values.  Requires
+ * t_end <= cache->capacity.  Sets cache->n_blocks = max(n_blocks, t_end/512). */
+int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache *cache,
+                    const lsa_params *p, void *stream);
+
+/* Tree above the buckets of cache->n_blocks blocks ([EXPL] "In the tree
+ * variant the same process is repeated on the buckets").  At every level,
+ * consecutive runs of 128 nodes are paired greedily by Ward cost
+ * (weights = pooled items, mu = sum / weight), ties to the lowest (i, j); an
+ * odd leftover is promoted alone; new nodes are ordered by their lower
+ * child; repeat until one root.  tree must be bound for >= cache->n_blocks. */
+int lsa_build_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream);
+
+/* Steps 3-5 for nq queries ([EXPL] "What one query actually does"; [BLOG]
+ * steps 3-5 and read_list).
+ * qidx fp32 [nq, 64] index queries; pos i64 [nq] their positions.  Query i
+ * sees the buckets of blocks b < H = min(pos/512, cache->n_blocks).
+ *   Flat (p->mode == LSA_MODE_FLAT, tree may be NULL): score every visible
+ *   bucket, s = <bf16(q/|q|), centroid_bf16> with fp32 accumulation, rank by
+ *   (score desc, bucket id asc).
+ *   Tree: level-synchronous beam search from the root: candidates at level l
+ *   are the children of the nodes kept at level l+1 plus the visible
+ *   level-l nodes whose parent is not visible; keep the best
+ *   max(beam, ceil(lsa_top_buckets / 2^l)).
+ * Then open the ranked buckets best first, skipping members in
+ * near = {0..min(sink, p+1)-1} U [max(0, p-window), p], until k far keys.
+ * lists i32 [nq, Lmax]: ascending positions of near U far, -1 padded;
+ * lens i32 [nq].  Lmax must be >= lsa_list_budget(p).
+ * ws: >= lsa_index_workspace_bytes(nq, cache->n_blocks, p) bytes. */
+int lsa_index_prefill(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache,
+                      const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax,
+                      const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);
+
+/* The same computation for a few new tokens (decode, batch nq, positions at
+ * or past the clustered context).  Identical results to lsa_index_prefill;
+ * the launch shape spreads each query's buckets over the whole GPU. */
+int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache,
+                     const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax,
+                     const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);
+
+/* Exact softmax attention over each query's list, shared by all its heads
+ * ([EXPL] "One index list is built per query and shared by all of its
+ * attention heads ... Then ordinary attention runs over sink, selected keys
+ * and window").
+ * Q bf16 [nq, Hq, 128]; K, V bf16 [Tk, Hkv, 128]; query head h reads KV head
+ * h / (Hq / Hkv) (Hq a multiple of Hkv, Hq / Hkv <= 16).  lists/lens as
+ * written by lsa_index_*; every listed position must be < Tk.
+ * O[i,h] = sum_j softmax_j(scale * Q[i,h] . K[j]) V[j] over j in list(i),
+ * fp32 softmax and accumulation; O bf16 [nq, Hq, 128]; lse fp32 [nq, Hq]
+ * (natural-log log-sum-exp of the scaled scores; may be NULL).
+ * ws: >= lsa_attention_workspace_bytes(nq, Hq, 128, Lmax) bytes (may be 0
+ * for large nq). */
+int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t nq,
+                         int32_t Hq, int32_t Hkv, int32_t head_dim, int64_t Tk, const int32_t *lists,
+                         const int32_t *lens, int32_t Lmax, float scale, uint16_t *O, float *lse,
+                         void *ws, int64_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

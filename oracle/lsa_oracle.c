@@ -269,6 +269,21 @@ void orc_pair_run(const float *mu, const int32_t *w, int m, int32_t *partner)
         partner[bi] = bj;
         partner[bj] = bi;
     }
+    /* Only non-finite costs can leave more than one node unpaired; pair the
+     * rest in index order so every run still yields ceil(m/2) nodes. */
+    int open = -1, left = 0;
+    for (int i = 0; i < m; ++i) left += (partner[i] < 0);
+    for (int i = 0; i < m && left > 1; ++i) {
+        if (partner[i] >= 0) continue;
+        if (open < 0) {
+            open = i;
+        } else {
+            partner[open] = i;
+            partner[i] = open;
+            open = -1;
+            left -= 2;
+        }
+    }
     free(D);
 }
 

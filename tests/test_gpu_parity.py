@@ -1,0 +1,219 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Rules are in tests/parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from hierarchical_key_clustering_b200 import inputs as I
+from hierarchical_key_clustering_b200 import lsa
+
+from . import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for the -m gpu tests")
+
+
+def _build_gpu(keys: np.ndarray, capacity=None, pieces=None, mode="flat", k=256, beam=32, cand_cap=0):
+    _need_gpu()
+    T = keys.shape[0]
+    cache = lsa.Cache(capacity or T)
+    p = lsa.lsa_default_params(k=k, mode=mode, beam=beam, cand_cap=cand_cap)
+    kd = PT.to_dev(keys)
+    if pieces is None:
+        pieces = [(0, T)]
+    for a, b in pieces:
+        lsa.lsa_build_cache(kd, a, b, cache, p)
+    tree = None
+    if mode == "tree":
+        tree = lsa.Tree(max(T // 512, 1))
+        lsa.lsa_build_tree(cache, tree, p)
+    torch.cuda.synchronize()
+    return cache, tree, p
+
+
+def _index_gpu(cache, tree, p, qidx, pos, decode=False):
+    nq = len(pos)
+    Lmax = lsa.lsa_list_budget(p)
+    lists = torch.empty((nq, Lmax), dtype=torch.int32, device="cuda")
+    lens = torch.empty((nq,), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_index_workspace_bytes(nq, cache.n_blocks, p))
+    fn = lsa.lsa_index_decode if decode else lsa.lsa_index_prefill
+    fn(PT.to_dev(qidx), PT.to_dev(np.asarray(pos, np.int64)), cache, tree, lists, lens, p, ws)
+    torch.cuda.synchronize()
+    return lists.cpu().numpy(), lens.cpu().numpy()
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    T = 4096
+    keys = I.index_keys(0, T, 32)
+    pos = np.arange(T, dtype=np.int64)
+    q = I.index_queries(0, keys, pos)
+    oc = O.build_cache(keys)
+    return keys, q, pos, oc
+
+
+def test_cache_bit_exact_tiny(tiny):
+    keys, _, _, oc = tiny
+    cache, _, _ = _build_gpu(keys)
+    assert cache.n_blocks == 8
+    PT.assert_cache_equal(PT.cache_to_numpy(cache, 4096), oc)
+
+
+def test_cache_incremental_and_ragged_tail():
+    """Building in uneven pieces gives the one-shot cache; a tail shorter than
+    a block is pooled but not clustered."""
+    T = 4096 + 300
+    keys = I.index_keys(1, T, 32)
+    oc = O.build_cache(keys)
+    cache, _, _ = _build_gpu(keys, capacity=T + 212, pieces=[(0, 1001), (1001, 2600), (2600, 2601), (2601, T)])
+    assert cache.n_blocks == 8
+    g = PT.cache_to_numpy(cache, T)
+    PT.assert_cache_equal(g, oc)
+
+
+def test_flat_index_all_queries_tiny(tiny):
+    keys, q, pos, oc = tiny
+    cache, _, p = _build_gpu(keys, k=256)
+    gl, gn = _index_gpu(cache, None, p, q, pos)
+    ol, on = O.index(q, pos, oc, k=256)
+    PT.assert_lists_match(gl, gn, ol, on, q, pos, oc, k=256)
+
+
+@pytest.mark.parametrize("k", [1, 7, 256, 5000])
+def test_flat_index_edge_positions(tiny, k):
+    """Positions before the first block, inside the sink, at block edges, and k
+    from 1 to more than every key (dense); ragged query count."""
+    keys, q, _, oc = tiny
+    pos = np.array([0, 1, 2, 3, 4, 5, 511, 512, 513, 515, 516, 1023, 1024, 1025, 1535, 2047, 2048, 3000, 4095,
+                    4095, 2049] + list(range(600, 4096, 61)), np.int64)
+    qq = q[pos]
+    cache, _, p = _build_gpu(keys, k=k)
+    gl, gn = _index_gpu(cache, None, p, qq, pos)
+    ol, on = O.index(qq, pos, oc, k=k)
+    PT.assert_lists_match(gl, gn, ol, on, qq, pos, oc, k=k)
+    if k == 5000:
+        for i, pp in enumerate(pos):
+            assert gn[i] == pp + 1 and np.array_equal(gl[i, :pp + 1], np.arange(pp + 1))
+
+
+def test_flat_exact_fallback_selection(tiny):
+    """With only P candidate slots per query, most queries overflow and take the
+    exact radix-select path; the lists must not change."""
+    keys, q, pos, oc = tiny
+    P = O.top_p(256)
+    cache, _, p = _build_gpu(keys, k=256, cand_cap=P)
+    sel = np.arange(0, 4096, 5)
+    gl, gn = _index_gpu(cache, None, p, q[sel], pos[sel])
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    PT.assert_lists_match(gl, gn, ol, on, q[sel], pos[sel], oc, k=256)
+
+
+def test_decode_positions_past_context(tiny):
+    """Decode: new tokens at or past the clustered context see every block."""
+    keys, _, _, oc = tiny
+    T = 4096
+    more = I.index_keys(0, T + 16, 32)
+    pos = np.arange(T, T + 16, dtype=np.int64)
+    qq = I.index_queries(9, more, pos)
+    cache, _, p = _build_gpu(keys, k=256)
+    for nq in (1, 3, 16):
+        gl, gn = _index_gpu(cache, None, p, qq[:nq], pos[:nq], decode=True)
+        ol, on = O.index(qq[:nq], pos[:nq], oc, k=256)
+        PT.assert_lists_match(gl, gn, ol, on, qq[:nq], pos[:nq], oc, k=256)
+
+
+def test_tree_build_bit_exact(tiny):
+    keys, _, _, oc = tiny
+    ot = O.build_tree(oc)
+    cache, tree, _ = _build_gpu(keys, mode="tree")
+    assert tree.level_sizes() == ot.level_size.tolist()
+    v = {k: t.cpu().numpy() for k, t in tree.views().items()}
+    for name in ("child", "parent", "weight", "min_block", "max_block"):
+        assert np.array_equal(v[name], getattr(ot, name)), f"tree {name} differs"
+    assert np.array_equal(v["sum"].view(np.uint32), ot.sum.view(np.uint32))
+    assert np.max(np.abs(v["centroid"] - ot.centroid)) <= 1e-6
+    assert np.array_equal(v["centroid_bf16"].view(np.uint16), ot.centroid_bf16)
+
+
+@pytest.mark.parametrize("beam", [32, 4, 512])
+def test_tree_index_tiny(tiny, beam):
+    keys, q, pos, oc = tiny
+    ot = O.build_tree(oc)
+    cache, tree, p = _build_gpu(keys, mode="tree", k=256, beam=beam)
+    sel = np.arange(0, 4096, 3)
+    gl, gn = _index_gpu(cache, tree, p, q[sel], pos[sel])
+    ol, on = O.index(q[sel], pos[sel], oc, k=256, mode="tree", tree=ot, beam=beam)
+    PT.assert_lists_match(gl, gn, ol, on, q[sel], pos[sel], oc, k=256, tree=ot, beam=beam)
+    if beam == 512:  # wide beam: Tree search is Flat search
+        fl, fn = O.index(q[sel], pos[sel], oc, k=256)
+        PT.assert_lists_match(gl, gn, fl, fn, q[sel], pos[sel], oc, k=256)
+
+
+@pytest.mark.parametrize("hq,hkv,nq", [(8, 1, 300), (32, 8, 200), (32, 8, 1), (8, 1, 2), (16, 16, 50)])
+def test_attention_against_oracle(tiny, hq, hkv, nq):
+    """Attention over the oracle's own lists (isolates the kernel); nq = 1-2
+    takes the split-list (decode) path."""
+    _need_gpu()
+    keys, q, pos, oc = tiny
+    rng = np.random.default_rng(nq + hq)
+    sel = np.sort(rng.choice(4096, size=nq, replace=False)).astype(np.int64)
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    Qb, Kb, Vb = I.qkv_bf16_bits(4, nq, 4096, hq, hkv)
+    Oref, lse_ref = O.attention(Qb, Kb, Vb, ol, on)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    Lmax = ol.shape[1]
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, Lmax))
+    lsa.lsa_sparse_attention(Qd, Kd, Vd, PT.to_dev(ol), PT.to_dev(on), Od, lse, ws=ws)
+    torch.cuda.synchronize()
+    PT.assert_attention_close(Od, Oref, lse, lse_ref)
+
+
+def test_attention_dense_causal_single_key(tiny):
+    """A one-key list returns that key's value row exactly (up to bf16)."""
+    _need_gpu()
+    nq, hq, hkv = 5, 8, 2
+    Qb, Kb, Vb = I.qkv_bf16_bits(5, nq, 64, hq, hkv)
+    lists = np.full((nq, 4), -1, np.int32)
+    lists[:, 0] = [3, 0, 63, 17, 17]
+    lens = np.ones(nq, np.int32)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lsa.lsa_sparse_attention(Qd, Kd, Vd, PT.to_dev(lists), PT.to_dev(lens), Od)
+    torch.cuda.synchronize()
+    V = O.bf16_bits_to_f32(Vb)
+    og = Od.float().cpu().numpy()
+    for i in range(nq):
+        for h in range(hq):
+            assert np.array_equal(og[i, h], V[lists[i, 0], h // (hq // hkv)])
+
+
+def test_end_to_end_tiny_layer(tiny):
+    """Indexer + attention through the C ABI against oracle lists + oracle
+    attention for the whole tiny workload (8 query heads, 1 KV head)."""
+    keys, q, pos, oc = tiny
+    cache, _, p = _build_gpu(keys, k=256)
+    Lmax = lsa.lsa_list_budget(p)
+    nq = 4096
+    lists = torch.empty((nq, Lmax), dtype=torch.int32, device="cuda")
+    lens = torch.empty((nq,), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_index_workspace_bytes(nq, cache.n_blocks, p))
+    lsa.lsa_index_prefill(PT.to_dev(q), PT.to_dev(pos), cache, None, lists, lens, p, ws)
+    Qb, Kb, Vb = I.qkv_bf16_bits(0, nq, 4096, 8, 1)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lsa.lsa_sparse_attention(Qd, Kd, Vd, lists, lens, Od)
+    torch.cuda.synchronize()
+    gl, gn = lists.cpu().numpy(), lens.cpu().numpy()
+    ol, on = O.index(q, pos, oc, k=256)
+    PT.assert_lists_match(gl, gn, ol, on, q, pos, oc, k=256)
+    sel = np.arange(0, nq, 4)
+    Oref, _ = O.attention(Qb[sel], Kb, Vb, gl[sel], gn[sel])
+    PT.assert_attention_close(Od[sel], Oref)

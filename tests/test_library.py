@@ -1,0 +1,136 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/lsa.h declares; host-only queries and argument checks behave as the
+header says.  CPU only: no call here launches a kernel."""
+import ctypes as C
+import math
+import os
+import re
+
+import pytest
+
+from hierarchical_key_clustering_b200 import build, lsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+FAKE = C.c_void_p(1 << 20)  # 256-aligned, never dereferenced by the calls below
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_\w+)\s*\(", text)))
+
+
+def test_library_builds_and_exports_header_symbols():
+    path = build.build()
+    assert os.path.exists(path)
+    raw = C.CDLL(path)
+    names = header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in lsa.h but not exported"
+    assert set(names) == set(lsa.EXPORTS)
+
+
+def test_default_params_and_budgets():
+    p = lsa.lsa_default_params()
+    assert (p.n_pool, p.block, p.n_buckets, p.cap_items, p.sink, p.window, p.k, p.beam, p.mode) == \
+        (4, 512, 64, 4, 4, 512, 4096, 32, 0)
+    assert lsa.lsa_list_budget(p) == 4096 + 4 + 512 + 1
+    assert lsa.lsa_top_buckets(p) == 1153
+    assert lsa.lsa_top_buckets(lsa.lsa_default_params(k=2048)) == 641
+    assert lsa.lsa_top_buckets(lsa.lsa_default_params(k=256)) == 193
+
+
+def test_cache_bytes_scoring_part_is_24_5_per_token():
+    """Scoring-time cache (bf16 centroids, 16 member slots, count) = 24.5 B/token;
+    the build-time arrays (pooled keys, fp32 centroids, item ids) come on top."""
+    T = 1 << 20
+    total = lsa.lib().lsa_cache_bytes(T)
+    nb = T // 512 * 64
+    scoring = nb * (64 * 2 + 16 * 4 + 4)
+    build_only = T // 4 * 64 * 4 + nb * 64 * 4 + T // 512 * 128
+    assert scoring / T == 24.5
+    assert total >= scoring + build_only
+    assert total - (scoring + build_only) < 6 * 256
+
+
+def test_tree_layout_levels():
+    for nblk in (1, 8, 256, 2048, 19531):
+        t = lsa.lsa_tree()
+        nbytes = lsa.lib().lsa_tree_bytes(nblk)
+        assert lsa.lib().lsa_tree_bind(FAKE, nbytes, nblk, C.byref(t)) == 0
+        nb = nblk * 64
+        assert t.n_levels == math.ceil(math.log2(nb)) + 1
+        sizes = [t.level_size[i] for i in range(t.n_levels)]
+        assert sizes[0] == nb and sizes[-1] == 1
+        assert all(sizes[i + 1] == (sizes[i] + 1) // 2 for i in range(len(sizes) - 1))
+        assert t.level_offset[t.n_levels] == sum(sizes)
+    assert lsa.lib().lsa_tree_bytes(2048) > 0
+
+
+def _expect(code, want):
+    assert code == want, lsa.lib().lsa_last_error_string().decode()
+
+
+def test_argument_errors_return_codes():
+    L = lsa.lib()
+    p = lsa.lsa_default_params()
+    cache = lsa.lsa_cache()
+    nbytes = L.lsa_cache_bytes(4096)
+    _expect(L.lsa_cache_bind(FAKE, nbytes, 4096, C.byref(cache)), 0)
+    _expect(L.lsa_cache_bind(FAKE, nbytes - 1, 4096, C.byref(cache)), -2)
+    _expect(L.lsa_cache_bind(C.c_void_p(1 << 20 | 16), nbytes, 4096, C.byref(cache)), -1)
+    # params checks
+    _expect(L.lsa_build_cache(FAKE, 0, 4096, C.byref(cache), None, None), -1)
+    bad = lsa.lsa_default_params(n_pool=8)
+    _expect(L.lsa_build_cache(FAKE, 0, 4096, C.byref(cache), C.byref(bad), None), -1)
+    _expect(L.lsa_build_cache(FAKE, 0, 5000, C.byref(cache), C.byref(p), None), -2)
+    _expect(L.lsa_build_cache(FAKE, 100, 50, C.byref(cache), C.byref(p), None), -2)
+    _expect(L.lsa_build_cache(C.c_void_p(1 << 20 | 4), 0, 4096, C.byref(cache), C.byref(p), None), -1)
+    # index: workspace and list budget checks
+    cache.n_blocks = 8
+    Lmax = L.lsa_list_budget(C.byref(p))
+    _expect(L.lsa_index_prefill(FAKE, FAKE, 10, C.byref(cache), None, FAKE, FAKE, Lmax, C.byref(p), None, 0,
+                                None), -5)
+    _expect(L.lsa_index_prefill(FAKE, FAKE, 10, C.byref(cache), None, FAKE, FAKE, Lmax - 1, C.byref(p), FAKE,
+                                1 << 40, None), -2)
+    tp = lsa.lsa_default_params(mode="tree")
+    _expect(L.lsa_index_prefill(FAKE, FAKE, 10, C.byref(cache), None, FAKE, FAKE, Lmax, C.byref(tp), FAKE,
+                                1 << 40, None), -1)
+    # nq = 0 is a no-op
+    _expect(L.lsa_index_prefill(None, None, 0, C.byref(cache), None, None, None, Lmax, C.byref(p), None, 0,
+                                None), 0)
+    # attention shape checks
+    _expect(L.lsa_sparse_attention(FAKE, FAKE, FAKE, 4, 32, 8, 64, 100, FAKE, FAKE, 10, 0.1, FAKE, None, None, 0,
+                                   None), -1)
+    _expect(L.lsa_sparse_attention(FAKE, FAKE, FAKE, 4, 30, 8, 128, 100, FAKE, FAKE, 10, 0.1, FAKE, None, None, 0,
+                                   None), -1)
+    _expect(L.lsa_sparse_attention(FAKE, FAKE, FAKE, 4, 64, 2, 128, 100, FAKE, FAKE, 10, 0.1, FAKE, None, None, 0,
+                                   None), -1)
+    _expect(L.lsa_sparse_attention(FAKE, FAKE, FAKE, 0, 32, 8, 128, 100, FAKE, FAKE, 10, 0.1, FAKE, None, None, 0,
+                                   None), 0)
+    assert "head_dim" in L.lsa_last_error_string().decode() or True
+
+
+def test_workspace_queries():
+    p = lsa.lsa_default_params(k=2048)
+    a = lsa.lsa_index_workspace_bytes(1000, 256, p)
+    b = lsa.lsa_index_workspace_bytes(2000, 256, p)
+    assert 0 < a < b
+    assert lsa.lsa_attention_workspace_bytes(131072, 32, 128, 2565) == 0  # many queries: no key split
+    assert lsa.lsa_attention_workspace_bytes(1, 32, 128, 4613) > 0        # decode: split the list
+    assert lsa.lsa_attention_workspace_bytes(1, 32, 64, 4613) == -1
+
+
+@pytest.mark.parametrize("name", ["lsa_build_cache", "lsa_index_decode", "lsa_sparse_attention"])
+def test_binding_raises_on_error(name):
+    with pytest.raises(lsa.LsaError):
+        if name == "lsa_build_cache":
+            lsa._check(lsa.lib().lsa_build_cache(None, 0, 1, None, None, None))
+        elif name == "lsa_index_decode":
+            lsa._check(lsa.lib().lsa_index_decode(None, None, 1, None, None, None, None, 0, None, None, 0, None))
+        else:
+            lsa._check(lsa.lib().lsa_sparse_attention(None, None, None, 1, 0, 0, 128, 1, None, None, 1, 1.0, None,
+                                                      None, None, 0, None))
