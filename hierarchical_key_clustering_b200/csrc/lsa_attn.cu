@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     const int g = (int)(qg % a.Hkv);
     const int64_t q = qg / a.Hkv;
     const int G = a.Hq / a.Hkv;
-    const int len = a.lens[q];
+    const int len = min(a.lens[q], a.Lmax);
     const int begin = split * keys_per_split;
     const int end = min(len, begin + keys_per_split);
     const int nch = end > begin ? (end - begin + KCH - 1) / KCH : 0;
