@@ -267,6 +267,11 @@ void count_launches(int n)
 {
     g_launches.fetch_add(n, std::memory_order_relaxed);
 }
+
+int report_error(int code, const char *msg)
+{
+    return fail(code, "%s", msg);
+}
 }  // namespace lsa
 
 extern "C" {

@@ -58,7 +58,8 @@ class lsa_tree(C.Structure):
 EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
-           "lsa_build_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention"]
+           "lsa_build_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
+           "lsa_index_decode_static"]
 
 _lib = None
 
@@ -96,6 +97,7 @@ def lib():
             "lsa_build_tree": (C.c_int, [pc, pt, pp, P]),
             "lsa_index_prefill": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P, i64, P]),
             "lsa_index_decode": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P, i64, P]),
+            "lsa_index_decode_static": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P]),
             "lsa_sparse_attention": (C.c_int, [P, P, P, i64, i32, i32, i32, i64, P, P, i32, f32, P, P, P,
                                                i64, P]),
         }
@@ -265,6 +267,16 @@ def lsa_index_prefill(qidx, pos, cache: Cache, tree: Tree | None, lists, lens, p
 
 def lsa_index_decode(qidx, pos, cache: Cache, tree: Tree | None, lists, lens, p: lsa_params, ws, stream=None):
     _index(lib().lsa_index_decode, qidx, pos, cache, tree, lists, lens, p, ws, stream)
+
+
+def lsa_index_decode_static(qidx, pos, cache: Cache, tree: Tree | None, lists, lens, p: lsa_params, stream=None):
+    """lsa_index_decode with the library's fixed device scratch (no workspace)."""
+    _check(lib().lsa_index_decode_static(_ptr(qidx), _ptr(pos), qidx.shape[0], C.byref(cache.c),
+                                         C.byref(tree.t) if tree is not None else None, _ptr(lists), _ptr(lens),
+                                         lists.shape[1], C.byref(p), _stream(stream)))
+
+
+STATIC_SCRATCH_BYTES = 4 << 20
 
 
 def lsa_sparse_attention(Q, K, V, lists, lens, O, lse=None, scale=None, ws=None, stream=None):

@@ -233,6 +233,36 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
                          const int32_t *lens, int32_t Lmax, float scale, uint16_t *O, float *lse,
                          void *ws, int64_t ws_bytes, void *stream);
 
+/* ---- decode indexing without a caller workspace ---- */
+
+/* Size of the fixed device scratch array behind lsa_index_decode_static. */
+#define LSA_STATIC_SCRATCH_BYTES (4u << 20)
+
+/* lsa_index_decode for callers that cannot allocate device memory (an engine
+ * that has reserved all device memory up front and gives its plugins no
+ * allocator, a host program that only holds pointers handed to it, a decode
+ * loop that must never stall on a cudaMalloc/cudaFree).  The LSA pages have
+ * no counterpart: this is a deployment convenience, not part of the method.
+ *
+ * Same arguments, results and errors as lsa_index_decode, without ws and
+ * ws_bytes: the scratch is one file-scope device array of
+ * LSA_STATIC_SCRATCH_BYTES (4 MiB) that every GPU loading the library holds
+ * until the process exits.  The call allocates nothing.  Requests needing more
+ * than that (lsa_index_workspace_bytes(nq, cache->n_blocks, p) > 4 MiB; e.g.
+ * more than 58 Flat queries at k = 4096 over 10M tokens) are rejected with
+ * LSA_ERR_WORKSPACE and a message saying so; nothing is enqueued then.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and keeps it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the previous call's
+ * contents (every value the kernels read is written earlier in the same
+ * call); calls whose GPU work overlaps in time -- on different streams, or
+ * from several host threads -- race on it and must be serialised by the
+ * caller. */
+int lsa_index_decode_static(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache,
+                            const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax,
+                            const lsa_params *p, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
