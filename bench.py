@@ -157,7 +157,9 @@ def attn_algorithmic_bytes(lens: np.ndarray, hq: int, hkv: int) -> int:
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = I.WORKLOADS[args.workload]
+    wl = dict(I.WORKLOADS[args.workload])
+    if args.queries:
+        wl["n_prefill"] = min(args.queries, wl["n_prefill"])
     T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
     keys_np, q_np, pos_np = make_prefill_inputs(wl)
     layer = SparseLayer(T, k=wl["k"], mode=wl["mode"], beam=wl.get("beam", 32), max_queries=nq, Hq=hq)
@@ -224,6 +226,10 @@ def run_ours(args, world, rank, local):
     # end to end: same calls, inputs from pinned host memory, output back to host
     e2e = run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
 
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=args.cpu_budget)
+
     decode = None
     if not args.no_decode:
         del Q, K, V, O, flush
@@ -234,7 +240,8 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "T": T, "queries": nq, "k": wl["k"], "sink": 4, "window": 512,
+        "config": {"workload": args.workload if not args.queries else f"{args.workload}[last {nq} queries]",
+                   "T": T, "queries": nq, "k": wl["k"], "sink": 4, "window": 512,
                    "mode": wl["mode"], "Hq": hq, "Hkv": hkv, "head_dim": 128, "index_dim": 64,
                    "mixture_components": wl["n_components"], "parallelism": "replicas",
                    "l2": "256 MiB buffer written between timed steps; Q/K/V (1.6 GB) exceed L2"},
@@ -246,8 +253,8 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
         "decode": decode,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=args.cpu_budget)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -290,8 +297,11 @@ def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, dev, world):
 
 
 def run_decode(args, dev):
-    """Decode at T = 1M (Flat, k = 4096): batch-1 index_decode + attention per
-    new token, 64 tokens; mean us/token over the timed tokens."""
+    """Decode at T = 1M (Flat, k = 4096): per new token, batch 1, the index of
+    that token (lsa_index_decode) and its sparse attention.  The two calls are
+    captured once in a CUDA graph; each token copies its query into the
+    graph's input buffers and replays it (both inside the timed region).
+    Mean us/token over 64 tokens; the eager (uncaptured) figure is kept too."""
     wl = I.WORKLOADS["flat_1m"]
     T, nd, hq, hkv = wl["T"], wl["n_decode"], wl["hq"], wl["hkv"]
     keys_all = I.index_keys(0, T + nd, wl["n_components"])
@@ -306,23 +316,64 @@ def run_decode(args, dev):
     Qd = torch.randn((nd, 1, hq, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
     qd = torch.from_numpy(q_np).to(dev)
     pd = torch.from_numpy(pos_np).to(dev)
+    q_in, p_in, Q_in = qd[:1].clone(), pd[:1].clone(), Qd[0].clone()
     O = torch.empty((1, hq, 128), dtype=torch.bfloat16, device=dev)
-    st = torch.cuda.current_stream()
+
+    def token():
+        layer.index(q_in, p_in, decode=True)
+        layer.attend(Q_in, K, V, O)
+
+    def feed(i):
+        q_in.copy_(qd[i:i + 1])
+        p_in.copy_(pd[i:i + 1])
+        Q_in.copy_(Qd[i])
+
     for i in range(4):
-        layer.index(qd[i:i + 1], pd[i:i + 1], decode=True)
-        layer.attend(Qd[i], K, V, O)
+        feed(i)
+        token()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    e0, e1 = ev(), ev()
+    e0.record()
     for i in range(nd):
-        layer.index(qd[i:i + 1], pd[i:i + 1], decode=True)
-        layer.attend(Qd[i], K, V, O)
-    e1.record(st)
+        feed(i)
+        token()
+    e1.record()
     torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / nd
-    lens = layer.lens[:1].item()
-    return {"workload": "flat_1m", "T": T, "tokens": nd, "us_per_token": round(us, 2), "list_len": int(lens),
-            "note": "batch 1; index_decode + sparse attention per token, launched eagerly"}
+    eager_us = e0.elapsed_time(e1) * 1e3 / nd
+    lens = int(layer.lens[:1].item())
+    graph_us, note = None, None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            token()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            token()
+        for i in range(4):
+            feed(i)
+            graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for i in range(nd):
+            feed(i)
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        graph_us = e0.elapsed_time(e1) * 1e3 / nd
+    except Exception as ex:  # report, keep the eager number
+        note = f"graph capture failed: {type(ex).__name__}: {ex}"[:200]
+    out = {"workload": "flat_1m", "T": T, "tokens": nd, "k": wl["k"], "list_len": lens,
+           "us_per_token": round(graph_us if graph_us is not None else eager_us, 2),
+           "us_per_token_eager": round(eager_us, 2),
+           "note": "batch 1; lsa_index_decode + lsa_sparse_attention per token, replayed from one CUDA graph"}
+    if note:
+        out["note"] = note
+    return out
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -381,7 +432,8 @@ def run_reference(args, world, rank):
             "warmup": args.warmup, "ms_per_step": round(nq / v * 1e3, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": args.workload, "T": T, "queries": nq, "k": wl["k"], "mode": wl["mode"],
+            "config": {"workload": args.workload if not args.queries else f"{args.workload}[last {nq} queries]",
+                   "T": T, "queries": nq, "k": wl["k"], "mode": wl["mode"],
                        "Hq": hq, "Hkv": hkv, "head_dim": 128, "parallelism": "host cores"},
             "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": vals[-1]["cores"], "kind": "oracle",
                              "sample": vals[-1]["sample"]},
@@ -397,6 +449,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="flat_128k", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--queries", type=int, default=0,
+                    help="time only the last N prefill queries of the workload (profiling slices)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)

@@ -138,9 +138,10 @@ TreeLayout tree_layout(int64_t nblk)
 }
 
 struct IndexLayout {
-    int64_t off[7];
+    int64_t off[8];
     int64_t bytes;
     int64_t gstride;
+    int64_t sstride;
     int64_t cap;
 };
 
@@ -154,9 +155,12 @@ IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
     IndexLayout L;
     L.gstride = G;
     L.cap = cand_cap(p);
-    const int64_t sz[7] = {nq * LSA_DIM * 2, nq * 4, nq * 4, nq * 4, nq * G * 4, nq * L.cap * 4, nq * L.cap * 4};
+    // small batches (decode) keep every score for the filter pass
+    L.sstride = (nq <= lsa::SMALL_NQ && p->mode == LSA_MODE_FLAT) ? N : 0;
+    const int64_t sz[8] = {nq * LSA_DIM * 2, nq * 4, nq * 4, nq * 4, nq * G * 4, nq * L.cap * 4, nq * L.cap * 4,
+                           nq * L.sstride * 4};
     int64_t o = 0;
-    for (int i = 0; i < 7; ++i) {
+    for (int i = 0; i < 8; ++i) {
         L.off[i] = o;
         o += align256(sz[i]);
     }
@@ -164,15 +168,20 @@ IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
     return L;
 }
 
+// Key splits per query: about 2048 warps in flight for small batches (one
+// warp per (query, KV head, split)), at least 32 keys per split.
 int attention_nsplit(int64_t nq, int32_t Hkv, int32_t Lmax)
 {
     const int64_t units = nq * (int64_t)Hkv;
     if (units >= 2048) return 1;
     int64_t s = (2048 + units - 1) / units;
-    const int64_t chunks = (Lmax + 15) / 16;
+    const int64_t chunks = (Lmax + 31) / 32;
     if (s > chunks) s = chunks;
+    if (s > 1024) s = 1024;  // the merge kernel holds at most 1024 split weights
     return (int)(s < 1 ? 1 : s);
 }
+
+
 
 int64_t attention_ws_bytes(int64_t nq, int32_t Hq, int32_t nsplit)
 {
@@ -224,7 +233,9 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     iw.gmax = (float *)(w + L.off[4]);
     iw.cand_s = (float *)(w + L.off[5]);
     iw.cand_id = (int32_t *)(w + L.off[6]);
+    iw.scores = L.sstride ? (float *)(w + L.off[7]) : nullptr;
     iw.gmax_stride = L.gstride;
+    iw.score_stride = L.sstride;
     iw.cap = (int32_t)L.cap;
     lsa::IndexArgs a;
     a.qidx = qidx;

@@ -11,9 +11,17 @@
 // head[, key split]) unit: its G = Hq/Hkv heads form the rows of a 16-row
 // mma.sync tile (rows >= G are zero), 16 gathered keys form a chunk, and an
 // fp32 online softmax carries the running max and sum.  K/V rows are
-// gathered with cp.async into a 3-stage ring in shared memory.  A decode
-// query (few queries, long list) splits its list over many warps and a
-// second kernel merges the partial results by log-sum-exp.
+// gathered with cp.async (16 B per lane) into a 3-stage ring in shared
+// memory; each warp loads the list indices of the next chunk one issue ahead,
+// so a gather never waits on a dependent index load.  The warps of a CTA are
+// independent (no CTA barrier), which keeps many gathers in flight per SM.
+// A decode query (few queries, long list) splits its list over many warps
+// and a second kernel merges the partial results by log-sum-exp.
+//
+// Measured alternative (kept out): one CTA per query fetching each 2 KB
+// position row of all 8 KV heads with cp.async.bulk into an mbarrier ring was
+// 1.5x slower on the 128K workload -- one pipeline per SM hides latency worse
+// than eight independent warp pipelines.
 #include <cuda_bf16.h>
 
 #include "lsa_common.cuh"
@@ -115,10 +123,17 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
         qa[kk][3] = r0 + 8 < G ? ld_u32(Qb + (r0 + 8) * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
     }
 
-    auto load = [&](int ch, int st) {
+    int pre = -1;  // index of lane's row in the chunk issued next
+    auto fetch_idx = [&](int ch) {
         const int base = begin + ch * KCH;
-        int my = -1;
-        if (lane < KCH && base + lane < end) my = lst[base + lane];
+        int v = -1;
+        if (lane < KCH && ch < nch && base + lane < end) v = lst[base + lane];
+        return v;
+    };
+    pre = fetch_idx(0);
+    auto load = [&](int ch, int st) {
+        int my = pre;
+        pre = fetch_idx(ch + 1);
         if (my >= a.Tk) my = -1;  // out-of-range entries are read as zeros, never fetched
         const uint32_t sK = sbase + st * STAGE_BYTES;
         const uint32_t sV = sK + KCH * ROWB * 2;
@@ -272,34 +287,61 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     }
 }
 
-// Merge the partial results of the key splits of one (query, head): one warp.
-__global__ void __launch_bounds__(256) k_attn_combine(AttnArgs a)
+// Merge the partial results of the key splits of one (query, head): one
+// 512-thread CTA.  The split weights 2^(m_s - M) are computed once in shared
+// memory; then 4 groups of 128 threads (one per output dim) each sum a
+// quarter of the splits and the groups are added.
+constexpr int MAX_SPLIT = 1024;
+__global__ void __launch_bounds__(512) k_attn_combine(AttnArgs a)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t unit = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (unit >= a.nq * a.Hq) return;
+    __shared__ float wts[MAX_SPLIT];
+    __shared__ float red[16];
+    __shared__ float part[3][LSA_HEAD];
+    const int64_t unit = blockIdx.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float *ml = a.part_ml + unit * a.nsplit * 2;
     float M = __int_as_float(0xff800000);
-    for (int s = 0; s < a.nsplit; ++s)
+    for (int s = t; s < a.nsplit; s += blockDim.x)
         if (ml[2 * s + 1] > 0.0f) M = fmaxf(M, ml[2 * s]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(LSA_FULL, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = red[0];
+    for (int w = 1; w < 16; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
     float L = 0.0f;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int s = 0; s < a.nsplit; ++s) {
+    for (int s = t; s < a.nsplit; s += blockDim.x) {
         const float l = ml[2 * s + 1];
-        if (!(l > 0.0f)) continue;
-        const float w = exp2f(ml[2 * s] - M);
+        const float w = (l > 0.0f) ? exp2f(ml[2 * s] - M) : 0.0f;
+        wts[s] = w;
         L += l * w;
-        const float4 v = *reinterpret_cast<const float4 *>(a.part_o + (unit * a.nsplit + s) * LSA_HEAD + lane * 4);
-        acc[0] += v.x * w;
-        acc[1] += v.y * w;
-        acc[2] += v.z * w;
-        acc[3] += v.w * w;
     }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    uint16_t *Ob = a.O + unit * LSA_HEAD + lane * 4;
-    *reinterpret_cast<uint32_t *>(Ob) = pack_bf16(acc[0] * inv, acc[1] * inv);
-    *reinterpret_cast<uint32_t *>(Ob + 2) = pack_bf16(acc[2] * inv, acc[3] * inv);
-    if (lane == 0 && a.lse) a.lse[unit] = M * LN2 + logf(L);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(LSA_FULL, L, o);
+    if (lane == 0) red[warp] = L;
+    __syncthreads();
+    L = 0.0f;
+    for (int w = 0; w < 16; ++w) L += red[w];
+    const int d = t & (LSA_HEAD - 1), grp = t >> 7;
+    const float *po = a.part_o + unit * a.nsplit * LSA_HEAD + d;
+    float acc = 0.0f;
+#pragma unroll 4
+    for (int s = grp; s < a.nsplit; s += 4) acc += (wts[s] > 0.0f) ? po[(int64_t)s * LSA_HEAD] * wts[s] : 0.0f;
+    if (grp > 0) part[grp - 1][d] = acc;
+    __syncthreads();
+    if (grp == 0) {
+        acc += part[0][d] + part[1][d] + part[2][d];
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        __nv_bfloat16 v = __float2bfloat16_rn(acc * inv);
+        a.O[unit * LSA_HEAD + d] = *reinterpret_cast<uint16_t *>(&v);
+        if (d == 0 && a.lse) a.lse[unit] = M * LN2 + logf(L);
+    }
+}
+
+int attention_list_cap()
+{
+    return 1 << 30;  // the list is streamed, not staged: any length
 }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
@@ -317,8 +359,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.nsplit > 1) {
-        const int64_t warps = a.nq * a.Hq;
-        k_attn_combine<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(a);
+        k_attn_combine<<<(unsigned)(a.nq * a.Hq), 512, 0, st>>>(a);
         count_launches(1);
         e = cudaGetLastError();
     }

@@ -110,7 +110,11 @@ __device__ __forceinline__ int32_t rank_key_id(uint64_t k)
 }
 
 // Block-wide bitonic sort (ascending) of n = power of two keys in shared
-// memory.  All threads of the block must call it.
+// memory.  All threads of the block must call it.  Thread t owns the pairs
+// whose lower index is t modulo blockDim, so a 32-aligned group of keys is
+// always handled by one warp: consecutive stages with strides below 32 only
+// need a warp barrier, and a block barrier is paid only around the wider
+// strides.
 template <typename T>
 __device__ void block_bitonic_sort(T *a, int n)
 {
@@ -127,9 +131,15 @@ __device__ void block_bitonic_sort(T *a, int n)
                     }
                 }
             }
-            __syncthreads();
+            const int next_j = (j > 1) ? (j >> 1) : k;
+            if (j < 32 && next_j < 32 && !(j == 1 && k == n)) {
+                __syncwarp();
+            } else {
+                __syncthreads();
+            }
         }
     }
+    if (n <= 1) __syncthreads();
 }
 
 __host__ __device__ __forceinline__ int64_t pow2_ceil64(int64_t x)

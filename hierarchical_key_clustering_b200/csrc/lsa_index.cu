@@ -203,6 +203,91 @@ __global__ void __launch_bounds__(256) k_score(int64_t nq, int64_t nb_total, con
 }
 
 // ---------------------------------------------------------------------------
+// Flat passes for small batches (decode): one thread per bucket, the bucket's
+// bf16 row held in registers and scored against each query with the same
+// fp32 chain as dot_bf16_row.  Pass 1 stores every score and the group
+// maxima; pass 2 filters the stored scores against tau.
+template <int MODE>
+__global__ void __launch_bounds__(256) k_dscore(int64_t nq, int64_t nb_total, const uint16_t *__restrict__ cbf,
+                                                int P, IndexWs ws)
+{
+    __shared__ float qf[SMALL_NQ][LSA_D];
+    // the centroid tile (256 rows of 144 B) and, once every thread holds its
+    // row, the scores of the tile share one buffer
+    __shared__ uint4 rows[256 * 9];
+    float(*S)[256] = reinterpret_cast<float(*)[256]>(rows);
+    __shared__ int Nq[SMALL_NQ], gq[SMALL_NQ];
+    __shared__ float tq[SMALL_NQ];
+    const int t = threadIdx.x;
+    for (int i = t; i < nq * LSA_D; i += 256) qf[i >> 6][i & 63] = bf_bits2f(ws.qhat[i]);
+    if (t < nq) {
+        Nq[t] = ws.horizon[t] * LSA_NBKT;
+        gq[t] = group_width(Nq[t], P);
+        tq[t] = (MODE == MODE_FILTER) ? ws.tau[t] : 0.0f;
+    }
+    __syncthreads();
+    const int64_t b0 = (int64_t)blockIdx.x * 256;
+    const int64_t b = b0 + t;
+    if (MODE == MODE_GMAX) {
+        // 256 rows x 128 B read with fully coalesced 16-B loads into rows of
+        // 144 B (conflict-free 16-B reads), then each thread takes its row
+        const uint4 *src = reinterpret_cast<const uint4 *>(cbf + b0 * LSA_D);
+        const int64_t nvalid = min((int64_t)256, nb_total - b0) * 8;
+#pragma unroll
+        for (int k2 = 0; k2 < 8; ++k2) {
+            const int i = k2 * 256 + t;
+            rows[(i >> 3) * 9 + (i & 7)] = (i < nvalid) ? __ldcs(src + i) : make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
+        uint32_t row[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const uint4 w = rows[t * 9 + v];
+            row[4 * v] = w.x;
+            row[4 * v + 1] = w.y;
+            row[4 * v + 2] = w.z;
+            row[4 * v + 3] = w.w;
+        }
+        __syncthreads();  // the tile is consumed: its space now holds scores
+        for (int qi = 0; qi < nq; ++qi) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                acc = fmaf(qf[qi][2 * i], __uint_as_float(row[i] << 16), acc);
+                acc = fmaf(qf[qi][2 * i + 1], __uint_as_float(row[i] & 0xffff0000u), acc);
+            }
+            S[qi][t] = acc;
+            if (b < Nq[qi]) ws.scores[qi * ws.score_stride + b] = acc;
+        }
+        __syncthreads();
+        const float NEG = __int_as_float(0xff800000);
+        for (int qi = 0; qi < nq; ++qi) {
+            const int g = gq[qi];
+            const int N = Nq[qi];
+            for (int j = t; j < 256 / g; j += 256) {
+                const int64_t start = b0 + (int64_t)j * g;
+                if (start >= N) continue;
+                float m = NEG;
+                for (int e = 0; e < g && start + e < N; ++e) m = fmaxf(m, S[qi][j * g + e]);
+                ws.gmax[qi * ws.gmax_stride + start / g] = m;
+            }
+        }
+    } else {
+        for (int qi = 0; qi < nq; ++qi) {
+            if (b >= Nq[qi]) continue;
+            const float s = ws.scores[qi * ws.score_stride + b];
+            if (s >= tq[qi]) {
+                const int slot = atomicAdd(ws.cnt + qi, 1);
+                if (slot < ws.cap) {
+                    ws.cand_s[qi * ws.cap + slot] = s;
+                    ws.cand_id[qi * ws.cap + slot] = (int32_t)b;
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Radix select: the P-th largest key (u = f2ord(score)) among values produced
 // by `get(i)` for i in [0, n); all threads of the block call it.
 template <typename Get>
@@ -213,23 +298,43 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-            uint32_t u = f2ord(get(i));
-            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1);
+        const int64_t n_round = ((n + blockDim.x - 1) / blockDim.x) * blockDim.x;
+        for (int64_t i = threadIdx.x; i < n_round; i += blockDim.x) {
+            const bool valid = i < n;
+            const uint32_t u = valid ? f2ord(get(i)) : 0u;
+            const int bin = (valid && (u & mask) == prefix) ? (int)((u >> shift) & 255) : -1;
+            // lanes with the same bin add once (scores cluster in few bins)
+            const unsigned peers = __match_any_sync(LSA_FULL, bin);
+            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int64_t acc = 0;
-            int digit = 0;
-            for (int d = 255; d >= 0; --d) {
-                if (acc + hist[d] >= rem) {
-                    digit = d;
-                    break;
-                }
-                acc += hist[d];
+        if (threadIdx.x < 32) {
+            // warp 0: lane l owns bins 255-8l .. 248-8l (descending); find the
+            // bin where the count from the top first reaches rem
+            const int lane = threadIdx.x;
+            int c8 = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) c8 += hist[255 - 8 * lane - e];
+            int incl = c8;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(LSA_FULL, incl, o);
+                if (lane >= o) incl += y;
             }
-            sh[0] = digit;
-            sh[1] = (int)(rem - acc);
+            const int excl = incl - c8;
+            if (excl < rem && rem <= incl) {
+                int acc = excl, digit = 255 - 8 * lane;
+                for (int e = 0; e < 8; ++e) {
+                    const int d = 255 - 8 * lane - e;
+                    if (acc + hist[d] >= rem) {
+                        digit = d;
+                        break;
+                    }
+                    acc += hist[d];
+                }
+                sh[0] = digit;
+                sh[1] = (int)(rem - acc);
+            }
         }
         __syncthreads();
         prefix |= ((uint32_t)sh[0]) << shift;
@@ -241,8 +346,11 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
 }
 
 // Threshold per query: P-th largest group maximum (or -inf when N <= P).
-__global__ void __launch_bounds__(256) k_select(int64_t nq, int P, IndexWs ws)
+// The group maxima of one query are staged in shared memory first (one
+// round of independent loads), then the four radix passes run from there.
+__global__ void __launch_bounds__(1024) k_select(int64_t nq, int P, IndexWs ws)
 {
+    extern __shared__ float gsm[];
     __shared__ int hist[256];
     __shared__ int sh[2];
     const int64_t q = blockIdx.x;
@@ -253,7 +361,9 @@ __global__ void __launch_bounds__(256) k_select(int64_t nq, int P, IndexWs ws)
         return;
     }
     const float *gm = ws.gmax + q * ws.gmax_stride;
-    uint32_t u = block_select_kth_largest(G, P, [&](int64_t i) { return gm[i]; }, hist, sh);
+    for (int64_t i = threadIdx.x; i < G; i += blockDim.x) gsm[i] = gm[i];
+    __syncthreads();
+    uint32_t u = block_select_kth_largest(G, P, [&](int64_t i) { return gsm[i]; }, hist, sh);
     if (threadIdx.x == 0) ws.tau[q] = ord2f(u);
 }
 
@@ -417,70 +527,208 @@ __device__ void block_inclusive_scan(int *a, int n, int *wsum)
     __syncthreads();
 }
 
+// Weighted radix select over 64-bit rank keys (ascending = best first):
+// the smallest key K with sum of w over keys <= K reaching `target`, and the
+// weight still needed from K itself.  All threads of the block call it.
+__device__ void block_weighted_select(const uint64_t *keys, const int32_t *w, int n, int target, int *hist,
+                                      uint64_t *out_key, int *out_rem)
+{
+    __shared__ int sh_digit, sh_rem;
+    uint64_t prefix = 0, mask = 0;
+    int rem = target;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        const int n_round = ((n + blockDim.x - 1) / blockDim.x) * blockDim.x;
+        for (int i = threadIdx.x; i < n_round; i += blockDim.x) {
+            int bin = -1, wt = 0;
+            if (i < n && (keys[i] & mask) == prefix) {
+                bin = (int)((keys[i] >> shift) & 255);
+                wt = w[i];
+            }
+            const unsigned peers = __match_any_sync(LSA_FULL, bin);
+            const int sum = __reduce_add_sync(peers, wt);
+            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], sum);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {  // ascending bins: lane l owns 8l .. 8l+7
+            const int lane = threadIdx.x;
+            int c8 = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) c8 += hist[8 * lane + e];
+            int incl = c8;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(LSA_FULL, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int excl = incl - c8;
+            if (excl < rem && rem <= incl) {
+                int acc = excl;
+                for (int e = 0; e < 8; ++e) {
+                    const int d = 8 * lane + e;
+                    if (acc + hist[d] >= rem) {
+                        sh_digit = d;
+                        sh_rem = rem - acc;
+                        break;
+                    }
+                    acc += hist[d];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= (uint64_t)sh_digit << shift;
+        mask |= (uint64_t)255 << shift;
+        rem = sh_rem;
+        __syncthreads();
+    }
+    *out_key = prefix;
+    *out_rem = rem;
+}
+
 // Rank the candidates of one query and expand them into its index list.
-__global__ void __launch_bounds__(256) k_rank_expand(const int64_t *__restrict__ pos, const int32_t *__restrict__ members,
-                                                     const int32_t *__restrict__ count, int32_t *__restrict__ lists,
-                                                     int32_t *__restrict__ lens, int Lmax, int k, int sink,
-                                                     int window, int P, int SM, int FM, IndexWs ws)
+//   1. count each candidate bucket's members outside near (its weight);
+//   2. the walk over buckets in (score desc, id asc) order stops at the
+//      bucket where the weights reach k: find that bucket (and how many of
+//      its keys are still needed) by a weighted radix select -- buckets
+//      ranked before it are taken whole, their order does not matter;
+//   3. mark the chosen positions in one 512-bit mask per touched block
+//      (blocks found through a bitmap over all visible blocks) and emit them
+//      block by block in ascending order -- the far keys come out sorted
+//      without sorting them;
+//   4. write sink, far keys and window.
+// Every bucket has >= 4 keys and at most sink + window clustered keys are
+// near, so when a query has >= P candidates its best P buckets already hold
+// k far keys: the cut never falls outside the top P.
+__global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict__ pos, const int32_t *__restrict__ members,
+                                                     int32_t *__restrict__ lists, int32_t *__restrict__ lens, int Lmax,
+                                                     int k, int sink, int window, int P, int CAP, int TW, IndexWs ws)
 {
     extern __shared__ uint64_t rsm[];
-    uint64_t *keys = rsm;                                 // [SM]
-    int32_t *cum = reinterpret_cast<int32_t *>(keys + SM);  // [P]
-    int32_t *far = cum + P;                               // [FM]
-    __shared__ int wsum[8];
+    uint64_t *keys = rsm;                                        // [CAP]
+    int32_t *wt = reinterpret_cast<int32_t *>(keys + CAP);       // [CAP]
+    uint32_t *masks = reinterpret_cast<uint32_t *>(wt + CAP);    // [P][16]
+    uint32_t *touched = masks + (size_t)P * 16;                  // [TW]
+    int32_t *wrank = reinterpret_cast<int32_t *>(touched + TW);  // [TW]
+    int32_t *slot_blk = wrank + TW;                              // [P]
+    int32_t *slot_off = slot_blk + P;                            // [P]
+    __shared__ int wsum[32];
+    __shared__ int hist[256];
+    __shared__ int tot_s;
 
     const int64_t q = blockIdx.x;
     const int t = threadIdx.x;
     const int64_t p = pos[q];
     const int n = min(ws.cnt[q], ws.cap);
-    const int S = (int)pow2_ceil64(n > 0 ? n : 1);
-    for (int i = t; i < S; i += blockDim.x)
-        keys[i] = (i < n) ? rank_key(ws.cand_s[q * ws.cap + i], ws.cand_id[q * ws.cap + i]) : ~0ull;
-    __syncthreads();
-    block_bitonic_sort(keys, S);
-    const int n_take = min(n, P);
     const int64_t w0 = p - window > 0 ? p - window : 0;
     const int64_t s_end = (int64_t)sink < p + 1 ? (int64_t)sink : p + 1;
-    for (int r = t; r < n_take; r += blockDim.x) {
-        const int32_t b = rank_key_id(keys[r]);
-        const int c = count[b];
+    if (t == 0) tot_s = 0;
+    for (int i = t; i < TW; i += blockDim.x) touched[i] = 0u;
+    __syncthreads();
+    int my_tot = 0;
+    for (int i = t; i < n; i += blockDim.x) {
+        const int32_t b = ws.cand_id[q * ws.cap + i];
+        keys[i] = rank_key(ws.cand_s[q * ws.cap + i], b);
+        const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
         int nn = 0;
-        for (int e = 0; e < c; ++e) {
-            int64_t m = members[(int64_t)b * LSA_NSLOT + e];
-            nn += !(m < s_end || (m >= w0 && m <= p));
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int4 w = __ldg(m4 + v);
+            const int mm[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int64_t m = mm[e];  // -1 pads are skipped
+                nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
+            }
         }
-        cum[r] = nn;
+        wt[i] = nn;
+        my_tot += nn;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) my_tot += __shfl_xor_sync(LSA_FULL, my_tot, o);
+    if ((t & 31) == 0) atomicAdd(&tot_s, my_tot);
+    __syncthreads();
+    const int nfar = min(k, tot_s);
+    uint64_t cut_key = 0;
+    int take = 0;
+    if (nfar > 0) block_weighted_select(keys, wt, n, nfar, hist, &cut_key, &take);
+    const bool any = nfar > 0;
+    for (int i = t; i < n; i += blockDim.x) {
+        if (any && keys[i] <= cut_key && wt[i] > 0) {
+            const int blk = rank_key_id(keys[i]) / LSA_NBKT;
+            atomicOr(&touched[blk >> 5], 1u << (blk & 31));
+        }
     }
     __syncthreads();
-    block_inclusive_scan(cum, n_take, wsum);
-    const int total = n_take > 0 ? cum[n_take - 1] : 0;
-    const int nfar = min(k, total);
-    for (int r = t; r < n_take; r += blockDim.x) {
-        const int prev = r > 0 ? cum[r - 1] : 0;
-        if (prev >= nfar) continue;
-        const int32_t b = rank_key_id(keys[r]);
-        const int c = count[b];
-        int idx = prev;
-        for (int e = 0; e < c && idx < nfar; ++e) {
-            int64_t m = members[(int64_t)b * LSA_NSLOT + e];
-            if (!(m < s_end || (m >= w0 && m <= p))) far[idx++] = (int32_t)m;
+    for (int i = t; i < TW; i += blockDim.x) wrank[i] = __popc(touched[i]);
+    __syncthreads();
+    block_inclusive_scan(wrank, TW, wsum);  // wrank[w] = touched blocks in words 0..w
+    const int nslots = TW > 0 ? wrank[TW - 1] : 0;
+    for (int i = t; i < nslots * 16; i += blockDim.x) masks[i] = 0u;
+    __syncthreads();
+    for (int i = t; i < n; i += blockDim.x) {
+        if (!(any && keys[i] <= cut_key && wt[i] > 0)) continue;
+        const int32_t b = rank_key_id(keys[i]);
+        const int limit = (keys[i] == cut_key) ? take : 16;
+        const int blk = b / LSA_NBKT;
+        const uint32_t word = touched[blk >> 5];
+        const int slot = wrank[blk >> 5] - __popc(word) + __popc(word & ((1u << (blk & 31)) - 1u));
+        slot_blk[slot] = blk;
+        const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
+        int idx = 0;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int4 w = __ldg(m4 + v);
+            const int mm[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int64_t m = mm[e];
+                if (m >= 0 && !(m < s_end || (m >= w0 && m <= p))) {
+                    if (idx < limit) atomicOr(&masks[slot * 16 + ((m & 511) >> 5)], 1u << (m & 31));
+                    ++idx;
+                }
+            }
         }
     }
-    const int F = (int)pow2_ceil64(nfar > 0 ? nfar : 1);
-    for (int i = nfar + t; i < F; i += blockDim.x) far[i] = 0x7fffffff;
     __syncthreads();
-    block_bitonic_sort(far, F);
+    for (int sl = t; sl < nslots; sl += blockDim.x) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) c += __popc(masks[sl * 16 + w]);
+        slot_off[sl] = c;
+    }
+    __syncthreads();
+    block_inclusive_scan(slot_off, nslots, wsum);
     const int n_sink = (int)min(s_end, w0);
+    int32_t *out = lists + q * (int64_t)Lmax;
+    {
+        const int lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
+        for (int sl = warp; sl < nslots; sl += nwarps) {
+            const uint32_t word = lane < 16 ? masks[sl * 16 + lane] : 0u;
+            const int c = __popc(word);
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) {
+                const int y = __shfl_up_sync(LSA_FULL, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int o = n_sink + slot_off[sl] - __shfl_sync(LSA_FULL, incl, 15) + incl - c;
+            const int32_t base = slot_blk[sl] * LSA_BLK + lane * 32;
+            uint32_t bits = word;
+            while (bits) {
+                const int bit = __ffs(bits) - 1;
+                out[o++] = base + bit;
+                bits &= bits - 1;
+            }
+        }
+    }
     const int nwin = (int)(p - w0 + 1);
     const int len = n_sink + nfar + nwin;
-    int32_t *out = lists + q * (int64_t)Lmax;
     for (int i = t; i < Lmax; i += blockDim.x) {
-        int32_t v;
-        if (i < n_sink) v = i;
-        else if (i < n_sink + nfar) v = far[i - n_sink];
-        else if (i < len) v = (int32_t)(w0 + (i - n_sink - nfar));
-        else v = -1;
-        out[i] = v;
+        if (i < n_sink) out[i] = i;
+        else if (i < n_sink + nfar) continue;
+        else if (i < len) out[i] = (int32_t)(w0 + (i - n_sink - nfar));
+        else out[i] = -1;
     }
     if (t == 0) lens[q] = len;
 }
@@ -498,7 +746,24 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int64_t nb_total = a.n_blocks * LSA_NBKT;
-    if (a.mode == 0) {
+    const bool small = a.nq <= SMALL_NQ;
+    const int big_block = small ? 1024 : 256;
+    cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(ws.gmax_stride * 4));
+    if (a.mode == 0 && small && nb_total > 0) {
+        const unsigned blocks = (unsigned)((nb_total + 255) / 256);
+        k_dscore<MODE_GMAX><<<blocks, 256, 0, st>>>(a.nq, nb_total, a.centroid_bf16, a.P, ws);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_select<<<(unsigned)a.nq, big_block, (size_t)ws.gmax_stride * 4, st>>>(a.nq, a.P, ws);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_dscore<MODE_FILTER><<<blocks, 256, 0, st>>>(a.nq, nb_total, a.centroid_bf16, a.P, ws);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_fallback<<<(unsigned)a.nq, 256, 0, st>>>(a.nq, a.centroid_bf16, a.P, ws);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else if (a.mode == 0) {
         if (nb_total > 0) {
             const int64_t qtiles = (a.nq + SQ - 1) / SQ;
             const int64_t tiles = (nb_total + SB - 1) / SB;
@@ -516,7 +781,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
             k_score<MODE_GMAX><<<grid, 256, sm1, st>>>(a.nq, nb_total, a.centroid_bf16, chunk, a.P, ws);
             count_launches(1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            k_select<<<(unsigned)a.nq, 256, 0, st>>>(a.nq, a.P, ws);
+            k_select<<<(unsigned)a.nq, 256, (size_t)ws.gmax_stride * 4, st>>>(a.nq, a.P, ws);
             count_launches(1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             k_score<MODE_FILTER><<<grid, 256, sm2, st>>>(a.nq, nb_total, a.centroid_bf16, chunk, a.P, ws);
@@ -538,12 +803,12 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const int SMK = (int)pow2_ceil64(ws.cap);
-    const int FM = (int)pow2_ceil64(a.k > 0 ? a.k : 1);
-    const size_t smr = (size_t)SMK * sizeof(uint64_t) + (size_t)a.P * sizeof(int32_t) + (size_t)FM * sizeof(int32_t);
+    const int TW = (int)((a.n_blocks + 31) / 32) + 1;
+    const int nslot_max = a.P;  // touched blocks <= buckets taken <= P (the cut is within any P buckets)
+    const size_t smr = (size_t)ws.cap * (8 + 4) + (size_t)nslot_max * (64 + 4 + 4) + (size_t)TW * 8;
     cudaFuncSetAttribute(k_rank_expand, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-    k_rank_expand<<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.lists, a.lens, a.Lmax, a.k, a.sink,
-                                                   a.window, a.P, SMK, FM, ws);
+    k_rank_expand<<<(unsigned)a.nq, big_block, smr, st>>>(a.pos, a.members, a.lists, a.lens, a.Lmax, a.k, a.sink,
+                                                         a.window, nslot_max, ws.cap, TW, ws);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -40,9 +40,15 @@ struct IndexWs {
     float *gmax;        // [nq, gmax_stride] group maxima
     float *cand_s;      // [nq, cap] candidate scores
     int32_t *cand_id;   // [nq, cap] candidate bucket ids
+    float *scores;      // [nq, score_stride] stored scores (small batches only)
     int64_t gmax_stride;
+    int64_t score_stride;
     int32_t cap;
 };
+
+// Batches up to this many queries take the small-batch (decode) path:
+// thread-per-bucket scoring with stored scores.
+constexpr int SMALL_NQ = 16;
 
 cudaError_t launch_pool_norm(const float *keys, int64_t item_begin, int64_t item_end, float *pooled,
                              cudaStream_t st, int n_sm);
@@ -86,5 +92,6 @@ struct AttnArgs {
 };
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm);
+int attention_list_cap();
 
 }  // namespace lsa

@@ -276,7 +276,7 @@ def lsa_index_decode_static(qidx, pos, cache: Cache, tree: Tree | None, lists, l
                                          lists.shape[1], C.byref(p), _stream(stream)))
 
 
-STATIC_SCRATCH_BYTES = 4 << 20
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 def lsa_sparse_attention(Q, K, V, lists, lens, O, lse=None, scale=None, ws=None, stream=None):

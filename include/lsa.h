@@ -141,6 +141,7 @@ const char *lsa_last_error_string(void);
  * since it was loaded: instrumentation for benchmarks and tests. */
 int64_t lsa_launch_count(void);
 
+
 /* Longest index list: sink + window + 1 (the query itself) + k. */
 int32_t lsa_list_budget(const lsa_params *p);
 
@@ -226,8 +227,10 @@ int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const ls
  * O[i,h] = sum_j softmax_j(scale * Q[i,h] . K[j]) V[j] over j in list(i),
  * fp32 softmax and accumulation; O bf16 [nq, Hq, 128]; lse fp32 [nq, Hq]
  * (natural-log log-sum-exp of the scaled scores; may be NULL).
- * ws: >= lsa_attention_workspace_bytes(nq, Hq, 128, Lmax) bytes (may be 0
- * for large nq). */
+ * ws: >= lsa_attention_workspace_bytes(nq, Hq, 128, Lmax) bytes.  It holds
+ * the partial results when few queries split their lists over many warps
+ * (decode); with a smaller workspace (or none) fewer splits are used, with
+ * the same results. */
 int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t nq,
                          int32_t Hq, int32_t Hkv, int32_t head_dim, int64_t Tk, const int32_t *lists,
                          const int32_t *lens, int32_t Lmax, float scale, uint16_t *O, float *lse,
@@ -236,7 +239,7 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
 /* ---- decode indexing without a caller workspace ---- */
 
 /* Size of the fixed device scratch array behind lsa_index_decode_static. */
-#define LSA_STATIC_SCRATCH_BYTES (4u << 20)
+#define LSA_STATIC_SCRATCH_BYTES (16u << 20)
 
 /* lsa_index_decode for callers that cannot allocate device memory (an engine
  * that has reserved all device memory up front and gives its plugins no
@@ -246,11 +249,13 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
  *
  * Same arguments, results and errors as lsa_index_decode, without ws and
  * ws_bytes: the scratch is one file-scope device array of
- * LSA_STATIC_SCRATCH_BYTES (4 MiB) that every GPU loading the library holds
+ * LSA_STATIC_SCRATCH_BYTES (16 MiB) that every GPU loading the library holds
  * until the process exits.  The call allocates nothing.  Requests needing more
- * than that (lsa_index_workspace_bytes(nq, cache->n_blocks, p) > 4 MiB; e.g.
- * more than 58 Flat queries at k = 4096 over 10M tokens) are rejected with
- * LSA_ERR_WORKSPACE and a message saying so; nothing is enqueued then.
+ * than that (lsa_index_workspace_bytes(nq, cache->n_blocks, p) > 16 MiB) are
+ * rejected with LSA_ERR_WORKSPACE and a message saying so; nothing is
+ * enqueued then.  At k = 4096 this admits up to 240 Flat queries over 1M
+ * tokens; over 10M tokens it admits 1-3 or 17-233 queries (batches of 16 or
+ * fewer keep every bucket score, 5 MB per query at 10M).
  *
  * The first call on a device looks up the array's device address (with that
  * device current) and keeps it; make that first call before any stream

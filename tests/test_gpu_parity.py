@@ -114,14 +114,17 @@ def test_flat_exact_fallback_selection(tiny):
     PT.assert_lists_match(gl, gn, ol, on, q[sel], pos[sel], oc, k=256)
 
 
-def test_decode_positions_past_context(tiny):
-    """Decode: new tokens at or past the clustered context see every block."""
+@pytest.mark.parametrize("cand_cap", [0, 193])
+def test_decode_positions_past_context(tiny, cand_cap):
+    """Decode: new tokens at or past the clustered context see every block
+    (small batches take the stored-score path; cand_cap = P forces its exact
+    fallback selection)."""
     keys, _, _, oc = tiny
     T = 4096
     more = I.index_keys(0, T + 16, 32)
     pos = np.arange(T, T + 16, dtype=np.int64)
     qq = I.index_queries(9, more, pos)
-    cache, _, p = _build_gpu(keys, k=256)
+    cache, _, p = _build_gpu(keys, k=256, cand_cap=cand_cap)
     for nq in (1, 3, 16):
         gl, gn = _index_gpu(cache, None, p, qq[:nq], pos[:nq], decode=True)
         ol, on = O.index(qq[:nq], pos[:nq], oc, k=256)
@@ -217,3 +220,15 @@ def test_end_to_end_tiny_layer(tiny):
     sel = np.arange(0, nq, 4)
     Oref, _ = O.attention(Qb[sel], Kb, Vb, gl[sel], gn[sel])
     PT.assert_attention_close(Od[sel], Oref)
+
+
+def test_small_and_large_batch_paths_agree(tiny):
+    """Batches of up to 16 queries (decode path) and larger batches (prefill
+    path) give bit-identical lists for the same queries."""
+    keys, q, pos, _ = tiny
+    cache, _, p = _build_gpu(keys, k=256)
+    sel = np.arange(100, 4096, 97)[:40].astype(np.int64)
+    big_l, big_n = _index_gpu(cache, None, p, q[sel], pos[sel])
+    for a in range(0, len(sel), 8):
+        sl, sn = _index_gpu(cache, None, p, q[sel[a:a + 8]], pos[sel[a:a + 8]], decode=True)
+        assert np.array_equal(sn, big_n[a:a + 8]) and np.array_equal(sl, big_l[a:a + 8])
