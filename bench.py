@@ -41,9 +41,11 @@ from hierarchical_key_clustering_b200.layer import SparseLayer  # noqa: E402
 METRIC = "indexer+sparse-attn prefill tokens/s & decode us/token per layer; % roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes per listed (query, KV head, key) measured by ncu for k_attn at the
-# 128K workload (profiles/k_attn_flat_128k.md); None until captured.
-ATTN_DRAM_BYTES_PER_ROW = None
+# DRAM bytes per listed (query, KV head, key) row that ncu measured for k_attn on
+# the last 16384 queries of the 128K workload (profiles/k_attn_flat_128k.md);
+# roofline.traffic scales it by the rows of a full launch.  Re-measure when
+# k_attn changes.
+ATTN_DRAM_BYTES_PER_ROW = 318.0
 
 
 def peaks():
@@ -221,7 +223,8 @@ def run_ours(args, world, rank, local):
         traffic = int(ATTN_DRAM_BYTES_PER_ROW * int(lens_np.sum()) * hkv)
     roofline = {"kernel": "k_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
-                "peak_source": pk["src"], "algorithmic_bytes": abytes}
+                "peak_source": pk["src"], "algorithmic_bytes": abytes,
+                "traffic_note": "ncu DRAM bytes per listed row on a 16384-query slice, scaled to the launch"}
 
     # end to end: same calls, inputs from pinned host memory, output back to host
     e2e = run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
