@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblsa.so")
-SOURCES = ["lsa_api.cu", "lsa_build.cu", "lsa_index.cu", "lsa_attn.cu", "lsa_noalloc.cu"]
+SOURCES = ["lsa_api.cu", "lsa_build.cu", "lsa_index.cu", "lsa_score_tc.cu", "lsa_attn.cu", "lsa_noalloc.cu"]
 HEADERS = ["lsa_common.cuh", "lsa_kernels.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

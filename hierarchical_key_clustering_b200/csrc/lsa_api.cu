@@ -147,17 +147,13 @@ struct IndexLayout {
 
 IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
 {
-    const int64_t P = top_buckets(p);
     const int64_t N = nblk * LSA_BUCKETS;
-    int64_t G = lsa::n_groups(N, P);
-    if (G < 8 * P) G = 8 * P;  // groups of any smaller visible range never exceed this
-    if (p->mode == LSA_MODE_TREE) G = 1;
     IndexLayout L;
-    L.gstride = G;
+    L.gstride = lsa::HIST_BINS;  // group-maximum histogram per query
     L.cap = cand_cap(p);
     // small batches (decode) keep every score for the filter pass
     L.sstride = (nq <= lsa::SMALL_NQ && p->mode == LSA_MODE_FLAT) ? N : 0;
-    const int64_t sz[8] = {nq * LSA_DIM * 2, nq * 4, nq * 4, nq * 4, nq * G * 4, nq * L.cap * 4, nq * L.cap * 4,
+    const int64_t sz[8] = {nq * LSA_DIM * 2, nq * 4, nq * 4, nq * 4, nq * L.gstride * 4, nq * L.cap * 4, nq * L.cap * 4,
                            nq * L.sstride * 4};
     int64_t o = 0;
     for (int i = 0; i < 8; ++i) {
@@ -170,6 +166,11 @@ IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
 
 // Key splits per query: about 2048 warps in flight for small batches (one
 // warp per (query, KV head, split)), at least 32 keys per split.
+// Bounded device-side waits: tries per wait, and the test hook that makes one
+// wait run out (lsa_debug_wait_test).
+uint32_t g_wait_limit = 1u << 20;
+uint32_t g_extra_tx = 0;
+
 int attention_nsplit(int64_t nq, int32_t Hkv, int32_t Lmax)
 {
     const int64_t units = nq * (int64_t)Hkv;
@@ -230,11 +231,10 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     iw.horizon = (int32_t *)(w + L.off[1]);
     iw.tau = (float *)(w + L.off[2]);
     iw.cnt = (int32_t *)(w + L.off[3]);
-    iw.gmax = (float *)(w + L.off[4]);
+    iw.ghist = (uint32_t *)(w + L.off[4]);
     iw.cand_s = (float *)(w + L.off[5]);
     iw.cand_id = (int32_t *)(w + L.off[6]);
     iw.scores = L.sstride ? (float *)(w + L.off[7]) : nullptr;
-    iw.gmax_stride = L.gstride;
     iw.score_stride = L.sstride;
     iw.cap = (int32_t)L.cap;
     lsa::IndexArgs a;
@@ -254,6 +254,9 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     a.beam = p->beam;
     a.mode = p->mode;
     a.P = (int32_t)P;
+    a.wait_limit = g_wait_limit;
+    a.extra_tx = g_extra_tx;
+    g_extra_tx = 0;
     lsa::TreeView tv;
     const lsa::TreeView *tvp = nullptr;
     if (p->mode == LSA_MODE_TREE && cache->n_blocks > 0) {
@@ -290,6 +293,20 @@ extern "C" {
 int64_t lsa_launch_count(void)
 {
     return g_launches.load(std::memory_order_relaxed);
+}
+
+int lsa_check_device_errors(void)
+{
+    int v = lsa::read_device_error(1);
+    if (v < 0) return fail(LSA_ERR_CUDA, "could not read the device error word");
+    if (v) fail(LSA_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    return v;
+}
+
+void lsa_debug_wait_test(int32_t enable)
+{
+    g_extra_tx = enable ? 16u : 0u;
+    g_wait_limit = enable ? 1024u : (1u << 20);
 }
 
 void lsa_default_params(lsa_params *p)

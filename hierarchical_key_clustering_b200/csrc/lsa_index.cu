@@ -9,12 +9,14 @@
 // that follows it; zhichai forum post, "Key points" (Flat vs Tree).
 //
 // Flat selection.  A query that sees N buckets needs its top P buckets,
-// P = ceil((k + sink + window) / 4).  Pass 1 scores every bucket and keeps
-// only the maximum of each group of g consecutive buckets (g a power of two
-// giving 4P..8P groups).  The P-th largest group maximum is a score of P
-// distinct buckets, so it is <= the P-th largest score: every bucket scoring
-// at least that value is kept by pass 2, which recomputes the same scores
-// bit for bit and appends the passing (score, id) pairs.  A query whose
+// P = ceil((k + sink + window) / 4).  Pass 1 (tcgen05, lsa_score_tc.cu)
+// scores every bucket and histograms the maximum of each group of g
+// consecutive buckets (g a power of two giving 4P..8P groups).  The P-th
+// largest group maximum is a score of P distinct buckets, so it is <= the
+// P-th largest score, and so is tau, the lower edge of its histogram bin:
+// every bucket scoring at least tau is kept by pass 2, which recomputes the same scores
+// bit for bit on the tensor cores (or, for <= 16 queries, reads the scores
+// pass 1 stored) and appends the passing (score, id) pairs.  A query whose
 // candidates overflow their slots is redone exactly (radix select on the
 // recomputed scores) by the fallback kernel.  The candidates are then ranked
 // by (score desc, id asc) and expanded.
@@ -23,12 +25,6 @@
 
 namespace lsa {
 
-constexpr int SQ = 64;    // queries per score CTA
-constexpr int SB = 128;   // buckets per score tile
-constexpr int QS = 65;    // padded row (floats)
-constexpr int SS = 129;   // padded score row
-constexpr int MODE_GMAX = 0;
-constexpr int MODE_FILTER = 1;
 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, const int64_t *__restrict__ pos,
@@ -49,11 +45,14 @@ __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, c
             ws.horizon[q] = (int32_t)H;
             ws.cnt[q] = 0;
         }
+        for (int i = lane; i < HIST_BINS; i += 32) ws.ghist[q * HIST_BINS + i] = 0u;
     }
 }
 
-// Score of one bucket: fp32 FMA chain over d = 0..63 of the bf16 operands.
-// k_score, k_fallback and k_tree_beam all use this exact order.
+// Score of one bucket on the CUDA cores: fp32 FMA chain over d = 0..63 of the
+// bf16 operands (k_fallback and k_tree_beam).  It can differ from the tensor
+// cores' sum of the same products in the last bit, which only matters for
+// scores within ~1e-6 of each other.
 __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *__restrict__ c)
 {
     const uint4 *c4 = reinterpret_cast<const uint4 *>(c);
@@ -72,216 +71,27 @@ __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *_
 }
 
 // ---------------------------------------------------------------------------
-// Flat passes 1 and 2.  CTA = 64 queries x a chunk of buckets, 128-bucket
-// tiles, 256 threads each computing 4 queries x 8 buckets.
-template <int MODE>
-__global__ void __launch_bounds__(256) k_score(int64_t nq, int64_t nb_total, const uint16_t *__restrict__ cbf,
-                                               int64_t chunk, int P, IndexWs ws)
+// Flat pass 2 for small batches (decode): the tensor-core pass 1 stored every
+// score; keep those >= tau (one thread per bucket, all queries of the batch).
+__global__ void __launch_bounds__(256) k_dfilter(int64_t nq, IndexWs ws)
 {
-    extern __shared__ float sm[];
-    float *qf = sm;                    // [64][65]
-    float *cf = qf + SQ * QS;          // [128][65]
-    float *S = cf + SB * QS;           // [64][129] (pass 1 only)
-    __shared__ int Nq[SQ];
-    __shared__ int gq[SQ];
-    __shared__ float tq[SQ];
-    __shared__ int nmax_s;
-
-    const int t = threadIdx.x;
-    const int64_t q0 = (int64_t)blockIdx.x * SQ;
-    if (t == 0) nmax_s = 0;
-    __syncthreads();
-    if (t < SQ) {
-        int64_t q = q0 + t;
-        int N = (q < nq) ? ws.horizon[q] * LSA_NBKT : 0;
-        Nq[t] = N;
-        gq[t] = group_width(N, P);
-        tq[t] = (MODE == MODE_FILTER && q < nq) ? ws.tau[q] : 0.0f;
-        atomicMax(&nmax_s, N);
-    }
-    for (int i = t; i < SQ * LSA_D; i += 256) {
-        int r = i >> 6, d = i & 63;
-        int64_t q = q0 + r;
-        qf[r * QS + d] = (q < nq) ? bf_bits2f(ws.qhat[q * LSA_D + d]) : 0.0f;
-    }
-    __syncthreads();
-    const int64_t b_begin = (int64_t)blockIdx.y * chunk;
-    const int64_t b_end = min(b_begin + chunk, (int64_t)nmax_s);
-    const int ty = t >> 4, tx = t & 15;
-
-    for (int64_t tile = b_begin; tile < b_end; tile += SB) {
-        // centroid tile -> float smem (bf16 rows of 128 B, uint4 loads)
-        for (int i = t; i < SB * 8; i += 256) {
-            int r = i >> 3, v = i & 7;
-            int64_t b = tile + r;
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (b < nb_total) w = __ldg(reinterpret_cast<const uint4 *>(cbf + b * LSA_D) + v);
-            uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                cf[r * QS + v * 8 + 2 * h] = __uint_as_float(ww[h] << 16);
-                cf[r * QS + v * 8 + 2 * h + 1] = __uint_as_float(ww[h] & 0xffff0000u);
-            }
-        }
-        __syncthreads();
-        float acc[4][8];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[r][i] = 0.0f;
-#pragma unroll 4
-        for (int d = 0; d < LSA_D; ++d) {
-            float qv[4], cv[8];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) qv[r] = qf[(ty * 4 + r) * QS + d];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cv[i] = cf[(tx + 16 * i) * QS + d];
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[r][i] = fmaf(qv[r], cv[i], acc[r][i]);
-        }
-        if (MODE == MODE_GMAX) {
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) S[(ty * 4 + r) * SS + tx + 16 * i] = acc[r][i];
-            __syncthreads();
-            const int warp = t >> 5, lane = t & 31;
-            for (int qi = warp * 8; qi < warp * 8 + 8; ++qi) {
-                const int N = Nq[qi];
-                if (tile >= N) continue;  // warp-uniform
-                const int g = gq[qi];
-                const float NEG = __int_as_float(0xff800000);
-                float v[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    int64_t b = tile + lane * 4 + e;
-                    v[e] = (b < N) ? S[qi * SS + lane * 4 + e] : NEG;
-                }
-                float *gm = ws.gmax + (q0 + qi) * ws.gmax_stride;
-                if (g == 1) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        int64_t b = tile + lane * 4 + e;
-                        if (b < N) gm[b] = v[e];
-                    }
-                } else if (g == 2) {
-#pragma unroll
-                    for (int e = 0; e < 4; e += 2) {
-                        int64_t b = tile + lane * 4 + e;
-                        if (b < N) gm[b >> 1] = fmaxf(v[e], v[e + 1]);
-                    }
-                } else {
-                    float m = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
-                    for (int s = 1; s < (g >> 2); s <<= 1) m = fmaxf(m, __shfl_xor_sync(LSA_FULL, m, s));
-                    int64_t b = tile + lane * 4;
-                    if ((lane & ((g >> 2) - 1)) == 0 && b < N) gm[b / g] = m;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int qi = ty * 4 + r;
-                const int N = Nq[qi];
-                const float tau = tq[qi];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    int64_t b = tile + tx + 16 * i;
-                    if (b < N && acc[r][i] >= tau) {
-                        int slot = atomicAdd(ws.cnt + q0 + qi, 1);
-                        if (slot < ws.cap) {
-                            ws.cand_s[(q0 + qi) * ws.cap + slot] = acc[r][i];
-                            ws.cand_id[(q0 + qi) * ws.cap + slot] = (int32_t)b;
-                        }
-                    }
-                }
-            }
-        }
-        __syncthreads();
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Flat passes for small batches (decode): one thread per bucket, the bucket's
-// bf16 row held in registers and scored against each query with the same
-// fp32 chain as dot_bf16_row.  Pass 1 stores every score and the group
-// maxima; pass 2 filters the stored scores against tau.
-template <int MODE>
-__global__ void __launch_bounds__(256) k_dscore(int64_t nq, int64_t nb_total, const uint16_t *__restrict__ cbf,
-                                                int P, IndexWs ws)
-{
-    __shared__ float qf[SMALL_NQ][LSA_D];
-    // the centroid tile (256 rows of 144 B) and, once every thread holds its
-    // row, the scores of the tile share one buffer
-    __shared__ uint4 rows[256 * 9];
-    float(*S)[256] = reinterpret_cast<float(*)[256]>(rows);
-    __shared__ int Nq[SMALL_NQ], gq[SMALL_NQ];
+    __shared__ int Nq[SMALL_NQ];
     __shared__ float tq[SMALL_NQ];
     const int t = threadIdx.x;
-    for (int i = t; i < nq * LSA_D; i += 256) qf[i >> 6][i & 63] = bf_bits2f(ws.qhat[i]);
     if (t < nq) {
         Nq[t] = ws.horizon[t] * LSA_NBKT;
-        gq[t] = group_width(Nq[t], P);
-        tq[t] = (MODE == MODE_FILTER) ? ws.tau[t] : 0.0f;
+        tq[t] = ws.tau[t];
     }
     __syncthreads();
-    const int64_t b0 = (int64_t)blockIdx.x * 256;
-    const int64_t b = b0 + t;
-    if (MODE == MODE_GMAX) {
-        // 256 rows x 128 B read with fully coalesced 16-B loads into rows of
-        // 144 B (conflict-free 16-B reads), then each thread takes its row
-        const uint4 *src = reinterpret_cast<const uint4 *>(cbf + b0 * LSA_D);
-        const int64_t nvalid = min((int64_t)256, nb_total - b0) * 8;
-#pragma unroll
-        for (int k2 = 0; k2 < 8; ++k2) {
-            const int i = k2 * 256 + t;
-            rows[(i >> 3) * 9 + (i & 7)] = (i < nvalid) ? __ldcs(src + i) : make_uint4(0, 0, 0, 0);
-        }
-        __syncthreads();
-        uint32_t row[32];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const uint4 w = rows[t * 9 + v];
-            row[4 * v] = w.x;
-            row[4 * v + 1] = w.y;
-            row[4 * v + 2] = w.z;
-            row[4 * v + 3] = w.w;
-        }
-        __syncthreads();  // the tile is consumed: its space now holds scores
-        for (int qi = 0; qi < nq; ++qi) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                acc = fmaf(qf[qi][2 * i], __uint_as_float(row[i] << 16), acc);
-                acc = fmaf(qf[qi][2 * i + 1], __uint_as_float(row[i] & 0xffff0000u), acc);
-            }
-            S[qi][t] = acc;
-            if (b < Nq[qi]) ws.scores[qi * ws.score_stride + b] = acc;
-        }
-        __syncthreads();
-        const float NEG = __int_as_float(0xff800000);
-        for (int qi = 0; qi < nq; ++qi) {
-            const int g = gq[qi];
-            const int N = Nq[qi];
-            for (int j = t; j < 256 / g; j += 256) {
-                const int64_t start = b0 + (int64_t)j * g;
-                if (start >= N) continue;
-                float m = NEG;
-                for (int e = 0; e < g && start + e < N; ++e) m = fmaxf(m, S[qi][j * g + e]);
-                ws.gmax[qi * ws.gmax_stride + start / g] = m;
-            }
-        }
-    } else {
-        for (int qi = 0; qi < nq; ++qi) {
-            if (b >= Nq[qi]) continue;
-            const float s = ws.scores[qi * ws.score_stride + b];
-            if (s >= tq[qi]) {
-                const int slot = atomicAdd(ws.cnt + qi, 1);
-                if (slot < ws.cap) {
-                    ws.cand_s[qi * ws.cap + slot] = s;
-                    ws.cand_id[qi * ws.cap + slot] = (int32_t)b;
-                }
+    const int64_t b = (int64_t)blockIdx.x * 256 + t;
+    for (int qi = 0; qi < nq; ++qi) {
+        if (b >= Nq[qi]) continue;
+        const float s = ws.scores[qi * ws.score_stride + b];
+        if (s >= tq[qi]) {
+            const int slot = atomicAdd(ws.cnt + qi, 1);
+            if (slot < ws.cap) {
+                ws.cand_s[qi * ws.cap + slot] = s;
+                ws.cand_id[qi * ws.cap + slot] = (int32_t)b;
             }
         }
     }
@@ -346,25 +156,50 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
 }
 
 // Threshold per query: P-th largest group maximum (or -inf when N <= P).
-// The group maxima of one query are staged in shared memory first (one
-// round of independent loads), then the four radix passes run from there.
-__global__ void __launch_bounds__(1024) k_select(int64_t nq, int P, IndexWs ws)
+// Threshold per query from its global group-maximum histogram (used when a
+// query's buckets were split over several score CTAs): tau = lower edge of
+// the bin holding the P-th largest group maximum, -inf when there are <= P
+// groups.  One warp per query.
+__global__ void __launch_bounds__(256) k_tau(int64_t nq, int P, IndexWs ws)
 {
-    extern __shared__ float gsm[];
-    __shared__ int hist[256];
-    __shared__ int sh[2];
-    const int64_t q = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (q >= nq) return;
     const int64_t N = (int64_t)ws.horizon[q] * LSA_NBKT;
-    const int64_t G = n_groups(N, P);
-    if (G <= P) {
-        if (threadIdx.x == 0) ws.tau[q] = __int_as_float(0xff800000);
+    const float NEG = __int_as_float(0xff800000);
+    if (n_groups(N, P) <= P) {
+        if (lane == 0) ws.tau[q] = NEG;
         return;
     }
-    const float *gm = ws.gmax + q * ws.gmax_stride;
-    for (int64_t i = threadIdx.x; i < G; i += blockDim.x) gsm[i] = gm[i];
-    __syncthreads();
-    uint32_t u = block_select_kth_largest(G, P, [&](int64_t i) { return gsm[i]; }, hist, sh);
-    if (threadIdx.x == 0) ws.tau[q] = ord2f(u);
+    // lane l owns bins 255-8l .. 248-8l (descending)
+    const uint32_t *h = ws.ghist + q * HIST_BINS;
+    int c8 = 0;
+    int cb[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        cb[e] = (int)h[HIST_BINS - 1 - 8 * lane - e];
+        c8 += cb[e];
+    }
+    int incl = c8;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(LSA_FULL, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int excl = incl - c8;
+    if (excl < P && P <= incl) {
+        int acc = excl;
+        int bin = HIST_BINS - 1 - 8 * lane;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            acc += cb[e];
+            if (acc >= P) {
+                bin = HIST_BINS - 1 - 8 * lane - e;
+                break;
+            }
+        }
+        ws.tau[q] = bin > 0 ? HIST_LO + bin * (2.0f * -HIST_LO / HIST_BINS) : NEG;
+    }
 }
 
 // Exact selection for queries whose candidates overflowed: radix select of
@@ -748,50 +583,39 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     const int64_t nb_total = a.n_blocks * LSA_NBKT;
     const bool small = a.nq <= SMALL_NQ;
     const int big_block = small ? 1024 : 256;
-    cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(ws.gmax_stride * 4));
-    if (a.mode == 0 && small && nb_total > 0) {
-        const unsigned blocks = (unsigned)((nb_total + 255) / 256);
-        k_dscore<MODE_GMAX><<<blocks, 256, 0, st>>>(a.nq, nb_total, a.centroid_bf16, a.P, ws);
-        count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        k_select<<<(unsigned)a.nq, big_block, (size_t)ws.gmax_stride * 4, st>>>(a.nq, a.P, ws);
-        count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        k_dscore<MODE_FILTER><<<blocks, 256, 0, st>>>(a.nq, nb_total, a.centroid_bf16, a.P, ws);
-        count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        k_fallback<<<(unsigned)a.nq, 256, 0, st>>>(a.nq, a.centroid_bf16, a.P, ws);
-        count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    } else if (a.mode == 0) {
-        if (nb_total > 0) {
-            const int64_t qtiles = (a.nq + SQ - 1) / SQ;
-            const int64_t tiles = (nb_total + SB - 1) / SB;
-            int64_t chunks = ((int64_t)n_sm * 8 + qtiles - 1) / qtiles;
-            if (chunks > tiles) chunks = tiles;
-            if (chunks < 1) chunks = 1;
-            if (chunks > 65535) chunks = 65535;
-            const int64_t chunk = ((tiles + chunks - 1) / chunks) * SB;
-            chunks = (nb_total + chunk - 1) / chunk;
-            const size_t sm1 = sizeof(float) * (SQ * QS + SB * QS + SQ * SS);
-            const size_t sm2 = sizeof(float) * (SQ * QS + SB * QS);
-            cudaFuncSetAttribute(k_score<MODE_GMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-            cudaFuncSetAttribute(k_score<MODE_FILTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-            dim3 grid((unsigned)qtiles, (unsigned)chunks);
-            k_score<MODE_GMAX><<<grid, 256, sm1, st>>>(a.nq, nb_total, a.centroid_bf16, chunk, a.P, ws);
-            count_launches(1);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            k_select<<<(unsigned)a.nq, 256, (size_t)ws.gmax_stride * 4, st>>>(a.nq, a.P, ws);
-            count_launches(1);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            k_score<MODE_FILTER><<<grid, 256, sm2, st>>>(a.nq, nb_total, a.centroid_bf16, chunk, a.P, ws);
-            count_launches(1);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            int64_t fb = a.nq < (int64_t)n_sm * 2 ? a.nq : (int64_t)n_sm * 2;
-            k_fallback<<<(unsigned)fb, 256, 0, st>>>(a.nq, a.centroid_bf16, a.P, ws);
+    if (a.mode == 0 && nb_total > 0) {
+        // pass 1 on the tensor cores: group maxima (+ every score for small batches)
+        ScoreTcArgs sa;
+        sa.nq = a.nq;
+        sa.nb_total = nb_total;
+        sa.P = a.P;
+        sa.mode = 0;
+        sa.store = small ? 1 : 0;
+        sa.chunk_tiles = 0;
+        sa.wait_limit = a.wait_limit;
+        sa.extra_tx = a.extra_tx;
+        int whole = 0;
+        if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, &whole)) != cudaSuccess) return e;
+        if (!whole) {  // thresholds from the merged histograms
+            k_tau<<<(unsigned)((a.nq + 7) / 8), 256, 0, st>>>(a.nq, a.P, ws);
             count_launches(1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
+        if (small) {  // pass 2 from the stored scores
+            const unsigned blocks = (unsigned)((nb_total + 255) / 256);
+            k_dfilter<<<blocks, 256, 0, st>>>(a.nq, ws);
+            count_launches(1);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        } else {  // pass 2 on the tensor cores: recompute the same scores, keep those >= tau
+            sa.mode = 1;
+            sa.store = 0;
+            sa.extra_tx = 0;
+            if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, nullptr)) != cudaSuccess) return e;
+        }
+        const int64_t fb = small ? a.nq : (a.nq < (int64_t)n_sm * 2 ? a.nq : (int64_t)n_sm * 2);
+        k_fallback<<<(unsigned)fb, 256, 0, st>>>(a.nq, a.centroid_bf16, a.P, ws);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else if (tree && tree->n_levels > 0) {
         int64_t B1 = ((int64_t)a.P + 1) / 2;
         if (B1 < a.beam) B1 = a.beam;

@@ -37,14 +37,18 @@ struct IndexWs {
     int32_t *horizon;   // [nq] visible blocks
     float *tau;         // [nq] Flat threshold
     int32_t *cnt;       // [nq] candidates written
-    float *gmax;        // [nq, gmax_stride] group maxima
+    uint32_t *ghist;    // [nq, HIST_BINS] group-maximum histograms (split ranges)
     float *cand_s;      // [nq, cap] candidate scores
     int32_t *cand_id;   // [nq, cap] candidate bucket ids
     float *scores;      // [nq, score_stride] stored scores (small batches only)
-    int64_t gmax_stride;
     int64_t score_stride;
     int32_t cap;
 };
+
+// Histogram of group maxima used to set the Flat threshold: HIST_BINS linear
+// bins over [HIST_LO, -HIST_LO] (scores of unit bf16 vectors lie inside).
+constexpr int HIST_BINS = 256;
+constexpr float HIST_LO = -1.0625f;
 
 // Batches up to this many queries take the small-batch (decode) path:
 // thread-per-bucket scoring with stored scores.
@@ -72,7 +76,28 @@ struct IndexArgs {
     int32_t Lmax;
     int32_t k, sink, window, beam, mode;
     int32_t P;  // top buckets kept
+    uint32_t wait_limit;  // tries per bounded device-side wait
+    uint32_t extra_tx;    // test hook (see lsa_debug_wait_test)
 };
+
+// Flat scoring on the tensor cores (lsa_score_tc.cu).  mode 0: threshold
+// histogram of group maxima (+ every score when store != 0); mode 1: append
+// scores >= tau.
+struct ScoreTcArgs {
+    int64_t nq;
+    int64_t nb_total;
+    int32_t P;
+    int32_t mode;
+    int32_t store;
+    int32_t whole_range;  // set by the launcher: one CTA covers each query's buckets
+    int64_t chunk_tiles;
+    uint32_t wait_limit;  // tries per bounded mbarrier wait
+    uint32_t extra_tx;    // test hook: non-zero skips the query-tile copy, so its barrier never completes
+};
+
+cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint16_t *centroid_bf16, cudaStream_t st,
+                            int n_sm, int *whole_range);
+int read_device_error(int clear);
 
 cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *tree, cudaStream_t st, int n_sm);
 

@@ -1,0 +1,491 @@
+// Flat search scores on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Method: Latent Sparse Attention pages -- learnaivisually explainer, "What
+// one query actually does" (the normalised query is scored against every
+// bucket centroid of the earlier cluster blocks); zhichai forum post, "Key
+// points" (Flat search scores all bucket centroids, ~T/8 per query).
+//
+// S = Q^ C^T is a dense 64-deep contraction: a CTA owns a tile of 128 queries
+// (the MMA M) and streams 256-centroid tiles (the MMA N) of its bucket range.
+//   warp 0        TMA producer: the query tile once, centroid tiles into a
+//                 4-stage ring (128B-swizzled, K-major), mbarrier completion;
+//   warp 1        allocates 512 TMEM columns; one thread issues
+//                 tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32, 4 x K=16) into
+//                 one of two 128 x 256 fp32 accumulators, and commits to the
+//                 stage's "empty" barrier and the accumulator's "full" one;
+//   warps 2..5    epilogue: thread r owns TMEM lane r = query q0 + r and reads
+//                 its 256 scores with tcgen05.ld, 32 columns at a time, while
+//                 the other accumulator is being filled.
+// The epilogue is fused with the pass's work, so the score matrix is never
+// stored (except, for batches of <= 16 queries, one row per query):
+//   GMAX    the maximum of each group of g consecutive buckets goes into the
+//           row's 256-bin histogram over [-1.0625, 1.0625] in shared memory
+//           (and, for small batches, every score is stored for the filter
+//           pass).  A CTA that covers the query's whole bucket range turns
+//           the histogram into the threshold tau itself: tau = lower edge of
+//           the bin that holds the P-th largest group maximum, a value <= the
+//           P-th largest group maximum <= the P-th largest score.  Otherwise
+//           the rows are added into a global per-query histogram and
+//           k_tau finishes;
+//   FILTER  append every score >= the query's threshold tau.
+// Causal masking: bucket b counts for query q only if b < 64 * H(q).
+// Every mbarrier wait is bounded: a wait that runs out sets the library's
+// device error word and the CTA leaves its loops, waits (bounded) for the
+// copies it issued, frees its TMEM and exits.
+#include <cuda.h>
+
+#include "lsa_common.cuh"
+#include "lsa_kernels.h"
+
+namespace lsa {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int TQ = 128;             // queries per tile (MMA M)
+constexpr int TB = 256;             // centroids per tile (MMA N)
+constexpr int NST = 4;              // centroid stages
+constexpr uint32_t A_BYTES = TQ * LSA_D * 2;   // 16 KB
+constexpr uint32_t B_BYTES = TB * LSA_D * 2;   // 32 KB
+constexpr int TMEM_COLS = 512;      // two 256-column fp32 accumulators
+constexpr int THREADS = 192;        // 6 warps
+constexpr int HSTRIDE = HIST_BINS / 2 + 1;  // 32-bit words per row histogram (2 x u16 bins per word, +1 pad)
+constexpr uint32_t HIST_BYTES = TQ * HSTRIDE * 4;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait; on expiry sets the device error word and the CTA abort flag.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit, volatile int *abort)
+{
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort) return false;
+    }
+    atomicExch(&g_device_error, 1);
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
+            "r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 B,
+// 8-row groups 1024 B apart (sm_100 descriptor format, version 1).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3fffu);          // start address
+    d |= (uint64_t)1 << 16;                           // leading byte offset (unused for SW128 K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset
+    d |= (uint64_t)1 << 46;                           // descriptor version
+    d |= (uint64_t)2 << 61;                           // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t IDESC = (1u << 4)               // D format fp32
+                           | (1u << 7)             // A bf16
+                           | (1u << 10)            // B bf16
+                           | ((uint32_t)(TB >> 3) << 17)
+                           | ((uint32_t)(TQ >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct TcSmem {
+    uint64_t full[NST];
+    uint64_t empty[NST];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t a_full;
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort;
+    int nmax;
+};
+
+}  // namespace
+
+// grid: x = query tile, y = bucket-tile chunk.  block = 192 threads.
+__global__ void __launch_bounds__(THREADS, 1)
+    k_score_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, ScoreTcArgs a,
+               IndexWs ws)
+{
+    extern __shared__ __align__(1024) uint8_t tsm_raw[];
+    // tiles first (1024-aligned for the 128B swizzle), control block after
+    uint8_t *tsm = tsm_raw + ((1024u - (smem_u32(tsm_raw) & 1023u)) & 1023u);
+    uint8_t *sA = tsm;
+    uint8_t *sB = tsm + A_BYTES;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(tsm + A_BYTES + NST * B_BYTES);  // [TQ][HSTRIDE]
+    TcSmem *cs = reinterpret_cast<TcSmem *>(tsm + A_BYTES + NST * B_BYTES + HIST_BYTES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t q0 = (int64_t)blockIdx.x * TQ;
+
+    if (threadIdx.x == 0) {
+        cs->nmax = 0;
+        cs->abort = 0;
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(smem_u32(&cs->full[s]), 1);
+            mbar_init(smem_u32(&cs->empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&cs->tfull[b]), 1);
+            mbar_init(smem_u32(&cs->tempty[b]), 4);
+        }
+        mbar_init(smem_u32(&cs->a_full), 1);
+        mbar_init(smem_u32(&cs->mma_done), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x < TQ) {
+        const int64_t q = q0 + threadIdx.x;
+        const int N = (q < a.nq) ? ws.horizon[q] * LSA_NBKT : 0;
+        atomicMax(&cs->nmax, N);
+    }
+    __syncthreads();
+    const int64_t tiles_all = ((int64_t)cs->nmax + TB - 1) / TB;
+    const int64_t j0 = (int64_t)blockIdx.y * a.chunk_tiles;
+    const int64_t j1 = min(j0 + a.chunk_tiles, tiles_all);
+    const int ntiles = j1 > j0 ? (int)(j1 - j0) : 0;
+    if (ntiles == 0) return;  // uniform: nothing allocated yet
+
+    volatile int *abort = &cs->abort;
+    if (warp == 1) {  // whole warp: TMEM allocation
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_u32(&cs->tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = cs->tmem_base;
+
+    int issued = 0;  // producer: centroid tiles issued
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmB) : "memory");
+        const uint32_t abar = smem_u32(&cs->a_full);
+        mbar_expect_tx(abar, A_BYTES);
+        if (a.extra_tx == 0) tma_load_2d(smem_u32(sA), &tmA, 0, (int)q0, abar);  // test hook: never arrives
+        for (int it = 0; it < ntiles; ++it) {
+            const int s = it % NST;
+            if (it >= NST && !wait_bounded(smem_u32(&cs->empty[s]), (uint32_t)(((it / NST) - 1) & 1), a.wait_limit,
+                                           abort))
+                break;
+            const uint32_t bar = smem_u32(&cs->full[s]);
+            mbar_expect_tx(bar, B_BYTES);
+            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, 0, (int)((j0 + it) * TB), bar);
+            ++issued;
+        }
+    } else if (warp == 1 && lane == 0) {
+        if (wait_bounded(smem_u32(&cs->a_full), 0, a.wait_limit, abort)) {
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA);
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % NST, buf = it & 1;
+                if (!wait_bounded(smem_u32(&cs->full[s]), (uint32_t)((it / NST) & 1), a.wait_limit, abort)) break;
+                if (it >= 2 &&
+                    !wait_bounded(smem_u32(&cs->tempty[buf]), (uint32_t)(((it >> 1) - 1) & 1), a.wait_limit, abort))
+                    break;
+                tc_fence_after();
+                const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
+                const uint32_t d = tmem + (uint32_t)(buf * TB);
+#pragma unroll
+                for (int k = 0; k < LSA_D / 16; ++k)
+                    mma_bf16(d, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), k > 0 ? 1u : 0u);
+                mma_commit(smem_u32(&cs->empty[s]));
+                mma_commit(smem_u32(&cs->tfull[buf]));
+            }
+        }
+    } else if (warp >= 2) {
+        // epilogue: thread owns TMEM lane (query row) r
+        const int sub = warp & 3;
+        const int r = sub * 32 + lane;
+        const int64_t q = q0 + r;
+        const int N = (q < a.nq) ? ws.horizon[q] * LSA_NBKT : 0;
+        const int g = group_width(N, a.P);
+        const float tau = (a.mode == 1 && q < a.nq) ? ws.tau[q] : 0.0f;
+        const float NEG = __int_as_float(0xff800000);
+        uint32_t *hrow = hist + r * HSTRIDE;
+        if (a.mode == 0)
+            for (int w = 0; w < HSTRIDE; ++w) hrow[w] = 0u;
+        // count one group maximum in the row histogram (saturating u16 bins)
+        auto count = [&](float m) {
+            int bin = __float2int_rd((m - HIST_LO) * (HIST_BINS / (2.0f * -HIST_LO)));
+            bin = min(max(bin, 0), HIST_BINS - 1);
+            const uint32_t w = hrow[bin >> 1];
+            const uint32_t sh = (bin & 1) * 16;
+            if (((w >> sh) & 0xffffu) != 0xffffu) hrow[bin >> 1] = w + (1u << sh);
+        };
+        float *sc = (a.store && q < a.nq) ? ws.scores + q * ws.score_stride : nullptr;
+        int own = 0;  // candidates this thread appended (FILTER)
+        for (int it = 0; it < ntiles; ++it) {
+            const int buf = it & 1;
+            const bool ok = wait_bounded(smem_u32(&cs->tfull[buf]), (uint32_t)((it >> 1) & 1), a.wait_limit, abort);
+            if (!__all_sync(LSA_FULL, ok)) break;  // warp-uniform: tcgen05.ld needs the whole warp
+            tc_fence_after();
+            const int64_t tb0 = (j0 + it) * TB;
+            float run = NEG;  // running maximum of a 64- or 128-bucket group
+#pragma unroll 1
+            for (int c = 0; c < TB / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + (uint32_t)(buf * TB + c * 32), v);
+                const int64_t b0 = tb0 + c * 32;
+                // N is a multiple of 64, so a 32-bucket chunk is wholly in or out
+                if (b0 >= N) continue;
+                if (a.mode == 0) {
+                    if (sc) {
+                        float4 *dst = reinterpret_cast<float4 *>(sc + b0);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                    if (g == 1) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) count(v[i]);
+                        continue;
+                    }
+                    // in-place max tree: after level L, v[i] (i a multiple of 2^L)
+                    // holds the maximum of buckets i .. i + 2^L - 1 of the chunk
+#pragma unroll
+                    for (int L = 1; L <= 5; ++L) {
+                        const int w = 1 << L;
+#pragma unroll
+                        for (int i = 0; i < 32; i += w) v[i] = fmaxf(v[i], v[i + w / 2]);
+                        if (w == g) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += w) count(v[i]);
+                        }
+                    }
+                    if (g > 32) {
+                        run = fmaxf(run, v[0]);
+                        const int per = g / 32;  // 2 or 4 chunks per group
+                        if ((c % per) == per - 1 || b0 + 32 >= N) {
+                            count(run);
+                            run = NEG;
+                        }
+                    }
+                } else {
+                    // count the chunk's candidates first, then reserve their
+                    // slots at once (no atomic when this CTA owns the query)
+                    int n = 0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) n += (v[i] >= tau);
+                    if (n) {
+                        int slot = a.whole_range ? own : atomicAdd(ws.cnt + q, n);
+                        own += n;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            if (v[i] >= tau) {
+                                if (slot < ws.cap) {
+                                    ws.cand_s[q * ws.cap + slot] = v[i];
+                                    ws.cand_id[q * ws.cap + slot] = (int32_t)(b0 + i);
+                                }
+                                ++slot;
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&cs->tempty[buf]));
+        }
+        if (a.mode == 1 && a.whole_range && q < a.nq) ws.cnt[q] = own;
+        if (a.mode == 0 && q < a.nq && N > 0 && !*abort) {
+            if (a.whole_range) {
+                // this CTA saw every bucket of the query: threshold from the histogram
+                const int64_t G = n_groups(N, a.P);
+                float t = NEG;
+                if (G > a.P) {
+                    int acc = 0;
+                    for (int bin = HIST_BINS - 1; bin > 0; --bin) {
+                        acc += (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
+                        if (acc >= a.P) {
+                            t = HIST_LO + bin * (2.0f * -HIST_LO / HIST_BINS);
+                            break;
+                        }
+                    }
+                }
+                ws.tau[q] = t;
+            } else {
+                uint32_t *gh = ws.ghist + q * HIST_BINS;
+                for (int bin = 0; bin < HIST_BINS; ++bin) {
+                    const uint32_t c = (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
+                    if (c) atomicAdd(gh + bin, c);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0 && lane == 0 && *abort) {
+        // copies issued but never consumed: wait for them (bounded) before exit
+        volatile int dummy = 0;
+        for (int it = 0; it < issued; ++it)
+            wait_bounded(smem_u32(&cs->full[it % NST]), (uint32_t)((it / NST) & 1), a.wait_limit, &dummy);
+    }
+    if (warp == 1 && lane == 0) {
+        // every MMA this thread issued has finished before its TMEM is freed
+        volatile int dummy = 0;
+        mma_commit(smem_u32(&cs->mma_done));
+        wait_bounded(smem_u32(&cs->mma_done), 0, a.wait_limit, &dummy);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch.
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Rows of 64 bf16 (128 B), box = box_rows x 64, 128B swizzle; rows past the
+// end read as zero.
+static bool make_map(CUtensorMap *m, const void *base, int64_t rows, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)LSA_D, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)LSA_D * 2};
+    cuuint32_t box[2] = {(cuuint32_t)LSA_D, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint16_t *centroid_bf16, cudaStream_t st,
+                            int n_sm, int *whole_range)
+{
+    if (a.nq <= 0 || a.nb_total <= 0) return cudaSuccess;
+    CUtensorMap tmA, tmB;
+    if (!make_map(&tmA, ws.qhat, a.nq, TQ) || !make_map(&tmB, centroid_bf16, a.nb_total, TB))
+        return cudaErrorInvalidValue;
+    const int64_t qtiles = (a.nq + TQ - 1) / TQ;
+    const int64_t tiles = (a.nb_total + TB - 1) / TB;
+    int64_t chunks = qtiles == 1 ? n_sm : (2LL * n_sm + qtiles - 1) / qtiles;
+    if (qtiles >= n_sm) chunks = 1;  // one CTA per query tile covers its whole range
+    if (chunks > tiles) chunks = tiles;
+    if (chunks < 1) chunks = 1;
+    if (chunks > 65535) chunks = 65535;
+    ScoreTcArgs b = a;
+    b.chunk_tiles = (tiles + chunks - 1) / chunks;
+    chunks = (tiles + b.chunk_tiles - 1) / b.chunk_tiles;
+    b.whole_range = (chunks == 1) ? 1 : 0;
+    if (whole_range) *whole_range = b.whole_range;
+    const size_t smem = A_BYTES + NST * B_BYTES + HIST_BYTES + sizeof(TcSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_score_tc<<<dim3((unsigned)qtiles, (unsigned)chunks), THREADS, smem, st>>>(tmA, tmB, b, ws);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+int read_device_error(int clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_device_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+}  // namespace lsa

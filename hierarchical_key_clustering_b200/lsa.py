@@ -55,7 +55,8 @@ class lsa_tree(C.Structure):
                 ("centroid", C.c_void_p), ("centroid_bf16", C.c_void_p)]
 
 
-EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_list_budget", "lsa_top_buckets",
+EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_check_device_errors",
+           "lsa_debug_wait_test", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
            "lsa_build_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
@@ -85,6 +86,8 @@ def lib():
             "lsa_default_params": (None, [pp]),
             "lsa_last_error_string": (C.c_char_p, []),
             "lsa_launch_count": (i64, []),
+            "lsa_check_device_errors": (C.c_int, []),
+            "lsa_debug_wait_test": (None, [i32]),
             "lsa_list_budget": (i32, [pp]),
             "lsa_top_buckets": (i32, [pp]),
             "lsa_cache_bytes": (i64, [i64]),
@@ -145,6 +148,15 @@ def lsa_default_params(**overrides) -> lsa_params:
 
 def lsa_launch_count() -> int:
     return lib().lsa_launch_count()
+
+
+def lsa_check_device_errors() -> int:
+    """0 if no bounded device-side wait ran out since the last check (clears it)."""
+    return lib().lsa_check_device_errors()
+
+
+def lsa_debug_wait_test(enable: bool):
+    lib().lsa_debug_wait_test(1 if enable else 0)
 
 
 def lsa_list_budget(p: lsa_params) -> int:

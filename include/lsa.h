@@ -141,6 +141,23 @@ const char *lsa_last_error_string(void);
  * since it was loaded: instrumentation for benchmarks and tests. */
 int64_t lsa_launch_count(void);
 
+/* Device-side failure detection.  Every wait inside a kernel (the mbarrier
+ * phases of the tensor-core score kernel's copy ring and accumulators) gives
+ * up after a bounded number of tries instead of spinning forever; one that
+ * gives up sets an error word on the device, and the kernel leaves its loops,
+ * waits (bounded) for the copies it issued, frees its tensor memory and
+ * exits, so the context stays usable.  lsa_check_device_errors() waits for
+ * the current device to go idle, reads and clears that word: 0 = no wait ran
+ * out, 1 = one did (outputs of that call are invalid and
+ * lsa_last_error_string() says so), < 0 = CUDA error.
+ * lsa_debug_wait_test(1) is a test hook: in the next lsa_index_* call in
+ * Flat mode every score CTA skips its query-tile copy, so the barrier that
+ * waits for it never completes, and waits are cut to a short limit; the error
+ * path then runs without hanging or faulting the GPU.
+ * lsa_debug_wait_test(0) restores the normal limit. */
+int lsa_check_device_errors(void);
+void lsa_debug_wait_test(int32_t enable);
+
 
 /* Longest index list: sink + window + 1 (the query itself) + k. */
 int32_t lsa_list_budget(const lsa_params *p);
