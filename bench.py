@@ -42,10 +42,11 @@ METRIC = "indexer+sparse-attn prefill tokens/s & decode us/token per layer; % ro
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per listed (query, KV head, key) row that ncu measured for k_attn on
-# the last 16384 queries of the 128K workload (dram__bytes_read.sum 106.86 GB
-# over 16384 x 2565 x 8 rows); roofline.traffic scales it by the rows of a full
-# launch.  Re-measure when k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = 318.0
+# the last 16384 queries of the 128K workload (dram__bytes_read.sum 7.17 GB over
+# 16384 x 2565 x 8 rows; head-major order keeps each head's K/V in L2);
+# roofline.traffic scales it by the rows of a full launch.  Re-measure when
+# k_attn changes.
+ATTN_DRAM_BYTES_PER_ROW = 21.3
 
 
 def peaks():

@@ -15,6 +15,9 @@
 // memory; each warp loads the list indices of the next chunk one issue ahead,
 // so a gather never waits on a dependent index load.  The warps of a CTA are
 // independent (no CTA barrier), which keeps many gathers in flight per SM.
+// Units run head-major (all queries of KV head 0, then head 1, ...): the K/V
+// rows of one head are 1/Hkv of the cache, so at 128K tokens (67 MB per
+// head) the rows that queries share stay in L2.
 // A decode query (few queries, long list) splits its list over many warps
 // and a second kernel merges the partial results by log-sum-exp.
 //
@@ -100,10 +103,12 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     const int64_t unit = (int64_t)blockIdx.x * AWARPS + warp;
     const int64_t total = a.nq * a.Hkv * a.nsplit;
     if (unit >= total) return;
+    // head-major order: the warps in flight all read one KV head, whose rows
+    // (Tk x 512 B of K+V) stay resident in L2 while its queries run
     const int split = (int)(unit % a.nsplit);
     const int64_t qg = unit / a.nsplit;
-    const int g = (int)(qg % a.Hkv);
-    const int64_t q = qg / a.Hkv;
+    const int g = (int)(qg / a.nq);
+    const int64_t q = qg % a.nq;
     const int G = a.Hq / a.Hkv;
     const int len = min(a.lens[q], a.Lmax);
     const int begin = split * keys_per_split;
@@ -224,12 +229,14 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
         l1 = l1 * al1 + rs1;
         m0 = mn0;
         m1 = mn1;
+        if (al0 != 1.0f || al1 != 1.0f) {  // the running max moved: rescale O
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            o[nt][0] *= al0;
-            o[nt][1] *= al0;
-            o[nt][2] *= al1;
-            o[nt][3] *= al1;
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][0] *= al0;
+                o[nt][1] *= al0;
+                o[nt][2] *= al1;
+                o[nt][3] *= al1;
+            }
         }
         uint32_t pa[4];
         pa[0] = pack_bf16(s[0][0], s[0][1]);
