@@ -11,7 +11,8 @@ of all 131072 queries, and sparse attention for all of them.
 value = prefill tokens (queries) per second, whole job.
 
 Also reported: decode us/token at T = 1,048,576 (index_decode + attention
-for 64 new tokens, batch 1), the roofline of the dominant kernel, the
+for 64 new tokens, batch 1; for the 1M and 10M workloads, at their own T),
+the roofline of the dominant kernel, the
 oracle's CPU time on a bounded sample, and an end-to-end number through the
 same C-ABI calls with inputs copied from pinned host memory every step and
 the output copied back.
@@ -163,6 +164,10 @@ def run_ours(args, world, rank, local):
     wl = dict(I.WORKLOADS[args.workload])
     if args.queries:
         wl["n_prefill"] = min(args.queries, wl["n_prefill"])
+    if args.mode:
+        wl["mode"] = args.mode
+    if wl["mode"] == "both":
+        wl["mode"] = "flat"
     T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
     keys_np, q_np, pos_np = make_prefill_inputs(wl)
     layer = SparseLayer(T, k=wl["k"], mode=wl["mode"], beam=wl.get("beam", 32), max_queries=nq, Hq=hq)
@@ -228,7 +233,7 @@ def run_ours(args, world, rank, local):
                 "traffic_note": "ncu DRAM bytes per listed row on a 16384-query slice, scaled to the launch"}
 
     # end to end: same calls, inputs from pinned host memory, output back to host
-    e2e = run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
+    e2e = None if args.no_e2e else run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -236,9 +241,10 @@ def run_ours(args, world, rank, local):
 
     decode = None
     if not args.no_decode:
-        del Q, K, V, O, flush
+        del Q, K, V, O, flush, layer
         torch.cuda.empty_cache()
-        decode = run_decode(args, dev)
+        dwl = "flat_1m" if args.workload == "flat_128k" else args.workload
+        decode = run_decode(args, dev, dwl, wl["mode"])
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -248,7 +254,7 @@ def run_ours(args, world, rank, local):
                    "T": T, "queries": nq, "k": wl["k"], "sink": 4, "window": 512,
                    "mode": wl["mode"], "Hq": hq, "Hkv": hkv, "head_dim": 128, "index_dim": 64,
                    "mixture_components": wl["n_components"], "parallelism": "replicas",
-                   "l2": "256 MiB buffer written between timed steps; Q/K/V (1.6 GB) exceed L2"},
+                   "l2": "256 MiB buffer written between timed steps; K/V exceed L2"},
         "breakdown_ms": {"build": round(float(per[:, 0].mean()), 3), "index": round(float(per[:, 1].mean()), 3),
                          "attention": round(attn_ms, 3)},
         "roofline": roofline,
@@ -300,18 +306,18 @@ def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, dev, world):
             "ms_per_step": round(ms / args.steps, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
-def run_decode(args, dev):
+def run_decode(args, dev, workload="flat_1m", mode="flat"):
     """Decode at T = 1M (Flat, k = 4096): per new token, batch 1, the index of
     that token (lsa_index_decode) and its sparse attention.  The two calls are
     captured once in a CUDA graph; each token copies its query into the
     graph's input buffers and replays it (both inside the timed region).
     Mean us/token over 64 tokens; the eager (uncaptured) figure is kept too."""
-    wl = I.WORKLOADS["flat_1m"]
+    wl = I.WORKLOADS[workload]
     T, nd, hq, hkv = wl["T"], wl["n_decode"], wl["hq"], wl["hkv"]
     keys_all = I.index_keys(0, T + nd, wl["n_components"])
     pos_np = np.arange(T, T + nd, dtype=np.int64)
     q_np = I.index_queries(0, keys_all, pos_np)
-    layer = SparseLayer(T, k=wl["k"], mode="flat", max_queries=1, Hq=hq)
+    layer = SparseLayer(T, k=wl["k"], mode=mode, beam=wl.get("beam", 32), max_queries=1, Hq=hq)
     layer.build(torch.from_numpy(keys_all[:T]).to(dev))
     g = torch.Generator(device=dev)
     g.manual_seed(77)
@@ -371,7 +377,7 @@ def run_decode(args, dev):
         graph_us = e0.elapsed_time(e1) * 1e3 / nd
     except Exception as ex:  # report, keep the eager number
         note = f"graph capture failed: {type(ex).__name__}: {ex}"[:200]
-    out = {"workload": "flat_1m", "T": T, "tokens": nd, "k": wl["k"], "list_len": lens,
+    out = {"workload": workload, "mode": mode, "T": T, "tokens": nd, "k": wl["k"], "list_len": lens,
            "us_per_token": round(graph_us if graph_us is not None else eager_us, 2),
            "us_per_token_eager": round(eager_us, 2),
            "note": "batch 1; lsa_index_decode + lsa_sparse_attention per token, replayed from one CUDA graph"}
@@ -392,6 +398,7 @@ def cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=20.0, sample=None
     nq = len(pos_np)
     t0 = time.perf_counter()
     oc = O.build_cache(keys_np)
+    ot = O.build_tree(oc) if wl["mode"] == "tree" else None
     t_build = time.perf_counter() - t0
     Kb = K.view(torch.int16).cpu().numpy().view(np.uint16)
     Vb = V.view(torch.int16).cpu().numpy().view(np.uint16)
@@ -403,7 +410,8 @@ def cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=20.0, sample=None
         sel = rng_idx[(np.arange(S) * 4096 // S)]
         Qb = I.normal_bf16_bits(1, I.STREAM_Q, (S, hq, 128))
         t0 = time.perf_counter()
-        lists, lens = O.index(q_np[sel], pos_np[sel], oc, k=wl["k"])
+        lists, lens = O.index(q_np[sel], pos_np[sel], oc, k=wl["k"], mode=wl["mode"], tree=ot,
+                              beam=wl.get("beam", 32))
         O.attention(Qb, Kb, Vb, lists, lens)
         t_q = time.perf_counter() - t0
         done = S
@@ -422,7 +430,8 @@ def run_reference(args, world, rank):
     """The reference arm: the CPU oracle on this host, same metric and workload."""
     if rank != 0:
         return
-    wl = I.WORKLOADS[args.workload]
+    wl = dict(I.WORKLOADS[args.workload])
+    wl["mode"] = args.mode or ("flat" if wl["mode"] == "both" else wl["mode"])
     keys_np, q_np, pos_np = make_prefill_inputs(wl)
     T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
     Kb = torch.from_numpy(I.normal_bf16_bits(0, I.STREAM_K, (T, hkv, 128)).view(np.int16)).view(torch.bfloat16)
@@ -455,7 +464,9 @@ def main():
     ap.add_argument("--workload", default="flat_128k", choices=sorted(I.WORKLOADS))
     ap.add_argument("--queries", type=int, default=0,
                     help="time only the last N prefill queries of the workload (profiling slices)")
+    ap.add_argument("--mode", default=None, choices=["flat", "tree"], help="override the workload's search mode")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()

@@ -50,9 +50,9 @@ __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, c
 }
 
 // Score of one bucket on the CUDA cores: fp32 FMA chain over d = 0..63 of the
-// bf16 operands (k_fallback and k_tree_beam).  It can differ from the tensor
-// cores' sum of the same products in the last bit, which only matters for
-// scores within ~1e-6 of each other.
+// bf16 operands (k_fallback).  It can differ from the tensor cores' sum of
+// the same products in the last bit, which only matters for scores within
+// ~1e-6 of each other, at the one cut a Flat search makes.
 __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *__restrict__ c)
 {
     const uint4 *c4 = reinterpret_cast<const uint4 *>(c);
@@ -68,6 +68,29 @@ __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *_
         }
     }
     return acc;
+}
+
+// Score of one tree node, rounded once to fp32 from the fp64 sum over
+// d = 0..63 of the bf16 products taken in that order.  A product of two bf16
+// values is exact in fp64, so each fused step rounds exactly like a separate
+// add and the result is the same fp32 value as a plain fp64 dot product
+// written out in index order.  A beam search cuts at every level; scoring
+// this way makes those cuts independent of the accumulation order.
+__device__ __forceinline__ float dot_bf16_row_f64(const float *qf, const uint16_t *__restrict__ c)
+{
+    const uint4 *c4 = reinterpret_cast<const uint4 *>(c);
+    double acc = 0.0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        uint4 w = __ldg(c4 + v);
+        uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            acc = __fma_rn((double)qf[v * 8 + 2 * h], (double)__uint_as_float(ww[h] << 16), acc);
+            acc = __fma_rn((double)qf[v * 8 + 2 * h + 1], (double)__uint_as_float(ww[h] & 0xffff0000u), acc);
+        }
+    }
+    return __double2float_rn(acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -311,7 +334,7 @@ __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int 
         for (int i = t; i < S; i += blockDim.x) {
             if (i < n) {
                 const int32_t u = cids[i];
-                keys[i] = rank_key(dot_bf16_row(qf, tv.centroid_bf16 + (off + u) * LSA_D), u);
+                keys[i] = rank_key(dot_bf16_row_f64(qf, tv.centroid_bf16 + (off + u) * LSA_D), u);
             } else {
                 keys[i] = ~0ull;
             }

@@ -1,0 +1,186 @@
+"""GPU parity at the measured workload sizes: T = 131072, 1,048,576 (Flat and
+Tree) and 10,000,000 tokens.  The bucket cache and the tree are compared in
+full; the index lists and the attention on sampled queries (the oracle
+computes those one by one), including decode positions past the context.
+Rules are in tests/parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from hierarchical_key_clustering_b200 import inputs as I
+from hierarchical_key_clustering_b200 import lsa
+
+from . import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for the -m gpu tests")
+
+
+def _gpu_index(cache, tree, p, q, pos, decode=False):
+    nq = len(pos)
+    Lmax = lsa.lsa_list_budget(p)
+    lists = torch.empty((nq, Lmax), dtype=torch.int32, device="cuda")
+    lens = torch.empty((nq,), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_index_workspace_bytes(nq, cache.n_blocks, p))
+    fn = lsa.lsa_index_decode if decode else lsa.lsa_index_prefill
+    fn(PT.to_dev(q), PT.to_dev(np.asarray(pos, np.int64)), cache, tree, lists, lens, p, ws)
+    torch.cuda.synchronize()
+    return lists, lens
+
+
+def _attention_sampled(lists_d, lens_d, sel, T_kv, hq, hkv, seed):
+    """GPU attention over all listed queries; oracle on the sampled rows, with
+    K/V rows gathered for exactly the listed positions."""
+    nq = lists_d.shape[0]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    Q = torch.randn((nq, hq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    K = torch.randn((T_kv, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((T_kv, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    O_ = torch.empty_like(Q)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, lists_d.shape[1]))
+    lsa.lsa_sparse_attention(Q, K, V, lists_d, lens_d, O_, lse, ws=ws)
+    torch.cuda.synchronize()
+    lists = lists_d[sel].cpu().numpy()
+    lens = lens_d[sel].cpu().numpy()
+    used = np.unique(lists[lists >= 0])
+    remap = {int(v): i for i, v in enumerate(used)}
+    ll = np.where(lists >= 0, np.vectorize(lambda v: remap.get(int(v), -1))(lists), -1).astype(np.int32)
+    ui = torch.from_numpy(used.astype(np.int64)).cuda()
+    bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
+    Oref, lse_ref = O.attention(bits(Q[torch.from_numpy(sel).cuda()]), bits(K.index_select(0, ui)),
+                                bits(V.index_select(0, ui)), ll, lens)
+    return PT.assert_attention_close(O_[torch.from_numpy(sel).cuda()], Oref, lse[torch.from_numpy(sel).cuda()],
+                                     lse_ref)
+
+
+def _check_tree(gtree, otree):
+    assert gtree.level_sizes() == otree.level_size.tolist()
+    v = {k: t.cpu().numpy() for k, t in gtree.views().items()}
+    for name in ("child", "parent", "weight", "min_block", "max_block"):
+        assert np.array_equal(v[name], getattr(otree, name)), f"tree {name} differs"
+    assert np.array_equal(v["sum"].view(np.uint32), otree.sum.view(np.uint32))
+    assert np.array_equal(v["centroid_bf16"].view(np.uint16), otree.centroid_bf16)
+
+
+def test_flat_128k_cache_index_attention():
+    _need_gpu()
+    wl = I.WORKLOADS["flat_128k"]
+    T, k = wl["T"], wl["k"]
+    keys = I.index_keys(0, T, wl["n_components"])
+    oc = O.build_cache(keys)
+    p = lsa.lsa_default_params(k=k)
+    cache = lsa.Cache(T)
+    lsa.lsa_build_cache(PT.to_dev(keys), 0, T, cache, p)
+    torch.cuda.synchronize()
+    PT.assert_cache_equal(PT.cache_to_numpy(cache, T), oc)
+    # all queries through the GPU (the benchmark's launch), 600 sampled for the oracle
+    pos = np.arange(T, dtype=np.int64)
+    q = I.index_queries(0, keys, pos)
+    lists_d, lens_d = _gpu_index(cache, None, p, q, pos)
+    sel = np.unique(np.concatenate([np.linspace(0, T - 1, 560).astype(np.int64),
+                                    [0, 3, 511, 512, 1023, 1024, 65535, 65536, T - 2, T - 1]]))
+    ol, on = O.index(q[sel], pos[sel], oc, k=k)
+    PT.assert_lists_match(lists_d[torch.from_numpy(sel).cuda()].cpu().numpy(),
+                          lens_d[torch.from_numpy(sel).cuda()].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
+    _attention_sampled(lists_d, lens_d, sel[::10], T, wl["hq"], wl["hkv"], seed=1)
+
+
+@pytest.fixture(scope="module")
+def big1m():
+    _need_gpu()
+    wl = I.WORKLOADS["flat_1m"]
+    T = wl["T"]
+    keys_all = I.index_keys(0, T + wl["n_decode"], wl["n_components"])
+    keys = keys_all[:T]
+    oc = O.build_cache(keys)
+    p = lsa.lsa_default_params(k=wl["k"], mode="tree", beam=32)
+    cache = lsa.Cache(T)
+    lsa.lsa_build_cache(PT.to_dev(keys), 0, T, cache, p)
+    tree = lsa.Tree(T // 512)
+    lsa.lsa_build_tree(cache, tree, p)
+    torch.cuda.synchronize()
+    return wl, keys_all, oc, cache, tree
+
+
+def test_1m_cache_and_tree_bit_exact(big1m):
+    wl, keys_all, oc, cache, tree = big1m
+    PT.assert_cache_equal(PT.cache_to_numpy(cache, wl["T"]), oc)
+    _check_tree(tree, O.build_tree(oc))
+
+
+def test_1m_flat_prefill_and_decode(big1m):
+    wl, keys_all, oc, cache, _ = big1m
+    T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
+    p = lsa.lsa_default_params(k=k)
+    pos = np.arange(T - npre, T, dtype=np.int64)
+    q = I.index_queries(0, keys_all, pos)
+    lists_d, lens_d = _gpu_index(cache, None, p, q, pos)
+    sel = np.linspace(0, npre - 1, 160).astype(np.int64)
+    ol, on = O.index(q[sel], pos[sel], oc, k=k)
+    PT.assert_lists_match(lists_d[torch.from_numpy(sel).cuda()].cpu().numpy(),
+                          lens_d[torch.from_numpy(sel).cuda()].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
+    _attention_sampled(lists_d, lens_d, sel[::8], T + ndec, wl["hq"], wl["hkv"], seed=2)
+    # decode: one token at a time, every decode position
+    dpos = np.arange(T, T + ndec, dtype=np.int64)
+    dq = I.index_queries(1, keys_all, dpos)
+    gl, gn = [], []
+    for i in range(ndec):
+        l1, n1 = _gpu_index(cache, None, p, dq[i:i + 1], dpos[i:i + 1], decode=True)
+        gl.append(l1.cpu().numpy()[0])
+        gn.append(int(n1.cpu().numpy()[0]))
+    ol, on = O.index(dq, dpos, oc, k=k)
+    PT.assert_lists_match(np.stack(gl), np.array(gn), ol, on, dq, dpos, oc, k=k)
+
+
+def test_1m_tree_prefill_and_decode(big1m):
+    wl, keys_all, oc, cache, tree = big1m
+    T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
+    ot = O.build_tree(oc)
+    p = lsa.lsa_default_params(k=k, mode="tree", beam=32)
+    pos = np.concatenate([np.arange(T - npre, T, dtype=np.int64)[np.linspace(0, npre - 1, 96).astype(np.int64)],
+                          np.arange(T, T + ndec, dtype=np.int64)[::4]])
+    q = I.index_queries(0, keys_all, pos)
+    gl, gn = _gpu_index(cache, tree, p, q, pos)
+    ol, on = O.index(q, pos, oc, k=k, mode="tree", tree=ot, beam=32)
+    PT.assert_lists_match(gl.cpu().numpy(), gn.cpu().numpy(), ol, on, q, pos, oc, k=k, tree=ot, beam=32)
+
+
+def test_10m_flat_and_tree():
+    """10,000,000 tokens: 19531 complete blocks and an unclustered tail of 128;
+    the full cache and tree bit-exact, sampled Flat and Tree lists of the
+    last 65536 positions and of decode tokens, attention over 41 GB of K/V."""
+    _need_gpu()
+    wl = I.WORKLOADS["flat_tree_10m"]
+    T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
+    keys_all = I.index_keys(0, T + ndec, wl["n_components"])
+    keys = keys_all[:T]
+    oc = O.build_cache(keys)
+    p = lsa.lsa_default_params(k=k)
+    cache = lsa.Cache(T)
+    lsa.lsa_build_cache(PT.to_dev(keys), 0, T, cache, p)
+    tree = lsa.Tree(T // 512)
+    lsa.lsa_build_tree(cache, tree, lsa.lsa_default_params(k=k, mode="tree"))
+    torch.cuda.synchronize()
+    assert cache.n_blocks == 19531
+    PT.assert_cache_equal(PT.cache_to_numpy(cache, T), oc)
+    ot = O.build_tree(oc)
+    _check_tree(tree, ot)
+    del keys
+    pos = np.concatenate([np.arange(T - npre, T, dtype=np.int64)[np.linspace(0, npre - 1, 48).astype(np.int64)],
+                          np.arange(T, T + ndec, dtype=np.int64)[::16]])
+    q = I.index_queries(0, keys_all, pos)
+    lists_d, lens_d = _gpu_index(cache, None, p, q, pos)
+    ol, on = O.index(q, pos, oc, k=k)
+    PT.assert_lists_match(lists_d.cpu().numpy(), lens_d.cpu().numpy(), ol, on, q, pos, oc, k=k)
+    pt = lsa.lsa_default_params(k=k, mode="tree", beam=32)
+    tl, tn = _gpu_index(cache, tree, pt, q, pos)
+    otl, otn = O.index(q, pos, oc, k=k, mode="tree", tree=ot, beam=32)
+    PT.assert_lists_match(tl.cpu().numpy(), tn.cpu().numpy(), otl, otn, q, pos, oc, k=k, tree=ot, beam=32)
+    _attention_sampled(lists_d, lens_d, np.arange(0, len(pos), 7), T + ndec, wl["hq"], wl["hkv"], seed=3)
