@@ -153,8 +153,8 @@ IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
     L.cap = cand_cap(p);
     // small batches (decode) keep every score for the filter pass
     L.sstride = (nq <= lsa::SMALL_NQ && p->mode == LSA_MODE_FLAT) ? N : 0;
-    const int64_t sz[8] = {nq * LSA_DIM * 2, nq * 4, nq * 4, nq * 4, nq * L.gstride * 4, nq * L.cap * 4, nq * L.cap * 4,
-                           nq * L.sstride * 4};
+    const int64_t sz[8] = {nq * LSA_DIM * 2, nq * 4,          nq * 4,          nq * 4, nq * L.gstride * 4,
+                           nq * L.cap * 16,  nq * L.cap * 4, nq * L.sstride * 4};
     int64_t o = 0;
     for (int i = 0; i < 8; ++i) {
         L.off[i] = o;
@@ -220,8 +220,9 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     IndexLayout L = index_layout(nq, cache->n_blocks, p);
     if (L.cap < P) return fail(LSA_ERR_ARG, "cand_cap %lld < top buckets %lld", (long long)L.cap, (long long)P);
     if (L.cap > 8192) return fail(LSA_ERR_ARG, "cand_cap %lld above 8192", (long long)L.cap);
-    if ((int64_t)lsa::pow2_ceil64(p->k > 0 ? p->k : 1) * 4 + lsa::pow2_ceil64(L.cap) * 8 + P * 4 > 200 * 1024)
-        return fail(LSA_ERR_ARG, "k %d too large for the expansion kernel", p->k);
+    if (lsa::rank_expand_smem_bytes((int)L.cap, cache->n_blocks) > 227 * 1024)
+        return fail(LSA_ERR_ARG, "cand_cap %lld / %lld blocks too large for the expansion kernel", (long long)L.cap,
+                    (long long)cache->n_blocks);
     if (!ws || ws_bytes < L.bytes)
         return fail(LSA_ERR_WORKSPACE, "index workspace %lld bytes < %lld", (long long)ws_bytes, (long long)L.bytes);
     if (((uintptr_t)ws & 255u) != 0) return fail(LSA_ERR_ARG, "workspace must be 256-byte aligned");
@@ -232,8 +233,8 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     iw.tau = (float *)(w + L.off[2]);
     iw.cnt = (int32_t *)(w + L.off[3]);
     iw.ghist = (uint32_t *)(w + L.off[4]);
-    iw.cand_s = (float *)(w + L.off[5]);
-    iw.cand_id = (int32_t *)(w + L.off[6]);
+    iw.cand4 = (float *)(w + L.off[5]);
+    iw.cand_g = (int32_t *)(w + L.off[6]);
     iw.scores = L.sstride ? (float *)(w + L.off[7]) : nullptr;
     iw.score_stride = L.sstride;
     iw.cap = (int32_t)L.cap;

@@ -9,17 +9,18 @@
 // that follows it; zhichai forum post, "Key points" (Flat vs Tree).
 //
 // Flat selection.  A query that sees N buckets needs its top P buckets,
-// P = ceil((k + sink + window) / 4).  Pass 1 (tcgen05, lsa_score_tc.cu)
-// scores every bucket and histograms the maximum of each group of g
-// consecutive buckets (g a power of two giving 4P..8P groups).  The P-th
-// largest group maximum is a score of P distinct buckets, so it is <= the
-// P-th largest score, and so is tau, the lower edge of its histogram bin:
-// every bucket scoring at least tau is kept by pass 2, which recomputes the same scores
-// bit for bit on the tensor cores (or, for <= 16 queries, reads the scores
-// pass 1 stored) and appends the passing (score, id) pairs.  A query whose
-// candidates overflow their slots is redone exactly (radix select on the
-// recomputed scores) by the fallback kernel.  The candidates are then ranked
-// by (score desc, id asc) and expanded.
+// P = ceil((k + sink + window) / 4).  Pass 1 scores every bucket and
+// histograms the maximum of each group of g consecutive buckets (g a power of
+// two giving 4P..8P groups).  The P-th largest group maximum is a score of P
+// distinct buckets, so it is <= the P-th largest score, and so is tau, the
+// lower edge of its histogram bin: every bucket scoring at least tau is a
+// candidate.  Pass 2 recomputes the same scores bit for bit on the tensor
+// cores (lsa_score_tc.cu) or, for <= 16 queries, reads the scores pass 1
+// stored (k_dscore streams the centroids once on the CUDA cores), and appends
+// every aligned group of 4 buckets whose best score is >= tau as one entry.
+// The expansion kernel keeps the scores >= tau, ranks them by (score desc,
+// id asc) and expands them; a query whose entries or candidates overflow
+// their slots is redone exactly there (radix select on recomputed scores).
 #include "lsa_common.cuh"
 #include "lsa_kernels.h"
 
@@ -94,33 +95,6 @@ __device__ __forceinline__ float dot_bf16_row_f64(const float *qf, const uint16_
 }
 
 // ---------------------------------------------------------------------------
-// Flat pass 2 for small batches (decode): the tensor-core pass 1 stored every
-// score; keep those >= tau (one thread per bucket, all queries of the batch).
-__global__ void __launch_bounds__(256) k_dfilter(int64_t nq, IndexWs ws)
-{
-    __shared__ int Nq[SMALL_NQ];
-    __shared__ float tq[SMALL_NQ];
-    const int t = threadIdx.x;
-    if (t < nq) {
-        Nq[t] = ws.horizon[t] * LSA_NBKT;
-        tq[t] = ws.tau[t];
-    }
-    __syncthreads();
-    const int64_t b = (int64_t)blockIdx.x * 256 + t;
-    for (int qi = 0; qi < nq; ++qi) {
-        if (b >= Nq[qi]) continue;
-        const float s = ws.scores[qi * ws.score_stride + b];
-        if (s >= tq[qi]) {
-            const int slot = atomicAdd(ws.cnt + qi, 1);
-            if (slot < ws.cap) {
-                ws.cand_s[qi * ws.cap + slot] = s;
-                ws.cand_id[qi * ws.cap + slot] = (int32_t)b;
-            }
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
 // Radix select: the P-th largest key (u = f2ord(score)) among values produced
 // by `get(i)` for i in [0, n); all threads of the block call it.
 template <typename Get>
@@ -176,111 +150,6 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
         __syncthreads();
     }
     return prefix;
-}
-
-// Threshold per query: P-th largest group maximum (or -inf when N <= P).
-// Threshold per query from its global group-maximum histogram (used when a
-// query's buckets were split over several score CTAs): tau = lower edge of
-// the bin holding the P-th largest group maximum, -inf when there are <= P
-// groups.  One warp per query.
-__global__ void __launch_bounds__(256) k_tau(int64_t nq, int P, IndexWs ws)
-{
-    const int lane = threadIdx.x & 31;
-    const int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (q >= nq) return;
-    const int64_t N = (int64_t)ws.horizon[q] * LSA_NBKT;
-    const float NEG = __int_as_float(0xff800000);
-    if (n_groups(N, P) <= P) {
-        if (lane == 0) ws.tau[q] = NEG;
-        return;
-    }
-    // lane l owns bins 255-8l .. 248-8l (descending)
-    const uint32_t *h = ws.ghist + q * HIST_BINS;
-    int c8 = 0;
-    int cb[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        cb[e] = (int)h[HIST_BINS - 1 - 8 * lane - e];
-        c8 += cb[e];
-    }
-    int incl = c8;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(LSA_FULL, incl, o);
-        if (lane >= o) incl += y;
-    }
-    const int excl = incl - c8;
-    if (excl < P && P <= incl) {
-        int acc = excl;
-        int bin = HIST_BINS - 1 - 8 * lane;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            acc += cb[e];
-            if (acc >= P) {
-                bin = HIST_BINS - 1 - 8 * lane - e;
-                break;
-            }
-        }
-        ws.tau[q] = bin > 0 ? HIST_LO + bin * (2.0f * -HIST_LO / HIST_BINS) : NEG;
-    }
-}
-
-// Exact selection for queries whose candidates overflowed: radix select of
-// the P-th largest recomputed score tau*, then all scores > tau* plus the
-// lowest-id buckets scoring exactly tau* up to P in all.
-__global__ void __launch_bounds__(256) k_fallback(int64_t nq, const uint16_t *__restrict__ cbf, int P, IndexWs ws)
-{
-    __shared__ int hist[256];
-    __shared__ int sh[2];
-    __shared__ float qf[LSA_D];
-    __shared__ int n_out;
-    __shared__ int wsum[8];
-    for (int64_t q = blockIdx.x; q < nq; q += gridDim.x) {
-        if (ws.cnt[q] <= ws.cap) continue;  // block-uniform
-        const int64_t N = (int64_t)ws.horizon[q] * LSA_NBKT;
-        if (threadIdx.x < LSA_D) qf[threadIdx.x] = bf_bits2f(ws.qhat[q * LSA_D + threadIdx.x]);
-        if (threadIdx.x == 0) n_out = 0;
-        __syncthreads();
-        auto score = [&](int64_t b) { return dot_bf16_row(qf, cbf + b * LSA_D); };
-        const float tau = ord2f(block_select_kth_largest(N, P, score, hist, sh));
-        float *cs = ws.cand_s + q * ws.cap;
-        int32_t *ci = ws.cand_id + q * ws.cap;
-        for (int64_t b = threadIdx.x; b < N; b += blockDim.x) {
-            float s = score(b);
-            if (s > tau) {
-                int slot = atomicAdd(&n_out, 1);
-                cs[slot] = s;
-                ci[slot] = (int32_t)b;
-            }
-        }
-        __syncthreads();
-        // ties at tau in ascending bucket order
-        for (int64_t base = 0; base < N; base += blockDim.x) {
-            if (n_out >= P) break;  // block-uniform (read after a barrier)
-            int64_t b = base + threadIdx.x;
-            bool tie = (b < N) && (score(b) == tau);
-            unsigned bal = __ballot_sync(LSA_FULL, tie);
-            const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-            if (lane == 0) wsum[w] = __popc(bal);
-            __syncthreads();
-            int before = n_out;
-            for (int k = 0; k < w; ++k) before += wsum[k];
-            before += __popc(bal & ((1u << lane) - 1u));
-            if (tie && before < P) {
-                cs[before] = tau;
-                ci[before] = (int32_t)b;
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                int tot = 0;
-                for (int k = 0; k < (int)(blockDim.x >> 5); ++k) tot += wsum[k];
-                n_out = min(P, n_out + tot);
-            }
-            __syncthreads();
-        }
-        if (threadIdx.x == 0) ws.cnt[q] = n_out;
-        __syncthreads();
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -345,12 +214,17 @@ __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int 
         if (B < W) B = W;
         const int nk = (int)min((int64_t)n, B);
         for (int i = t; i < nk; i += blockDim.x) kept[i] = rank_key_id(keys[i]);
-        if (l == 0) {
+        if (l == 0) {  // one candidate entry per kept bucket; tau = -inf keeps them all
+            const float NEG = __int_as_float(0xff800000);
+            float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
             for (int i = t; i < nk; i += blockDim.x) {
-                ws.cand_s[q * ws.cap + i] = rank_key_score(keys[i]);
-                ws.cand_id[q * ws.cap + i] = rank_key_id(keys[i]);
+                c4[i] = make_float4(rank_key_score(keys[i]), NEG, NEG, NEG);
+                ws.cand_g[q * ws.cap + i] = rank_key_id(keys[i]);
             }
-            if (t == 0) ws.cnt[q] = nk;
+            if (t == 0) {
+                ws.cnt[q] = nk;
+                ws.tau[q] = NEG;
+            }
         }
         if (t == 0) n_kept = nk;
         __syncthreads();
@@ -358,135 +232,334 @@ __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int 
 }
 
 // ---------------------------------------------------------------------------
-// Block-wide inclusive scan of a[0..n) in shared memory (256 threads).
-__device__ void block_inclusive_scan(int *a, int n, int *wsum)
+// Block-wide inclusive scan of a[0..n) in shared memory (any block size up
+// to 1024 threads).
+template <typename T>
+__device__ void block_inclusive_scan(T *a, int n, T *wsum)
 {
     const int t = threadIdx.x;
     const int per = (n + blockDim.x - 1) / blockDim.x;
     const int lo = min(n, t * per), hi = min(n, lo + per);
-    int s = 0;
+    T s = 0;
     for (int i = lo; i < hi; ++i) {
         s += a[i];
         a[i] = s;
     }
     // exclusive scan of per-thread totals
     const int lane = t & 31, w = t >> 5;
-    int x = s;
+    T x = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(LSA_FULL, x, o);
+        T y = __shfl_up_sync(LSA_FULL, x, o);
         if (lane >= o) x += y;
     }
     if (lane == 31) wsum[w] = x;
     __syncthreads();
-    int before = x - s;
+    T before = x - s;
     for (int k = 0; k < w; ++k) before += wsum[k];
     for (int i = lo; i < hi; ++i) a[i] += before;
     __syncthreads();
 }
 
-// Weighted radix select over 64-bit rank keys (ascending = best first):
-// the smallest key K with sum of w over keys <= K reaching `target`, and the
-// weight still needed from K itself.  All threads of the block call it.
-__device__ void block_weighted_select(const uint64_t *keys, const int32_t *w, int n, int target, int *hist,
-                                      uint64_t *out_key, int *out_rem)
+// Threshold of one query from its group-maximum histogram (warp-collective,
+// every lane returns it): the lower edge of the bin holding the P-th largest
+// group maximum, -inf when the query has <= P groups.
+__device__ float tau_from_hist(const uint32_t *h, int64_t N, int P)
 {
-    __shared__ int sh_digit, sh_rem;
-    uint64_t prefix = 0, mask = 0;
-    int rem = target;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        const int n_round = ((n + blockDim.x - 1) / blockDim.x) * blockDim.x;
-        for (int i = threadIdx.x; i < n_round; i += blockDim.x) {
-            int bin = -1, wt = 0;
-            if (i < n && (keys[i] & mask) == prefix) {
-                bin = (int)((keys[i] >> shift) & 255);
-                wt = w[i];
+    const int lane = threadIdx.x & 31;
+    const float NEG = __int_as_float(0xff800000);
+    if (n_groups(N, P) <= P) return NEG;
+    // lane l owns bins 255-8l .. 248-8l (descending)
+    int cb[8], c8 = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        cb[e] = (int)h[HIST_BINS - 1 - 8 * lane - e];
+        c8 += cb[e];
+    }
+    int incl = c8;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(LSA_FULL, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int excl = incl - c8;
+    int bin = -1;
+    if (excl < P && P <= incl) {
+        int acc = excl;
+        bin = HIST_BINS - 1 - 8 * lane;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            acc += cb[e];
+            if (acc >= P) {
+                bin = HIST_BINS - 1 - 8 * lane - e;
+                break;
             }
-            const unsigned peers = __match_any_sync(LSA_FULL, bin);
-            const int sum = __reduce_add_sync(peers, wt);
-            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], sum);
         }
-        __syncthreads();
-        if (threadIdx.x < 32) {  // ascending bins: lane l owns 8l .. 8l+7
-            const int lane = threadIdx.x;
-            int c8 = 0;
+    }
+    const unsigned who = __ballot_sync(LSA_FULL, bin >= 0);
+    bin = who ? __shfl_sync(LSA_FULL, bin, __ffs(who) - 1) : 0;
+    return bin > 0 ? hist_edge(bin) : NEG;
+}
+
+// Threshold per query from its global group-maximum histogram, for queries
+// whose buckets were split over several score CTAs.  One warp per query.
+__global__ void __launch_bounds__(256) k_tau(int64_t nq, int P, IndexWs ws)
+{
+    const int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (q >= nq) return;
+    const float t = tau_from_hist(ws.ghist + q * HIST_BINS, (int64_t)ws.horizon[q] * LSA_NBKT, P);
+    if ((threadIdx.x & 31) == 0) ws.tau[q] = t;
+}
+
+// ---------------------------------------------------------------------------
+// Small batches (<= SMALL_NQ queries, decode), pass 1: every score on the
+// CUDA cores, each centroid row streamed once from HBM for all queries of
+// the batch, stored for the filter pass, with each query's group maxima
+// counted into its global histogram.  A CTA of DS_WARPS warps takes
+// DS_WARPS * 128 consecutive buckets; a warp takes an aligned run of 128
+// (groups are at most 128 buckets, so none straddles two warps), 32 at a time,
+// one bucket per lane.
+constexpr int DS_WARPS = 4;
+constexpr int DS_SPAN = DS_WARPS * 128;
+
+__global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb_total,
+                                                          const uint16_t *__restrict__ cbf, int P, IndexWs ws)
+{
+    __shared__ __align__(16) float qf[SMALL_NQ][LSA_D];
+    __shared__ uint32_t hs[SMALL_NQ][HIST_BINS];
+    __shared__ int Nq[SMALL_NQ], gq[SMALL_NQ];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    for (int i = t; i < nq * LSA_D; i += blockDim.x) qf[i / LSA_D][i % LSA_D] = bf_bits2f(ws.qhat[i]);
+    for (int i = t; i < nq * HIST_BINS; i += blockDim.x) hs[i / HIST_BINS][i % HIST_BINS] = 0u;
+    if (t < nq) {
+        const int N = ws.horizon[t] * LSA_NBKT;
+        Nq[t] = N;
+        gq[t] = group_width(N, P);
+    }
+    __syncthreads();
+    const float NEG = __int_as_float(0xff800000);
+    const int64_t wbase = (int64_t)blockIdx.x * DS_SPAN + warp * 128;
+    float run[SMALL_NQ];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) c8 += hist[8 * lane + e];
-            int incl = c8;
+    for (int i = 0; i < SMALL_NQ; ++i) run[i] = NEG;
+    for (int r = 0; r < 4; ++r) {
+        const int64_t b = wbase + r * 32 + lane;
+        uint32_t cw[32];
+        if (b < nb_total) {
+            const uint4 *c4 = reinterpret_cast<const uint4 *>(cbf + b * LSA_D);
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(LSA_FULL, incl, o);
-                if (lane >= o) incl += y;
+            for (int v = 0; v < 8; ++v) {
+                const uint4 w = __ldg(c4 + v);
+                cw[4 * v] = w.x;
+                cw[4 * v + 1] = w.y;
+                cw[4 * v + 2] = w.z;
+                cw[4 * v + 3] = w.w;
             }
-            const int excl = incl - c8;
-            if (excl < rem && rem <= incl) {
-                int acc = excl;
-                for (int e = 0; e < 8; ++e) {
-                    const int d = 8 * lane + e;
-                    if (acc + hist[d] >= rem) {
-                        sh_digit = d;
-                        sh_rem = rem - acc;
-                        break;
-                    }
-                    acc += hist[d];
+        } else {
+#pragma unroll
+            for (int v = 0; v < 32; ++v) cw[v] = 0u;
+        }
+#pragma unroll
+        for (int qi = 0; qi < SMALL_NQ; ++qi) {
+            if (qi >= nq) break;  // uniform
+            const float4 *qv = reinterpret_cast<const float4 *>(qf[qi]);
+            float acc = 0.0f;
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+                const float4 x = qv[v];
+                acc = fmaf(x.x, __uint_as_float(cw[2 * v] << 16), acc);
+                acc = fmaf(x.y, __uint_as_float(cw[2 * v] & 0xffff0000u), acc);
+                acc = fmaf(x.z, __uint_as_float(cw[2 * v + 1] << 16), acc);
+                acc = fmaf(x.w, __uint_as_float(cw[2 * v + 1] & 0xffff0000u), acc);
+            }
+            const bool valid = b < Nq[qi];
+            if (valid) ws.scores[qi * ws.score_stride + b] = acc;
+            const int g = gq[qi];
+            float m = valid ? acc : NEG;
+            if (g <= 32) {
+                for (int o = 1; o < g; o <<= 1) m = fmaxf(m, __shfl_xor_sync(LSA_FULL, m, o));
+                if (valid && (lane & (g - 1)) == 0) atomicAdd(&hs[qi][hist_bin(m)], 1u);
+            } else {
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(LSA_FULL, m, o));
+                run[qi] = fmaxf(run[qi], m);
+                const int per = g >> 5;  // 2 or 4 rounds per group
+                if ((r & (per - 1)) == per - 1) {
+                    const int64_t gstart = wbase + (int64_t)(r - per + 1) * 32;
+                    if (lane == 0 && gstart < Nq[qi]) atomicAdd(&hs[qi][hist_bin(run[qi])], 1u);
+                    run[qi] = NEG;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = t; i < nq * HIST_BINS; i += blockDim.x) {
+        const uint32_t c = hs[i / HIST_BINS][i % HIST_BINS];
+        if (c) atomicAdd(ws.ghist + i, c);
+    }
+}
+
+// Small batches, pass 2: each CTA derives every query's threshold from its
+// histogram (CTA 0 also stores it), then one thread per aligned group of 4
+// stored scores appends the group as a candidate entry when its best score
+// is >= tau.
+__global__ void __launch_bounds__(256) k_dfilter(int64_t nq, int P, IndexWs ws)
+{
+    __shared__ float tq[SMALL_NQ];
+    __shared__ int Nq[SMALL_NQ];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    for (int qi = warp; qi < nq; qi += blockDim.x >> 5) {
+        const int64_t N = (int64_t)ws.horizon[qi] * LSA_NBKT;
+        const float tau = tau_from_hist(ws.ghist + qi * HIST_BINS, N, P);
+        if (lane == 0) {
+            tq[qi] = tau;
+            Nq[qi] = (int)N;
+            if (blockIdx.x == 0) ws.tau[qi] = tau;
+        }
+    }
+    __syncthreads();
+    const int64_t b4 = ((int64_t)blockIdx.x * blockDim.x + t) * 4;
+    for (int qi = 0; qi < nq; ++qi) {
+        if (b4 >= Nq[qi]) continue;
+        const float4 s = *reinterpret_cast<const float4 *>(ws.scores + qi * ws.score_stride + b4);
+        if (fmaxf(fmaxf(s.x, s.y), fmaxf(s.z, s.w)) >= tq[qi]) {
+            const int slot = atomicAdd(ws.cnt + qi, 1);
+            if (slot < ws.cap) {
+                reinterpret_cast<float4 *>(ws.cand4)[qi * ws.cap + slot] = s;
+                ws.cand_g[qi * ws.cap + slot] = (int32_t)b4;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Rank the candidates of one query and expand them into its index list.
+//   1. candidates: every listed score >= tau (a Flat query whose entries or
+//      candidates overflow is redone exactly here: radix select of the P-th
+//      largest score recomputed on the CUDA cores, then every bucket above it
+//      and the lowest-id buckets equal to it, P in all);
+//   2. each candidate's weight: its members outside near;
+//   3. the walk over buckets in (score desc, id asc) order stops at the
+//      bucket where the weights reach k: found by histogramming the weights
+//      over the candidates' rank keys (4096 bins over the remaining key range)
+//      and narrowing to the bin where k is reached until it holds one key --
+//      buckets ranked before it are taken whole, their order does not matter;
+//   4. the chosen positions are marked in one 512-bit mask per touched block
+//      (blocks found through a bitmap over all visible blocks, RX_SLOTS
+//      blocks at a time) and emitted block by block in ascending order -- the
+//      far keys come out sorted without sorting them;
+//   5. sink, far keys and window are written.
+// Every bucket has >= 4 keys and at most sink + window clustered keys are
+// near, so the best P buckets already hold k far keys: the cut never falls
+// outside the top P.
+constexpr int RX_SLOTS = 512;  // touched blocks per emit batch
+constexpr int RX_BINS = 4096;  // bins of the cut search (aliases the masks)
+
+__host__ __device__ inline size_t rank_expand_smem(int KC, int TW)
+{
+    return (size_t)KC * 8 + (size_t)RX_SLOTS * 64 + (size_t)TW * 8 + (size_t)RX_SLOTS * 8 + (size_t)KC;
+}
+
+__global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict__ pos,
+                                                      const int32_t *__restrict__ members,
+                                                      const uint16_t *__restrict__ cbf, int32_t *__restrict__ lists,
+                                                      int32_t *__restrict__ lens, int Lmax, int k, int sink,
+                                                      int window, int P, int KC, int TW, IndexWs ws)
+{
+    extern __shared__ uint64_t rsm[];
+    uint64_t *keys = rsm;                                           // [KC]
+    uint32_t *masks = reinterpret_cast<uint32_t *>(keys + KC);      // [RX_SLOTS][16]
+    uint32_t *bins = masks;                                         // [RX_BINS] (before the masks are used)
+    uint32_t *touched = masks + RX_SLOTS * 16;                      // [TW]
+    int32_t *wrank = reinterpret_cast<int32_t *>(touched + TW);     // [TW]
+    int32_t *slot_blk = wrank + TW;                                 // [RX_SLOTS]
+    int32_t *slot_off = slot_blk + RX_SLOTS;                        // [RX_SLOTS]
+    uint8_t *wt = reinterpret_cast<uint8_t *>(slot_off + RX_SLOTS);  // [KC]
+    __shared__ int wsum[32];
+    __shared__ int hist[256];
+    __shared__ int sh[4];
+    __shared__ float qf[LSA_D];
+    __shared__ int nk_s, fb_s, tot_s, cnt_s, excl_s;
+    __shared__ unsigned long long lo_s, hi_s, cut_s;
+
+    const int64_t q = blockIdx.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
+    const int64_t p = pos[q];
+    const int64_t w0 = p - window > 0 ? p - window : 0;
+    const int64_t s_end = (int64_t)sink < p + 1 ? (int64_t)sink : p + 1;
+    const int64_t N = (int64_t)ws.horizon[q] * LSA_NBKT;
+    const float NEG = __int_as_float(0xff800000);
+    const int ne = ws.cnt[q];
+    if (t == 0) {
+        nk_s = 0;
+        fb_s = ne > ws.cap;
+        tot_s = 0;
+        lo_s = ~0ull;
+        hi_s = 0ull;
+    }
+    for (int i = t; i < TW; i += blockDim.x) touched[i] = 0u;
+    __syncthreads();
+
+    // 1. candidates
+    if (!fb_s) {
+        const float tau = ws.tau[q];
+        const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + q * ws.cap;
+        const int32_t *cg = ws.cand_g + q * ws.cap;
+        for (int i = t; i < ne; i += blockDim.x) {
+            const float4 s4 = c4[i];
+            const int32_t g = cg[i];
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (sv[e] >= tau && sv[e] > NEG) {
+                    const int slot = atomicAdd(&nk_s, 1);
+                    if (slot < KC) keys[slot] = rank_key(sv[e], g + e);
                 }
             }
         }
         __syncthreads();
-        prefix |= (uint64_t)sh_digit << shift;
-        mask |= (uint64_t)255 << shift;
-        rem = sh_rem;
+        if (t == 0 && nk_s > KC) fb_s = 1;
         __syncthreads();
     }
-    *out_key = prefix;
-    *out_rem = rem;
-}
+    if (fb_s) {  // block-uniform: exact selection of the top P
+        if (t < LSA_D) qf[t] = bf_bits2f(ws.qhat[q * LSA_D + t]);
+        if (t == 0) nk_s = 0;
+        __syncthreads();
+        auto score = [&](int64_t b) { return dot_bf16_row(qf, cbf + b * LSA_D); };
+        const float ts = ord2f(block_select_kth_largest(N, P, score, hist, sh));
+        for (int64_t b = t; b < N; b += blockDim.x) {
+            const float s = score(b);
+            if (s > ts) keys[atomicAdd(&nk_s, 1)] = rank_key(s, (int32_t)b);
+        }
+        __syncthreads();
+        // ties at ts in ascending bucket order, up to P candidates in all
+        for (int64_t base = 0; base < N; base += blockDim.x) {
+            if (nk_s >= P) break;  // block-uniform (read after a barrier)
+            const int64_t b = base + t;
+            const bool tie = (b < N) && (score(b) == ts);
+            const unsigned bal = __ballot_sync(LSA_FULL, tie);
+            if (lane == 0) wsum[warp] = __popc(bal);
+            __syncthreads();
+            int before = nk_s;
+            for (int w = 0; w < warp; ++w) before += wsum[w];
+            before += __popc(bal & ((1u << lane) - 1u));
+            if (tie && before < P) keys[before] = rank_key(ts, (int32_t)b);
+            __syncthreads();
+            if (t == 0) {
+                int tot = 0;
+                for (int w = 0; w < nwarps; ++w) tot += wsum[w];
+                nk_s = min(P, nk_s + tot);
+            }
+            __syncthreads();
+        }
+    }
+    const int n = nk_s;
 
-// Rank the candidates of one query and expand them into its index list.
-//   1. count each candidate bucket's members outside near (its weight);
-//   2. the walk over buckets in (score desc, id asc) order stops at the
-//      bucket where the weights reach k: find that bucket (and how many of
-//      its keys are still needed) by a weighted radix select -- buckets
-//      ranked before it are taken whole, their order does not matter;
-//   3. mark the chosen positions in one 512-bit mask per touched block
-//      (blocks found through a bitmap over all visible blocks) and emit them
-//      block by block in ascending order -- the far keys come out sorted
-//      without sorting them;
-//   4. write sink, far keys and window.
-// Every bucket has >= 4 keys and at most sink + window clustered keys are
-// near, so when a query has >= P candidates its best P buckets already hold
-// k far keys: the cut never falls outside the top P.
-__global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict__ pos, const int32_t *__restrict__ members,
-                                                     int32_t *__restrict__ lists, int32_t *__restrict__ lens, int Lmax,
-                                                     int k, int sink, int window, int P, int CAP, int TW, IndexWs ws)
-{
-    extern __shared__ uint64_t rsm[];
-    uint64_t *keys = rsm;                                        // [CAP]
-    int32_t *wt = reinterpret_cast<int32_t *>(keys + CAP);       // [CAP]
-    uint32_t *masks = reinterpret_cast<uint32_t *>(wt + CAP);    // [P][16]
-    uint32_t *touched = masks + (size_t)P * 16;                  // [TW]
-    int32_t *wrank = reinterpret_cast<int32_t *>(touched + TW);  // [TW]
-    int32_t *slot_blk = wrank + TW;                              // [P]
-    int32_t *slot_off = slot_blk + P;                            // [P]
-    __shared__ int wsum[32];
-    __shared__ int hist[256];
-    __shared__ int tot_s;
-
-    const int64_t q = blockIdx.x;
-    const int t = threadIdx.x;
-    const int64_t p = pos[q];
-    const int n = min(ws.cnt[q], ws.cap);
-    const int64_t w0 = p - window > 0 ? p - window : 0;
-    const int64_t s_end = (int64_t)sink < p + 1 ? (int64_t)sink : p + 1;
-    if (t == 0) tot_s = 0;
-    for (int i = t; i < TW; i += blockDim.x) touched[i] = 0u;
-    __syncthreads();
+    // 2. weights (members outside near) and the key range of weighted candidates
     int my_tot = 0;
+    unsigned long long my_lo = ~0ull, my_hi = 0ull;
     for (int i = t; i < n; i += blockDim.x) {
-        const int32_t b = ws.cand_id[q * ws.cap + i];
-        keys[i] = rank_key(ws.cand_s[q * ws.cap + i], b);
+        const int32_t b = rank_key_id(keys[i]);
         const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
         int nn = 0;
 #pragma unroll
@@ -499,20 +572,80 @@ __global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict_
                 nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
             }
         }
-        wt[i] = nn;
+        wt[i] = (uint8_t)nn;
         my_tot += nn;
+        if (nn > 0) {
+            my_lo = min(my_lo, (unsigned long long)keys[i]);
+            my_hi = max(my_hi, (unsigned long long)keys[i]);
+        }
     }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) my_tot += __shfl_xor_sync(LSA_FULL, my_tot, o);
-    if ((t & 31) == 0) atomicAdd(&tot_s, my_tot);
+    for (int o = 16; o >= 1; o >>= 1) {
+        my_tot += __shfl_xor_sync(LSA_FULL, my_tot, o);
+        my_lo = min(my_lo, __shfl_xor_sync(LSA_FULL, my_lo, o));
+        my_hi = max(my_hi, __shfl_xor_sync(LSA_FULL, my_hi, o));
+    }
+    if (lane == 0) {
+        atomicAdd(&tot_s, my_tot);
+        atomicMin(&lo_s, my_lo);
+        atomicMax(&hi_s, my_hi);
+    }
     __syncthreads();
     const int nfar = min(k, tot_s);
-    uint64_t cut_key = 0;
+
+    // 3. the cut: smallest key K with (weight of keys <= K) >= nfar, and the
+    //    number of K's far keys still needed (take)
+    uint64_t cut = 0;
     int take = 0;
-    if (nfar > 0) block_weighted_select(keys, wt, n, nfar, hist, &cut_key, &take);
+    if (nfar > 0) {
+        uint64_t lo = lo_s, hi = hi_s;
+        int rem = nfar;
+        for (int round = 0;; ++round) {  // block-uniform
+            const uint64_t span = hi - lo;
+            const int shift = (span >> 12) == 0 ? 0 : (64 - __clzll((long long)span)) - 12;
+            for (int i = t; i < RX_BINS; i += blockDim.x) bins[i] = 0u;
+            if (t == 0) cut_s = ~0ull;
+            __syncthreads();
+            for (int i = t; i < n; i += blockDim.x) {
+                const uint64_t key = keys[i];
+                if (wt[i] > 0 && key >= lo && key <= hi)
+                    atomicAdd(&bins[(key - lo) >> shift], (1u << 18) | (uint32_t)wt[i]);
+            }
+            __syncthreads();
+            block_inclusive_scan(bins, RX_BINS, reinterpret_cast<uint32_t *>(wsum));  // count << 18 | weight
+            for (int c = t; c < RX_BINS; c += blockDim.x) {
+                const uint32_t inc = bins[c], exc = c > 0 ? bins[c - 1] : 0u;
+                if ((int)(exc & 0x3ffffu) < rem && rem <= (int)(inc & 0x3ffffu)) {
+                    sh[0] = c;
+                    excl_s = (int)(exc & 0x3ffffu);
+                    cnt_s = (int)((inc >> 18) - (exc >> 18));
+                }
+            }
+            __syncthreads();
+            const int c = sh[0];
+            const uint64_t blo = lo + ((uint64_t)c << shift);
+            const uint64_t bhi = min(hi, blo + (((uint64_t)1 << shift) - 1));
+            rem -= excl_s;
+            // one weighted key left in [blo, bhi] (always so once a bin is one
+            // key wide, since keys are distinct): it is the cut
+            if (cnt_s == 1 || shift == 0 || round == 7) {
+                for (int i = t; i < n; i += blockDim.x)
+                    if (wt[i] > 0 && keys[i] >= blo && keys[i] <= bhi) atomicMin(&cut_s, (unsigned long long)keys[i]);
+                __syncthreads();
+                cut = cut_s;
+                take = rem;
+                break;
+            }
+            lo = blo;
+            hi = bhi;
+            __syncthreads();
+        }
+    }
     const bool any = nfar > 0;
+
+    // 4. touched blocks, then masks and emission RX_SLOTS blocks at a time
     for (int i = t; i < n; i += blockDim.x) {
-        if (any && keys[i] <= cut_key && wt[i] > 0) {
+        if (any && wt[i] > 0 && keys[i] <= cut) {
             const int blk = rank_key_id(keys[i]) / LSA_NBKT;
             atomicOr(&touched[blk >> 5], 1u << (blk & 31));
         }
@@ -522,46 +655,48 @@ __global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict_
     __syncthreads();
     block_inclusive_scan(wrank, TW, wsum);  // wrank[w] = touched blocks in words 0..w
     const int nslots = TW > 0 ? wrank[TW - 1] : 0;
-    for (int i = t; i < nslots * 16; i += blockDim.x) masks[i] = 0u;
-    __syncthreads();
-    for (int i = t; i < n; i += blockDim.x) {
-        if (!(any && keys[i] <= cut_key && wt[i] > 0)) continue;
-        const int32_t b = rank_key_id(keys[i]);
-        const int limit = (keys[i] == cut_key) ? take : 16;
-        const int blk = b / LSA_NBKT;
-        const uint32_t word = touched[blk >> 5];
-        const int slot = wrank[blk >> 5] - __popc(word) + __popc(word & ((1u << (blk & 31)) - 1u));
-        slot_blk[slot] = blk;
-        const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
-        int idx = 0;
+    const int n_sink = (int)min(s_end, w0);
+    int32_t *out = lists + q * (int64_t)Lmax;
+    int emitted = 0;
+    for (int b0 = 0; b0 < nslots; b0 += RX_SLOTS) {
+        const int nb = min(RX_SLOTS, nslots - b0);
+        for (int i = t; i < nb * 16; i += blockDim.x) masks[i] = 0u;
+        __syncthreads();
+        for (int i = t; i < n; i += blockDim.x) {
+            if (!(any && wt[i] > 0 && keys[i] <= cut)) continue;
+            const int32_t b = rank_key_id(keys[i]);
+            const int blk = b / LSA_NBKT;
+            const uint32_t word = touched[blk >> 5];
+            const int slot = wrank[blk >> 5] - __popc(word) + __popc(word & ((1u << (blk & 31)) - 1u)) - b0;
+            if (slot < 0 || slot >= nb) continue;
+            slot_blk[slot] = blk;
+            const int limit = (keys[i] == cut) ? take : 16;
+            const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
+            int idx = 0;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const int4 w = __ldg(m4 + v);
-            const int mm[4] = {w.x, w.y, w.z, w.w};
+            for (int v = 0; v < 4; ++v) {
+                const int4 w = __ldg(m4 + v);
+                const int mm[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int64_t m = mm[e];
-                if (m >= 0 && !(m < s_end || (m >= w0 && m <= p))) {
-                    if (idx < limit) atomicOr(&masks[slot * 16 + ((m & 511) >> 5)], 1u << (m & 31));
-                    ++idx;
+                for (int e = 0; e < 4; ++e) {
+                    const int64_t m = mm[e];
+                    if (m >= 0 && !(m < s_end || (m >= w0 && m <= p))) {
+                        if (idx < limit) atomicOr(&masks[slot * 16 + ((m & 511) >> 5)], 1u << (m & 31));
+                        ++idx;
+                    }
                 }
             }
         }
-    }
-    __syncthreads();
-    for (int sl = t; sl < nslots; sl += blockDim.x) {
-        int c = 0;
+        __syncthreads();
+        for (int sl = t; sl < nb; sl += blockDim.x) {
+            int c = 0;
 #pragma unroll
-        for (int w = 0; w < 16; ++w) c += __popc(masks[sl * 16 + w]);
-        slot_off[sl] = c;
-    }
-    __syncthreads();
-    block_inclusive_scan(slot_off, nslots, wsum);
-    const int n_sink = (int)min(s_end, w0);
-    int32_t *out = lists + q * (int64_t)Lmax;
-    {
-        const int lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
-        for (int sl = warp; sl < nslots; sl += nwarps) {
+            for (int w = 0; w < 16; ++w) c += __popc(masks[sl * 16 + w]);
+            slot_off[sl] = c;
+        }
+        __syncthreads();
+        block_inclusive_scan(slot_off, nb, wsum);
+        for (int sl = warp; sl < nb; sl += nwarps) {
             const uint32_t word = lane < 16 ? masks[sl * 16 + lane] : 0u;
             const int c = __popc(word);
             int incl = c;
@@ -570,7 +705,7 @@ __global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict_
                 const int y = __shfl_up_sync(LSA_FULL, incl, o);
                 if (lane >= o) incl += y;
             }
-            int o = n_sink + slot_off[sl] - __shfl_sync(LSA_FULL, incl, 15) + incl - c;
+            int o = n_sink + emitted + slot_off[sl] - __shfl_sync(LSA_FULL, incl, 15) + incl - c;
             const int32_t base = slot_blk[sl] * LSA_BLK + lane * 32;
             uint32_t bits = word;
             while (bits) {
@@ -579,16 +714,25 @@ __global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict_
                 bits &= bits - 1;
             }
         }
+        emitted += slot_off[nb - 1];
+        __syncthreads();
     }
+    // emitted == nfar (the marks add up to the weights before the cut plus
+    // take); the list is laid out from what was written either way
     const int nwin = (int)(p - w0 + 1);
-    const int len = n_sink + nfar + nwin;
+    const int len = n_sink + emitted + nwin;
     for (int i = t; i < Lmax; i += blockDim.x) {
         if (i < n_sink) out[i] = i;
-        else if (i < n_sink + nfar) continue;
-        else if (i < len) out[i] = (int32_t)(w0 + (i - n_sink - nfar));
+        else if (i < n_sink + emitted) continue;
+        else if (i < len) out[i] = (int32_t)(w0 + (i - n_sink - emitted));
         else out[i] = -1;
     }
     if (t == 0) lens[q] = len;
+}
+
+size_t rank_expand_smem_bytes(int cap, int64_t n_blocks)
+{
+    return rank_expand_smem(cap, (int)((n_blocks + 31) / 32) + 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -605,40 +749,35 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     }
     const int64_t nb_total = a.n_blocks * LSA_NBKT;
     const bool small = a.nq <= SMALL_NQ;
-    const int big_block = small ? 1024 : 256;
     if (a.mode == 0 && nb_total > 0) {
-        // pass 1 on the tensor cores: group maxima (+ every score for small batches)
-        ScoreTcArgs sa;
-        sa.nq = a.nq;
-        sa.nb_total = nb_total;
-        sa.P = a.P;
-        sa.mode = 0;
-        sa.store = small ? 1 : 0;
-        sa.chunk_tiles = 0;
-        sa.wait_limit = a.wait_limit;
-        sa.extra_tx = a.extra_tx;
-        int whole = 0;
-        if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, &whole)) != cudaSuccess) return e;
-        if (!whole) {  // thresholds from the merged histograms
-            k_tau<<<(unsigned)((a.nq + 7) / 8), 256, 0, st>>>(a.nq, a.P, ws);
+        if (small) {  // stream every centroid once for the whole batch, keep the scores
+            k_dscore<<<(unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN), DS_WARPS * 32, 0, st>>>(a.nq, nb_total,
+                                                                                               a.centroid_bf16, a.P, ws);
             count_launches(1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-        if (small) {  // pass 2 from the stored scores
-            const unsigned blocks = (unsigned)((nb_total + 255) / 256);
-            k_dfilter<<<blocks, 256, 0, st>>>(a.nq, ws);
+            k_dfilter<<<(unsigned)((nb_total / 4 + 255) / 256), 256, 0, st>>>(a.nq, a.P, ws);
             count_launches(1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        } else {  // pass 2 on the tensor cores: recompute the same scores, keep those >= tau
+        } else {  // two passes on the tensor cores: threshold, then filter
+            ScoreTcArgs sa;
+            sa.nq = a.nq;
+            sa.nb_total = nb_total;
+            sa.P = a.P;
+            sa.mode = 0;
+            sa.chunk_tiles = 0;
+            sa.wait_limit = a.wait_limit;
+            sa.extra_tx = a.extra_tx;
+            int whole = 0;
+            if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, &whole)) != cudaSuccess) return e;
+            if (!whole) {  // thresholds from the merged histograms
+                k_tau<<<(unsigned)((a.nq + 7) / 8), 256, 0, st>>>(a.nq, a.P, ws);
+                count_launches(1);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
             sa.mode = 1;
-            sa.store = 0;
             sa.extra_tx = 0;
             if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, nullptr)) != cudaSuccess) return e;
         }
-        const int64_t fb = small ? a.nq : (a.nq < (int64_t)n_sm * 2 ? a.nq : (int64_t)n_sm * 2);
-        k_fallback<<<(unsigned)fb, 256, 0, st>>>(a.nq, a.centroid_bf16, a.P, ws);
-        count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else if (tree && tree->n_levels > 0) {
         int64_t B1 = ((int64_t)a.P + 1) / 2;
         if (B1 < a.beam) B1 = a.beam;
@@ -651,11 +790,12 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
-    const int nslot_max = a.P;  // touched blocks <= buckets taken <= P (the cut is within any P buckets)
-    const size_t smr = (size_t)ws.cap * (8 + 4) + (size_t)nslot_max * (64 + 4 + 4) + (size_t)TW * 8;
+    const int KC = ws.cap;
+    const size_t smr = rank_expand_smem(KC, TW);
     cudaFuncSetAttribute(k_rank_expand, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-    k_rank_expand<<<(unsigned)a.nq, big_block, smr, st>>>(a.pos, a.members, a.lists, a.lens, a.Lmax, a.k, a.sink,
-                                                         a.window, nslot_max, ws.cap, TW, ws);
+    k_rank_expand<<<(unsigned)a.nq, small ? 1024 : 256, smr, st>>>(a.pos, a.members, a.centroid_bf16, a.lists,
+                                                                   a.lens, a.Lmax, a.k, a.sink, a.window, a.P, KC,
+                                                                   TW, ws);
     count_launches(1);
     return cudaGetLastError();
 }

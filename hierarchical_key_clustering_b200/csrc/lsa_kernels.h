@@ -32,26 +32,44 @@ struct TreeView {
 };
 
 // Per-call index workspace (device pointers carved by the C ABI).
+// Candidates are entries of up to 4 buckets: cand_g holds the first bucket
+// id, cand4 the scores of buckets cand_g .. cand_g + 3; a score of -inf marks
+// a bucket that is not a candidate.  The expansion keeps the scores >= tau.
 struct IndexWs {
     uint16_t *qhat;     // [nq, 64] bf16 normalised queries
     int32_t *horizon;   // [nq] visible blocks
-    float *tau;         // [nq] Flat threshold
-    int32_t *cnt;       // [nq] candidates written
+    float *tau;         // [nq] Flat threshold (-inf: keep every listed score)
+    int32_t *cnt;       // [nq] candidate entries appended (may exceed cap)
     uint32_t *ghist;    // [nq, HIST_BINS] group-maximum histograms (split ranges)
-    float *cand_s;      // [nq, cap] candidate scores
-    int32_t *cand_id;   // [nq, cap] candidate bucket ids
+    float *cand4;       // [nq, cap, 4] candidate scores
+    int32_t *cand_g;    // [nq, cap] first bucket of each entry
     float *scores;      // [nq, score_stride] stored scores (small batches only)
     int64_t score_stride;
-    int32_t cap;
+    int32_t cap;        // entries per query
 };
-
 // Histogram of group maxima used to set the Flat threshold: HIST_BINS linear
 // bins over [HIST_LO, -HIST_LO] (scores of unit bf16 vectors lie inside).
 constexpr int HIST_BINS = 256;
 constexpr float HIST_LO = -1.0625f;
+constexpr float HIST_BIN_W = 2.0f * -HIST_LO / HIST_BINS;  // 17/2048: every bin edge is an exact float
+#ifdef __CUDACC__
+__device__ __forceinline__ float hist_edge(int bin)
+{
+    return HIST_LO + (float)bin * HIST_BIN_W;
+}
+// Bin of a group maximum m, rounded so that its lower edge is <= m.
+__device__ __forceinline__ int hist_bin(float m)
+{
+    int bin = __float2int_rd(__fmul_rn(__fsub_rn(m, HIST_LO), 1.0f / HIST_BIN_W));
+    bin = min(max(bin, 0), HIST_BINS - 1);
+    if (bin > 0 && m < hist_edge(bin)) --bin;
+    return bin;
+}
+#endif
 
 // Batches up to this many queries take the small-batch (decode) path:
-// thread-per-bucket scoring with stored scores.
+// streaming thread-per-bucket scoring on the CUDA cores, scores stored for
+// the filter pass.
 constexpr int SMALL_NQ = 16;
 
 cudaError_t launch_pool_norm(const float *keys, int64_t item_begin, int64_t item_end, float *pooled,
@@ -81,25 +99,26 @@ struct IndexArgs {
 };
 
 // Flat scoring on the tensor cores (lsa_score_tc.cu).  mode 0: threshold
-// histogram of group maxima (+ every score when store != 0); mode 1: append
-// scores >= tau.
+// histogram of group maxima; mode 1: append the groups of 4 buckets whose
+// best score is >= tau.
 struct ScoreTcArgs {
     int64_t nq;
     int64_t nb_total;
     int32_t P;
     int32_t mode;
-    int32_t store;
     int32_t whole_range;  // set by the launcher: one CTA covers each query's buckets
     int64_t chunk_tiles;
     uint32_t wait_limit;  // tries per bounded mbarrier wait
     uint32_t extra_tx;    // test hook: non-zero skips the query-tile copy, so its barrier never completes
 };
-
 cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint16_t *centroid_bf16, cudaStream_t st,
                             int n_sm, int *whole_range);
 int read_device_error(int clear);
 
 cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *tree, cudaStream_t st, int n_sm);
+// Shared memory the expansion kernel needs for `cap` candidates over a cache
+// of n_blocks blocks.
+size_t rank_expand_smem_bytes(int cap, int64_t n_blocks);
 
 struct AttnArgs {
     const uint16_t *Q, *K, *V;

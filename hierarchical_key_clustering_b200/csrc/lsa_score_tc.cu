@@ -5,30 +5,38 @@
 // bucket centroid of the earlier cluster blocks); zhichai forum post, "Key
 // points" (Flat search scores all bucket centroids, ~T/8 per query).
 //
-// S = Q^ C^T is a dense 64-deep contraction: a CTA owns a tile of 128 queries
-// (the MMA M) and streams 256-centroid tiles (the MMA N) of its bucket range.
-//   warp 0        TMA producer: the query tile once, centroid tiles into a
-//                 4-stage ring (128B-swizzled, K-major), mbarrier completion;
-//   warp 1        allocates 512 TMEM columns; one thread issues
-//                 tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32, 4 x K=16) into
-//                 one of two 128 x 256 fp32 accumulators, and commits to the
-//                 stage's "empty" barrier and the accumulator's "full" one;
-//   warps 2..5    epilogue: thread r owns TMEM lane r = query q0 + r and reads
-//                 its 256 scores with tcgen05.ld, 32 columns at a time, while
-//                 the other accumulator is being filled.
+// S = Q^ C^T is a dense 64-deep contraction.  A CTA owns two tiles of 128
+// queries (two MMA M operands) and streams 128-centroid tiles (the MMA N) of
+// its bucket range; each centroid tile feeds both query tiles, which halves
+// the centroid bytes per score the CTA pulls from L2.
+//   warp 0        TMA producer: both query tiles once (one 256-row box),
+//                 centroid tiles into a ring of 4 (threshold pass) or 8
+//                 (filter pass) stages, 128B-swizzled, K-major;
+//   warp 1        allocates 512 TMEM columns = [query tile][2 buffers] x 128
+//                 fp32 columns; one thread issues tcgen05.mma.kind::f16
+//                 (bf16 x bf16 -> fp32, 4 x K=16 per query tile) and commits
+//                 to the stage's "empty" barrier and the buffer's "full" one;
+//   warps 2..9    epilogue, two warps per TMEM lane quadrant: warp w reads
+//                 lanes 32 (w % 4) .. +31 of query tile (w - 2) / 4, so each
+//                 thread owns one query row; it copies its 128 scores out of
+//                 TMEM (4 loads, one wait), frees the buffer for the next MMA
+//                 and then works on registers.
 // The epilogue is fused with the pass's work, so the score matrix is never
-// stored (except, for batches of <= 16 queries, one row per query):
+// stored:
 //   GMAX    the maximum of each group of g consecutive buckets goes into the
-//           row's 256-bin histogram over [-1.0625, 1.0625] in shared memory
-//           (and, for small batches, every score is stored for the filter
-//           pass).  A CTA that covers the query's whole bucket range turns
-//           the histogram into the threshold tau itself: tau = lower edge of
-//           the bin that holds the P-th largest group maximum, a value <= the
+//           row's 256-bin histogram over [-1.0625, 1.0625] in shared memory.
+//           A CTA that covers the query's whole bucket range turns the
+//           histogram into the threshold tau itself: tau = lower edge of the
+//           bin that holds the P-th largest group maximum, a value <= the
 //           P-th largest group maximum <= the P-th largest score.  Otherwise
-//           the rows are added into a global per-query histogram and
-//           k_tau finishes;
-//   FILTER  append every score >= the query's threshold tau.
-// Causal masking: bucket b counts for query q only if b < 64 * H(q).
+//           the rows are added into a global per-query histogram and k_tau
+//           finishes;
+//   FILTER  every aligned group of 4 buckets whose best score is >= tau is
+//           appended as one entry (first bucket id, its 4 scores); the
+//           expansion kernel keeps the scores >= tau.
+// Causal masking: bucket b counts for query q only if b < 64 * H(q); N =
+// 64 * H is a multiple of 64, so every 64-column half tile is wholly inside
+// or outside a query's range.
 // Every mbarrier wait is bounded: a wait that runs out sets the library's
 // device error word and the CTA leaves its loops, waits (bounded) for the
 // copies it issued, frees its TMEM and exits.
@@ -44,14 +52,18 @@ __device__ int g_device_error = 0;
 namespace {
 
 constexpr int TQ = 128;             // queries per tile (MMA M)
-constexpr int TB = 256;             // centroids per tile (MMA N)
-constexpr int NST = 4;              // centroid stages
-constexpr uint32_t A_BYTES = TQ * LSA_D * 2;   // 16 KB
-constexpr uint32_t B_BYTES = TB * LSA_D * 2;   // 32 KB
-constexpr int TMEM_COLS = 512;      // two 256-column fp32 accumulators
-constexpr int THREADS = 192;        // 6 warps
-constexpr int HSTRIDE = HIST_BINS / 2 + 1;  // 32-bit words per row histogram (2 x u16 bins per word, +1 pad)
-constexpr uint32_t HIST_BYTES = TQ * HSTRIDE * 4;
+constexpr int QT = 2;               // query tiles per CTA
+constexpr int TB = 128;             // centroids per tile (MMA N)
+constexpr int NST_GMAX = 4;         // centroid stages, threshold pass (its histograms take the rest)
+constexpr int NST_FILTER = 8;       // centroid stages, filter pass
+constexpr int NST_MAX = 8;
+constexpr uint32_t A_BYTES = QT * TQ * LSA_D * 2;  // 32 KB
+constexpr uint32_t B_BYTES = TB * LSA_D * 2;       // 16 KB
+constexpr int TMEM_COLS = 512;      // [query tile][buffer] x 128 fp32 columns
+constexpr int EPI_WARPS = 4 * QT;   // 8
+constexpr int THREADS = 64 + 32 * EPI_WARPS;  // 320
+constexpr int HSTRIDE = HIST_BINS / 2 + 1;   // 32-bit words per row histogram (2 x u16 bins per word, +1 pad)
+constexpr uint32_t HIST_BYTES = QT * TQ * HSTRIDE * 4;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -119,7 +131,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr)
 }
 
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
-// N = 256, M = 128.
+// N = 128, M = 128.
 constexpr uint32_t IDESC = (1u << 4)               // D format fp32
                            | (1u << 7)             // A bf16
                            | (1u << 10)            // B bf16
@@ -151,7 +163,8 @@ __device__ __forceinline__ void tc_fence_after()
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (no wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float *v)
 {
     uint32_t r[32];
     asm volatile(
@@ -162,14 +175,35 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_wait_ld()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float max4f(const float *v)
+{
+    return fmaxf(max3f(v[0], v[1], v[2]), v[3]);
+}
+
+__device__ __forceinline__ float max8f(const float *v)
+{
+    return max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+}
+
 struct TcSmem {
-    uint64_t full[NST];
-    uint64_t empty[NST];
+    uint64_t full[NST_MAX];
+    uint64_t empty[NST_MAX];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t a_full;
@@ -181,7 +215,7 @@ struct TcSmem {
 
 }  // namespace
 
-// grid: x = query tile, y = bucket-tile chunk.  block = 192 threads.
+// grid: x = pair of query tiles, y = bucket-tile chunk.  block = 320 threads.
 __global__ void __launch_bounds__(THREADS, 1)
     k_score_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, ScoreTcArgs a,
                IndexWs ws)
@@ -189,31 +223,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ __align__(1024) uint8_t tsm_raw[];
     // tiles first (1024-aligned for the 128B swizzle), control block after
     uint8_t *tsm = tsm_raw + ((1024u - (smem_u32(tsm_raw) & 1023u)) & 1023u);
+    const int nst = a.mode == 0 ? NST_GMAX : NST_FILTER;
     uint8_t *sA = tsm;
     uint8_t *sB = tsm + A_BYTES;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(tsm + A_BYTES + NST * B_BYTES);  // [TQ][HSTRIDE]
-    TcSmem *cs = reinterpret_cast<TcSmem *>(tsm + A_BYTES + NST * B_BYTES + HIST_BYTES);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(tsm + A_BYTES + nst * B_BYTES);  // [QT*TQ][HSTRIDE], GMAX only
+    TcSmem *cs = reinterpret_cast<TcSmem *>(tsm + A_BYTES + nst * B_BYTES + (a.mode == 0 ? HIST_BYTES : 0));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t q0 = (int64_t)blockIdx.x * TQ;
+    const int64_t q0 = (int64_t)blockIdx.x * (QT * TQ);
 
     if (threadIdx.x == 0) {
         cs->nmax = 0;
         cs->abort = 0;
-        for (int s = 0; s < NST; ++s) {
+        for (int s = 0; s < nst; ++s) {
             mbar_init(smem_u32(&cs->full[s]), 1);
             mbar_init(smem_u32(&cs->empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&cs->tfull[b]), 1);
-            mbar_init(smem_u32(&cs->tempty[b]), 4);
+            mbar_init(smem_u32(&cs->tempty[b]), EPI_WARPS);
         }
         mbar_init(smem_u32(&cs->a_full), 1);
         mbar_init(smem_u32(&cs->mma_done), 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
-    if (threadIdx.x < TQ) {
+    if (threadIdx.x < QT * TQ) {
         const int64_t q = q0 + threadIdx.x;
         const int N = (q < a.nq) ? ws.horizon[q] * LSA_NBKT : 0;
         atomicMax(&cs->nmax, N);
@@ -245,128 +280,155 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t abar = smem_u32(&cs->a_full);
         mbar_expect_tx(abar, A_BYTES);
         if (a.extra_tx == 0) tma_load_2d(smem_u32(sA), &tmA, 0, (int)q0, abar);  // test hook: never arrives
+        int s = 0, ph = 0;
         for (int it = 0; it < ntiles; ++it) {
-            const int s = it % NST;
-            if (it >= NST && !wait_bounded(smem_u32(&cs->empty[s]), (uint32_t)(((it / NST) - 1) & 1), a.wait_limit,
-                                           abort))
-                break;
+            if (it >= nst && !wait_bounded(smem_u32(&cs->empty[s]), (uint32_t)(ph ^ 1), a.wait_limit, abort)) break;
             const uint32_t bar = smem_u32(&cs->full[s]);
             mbar_expect_tx(bar, B_BYTES);
             tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, 0, (int)((j0 + it) * TB), bar);
             ++issued;
+            if (++s == nst) {
+                s = 0;
+                ph ^= 1;
+            }
         }
     } else if (warp == 1 && lane == 0) {
         if (wait_bounded(smem_u32(&cs->a_full), 0, a.wait_limit, abort)) {
             tc_fence_after();
             const uint32_t a_addr = smem_u32(sA);
+            int s = 0, ph = 0;
             for (int it = 0; it < ntiles; ++it) {
-                const int s = it % NST, buf = it & 1;
-                if (!wait_bounded(smem_u32(&cs->full[s]), (uint32_t)((it / NST) & 1), a.wait_limit, abort)) break;
+                const int buf = it & 1;
+                if (!wait_bounded(smem_u32(&cs->full[s]), (uint32_t)ph, a.wait_limit, abort)) break;
                 if (it >= 2 &&
                     !wait_bounded(smem_u32(&cs->tempty[buf]), (uint32_t)(((it >> 1) - 1) & 1), a.wait_limit, abort))
                     break;
                 tc_fence_after();
                 const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
-                const uint32_t d = tmem + (uint32_t)(buf * TB);
 #pragma unroll
-                for (int k = 0; k < LSA_D / 16; ++k)
-                    mma_bf16(d, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), k > 0 ? 1u : 0u);
+                for (int qt = 0; qt < QT; ++qt) {
+                    const uint32_t d = tmem + (uint32_t)((qt * 2 + buf) * TB);
+                    const uint32_t aq = a_addr + (uint32_t)(qt * TQ * LSA_D * 2);
+#pragma unroll
+                    for (int k = 0; k < LSA_D / 16; ++k)
+                        mma_bf16(d, smem_desc(aq + k * 32), smem_desc(b_addr + k * 32), k > 0 ? 1u : 0u);
+                }
                 mma_commit(smem_u32(&cs->empty[s]));
                 mma_commit(smem_u32(&cs->tfull[buf]));
+                if (++s == nst) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
         }
     } else if (warp >= 2) {
-        // epilogue: thread owns TMEM lane (query row) r
-        const int sub = warp & 3;
-        const int r = sub * 32 + lane;
-        const int64_t q = q0 + r;
+        // epilogue: thread owns row r of query tile qt (TMEM lane 32 * quad + lane)
+        const int quad = warp & 3;
+        const int qt = (warp - 2) >> 2;
+        const int r = quad * 32 + lane;
+        const int64_t q = q0 + qt * TQ + r;
         const int N = (q < a.nq) ? ws.horizon[q] * LSA_NBKT : 0;
         const int g = group_width(N, a.P);
         const float tau = (a.mode == 1 && q < a.nq) ? ws.tau[q] : 0.0f;
         const float NEG = __int_as_float(0xff800000);
-        uint32_t *hrow = hist + r * HSTRIDE;
+        uint32_t *hrow = hist + (qt * TQ + r) * HSTRIDE;
         if (a.mode == 0)
             for (int w = 0; w < HSTRIDE; ++w) hrow[w] = 0u;
         // count one group maximum in the row histogram (saturating u16 bins)
         auto count = [&](float m) {
-            int bin = __float2int_rd((m - HIST_LO) * (HIST_BINS / (2.0f * -HIST_LO)));
-            bin = min(max(bin, 0), HIST_BINS - 1);
+            const int bin = hist_bin(m);
             const uint32_t w = hrow[bin >> 1];
             const uint32_t sh = (bin & 1) * 16;
             if (((w >> sh) & 0xffffu) != 0xffffu) hrow[bin >> 1] = w + (1u << sh);
         };
-        float *sc = (a.store && q < a.nq) ? ws.scores + q * ws.score_stride : nullptr;
-        int own = 0;  // candidates this thread appended (FILTER)
+        float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
+        int32_t *cg = ws.cand_g + q * ws.cap;
+        int own = 0;  // group entries this thread appended (FILTER)
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(qt * 2 * TB);
         for (int it = 0; it < ntiles; ++it) {
             const int buf = it & 1;
             const bool ok = wait_bounded(smem_u32(&cs->tfull[buf]), (uint32_t)((it >> 1) & 1), a.wait_limit, abort);
             if (!__all_sync(LSA_FULL, ok)) break;  // warp-uniform: tcgen05.ld needs the whole warp
             tc_fence_after();
+            float v[TB];
+#pragma unroll
+            for (int c = 0; c < TB / 32; ++c) tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + c * 32), v + c * 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&cs->tempty[buf]));  // the MMA may refill this buffer now
             const int64_t tb0 = (j0 + it) * TB;
-            float run = NEG;  // running maximum of a 64- or 128-bucket group
-#pragma unroll 1
-            for (int c = 0; c < TB / 32; ++c) {
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + (uint32_t)(buf * TB + c * 32), v);
-                const int64_t b0 = tb0 + c * 32;
-                // N is a multiple of 64, so a 32-bucket chunk is wholly in or out
-                if (b0 >= N) continue;
+            float run = NEG;  // g = 128: maximum over the whole tile
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float *x = v + 64 * h;
+                const int64_t b0 = tb0 + 64 * h;
+                const bool in = b0 < N;
                 if (a.mode == 0) {
-                    if (sc) {
-                        float4 *dst = reinterpret_cast<float4 *>(sc + b0);
+                    if (!in) continue;
+                    if (g >= 8) {
+                        float m8[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                    }
-                    if (g == 1) {
+                        for (int j = 0; j < 8; ++j) m8[j] = max8f(x + 8 * j);
+                        if (g == 8) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) count(v[i]);
-                        continue;
-                    }
-                    // in-place max tree: after level L, v[i] (i a multiple of 2^L)
-                    // holds the maximum of buckets i .. i + 2^L - 1 of the chunk
+                            for (int j = 0; j < 8; ++j) count(m8[j]);
+                        } else if (g == 16) {
 #pragma unroll
-                    for (int L = 1; L <= 5; ++L) {
-                        const int w = 1 << L;
-#pragma unroll
-                        for (int i = 0; i < 32; i += w) v[i] = fmaxf(v[i], v[i + w / 2]);
-                        if (w == g) {
-#pragma unroll
-                            for (int i = 0; i < 32; i += w) count(v[i]);
+                            for (int j = 0; j < 4; ++j) count(fmaxf(m8[2 * j], m8[2 * j + 1]));
+                        } else if (g == 32) {
+                            count(max4f(m8));
+                            count(max4f(m8 + 4));
+                        } else {
+                            const float m64 = max8f(m8);
+                            if (g == 64) {
+                                count(m64);
+                            } else {  // g == 128: one group per tile (or its valid first half)
+                                run = fmaxf(run, m64);
+                                if (h == 1 || b0 + 64 >= N) count(run);
+                            }
                         }
-                    }
-                    if (g > 32) {
-                        run = fmaxf(run, v[0]);
-                        const int per = g / 32;  // 2 or 4 chunks per group
-                        if ((c % per) == per - 1 || b0 + 32 >= N) {
-                            count(run);
-                            run = NEG;
-                        }
+                    } else if (g == 4) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) count(max4f(x + 4 * j));
+                    } else if (g == 2) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) count(fmaxf(x[2 * j], x[2 * j + 1]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) count(x[j]);
                     }
                 } else {
-                    // count the chunk's candidates first, then reserve their
-                    // slots at once (no atomic when this CTA owns the query)
-                    int n = 0;
+                    float m4[16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) n += (v[i] >= tau);
-                    if (n) {
-                        int slot = a.whole_range ? own : atomicAdd(ws.cnt + q, n);
-                        own += n;
+                    for (int j = 0; j < 16; ++j) m4[j] = max4f(x + 4 * j);
+                    const float m64 = fmaxf(max3f(max3f(m4[0], m4[1], m4[2]), max3f(m4[3], m4[4], m4[5]),
+                                                  max3f(m4[6], m4[7], m4[8])),
+                                            max3f(max3f(m4[9], m4[10], m4[11]), max3f(m4[12], m4[13], m4[14]), m4[15]));
+                    const bool hit = in && m64 >= tau;
+                    if (!__any_sync(LSA_FULL, hit)) continue;
+                    if (hit) {
+                        int slot = own;
+                        if (!a.whole_range) {
+                            int n = 0;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            if (v[i] >= tau) {
+                            for (int j = 0; j < 16; ++j) n += m4[j] >= tau;
+                            slot = atomicAdd(ws.cnt + q, n);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (m4[j] >= tau) {
                                 if (slot < ws.cap) {
-                                    ws.cand_s[q * ws.cap + slot] = v[i];
-                                    ws.cand_id[q * ws.cap + slot] = (int32_t)(b0 + i);
+                                    c4[slot] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+                                    cg[slot] = (int32_t)(b0 + 4 * j);
                                 }
                                 ++slot;
+                                ++own;
                             }
                         }
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&cs->tempty[buf]));
         }
         if (a.mode == 1 && a.whole_range && q < a.nq) ws.cnt[q] = own;
         if (a.mode == 0 && q < a.nq && N > 0 && !*abort) {
@@ -379,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int bin = HIST_BINS - 1; bin > 0; --bin) {
                         acc += (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
                         if (acc >= a.P) {
-                            t = HIST_LO + bin * (2.0f * -HIST_LO / HIST_BINS);
+                            t = hist_edge(bin);
                             break;
                         }
                     }
@@ -396,10 +458,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncthreads();
     if (warp == 0 && lane == 0 && *abort) {
-        // copies issued but never consumed: wait for them (bounded) before exit
+        // copies that may still be in flight (the producer reused a stage only
+        // after the MMA had consumed its previous copy): wait for the last
+        // nst of them (bounded) before exit
         volatile int dummy = 0;
-        for (int it = 0; it < issued; ++it)
-            wait_bounded(smem_u32(&cs->full[it % NST]), (uint32_t)((it / NST) & 1), a.wait_limit, &dummy);
+        for (int it = max(0, issued - nst); it < issued; ++it)
+            wait_bounded(smem_u32(&cs->full[it % nst]), (uint32_t)((it / nst) & 1), a.wait_limit, &dummy);
     }
     if (warp == 1 && lane == 0) {
         // every MMA this thread issued has finished before its TMEM is freed
@@ -455,12 +519,15 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
 {
     if (a.nq <= 0 || a.nb_total <= 0) return cudaSuccess;
     CUtensorMap tmA, tmB;
-    if (!make_map(&tmA, ws.qhat, a.nq, TQ) || !make_map(&tmB, centroid_bf16, a.nb_total, TB))
+    if (!make_map(&tmA, ws.qhat, a.nq, QT * TQ) || !make_map(&tmB, centroid_bf16, a.nb_total, TB))
         return cudaErrorInvalidValue;
-    const int64_t qtiles = (a.nq + TQ - 1) / TQ;
+    const int64_t qpairs = (a.nq + QT * TQ - 1) / (QT * TQ);
     const int64_t tiles = (a.nb_total + TB - 1) / TB;
-    int64_t chunks = qtiles == 1 ? n_sm : (2LL * n_sm + qtiles - 1) / qtiles;
-    if (qtiles >= n_sm) chunks = 1;  // one CTA per query tile covers its whole range
+    // One CTA per pair of query tiles over its whole bucket range when that
+    // fills most SMs (no atomics, threshold set in place); otherwise split the
+    // range so that about four waves of CTAs balance the SMs.
+    int64_t chunks = 1;
+    if (qpairs * 4 < (int64_t)n_sm * 3) chunks = (4LL * n_sm + qpairs - 1) / qpairs;
     if (chunks > tiles) chunks = tiles;
     if (chunks < 1) chunks = 1;
     if (chunks > 65535) chunks = 65535;
@@ -469,10 +536,11 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
     chunks = (tiles + b.chunk_tiles - 1) / b.chunk_tiles;
     b.whole_range = (chunks == 1) ? 1 : 0;
     if (whole_range) *whole_range = b.whole_range;
-    const size_t smem = A_BYTES + NST * B_BYTES + HIST_BYTES + sizeof(TcSmem) + 1024;
+    const size_t smem = A_BYTES + (size_t)(a.mode == 0 ? NST_GMAX : NST_FILTER) * B_BYTES +
+                        (a.mode == 0 ? HIST_BYTES : 0) + sizeof(TcSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_score_tc<<<dim3((unsigned)qtiles, (unsigned)chunks), THREADS, smem, st>>>(tmA, tmB, b, ws);
+    k_score_tc<<<dim3((unsigned)qpairs, (unsigned)chunks), THREADS, smem, st>>>(tmA, tmB, b, ws);
     count_launches(1);
     return cudaGetLastError();
 }

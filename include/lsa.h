@@ -270,8 +270,8 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
  * until the process exits.  The call allocates nothing.  Requests needing more
  * than that (lsa_index_workspace_bytes(nq, cache->n_blocks, p) > 16 MiB) are
  * rejected with LSA_ERR_WORKSPACE and a message saying so; nothing is
- * enqueued then.  At k = 4096 this admits up to 240 Flat queries over 1M
- * tokens; over 10M tokens it admits 1-3 or 17-233 queries (batches of 16 or
+ * enqueued then.  At k = 4096 this admits up to 201 Flat queries over 1M
+ * tokens; over 10M tokens it admits 1-3 or 17-201 queries (batches of 16 or
  * fewer keep every bucket score, 5 MB per query at 10M).
  *
  * The first call on a device looks up the array's device address (with that

@@ -223,12 +223,19 @@ def test_end_to_end_tiny_layer(tiny):
 
 
 def test_small_and_large_batch_paths_agree(tiny):
-    """Batches of up to 16 queries (decode path) and larger batches (prefill
-    path) give bit-identical lists for the same queries."""
-    keys, q, pos, _ = tiny
+    """Batches of up to 16 queries (decode path: CUDA-core scores) and larger
+    batches (prefill path: tensor-core scores) give the oracle's lists for the
+    same queries; the two score sums may differ in the last bit, so lists may
+    differ only by near-ties at the k cut, and almost never do."""
+    keys, q, pos, oc = tiny
     cache, _, p = _build_gpu(keys, k=256)
     sel = np.arange(100, 4096, 97)[:40].astype(np.int64)
     big_l, big_n = _index_gpu(cache, None, p, q[sel], pos[sel])
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    PT.assert_lists_match(big_l, big_n, ol, on, q[sel], pos[sel], oc, k=256)
+    same = 0
     for a in range(0, len(sel), 8):
         sl, sn = _index_gpu(cache, None, p, q[sel[a:a + 8]], pos[sel[a:a + 8]], decode=True)
-        assert np.array_equal(sn, big_n[a:a + 8]) and np.array_equal(sl, big_l[a:a + 8])
+        PT.assert_lists_match(sl, sn, ol[a:a + 8], on[a:a + 8], q[sel[a:a + 8]], pos[sel[a:a + 8]], oc, k=256)
+        same += sum(int(sn[i] == big_n[a + i] and np.array_equal(sl[i], big_l[a + i])) for i in range(len(sn)))
+    assert same >= len(sel) - 2
