@@ -232,32 +232,34 @@ __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int 
 }
 
 // ---------------------------------------------------------------------------
-// Block-wide inclusive scan of a[0..n) in shared memory (any block size up
-// to 1024 threads).
+// Block-wide inclusive scan of a[0..n) in shared memory.  Warp w scans the
+// contiguous segment [w * seg, (w + 1) * seg) 32 elements at a time, lane i
+// on element i (no bank conflicts), carrying the running total; then the
+// segment totals are added in.  Any block size up to 1024 threads.
 template <typename T>
 __device__ void block_inclusive_scan(T *a, int n, T *wsum)
 {
-    const int t = threadIdx.x;
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int lo = min(n, t * per), hi = min(n, lo + per);
-    T s = 0;
-    for (int i = lo; i < hi; ++i) {
-        s += a[i];
-        a[i] = s;
-    }
-    // exclusive scan of per-thread totals
-    const int lane = t & 31, w = t >> 5;
-    T x = s;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int seg = (((n + nw - 1) / nw) + 31) & ~31;
+    const int lo = min(n, w * seg), hi = min(n, lo + seg);
+    T carry = 0;
+    for (int base = lo; base < hi; base += 32) {  // warp-uniform
+        const int i = base + lane;
+        T x = i < hi ? a[i] : T(0);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        T y = __shfl_up_sync(LSA_FULL, x, o);
-        if (lane >= o) x += y;
+        for (int o = 1; o < 32; o <<= 1) {
+            const T y = __shfl_up_sync(LSA_FULL, x, o);
+            if (lane >= o) x += y;
+        }
+        if (i < hi) a[i] = x + carry;
+        carry += __shfl_sync(LSA_FULL, x, 31);
     }
-    if (lane == 31) wsum[w] = x;
+    if (lane == 0) wsum[w] = carry;
     __syncthreads();
-    T before = x - s;
+    T before = 0;
     for (int k = 0; k < w; ++k) before += wsum[k];
-    for (int i = lo; i < hi; ++i) a[i] += before;
+    if (before != T(0))
+        for (int i = lo + lane; i < hi; i += 32) a[i] += before;
     __syncthreads();
 }
 
@@ -317,16 +319,25 @@ __global__ void __launch_bounds__(256) k_tau(int64_t nq, int P, IndexWs ws)
 // the batch, stored for the filter pass, with each query's group maxima
 // counted into its global histogram.  A CTA of DS_WARPS warps takes
 // DS_WARPS * 128 consecutive buckets; a warp takes an aligned run of 128
-// (groups are at most 128 buckets, so none straddles two warps), 32 at a time,
-// one bucket per lane.
+// (groups are at most 128 buckets, so none straddles two warps), 32 rows at
+// a time: the rows are copied with coalesced 16-byte cp.async (a warp
+// instruction moves 4 whole rows) into a padded shared tile, double-buffered,
+// and lane i then scores row i from there.
 constexpr int DS_WARPS = 4;
 constexpr int DS_SPAN = DS_WARPS * 128;
+constexpr int DS_ROW = 144;  // bytes per staged row: 128 + 16 (bank-conflict-free 16-byte reads)
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
 
 __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb_total,
                                                           const uint16_t *__restrict__ cbf, int P, IndexWs ws)
 {
     __shared__ __align__(16) float qf[SMALL_NQ][LSA_D];
     __shared__ uint32_t hs[SMALL_NQ][HIST_BINS];
+    extern __shared__ __align__(16) uint8_t ds_dyn[];  // [DS_WARPS][2][32 * DS_ROW] staged rows
     __shared__ int Nq[SMALL_NQ], gq[SMALL_NQ];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     for (int i = t; i < nq * LSA_D; i += blockDim.x) qf[i / LSA_D][i % LSA_D] = bf_bits2f(ws.qhat[i]);
@@ -336,29 +347,48 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
         Nq[t] = N;
         gq[t] = group_width(N, P);
     }
-    __syncthreads();
     const float NEG = __int_as_float(0xff800000);
     const int64_t wbase = (int64_t)blockIdx.x * DS_SPAN + warp * 128;
+    // copy the 32 rows of round r into stage[warp][r & 1]: instruction v moves
+    // rows 4v .. 4v + 3, lane l the 16 bytes l % 8 of row 4v + l / 8; rows past
+    // the end are zero-filled (source clamped to row 0, nothing read)
+    auto issue = [&](int r) {
+        const uint32_t dst0 = (uint32_t)__cvta_generic_to_shared(ds_dyn + (warp * 2 + (r & 1)) * 32 * DS_ROW);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const int row = 4 * v + (lane >> 3);
+            const int64_t b = wbase + r * 32 + row;
+            const bool ok = b < nb_total;
+            cp_async16(dst0 + row * DS_ROW + (lane & 7) * 16, cbf + (ok ? b : 0) * LSA_D + (lane & 7) * 8,
+                       ok ? 16u : 0u);
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    issue(0);
+    __syncthreads();
     float run[SMALL_NQ];
 #pragma unroll
     for (int i = 0; i < SMALL_NQ; ++i) run[i] = NEG;
     for (int r = 0; r < 4; ++r) {
+        if (r + 1 < 4) {
+            issue(r + 1);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+        }
+        __syncwarp();
         const int64_t b = wbase + r * 32 + lane;
         uint32_t cw[32];
-        if (b < nb_total) {
-            const uint4 *c4 = reinterpret_cast<const uint4 *>(cbf + b * LSA_D);
+        const uint4 *src = reinterpret_cast<const uint4 *>(ds_dyn + (warp * 2 + (r & 1)) * 32 * DS_ROW + lane * DS_ROW);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                const uint4 w = __ldg(c4 + v);
-                cw[4 * v] = w.x;
-                cw[4 * v + 1] = w.y;
-                cw[4 * v + 2] = w.z;
-                cw[4 * v + 3] = w.w;
-            }
-        } else {
-#pragma unroll
-            for (int v = 0; v < 32; ++v) cw[v] = 0u;
+        for (int v = 0; v < 8; ++v) {
+            const uint4 w = src[v];
+            cw[4 * v] = w.x;
+            cw[4 * v + 1] = w.y;
+            cw[4 * v + 2] = w.z;
+            cw[4 * v + 3] = w.w;
         }
+        __syncwarp();  // this buffer is refilled two rounds later
 #pragma unroll
         for (int qi = 0; qi < SMALL_NQ; ++qi) {
             if (qi >= nq) break;  // uniform
@@ -460,7 +490,8 @@ __host__ __device__ inline size_t rank_expand_smem(int KC, int TW)
     return (size_t)KC * 8 + (size_t)RX_SLOTS * 64 + (size_t)TW * 8 + (size_t)RX_SLOTS * 8 + (size_t)KC;
 }
 
-__global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict__ pos,
+template <int NT>
+__global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ pos,
                                                       const int32_t *__restrict__ members,
                                                       const uint16_t *__restrict__ cbf, int32_t *__restrict__ lists,
                                                       int32_t *__restrict__ lens, int Lmax, int k, int sink,
@@ -505,15 +536,36 @@ __global__ void __launch_bounds__(1024) k_rank_expand(const int64_t *__restrict_
         const float tau = ws.tau[q];
         const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + q * ws.cap;
         const int32_t *cg = ws.cand_g + q * ws.cap;
-        for (int i = t; i < ne; i += blockDim.x) {
-            const float4 s4 = c4[i];
-            const int32_t g = cg[i];
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        for (int i0 = 0; i0 < ne; i0 += blockDim.x) {  // block-uniform trip count
+            const int i = i0 + t;
+            float sv[4] = {NEG, NEG, NEG, NEG};
+            int32_t g = 0;
+            if (i < ne) {
+                const float4 s4 = c4[i];
+                g = cg[i];
+                sv[0] = s4.x;
+                sv[1] = s4.y;
+                sv[2] = s4.z;
+                sv[3] = s4.w;
+            }
+            int nc = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) nc += sv[e] >= tau && sv[e] > NEG;
+            // one shared-memory atomic per warp
+            int incl = nc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(LSA_FULL, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int base = 0;
+            if (lane == 31 && incl > 0) base = atomicAdd(&nk_s, incl);
+            int slot = __shfl_sync(LSA_FULL, base, 31) + incl - nc;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 if (sv[e] >= tau && sv[e] > NEG) {
-                    const int slot = atomicAdd(&nk_s, 1);
                     if (slot < KC) keys[slot] = rank_key(sv[e], g + e);
+                    ++slot;
                 }
             }
         }
@@ -751,8 +803,10 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     const bool small = a.nq <= SMALL_NQ;
     if (a.mode == 0 && nb_total > 0) {
         if (small) {  // stream every centroid once for the whole batch, keep the scores
-            k_dscore<<<(unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN), DS_WARPS * 32, 0, st>>>(a.nq, nb_total,
-                                                                                               a.centroid_bf16, a.P, ws);
+            const int dsm = DS_WARPS * 2 * 32 * DS_ROW;
+            cudaFuncSetAttribute(k_dscore, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+            k_dscore<<<(unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN), DS_WARPS * 32, dsm, st>>>(
+                a.nq, nb_total, a.centroid_bf16, a.P, ws);
             count_launches(1);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             k_dfilter<<<(unsigned)((nb_total / 4 + 255) / 256), 256, 0, st>>>(a.nq, a.P, ws);
@@ -792,10 +846,15 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
     const int KC = ws.cap;
     const size_t smr = rank_expand_smem(KC, TW);
-    cudaFuncSetAttribute(k_rank_expand, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-    k_rank_expand<<<(unsigned)a.nq, small ? 1024 : 256, smr, st>>>(a.pos, a.members, a.centroid_bf16, a.lists,
-                                                                   a.lens, a.Lmax, a.k, a.sink, a.window, a.P, KC,
-                                                                   TW, ws);
+    if (small) {  // one CTA per query, few queries: widest blocks
+        cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        k_rank_expand<1024><<<(unsigned)a.nq, 1024, smr, st>>>(a.pos, a.members, a.centroid_bf16, a.lists, a.lens,
+                                                               a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ws);
+    } else {
+        cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.centroid_bf16, a.lists, a.lens,
+                                                             a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ws);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

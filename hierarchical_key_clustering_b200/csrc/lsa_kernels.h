@@ -57,13 +57,16 @@ __device__ __forceinline__ float hist_edge(int bin)
 {
     return HIST_LO + (float)bin * HIST_BIN_W;
 }
-// Bin of a group maximum m, rounded so that its lower edge is <= m.
+// Bin of a group maximum m, rounded so that its lower edge is <= m: the bin
+// coordinate (m - HIST_LO) / HIST_BIN_W is computed with one fused multiply-add
+// and lowered by 1e-4 of a bin, more than that multiply-add's total rounding
+// error (< 4e-5 of a bin for |m| <= 1.0625), so its floor never exceeds the
+// exact one.  A maximum within 1e-4 of a bin above an edge may land one bin
+// low, which only lowers tau.
 __device__ __forceinline__ int hist_bin(float m)
 {
-    int bin = __float2int_rd(__fmul_rn(__fsub_rn(m, HIST_LO), 1.0f / HIST_BIN_W));
-    bin = min(max(bin, 0), HIST_BINS - 1);
-    if (bin > 0 && m < hist_edge(bin)) --bin;
-    return bin;
+    const float c = fmaf(m, 1.0f / HIST_BIN_W, -HIST_LO / HIST_BIN_W - 1e-4f);
+    return min(max(__float2int_rd(c), 0), HIST_BINS - 1);
 }
 #endif
 

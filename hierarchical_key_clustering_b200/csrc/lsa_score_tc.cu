@@ -201,6 +201,17 @@ __device__ __forceinline__ float max8f(const float *v)
     return max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
 }
 
+// Candidate entry (4 scores + first bucket id), stored only when p != 0.
+__device__ __forceinline__ void st_entry_if(int p, float4 *d4, int32_t *dg, const float *x, int32_t g)
+{
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n"
+        " @q st.global.v4.f32 [%1], {%2, %3, %4, %5};\n"
+        " @q st.global.b32 [%6], %7;\n}\n" ::"r"(p),
+        "l"(d4), "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "l"(dg), "r"(g)
+        : "memory");
+}
+
 struct TcSmem {
     uint64_t full[NST_MAX];
     uint64_t empty[NST_MAX];
@@ -334,12 +345,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t *hrow = hist + (qt * TQ + r) * HSTRIDE;
         if (a.mode == 0)
             for (int w = 0; w < HSTRIDE; ++w) hrow[w] = 0u;
-        // count one group maximum in the row histogram (saturating u16 bins)
+        // Count one group maximum in the row histogram (saturating u16 bins).
+        // bL tracks the bin holding the P-th largest maximum counted so far
+        // (S = counts in bins >= bL); once P maxima are at or above its edge
+        // lm, a smaller maximum can only land below the final threshold bin
+        // (bL never falls, here or in the merged histogram of a split range),
+        // so it is not counted.
+        int bL = 0, S = 0;
+        float lm = NEG;
+        auto hcount = [&](int b) { return (int)((hrow[b >> 1] >> ((b & 1) * 16)) & 0xffffu); };
         auto count = [&](float m) {
+            if (m < lm) return;
             const int bin = hist_bin(m);
             const uint32_t w = hrow[bin >> 1];
             const uint32_t sh = (bin & 1) * 16;
-            if (((w >> sh) & 0xffffu) != 0xffffu) hrow[bin >> 1] = w + (1u << sh);
+            if (((w >> sh) & 0xffffu) == 0xffffu) return;
+            hrow[bin >> 1] = w + (1u << sh);
+            if (bin < bL) return;
+            ++S;
+            while (S - hcount(bL) >= a.P) S -= hcount(bL++);
+            if (S >= a.P) lm = hist_edge(bL);
         };
         float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
         int32_t *cg = ws.cand_g + q * ws.cap;
@@ -350,18 +375,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool ok = wait_bounded(smem_u32(&cs->tfull[buf]), (uint32_t)((it >> 1) & 1), a.wait_limit, abort);
             if (!__all_sync(LSA_FULL, ok)) break;  // warp-uniform: tcgen05.ld needs the whole warp
             tc_fence_after();
-            float v[TB];
-#pragma unroll
-            for (int c = 0; c < TB / 32; ++c) tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + c * 32), v + c * 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&cs->tempty[buf]));  // the MMA may refill this buffer now
             const int64_t tb0 = (j0 + it) * TB;
             float run = NEG;  // g = 128: maximum over the whole tile
-#pragma unroll
+#pragma unroll 1
             for (int h = 0; h < 2; ++h) {
-                const float *x = v + 64 * h;
+                // one 64-column half at a time (registers); after the second
+                // half is read the MMA may refill this buffer
+                float x[64];
+                tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + h * 64), x);
+                tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + h * 64 + 32), x + 32);
+                tmem_wait_ld();
+                if (h == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&cs->tempty[buf]));
+                }
                 const int64_t b0 = tb0 + 64 * h;
                 const bool in = b0 < N;
                 if (a.mode == 0) {
@@ -409,21 +437,28 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (!__any_sync(LSA_FULL, hit)) continue;
                     if (hit) {
                         int slot = own;
-                        if (!a.whole_range) {
+                        if (!a.whole_range) {  // reserve this half tile's entries
                             int n = 0;
 #pragma unroll
                             for (int j = 0; j < 16; ++j) n += m4[j] >= tau;
                             slot = atomicAdd(ws.cnt + q, n);
                         }
+                        if (slot + 16 <= ws.cap) {  // every entry fits: predicated stores, no branches
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (m4[j] >= tau) {
-                                if (slot < ws.cap) {
-                                    c4[slot] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
-                                    cg[slot] = (int32_t)(b0 + 4 * j);
+                            for (int j = 0; j < 16; ++j) {
+                                const int pj = m4[j] >= tau;
+                                st_entry_if(pj, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
+                                slot += pj;
+                                own += pj;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                if (m4[j] >= tau) {
+                                    if (slot < ws.cap) st_entry_if(1, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
+                                    ++slot;
+                                    ++own;
                                 }
-                                ++slot;
-                                ++own;
                             }
                         }
                     }
