@@ -201,6 +201,32 @@ __device__ __forceinline__ float max8f(const float *v)
     return max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
 }
 
+// One query row's group-maximum histogram in shared memory (256 saturating
+// u16 bins, two per word).  bL tracks the bin holding the P-th largest
+// maximum counted so far and S the counts in bins >= bL; once P maxima are at
+// or above its edge lm, a smaller maximum can only land below the final
+// threshold bin (bL never falls, here or in the merged histogram of a split
+// range), so it is not counted.
+struct RowHist {
+    uint32_t *h;
+    int bL, S;
+    float lm;
+    __device__ __forceinline__ int at(int b) const { return (int)((h[b >> 1] >> ((b & 1) * 16)) & 0xffffu); }
+    __device__ __forceinline__ void add(float m, int P)
+    {
+        if (m < lm) return;
+        const int bin = hist_bin(m);
+        const uint32_t w = h[bin >> 1];
+        const uint32_t sh = (bin & 1) * 16;
+        if (((w >> sh) & 0xffffu) == 0xffffu) return;
+        h[bin >> 1] = w + (1u << sh);
+        if (bin < bL) return;
+        ++S;
+        while (S - at(bL) >= P) S -= at(bL++);
+        if (S >= P) lm = hist_edge(bL);
+    }
+};
+
 // Candidate entry (4 scores + first bucket id), stored only when p != 0.
 __device__ __forceinline__ void st_entry_if(int p, float4 *d4, int32_t *dg, const float *x, int32_t g)
 {
@@ -270,6 +296,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int64_t j1 = min(j0 + a.chunk_tiles, tiles_all);
     const int ntiles = j1 > j0 ? (int)(j1 - j0) : 0;
     if (ntiles == 0) return;  // uniform: nothing allocated yet
+    // CTAs start their walk at evenly spread tiles of the range (and wrap), so
+    // that at any moment they read different centroid tiles instead of all
+    // pulling the same lines from the same L2 slices
+    const int rot = (int)(((int64_t)blockIdx.x * ntiles) / gridDim.x);
+    auto tile_of = [&](int it) {
+        const int r = it + rot;
+        return j0 + (r >= ntiles ? r - ntiles : r);
+    };
 
     volatile int *abort = &cs->abort;
     if (warp == 1) {  // whole warp: TMEM allocation
@@ -296,7 +330,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (it >= nst && !wait_bounded(smem_u32(&cs->empty[s]), (uint32_t)(ph ^ 1), a.wait_limit, abort)) break;
             const uint32_t bar = smem_u32(&cs->full[s]);
             mbar_expect_tx(bar, B_BYTES);
-            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, 0, (int)((j0 + it) * TB), bar);
+            tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, 0, (int)(tile_of(it) * TB), bar);
             ++issued;
             if (++s == nst) {
                 s = 0;
@@ -345,27 +379,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t *hrow = hist + (qt * TQ + r) * HSTRIDE;
         if (a.mode == 0)
             for (int w = 0; w < HSTRIDE; ++w) hrow[w] = 0u;
-        // Count one group maximum in the row histogram (saturating u16 bins).
-        // bL tracks the bin holding the P-th largest maximum counted so far
-        // (S = counts in bins >= bL); once P maxima are at or above its edge
-        // lm, a smaller maximum can only land below the final threshold bin
-        // (bL never falls, here or in the merged histogram of a split range),
-        // so it is not counted.
-        int bL = 0, S = 0;
-        float lm = NEG;
-        auto hcount = [&](int b) { return (int)((hrow[b >> 1] >> ((b & 1) * 16)) & 0xffffu); };
-        auto count = [&](float m) {
-            if (m < lm) return;
-            const int bin = hist_bin(m);
-            const uint32_t w = hrow[bin >> 1];
-            const uint32_t sh = (bin & 1) * 16;
-            if (((w >> sh) & 0xffffu) == 0xffffu) return;
-            hrow[bin >> 1] = w + (1u << sh);
-            if (bin < bL) return;
-            ++S;
-            while (S - hcount(bL) >= a.P) S -= hcount(bL++);
-            if (S >= a.P) lm = hist_edge(bL);
-        };
+        // Count one group maximum in the row histogram (saturating u16 bins);
+        // see RowHist for the bound that lets most maxima go uncounted.
+        RowHist rh{hrow, 0, 0, NEG};
+        auto count = [&](float m) { rh.add(m, a.P); };
         float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
         int32_t *cg = ws.cand_g + q * ws.cap;
         int own = 0;  // group entries this thread appended (FILTER)
@@ -375,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool ok = wait_bounded(smem_u32(&cs->tfull[buf]), (uint32_t)((it >> 1) & 1), a.wait_limit, abort);
             if (!__all_sync(LSA_FULL, ok)) break;  // warp-uniform: tcgen05.ld needs the whole warp
             tc_fence_after();
-            const int64_t tb0 = (j0 + it) * TB;
+            const int64_t tb0 = tile_of(it) * TB;
             float run = NEG;  // g = 128: maximum over the whole tile
 #pragma unroll 1
             for (int h = 0; h < 2; ++h) {
@@ -427,12 +444,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int j = 0; j < 64; ++j) count(x[j]);
                     }
                 } else {
-                    float m4[16];
+                    float m4[16], m16[4];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) m4[j] = max4f(x + 4 * j);
-                    const float m64 = fmaxf(max3f(max3f(m4[0], m4[1], m4[2]), max3f(m4[3], m4[4], m4[5]),
-                                                  max3f(m4[6], m4[7], m4[8])),
-                                            max3f(max3f(m4[9], m4[10], m4[11]), max3f(m4[12], m4[13], m4[14]), m4[15]));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) m16[j] = max4f(m4 + 4 * j);
+                    const float m64 = max4f(m16);
                     const bool hit = in && m64 >= tau;
                     if (!__any_sync(LSA_FULL, hit)) continue;
                     if (hit) {
@@ -443,13 +460,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                             for (int j = 0; j < 16; ++j) n += m4[j] >= tau;
                             slot = atomicAdd(ws.cnt + q, n);
                         }
-                        if (slot + 16 <= ws.cap) {  // every entry fits: predicated stores, no branches
+                        if (slot + 16 <= ws.cap) {  // every entry fits: predicated stores per 16-bucket block
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int pj = m4[j] >= tau;
-                                st_entry_if(pj, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
-                                slot += pj;
-                                own += pj;
+                            for (int kb = 0; kb < 4; ++kb) {
+                                if (m16[kb] < tau) continue;
+#pragma unroll
+                                for (int j = 4 * kb; j < 4 * kb + 4; ++j) {
+                                    const int pj = m4[j] >= tau;
+                                    st_entry_if(pj, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
+                                    slot += pj;
+                                    own += pj;
+                                }
                             }
                         } else {
 #pragma unroll
