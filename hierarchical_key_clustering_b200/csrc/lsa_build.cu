@@ -92,6 +92,41 @@ __device__ __forceinline__ ArgMin block_argmin128(float d, int ij, float *red_d,
     return r;
 }
 
+// Minimum of row r over the columns j < m, j != r, with ok(j), ties to the
+// lowest j -- exactly what an ascending scan keeping the first strictly
+// smaller value finds ((+inf, -1) when no column qualifies).  The whole warp
+// computes it (lane l looks at columns l, l + 32, l + 64, l + 96) and every
+// lane gets it.
+template <typename Ok>
+__device__ __forceinline__ void warp_row_min(const float *row, int r, int m, Ok ok, float &best, int &bj)
+{
+    const int lane = threadIdx.x & 31;
+    float b = __int_as_float(0x7f800000);
+    int jb = -1;
+#pragma unroll
+    for (int k = 0; k < LSA_NITEMS / 32; ++k) {
+        const int j = lane + 32 * k;
+        if (j < m && j != r && ok(j)) {
+            const float v = row[j];
+            if (v < b) {
+                b = v;
+                jb = j;
+            }
+        }
+    }
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const float b2 = __shfl_xor_sync(LSA_FULL, b, s);
+        const int j2 = __shfl_xor_sync(LSA_FULL, jb, s);
+        if (j2 >= 0 && (jb < 0 || b2 < b || (b2 == b && j2 < jb))) {
+            b = b2;
+            jb = j2;
+        }
+    }
+    best = b;
+    bj = jb;
+}
+
 // Fill D[i][j] = f_ij * |Y_i - Y_j|^2 (fixed order), where f_ij = fac(i, j).
 // Thread t handles pairs (t, (t + delta) mod 128), delta = 1..63, and
 // delta = 64 for t < 64: every unordered pair exactly once.
@@ -155,22 +190,28 @@ __global__ void __launch_bounds__(128) k_ward(const float *__restrict__ pooled, 
     __syncthreads();
 
     const int DEAD = 1000;
+    const float INF = __int_as_float(0x7f800000);
     bool failed = false;
-    for (int it = 0; it < LSA_NITEMS - LSA_NBKT; ++it) {
-        float best = __int_as_float(0x7f800000);
-        int bj = -1;
-        const int nt = nl[t];
-        if (nt < DEAD) {
-            const float *row = D + t * DS;
-            for (int j = 0; j < LSA_NITEMS; ++j) {
-                if (j == t || nt + nl[j] > cap) continue;
-                float v = row[j];
-                if (v < best) {
-                    best = v;
-                    bj = j;
-                }
+    // Row minima: thread t keeps the cheapest eligible partner of cluster t
+    // (n_t + n_j <= cap, ties to the lowest j).  A merge of (i, j) into i
+    // changes only column i (new costs) and column j (gone), so a row needs a
+    // rescan only if it is row i or its partner was i or j; every other row
+    // just weighs its new cost to i.
+    float best = INF;
+    int bj = -1;
+    {
+        const float *row = D + t * DS;
+        for (int j = 0; j < LSA_NITEMS; ++j) {
+            if (j == t || 1 + nl[j] > cap) continue;
+            const float v = row[j];
+            if (v < best) {
+                best = v;
+                bj = j;
             }
         }
+    }
+    for (int it = 0; it < LSA_NITEMS - LSA_NBKT; ++it) {
+        const int nt = nl[t];
         int ij = (bj < 0) ? 0x7fffffff : (min(t, bj) * LSA_NITEMS + max(t, bj));
         ArgMin am = block_argmin128(best, ij, red_d, red_ij);
         if (am.ij == 0x7fffffff) {  // no finite eligible cost: non-finite keys
@@ -193,6 +234,31 @@ __global__ void __launch_bounds__(128) k_ward(const float *__restrict__ pooled, 
         if (t == bi) nl[t] = ni + nj;
         if (t == bjj) nl[t] = DEAD;
         __syncthreads();
+        const int ntn = nl[t];
+        const bool live = ntn < DEAD;
+        const bool need = live && (t == bi || bj == bi || bj == bjj);
+        if (!live) {
+            best = INF;
+            bj = -1;
+        } else if (!need && ntn + nl[bi] <= cap) {
+            const float v = D[t * DS + bi];
+            if (v < best || (v == best && bi < bj)) {
+                best = v;
+                bj = bi;
+            }
+        }
+        for (unsigned pend = __ballot_sync(LSA_FULL, need); pend; pend &= pend - 1) {
+            const int l = __ffs(pend) - 1;
+            const int r = (t & ~31) + l;
+            const int nr = nl[r];
+            float b2;
+            int j2;
+            warp_row_min(D + r * DS, r, LSA_NITEMS, [&](int j) { return nr + nl[j] <= cap; }, b2, j2);
+            if ((t & 31) == l) {
+                best = b2;
+                bj = j2;
+            }
+        }
     }
 
     if (failed) {  // leave this block's buckets empty rather than write out of range
@@ -318,20 +384,23 @@ __global__ void __launch_bounds__(128) k_tree_pair(TreeDev tr, int64_t off_prev,
     });
     __syncthreads();
 
-    for (int it = 0; it < m / 2; ++it) {
-        float best = __int_as_float(0x7f800000);
-        int bj = -1;
-        if (partner[t] == -1) {
-            const float *row = D + t * DS;
-            for (int j = 0; j < m; ++j) {
-                if (j == t || partner[j] != -1) continue;
-                float v = row[j];
-                if (v < best) {
-                    best = v;
-                    bj = j;
-                }
+    // Row minima over unpaired partners (ties to the lowest j); pairing (i, j)
+    // removes columns i and j, so only rows whose partner was i or j rescan.
+    const float INF = __int_as_float(0x7f800000);
+    float best = INF;
+    int bj = -1;
+    if (partner[t] == -1) {
+        const float *row = D + t * DS;
+        for (int j = 0; j < m; ++j) {
+            if (j == t || partner[j] != -1) continue;
+            const float v = row[j];
+            if (v < best) {
+                best = v;
+                bj = j;
             }
         }
+    }
+    for (int it = 0; it < m / 2; ++it) {
         int ij = (bj < 0) ? 0x7fffffff : (min(t, bj) * LSA_NITEMS + max(t, bj));
         ArgMin am = block_argmin128(best, ij, red_d, red_ij);
         if (am.ij == 0x7fffffff) break;  // only non-finite costs left
@@ -339,6 +408,23 @@ __global__ void __launch_bounds__(128) k_tree_pair(TreeDev tr, int64_t off_prev,
         if (t == bi) partner[t] = bjj;
         if (t == bjj) partner[t] = bi;
         __syncthreads();
+        const bool open = partner[t] == -1;
+        const bool need = open && (bj == bi || bj == bjj);
+        if (!open) {
+            best = INF;
+            bj = -1;
+        }
+        for (unsigned pend = __ballot_sync(LSA_FULL, need); pend; pend &= pend - 1) {
+            const int l = __ffs(pend) - 1;
+            const int r = (t & ~31) + l;
+            float b2;
+            int j2;
+            warp_row_min(D + r * DS, r, m, [&](int j) { return partner[j] == -1; }, b2, j2);
+            if ((t & 31) == l) {
+                best = b2;
+                bj = j2;
+            }
+        }
     }
     if (t == 0) {  // pair whatever is still unpaired in index order (no-op for finite costs)
         int open = -1, left = 0;
