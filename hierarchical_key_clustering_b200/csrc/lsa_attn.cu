@@ -11,8 +11,8 @@
 // head[, key split]) unit: its G = Hq/Hkv heads form the rows of a 16-row
 // mma.sync tile (rows >= G are zero), 16 gathered keys form a chunk, and an
 // fp32 online softmax carries the running max and sum.  K/V rows are
-// gathered with cp.async (16 B per lane) into a 3-stage ring in shared
-// memory; each warp loads the list indices of the next chunk one issue ahead,
+// gathered with cp.async (16 B per lane) into a 3-stage ring of swizzled
+// 256-byte rows in shared memory; each warp loads the list indices of the next chunk one issue ahead,
 // so a gather never waits on a dependent index load.  The warps of a CTA are
 // independent (no CTA barrier), which keeps many gathers in flight per SM.
 // Units run head-major (all queries of KV head 0, then head 1, ...): the K/V
@@ -33,13 +33,23 @@
 namespace lsa {
 
 constexpr int KCH = 16;                          // keys per chunk
-constexpr int ROWB = 136;                        // bf16 per smem row (128 + 8 pad)
+constexpr int ROWB = 128;                        // bf16 per smem row (256 B, 16-byte segments XOR-swizzled)
 constexpr int NST = 3;                           // pipeline stages
 constexpr int STAGE_BYTES = 2 * KCH * ROWB * 2;  // K + V
 constexpr int WARP_BYTES = NST * STAGE_BYTES;
 constexpr int AWARPS = 4;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
+
+// Byte offset of the 16-byte segment `seg` (dims 8 seg .. 8 seg + 7) of row
+// `row` in a staged K or V tile.  Rows are 256 B, so every 32-byte sector of
+// a gathered row lands in one aligned 32-byte piece of shared memory (the XOR
+// keeps segment pairs 2k, 2k + 1 together), and the XOR with row & 7 puts the
+// 8 rows an ldmatrix reads at one logical segment in 8 different bank groups.
+__device__ __forceinline__ uint32_t tile_off(int row, int seg)
+{
+    return (uint32_t)(row * (ROWB * 2) + ((seg ^ (row & 7)) << 4));
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -96,6 +106,23 @@ __device__ __forceinline__ uint32_t ld_u32(const uint16_t *p)
     return *reinterpret_cast<const uint32_t *>(p);
 }
 
+// 8x8 b16 transpose across the warp (fragment layout of mma.m16n8k16).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// One warp per (query, KV head[, key split]).  Scores are computed
+// transposed, S^T = K Q^T: the 16 keys of a chunk are the MMA rows and the
+// G query heads the columns (NT tiles of 8), so a chunk takes 8 MMAs per
+// column tile for S^T and 8 for O^T += V^T P^T, with no rows wasted on
+// padding heads.  Lane (r0 = lane / 4, c = lane % 4) holds keys r0, r0 + 8 of
+// heads 2c, 2c + 1 of each column tile, and keeps the running max / sum of
+// those two heads; P^T turns into the B operand of the PV product by one
+// movmatrix transpose per 8 x 8 block.
+template <int NT>
 __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_split)
 {
     extern __shared__ __align__(128) uint8_t asmem[];
@@ -119,13 +146,16 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
 
     const int r0 = lane >> 2, c = lane & 3;
     const uint16_t *Qb = a.Q + ((q * a.Hq) + (int64_t)g * G) * LSA_HEAD;
-    uint32_t qa[8][4];
+    // B operand Q^T: dims 2c, 2c + 1 (and + 8) of dim block kk, head 8 nt + r0
+    uint32_t qb[NT][8][2];
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        qa[kk][0] = r0 < G ? ld_u32(Qb + r0 * LSA_HEAD + kk * 16 + 2 * c) : 0u;
-        qa[kk][1] = r0 + 8 < G ? ld_u32(Qb + (r0 + 8) * LSA_HEAD + kk * 16 + 2 * c) : 0u;
-        qa[kk][2] = r0 < G ? ld_u32(Qb + r0 * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
-        qa[kk][3] = r0 + 8 < G ? ld_u32(Qb + (r0 + 8) * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = nt * 8 + r0;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            qb[nt][kk][0] = h < G ? ld_u32(Qb + h * LSA_HEAD + kk * 16 + 2 * c) : 0u;
+            qb[nt][kk][1] = h < G ? ld_u32(Qb + h * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
+        }
     }
 
     int pre = -1;  // index of lane's row in the chunk issued next
@@ -149,20 +179,24 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
             const int idx = __shfl_sync(LSA_FULL, my, row);
             const int64_t off = ((int64_t)(idx < 0 ? 0 : idx) * a.Hkv + g) * LSA_HEAD + seg * 8;
             const int bytes = idx < 0 ? 0 : 16;
-            const uint32_t so = (uint32_t)((row * ROWB + seg * 8) * 2);
+            const uint32_t so = tile_off(row, seg);
             cp_async16(sK + so, a.K + off, bytes);
             cp_async16(sV + so, a.V + off, bytes);
         }
         cp_commit();
     };
 
-    float o[16][4];
+    float o[NT][8][4];  // O^T: dims 16 mt + r0 (+ 8) x heads 8 nt + 2c (+ 1)
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) o[nt][j] = 0.0f;
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[nt][mt][j] = 0.0f;
     const float NEG = __int_as_float(0xff800000);
-    float m0 = NEG, m1 = NEG, l0 = 0.0f, l1 = 0.0f;
+    float m[NT][2], l[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = NEG, l[nt][0] = l[nt][1] = 0.0f;
     const float sl2 = a.scale * LOG2E;
 
 #pragma unroll
@@ -178,81 +212,80 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
         __syncwarp();
         const uint32_t sK = sbase + (ch % NST) * STAGE_BYTES;
         const uint32_t sV = sK + KCH * ROWB * 2;
-        float s[2][4];
+        float s[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int j = 0; j < 4; ++j) s[nt][j] = 0.0f;
         {
-            const int mat = lane >> 3, rr = lane & 7;
-            const int key = rr + ((mat >> 1) << 3);
+            // A = K chunk (16 keys x 16 dims): matrix mm = lane / 8 is keys
+            // 8 (mm & 1) .., dims 8 (mm >> 1) ..
+            const int key = (lane & 7) + (((lane >> 3) & 1) << 3);
+            const int dsub = (lane >> 4) << 3;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                uint32_t b[4];
-                const int dim = kk * 16 + ((mat & 1) << 3);
-                ldsm_x4(b, sK + (uint32_t)((key * ROWB + dim) * 2));
-                mma16816(s[0], qa[kk], b[0], b[1]);
-                mma16816(s[1], qa[kk], b[2], b[3]);
+                uint32_t ka[4];
+                ldsm_x4(ka, sK + tile_off(key, 2 * kk + (dsub >> 3)));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma16816(s[nt], ka, qb[nt][kk][0], qb[nt][kk][1]);
             }
         }
         const int base = begin + ch * KCH;
+        const bool v0 = base + r0 < end, v1 = base + r0 + 8 < end;
+        uint32_t pb[NT][2];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < NT; ++nt) {
+            s[nt][0] = v0 ? s[nt][0] * sl2 : NEG;
+            s[nt][1] = v0 ? s[nt][1] * sl2 : NEG;
+            s[nt][2] = v1 ? s[nt][2] * sl2 : NEG;
+            s[nt][3] = v1 ? s[nt][3] * sl2 : NEG;
+            // column (head) maxima over the 16 keys: lanes with equal c
+            float mx0 = fmaxf(s[nt][0], s[nt][2]), mx1 = fmaxf(s[nt][1], s[nt][3]);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int kidx = nt * 8 + 2 * c + (j & 1);
-                s[nt][j] = (base + kidx < end) ? s[nt][j] * sl2 : NEG;
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(LSA_FULL, mx0, o2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(LSA_FULL, mx1, o2));
             }
-        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(LSA_FULL, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(LSA_FULL, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(LSA_FULL, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(LSA_FULL, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-        float rs0 = 0.0f, rs1 = 0.0f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+            const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+            const float al0 = exp2f(m[nt][0] - mn0), al1 = exp2f(m[nt][1] - mn1);
             s[nt][0] = exp2f(s[nt][0] - mn0);
-            s[nt][1] = exp2f(s[nt][1] - mn0);
-            s[nt][2] = exp2f(s[nt][2] - mn1);
+            s[nt][1] = exp2f(s[nt][1] - mn1);
+            s[nt][2] = exp2f(s[nt][2] - mn0);
             s[nt][3] = exp2f(s[nt][3] - mn1);
-            rs0 += s[nt][0] + s[nt][1];
-            rs1 += s[nt][2] + s[nt][3];
-        }
-        rs0 += __shfl_xor_sync(LSA_FULL, rs0, 1);
-        rs0 += __shfl_xor_sync(LSA_FULL, rs0, 2);
-        rs1 += __shfl_xor_sync(LSA_FULL, rs1, 1);
-        rs1 += __shfl_xor_sync(LSA_FULL, rs1, 2);
-        l0 = l0 * al0 + rs0;
-        l1 = l1 * al1 + rs1;
-        m0 = mn0;
-        m1 = mn1;
-        if (al0 != 1.0f || al1 != 1.0f) {  // the running max moved: rescale O
+            float rs0 = s[nt][0] + s[nt][2], rs1 = s[nt][1] + s[nt][3];
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                o[nt][0] *= al0;
-                o[nt][1] *= al0;
-                o[nt][2] *= al1;
-                o[nt][3] *= al1;
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                rs0 += __shfl_xor_sync(LSA_FULL, rs0, o2);
+                rs1 += __shfl_xor_sync(LSA_FULL, rs1, o2);
             }
-        }
-        uint32_t pa[4];
-        pa[0] = pack_bf16(s[0][0], s[0][1]);
-        pa[1] = pack_bf16(s[0][2], s[0][3]);
-        pa[2] = pack_bf16(s[1][0], s[1][1]);
-        pa[3] = pack_bf16(s[1][2], s[1][3]);
-        {
-            const int mat = lane >> 3, rr = lane & 7;
-            const int key = rr + ((mat & 1) << 3);
+            l[nt][0] = l[nt][0] * al0 + rs0;
+            l[nt][1] = l[nt][1] * al1 + rs1;
+            m[nt][0] = mn0;
+            m[nt][1] = mn1;
+            if (al0 != 1.0f || al1 != 1.0f) {  // the running max moved: rescale O^T
 #pragma unroll
-            for (int nt2 = 0; nt2 < 8; ++nt2) {
-                uint32_t b[4];
-                const int dim = nt2 * 16 + ((mat >> 1) << 3);
-                ldsm_x4_t(b, sV + (uint32_t)((key * ROWB + dim) * 2));
-                mma16816(o[2 * nt2], pa, b[0], b[1]);
-                mma16816(o[2 * nt2 + 1], pa, b[2], b[3]);
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[nt][mt][0] *= al0;
+                    o[nt][mt][1] *= al1;
+                    o[nt][mt][2] *= al0;
+                    o[nt][mt][3] *= al1;
+                }
+            }
+            // P^T blocks (keys r0 / r0 + 8, heads 2c, 2c + 1) -> B fragments
+            pb[nt][0] = movmatrix_t(pack_bf16(s[nt][0], s[nt][1]));
+            pb[nt][1] = movmatrix_t(pack_bf16(s[nt][2], s[nt][3]));
+        }
+        {
+            // A = V^T (16 dims x 16 keys) by transposing loads of V rows:
+            // matrix mm = lane / 8 is dims 8 (mm & 1) .., keys 8 (mm >> 1) ..
+            const int key = (lane & 7) + ((lane >> 4) << 3);
+            const int dsub = ((lane >> 3) & 1) << 3;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t va[4];
+                ldsm_x4_t(va, sV + tile_off(key, 2 * mt + (dsub >> 3)));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma16816(o[nt][mt], va, pb[nt][0], pb[nt][1]);
             }
         }
         __syncwarp();
@@ -260,37 +293,46 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     cp_wait<0>();
 
     if (a.nsplit == 1) {
-        const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
         uint16_t *Ob = a.O + ((q * a.Hq) + (int64_t)g * G) * LSA_HEAD;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int dim = nt * 8 + 2 * c;
-            if (r0 < G)
-                *reinterpret_cast<uint32_t *>(Ob + r0 * LSA_HEAD + dim) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
-            if (r0 + 8 < G)
-                *reinterpret_cast<uint32_t *>(Ob + (r0 + 8) * LSA_HEAD + dim) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
-        }
-        if (c == 0 && a.lse) {
-            if (r0 < G) a.lse[q * a.Hq + g * G + r0] = m0 * LN2 + logf(l0);
-            if (r0 + 8 < G) a.lse[q * a.Hq + g * G + r0 + 8] = m1 * LN2 + logf(l1);
+        for (int nt = 0; nt < NT; ++nt) {
+            const float i0 = l[nt][0] > 0.0f ? 1.0f / l[nt][0] : 0.0f;
+            const float i1 = l[nt][1] > 0.0f ? 1.0f / l[nt][1] : 0.0f;
+            const int h = nt * 8 + r0;  // after the transpose: head row r0, dims 2c, 2c + 1
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const uint32_t lo = movmatrix_t(pack_bf16(o[nt][mt][0] * i0, o[nt][mt][1] * i1));
+                const uint32_t hi = movmatrix_t(pack_bf16(o[nt][mt][2] * i0, o[nt][mt][3] * i1));
+                if (h < G) {
+                    *reinterpret_cast<uint32_t *>(Ob + h * LSA_HEAD + mt * 16 + 2 * c) = lo;
+                    *reinterpret_cast<uint32_t *>(Ob + h * LSA_HEAD + mt * 16 + 8 + 2 * c) = hi;
+                }
+            }
+            if (r0 == 0 && a.lse) {
+                if (nt * 8 + 2 * c < G) a.lse[q * a.Hq + g * G + nt * 8 + 2 * c] = m[nt][0] * LN2 + logf(l[nt][0]);
+                if (nt * 8 + 2 * c + 1 < G)
+                    a.lse[q * a.Hq + g * G + nt * 8 + 2 * c + 1] = m[nt][1] * LN2 + logf(l[nt][1]);
+            }
         }
     } else {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int r = r0 + 8 * half;
-            if (r >= G) continue;
-            const int64_t pidx = ((q * a.Hq) + (int64_t)g * G + r) * a.nsplit + split;
-            float *po = a.part_o + pidx * LSA_HEAD;
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const int dim = nt * 8 + 2 * c;
-                *reinterpret_cast<float2 *>(po + dim) = make_float2(o[nt][2 * half], o[nt][2 * half + 1]);
+            for (int e = 0; e < 2; ++e) {
+                const int h = nt * 8 + 2 * c + e;
+                if (h >= G) continue;
+                const int64_t pidx = ((q * a.Hq) + (int64_t)g * G + h) * a.nsplit + split;
+                float *po = a.part_o + pidx * LSA_HEAD;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    po[mt * 16 + r0] = o[nt][mt][e];
+                    po[mt * 16 + 8 + r0] = o[nt][mt][2 + e];
+                }
+                if (r0 == 0) {
+                    a.part_ml[pidx * 2] = m[nt][e];
+                    a.part_ml[pidx * 2 + 1] = l[nt][e];
+                }
             }
-            if (c == 0) {
-                a.part_ml[pidx * 2] = half ? m1 : m0;
-                a.part_ml[pidx * 2 + 1] = half ? l1 : l0;
-            }
-        }
     }
 }
 
@@ -356,13 +398,15 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     (void)n_sm;
     if (a.nq <= 0) return cudaSuccess;
     const int smem = AWARPS * WARP_BYTES;
-    cudaError_t e = cudaFuncSetAttribute(k_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int G = a.Hq / a.Hkv;
+    auto kern = G <= 8 ? k_attn<1> : k_attn<2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int kps = (a.Lmax + a.nsplit - 1) / a.nsplit;
     kps = ((kps + KCH - 1) / KCH) * KCH;
     const int64_t units = a.nq * a.Hkv * a.nsplit;
     const int64_t blocks = (units + AWARPS - 1) / AWARPS;
-    k_attn<<<(unsigned)blocks, AWARPS * 32, smem, st>>>(a, kps);
+    kern<<<(unsigned)blocks, AWARPS * 32, smem, st>>>(a, kps);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.nsplit > 1) {
