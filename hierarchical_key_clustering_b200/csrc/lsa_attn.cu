@@ -11,8 +11,9 @@
 // head[, key split]) unit: its G = Hq/Hkv heads form the rows of a 16-row
 // mma.sync tile (rows >= G are zero), 16 gathered keys form a chunk, and an
 // fp32 online softmax carries the running max and sum.  K/V rows are
-// gathered with cp.async (16 B per lane) into a 3-stage ring of swizzled
-// 256-byte rows in shared memory; each warp loads the list indices of the next chunk one issue ahead,
+// gathered with cp.async (16 B per lane) into a 2-stage ring of swizzled
+// 256-byte rows in shared memory (2 stages leave room for 12 warps per SM,
+// which hides the gather latency better than deeper rings with 8 warps); each warp loads the list indices of the next chunk one issue ahead,
 // so a gather never waits on a dependent index load.  The warps of a CTA are
 // independent (no CTA barrier), which keeps many gathers in flight per SM.
 // Units run head-major (all queries of KV head 0, then head 1, ...): the K/V
@@ -34,7 +35,7 @@ namespace lsa {
 
 constexpr int KCH = 16;                          // keys per chunk
 constexpr int ROWB = 128;                        // bf16 per smem row (256 B, 16-byte segments XOR-swizzled)
-constexpr int NST = 3;                           // pipeline stages
+constexpr int NST = 2;                           // pipeline stages (2 x 8 KB per warp: 3 CTAs of 4 warps per SM)
 constexpr int STAGE_BYTES = 2 * KCH * ROWB * 2;  // K + V
 constexpr int WARP_BYTES = NST * STAGE_BYTES;
 constexpr int AWARPS = 4;
