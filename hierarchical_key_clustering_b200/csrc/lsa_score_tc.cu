@@ -201,29 +201,17 @@ __device__ __forceinline__ float max8f(const float *v)
     return max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
 }
 
-// One query row's group-maximum histogram in shared memory (256 saturating
-// u16 bins, two per word).  bL tracks the bin holding the P-th largest
-// maximum counted so far and S the counts in bins >= bL; once P maxima are at
-// or above its edge lm, a smaller maximum can only land below the final
-// threshold bin (bL never falls, here or in the merged histogram of a split
-// range), so it is not counted.
+// One query row's group-maximum histogram in shared memory: 256 saturating
+// u16 bins, two per word.  (Skipping maxima below a running P-th-largest
+// bound was tried: its bookkeeping cost more than the counts it saved.)
 struct RowHist {
     uint32_t *h;
-    int bL, S;
-    float lm;
-    __device__ __forceinline__ int at(int b) const { return (int)((h[b >> 1] >> ((b & 1) * 16)) & 0xffffu); }
-    __device__ __forceinline__ void add(float m, int P)
+    __device__ __forceinline__ void add(float m) const
     {
-        if (m < lm) return;
         const int bin = hist_bin(m);
         const uint32_t w = h[bin >> 1];
         const uint32_t sh = (bin & 1) * 16;
-        if (((w >> sh) & 0xffffu) == 0xffffu) return;
-        h[bin >> 1] = w + (1u << sh);
-        if (bin < bL) return;
-        ++S;
-        while (S - at(bL) >= P) S -= at(bL++);
-        if (S >= P) lm = hist_edge(bL);
+        if (((w >> sh) & 0xffffu) != 0xffffu) h[bin >> 1] = w + (1u << sh);
     }
 };
 
@@ -379,10 +367,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t *hrow = hist + (qt * TQ + r) * HSTRIDE;
         if (a.mode == 0)
             for (int w = 0; w < HSTRIDE; ++w) hrow[w] = 0u;
-        // Count one group maximum in the row histogram (saturating u16 bins);
-        // see RowHist for the bound that lets most maxima go uncounted.
-        RowHist rh{hrow, 0, 0, NEG};
-        auto count = [&](float m) { rh.add(m, a.P); };
+        const RowHist rh{hrow};
+        auto count = [&](float m) { rh.add(m); };
         float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
         int32_t *cg = ws.cand_g + q * ws.cap;
         int own = 0;  // group entries this thread appended (FILTER)
@@ -394,7 +380,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const int64_t tb0 = tile_of(it) * TB;
             float run = NEG;  // g = 128: maximum over the whole tile
-#pragma unroll 1
+#pragma unroll
             for (int h = 0; h < 2; ++h) {
                 // one 64-column half at a time (registers); after the second
                 // half is read the MMA may refill this buffer
