@@ -485,9 +485,11 @@ __global__ void __launch_bounds__(256) k_dfilter(int64_t nq, int P, IndexWs ws)
 constexpr int RX_SLOTS = 512;  // touched blocks per emit batch
 constexpr int RX_BINS = 4096;  // bins of the cut search (aliases the masks)
 
+constexpr int RX_MW = 17;      // words per touched block's mask row (16 + 1 pad: conflict-free per-slot reads)
+
 __host__ __device__ inline size_t rank_expand_smem(int KC, int TW)
 {
-    return (size_t)KC * 8 + (size_t)RX_SLOTS * 64 + (size_t)TW * 8 + (size_t)RX_SLOTS * 8 + (size_t)KC;
+    return (size_t)KC * 8 + (size_t)RX_SLOTS * RX_MW * 4 + (size_t)TW * 8 + (size_t)RX_SLOTS * 8 + (size_t)KC;
 }
 
 template <int NT>
@@ -499,9 +501,9 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
 {
     extern __shared__ uint64_t rsm[];
     uint64_t *keys = rsm;                                           // [KC]
-    uint32_t *masks = reinterpret_cast<uint32_t *>(keys + KC);      // [RX_SLOTS][16]
+    uint32_t *masks = reinterpret_cast<uint32_t *>(keys + KC);      // [RX_SLOTS][RX_MW]
     uint32_t *bins = masks;                                         // [RX_BINS] (before the masks are used)
-    uint32_t *touched = masks + RX_SLOTS * 16;                      // [TW]
+    uint32_t *touched = masks + RX_SLOTS * RX_MW;                   // [TW]
     int32_t *wrank = reinterpret_cast<int32_t *>(touched + TW);     // [TW]
     int32_t *slot_blk = wrank + TW;                                 // [RX_SLOTS]
     int32_t *slot_off = slot_blk + RX_SLOTS;                        // [RX_SLOTS]
@@ -712,7 +714,7 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     int emitted = 0;
     for (int b0 = 0; b0 < nslots; b0 += RX_SLOTS) {
         const int nb = min(RX_SLOTS, nslots - b0);
-        for (int i = t; i < nb * 16; i += blockDim.x) masks[i] = 0u;
+        for (int i = t; i < nb * RX_MW; i += blockDim.x) masks[i] = 0u;
         __syncthreads();
         for (int i = t; i < n; i += blockDim.x) {
             if (!(any && wt[i] > 0 && keys[i] <= cut)) continue;
@@ -733,7 +735,7 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                 for (int e = 0; e < 4; ++e) {
                     const int64_t m = mm[e];
                     if (m >= 0 && !(m < s_end || (m >= w0 && m <= p))) {
-                        if (idx < limit) atomicOr(&masks[slot * 16 + ((m & 511) >> 5)], 1u << (m & 31));
+                        if (idx < limit) atomicOr(&masks[slot * RX_MW + ((m & 511) >> 5)], 1u << (m & 31));
                         ++idx;
                     }
                 }
@@ -743,27 +745,22 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
         for (int sl = t; sl < nb; sl += blockDim.x) {
             int c = 0;
 #pragma unroll
-            for (int w = 0; w < 16; ++w) c += __popc(masks[sl * 16 + w]);
+            for (int w = 0; w < 16; ++w) c += __popc(masks[sl * RX_MW + w]);
             slot_off[sl] = c;
         }
         __syncthreads();
         block_inclusive_scan(slot_off, nb, wsum);
-        for (int sl = warp; sl < nb; sl += nwarps) {
-            const uint32_t word = lane < 16 ? masks[sl * 16 + lane] : 0u;
-            const int c = __popc(word);
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) {
-                const int y = __shfl_up_sync(LSA_FULL, incl, o);
-                if (lane >= o) incl += y;
-            }
-            int o = n_sink + emitted + slot_off[sl] - __shfl_sync(LSA_FULL, incl, 15) + incl - c;
-            const int32_t base = slot_blk[sl] * LSA_BLK + lane * 32;
-            uint32_t bits = word;
-            while (bits) {
-                const int bit = __ffs(bits) - 1;
-                out[o++] = base + bit;
-                bits &= bits - 1;
+        // one thread per touched block: its positions in ascending order
+        for (int sl = t; sl < nb; sl += blockDim.x) {
+            int o = n_sink + emitted + (sl > 0 ? slot_off[sl - 1] : 0);
+            const int32_t base = slot_blk[sl] * LSA_BLK;
+#pragma unroll 4
+            for (int w = 0; w < 16; ++w) {
+                uint32_t bits = masks[sl * RX_MW + w];
+                while (bits) {
+                    out[o++] = base + 32 * w + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                }
             }
         }
         emitted += slot_off[nb - 1];
