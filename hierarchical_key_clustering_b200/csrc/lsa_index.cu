@@ -495,6 +495,7 @@ __host__ __device__ inline size_t rank_expand_smem(int KC, int TW)
 template <int NT>
 __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ pos,
                                                       const int32_t *__restrict__ members,
+                                                      const int32_t *__restrict__ count,
                                                       const uint16_t *__restrict__ cbf, int32_t *__restrict__ lists,
                                                       int32_t *__restrict__ lens, int Lmax, int k, int sink,
                                                       int window, int P, int KC, int TW, IndexWs ws)
@@ -609,21 +610,28 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     }
     const int n = nk_s;
 
-    // 2. weights (members outside near) and the key range of weighted candidates
+    // 2. weights (members outside near) and the key range of weighted candidates.
+    //    Only a block that overlaps the sink or the window can hold near keys;
+    //    a bucket of any other block weighs its member count.
     int my_tot = 0;
     unsigned long long my_lo = ~0ull, my_hi = 0ull;
     for (int i = t; i < n; i += blockDim.x) {
         const int32_t b = rank_key_id(keys[i]);
-        const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
+        const int64_t blo = (int64_t)(b / LSA_NBKT) * LSA_BLK;
         int nn = 0;
+        if (blo >= s_end && blo + LSA_BLK <= w0) {
+            nn = __ldg(count + b);
+        } else {
+            const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const int4 w = __ldg(m4 + v);
-            const int mm[4] = {w.x, w.y, w.z, w.w};
+            for (int v = 0; v < 4; ++v) {
+                const int4 w = __ldg(m4 + v);
+                const int mm[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int64_t m = mm[e];  // -1 pads are skipped
-                nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
+                for (int e = 0; e < 4; ++e) {
+                    const int64_t m = mm[e];  // -1 pads are skipped
+                    nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
+                }
             }
         }
         wt[i] = (uint8_t)nn;
@@ -712,6 +720,10 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     const int n_sink = (int)min(s_end, w0);
     int32_t *out = lists + q * (int64_t)Lmax;
     int emitted = 0;
+    // one batch whose far keys fit in the candidate keys' space (free once the
+    // marks are set): stage them there and copy the whole list out coalesced
+    const bool stage = nslots <= RX_SLOTS && nfar <= 2 * KC;
+    int32_t *stg = reinterpret_cast<int32_t *>(keys);
     for (int b0 = 0; b0 < nslots; b0 += RX_SLOTS) {
         const int nb = min(RX_SLOTS, nslots - b0);
         for (int i = t; i < nb * RX_MW; i += blockDim.x) masks[i] = 0u;
@@ -752,13 +764,14 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
         block_inclusive_scan(slot_off, nb, wsum);
         // one thread per touched block: its positions in ascending order
         for (int sl = t; sl < nb; sl += blockDim.x) {
-            int o = n_sink + emitted + (sl > 0 ? slot_off[sl - 1] : 0);
+            int o = (stage ? 0 : n_sink) + emitted + (sl > 0 ? slot_off[sl - 1] : 0);
+            int32_t *dst = stage ? stg : out;
             const int32_t base = slot_blk[sl] * LSA_BLK;
 #pragma unroll 4
             for (int w = 0; w < 16; ++w) {
                 uint32_t bits = masks[sl * RX_MW + w];
                 while (bits) {
-                    out[o++] = base + 32 * w + __ffs(bits) - 1;
+                    dst[o++] = base + 32 * w + __ffs(bits) - 1;
                     bits &= bits - 1;
                 }
             }
@@ -772,7 +785,9 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     const int len = n_sink + emitted + nwin;
     for (int i = t; i < Lmax; i += blockDim.x) {
         if (i < n_sink) out[i] = i;
-        else if (i < n_sink + emitted) continue;
+        else if (i < n_sink + emitted) {
+            if (stage) out[i] = stg[i - n_sink];
+        }
         else if (i < len) out[i] = (int32_t)(w0 + (i - n_sink - emitted));
         else out[i] = -1;
     }
@@ -845,11 +860,11 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     const size_t smr = rank_expand_smem(KC, TW);
     if (small) {  // one CTA per query, few queries: widest blocks
         cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        k_rank_expand<1024><<<(unsigned)a.nq, 1024, smr, st>>>(a.pos, a.members, a.centroid_bf16, a.lists, a.lens,
+        k_rank_expand<1024><<<(unsigned)a.nq, 1024, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,
                                                                a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ws);
     } else {
         cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.centroid_bf16, a.lists, a.lens,
+        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,
                                                              a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ws);
     }
     count_launches(1);
