@@ -47,7 +47,7 @@ L2_FLUSH_BYTES = 256 << 20
 # 16384 x 2565 x 8 rows; head-major order keeps each head's K/V in L2);
 # roofline.traffic scales it by the rows of a full launch.  Re-measure when
 # k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = 21.3
+ATTN_DRAM_BYTES_PER_ROW = 21.0
 
 
 def peaks():
