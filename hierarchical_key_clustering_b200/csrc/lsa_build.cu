@@ -4,7 +4,7 @@
 // Method: Latent Sparse Attention pages -- learnaivisually explainer, "How
 // the hierarchy is built" (normalise, sum n_pool = 4 consecutive keys, Ward
 // merge of each full block into a fixed number of buckets, centroid + key
-// table per bucket, "the same process is repeated on the buckets" for the
+// table per bucket, and the same merging again on the buckets for the
 // tree); zhichai forum post, "Key points" (64-dim, 512-key blocks, buckets of
 // ~8 and at most 16 keys); sotaaz blog, "The same steps in general", step 2.
 #include "lsa_common.cuh"

@@ -64,8 +64,9 @@ enum { LSA_MODE_FLAT = 0, LSA_MODE_TREE = 1 };
 
 /* Parameters of the method.  lsa_default_params() fills the pages' values:
  * n_pool 4, block 512, n_buckets 64, cap_items 4, sink 4, window 512 ([BLOG]
- * step 5: "the first 4 keys and the latest 512 are always read"), k 4096
- * ([BLOG] step 4: "On Qwen3.8-27B that is 4,096 keys"), beam 32, mode Flat.
+ * step 5: four sink keys and the newest 512 keys are always read), k 4096
+ * ([BLOG] step 4: the long-range key budget given for the Qwen model),
+ * beam 32, mode Flat.
  * cand_cap: per-query candidate slots of the Flat search (0 = automatic).
  * A smaller value only routes more queries through the exact fallback
  * selection; results do not change. */
@@ -82,9 +83,9 @@ typedef struct lsa_params {
     int32_t cand_cap;
 } lsa_params;
 
-/* Bucket cache ([EXPL] "Each bucket stores one centroid and a table of the
- * key positions it contains, and once a block is clustered its buckets never
- * change").  Bucket g = 64*b + r is the r-th bucket of block b, buckets of a
+/* Bucket cache ([EXPL] "How the hierarchy is built": a bucket keeps a
+ * centroid and the positions of its keys, and a clustered block is never
+ * touched again).  Bucket g = 64*b + r is the r-th bucket of block b, buckets of a
  * block ordered by their lowest pooled item.
  *   pooled        fp32 [capacity/4, 64]   sum of 4 normalised keys per item
  *   item_bucket   u8   [capacity/512, 128] bucket (0..63) of each pooled item
@@ -105,9 +106,9 @@ typedef struct lsa_cache {
     uint16_t *centroid_bf16;
 } lsa_cache;
 
-/* Tree of merged buckets ([EXPL] "In the tree variant the same process is
- * repeated on the buckets to form higher levels"; [FORUM] "binary tree of
- * merged buckets").  Level 0 = the buckets; level l has ceil(n_{l-1}/2)
+/* Tree of merged buckets ([EXPL] "How the hierarchy is built": the tree
+ * variant merges buckets again, level after level; [FORUM] "Key points": a
+ * binary tree over the buckets).  Level 0 = the buckets; level l has ceil(n_{l-1}/2)
  * nodes; the top level holds the root.  Node arrays are indexed by global
  * id = level_offset[l] + local id; child/parent hold LOCAL ids of the level
  * below/above.
@@ -199,8 +200,8 @@ int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, 
 int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache *cache,
                     const lsa_params *p, void *stream);
 
-/* Tree above the buckets of cache->n_blocks blocks ([EXPL] "In the tree
- * variant the same process is repeated on the buckets").  At every level,
+/* Tree above the buckets of cache->n_blocks blocks ([EXPL] "How the
+ * hierarchy is built", tree variant).  At every level,
  * consecutive runs of 128 nodes are paired greedily by Ward cost
  * (weights = pooled items, mu = sum / weight), ties to the lowest (i, j); an
  * odd leftover is promoted alone; new nodes are ordered by their lower
@@ -235,12 +236,12 @@ int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const ls
                      const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);
 
 /* Exact softmax attention over each query's list, shared by all its heads
- * ([EXPL] "One index list is built per query and shared by all of its
- * attention heads ... Then ordinary attention runs over sink, selected keys
- * and window").
+ * ([EXPL] "What one query actually does": one list per query serves every
+ * head of that query, and plain softmax attention runs over it).
  * Q bf16 [nq, Hq, 128]; K, V bf16 [Tk, Hkv, 128]; query head h reads KV head
  * h / (Hq / Hkv) (Hq a multiple of Hkv, Hq / Hkv <= 16).  lists/lens as
- * written by lsa_index_*; every listed position must be < Tk.
+ * written by lsa_index_*: each list strictly increasing, every listed
+ * position < Tk.
  * O[i,h] = sum_j softmax_j(scale * Q[i,h] . K[j]) V[j] over j in list(i),
  * fp32 softmax and accumulation; O bf16 [nq, Hq, 128]; lse fp32 [nq, Hq]
  * (natural-log log-sum-exp of the scaled scores; may be NULL).

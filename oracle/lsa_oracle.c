@@ -102,8 +102,9 @@ float orc_sqdist(const float *a, const float *b)
     return r1_sum(sq);
 }
 
-/* Length-normalise: out = x / sqrt(sum x^2) ([EXPL] "each index key is
- * length-normalized"; [FORUM] "L2-normalized").  Zero vector -> zero. */
+/* Length-normalise: out = x / sqrt(sum x^2) ([EXPL] "How the hierarchy is
+ * built" and [FORUM] "Key points": keys are scaled to unit length).  Zero
+ * vector -> zero. */
 void orc_normalize(const float *x, float *out)
 {
     float n = sqrtf(orc_sumsq(x));
@@ -128,9 +129,10 @@ void orc_pool_norm(const float *keys, int64_t n_items, float *pooled)
 
 /* ---------- step a2: Ward clustering of one block ---------- */
 
-/* [EXPL] "When a block is full, its pooled keys are merged bottom-up with
- * Ward's method into a fixed number of buckets"; [BLOG] step 2 "buckets of
- * about 8 keys, 16 at most"; Ward 1963 for the criterion.
+/* [EXPL] "How the hierarchy is built": a full block's pooled keys are
+ * clustered bottom-up by Ward's criterion down to a fixed bucket count;
+ * [BLOG] step 2: buckets average 8 keys and hold no more than 16; Ward 1963
+ * for the criterion.
  *
  * items: [m, 64] pooled keys (unit weight each).  Merge cost of clusters A, B:
  *   D(A,B) = n_A n_B / (n_A + n_B) * |mu_A - mu_B|^2   (increase of the SSE),
@@ -239,9 +241,9 @@ int64_t orc_build_cache(const float *keys, int64_t T, int cap_items, int n_bucke
 
 /* ---------- step a3: the tree of merged buckets ---------- */
 
-/* Greedy Ward pairing of one run of m nodes ([EXPL] "In the tree variant the
- * same process is repeated on the buckets"; [FORUM] "binary tree of merged
- * buckets").  mu: [m, 64] node means, w: [m] weights (pooled items).
+/* Greedy Ward pairing of one run of m nodes ([EXPL] "How the hierarchy is
+ * built", tree variant: the buckets are merged again, level after level;
+ * [FORUM] "Key points": a binary tree over the buckets).  mu: [m, 64] node means, w: [m] weights (pooled items).
  * D(A,B) = (w_A w_B / (w_A + w_B)) |mu_A - mu_B|^2; repeatedly pair the two
  * unpaired nodes of least cost (ties to the lowest (i, j)).  partner[i] <- the
  * node paired with i, or -1 if i stays alone. */
@@ -380,8 +382,8 @@ int orc_build_tree(const float *pooled, const int32_t *members, const int32_t *c
 
 /* ---------- steps a4-a7: one query ---------- */
 
-/* [EXPL] "What one query actually does": the query is normalized; R9: bf16
- * copy of the normalised query. */
+/* [EXPL] "What one query actually does": the query is scaled to unit
+ * length first; R9: bf16 copy of the normalised query. */
 void orc_qnorm(const float *q, int64_t nq, uint16_t *qhat)
 {
     for (int64_t i = 0; i < nq; ++i) {
@@ -410,10 +412,10 @@ static int cmp_rank(const void *a, const void *b)
     return (x->id > y->id) - (x->id < y->id);
 }
 
-/* Flat search ([EXPL] "it scores every bucket centroid from earlier cluster
- * blocks and takes the top buckets"; [FORUM] "Flat search scores all bucket
- * centroids"): score every bucket of blocks 0..H-1, rank by (score desc,
- * id asc).  Writes all 64*H ranked ids/scores; returns their number. */
+/* Flat search ([EXPL] "What one query actually does": every centroid of the
+ * earlier blocks is scored and the best buckets are kept; [FORUM] "Key
+ * points", Flat vs Tree): score every bucket of blocks 0..H-1, rank by
+ * (score desc, id asc).  Writes all 64*H ranked ids/scores; returns their number. */
 int64_t orc_flat_rank(const uint16_t *qhat, int64_t H, int n_buckets, const uint16_t *cbf,
                       int32_t *ids, float *scores)
 {
@@ -426,8 +428,9 @@ int64_t orc_flat_rank(const uint16_t *qhat, int64_t H, int n_buckets, const uint
     return n;
 }
 
-/* Tree search (R8; [EXPL] "at each level it expands only the best nodes it
- * kept"; [FORUM] "beam search per level").  A node is visible iff all its
+/* Tree search (R8; [EXPL] "What one query actually does" and the
+ * search-style table: each level opens only the children of the nodes kept at
+ * the level above; [FORUM] "Key points": a beam per level).  A node is visible iff all its
  * blocks are < H.  Candidates at level l = children of the nodes kept at
  * level l+1, plus visible level-l nodes whose parent is not visible (or that
  * have no parent).  Keep the best max(W, ceil(P / 2^l)) by (score desc, id
@@ -478,8 +481,9 @@ static int cmp_i32(const void *a, const void *b)
 }
 
 /* Open the ranked buckets best first and add sink + window ([BLOG] steps 4-5
- * and read_list; [EXPL] "expanded into key positions, best first, until k
- * long-range keys are collected.  Two things are always added").
+ * and read_list; [EXPL] "What one query actually does": buckets turn into
+ * key positions in rank order until k long-range keys are in, and the sink
+ * and the recent window are always added).
  * near = {0..min(sink,p+1)-1} U [max(0,p-window), p]; members already in
  * near are skipped and the next one takes their place; stop at k far keys.
  * out[0..len) = sorted(near U far), out[len..Lmax) = -1.  Returns len. */
@@ -542,8 +546,9 @@ int orc_index(const float *qidx, const int64_t *pos, int64_t nq, int64_t nblk, i
 
 /* ---------- step a8: exact softmax attention over each list ---------- */
 
-/* [EXPL] "Then ordinary attention runs over sink, selected keys and window";
- * one list per query shared by all its heads.  Q [nq,Hq,dh], K/V [Tk,Hkv,dh]
+/* [EXPL] "What one query actually does": plain softmax attention over the
+ * sink, the chosen keys and the window; one list per query serves all its
+ * heads.  Q [nq,Hq,dh], K/V [Tk,Hkv,dh]
  * as bf16 bits; query head h reads KV head floor(h*Hkv/Hq).  Computed in fp64:
  * O = sum_j softmax_j(scale * q.k_j) v_j; lse = max + log(sum exp).  O, lse
  * are rounded to fp32 at the end. */
