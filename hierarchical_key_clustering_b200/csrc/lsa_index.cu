@@ -153,6 +153,55 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
 }
 
 // ---------------------------------------------------------------------------
+// Ascending bitonic sort of 32 E keys held by one warp: element E * lane + r
+// is v[r].  Pairs E or more apart are exchanged across lanes with shuffles,
+// closer pairs inside a lane's registers; no shared memory, no barriers.
+template <int E>
+__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[E])
+{
+    const int lane = threadIdx.x & 31;
+    for (int k = 2; k <= 32 * E; k <<= 1) {
+        for (int j = k >> 1; j >= E; j >>= 1) {
+            const int lj = j / E;  // lane distance of the pair
+            const bool lower = (lane & lj) == 0;
+#pragma unroll
+            for (int r = 0; r < E; ++r) {
+                const uint64_t o = __shfl_xor_sync(LSA_FULL, v[r], lj);
+                const bool up = ((E * lane + r) & k) == 0;
+                v[r] = (lower == up) ? (v[r] < o ? v[r] : o) : (v[r] > o ? v[r] : o);
+            }
+        }
+#pragma unroll
+        for (int j = E / 2; j > 0; j >>= 1) {
+            if (j >= k) continue;
+#pragma unroll
+            for (int r = 0; r < E; ++r) {
+                if ((r ^ j) <= r) continue;
+                const bool up = ((E * lane + r) & k) == 0;
+                const uint64_t x = v[r], y = v[r ^ j];
+                if ((x > y) == up) {
+                    v[r] = y;
+                    v[r ^ j] = x;
+                }
+            }
+        }
+    }
+}
+
+// keys[0..S) ascending by one warp (S = 32 E); the other warps idle.
+template <int E>
+__device__ __forceinline__ void warp_sort_smem(uint64_t *keys)
+{
+    const int lane = threadIdx.x & 31;
+    uint64_t v[E];
+#pragma unroll
+    for (int r = 0; r < E; ++r) v[r] = keys[E * lane + r];
+    warp_bitonic_sort<E>(v);
+#pragma unroll
+    for (int r = 0; r < E; ++r) keys[E * lane + r] = v[r];
+}
+
+// ---------------------------------------------------------------------------
 // Tree beam search: one CTA per query, level by level from the root.
 __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, IndexWs ws)
 {
@@ -200,7 +249,8 @@ __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int 
         __syncthreads();
         const int n = nc;
         const int S = (int)pow2_ceil64(n > 0 ? n : 1);
-        for (int i = t; i < S; i += blockDim.x) {
+        const int Sp = S < 32 ? 32 : S;  // a warp sorts at least 32 keys
+        for (int i = t; i < Sp; i += blockDim.x) {
             if (i < n) {
                 const int32_t u = cids[i];
                 keys[i] = rank_key(dot_bf16_row_f64(qf, tv.centroid_bf16 + (off + u) * LSA_D), u);
@@ -209,7 +259,18 @@ __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int 
             }
         }
         __syncthreads();
-        block_bitonic_sort(keys, S);
+        if (Sp <= 512) {  // small levels (every level above the last few): one warp, registers only
+            if (t < 32) {
+                if (Sp == 32) warp_sort_smem<1>(keys);
+                else if (Sp == 64) warp_sort_smem<2>(keys);
+                else if (Sp == 128) warp_sort_smem<4>(keys);
+                else if (Sp == 256) warp_sort_smem<8>(keys);
+                else warp_sort_smem<16>(keys);
+            }
+            __syncthreads();
+        } else {
+            block_bitonic_sort(keys, S);
+        }
         int64_t B = ((int64_t)P + ((int64_t)1 << l) - 1) >> l;
         if (B < W) B = W;
         const int nk = (int)min((int64_t)n, B);
