@@ -217,6 +217,10 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
             return fail(LSA_ERR_ARG, "beam %d / k %d too large for the beam kernel", p->beam, p->k);
     }
     const int64_t P = top_buckets(p);
+    // Flat threshold histograms count at most 2^16 - 1 group maxima per query
+    // (groups of up to 64 buckets, 4P..8P of them)
+    if (p->mode == LSA_MODE_FLAT && (cache->n_blocks > 65535 || P >= 8192))
+        return fail(LSA_ERR_SHAPE, "Flat search supports up to 65535 blocks and k + sink + window < 32768");
     IndexLayout L = index_layout(nq, cache->n_blocks, p);
     if (L.cap < P) return fail(LSA_ERR_ARG, "cand_cap %lld < top buckets %lld", (long long)L.cap, (long long)P);
     if (L.cap > 8192) return fail(LSA_ERR_ARG, "cand_cap %lld above 8192", (long long)L.cap);

@@ -157,12 +157,12 @@ __host__ __device__ __forceinline__ int64_t pow2_floor64(int64_t x)
 }
 
 // Group width of the Flat threshold pass for a query that sees N buckets:
-// the largest power of two <= N / (4P), clamped to [1, 128], so a query has
+// the largest power of two <= N / (4P), clamped to [1, 64], so a query has
 // between 4P and 8P group maxima (or N of them when N is small).
 __host__ __device__ __forceinline__ int group_width(int64_t N, int64_t P)
 {
     int64_t g = (N >= 4 * P) ? pow2_floor64(N / (4 * P)) : 1;
-    if (g > 128) g = 128;
+    if (g > 64) g = 64;
     return (int)g;
 }
 

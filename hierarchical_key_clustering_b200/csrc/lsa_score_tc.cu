@@ -60,10 +60,11 @@ constexpr int NST_MAX = 8;
 constexpr uint32_t A_BYTES = QT * TQ * LSA_D * 2;  // 32 KB
 constexpr uint32_t B_BYTES = TB * LSA_D * 2;       // 16 KB
 constexpr int TMEM_COLS = 512;      // [query tile][buffer] x 128 fp32 columns
-constexpr int EPI_WARPS = 4 * QT;   // 8
-constexpr int THREADS = 64 + 32 * EPI_WARPS;  // 320
+constexpr int EPI_WARPS = 8 * QT;   // 16: TMEM lane quadrant x query tile x column half
+constexpr int THREADS = 64 + 32 * EPI_WARPS;  // 576
 constexpr int HSTRIDE = HIST_BINS / 2 + 1;   // 32-bit words per row histogram (2 x u16 bins per word, +1 pad)
 constexpr uint32_t HIST_BYTES = QT * TQ * HSTRIDE * 4;
+constexpr uint32_t ROWCNT_BYTES = QT * TQ * 4;  // per-row entry counters of the filter pass
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -201,20 +202,6 @@ __device__ __forceinline__ float max8f(const float *v)
     return max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
 }
 
-// One query row's group-maximum histogram in shared memory: 256 saturating
-// u16 bins, two per word.  (Skipping maxima below a running P-th-largest
-// bound was tried: its bookkeeping cost more than the counts it saved.)
-struct RowHist {
-    uint32_t *h;
-    __device__ __forceinline__ void add(float m) const
-    {
-        const int bin = hist_bin(m);
-        const uint32_t w = h[bin >> 1];
-        const uint32_t sh = (bin & 1) * 16;
-        if (((w >> sh) & 0xffffu) != 0xffffu) h[bin >> 1] = w + (1u << sh);
-    }
-};
-
 // Candidate entry (4 scores + first bucket id), stored only when p != 0.
 __device__ __forceinline__ void st_entry_if(int p, float4 *d4, int32_t *dg, const float *x, int32_t g)
 {
@@ -252,10 +239,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t *sA = tsm;
     uint8_t *sB = tsm + A_BYTES;
     uint32_t *hist = reinterpret_cast<uint32_t *>(tsm + A_BYTES + nst * B_BYTES);  // [QT*TQ][HSTRIDE], GMAX only
-    TcSmem *cs = reinterpret_cast<TcSmem *>(tsm + A_BYTES + nst * B_BYTES + (a.mode == 0 ? HIST_BYTES : 0));
+    int *rowcnt = reinterpret_cast<int *>(tsm + A_BYTES + nst * B_BYTES);           // [QT*TQ], FILTER only
+    TcSmem *cs = reinterpret_cast<TcSmem *>(tsm + A_BYTES + nst * B_BYTES + (a.mode == 0 ? HIST_BYTES : ROWCNT_BYTES));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t q0 = (int64_t)blockIdx.x * (QT * TQ);
+    // epilogue identity of this thread (meaningful for warps >= 2)
+    const int ep_quad = warp & 3, ep_sel = (warp - 2) >> 2;
+    const int ep_qt = ep_sel & 1, ep_half = ep_sel >> 1;
+    const int ep_r = ep_quad * 32 + lane;
+    const int64_t ep_q = q0 + ep_qt * TQ + ep_r;
+    const int ep_N = (warp >= 2 && ep_q < a.nq) ? ws.horizon[ep_q] * LSA_NBKT : 0;
+    if (a.mode == 0)
+        for (int i = threadIdx.x; i < QT * TQ * HSTRIDE; i += THREADS) hist[i] = 0u;
+    else
+        for (int i = threadIdx.x; i < QT * TQ; i += THREADS) rowcnt[i] = 0;
 
     if (threadIdx.x == 0) {
         cs->nmax = 0;
@@ -355,150 +353,132 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (warp >= 2) {
-        // epilogue: thread owns row r of query tile qt (TMEM lane 32 * quad + lane)
-        const int quad = warp & 3;
-        const int qt = (warp - 2) >> 2;
-        const int r = quad * 32 + lane;
-        const int64_t q = q0 + qt * TQ + r;
-        const int N = (q < a.nq) ? ws.horizon[q] * LSA_NBKT : 0;
-        const int g = group_width(N, a.P);
-        const float tau = (a.mode == 1 && q < a.nq) ? ws.tau[q] : 0.0f;
+        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows of query
+        // tile qt) and one 64-column half of each 128-column accumulator, 32
+        // columns at a time; the row's two halves go to two warps
         const float NEG = __int_as_float(0xff800000);
-        uint32_t *hrow = hist + (qt * TQ + r) * HSTRIDE;
-        if (a.mode == 0)
-            for (int w = 0; w < HSTRIDE; ++w) hrow[w] = 0u;
-        const RowHist rh{hrow};
-        auto count = [&](float m) { rh.add(m); };
-        float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
-        int32_t *cg = ws.cand_g + q * ws.cap;
-        int own = 0;  // group entries this thread appended (FILTER)
-        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(qt * 2 * TB);
+        const int g = ep_N > 0 ? group_width(ep_N, a.P) : 1;  // <= 64: a group never spans two halves
+        const float tau = (a.mode == 1 && ep_q < a.nq) ? ws.tau[ep_q] : 0.0f;
+        uint32_t *hrow = hist + (ep_qt * TQ + ep_r) * HSTRIDE;
+        auto count = [&](float m) {  // counts per bin stay below 2^16 (at most 2^16 - 1 groups per query)
+            const int bin = hist_bin(m);
+            atomicAdd(&hrow[bin >> 1], 1u << ((bin & 1) * 16));
+        };
+        float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + ep_q * ws.cap;
+        int32_t *cg = ws.cand_g + ep_q * ws.cap;
+        const uint32_t lane_base = tmem + ((uint32_t)(ep_quad * 32) << 16) + (uint32_t)(ep_qt * 2 * TB + ep_half * 64);
         for (int it = 0; it < ntiles; ++it) {
             const int buf = it & 1;
             const bool ok = wait_bounded(smem_u32(&cs->tfull[buf]), (uint32_t)((it >> 1) & 1), a.wait_limit, abort);
             if (!__all_sync(LSA_FULL, ok)) break;  // warp-uniform: tcgen05.ld needs the whole warp
             tc_fence_after();
-            const int64_t tb0 = tile_of(it) * TB;
-            float run = NEG;  // g = 128: maximum over the whole tile
+            const int64_t bh = tile_of(it) * TB + 64 * ep_half;  // first bucket of this half
+            float run = NEG;                                     // g = 64: maximum over the half
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                // one 64-column half at a time (registers); after the second
-                // half is read the MMA may refill this buffer
-                float x[64];
-                tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + h * 64), x);
-                tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + h * 64 + 32), x + 32);
+            for (int c = 0; c < 2; ++c) {
+                float x[32];
+                tmem_ld32_nowait(lane_base + (uint32_t)(buf * TB + 32 * c), x);
                 tmem_wait_ld();
-                if (h == 1) {
+                if (c == 1) {  // this warp has read its half: the MMA may refill the buffer
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&cs->tempty[buf]));
                 }
-                const int64_t b0 = tb0 + 64 * h;
-                const bool in = b0 < N;
+                const int64_t b0 = bh + 32 * c;
+                const bool in = bh < ep_N;  // N is a multiple of 64: the half is wholly in or out
                 if (a.mode == 0) {
-                    if (!in) continue;
+                    if (!in) continue;  // nothing warp-wide below in this pass
                     if (g >= 8) {
-                        float m8[8];
+                        float m8[4];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) m8[j] = max8f(x + 8 * j);
+                        for (int j = 0; j < 4; ++j) m8[j] = max8f(x + 8 * j);
                         if (g == 8) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) count(m8[j]);
+                            for (int j = 0; j < 4; ++j) count(m8[j]);
                         } else if (g == 16) {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) count(fmaxf(m8[2 * j], m8[2 * j + 1]));
-                        } else if (g == 32) {
-                            count(max4f(m8));
-                            count(max4f(m8 + 4));
+                            count(fmaxf(m8[0], m8[1]));
+                            count(fmaxf(m8[2], m8[3]));
                         } else {
-                            const float m64 = max8f(m8);
-                            if (g == 64) {
-                                count(m64);
-                            } else {  // g == 128: one group per tile (or its valid first half)
-                                run = fmaxf(run, m64);
-                                if (h == 1 || b0 + 64 >= N) count(run);
+                            const float m32 = max4f(m8);
+                            if (g == 32) {
+                                count(m32);
+                            } else {  // g == 64: both 32-column parts
+                                run = fmaxf(run, m32);
+                                if (c == 1) count(run);
                             }
                         }
                     } else if (g == 4) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) count(max4f(x + 4 * j));
+                        for (int j = 0; j < 8; ++j) count(max4f(x + 4 * j));
                     } else if (g == 2) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) count(fmaxf(x[2 * j], x[2 * j + 1]));
+                        for (int j = 0; j < 16; ++j) count(fmaxf(x[2 * j], x[2 * j + 1]));
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 64; ++j) count(x[j]);
+                        for (int j = 0; j < 32; ++j) count(x[j]);
                     }
                 } else {
-                    float m4[16], m16[4];
+                    float m4[8];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) m4[j] = max4f(x + 4 * j);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) m16[j] = max4f(m4 + 4 * j);
-                    const float m64 = max4f(m16);
-                    const bool hit = in && m64 >= tau;
-                    if (!__any_sync(LSA_FULL, hit)) continue;
+                    for (int j = 0; j < 8; ++j) m4[j] = max4f(x + 4 * j);
+                    const float m32 = fmaxf(max4f(m4), max4f(m4 + 4));
+                    const bool hit = in && m32 >= tau;
+                    if (!__any_sync(LSA_FULL, hit)) continue;  // every lane votes
                     if (hit) {
-                        int slot = own;
-                        if (!a.whole_range) {  // reserve this half tile's entries
-                            int n = 0;
+                        int n = 0;
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) n += m4[j] >= tau;
-                            slot = atomicAdd(ws.cnt + q, n);
-                        }
-                        if (slot + 16 <= ws.cap) {  // every entry fits: predicated stores per 16-bucket block
+                        for (int j = 0; j < 8; ++j) n += m4[j] >= tau;
+                        int slot = a.whole_range ? atomicAdd(&rowcnt[ep_qt * TQ + ep_r], n) : atomicAdd(ws.cnt + ep_q, n);
+                        if (slot + n <= ws.cap) {  // every entry fits: predicated stores, no branches
 #pragma unroll
-                            for (int kb = 0; kb < 4; ++kb) {
-                                if (m16[kb] < tau) continue;
-#pragma unroll
-                                for (int j = 4 * kb; j < 4 * kb + 4; ++j) {
-                                    const int pj = m4[j] >= tau;
-                                    st_entry_if(pj, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
-                                    slot += pj;
-                                    own += pj;
-                                }
+                            for (int j = 0; j < 8; ++j) {
+                                const int pj = m4[j] >= tau;
+                                st_entry_if(pj, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
+                                slot += pj;
                             }
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
+                            for (int j = 0; j < 8; ++j) {
                                 if (m4[j] >= tau) {
                                     if (slot < ws.cap) st_entry_if(1, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
                                     ++slot;
-                                    ++own;
                                 }
                             }
                         }
                     }
-                }
-            }
-        }
-        if (a.mode == 1 && a.whole_range && q < a.nq) ws.cnt[q] = own;
-        if (a.mode == 0 && q < a.nq && N > 0 && !*abort) {
-            if (a.whole_range) {
-                // this CTA saw every bucket of the query: threshold from the histogram
-                const int64_t G = n_groups(N, a.P);
-                float t = NEG;
-                if (G > a.P) {
-                    int acc = 0;
-                    for (int bin = HIST_BINS - 1; bin > 0; --bin) {
-                        acc += (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
-                        if (acc >= a.P) {
-                            t = hist_edge(bin);
-                            break;
-                        }
-                    }
-                }
-                ws.tau[q] = t;
-            } else {
-                uint32_t *gh = ws.ghist + q * HIST_BINS;
-                for (int bin = 0; bin < HIST_BINS; ++bin) {
-                    const uint32_t c = (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
-                    if (c) atomicAdd(gh + bin, c);
                 }
             }
         }
     }
     __syncthreads();
+    // per-row results, once both halves of every row are in: one thread per row
+    if (warp >= 2 && ep_half == 0 && ep_q < a.nq && ep_N > 0 && !*abort) {
+        uint32_t *hrow = hist + (ep_qt * TQ + ep_r) * HSTRIDE;
+        if (a.mode == 1) {
+            if (a.whole_range) ws.cnt[ep_q] = rowcnt[ep_qt * TQ + ep_r];
+        } else if (a.whole_range) {
+            // this CTA saw every bucket of the query: threshold from the histogram
+            const int64_t G = n_groups(ep_N, a.P);
+            float t = __int_as_float(0xff800000);
+            if (G > a.P) {
+                int acc = 0;
+                for (int bin = HIST_BINS - 1; bin > 0; --bin) {
+                    acc += (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
+                    if (acc >= a.P) {
+                        t = hist_edge(bin);
+                        break;
+                    }
+                }
+            }
+            ws.tau[ep_q] = t;
+        } else {
+            uint32_t *gh = ws.ghist + ep_q * HIST_BINS;
+            for (int bin = 0; bin < HIST_BINS; ++bin) {
+                const uint32_t c = (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
+                if (c) atomicAdd(gh + bin, c);
+            }
+        }
+    }
     if (warp == 0 && lane == 0 && *abort) {
         // copies that may still be in flight (the producer reused a stage only
         // after the MMA had consumed its previous copy): wait for the last
@@ -579,7 +559,7 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
     b.whole_range = (chunks == 1) ? 1 : 0;
     if (whole_range) *whole_range = b.whole_range;
     const size_t smem = A_BYTES + (size_t)(a.mode == 0 ? NST_GMAX : NST_FILTER) * B_BYTES +
-                        (a.mode == 0 ? HIST_BYTES : 0) + sizeof(TcSmem) + 1024;
+                        (a.mode == 0 ? HIST_BYTES : ROWCNT_BYTES) + sizeof(TcSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k_score_tc<<<dim3((unsigned)qpairs, (unsigned)chunks), THREADS, smem, st>>>(tmA, tmB, b, ws);

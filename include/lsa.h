@@ -214,7 +214,9 @@ int lsa_build_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, 
  * sees the buckets of blocks b < H = min(pos/512, cache->n_blocks).
  *   Flat (p->mode == LSA_MODE_FLAT, tree may be NULL): score every visible
  *   bucket, s = <bf16(q/|q|), centroid_bf16> with fp32 accumulation, rank by
- *   (score desc, bucket id asc).
+ *   (score desc, bucket id asc).  Supports caches of up to 65535 blocks
+ *   (33.5M tokens) and k + sink + window < 32768; larger requests return
+ *   LSA_ERR_SHAPE.
  *   Tree: level-synchronous beam search from the root: candidates at level l
  *   are the children of the nodes kept at level l+1 plus the visible
  *   level-l nodes whose parent is not visible; keep the best
