@@ -202,17 +202,6 @@ __device__ __forceinline__ float max8f(const float *v)
     return max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
 }
 
-// Candidate entry (4 scores + first bucket id), stored only when p != 0.
-__device__ __forceinline__ void st_entry_if(int p, float4 *d4, int32_t *dg, const float *x, int32_t g)
-{
-    asm volatile(
-        "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n"
-        " @q st.global.v4.f32 [%1], {%2, %3, %4, %5};\n"
-        " @q st.global.b32 [%6], %7;\n}\n" ::"r"(p),
-        "l"(d4), "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "l"(dg), "r"(g)
-        : "memory");
-}
-
 struct TcSmem {
     uint64_t full[NST_MAX];
     uint64_t empty[NST_MAX];
@@ -425,25 +414,29 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const bool hit = in && m32 >= tau;
                     if (!__any_sync(LSA_FULL, hit)) continue;  // every lane votes
                     if (hit) {
-                        int n = 0;
+                        // one bit per 4-bucket group at or above tau; entries are
+                        // written only for those (usually one per hit lane)
+                        unsigned mask = 0;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) n += m4[j] >= tau;
+                        for (int j = 0; j < 8; ++j) mask |= (m4[j] >= tau ? 1u : 0u) << j;
+                        const int n = __popc(mask);
                         int slot = a.whole_range ? atomicAdd(&rowcnt[ep_qt * TQ + ep_r], n) : atomicAdd(ws.cnt + ep_q, n);
-                        if (slot + n <= ws.cap) {  // every entry fits: predicated stores, no branches
+                        while (mask) {
+                            const int j = __ffs(mask) - 1;
+                            mask &= mask - 1;
+                            // x[4j .. 4j+3] for a runtime j: select on its bits
+                            float4 v[4];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const int pj = m4[j] >= tau;
-                                st_entry_if(pj, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
-                                slot += pj;
+                            for (int i = 0; i < 4; ++i)
+                                v[i] = (j & 1) ? make_float4(x[8 * i + 4], x[8 * i + 5], x[8 * i + 6], x[8 * i + 7])
+                                               : make_float4(x[8 * i], x[8 * i + 1], x[8 * i + 2], x[8 * i + 3]);
+                            const float4 w0 = (j & 2) ? v[1] : v[0], w1 = (j & 2) ? v[3] : v[2];
+                            const float4 e = (j & 4) ? w1 : w0;
+                            if (slot < ws.cap) {
+                                c4[slot] = e;
+                                cg[slot] = (int32_t)(b0 + 4 * j);
                             }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                if (m4[j] >= tau) {
-                                    if (slot < ws.cap) st_entry_if(1, c4 + slot, cg + slot, x + 4 * j, (int32_t)(b0 + 4 * j));
-                                    ++slot;
-                                }
-                            }
+                            ++slot;
                         }
                     }
                 }
