@@ -42,12 +42,16 @@ from hierarchical_key_clustering_b200.layer import SparseLayer  # noqa: E402
 METRIC = "indexer+sparse-attn prefill tokens/s & decode us/token per layer; % roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes per listed (query, KV head, key) row that ncu measured for k_attn on
-# the last 16384 queries of the 128K workload (dram__bytes_read.sum 7.17 GB over
-# 16384 x 2565 x 8 rows; head-major order keeps each head's K/V in L2);
-# roofline.traffic scales it by the rows of a full launch.  Re-measure when
-# k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = 21.0
+# DRAM bytes per listed (query, KV head, key) row that ncu measured for the
+# k_attn launch of each Flat workload (dram__bytes_read.sum + write, divided by
+# the launch's listed rows x Hkv):
+#   flat_128k      7.06 GB + 0.14 GB over the last 16384 queries (a slice: the
+#                  full launch is scaled from it), 2565 x 8 rows each;
+#   flat_1m        437.8 GB + 0.28 GB over 32768 x 4613 x 8 rows (full launch);
+#   flat_tree_10m  1.09 TB + 0.55 GB over 65536 x 4613 x 8 rows (full launch).
+# K/V fit in L2 at 128K (one head's 67 MB stays resident); at 1M and 10M the
+# far keys come from HBM.  Re-measure when k_attn changes.
+ATTN_DRAM_BYTES_PER_ROW = {"flat_128k": 21.4, "flat_1m": 362.3, "flat_tree_10m": 450.8}
 
 
 def peaks():
@@ -225,12 +229,16 @@ def run_ours(args, world, rank, local):
     abytes = attn_algorithmic_bytes(lens_np, hq, hkv)
     achieved = abytes / (attn_ms / 1e3) / 1e9
     traffic = None
-    if ATTN_DRAM_BYTES_PER_ROW is not None:
-        traffic = int(ATTN_DRAM_BYTES_PER_ROW * int(lens_np.sum()) * hkv)
+    per_row = ATTN_DRAM_BYTES_PER_ROW.get(args.workload) if wl["mode"] == "flat" else None
+    if per_row is not None:
+        traffic = int(per_row * int(lens_np.sum()) * hkv)
     roofline = {"kernel": "k_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
                 "peak_source": pk["src"], "algorithmic_bytes": abytes,
-                "traffic_note": "ncu DRAM bytes per listed row on a 16384-query slice, scaled to the launch"}
+                "traffic_note": "ncu DRAM bytes per listed row of this workload's launch, times its rows"}
+    if traffic is not None:  # the same launch measured on the DRAM side: bytes that really crossed HBM
+        roofline["dram_achieved"] = round(traffic / (attn_ms / 1e3) / 1e9, 1)
+        roofline["dram_frac"] = round(traffic / (attn_ms / 1e3) / 1e9 / pk["hbm"], 4)
 
     # end to end: same calls, inputs from pinned host memory, output back to host
     e2e = None if args.no_e2e else run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
