@@ -126,6 +126,8 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x)
 template <int NT>
 __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_split)
 {
+    pdl_wait();
+    pdl_release();
     extern __shared__ __align__(128) uint8_t asmem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t unit = (int64_t)blockIdx.x * AWARPS + warp;
@@ -344,6 +346,8 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
 constexpr int MAX_SPLIT = 1024;
 __global__ void __launch_bounds__(512) k_attn_combine(AttnArgs a)
 {
+    pdl_wait();
+    pdl_release();
     __shared__ float wts[MAX_SPLIT];
     __shared__ float red[16];
     __shared__ float part[3][LSA_HEAD];
@@ -407,13 +411,14 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     kps = ((kps + KCH - 1) / KCH) * KCH;
     const int64_t units = a.nq * a.Hkv * a.nsplit;
     const int64_t blocks = (units + AWARPS - 1) / AWARPS;
-    kern<<<(unsigned)blocks, AWARPS * 32, smem, st>>>(a, kps);
+    // split lists (few queries, decode): short kernels, launched back to back
+    if ((e = launch_k(a.nsplit > 1, kern, dim3((unsigned)blocks), dim3(AWARPS * 32), (size_t)smem, st, a, kps)) !=
+        cudaSuccess)
+        return e;
     count_launches(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.nsplit > 1) {
-        k_attn_combine<<<(unsigned)(a.nq * a.Hq), 512, 0, st>>>(a);
+        e = launch_k(true, k_attn_combine, dim3((unsigned)(a.nq * a.Hq)), dim3(512), 0, st, a);
         count_launches(1);
-        e = cudaGetLastError();
     }
     return e;
 }

@@ -142,6 +142,19 @@ __device__ void block_bitonic_sort(T *a, int n)
     if (n <= 1) __syncthreads();
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the grids this one
+// depends on have completed and their writes are visible (a no-op for an
+// ordinary launch); pdl_release: let the next kernel of the stream start
+// launching, so that its launch and prologue overlap this grid's tail.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void pdl_release()
+{
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 __host__ __device__ __forceinline__ int64_t pow2_ceil64(int64_t x)
 {
     int64_t p = 1;

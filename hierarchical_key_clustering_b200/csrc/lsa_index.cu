@@ -31,6 +31,8 @@ namespace lsa {
 __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, const int64_t *__restrict__ pos,
                                                int64_t nq, int64_t n_blocks, IndexWs ws)
 {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -205,6 +207,8 @@ __device__ __forceinline__ void warp_sort_smem(uint64_t *keys)
 // Tree beam search: one CTA per query, level by level from the root.
 __global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, IndexWs ws)
 {
+    pdl_wait();
+    pdl_release();
     extern __shared__ uint64_t tsm[];
     uint64_t *keys = tsm;                                    // [CM]
     int32_t *cids = reinterpret_cast<int32_t *>(keys + CM);  // [CM]
@@ -396,6 +400,8 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb_total,
                                                           const uint16_t *__restrict__ cbf, int P, IndexWs ws)
 {
+    pdl_wait();
+    pdl_release();
     __shared__ __align__(16) float qf[SMALL_NQ][LSA_D];
     __shared__ uint32_t hs[SMALL_NQ][HIST_BINS];
     extern __shared__ __align__(16) uint8_t ds_dyn[];  // [DS_WARPS][2][32 * DS_ROW] staged rows
@@ -496,6 +502,8 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
 // is >= tau.
 __global__ void __launch_bounds__(256) k_dfilter(int64_t nq, int P, IndexWs ws)
 {
+    pdl_wait();
+    pdl_release();
     __shared__ float tq[SMALL_NQ];
     __shared__ int Nq[SMALL_NQ];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -566,6 +574,8 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                                                       int32_t *__restrict__ lens, int Lmax, int k, int sink,
                                                       int window, int P, int KC, int TW, IndexWs ws)
 {
+    pdl_wait();
+    pdl_release();
     extern __shared__ uint64_t rsm[];
     uint64_t *keys = rsm;                                           // [KC]
     uint32_t *masks = reinterpret_cast<uint32_t *>(keys + KC);      // [RX_SLOTS][RX_MW]
@@ -873,9 +883,10 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     {
         int64_t blocks = (a.nq + 7) / 8;
         if (blocks > (int64_t)n_sm * 32) blocks = (int64_t)n_sm * 32;
-        k_qnorm<<<(unsigned)blocks, 256, 0, st>>>(a.qidx, a.pos, a.nq, a.n_blocks, ws);
+        if ((e = launch_k(a.nq <= SMALL_NQ, k_qnorm, dim3((unsigned)blocks), dim3(256), 0, st, a.qidx, a.pos, a.nq,
+                          a.n_blocks, ws)) != cudaSuccess)
+            return e;
         count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int64_t nb_total = a.n_blocks * LSA_NBKT;
     const bool small = a.nq <= SMALL_NQ;
@@ -883,13 +894,14 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         if (small) {  // stream every centroid once for the whole batch, keep the scores
             const int dsm = DS_WARPS * 2 * 32 * DS_ROW;
             cudaFuncSetAttribute(k_dscore, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-            k_dscore<<<(unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN), DS_WARPS * 32, dsm, st>>>(
-                a.nq, nb_total, a.centroid_bf16, a.P, ws);
+            if ((e = launch_k(true, k_dscore, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
+                              (size_t)dsm, st, a.nq, nb_total, a.centroid_bf16, a.P, ws)) != cudaSuccess)
+                return e;
             count_launches(1);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            k_dfilter<<<(unsigned)((nb_total / 4 + 255) / 256), 256, 0, st>>>(a.nq, a.P, ws);
+            if ((e = launch_k(true, k_dfilter, dim3((unsigned)((nb_total / 4 + 255) / 256)), dim3(256), 0, st, a.nq, a.P,
+                              ws)) != cudaSuccess)
+                return e;
             count_launches(1);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
         } else {  // two passes on the tensor cores: threshold, then filter
             ScoreTcArgs sa;
             sa.nq = a.nq;
@@ -917,9 +929,10 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         const int KM = a.beam > a.P ? a.beam : a.P;
         const size_t smt = (size_t)CM * (sizeof(uint64_t) + sizeof(int32_t)) + (size_t)KM * sizeof(int32_t);
         cudaFuncSetAttribute(k_tree_beam, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smt);
-        k_tree_beam<<<(unsigned)a.nq, 256, smt, st>>>(a.nq, *tree, a.beam, a.P, CM, ws);
+        if ((e = launch_k(small, k_tree_beam, dim3((unsigned)a.nq), dim3(256), smt, st, a.nq, *tree, a.beam, a.P, CM,
+                          ws)) != cudaSuccess)
+            return e;
         count_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
     // candidates held in shared memory: the filter keeps about 1.2-1.45 P per
@@ -928,8 +941,10 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     const size_t smr = rank_expand_smem(KC, TW);
     if (small) {  // one CTA per query, few queries: widest blocks
         cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        k_rank_expand<1024><<<(unsigned)a.nq, 1024, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,
-                                                               a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ws);
+        const cudaError_t el = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
+                                        a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
+                                        a.window, a.P, KC, TW, ws);
+        if (el != cudaSuccess) return el;
     } else {
         cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,

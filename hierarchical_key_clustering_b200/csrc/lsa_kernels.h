@@ -75,6 +75,27 @@ __device__ __forceinline__ int hist_bin(float m)
 // the filter pass.
 constexpr int SMALL_NQ = 16;
 
+// Launch `kern` on `st`; with pdl the launch may begin before the previous
+// kernel of the stream finishes (the kernel waits for it with pdl_wait before
+// reading anything it wrote).  Used on the small-batch (decode) path, where a
+// token's kernels are short and launch latency adds up.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? at : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_pool_norm(const float *keys, int64_t item_begin, int64_t item_end, float *pooled,
                              cudaStream_t st, int n_sm);
 cudaError_t launch_ward(const float *pooled, int64_t blk_begin, int64_t blk_end, int cap, uint8_t *item_bucket,
