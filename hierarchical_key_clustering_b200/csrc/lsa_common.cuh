@@ -109,39 +109,6 @@ __device__ __forceinline__ int32_t rank_key_id(uint64_t k)
     return (int32_t)(uint32_t)(k & 0xffffffffu);
 }
 
-// Block-wide bitonic sort (ascending) of n = power of two keys in shared
-// memory.  All threads of the block must call it.  Thread t owns the pairs
-// whose lower index is t modulo blockDim, so a 32-aligned group of keys is
-// always handled by one warp: consecutive stages with strides below 32 only
-// need a warp barrier, and a block barrier is paid only around the wider
-// strides.
-template <typename T>
-__device__ void block_bitonic_sort(T *a, int n)
-{
-    for (int k = 2; k <= n; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < n; i += blockDim.x) {
-                int ixj = i ^ j;
-                if (ixj > i) {
-                    T x = a[i], y = a[ixj];
-                    bool up = ((i & k) == 0);
-                    if ((x > y) == up) {
-                        a[i] = y;
-                        a[ixj] = x;
-                    }
-                }
-            }
-            const int next_j = (j > 1) ? (j >> 1) : k;
-            if (j < 32 && next_j < 32 && !(j == 1 && k == n)) {
-                __syncwarp();
-            } else {
-                __syncthreads();
-            }
-        }
-    }
-    if (n <= 1) __syncthreads();
-}
-
 // Programmatic dependent launch.  pdl_wait: block until the grids this one
 // depends on have completed and their writes are visible (a no-op for an
 // ordinary launch); pdl_release: let the next kernel of the stream start

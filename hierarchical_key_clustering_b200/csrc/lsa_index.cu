@@ -73,29 +73,6 @@ __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *_
     return acc;
 }
 
-// Score of one tree node, rounded once to fp32 from the fp64 sum over
-// d = 0..63 of the bf16 products taken in that order.  A product of two bf16
-// values is exact in fp64, so each fused step rounds exactly like a separate
-// add and the result is the same fp32 value as a plain fp64 dot product
-// written out in index order.  A beam search cuts at every level; scoring
-// this way makes those cuts independent of the accumulation order.
-__device__ __forceinline__ float dot_bf16_row_f64(const float *qf, const uint16_t *__restrict__ c)
-{
-    const uint4 *c4 = reinterpret_cast<const uint4 *>(c);
-    double acc = 0.0;
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-        uint4 w = __ldg(c4 + v);
-        uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            acc = __fma_rn((double)qf[v * 8 + 2 * h], (double)__uint_as_float(ww[h] << 16), acc);
-            acc = __fma_rn((double)qf[v * 8 + 2 * h + 1], (double)__uint_as_float(ww[h] & 0xffff0000u), acc);
-        }
-    }
-    return __double2float_rn(acc);
-}
-
 // ---------------------------------------------------------------------------
 // Radix select: the P-th largest key (u = f2ord(score)) among values produced
 // by `get(i)` for i in [0, n); all threads of the block call it.
@@ -155,144 +132,357 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
 }
 
 // ---------------------------------------------------------------------------
-// Ascending bitonic sort of 32 E keys held by one warp: element E * lane + r
-// is v[r].  Pairs E or more apart are exchanged across lanes with shuffles,
-// closer pairs inside a lane's registers; no shared memory, no barriers.
-template <int E>
-__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[E])
+// Tree beam search, level by level from the root, one query per team of TEAM
+// warps: TEAM = 1 for many queries (a CTA then holds several independent
+// queries and never synchronises as a whole), TEAM = 8 for a few (latency).
+// Per level the candidates are gathered, scored (fp64 in-order sums, rounded
+// once) and the best B kept.  Keeping the best B is a selection, not a sort:
+// a 256-bin histogram of the scores over their own [min, max] range finds the
+// bin holding the B-th best; the bins above it are kept whole, and the
+// boundary bin's members are ranked exactly by their rank keys (score desc,
+// id asc): by pairwise counting when they are few, by a radix select over the
+// 64-bit keys otherwise.  Rank keys are unique, so the kept set is the one a
+// full sort gives; its order is free (the expansion ranks the entries itself).
+constexpr int TB_BINS = 256;
+constexpr int TB_SMALL = 128;  // boundary members ranked by pairwise counting
+
+// Shared memory of one team: qd double[64] | hist int[256] (later the
+// boundary list, uint64[128]) | ctl int[16] + float[16] | keys uint64[CM] |
+// kept int32[KM].
+__host__ __device__ __forceinline__ size_t tree_beam_team_bytes(int CM, int KM)
 {
-    const int lane = threadIdx.x & 31;
-    for (int k = 2; k <= 32 * E; k <<= 1) {
-        for (int j = k >> 1; j >= E; j >>= 1) {
-            const int lj = j / E;  // lane distance of the pair
-            const bool lower = (lane & lj) == 0;
+    return 512 + 1024 + 128 + 8 * (size_t)CM + ((4 * (size_t)KM + 15) & ~(size_t)15);
+}
+
+template <int TEAM>
+__device__ __forceinline__ void team_sync()
+{
+    if constexpr (TEAM == 1) __syncwarp();
+    else __syncthreads();
+}
+
+// Team-wide minimum and maximum; every thread returns both.
+template <int TEAM>
+__device__ __forceinline__ void team_min_max(float &lo, float &hi, float *red)
+{
 #pragma unroll
-            for (int r = 0; r < E; ++r) {
-                const uint64_t o = __shfl_xor_sync(LSA_FULL, v[r], lj);
-                const bool up = ((E * lane + r) & k) == 0;
-                v[r] = (lower == up) ? (v[r] < o ? v[r] : o) : (v[r] > o ? v[r] : o);
-            }
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(LSA_FULL, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(LSA_FULL, hi, o));
+    }
+    if constexpr (TEAM > 1) {
+        const int w = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) {
+            red[w] = lo;
+            red[TEAM + w] = hi;
         }
+        __syncthreads();
+        lo = red[0];
+        hi = red[TEAM];
 #pragma unroll
-        for (int j = E / 2; j > 0; j >>= 1) {
-            if (j >= k) continue;
-#pragma unroll
-            for (int r = 0; r < E; ++r) {
-                if ((r ^ j) <= r) continue;
-                const bool up = ((E * lane + r) & k) == 0;
-                const uint64_t x = v[r], y = v[r ^ j];
-                if ((x > y) == up) {
-                    v[r] = y;
-                    v[r ^ j] = x;
-                }
-            }
+        for (int k = 1; k < TEAM; ++k) {
+            lo = fminf(lo, red[k]);
+            hi = fmaxf(hi, red[TEAM + k]);
         }
+        __syncthreads();
     }
 }
 
-// keys[0..S) ascending by one warp (S = 32 E); the other warps idle.
-template <int E>
-__device__ __forceinline__ void warp_sort_smem(uint64_t *keys)
+// One warp over a 256-bin histogram: the bin at which the count, taken bin by
+// bin in scan order (descending bins when desc), first reaches need, and the
+// count in the bins scanned before it.  Lane l owns scan positions 8l..8l+7.
+__device__ __forceinline__ void warp_hist_pick(const int *h, int need, bool desc, int &sel, int &before)
 {
     const int lane = threadIdx.x & 31;
-    uint64_t v[E];
+    int c[8], c8 = 0;
 #pragma unroll
-    for (int r = 0; r < E; ++r) v[r] = keys[E * lane + r];
-    warp_bitonic_sort<E>(v);
+    for (int e = 0; e < 8; ++e) {
+        c[e] = h[desc ? 255 - 8 * lane - e : 8 * lane + e];
+        c8 += c[e];
+    }
+    int incl = c8;
 #pragma unroll
-    for (int r = 0; r < E; ++r) keys[E * lane + r] = v[r];
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(LSA_FULL, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int excl = incl - c8;
+    int e_hit = -1, acc = excl;
+    if (excl < need && need <= incl) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (e_hit < 0) {
+                if (acc + c[e] >= need) e_hit = e;
+                else acc += c[e];
+            }
+        }
+    }
+    const unsigned who = __ballot_sync(LSA_FULL, e_hit >= 0);
+    const int src = who ? __ffs(who) - 1 : 0;
+    e_hit = __shfl_sync(LSA_FULL, e_hit, src);
+    acc = __shfl_sync(LSA_FULL, acc, src);
+    if (!who) {  // need exceeds the total: cannot happen; keep the index in range
+        e_hit = 7;
+        acc = 0;
+    }
+    sel = desc ? 255 - 8 * src - e_hit : 8 * src + e_hit;
+    before = acc;
 }
 
-// ---------------------------------------------------------------------------
-// Tree beam search: one CTA per query, level by level from the root.
-__global__ void __launch_bounds__(256) k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, IndexWs ws)
+// Scores of two tree nodes at once (two independent fp64 chains, for latency
+// hiding).  Each is rounded once to fp32 from the fp64 sum over d = 0..63 of
+// the bf16 products taken in that order.  A product of two bf16 values is
+// exact in fp64, so each fused step rounds exactly like a separate add and the
+// result is the fp32 value of a plain fp64 dot product written out in index
+// order.  A beam search cuts at every level; scoring this way makes those cuts
+// independent of the accumulation order.
+__device__ __forceinline__ void dot2_bf16_f64(const double *qd, const uint16_t *__restrict__ ca,
+                                              const uint16_t *__restrict__ cb, float &sa, float &sb)
+{
+    const uint4 *a4 = reinterpret_cast<const uint4 *>(ca);
+    const uint4 *b4 = reinterpret_cast<const uint4 *>(cb);
+    uint4 wa[8], wb[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        wa[v] = __ldg(a4 + v);
+        wb[v] = __ldg(b4 + v);
+    }
+    double x = 0.0, y = 0.0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        const uint32_t ua[4] = {wa[v].x, wa[v].y, wa[v].z, wa[v].w};
+        const uint32_t ub[4] = {wb[v].x, wb[v].y, wb[v].z, wb[v].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const double2 qq = *reinterpret_cast<const double2 *>(qd + v * 8 + 2 * h);
+            x = __fma_rn(qq.x, (double)__uint_as_float(ua[h] << 16), x);
+            y = __fma_rn(qq.x, (double)__uint_as_float(ub[h] << 16), y);
+            x = __fma_rn(qq.y, (double)__uint_as_float(ua[h] & 0xffff0000u), x);
+            y = __fma_rn(qq.y, (double)__uint_as_float(ub[h] & 0xffff0000u), y);
+        }
+    }
+    sa = __double2float_rn(x);
+    sb = __double2float_rn(y);
+}
+
+// Warp-aggregated append: the lanes with pred get consecutive slots from the
+// shared counter *ctr (one atomic per warp); returns the lane's slot.
+__device__ __forceinline__ int warp_append(bool pred, int *ctr)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned m = __ballot_sync(LSA_FULL, pred);
+    int base = 0;
+    if (lane == 0 && m) base = atomicAdd(ctr, __popc(m));
+    base = __shfl_sync(LSA_FULL, base, 0);
+    return base + __popc(m & ((1u << lane) - 1u));
+}
+
+template <int TEAM>
+__global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, int KM, IndexWs ws)
 {
     pdl_wait();
     pdl_release();
-    extern __shared__ uint64_t tsm[];
-    uint64_t *keys = tsm;                                    // [CM]
-    int32_t *cids = reinterpret_cast<int32_t *>(keys + CM);  // [CM]
-    int32_t *kept = cids + CM;                               // [max(W, P)]
-    __shared__ float qf[LSA_D];
-    __shared__ int nc;
-    __shared__ int n_kept;
+    extern __shared__ __align__(16) unsigned char tb_smem[];
+    const int lane = threadIdx.x & 31;
+    constexpr int TT = TEAM * 32;
+    const int tw = TEAM == 1 ? lane : (int)threadIdx.x;
+    const int team = TEAM == 1 ? (int)(threadIdx.x >> 5) : 0;
+    const int64_t q = TEAM == 1 ? (int64_t)blockIdx.x * (blockDim.x >> 5) + team : (int64_t)blockIdx.x;
+    if (q >= nq) return;  // warp-uniform (TEAM 1) or block-uniform (TEAM > 1)
+    unsigned char *base = tb_smem + (size_t)team * tree_beam_team_bytes(CM, KM);
+    double *qd = reinterpret_cast<double *>(base);
+    int *hist = reinterpret_cast<int *>(base + 512);
+    uint64_t *small = reinterpret_cast<uint64_t *>(base + 512);
+    int *ctl = reinterpret_cast<int *>(base + 1536);  // 0 candidates, 1 kept, 2 boundary list, 3.. picks
+    float *red = reinterpret_cast<float *>(base + 1536 + 64);
+    uint64_t *keys = reinterpret_cast<uint64_t *>(base + 1664);
+    int32_t *kept = reinterpret_cast<int32_t *>(keys + CM);
+    const float NEG = __int_as_float(0xff800000);
+    float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
+    int32_t *cg = ws.cand_g + q * ws.cap;
 
-    const int64_t q = blockIdx.x;
-    const int t = threadIdx.x;
     const int H = ws.horizon[q];
-    if (t < LSA_D) qf[t] = bf_bits2f(ws.qhat[q * LSA_D + t]);
-    if (t == 0) n_kept = 0;
-    __syncthreads();
+    for (int d = tw; d < LSA_D; d += TT) qd[d] = (double)bf_bits2f(ws.qhat[q * LSA_D + d]);
+    int n_kept = 0;
     const int top = tv.n_levels - 1;
     for (int l = top; l >= 0; --l) {
-        if (t == 0) nc = 0;
-        __syncthreads();
         const int64_t off = tv.level_offset[l];
+        const int64_t offp = tv.level_offset[l + 1];
         const int64_t size = tv.level_size[l];
-        for (int i = t; i < n_kept; i += blockDim.x) {
-            const int64_t v = tv.level_offset[l + 1] + kept[i];
-            const int32_t c0 = tv.child[2 * v], c1 = tv.child[2 * v + 1];
-            int slot = atomicAdd(&nc, c1 >= 0 ? 2 : 1);
-            cids[slot] = c0;
-            if (c1 >= 0) cids[slot + 1] = c1;
+        if (tw == 0) ctl[0] = ctl[1] = ctl[2] = 0;
+        for (int i = tw; i < TB_BINS; i += TT) hist[i] = 0;
+        team_sync<TEAM>();
+        // candidates: children of the kept nodes, then the visible nodes whose
+        // parent is not visible (only the run of 128 nodes holding block H can
+        // mix the two; at the top level, every visible node)
+        for (int b0 = 0; b0 < n_kept; b0 += TT) {
+            const int i = b0 + tw;
+            int32_t c0 = -1, c1 = -1;
+            if (i < n_kept) {
+                const int64_t v = offp + kept[i];
+                c0 = tv.child[2 * v];
+                c1 = tv.child[2 * v + 1];
+            }
+            const unsigned m0 = __ballot_sync(LSA_FULL, c0 >= 0), m1 = __ballot_sync(LSA_FULL, c1 >= 0);
+            const unsigned lt = (1u << lane) - 1u;
+            const int o = __popc(m0 & lt) + __popc(m1 & lt);
+            int wb = 0;
+            if (lane == 0 && (m0 | m1)) wb = atomicAdd(&ctl[0], __popc(m0) + __popc(m1));
+            wb = __shfl_sync(LSA_FULL, wb, 0) + o;
+            if (c0 >= 0 && wb < CM) keys[wb] = (uint32_t)c0;
+            wb += c0 >= 0;
+            if (c1 >= 0 && wb < CM) keys[wb] = (uint32_t)c1;
         }
-        if (l == top) {
-            for (int64_t u = t; u < size; u += blockDim.x)
-                if (tv.max_block[off + u] < H) cids[atomicAdd(&nc, 1)] = (int32_t)u;
-        } else {
-            // only the run of 128 nodes holding block H can mix visible
-            // nodes with parents that are not visible
-            const int64_t lo = ((int64_t)H >> (l + 1)) * LSA_RUN;
-            const int64_t hi = min(lo + LSA_RUN, size);
-            for (int64_t u = lo + t; u < hi; u += blockDim.x) {
-                const int64_t v = off + u;
-                if (tv.max_block[v] < H && tv.max_block[tv.level_offset[l + 1] + tv.parent[v]] >= H)
-                    cids[atomicAdd(&nc, 1)] = (int32_t)u;
+        {
+            const int64_t lo = l == top ? 0 : ((int64_t)H >> (l + 1)) * LSA_RUN;
+            const int64_t hi = l == top ? size : min(lo + LSA_RUN, size);
+            for (int64_t u0 = lo; u0 < hi; u0 += TT) {
+                const int64_t u = u0 + tw;
+                bool ok = false;
+                if (u < hi) {
+                    const int64_t v = off + u;
+                    ok = tv.max_block[v] < H && (l == top || tv.max_block[offp + tv.parent[v]] >= H);
+                }
+                const int slot = warp_append(ok, &ctl[0]);
+                if (ok && slot < CM) keys[slot] = (uint32_t)u;
             }
         }
-        __syncthreads();
-        const int n = nc;
-        const int S = (int)pow2_ceil64(n > 0 ? n : 1);
-        const int Sp = S < 32 ? 32 : S;  // a warp sorts at least 32 keys
-        for (int i = t; i < Sp; i += blockDim.x) {
-            if (i < n) {
-                const int32_t u = cids[i];
-                keys[i] = rank_key(dot_bf16_row_f64(qf, tv.centroid_bf16 + (off + u) * LSA_D), u);
+        team_sync<TEAM>();
+        const int n = min(ctl[0], CM);
+        int64_t Bl = ((int64_t)P + ((int64_t)1 << l) - 1) >> l;
+        if (Bl < W) Bl = W;
+        const int B = (int)min((int64_t)n, Bl);
+        float smin = __int_as_float(0x7f800000), smax = NEG;
+        if (n > Bl || l == 0) {
+            // scores (rank keys in place of the ids)
+            for (int i0 = tw; i0 < n; i0 += 2 * TT) {
+                const int i1 = i0 + TT;
+                const uint32_t ua = (uint32_t)keys[i0];
+                const uint32_t ub = i1 < n ? (uint32_t)keys[i1] : ua;
+                float sa, sb;
+                dot2_bf16_f64(qd, tv.centroid_bf16 + (off + ua) * LSA_D, tv.centroid_bf16 + (off + ub) * LSA_D, sa, sb);
+                keys[i0] = rank_key(sa, (int32_t)ua);
+                smin = fminf(smin, sa);
+                smax = fmaxf(smax, sa);
+                if (i1 < n) {
+                    keys[i1] = rank_key(sb, (int32_t)ub);
+                    smin = fminf(smin, sb);
+                    smax = fmaxf(smax, sb);
+                }
+            }
+            if (n > Bl) team_min_max<TEAM>(smin, smax, red);
+        }
+        // emit the key as kept (levels above the buckets) or as a candidate
+        // entry (bucket level; one bucket per entry)
+        auto emit = [&](uint64_t key, int slot) {
+            if (l > 0) {
+                if (slot < KM) kept[slot] = rank_key_id(key);
+            } else if (slot < ws.cap) {
+                c4[slot] = make_float4(rank_key_score(key), NEG, NEG, NEG);
+                cg[slot] = rank_key_id(key);
+            }
+        };
+        if (n <= Bl) {
+            for (int i = tw; i < n; i += TT) emit(keys[i], i);
+        } else {
+            // monotone bin of a score over [smin, smax]; equal scores share a bin
+            float scale = smax > smin ? __fdiv_rn((float)TB_BINS, __fsub_rn(smax, smin)) : 0.0f;
+            if (!(scale < 1e30f)) scale = 0.0f;
+            auto binof = [&](uint64_t key) -> int {
+                const int b = (int)__fmul_rn(__fsub_rn(rank_key_score(key), smin), scale);
+                return min(max(b, 0), TB_BINS - 1);
+            };
+            for (int i = tw; i < n; i += TT) atomicAdd(&hist[binof(keys[i])], 1);
+            team_sync<TEAM>();
+            if (TEAM == 1 || threadIdx.x < 32) {
+                int sel, before;
+                warp_hist_pick(hist, B, true, sel, before);
+                if (lane == 0) {
+                    ctl[3] = sel;
+                    ctl[4] = B - before;
+                    ctl[5] = hist[sel];
+                }
+            }
+            team_sync<TEAM>();
+            const int bsel = ctl[3], r = ctl[4], m1 = ctl[5];
+            if (m1 <= TB_SMALL) {
+                // bins above the boundary kept; the boundary bin's members
+                // listed, then ranked by counting
+                for (int b0 = 0; b0 < n; b0 += TT) {
+                    const int i = b0 + tw;
+                    uint64_t key = 0;
+                    int bn = -1;
+                    if (i < n) {
+                        key = keys[i];
+                        bn = binof(key);
+                    }
+                    const int ks = warp_append(bn > bsel, &ctl[1]);
+                    if (bn > bsel) emit(key, ks);
+                    const int ss = warp_append(bn == bsel, &ctl[2]);
+                    if (bn == bsel && ss < TB_SMALL) small[ss] = key;
+                }
+                team_sync<TEAM>();
+                if (TEAM == 1 || threadIdx.x < 32) {
+                    for (int e0 = 0; e0 < m1; e0 += 32) {
+                        const int e = e0 + lane;
+                        const uint64_t ke = e < m1 ? small[e] : ~0ull;
+                        int rank = 0;
+                        for (int j = 0; j < m1; ++j) rank += small[j] < ke;
+                        const bool keep = e < m1 && rank < r;
+                        const int ks = warp_append(keep, &ctl[1]);
+                        if (keep) emit(ke, ks);
+                    }
+                }
             } else {
-                keys[i] = ~0ull;
+                // many members share the boundary bin (near-equal scores):
+                // radix select of the r-th smallest rank key among them
+                uint64_t prefix = 0, mask = 0;
+                int rem = r;
+                for (int shift = 56; shift >= 0; shift -= 8) {
+                    for (int i = tw; i < TB_BINS; i += TT) hist[i] = 0;
+                    team_sync<TEAM>();
+                    for (int i = tw; i < n; i += TT) {
+                        const uint64_t key = keys[i];
+                        if (binof(key) == bsel && (key & mask) == prefix) atomicAdd(&hist[(int)((key >> shift) & 255u)], 1);
+                    }
+                    team_sync<TEAM>();
+                    if (TEAM == 1 || threadIdx.x < 32) {
+                        int sel, before;
+                        warp_hist_pick(hist, rem, false, sel, before);
+                        if (lane == 0) {
+                            ctl[6] = sel;
+                            ctl[7] = before;
+                            ctl[8] = hist[sel];
+                        }
+                    }
+                    team_sync<TEAM>();
+                    prefix |= (uint64_t)ctl[6] << shift;
+                    mask |= (uint64_t)255u << shift;
+                    rem -= ctl[7];
+                    const bool done = ctl[8] == rem;
+                    team_sync<TEAM>();
+                    if (done) break;
+                }
+                for (int b0 = 0; b0 < n; b0 += TT) {
+                    const int i = b0 + tw;
+                    bool keep = false;
+                    uint64_t key = 0;
+                    if (i < n) {
+                        key = keys[i];
+                        const int bn = binof(key);
+                        keep = bn > bsel || (bn == bsel && (key & mask) <= prefix);
+                    }
+                    const int ks = warp_append(keep, &ctl[1]);
+                    if (keep) emit(key, ks);
+                }
             }
         }
-        __syncthreads();
-        if (Sp <= 512) {  // small levels (every level above the last few): one warp, registers only
-            if (t < 32) {
-                if (Sp == 32) warp_sort_smem<1>(keys);
-                else if (Sp == 64) warp_sort_smem<2>(keys);
-                else if (Sp == 128) warp_sort_smem<4>(keys);
-                else if (Sp == 256) warp_sort_smem<8>(keys);
-                else warp_sort_smem<16>(keys);
-            }
-            __syncthreads();
-        } else {
-            block_bitonic_sort(keys, S);
+        if (l == 0 && tw == 0) {  // tau = -inf keeps every entry
+            ws.cnt[q] = B;
+            ws.tau[q] = NEG;
         }
-        int64_t B = ((int64_t)P + ((int64_t)1 << l) - 1) >> l;
-        if (B < W) B = W;
-        const int nk = (int)min((int64_t)n, B);
-        for (int i = t; i < nk; i += blockDim.x) kept[i] = rank_key_id(keys[i]);
-        if (l == 0) {  // one candidate entry per kept bucket; tau = -inf keeps them all
-            const float NEG = __int_as_float(0xff800000);
-            float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
-            for (int i = t; i < nk; i += blockDim.x) {
-                c4[i] = make_float4(rank_key_score(keys[i]), NEG, NEG, NEG);
-                ws.cand_g[q * ws.cap + i] = rank_key_id(keys[i]);
-            }
-            if (t == 0) {
-                ws.cnt[q] = nk;
-                ws.tau[q] = NEG;
-            }
-        }
-        if (t == 0) n_kept = nk;
-        __syncthreads();
+        n_kept = B;
+        team_sync<TEAM>();
     }
 }
 
@@ -925,13 +1115,21 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
     } else if (tree && tree->n_levels > 0) {
         int64_t B1 = ((int64_t)a.P + 1) / 2;
         if (B1 < a.beam) B1 = a.beam;
-        const int CM = (int)pow2_ceil64(2 * B1 + LSA_RUN + 2);
-        const int KM = a.beam > a.P ? a.beam : a.P;
-        const size_t smt = (size_t)CM * (sizeof(uint64_t) + sizeof(int32_t)) + (size_t)KM * sizeof(int32_t);
-        cudaFuncSetAttribute(k_tree_beam, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smt);
-        if ((e = launch_k(small, k_tree_beam, dim3((unsigned)a.nq), dim3(256), smt, st, a.nq, *tree, a.beam, a.P, CM,
-                          ws)) != cudaSuccess)
-            return e;
+        // candidates per level: the children of at most B1 kept nodes plus one run
+        const int CM = (int)(2 * B1 + LSA_RUN + 2);
+        const int KM = (int)B1;
+        const size_t tb = tree_beam_team_bytes(CM, KM);
+        if (small) {  // one query per CTA of 8 warps
+            cudaFuncSetAttribute(k_tree_beam<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb);
+            e = launch_k(true, k_tree_beam<8>, dim3((unsigned)a.nq), dim3(256), tb, st, a.nq, *tree, a.beam, a.P, CM,
+                         KM, ws);
+        } else {  // one query per warp, up to 8 per CTA, two CTAs per SM
+            const int qpb = (int)max((size_t)1, min((size_t)8, (size_t)(113 * 1024) / tb));
+            cudaFuncSetAttribute(k_tree_beam<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(qpb * tb));
+            e = launch_k(false, k_tree_beam<1>, dim3((unsigned)((a.nq + qpb - 1) / qpb)), dim3(32 * qpb), qpb * tb, st,
+                         a.nq, *tree, a.beam, a.P, CM, KM, ws);
+        }
+        if (e != cudaSuccess) return e;
         count_launches(1);
     }
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
