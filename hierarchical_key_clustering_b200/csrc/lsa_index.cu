@@ -133,37 +133,72 @@ __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int 
 
 // ---------------------------------------------------------------------------
 // Tree beam search, level by level from the root, one query per team of TEAM
-// warps: TEAM = 1 for many queries (a CTA then holds several independent
-// queries and never synchronises as a whole), TEAM = 8 for a few (latency).
-// Per level the candidates are gathered, scored (fp64 in-order sums, rounded
-// once) and the best B kept.  Keeping the best B is a selection, not a sort:
-// a 256-bin histogram of the scores over their own [min, max] range finds the
-// bin holding the B-th best; the bins above it are kept whole, and the
-// boundary bin's members are ranked exactly by their rank keys (score desc,
-// id asc): by pairwise counting when they are few, by a radix select over the
-// 64-bit keys otherwise.  Rank keys are unique, so the kept set is the one a
-// full sort gives; its order is free (the expansion ranks the entries itself).
+// warps (teams of a CTA are independent: TEAM = 2 for many queries, 8 for a
+// few).  Per level the candidates are gathered, scored and the best B kept.
+// Keeping the best B is a selection, not a sort: a 256-bin histogram of the
+// scores over their own [min, max] range finds the bin holding the B-th best;
+// the bins above it are kept whole, and the boundary bin's members are ranked
+// exactly by their rank keys (score desc, id asc): by pairwise counting when
+// they are few, by a radix select over the 64-bit keys otherwise.  Rank keys
+// are unique, so the kept set is the one a full sort gives; its order is free
+// (the expansion ranks the entries itself).
+//
+// Candidate slots: the children of kept node i sit at slots 2i and 2i + 1 (a
+// node with one child leaves a hole, key ~0, skipped everywhere), then the
+// visible nodes whose parent is not visible.  Centroid rows are scored from
+// shared memory: a warp copies 32 rows with coalesced 16-byte loads (eight
+// lanes per row, so one load instruction touches 4 lines, not 32), then each
+// lane scores one row.
 constexpr int TB_BINS = 256;
 constexpr int TB_SMALL = 128;  // boundary members ranked by pairwise counting
+constexpr int TB_STAGE = 32 * LSA_D * 2;  // bytes of one warp's staged rows
+constexpr uint64_t TB_HOLE = ~0ull;
+// many queries: teams of BEAM_TEAM warps, BEAM_MINB CTAs per SM sharing its
+// 228 KB of shared memory (1 KB of which each CTA reserves)
+constexpr int BEAM_TEAM = 2, BEAM_MINB = 3;
+constexpr size_t SM_SMEM = 233472;
 
 // Shared memory of one team: qd double[64] | hist int[256] (later the
-// boundary list, uint64[128]) | ctl int[16] + float[16] | keys uint64[CM] |
-// kept int32[KM].
-__host__ __device__ __forceinline__ size_t tree_beam_team_bytes(int CM, int KM)
+// boundary list, uint64[128]) | ctl int[16] + red float[16] | keys uint64[CM]
+// | kept int32[KM] | staged rows, TB_STAGE bytes per warp.
+__host__ __device__ __forceinline__ size_t tree_beam_keys_bytes(int CM) { return (8 * (size_t)CM + 15) & ~(size_t)15; }
+__host__ __device__ __forceinline__ size_t tree_beam_kept_bytes(int KM) { return (4 * (size_t)KM + 15) & ~(size_t)15; }
+__host__ __device__ __forceinline__ size_t tree_beam_team_bytes(int CM, int KM, int team_warps)
 {
-    return 512 + 1024 + 128 + 8 * (size_t)CM + ((4 * (size_t)KM + 15) & ~(size_t)15);
+    return 1664 + tree_beam_keys_bytes(CM) + tree_beam_kept_bytes(KM) + (size_t)team_warps * TB_STAGE;
 }
 
+// Barrier of one team: a warp barrier for one warp, else the named barrier
+// 1 + team over the team's 32 TEAM threads (teams of a CTA never wait on one
+// another).
 template <int TEAM>
-__device__ __forceinline__ void team_sync()
+__device__ __forceinline__ void team_sync(int team)
 {
     if constexpr (TEAM == 1) __syncwarp();
-    else __syncthreads();
+    else asm volatile("bar.sync %0, %1;\n" ::"r"(team + 1), "r"(TEAM * 32) : "memory");
+}
+
+// Team-wide sum of an int; every thread returns it.
+template <int TEAM>
+__device__ __forceinline__ int team_sum(int x, int *red, int team)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(LSA_FULL, x, o);
+    if constexpr (TEAM > 1) {
+        const int w = (threadIdx.x >> 5) % TEAM;
+        if ((threadIdx.x & 31) == 0) red[w] = x;
+        team_sync<TEAM>(team);
+        x = 0;
+#pragma unroll
+        for (int k = 0; k < TEAM; ++k) x += red[k];
+        team_sync<TEAM>(team);
+    }
+    return x;
 }
 
 // Team-wide minimum and maximum; every thread returns both.
 template <int TEAM>
-__device__ __forceinline__ void team_min_max(float &lo, float &hi, float *red)
+__device__ __forceinline__ void team_min_max(float &lo, float &hi, float *red, int team)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -171,12 +206,12 @@ __device__ __forceinline__ void team_min_max(float &lo, float &hi, float *red)
         hi = fmaxf(hi, __shfl_xor_sync(LSA_FULL, hi, o));
     }
     if constexpr (TEAM > 1) {
-        const int w = threadIdx.x >> 5;
+        const int w = (threadIdx.x >> 5) % TEAM;
         if ((threadIdx.x & 31) == 0) {
             red[w] = lo;
             red[TEAM + w] = hi;
         }
-        __syncthreads();
+        team_sync<TEAM>(team);
         lo = red[0];
         hi = red[TEAM];
 #pragma unroll
@@ -184,7 +219,7 @@ __device__ __forceinline__ void team_min_max(float &lo, float &hi, float *red)
             lo = fminf(lo, red[k]);
             hi = fmaxf(hi, red[TEAM + k]);
         }
-        __syncthreads();
+        team_sync<TEAM>(team);
     }
 }
 
@@ -229,40 +264,28 @@ __device__ __forceinline__ void warp_hist_pick(const int *h, int need, bool desc
     before = acc;
 }
 
-// Scores of two tree nodes at once (two independent fp64 chains, for latency
-// hiding).  Each is rounded once to fp32 from the fp64 sum over d = 0..63 of
-// the bf16 products taken in that order.  A product of two bf16 values is
-// exact in fp64, so each fused step rounds exactly like a separate add and the
+// Score of one tree node from its staged row (16-byte segments stored at
+// segment ^ sw), rounded once to fp32 from the fp64 sum over d = 0..63 of the
+// bf16 products taken in that order.  A product of two bf16 values is exact
+// in fp64, so each fused step rounds exactly like a separate add and the
 // result is the fp32 value of a plain fp64 dot product written out in index
-// order.  A beam search cuts at every level; scoring this way makes those cuts
-// independent of the accumulation order.
-__device__ __forceinline__ void dot2_bf16_f64(const double *qd, const uint16_t *__restrict__ ca,
-                                              const uint16_t *__restrict__ cb, float &sa, float &sb)
+// order.  A beam search cuts at every level; scoring this way makes those
+// cuts independent of the accumulation order.
+__device__ __forceinline__ float dot_staged_f64(const double *qd, const uint4 *row, int sw)
 {
-    const uint4 *a4 = reinterpret_cast<const uint4 *>(ca);
-    const uint4 *b4 = reinterpret_cast<const uint4 *>(cb);
-    uint4 wa[8], wb[8];
+    double x = 0.0;
 #pragma unroll
     for (int v = 0; v < 8; ++v) {
-        wa[v] = __ldg(a4 + v);
-        wb[v] = __ldg(b4 + v);
-    }
-    double x = 0.0, y = 0.0;
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-        const uint32_t ua[4] = {wa[v].x, wa[v].y, wa[v].z, wa[v].w};
-        const uint32_t ub[4] = {wb[v].x, wb[v].y, wb[v].z, wb[v].w};
+        const uint4 w = row[v ^ sw];
+        const uint32_t ua[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
             const double2 qq = *reinterpret_cast<const double2 *>(qd + v * 8 + 2 * h);
             x = __fma_rn(qq.x, (double)__uint_as_float(ua[h] << 16), x);
-            y = __fma_rn(qq.x, (double)__uint_as_float(ub[h] << 16), y);
             x = __fma_rn(qq.y, (double)__uint_as_float(ua[h] & 0xffff0000u), x);
-            y = __fma_rn(qq.y, (double)__uint_as_float(ub[h] & 0xffff0000u), y);
         }
     }
-    sa = __double2float_rn(x);
-    sb = __double2float_rn(y);
+    return __double2float_rn(x);
 }
 
 // Warp-aggregated append: the lanes with pred get consecutive slots from the
@@ -277,29 +300,36 @@ __device__ __forceinline__ int warp_append(bool pred, int *ctr)
     return base + __popc(m & ((1u << lane) - 1u));
 }
 
-template <int TEAM>
-__global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, int KM, IndexWs ws)
+// TEAM warps per query, MINB CTAs per SM (register budget).
+template <int TEAM, int MINB>
+__global__ void __launch_bounds__(256, MINB)
+    k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, int KM, IndexWs ws)
 {
     pdl_wait();
     pdl_release();
     extern __shared__ __align__(16) unsigned char tb_smem[];
     const int lane = threadIdx.x & 31;
     constexpr int TT = TEAM * 32;
-    const int tw = TEAM == 1 ? lane : (int)threadIdx.x;
-    const int team = TEAM == 1 ? (int)(threadIdx.x >> 5) : 0;
-    const int64_t q = TEAM == 1 ? (int64_t)blockIdx.x * (blockDim.x >> 5) + team : (int64_t)blockIdx.x;
-    if (q >= nq) return;  // warp-uniform (TEAM 1) or block-uniform (TEAM > 1)
-    unsigned char *base = tb_smem + (size_t)team * tree_beam_team_bytes(CM, KM);
+    constexpr int RUNP = (LSA_RUN + TT - 1) / TT;
+    const int tw = (int)threadIdx.x % TT;
+    const int wi = tw >> 5;
+    const int team = (int)threadIdx.x / TT;
+    const int64_t q = (int64_t)blockIdx.x * (blockDim.x / TT) + team;
+    if (q >= nq) return;  // team-uniform; teams synchronise only among themselves
+    unsigned char *base = tb_smem + (size_t)team * tree_beam_team_bytes(CM, KM, TEAM);
     double *qd = reinterpret_cast<double *>(base);
     int *hist = reinterpret_cast<int *>(base + 512);
     uint64_t *small = reinterpret_cast<uint64_t *>(base + 512);
     int *ctl = reinterpret_cast<int *>(base + 1536);  // 0 candidates, 1 kept, 2 boundary list, 3.. picks
     float *red = reinterpret_cast<float *>(base + 1536 + 64);
     uint64_t *keys = reinterpret_cast<uint64_t *>(base + 1664);
-    int32_t *kept = reinterpret_cast<int32_t *>(keys + CM);
+    int32_t *kept = reinterpret_cast<int32_t *>(base + 1664 + tree_beam_keys_bytes(CM));
+    uint4 *stage = reinterpret_cast<uint4 *>(base + 1664 + tree_beam_keys_bytes(CM) + tree_beam_kept_bytes(KM)) +
+                   wi * (TB_STAGE / 16);
     const float NEG = __int_as_float(0xff800000);
     float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
     int32_t *cg = ws.cand_g + q * ws.cap;
+    const int2 *child2 = reinterpret_cast<const int2 *>(tv.child);
 
     const int H = ws.horizon[q];
     for (int d = tw; d < LSA_D; d += TT) qd[d] = (double)bf_bits2f(ws.qhat[q * LSA_D + d]);
@@ -309,68 +339,90 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
         const int64_t off = tv.level_offset[l];
         const int64_t offp = tv.level_offset[l + 1];
         const int64_t size = tv.level_size[l];
-        if (tw == 0) ctl[0] = ctl[1] = ctl[2] = 0;
-        for (int i = tw; i < TB_BINS; i += TT) hist[i] = 0;
-        team_sync<TEAM>();
-        // candidates: children of the kept nodes, then the visible nodes whose
-        // parent is not visible (only the run of 128 nodes holding block H can
-        // mix the two; at the top level, every visible node)
-        for (int b0 = 0; b0 < n_kept; b0 += TT) {
-            const int i = b0 + tw;
-            int32_t c0 = -1, c1 = -1;
-            if (i < n_kept) {
-                const int64_t v = offp + kept[i];
-                c0 = tv.child[2 * v];
-                c1 = tv.child[2 * v + 1];
-            }
-            const unsigned m0 = __ballot_sync(LSA_FULL, c0 >= 0), m1 = __ballot_sync(LSA_FULL, c1 >= 0);
-            const unsigned lt = (1u << lane) - 1u;
-            const int o = __popc(m0 & lt) + __popc(m1 & lt);
-            int wb = 0;
-            if (lane == 0 && (m0 | m1)) wb = atomicAdd(&ctl[0], __popc(m0) + __popc(m1));
-            wb = __shfl_sync(LSA_FULL, wb, 0) + o;
-            if (c0 >= 0 && wb < CM) keys[wb] = (uint32_t)c0;
-            wb += c0 >= 0;
-            if (c1 >= 0 && wb < CM) keys[wb] = (uint32_t)c1;
-        }
+        const int nch = min(2 * n_kept, CM);  // children slots
+        // visible nodes whose parent is not visible: only the run of 128 nodes
+        // holding block H can mix the two (at the top level, every visible node)
+        bool run_ok[RUNP];
         {
             const int64_t lo = l == top ? 0 : ((int64_t)H >> (l + 1)) * LSA_RUN;
-            const int64_t hi = l == top ? size : min(lo + LSA_RUN, size);
-            for (int64_t u0 = lo; u0 < hi; u0 += TT) {
-                const int64_t u = u0 + tw;
+            const int64_t hi = min(min(l == top ? size : lo + LSA_RUN, size), lo + (int64_t)RUNP * TT);
+#pragma unroll
+            for (int k = 0; k < RUNP; ++k) {
+                const int64_t u = lo + k * TT + tw;
                 bool ok = false;
                 if (u < hi) {
                     const int64_t v = off + u;
                     ok = tv.max_block[v] < H && (l == top || tv.max_block[offp + tv.parent[v]] >= H);
                 }
-                const int slot = warp_append(ok, &ctl[0]);
-                if (ok && slot < CM) keys[slot] = (uint32_t)u;
+                run_ok[k] = ok;
             }
         }
-        team_sync<TEAM>();
-        const int n = min(ctl[0], CM);
+        // children of the kept nodes at fixed slots
+        int holes = 0;
+        for (int i = tw; i < n_kept; i += TT) {
+            const int2 c = __ldg(child2 + offp + kept[i]);
+            if (2 * i + 1 < CM) {
+                keys[2 * i] = c.x >= 0 ? (uint64_t)(uint32_t)c.x : TB_HOLE;
+                keys[2 * i + 1] = c.y >= 0 ? (uint64_t)(uint32_t)c.y : TB_HOLE;
+            }
+            holes += (c.x < 0) + (c.y < 0);
+        }
+        if (tw == 0) {
+            ctl[0] = nch;
+            ctl[1] = ctl[2] = 0;
+        }
+        for (int i = tw; i < TB_BINS; i += TT) hist[i] = 0;
+        team_sync<TEAM>(team);
+        {
+            const int64_t lo = l == top ? 0 : ((int64_t)H >> (l + 1)) * LSA_RUN;
+#pragma unroll
+            for (int k = 0; k < RUNP; ++k) {
+                const int slot = warp_append(run_ok[k], &ctl[0]);
+                if (run_ok[k] && slot < CM) keys[slot] = (uint64_t)(lo + k * TT + tw);
+            }
+        }
+        const int nvalid_hint = team_sum<TEAM>(holes, reinterpret_cast<int *>(red), team);
+        team_sync<TEAM>(team);
+        const int ns = min(ctl[0], CM);   // slots
+        const int n = ns - nvalid_hint;   // valid candidates (slots minus holes)
         int64_t Bl = ((int64_t)P + ((int64_t)1 << l) - 1) >> l;
         if (Bl < W) Bl = W;
         const int B = (int)min((int64_t)n, Bl);
         float smin = __int_as_float(0x7f800000), smax = NEG;
         if (n > Bl || l == 0) {
-            // scores (rank keys in place of the ids)
-            for (int i0 = tw; i0 < n; i0 += 2 * TT) {
-                const int i1 = i0 + TT;
-                const uint32_t ua = (uint32_t)keys[i0];
-                const uint32_t ub = i1 < n ? (uint32_t)keys[i1] : ua;
-                float sa, sb;
-                dot2_bf16_f64(qd, tv.centroid_bf16 + (off + ua) * LSA_D, tv.centroid_bf16 + (off + ub) * LSA_D, sa, sb);
-                keys[i0] = rank_key(sa, (int32_t)ua);
-                smin = fminf(smin, sa);
-                smax = fmaxf(smax, sa);
-                if (i1 < n) {
-                    keys[i1] = rank_key(sb, (int32_t)ub);
-                    smin = fminf(smin, sb);
-                    smax = fmaxf(smax, sb);
+            // scores (rank keys in place of the ids), 32 staged rows at a time
+            const uint16_t *crow = tv.centroid_bf16 + off * LSA_D;
+            for (int c0 = wi * 32; c0 < ns; c0 += TT) {
+                const int m = min(32, ns - c0);
+                uint4 v[8];
+                bool ok[8];
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const int r = 4 * p + (lane >> 3);
+                    const uint64_t id = r < m ? keys[c0 + r] : TB_HOLE;
+                    ok[p] = id != TB_HOLE;
+                    v[p] = ok[p] ? __ldg(reinterpret_cast<const uint4 *>(crow + (int64_t)(uint32_t)id * LSA_D) + (lane & 7))
+                                 : make_uint4(0, 0, 0, 0);
                 }
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const int r = 4 * p + (lane >> 3);
+                    if (ok[p]) stage[r * 8 + ((lane & 7) ^ (r & 7))] = v[p];
+                }
+                __syncwarp();
+                if (lane < m) {
+                    const uint64_t id = keys[c0 + lane];
+                    if (id != TB_HOLE) {
+                        const float s = dot_staged_f64(qd, stage + lane * 8, lane & 7);
+                        keys[c0 + lane] = rank_key(s, (int32_t)(uint32_t)id);
+                        smin = fminf(smin, s);
+                        smax = fmaxf(smax, s);
+                    }
+                }
+                __syncwarp();
             }
-            if (n > Bl) team_min_max<TEAM>(smin, smax, red);
+            team_sync<TEAM>(team);
+            if (n > Bl) team_min_max<TEAM>(smin, smax, red, team);
         }
         // emit the key as kept (levels above the buckets) or as a candidate
         // entry (bucket level; one bucket per entry)
@@ -383,18 +435,27 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
             }
         };
         if (n <= Bl) {
-            for (int i = tw; i < n; i += TT) emit(keys[i], i);
+            for (int b0 = 0; b0 < ns; b0 += TT) {
+                const int i = b0 + tw;
+                const uint64_t key = i < ns ? keys[i] : TB_HOLE;
+                const int ks = warp_append(key != TB_HOLE, &ctl[1]);
+                if (key != TB_HOLE) emit(key, ks);
+            }
         } else {
             // monotone bin of a score over [smin, smax]; equal scores share a bin
             float scale = smax > smin ? __fdiv_rn((float)TB_BINS, __fsub_rn(smax, smin)) : 0.0f;
             if (!(scale < 1e30f)) scale = 0.0f;
             auto binof = [&](uint64_t key) -> int {
+                if (key == TB_HOLE) return -1;
                 const int b = (int)__fmul_rn(__fsub_rn(rank_key_score(key), smin), scale);
                 return min(max(b, 0), TB_BINS - 1);
             };
-            for (int i = tw; i < n; i += TT) atomicAdd(&hist[binof(keys[i])], 1);
-            team_sync<TEAM>();
-            if (TEAM == 1 || threadIdx.x < 32) {
+            for (int i = tw; i < ns; i += TT) {
+                const int b = binof(keys[i]);
+                if (b >= 0) atomicAdd(&hist[b], 1);
+            }
+            team_sync<TEAM>(team);
+            if (tw < 32) {
                 int sel, before;
                 warp_hist_pick(hist, B, true, sel, before);
                 if (lane == 0) {
@@ -403,16 +464,16 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
                     ctl[5] = hist[sel];
                 }
             }
-            team_sync<TEAM>();
+            team_sync<TEAM>(team);
             const int bsel = ctl[3], r = ctl[4], m1 = ctl[5];
             if (m1 <= TB_SMALL) {
                 // bins above the boundary kept; the boundary bin's members
                 // listed, then ranked by counting
-                for (int b0 = 0; b0 < n; b0 += TT) {
+                for (int b0 = 0; b0 < ns; b0 += TT) {
                     const int i = b0 + tw;
                     uint64_t key = 0;
                     int bn = -1;
-                    if (i < n) {
+                    if (i < ns) {
                         key = keys[i];
                         bn = binof(key);
                     }
@@ -421,8 +482,8 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
                     const int ss = warp_append(bn == bsel, &ctl[2]);
                     if (bn == bsel && ss < TB_SMALL) small[ss] = key;
                 }
-                team_sync<TEAM>();
-                if (TEAM == 1 || threadIdx.x < 32) {
+                team_sync<TEAM>(team);
+                if (tw < 32) {
                     for (int e0 = 0; e0 < m1; e0 += 32) {
                         const int e = e0 + lane;
                         const uint64_t ke = e < m1 ? small[e] : ~0ull;
@@ -440,13 +501,14 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
                 int rem = r;
                 for (int shift = 56; shift >= 0; shift -= 8) {
                     for (int i = tw; i < TB_BINS; i += TT) hist[i] = 0;
-                    team_sync<TEAM>();
-                    for (int i = tw; i < n; i += TT) {
+                    team_sync<TEAM>(team);
+                    for (int i = tw; i < ns; i += TT) {
                         const uint64_t key = keys[i];
-                        if (binof(key) == bsel && (key & mask) == prefix) atomicAdd(&hist[(int)((key >> shift) & 255u)], 1);
+                        if (binof(key) == bsel && (key & mask) == prefix)
+                            atomicAdd(&hist[(int)((key >> shift) & 255u)], 1);
                     }
-                    team_sync<TEAM>();
-                    if (TEAM == 1 || threadIdx.x < 32) {
+                    team_sync<TEAM>(team);
+                    if (tw < 32) {
                         int sel, before;
                         warp_hist_pick(hist, rem, false, sel, before);
                         if (lane == 0) {
@@ -455,19 +517,19 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
                             ctl[8] = hist[sel];
                         }
                     }
-                    team_sync<TEAM>();
+                    team_sync<TEAM>(team);
                     prefix |= (uint64_t)ctl[6] << shift;
                     mask |= (uint64_t)255u << shift;
                     rem -= ctl[7];
                     const bool done = ctl[8] == rem;
-                    team_sync<TEAM>();
+                    team_sync<TEAM>(team);
                     if (done) break;
                 }
-                for (int b0 = 0; b0 < n; b0 += TT) {
+                for (int b0 = 0; b0 < ns; b0 += TT) {
                     const int i = b0 + tw;
                     bool keep = false;
                     uint64_t key = 0;
-                    if (i < n) {
+                    if (i < ns) {
                         key = keys[i];
                         const int bn = binof(key);
                         keep = bn > bsel || (bn == bsel && (key & mask) <= prefix);
@@ -482,7 +544,7 @@ __global__ void __launch_bounds__(256, 2) k_tree_beam(int64_t nq, TreeView tv, i
             ws.tau[q] = NEG;
         }
         n_kept = B;
-        team_sync<TEAM>();
+        team_sync<TEAM>(team);
     }
 }
 
@@ -1118,16 +1180,19 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         // candidates per level: the children of at most B1 kept nodes plus one run
         const int CM = (int)(2 * B1 + LSA_RUN + 2);
         const int KM = (int)B1;
-        const size_t tb = tree_beam_team_bytes(CM, KM);
         if (small) {  // one query per CTA of 8 warps
-            cudaFuncSetAttribute(k_tree_beam<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb);
-            e = launch_k(true, k_tree_beam<8>, dim3((unsigned)a.nq), dim3(256), tb, st, a.nq, *tree, a.beam, a.P, CM,
-                         KM, ws);
-        } else {  // one query per warp, up to 8 per CTA, two CTAs per SM
-            const int qpb = (int)max((size_t)1, min((size_t)8, (size_t)(113 * 1024) / tb));
-            cudaFuncSetAttribute(k_tree_beam<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(qpb * tb));
-            e = launch_k(false, k_tree_beam<1>, dim3((unsigned)((a.nq + qpb - 1) / qpb)), dim3(32 * qpb), qpb * tb, st,
-                         a.nq, *tree, a.beam, a.P, CM, KM, ws);
+            auto kern = k_tree_beam<8, 1>;
+            const size_t tb = tree_beam_team_bytes(CM, KM, 8);
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb);
+            e = launch_k(true, kern, dim3((unsigned)a.nq), dim3(256), tb, st, a.nq, *tree, a.beam, a.P, CM, KM, ws);
+        } else {  // BEAM_TEAM warps per query, teams of a CTA independent
+            auto kern = k_tree_beam<BEAM_TEAM, BEAM_MINB>;
+            const size_t tb = tree_beam_team_bytes(CM, KM, BEAM_TEAM);
+            const int per_cta = 8 / BEAM_TEAM;
+            const int qpb = (int)max((size_t)1, min((size_t)per_cta, (SM_SMEM / BEAM_MINB - 1024) / tb));
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(qpb * tb));
+            e = launch_k(false, kern, dim3((unsigned)((a.nq + qpb - 1) / qpb)), dim3(32 * BEAM_TEAM * qpb), qpb * tb,
+                         st, a.nq, *tree, a.beam, a.P, CM, KM, ws);
         }
         if (e != cudaSuccess) return e;
         count_launches(1);
