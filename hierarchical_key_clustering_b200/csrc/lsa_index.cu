@@ -159,13 +159,15 @@ constexpr int BEAM_TEAM = 2, BEAM_MINB = 3;
 constexpr size_t SM_SMEM = 233472;
 
 // Shared memory of one team: qd double[64] | hist int[256] (later the
-// boundary list, uint64[128]) | ctl int[16] + red float[16] | keys uint64[CM]
-// | kept int32[KM] | staged rows, TB_STAGE bytes per warp.
+// boundary list, uint64[128]) | ctl int[16] | red float[32] (two per warp of
+// a team of up to 16) | keys uint64[CM] | kept int32[KM] | staged rows,
+// TB_STAGE bytes per warp.
+constexpr int TB_KEYS_OFF = 512 + 1024 + 64 + 128;
 __host__ __device__ __forceinline__ size_t tree_beam_keys_bytes(int CM) { return (8 * (size_t)CM + 15) & ~(size_t)15; }
 __host__ __device__ __forceinline__ size_t tree_beam_kept_bytes(int KM) { return (4 * (size_t)KM + 15) & ~(size_t)15; }
 __host__ __device__ __forceinline__ size_t tree_beam_team_bytes(int CM, int KM, int team_warps)
 {
-    return 1664 + tree_beam_keys_bytes(CM) + tree_beam_kept_bytes(KM) + (size_t)team_warps * TB_STAGE;
+    return TB_KEYS_OFF + tree_beam_keys_bytes(CM) + tree_beam_kept_bytes(KM) + (size_t)team_warps * TB_STAGE;
 }
 
 // Barrier of one team: a warp barrier for one warp, else the named barrier
@@ -302,13 +304,14 @@ __device__ __forceinline__ int warp_append(bool pred, int *ctr)
 
 // TEAM warps per query, MINB CTAs per SM (register budget).
 template <int TEAM, int MINB>
-__global__ void __launch_bounds__(256, MINB)
+__global__ void __launch_bounds__(TEAM >= 8 ? 32 * TEAM : 256, MINB)
     k_tree_beam(int64_t nq, TreeView tv, int W, int P, int CM, int KM, IndexWs ws)
 {
     pdl_wait();
     pdl_release();
     extern __shared__ __align__(16) unsigned char tb_smem[];
     const int lane = threadIdx.x & 31;
+    static_assert(TEAM >= 1 && TEAM <= 16 && 256 / (32 * TEAM) <= 15, "team reductions hold 2 floats per warp of <= 16; barrier ids 1..15");
     constexpr int TT = TEAM * 32;
     constexpr int RUNP = (LSA_RUN + TT - 1) / TT;
     const int tw = (int)threadIdx.x % TT;
@@ -322,10 +325,11 @@ __global__ void __launch_bounds__(256, MINB)
     uint64_t *small = reinterpret_cast<uint64_t *>(base + 512);
     int *ctl = reinterpret_cast<int *>(base + 1536);  // 0 candidates, 1 kept, 2 boundary list, 3.. picks
     float *red = reinterpret_cast<float *>(base + 1536 + 64);
-    uint64_t *keys = reinterpret_cast<uint64_t *>(base + 1664);
-    int32_t *kept = reinterpret_cast<int32_t *>(base + 1664 + tree_beam_keys_bytes(CM));
-    uint4 *stage = reinterpret_cast<uint4 *>(base + 1664 + tree_beam_keys_bytes(CM) + tree_beam_kept_bytes(KM)) +
-                   wi * (TB_STAGE / 16);
+    uint64_t *keys = reinterpret_cast<uint64_t *>(base + TB_KEYS_OFF);
+    int32_t *kept = reinterpret_cast<int32_t *>(base + TB_KEYS_OFF + tree_beam_keys_bytes(CM));
+    uint4 *stage =
+        reinterpret_cast<uint4 *>(base + TB_KEYS_OFF + tree_beam_keys_bytes(CM) + tree_beam_kept_bytes(KM)) +
+        wi * (TB_STAGE / 16);
     const float NEG = __int_as_float(0xff800000);
     float4 *c4 = reinterpret_cast<float4 *>(ws.cand4) + q * ws.cap;
     int32_t *cg = ws.cand_g + q * ws.cap;
@@ -335,26 +339,36 @@ __global__ void __launch_bounds__(256, MINB)
     for (int d = tw; d < LSA_D; d += TT) qd[d] = (double)bf_bits2f(ws.qhat[q * LSA_D + d]);
     int n_kept = 0;
     const int top = tv.n_levels - 1;
+    // Visible nodes whose parent is not visible: only the run of 128 nodes
+    // holding block H can mix the two (at the top level, every visible node).
+    // Each level's flags are loaded while the level above is processed.
+    bool run_ok[RUNP];
+    int32_t rmb[RUNP], rpar[RUNP];
+    {
+        const int64_t off = tv.level_offset[top], hi = min(tv.level_size[top], (int64_t)RUNP * TT);
+#pragma unroll
+        for (int k = 0; k < RUNP; ++k) {
+            const int64_t u = k * TT + tw;
+            run_ok[k] = u < hi && tv.max_block[off + u] < H;
+        }
+    }
     for (int l = top; l >= 0; --l) {
         const int64_t off = tv.level_offset[l];
         const int64_t offp = tv.level_offset[l + 1];
-        const int64_t size = tv.level_size[l];
         const int nch = min(2 * n_kept, CM);  // children slots
-        // visible nodes whose parent is not visible: only the run of 128 nodes
-        // holding block H can mix the two (at the top level, every visible node)
-        bool run_ok[RUNP];
-        {
-            const int64_t lo = l == top ? 0 : ((int64_t)H >> (l + 1)) * LSA_RUN;
-            const int64_t hi = min(min(l == top ? size : lo + LSA_RUN, size), lo + (int64_t)RUNP * TT);
+        if (l > 0) {  // the next level's run: visibility and parents
+            const int64_t rlo = ((int64_t)H >> l) * LSA_RUN;
+            const int64_t rhi = min(min(rlo + LSA_RUN, tv.level_size[l - 1]), rlo + (int64_t)RUNP * TT);
+            const int64_t offn = tv.level_offset[l - 1];
 #pragma unroll
             for (int k = 0; k < RUNP; ++k) {
-                const int64_t u = lo + k * TT + tw;
-                bool ok = false;
-                if (u < hi) {
-                    const int64_t v = off + u;
-                    ok = tv.max_block[v] < H && (l == top || tv.max_block[offp + tv.parent[v]] >= H);
+                const int64_t u = rlo + k * TT + tw;
+                rmb[k] = INT_MAX;
+                rpar[k] = 0;
+                if (u < rhi) {
+                    rmb[k] = tv.max_block[offn + u];
+                    rpar[k] = tv.parent[offn + u];
                 }
-                run_ok[k] = ok;
             }
         }
         // children of the kept nodes at fixed slots
@@ -381,10 +395,10 @@ __global__ void __launch_bounds__(256, MINB)
                 if (run_ok[k] && slot < CM) keys[slot] = (uint64_t)(lo + k * TT + tw);
             }
         }
-        const int nvalid_hint = team_sum<TEAM>(holes, reinterpret_cast<int *>(red), team);
+        const int nholes = team_sum<TEAM>(holes, reinterpret_cast<int *>(red), team);
         team_sync<TEAM>(team);
-        const int ns = min(ctl[0], CM);   // slots
-        const int n = ns - nvalid_hint;   // valid candidates (slots minus holes)
+        const int ns = min(ctl[0], CM);  // slots
+        const int n = ns - nholes;  // valid candidates
         int64_t Bl = ((int64_t)P + ((int64_t)1 << l) - 1) >> l;
         if (Bl < W) Bl = W;
         const int B = (int)min((int64_t)n, Bl);
@@ -542,6 +556,10 @@ __global__ void __launch_bounds__(256, MINB)
         if (l == 0 && tw == 0) {  // tau = -inf keeps every entry
             ws.cnt[q] = B;
             ws.tau[q] = NEG;
+        }
+        if (l > 0) {  // parents of the next level's run sit at this level
+#pragma unroll
+            for (int k = 0; k < RUNP; ++k) run_ok[k] = rmb[k] < H && tv.max_block[off + rpar[k]] >= H;
         }
         n_kept = B;
         team_sync<TEAM>(team);
@@ -1180,11 +1198,11 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         // candidates per level: the children of at most B1 kept nodes plus one run
         const int CM = (int)(2 * B1 + LSA_RUN + 2);
         const int KM = (int)B1;
-        if (small) {  // one query per CTA of 8 warps
-            auto kern = k_tree_beam<8, 1>;
-            const size_t tb = tree_beam_team_bytes(CM, KM, 8);
+        if (small) {  // one query per CTA of 16 warps
+            auto kern = k_tree_beam<16, 1>;
+            const size_t tb = tree_beam_team_bytes(CM, KM, 16);
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb);
-            e = launch_k(true, kern, dim3((unsigned)a.nq), dim3(256), tb, st, a.nq, *tree, a.beam, a.P, CM, KM, ws);
+            e = launch_k(true, kern, dim3((unsigned)a.nq), dim3(512), tb, st, a.nq, *tree, a.beam, a.P, CM, KM, ws);
         } else {  // BEAM_TEAM warps per query, teams of a CTA independent
             auto kern = k_tree_beam<BEAM_TEAM, BEAM_MINB>;
             const size_t tb = tree_beam_team_bytes(CM, KM, BEAM_TEAM);
