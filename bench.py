@@ -279,25 +279,20 @@ def run_ours(args, world, rank, local):
 
 
 def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, dev, world):
+    """The step through SparseLayer.prefill_from_host: inputs from pinned host
+    memory, O back to pinned host memory, every step (transfers overlapped
+    with the kernels on copy streams, the step still ends after its last
+    copy back)."""
     st = torch.cuda.current_stream()
     pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
     h_keys, h_q, h_pos = pin(keys_np), pin(q_np), pin(pos_np)
     h_Q, h_K, h_V = Qd.cpu().pin_memory(), Kd.cpu().pin_memory(), Vd.cpu().pin_memory()
     h_O = torch.empty(Qd.shape, dtype=Qd.dtype).pin_memory()
-    d_keys, d_q, d_pos = torch.empty_like(h_keys, device=dev), torch.empty_like(h_q, device=dev), \
-        torch.empty_like(h_pos, device=dev)
-    d_Q, d_K, d_V = torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd)
-    d_O = torch.empty_like(Qd)
     h2d = sum(t.numel() * t.element_size() for t in (h_keys, h_q, h_pos, h_Q, h_K, h_V))
     d2h = h_O.numel() * h_O.element_size()
 
     def step():
-        for d, h in ((d_keys, h_keys), (d_q, h_q), (d_pos, h_pos), (d_Q, h_Q), (d_K, h_K), (d_V, h_V)):
-            d.copy_(h, non_blocking=True)
-        layer.build(d_keys)
-        layer.index(d_q, d_pos)
-        layer.attend(d_Q, d_K, d_V, d_O)
-        h_O.copy_(d_O, non_blocking=True)
+        layer.prefill_from_host(h_keys, h_q, h_pos, h_Q, h_K, h_V, h_O)
 
     for _ in range(max(1, args.warmup)):
         step()

@@ -190,6 +190,18 @@ int64_t attention_ws_bytes(int64_t nq, int32_t Hq, int32_t nsplit)
     return align256(nq * Hq * (int64_t)nsplit * LSA_HEAD_DIM * 4) + align256(nq * Hq * (int64_t)nsplit * 2 * 4);
 }
 
+// Batches of at least this many queries take the near-set path (a tile of
+// consecutive queries shares its sink and window rows); its workspace holds
+// one partial result per (query, head) and one plan per query.
+constexpr int64_t NEAR_MIN_NQ = 64;
+int64_t near_ws_bytes(int64_t nq, int32_t Hq)
+{
+    if (nq < NEAR_MIN_NQ) return 0;
+    // tiles hold at least one query: nq tile records bound every tile count
+    return align256(nq * Hq * (int64_t)LSA_HEAD_DIM * 4) + align256(nq * Hq * (int64_t)2 * 4) + align256(nq * 8) +
+           align256(nq * 16);
+}
+
 int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache, const lsa_tree *tree,
                int32_t *lists, int32_t *lens, int32_t Lmax, const lsa_params *p, void *ws, int64_t ws_bytes,
                void *stream)
@@ -413,7 +425,9 @@ int64_t lsa_index_workspace_bytes(int64_t nq, int64_t n_blocks, const lsa_params
 int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, int32_t Lmax)
 {
     if (nq < 0 || Hq < 1 || head_dim != LSA_HEAD_DIM || Lmax < 1) return -1;
-    return attention_ws_bytes(nq, Hq, attention_nsplit(nq, 1, Lmax));
+    const int64_t split = attention_ws_bytes(nq, Hq, attention_nsplit(nq, 1, Lmax));
+    const int64_t near = near_ws_bytes(nq, Hq);
+    return split > near ? split : near;
 }
 
 int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache *cache, const lsa_params *p,
@@ -513,6 +527,18 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
     a.nsplit = nsplit;
     a.part_o = nullptr;
     a.part_ml = nullptr;
+    a.near_plan = nullptr;
+    a.near_tile = nullptr;
+    a.near_o = nullptr;
+    a.near_ml = nullptr;
+    const int64_t nb = near_ws_bytes(nq, Hq);
+    if (nsplit == 1 && nb > 0 && lsa::near_tile_queries(Hq / Hkv) > 0 && ws && ws_bytes >= nb &&
+        ((uintptr_t)ws & 255u) == 0) {
+        a.near_o = (float *)ws;
+        a.near_ml = (float *)((char *)ws + align256(nq * Hq * (int64_t)LSA_HEAD_DIM * 4));
+        a.near_plan = (int2 *)((char *)a.near_ml + align256(nq * Hq * (int64_t)2 * 4));
+        a.near_tile = (int4 *)((char *)a.near_plan + align256(nq * 8));
+    }
     if (nsplit > 1) {
         if (((uintptr_t)ws & 255u) != 0) return fail(LSA_ERR_ARG, "workspace must be 256-byte aligned");
         a.part_o = (float *)ws;

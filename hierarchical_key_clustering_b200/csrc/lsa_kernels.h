@@ -157,7 +157,18 @@ struct AttnArgs {
     float *part_o;   // [nq, Hq, nsplit, 128] (nsplit > 1 only)
     float *part_ml;  // [nq, Hq, nsplit, 2]
     int32_t nsplit;
+    // near-set split (nsplit == 1 only; NULL = off): per query the sink
+    // prefix and window suffix of its list taken densely, and their partial
+    // results [nq, Hq, 128] / [nq, Hq, 2] (running max in log2 units, sum)
+    int2 *near_plan;
+    int4 *near_tile;  // per tile: {usable, first position, lowest near key, longest sink prefix}
+    float *near_o;
+    float *near_ml;
 };
+
+// Queries per near-set tile for G query heads per KV head, 0 = no near path.
+constexpr int NEAR_ROWS = 128;
+__host__ __device__ inline int near_tile_queries(int G) { return (G >= 1 && NEAR_ROWS % G == 0) ? NEAR_ROWS / G : 0; }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm);
 int attention_list_cap();

@@ -28,6 +28,8 @@ class SparseLayer:
                                      device)
         self.lists = torch.empty((max_queries, self.Lmax), dtype=torch.int32, device=device)
         self.lens = torch.empty((max_queries,), dtype=torch.int32, device=device)
+        self._h2d = self._d2h = None  # copy streams of prefill_from_host
+        self._dbuf, self._dbuf_key = None, None
 
     def build(self, keys: torch.Tensor, t_begin: int = 0, t_end: int | None = None, stream=None):
         t_end = keys.shape[0] if t_end is None else t_end
@@ -47,3 +49,67 @@ class SparseLayer:
         lsa.lsa_sparse_attention(Q, K, V, self.lists[:nq], self.lens[:nq], O, lse, ws=self.ws_attn,
                                  stream=stream)
         return O
+
+    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int = 8):
+        """One prefill step whose inputs and output live in pinned host memory.
+
+        Three streams overlap the transfers with the kernels: the index
+        inputs go first and the cache build and index start as soon as they
+        land, while K and V follow; Q then arrives in query chunks (multiples
+        of 128 queries, so the near-set tiles of the attention do not change)
+        and each chunk's attention starts when its Q is on the device; each
+        chunk's O is copied back while the next chunks compute.  Every copy
+        and kernel of the call is ordered after the work already queued on
+        the current stream, and the current stream waits for the last copy
+        back, so the call behaves as one stream-ordered step.  The results are
+        those of build + index + attend on device copies of the inputs, up to
+        the attention's summation order when a chunk holds so few (query, KV
+        head) units that the attention splits lists over warps.
+        """
+        nq = h_Q.shape[0]
+        assert nq <= self.max_queries
+        dev = self.lists.device
+        cs = torch.cuda.current_stream(dev)
+        if self._h2d is None:
+            self._h2d, self._d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        hs = (h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O)
+        key = tuple((tuple(t.shape), t.dtype) for t in hs)
+        if self._dbuf_key != key:
+            self._dbuf = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hs]
+            self._dbuf_key = key
+        d_keys, d_q, d_pos, d_Q, d_K, d_V, d_O = self._dbuf
+        step = -(-nq // max(1, chunks))
+        step = -(-step // 128) * 128
+        bounds = [(c0, min(nq, c0 + step)) for c0 in range(0, nq, step)]
+        self._h2d.wait_stream(cs)
+        with torch.cuda.stream(self._h2d):
+            for d, h in ((d_keys, h_keys), (d_q, h_qidx), (d_pos, h_pos)):
+                d.copy_(h, non_blocking=True)
+            e_idx = torch.cuda.Event()
+            e_idx.record()
+            d_K.copy_(h_K, non_blocking=True)
+            d_V.copy_(h_V, non_blocking=True)
+            e_kv = torch.cuda.Event()
+            e_kv.record()
+            e_q = []
+            for c0, c1 in bounds:
+                d_Q[c0:c1].copy_(h_Q[c0:c1], non_blocking=True)
+                e_q.append(torch.cuda.Event())
+                e_q[-1].record()
+        cs.wait_event(e_idx)
+        self.build(d_keys, stream=cs)
+        self.index(d_q, d_pos, stream=cs)
+        cs.wait_event(e_kv)
+        e_o = []
+        for (c0, c1), eq in zip(bounds, e_q):
+            cs.wait_event(eq)
+            lsa.lsa_sparse_attention(d_Q[c0:c1], d_K, d_V, self.lists[c0:c1], self.lens[c0:c1], d_O[c0:c1],
+                                     None if lse is None else lse[c0:c1], ws=self.ws_attn, stream=cs)
+            e_o.append(torch.cuda.Event())
+            e_o[-1].record(cs)
+        with torch.cuda.stream(self._d2h):
+            for (c0, c1), eo in zip(bounds, e_o):
+                self._d2h.wait_event(eo)
+                h_O[c0:c1].copy_(d_O[c0:c1], non_blocking=True)
+        cs.wait_stream(self._d2h)
+        return h_O

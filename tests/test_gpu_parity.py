@@ -179,6 +179,58 @@ def test_attention_against_oracle(tiny, hq, hkv, nq):
     PT.assert_attention_close(Od, Oref, lse, lse_ref)
 
 
+@pytest.mark.parametrize("hq,hkv,p0,nq", [(32, 8, 1000, 300), (8, 1, 0, 200), (16, 1, 3000, 100), (16, 16, 2000, 130),
+                                          (32, 8, 500, 64)])
+def test_attention_near_tiles_against_oracle(tiny, hq, hkv, p0, nq):
+    """Consecutive queries: their sink and window keys go through the
+    near-set tiles (from position 0, where sink and window meet, up), the rest
+    of each list through the gather; the merge must match the oracle."""
+    _need_gpu()
+    keys, q, pos, oc = tiny
+    sel = np.arange(p0, p0 + nq, dtype=np.int64)
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    Qb, Kb, Vb = I.qkv_bf16_bits(7, nq, 4096, hq, hkv)
+    Oref, lse_ref = O.attention(Qb, Kb, Vb, ol, on)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, ol.shape[1]))
+    lsa.lsa_sparse_attention(Qd, Kd, Vd, PT.to_dev(ol), PT.to_dev(on), Od, lse, ws=ws)
+    torch.cuda.synchronize()
+    PT.assert_attention_close(Od, Oref, lse, lse_ref)
+
+
+def test_attention_near_tiles_irregular_lists(tiny):
+    """Lists without a window (random subsets ending at the query's position),
+    and a batch whose positions jump inside a tile: the near-set plan must
+    take only what each list holds and fall back to the gather otherwise."""
+    _need_gpu()
+    rng = np.random.default_rng(11)
+    nq, hq, hkv, T = 257, 32, 8, 4096
+    p = np.arange(1500, 1500 + nq, dtype=np.int64)
+    p[100:] += 7  # tiles 3 (queries 96..127) and up: 3 is not consecutive
+    Lmax = 600
+    lists = np.full((nq, Lmax), -1, np.int32)
+    lens = np.zeros(nq, np.int32)
+    for i in range(nq):
+        if i % 3 == 0:  # dense tail and head, random middle
+            mid = np.sort(rng.choice(np.arange(6, p[i] - 300), size=100, replace=False))
+            li = np.concatenate([np.arange(0, 6), mid, np.arange(p[i] - 299, p[i] + 1)])
+        else:  # random subset that ends at p
+            li = np.concatenate([np.sort(rng.choice(p[i], size=rng.integers(1, 500), replace=False)), [p[i]]])
+        lists[i, :len(li)] = li
+        lens[i] = len(li)
+    Qb, Kb, Vb = I.qkv_bf16_bits(8, nq, T, hq, hkv)
+    Oref, lse_ref = O.attention(Qb, Kb, Vb, lists, lens)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, Lmax))
+    lsa.lsa_sparse_attention(Qd, Kd, Vd, PT.to_dev(lists), PT.to_dev(lens), Od, lse, ws=ws)
+    torch.cuda.synchronize()
+    PT.assert_attention_close(Od, Oref, lse, lse_ref)
+
+
 def test_attention_dense_causal_single_key(tiny):
     """A one-key list returns that key's value row exactly (up to bf16)."""
     _need_gpu()
@@ -239,3 +291,29 @@ def test_small_and_large_batch_paths_agree(tiny):
         PT.assert_lists_match(sl, sn, ol[a:a + 8], on[a:a + 8], q[sel[a:a + 8]], pos[sel[a:a + 8]], oc, k=256)
         same += sum(int(sn[i] == big_n[a + i] and np.array_equal(sl[i], big_l[a + i])) for i in range(len(sn)))
     assert same >= len(sel) - 2
+
+
+def test_prefill_from_host_matches_device_path(tiny):
+    """The pipelined host-memory step (copy streams, query chunks) gives the
+    same O, bit for bit, as build + index + attend on device inputs (8 KV
+    heads: every chunk has enough (query, head) units to keep whole lists)."""
+    _need_gpu()
+    from hierarchical_key_clustering_b200.layer import SparseLayer
+    keys, q, pos, _ = tiny
+    nq, hq, hkv = 4096, 32, 8
+    Qb, Kb, Vb = I.qkv_bf16_bits(9, nq, 4096, hq, hkv)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    dev_layer = SparseLayer(4096, k=256, max_queries=nq, Hq=hq)
+    dev_layer.build(PT.to_dev(keys))
+    dev_layer.index(PT.to_dev(q), PT.to_dev(pos))
+    Od = torch.empty_like(Qd)
+    dev_layer.attend(Qd, Kd, Vd, Od)
+    host_layer = SparseLayer(4096, k=256, max_queries=nq, Hq=hq)
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_O = torch.empty(Qd.shape, dtype=Qd.dtype).pin_memory()
+    for chunks in (5, 1):
+        h_O.zero_()
+        host_layer.prefill_from_host(pin(torch.from_numpy(keys)), pin(torch.from_numpy(q)),
+                                     pin(torch.from_numpy(pos)), pin(Qd), pin(Kd), pin(Vd), h_O, chunks=chunks)
+        torch.cuda.synchronize()
+        assert torch.equal(h_O, Od.cpu())
