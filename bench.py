@@ -42,16 +42,19 @@ from hierarchical_key_clustering_b200.layer import SparseLayer  # noqa: E402
 METRIC = "indexer+sparse-attn prefill tokens/s & decode us/token per layer; % roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes per listed (query, KV head, key) row that ncu measured for the
-# k_attn launch of each Flat workload (dram__bytes_read.sum + write, divided by
-# the launch's listed rows x Hkv):
-#   flat_128k      7.06 GB + 0.14 GB over the last 16384 queries (a slice: the
-#                  full launch is scaled from it), 2565 x 8 rows each;
-#   flat_1m        437.8 GB + 0.28 GB over 32768 x 4613 x 8 rows (full launch);
-#   flat_tree_10m  1.09 TB + 0.55 GB over 65536 x 4613 x 8 rows (full launch).
-# K/V fit in L2 at 128K (one head's 67 MB stays resident); at 1M and 10M the
-# far keys come from HBM.  Re-measure when k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = {"flat_128k": 21.4, "flat_1m": 362.3, "flat_tree_10m": 450.8}
+# DRAM bytes per far (query, KV head, key) row -- a list entry the gather
+# kernel k_attn reads -- that ncu measured for the k_attn launch of each Flat
+# workload (dram__bytes_read.sum + dram__bytes_write.sum of the full launch
+# divided by the launch's far rows x Hkv):
+#   flat_128k      20.21 GB + 1.08 GB over 131072 x 2048 x 8 far rows (the
+#                  near-set tiles take sink and window; k_attn's reads include
+#                  the tiles' partial results);
+#   flat_1m        437.8 GB + 0.28 GB over 32768 x 4613 x 8 rows;
+#   flat_tree_10m  1.09 TB + 0.55 GB over 65536 x 4613 x 8 rows (at 1M and
+#                  10M a KV head does not fit in L2, the library keeps the
+#                  near set in the gather, and every listed row is a far row).
+# Re-measure when k_attn changes.
+ATTN_DRAM_BYTES_PER_FAR_ROW = {"flat_128k": 9.92, "flat_1m": 362.3, "flat_tree_10m": 450.8}
 
 
 def peaks():
@@ -156,11 +159,34 @@ def device_qkv(nq, n_kv, hq, hkv, seed=0, dev="cuda"):
     return Q, K, V
 
 
-def attn_algorithmic_bytes(lens: np.ndarray, hq: int, hkv: int) -> int:
-    """K and V rows of every listed (query, KV head, key) + Q read + O write +
-    the lists themselves."""
-    rows = int(lens.astype(np.int64).sum())
-    return rows * hkv * 2 * 256 + len(lens) * hq * 128 * 2 * 2 + rows * 4
+def near_split_rows(lists: torch.Tensor, lens: torch.Tensor, chunk: int = 4096):
+    """Per list, the rows the near-set tiles take -- the run of consecutive
+    positions that ends the list (at most 1024) and the run 0, 1, .. that
+    starts it (at most 16, disjoint from the first) -- as the attention's plan
+    finds them for a tile of consecutive queries (the bench's queries are
+    consecutive).  Returns (near rows, far rows) summed over the lists."""
+    nq, lmax = lists.shape
+    dev = lists.device
+    ar_d = torch.arange(1024, device=dev)
+    ar_s = torch.arange(min(16, lmax), device=dev)
+    near = far = 0
+    for c0 in range(0, nq, chunk):
+        lst = lists[c0:c0 + chunk].long()
+        n = lens[c0:c0 + chunk].long().clamp(max=lmax)
+        tail = torch.gather(lst, 1, (n[:, None] - 1 - ar_d[None, :]).clamp(min=0))
+        d = ((tail == tail[:, :1] - ar_d[None, :]) & (ar_d[None, :] < n[:, None])).int().cumprod(1).sum(1)
+        head = lst[:, :len(ar_s)]
+        s = ((head == ar_s[None, :]) & (ar_s[None, :] < (n - d)[:, None])).int().cumprod(1).sum(1)
+        near += int((s + d).sum())
+        far += int((n - s - d).sum())
+    return near, far
+
+
+def attn_algorithmic_bytes(far_rows: int, nq: int, hq: int, hkv: int) -> int:
+    """Gather kernel k_attn: K and V rows of every far (query, KV head, key)
+    + their list entries + Q read + O write + the near-set partial results
+    (fp32 O and max/sum per (query, head)) it merges."""
+    return far_rows * hkv * 2 * 256 + far_rows * 4 + nq * hq * 128 * 2 * 2 + nq * hq * 130 * 4
 
 
 def run_ours(args, world, rank, local):
@@ -205,6 +231,8 @@ def run_ours(args, world, rank, local):
     lens_np = layer.lens[:nq].cpu().numpy()
 
     launches0 = lsa.lsa_launch_count()
+    lsa.lsa_attention_timing_read()  # drop the warm-up calls' events
+    lsa.lsa_attention_timing(True)
     clk = Clocks(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -217,6 +245,8 @@ def run_ours(args, world, rank, local):
     clocks = clk.stop()
     barrier(world)
     launches = lsa.lsa_launch_count() - launches0
+    lsa.lsa_attention_timing(False)
+    near_ms, gather_ms, n_calls = lsa.lsa_attention_timing_read()
     per = np.array([[a.elapsed_time(b), b.elapsed_time(c), c.elapsed_time(d), a.elapsed_time(d)]
                     for a, b, c, d in times])
     total_ms = float(per[:, 3].sum())
@@ -224,19 +254,27 @@ def run_ours(args, world, rank, local):
     ms_step = total_ms / args.steps
     value = world * nq * args.steps / (total_ms / 1e3)
 
-    # roofline of the dominant kernel (attention: one k_attn launch per step)
+    # roofline of the dominant kernel: k_attn, the far-key gather (one launch
+    # per step), timed by the library's events around it on the step's stream
     pk = peaks()
-    attn_ms = float(per[:, 2].mean())
-    abytes = attn_algorithmic_bytes(lens_np, hq, hkv)
+    if near_ms > 0.0:  # the near-set tiles ran
+        near_rows, far_rows = near_split_rows(layer.lists[:nq], layer.lens[:nq])
+    else:
+        near_rows, far_rows = 0, int(lens_np.astype(np.int64).sum())
+    attn_ms = gather_ms / max(1, n_calls)
+    abytes = attn_algorithmic_bytes(far_rows, nq, hq, hkv)
     achieved = abytes / (attn_ms / 1e3) / 1e9
     traffic = None
-    per_row = ATTN_DRAM_BYTES_PER_ROW.get(args.workload) if wl["mode"] == "flat" else None
+    per_row = ATTN_DRAM_BYTES_PER_FAR_ROW.get(args.workload) if wl["mode"] == "flat" else None
     if per_row is not None:
-        traffic = int(per_row * int(lens_np.sum()) * hkv)
+        traffic = int(per_row * far_rows * hkv)
     roofline = {"kernel": "k_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
-                "peak_source": pk["src"], "algorithmic_bytes": abytes,
-                "traffic_note": "ncu DRAM bytes per listed row of this workload's launch, times its rows"}
+                "peak_source": pk["src"], "algorithmic_bytes": abytes, "launch_ms": round(attn_ms, 3),
+                "traffic_note": "ncu DRAM bytes per far row of this workload's launch, times its far rows",
+                "near": {"kernels": "k_near_plan + k_attn_near", "ms": round(near_ms / max(1, n_calls), 3),
+                         "rows_per_query": round(near_rows / nq, 1),
+                         "far_rows_per_query": round(far_rows / nq, 1)}}
     if traffic is not None:  # the same launch measured on the DRAM side: bytes that really crossed HBM
         roofline["dram_achieved"] = round(traffic / (attn_ms / 1e3) / 1e9, 1)
         roofline["dram_frac"] = round(traffic / (attn_ms / 1e3) / 1e9 / pk["hbm"], 4)
@@ -265,7 +303,7 @@ def run_ours(args, world, rank, local):
                    "mixture_components": wl["n_components"], "parallelism": "replicas",
                    "l2": "256 MiB buffer written between timed steps; K/V exceed L2"},
         "breakdown_ms": {"build": round(float(per[:, 0].mean()), 3), "index": round(float(per[:, 1].mean()), 3),
-                         "attention": round(attn_ms, 3)},
+                         "attention": round(float(per[:, 2].mean()), 3)},
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": int(launches),

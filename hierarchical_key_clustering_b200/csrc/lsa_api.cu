@@ -47,6 +47,13 @@ int sm_count()
     return n > 0 ? n : 148;
 }
 
+int64_t l2_bytes()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev);
+    return n > 0 ? n : (int64_t)126 << 20;
+}
+
 int check_params(const lsa_params *p)
 {
     if (!p) return fail(LSA_ERR_ARG, "params is NULL");
@@ -320,6 +327,23 @@ int lsa_check_device_errors(void)
     return v;
 }
 
+void lsa_attention_timing(int32_t enable)
+{
+    lsa::attention_timing(enable != 0);
+}
+
+int lsa_attention_timing_read(double *near_ms, double *gather_ms, int32_t *calls)
+{
+    double a = 0.0, b = 0.0;
+    int n = 0;
+    cudaError_t e = lsa::attention_timing_read(a, b, n);
+    if (near_ms) *near_ms = a;
+    if (gather_ms) *gather_ms = b;
+    if (calls) *calls = n;
+    if (e != cudaSuccess) return cuda_fail(e, "attention timing events");
+    return LSA_OK;
+}
+
 void lsa_debug_wait_test(int32_t enable)
 {
     g_extra_tx = enable ? 16u : 0u;
@@ -531,8 +555,14 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
     a.near_tile = nullptr;
     a.near_o = nullptr;
     a.near_ml = nullptr;
+    // The near-set tiles pay where the gather is bound by L2 throughput: when
+    // one KV head's K + V (Tk x 512 B) stays in L2 while its queries run, the
+    // window rows that every query re-reads cost as much as its far rows.
+    // Past that the gather is bound by HBM, where the re-read window rows are
+    // L2 hits that cost little, and the tiles would only add their own time.
     const int64_t nb = near_ws_bytes(nq, Hq);
-    if (nsplit == 1 && nb > 0 && lsa::near_tile_queries(Hq / Hkv) > 0 && ws && ws_bytes >= nb &&
+    const bool near_pays = Tk * 2 * LSA_HEAD_DIM * 2 <= l2_bytes() * 3 / 4;
+    if (nsplit == 1 && nb > 0 && near_pays && lsa::near_tile_queries(Hq / Hkv) > 0 && ws && ws_bytes >= nb &&
         ((uintptr_t)ws & 255u) == 0) {
         a.near_o = (float *)ws;
         a.near_ml = (float *)((char *)ws + align256(nq * Hq * (int64_t)LSA_HEAD_DIM * 4));

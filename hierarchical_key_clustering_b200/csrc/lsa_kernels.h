@@ -171,6 +171,8 @@ constexpr int NEAR_ROWS = 128;
 __host__ __device__ inline int near_tile_queries(int G) { return (G >= 1 && NEAR_ROWS % G == 0) ? NEAR_ROWS / G : 0; }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm);
+void attention_timing(bool on);
+cudaError_t attention_timing_read(double &near_ms, double &gather_ms, int &calls);
 int attention_list_cap();
 
 }  // namespace lsa

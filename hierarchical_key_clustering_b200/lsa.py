@@ -56,7 +56,7 @@ class lsa_tree(C.Structure):
 
 
 EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_check_device_errors",
-           "lsa_debug_wait_test", "lsa_list_budget", "lsa_top_buckets",
+           "lsa_debug_wait_test", "lsa_attention_timing", "lsa_attention_timing_read", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
            "lsa_build_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
@@ -88,6 +88,8 @@ def lib():
             "lsa_launch_count": (i64, []),
             "lsa_check_device_errors": (C.c_int, []),
             "lsa_debug_wait_test": (None, [i32]),
+            "lsa_attention_timing": (None, [i32]),
+            "lsa_attention_timing_read": (C.c_int, [C.POINTER(C.c_double), C.POINTER(C.c_double), C.POINTER(i32)]),
             "lsa_list_budget": (i32, [pp]),
             "lsa_top_buckets": (i32, [pp]),
             "lsa_cache_bytes": (i64, [i64]),
@@ -148,6 +150,18 @@ def lsa_default_params(**overrides) -> lsa_params:
 
 def lsa_launch_count() -> int:
     return lib().lsa_launch_count()
+
+
+def lsa_attention_timing(enable: bool) -> None:
+    """Record per-kernel CUDA events in every lsa_sparse_attention call (profiling aid)."""
+    lib().lsa_attention_timing(1 if enable else 0)
+
+
+def lsa_attention_timing_read():
+    """(near-set ms, gather ms, calls) summed since the last read; waits for the events."""
+    a, b, n = C.c_double(), C.c_double(), C.c_int32()
+    _check(lib().lsa_attention_timing_read(C.byref(a), C.byref(b), C.byref(n)))
+    return a.value, b.value, n.value
 
 
 def lsa_check_device_errors() -> int:

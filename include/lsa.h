@@ -159,6 +159,17 @@ int64_t lsa_launch_count(void);
 int lsa_check_device_errors(void);
 void lsa_debug_wait_test(int32_t enable);
 
+/* Per-kernel timing of lsa_sparse_attention, a profiling aid.  While enabled
+ * (lsa_attention_timing(1)), every call records three CUDA events on its own
+ * stream: before its near-set kernels (plan + dense tiles), between them and
+ * the gather kernel (with its split merge), and after; nothing else changes.
+ * lsa_attention_timing_read waits for the recorded events and returns the
+ * milliseconds summed over the calls since the last read (near set, 0 for a
+ * call that did not take it; gather) and their count, then forgets them.  Returns LSA_OK or LSA_ERR_CUDA.  Not
+ * thread-safe: enable, call and read from one host thread. */
+void lsa_attention_timing(int32_t enable);
+int lsa_attention_timing_read(double *near_ms, double *gather_ms, int32_t *calls);
+
 
 /* Longest index list: sink + window + 1 (the query itself) + k. */
 int32_t lsa_list_budget(const lsa_params *p);
@@ -249,8 +260,13 @@ int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const ls
  * (natural-log log-sum-exp of the scaled scores; may be NULL).
  * ws: >= lsa_attention_workspace_bytes(nq, Hq, 128, Lmax) bytes.  It holds
  * the partial results when few queries split their lists over many warps
- * (decode); with a smaller workspace (or none) fewer splits are used, with
- * the same results. */
+ * (decode), or, for batches of at least 64 queries whose KV head fits in
+ * three quarters of L2 (Tk x 512 B), the near-set results of tiles of
+ * consecutive queries: the run of consecutive positions that ends a list and
+ * the run 0, 1, .. that starts it are read once per tile and merged with the
+ * rest of each list by log-sum-exp.  With a smaller workspace (or none) fewer
+ * splits, or no tiles, are used; results are the same up to fp32 summation
+ * order. */
 int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t nq,
                          int32_t Hq, int32_t Hkv, int32_t head_dim, int64_t Tk, const int32_t *lists,
                          const int32_t *lens, int32_t Lmax, float scale, uint16_t *O, float *lse,
