@@ -50,17 +50,19 @@ class SparseLayer:
                                  stream=stream)
         return O
 
-    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int = 8):
+    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int = 16):
         """One prefill step whose inputs and output live in pinned host memory.
 
-        Three streams overlap the transfers with the kernels: the index
-        inputs go first and the cache build and index start as soon as they
-        land, while K and V follow; Q then arrives in query chunks (multiples
-        of 128 queries, so the near-set tiles of the attention do not change)
-        and each chunk's attention starts when its Q is on the device; each
-        chunk's O is copied back while the next chunks compute.  Every copy
-        and kernel of the call is ordered after the work already queued on
-        the current stream, and the current stream waits for the last copy
+        Three streams overlap the transfers with the kernels.  The index
+        inputs go first, and the cache build and index start as soon as they
+        land.  Q then arrives in query chunks (multiples of 128 queries, so
+        the near-set tiles of the attention do not change), each preceded by
+        the K and V rows its queries can list (positions up to the chunk's
+        largest query position; the rest of K and V follows the last chunk),
+        and each chunk's attention starts when its rows are on the device;
+        each chunk's O is copied back while the next chunks compute.  Every
+        copy and kernel of the call is ordered after the work already queued
+        on the current stream, and the current stream waits for the last copy
         back, so the call behaves as one stream-ordered step.  The results are
         those of build + index + attend on device copies of the inputs, up to
         the attention's summation order when a chunk holds so few (query, KV
@@ -78,31 +80,38 @@ class SparseLayer:
             self._dbuf = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hs]
             self._dbuf_key = key
         d_keys, d_q, d_pos, d_Q, d_K, d_V, d_O = self._dbuf
+        tk = h_K.shape[0]
         step = -(-nq // max(1, chunks))
         step = -(-step // 128) * 128
         bounds = [(c0, min(nq, c0 + step)) for c0 in range(0, nq, step)]
+        # K/V rows each chunk needs: its lists hold positions <= its largest query position
+        need = [min(tk, int(h_pos[c0:c1].max()) + 1) for c0, c1 in bounds]
         self._h2d.wait_stream(cs)
         with torch.cuda.stream(self._h2d):
             for d, h in ((d_keys, h_keys), (d_q, h_qidx), (d_pos, h_pos)):
                 d.copy_(h, non_blocking=True)
             e_idx = torch.cuda.Event()
             e_idx.record()
-            d_K.copy_(h_K, non_blocking=True)
-            d_V.copy_(h_V, non_blocking=True)
-            e_kv = torch.cuda.Event()
-            e_kv.record()
-            e_q = []
-            for c0, c1 in bounds:
+            e_in, have = [], 0
+            for (c0, c1), n in zip(bounds, need):
+                if n > have:
+                    d_K[have:n].copy_(h_K[have:n], non_blocking=True)
+                    d_V[have:n].copy_(h_V[have:n], non_blocking=True)
+                    have = n
                 d_Q[c0:c1].copy_(h_Q[c0:c1], non_blocking=True)
-                e_q.append(torch.cuda.Event())
-                e_q[-1].record()
+                e_in.append(torch.cuda.Event())
+                e_in[-1].record()
+            if have < tk:
+                d_K[have:].copy_(h_K[have:], non_blocking=True)
+                d_V[have:].copy_(h_V[have:], non_blocking=True)
+            e_all = torch.cuda.Event()
+            e_all.record()
         cs.wait_event(e_idx)
         self.build(d_keys, stream=cs)
         self.index(d_q, d_pos, stream=cs)
-        cs.wait_event(e_kv)
         e_o = []
-        for (c0, c1), eq in zip(bounds, e_q):
-            cs.wait_event(eq)
+        for (c0, c1), ei in zip(bounds, e_in):
+            cs.wait_event(ei)
             lsa.lsa_sparse_attention(d_Q[c0:c1], d_K, d_V, self.lists[c0:c1], self.lens[c0:c1], d_O[c0:c1],
                                      None if lse is None else lse[c0:c1], ws=self.ws_attn, stream=cs)
             e_o.append(torch.cuda.Event())
@@ -112,4 +121,5 @@ class SparseLayer:
                 self._d2h.wait_event(eo)
                 h_O[c0:c1].copy_(d_O[c0:c1], non_blocking=True)
         cs.wait_stream(self._d2h)
+        cs.wait_event(e_all)
         return h_O
