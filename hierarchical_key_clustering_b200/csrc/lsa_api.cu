@@ -422,6 +422,7 @@ int lsa_tree_bind(void *base, int64_t bytes, int64_t n_blocks, lsa_tree *out)
     int64_t size[LSA_MAX_LEVELS + 1], offset[LSA_MAX_LEVELS + 2];
     int L = tree_levels(n_blocks * LSA_BUCKETS, size, offset);
     out->n_blocks = 0;
+    out->cap_blocks = (int32_t)n_blocks;
     out->n_levels = L;
     for (int l = 0; l < L; ++l) {
         out->level_size[l] = size[l];
@@ -481,26 +482,50 @@ int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache
     return LSA_OK;
 }
 
-int lsa_build_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream)
+// Shared by lsa_build_tree and lsa_update_tree: the tree's level sizes for
+// the cache's blocks, its offsets fixed by the capacity it was bound for, and
+// the launches for the leaves from block b_first on and the runs above them.
+static int tree_grow(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, int64_t b_first, void *stream)
 {
     int rc = check_params(p);
     if (rc) return rc;
     if (!cache || !tree) return fail(LSA_ERR_ARG, "cache and tree must be non-NULL");
     if (cache->n_blocks < 1) return fail(LSA_ERR_SHAPE, "the cache has no complete block");
+    if (!tree->child || !tree->sum || tree->cap_blocks < 1)
+        return fail(LSA_ERR_ARG, "tree is not bound (lsa_tree_bind)");
+    if (cache->n_blocks > tree->cap_blocks)
+        return fail(LSA_ERR_SHAPE, "tree bound for %d blocks, the cache holds %lld", tree->cap_blocks,
+                    (long long)cache->n_blocks);
     int64_t size[LSA_MAX_LEVELS + 1], offset[LSA_MAX_LEVELS + 2];
-    int L = tree_levels(cache->n_blocks * LSA_BUCKETS, size, offset);
-    if (tree->n_levels < L || tree->level_offset[tree->n_levels] < offset[L] || !tree->child || !tree->sum)
-        return fail(LSA_ERR_SHAPE, "tree buffer bound for fewer blocks than the cache holds");
+    int64_t csize[LSA_MAX_LEVELS + 1], coff[LSA_MAX_LEVELS + 2];
+    const int L = tree_levels(cache->n_blocks * LSA_BUCKETS, size, offset);
+    const int LC = tree_levels((int64_t)tree->cap_blocks * LSA_BUCKETS, csize, coff);
+    if (L > LC) return fail(LSA_ERR_SHAPE, "tree levels exceed its capacity");
     tree->n_levels = L;
     for (int l = 0; l < LSA_MAX_LEVELS; ++l) tree->level_size[l] = l < L ? size[l] : 0;
-    for (int l = 0; l <= LSA_MAX_LEVELS; ++l) tree->level_offset[l] = l <= L ? offset[l] : offset[L];
+    for (int l = 0; l <= LSA_MAX_LEVELS; ++l) tree->level_offset[l] = l <= LC ? coff[l] : coff[LC];
     lsa::TreeDev td{tree->child, tree->parent, tree->weight, tree->min_block, tree->max_block,
                     tree->sum, tree->centroid, tree->centroid_bf16};
-    cudaError_t e = lsa::launch_tree(cache->pooled, cache->members, cache->count, size[0], td, size, offset, L,
-                                     (cudaStream_t)stream, sm_count());
+    cudaError_t e = lsa::launch_tree(cache->pooled, cache->members, cache->count, b_first * LSA_BUCKETS, size[0], td,
+                                     size, tree->level_offset, L, (cudaStream_t)stream, sm_count());
     if (e != cudaSuccess) return cuda_fail(e, "tree launch");
     tree->n_blocks = cache->n_blocks;
     return LSA_OK;
+}
+
+int lsa_build_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream)
+{
+    return tree_grow(cache, tree, p, 0, stream);
+}
+
+int lsa_update_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream)
+{
+    if (!cache || !tree) return fail(LSA_ERR_ARG, "cache and tree must be non-NULL");
+    if (cache->n_blocks < tree->n_blocks)
+        return fail(LSA_ERR_SHAPE, "the cache holds %lld blocks, fewer than the tree's %lld",
+                    (long long)cache->n_blocks, (long long)tree->n_blocks);
+    if (tree->n_blocks > 0 && cache->n_blocks == tree->n_blocks) return check_params(p);
+    return tree_grow(cache, tree, p, tree->n_blocks, stream);
 }
 
 int lsa_index_prefill(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache,

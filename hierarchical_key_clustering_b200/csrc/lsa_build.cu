@@ -320,13 +320,13 @@ __global__ void __launch_bounds__(128) k_ward(const float *__restrict__ pooled, 
 // ascending item order, weight = items, min/max block = its block.
 __global__ void __launch_bounds__(256) k_tree_leaves(const float *__restrict__ pooled,
                                                      const int32_t *__restrict__ members,
-                                                     const int32_t *__restrict__ count, int64_t nb,
-                                                     TreeDev tr)
+                                                     const int32_t *__restrict__ count, int64_t g_first,
+                                                     int64_t nb, TreeDev tr)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t g = warp; g < nb; g += nwarps) {
+    for (int64_t g = g_first + warp; g < nb; g += nwarps) {
         const int cnt = count[g];
         float sa = 0.0f, sb = 0.0f;
         for (int e = 0; e < cnt; e += LSA_NP) {
@@ -355,7 +355,8 @@ __global__ void __launch_bounds__(256) k_tree_leaves(const float *__restrict__ p
 // with mu = sum / w; repeatedly pair the cheapest two unpaired nodes (ties to
 // the lowest (i, j)).  New nodes (pairs at their lower member, lone leftover
 // as itself) are written in ascending order of that member.
-__global__ void __launch_bounds__(128) k_tree_pair(TreeDev tr, int64_t off_prev, int64_t n_prev, int64_t off)
+__global__ void __launch_bounds__(128) k_tree_pair(TreeDev tr, int64_t run0, int64_t off_prev, int64_t n_prev,
+                                                   int64_t off)
 {
     extern __shared__ float smem[];
     float *Y = smem;
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(128) k_tree_pair(TreeDev tr, int64_t off_prev,
     __shared__ int warp_cnt[4];
 
     const int t = threadIdx.x;
-    const int64_t first = (int64_t)blockIdx.x * LSA_RUN;
+    const int64_t first = (run0 + blockIdx.x) * LSA_RUN;
     const int m = (int)min((int64_t)LSA_RUN, n_prev - first);
     const int64_t base = off_prev + first;
     if (t < m) w_s[t] = tr.weight[base + t];
@@ -527,26 +528,35 @@ cudaError_t launch_ward(const float *pooled, int64_t blk_begin, int64_t blk_end,
     return cudaGetLastError();
 }
 
-cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32_t *count, int64_t nb,
-                        const TreeDev &tr, const int64_t *level_size, const int64_t *level_offset, int n_levels,
-                        cudaStream_t st, int n_sm)
+cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32_t *count, int64_t g_first,
+                        int64_t nb, const TreeDev &tr, const int64_t *level_size, const int64_t *level_offset,
+                        int n_levels, cudaStream_t st, int n_sm)
 {
     cudaError_t e = cudaFuncSetAttribute(k_tree_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WARD_SMEM);
     if (e != cudaSuccess) return e;
-    int64_t blocks = (nb + 7) / 8;
+    int64_t blocks = (nb - g_first + 7) / 8;
     if (blocks > (int64_t)n_sm * 16) blocks = (int64_t)n_sm * 16;
     if (blocks < 1) blocks = 1;
-    k_tree_leaves<<<(unsigned)blocks, 256, 0, st>>>(pooled, members, count, nb, tr);
+    k_tree_leaves<<<(unsigned)blocks, 256, 0, st>>>(pooled, members, count, g_first, nb, tr);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    // a run of 128 nodes is paired from its own nodes alone, and every run
+    // but a level's last is full (its 64 parents start at 64 x its index):
+    // only the runs from the first changed node on change, level by level
+    int64_t changed = g_first;
     for (int l = 1; l < n_levels; ++l) {
-        int64_t n_prev = level_size[l - 1];
-        int64_t runs = (n_prev + LSA_RUN - 1) / LSA_RUN;
-        k_tree_pair<<<(unsigned)runs, 128, WARD_SMEM, st>>>(tr, level_offset[l - 1], n_prev, level_offset[l]);
-        count_launches(1);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+        const int64_t n_prev = level_size[l - 1];
+        const int64_t runs = (n_prev + LSA_RUN - 1) / LSA_RUN;
+        const int64_t run0 = changed / LSA_RUN;
+        if (runs > run0) {
+            k_tree_pair<<<(unsigned)(runs - run0), 128, WARD_SMEM, st>>>(tr, run0, level_offset[l - 1], n_prev,
+                                                                        level_offset[l]);
+            count_launches(1);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        changed = run0 * (LSA_RUN / 2);
     }
     return cudaSuccess;
 }

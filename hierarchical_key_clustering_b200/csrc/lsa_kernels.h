@@ -101,9 +101,11 @@ cudaError_t launch_pool_norm(const float *keys, int64_t item_begin, int64_t item
 cudaError_t launch_ward(const float *pooled, int64_t blk_begin, int64_t blk_end, int cap, uint8_t *item_bucket,
                         int32_t *members, int32_t *count, float *centroid, uint16_t *centroid_bf16,
                         cudaStream_t st);
-cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32_t *count, int64_t nb,
-                        const TreeDev &tr, const int64_t *level_size, const int64_t *level_offset, int n_levels,
-                        cudaStream_t st, int n_sm);
+// Leaves from bucket g_first on (g_first = 0: the whole tree) and, level by
+// level, the runs of 128 nodes from the first changed node on.
+cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32_t *count, int64_t g_first,
+                        int64_t nb, const TreeDev &tr, const int64_t *level_size, const int64_t *level_offset,
+                        int n_levels, cudaStream_t st, int n_sm);
 
 struct IndexArgs {
     const float *qidx;

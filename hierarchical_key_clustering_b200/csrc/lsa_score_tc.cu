@@ -44,6 +44,7 @@
 
 #include "lsa_common.cuh"
 #include "lsa_kernels.h"
+#include "lsa_tc.cuh"
 
 namespace lsa {
 
@@ -66,124 +67,32 @@ constexpr int HSTRIDE = HIST_BINS / 2 + 1;   // 32-bit words per row histogram (
 constexpr uint32_t HIST_BYTES = QT * TQ * HSTRIDE * 4;
 constexpr uint32_t ROWCNT_BYTES = QT * TQ * 4;  // per-row entry counters of the filter pass
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
+using tc::mbar_arrive;
+using tc::mbar_expect_tx;
+using tc::mbar_init;
+using tc::smem_desc;
+using tc::smem_u32;
+using tc::tma_load_2d;
+using tc::tmem_ld32_nowait;
+using tc::tmem_wait_ld;
+using tc::mma_commit;
 
 // Bounded wait; on expiry sets the device error word and the CTA abort flag.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit, volatile int *abort)
 {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort) return false;
-    }
-    atomicExch(&g_device_error, 1);
-    *abort = 1;
-    return false;
+    return tc::wait_bounded(bar, parity, limit, abort, &g_device_error);
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
-            "r"(dst),
-        "l"(map), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 B,
-// 8-row groups 1024 B apart (sm_100 descriptor format, version 1).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr)
-{
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3fffu);          // start address
-    d |= (uint64_t)1 << 16;                           // leading byte offset (unused for SW128 K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset
-    d |= (uint64_t)1 << 46;                           // descriptor version
-    d |= (uint64_t)2 << 61;                           // SWIZZLE_128B
-    return d;
-}
-
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
-// N = 128, M = 128.
-constexpr uint32_t IDESC = (1u << 4)               // D format fp32
-                           | (1u << 7)             // A bf16
-                           | (1u << 10)            // B bf16
-                           | ((uint32_t)(TB >> 3) << 17)
-                           | ((uint32_t)(TQ >> 4) << 24);
+// kind::f16: D fp32, A and B bf16, both K-major, N = 128, M = 128.
+constexpr uint32_t IDESC = tc::idesc_bf16(TQ, TB);
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
 {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
-        : "memory");
+    tc::mma_bf16(tmem_d, adesc, bdesc, IDESC, accumulate);
 }
 
-__device__ __forceinline__ void mma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before()
-{
-    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after()
-{
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-
-// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (no wait).
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float *v)
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_wait_ld()
-{
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
+__device__ __forceinline__ void tc_fence_before() { tc::fence_before(); }
+__device__ __forceinline__ void tc_fence_after() { tc::fence_after(); }
 
 __device__ __forceinline__ float max3f(float a, float b, float c)
 {
@@ -497,11 +406,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 // ---------------------------------------------------------------------------
 // Host side: tensor maps and launch.
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
+EncodeTiledFn tensor_map_encoder()
 {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
@@ -518,7 +423,7 @@ static EncodeTiledFn encode_fn()
 // end read as zero.
 static bool make_map(CUtensorMap *m, const void *base, int64_t rows, int box_rows)
 {
-    EncodeTiledFn fn = encode_fn();
+    EncodeTiledFn fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)LSA_D, (cuuint64_t)(rows > 0 ? rows : 1)};
     cuuint64_t strides[1] = {(cuuint64_t)LSA_D * 2};

@@ -37,6 +37,14 @@ class SparseLayer:
         if self.tree is not None:
             lsa.lsa_build_tree(self.cache, self.tree, self.p, stream)
 
+    def append(self, keys: torch.Tensor, t_begin: int, t_end: int, stream=None):
+        """Grow the cache with the index keys of positions t_begin..t_end-1
+        (keys holds positions 0..t_end-1): items and blocks that complete are
+        pooled and clustered, and the tree, if any, is extended in place."""
+        lsa.lsa_build_cache(keys, t_begin, t_end, self.cache, self.p, stream)
+        if self.tree is not None and self.cache.n_blocks > 0:
+            lsa.lsa_update_tree(self.cache, self.tree, self.p, stream)
+
     def index(self, qidx: torch.Tensor, pos: torch.Tensor, decode: bool = False, stream=None):
         nq = qidx.shape[0]
         assert nq <= self.max_queries

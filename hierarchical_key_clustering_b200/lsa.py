@@ -48,7 +48,7 @@ class lsa_cache(C.Structure):
 
 
 class lsa_tree(C.Structure):
-    _fields_ = [("n_blocks", C.c_int64), ("n_levels", C.c_int32), ("reserved", C.c_int32),
+    _fields_ = [("n_blocks", C.c_int64), ("n_levels", C.c_int32), ("cap_blocks", C.c_int32),
                 ("level_size", C.c_int64 * MAX_LEVELS), ("level_offset", C.c_int64 * (MAX_LEVELS + 1)),
                 ("child", C.c_void_p), ("parent", C.c_void_p), ("weight", C.c_void_p),
                 ("min_block", C.c_void_p), ("max_block", C.c_void_p), ("sum", C.c_void_p),
@@ -59,7 +59,7 @@ EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "l
            "lsa_debug_wait_test", "lsa_attention_timing", "lsa_attention_timing_read", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
-           "lsa_build_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
+           "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
            "lsa_index_decode_static"]
 
 _lib = None
@@ -100,6 +100,7 @@ def lib():
             "lsa_attention_workspace_bytes": (i64, [i64, i32, i32, i32]),
             "lsa_build_cache": (C.c_int, [P, i64, i64, pc, pp, P]),
             "lsa_build_tree": (C.c_int, [pc, pt, pp, P]),
+            "lsa_update_tree": (C.c_int, [pc, pt, pp, P]),
             "lsa_index_prefill": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P, i64, P]),
             "lsa_index_decode": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P, i64, P]),
             "lsa_index_decode_static": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P]),
@@ -277,6 +278,10 @@ def lsa_build_cache(keys: torch.Tensor, t_begin: int, t_end: int, cache: Cache, 
 
 def lsa_build_tree(cache: Cache, tree: Tree, p: lsa_params, stream=None):
     _check(lib().lsa_build_tree(C.byref(cache.c), C.byref(tree.t), C.byref(p), _stream(stream)))
+
+
+def lsa_update_tree(cache: Cache, tree: Tree, p: lsa_params, stream=None):
+    _check(lib().lsa_update_tree(C.byref(cache.c), C.byref(tree.t), C.byref(p), _stream(stream)))
 
 
 def _index(fn, qidx, pos, cache, tree, lists, lens, p, ws, stream):

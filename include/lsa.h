@@ -116,11 +116,13 @@ typedef struct lsa_cache {
  *   items below), min_block / max_block [n], sum fp32 [n,64] (sum of the
  *   leaves' pooled keys), centroid fp32 [n,64] = normalise(sum),
  *   centroid_bf16 [n,64].
- * Fill with lsa_tree_bind; lsa_build_tree sets n_blocks. */
+ * Fill with lsa_tree_bind, which lays the levels out for its capacity
+ * (level_offset fixed, level_size growing with the cache), so that a tree can
+ * grow in place; lsa_build_tree / lsa_update_tree set n_blocks. */
 typedef struct lsa_tree {
     int64_t n_blocks;
     int32_t n_levels;
-    int32_t reserved;
+    int32_t cap_blocks; /* capacity the buffer was bound for; level_offset is laid out for it */
     int64_t level_size[LSA_MAX_LEVELS];
     int64_t level_offset[LSA_MAX_LEVELS + 1];
     int32_t *child;
@@ -218,6 +220,17 @@ int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache
  * odd leftover is promoted alone; new nodes are ordered by their lower
  * child; repeat until one root.  tree must be bound for >= cache->n_blocks. */
 int lsa_build_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream);
+
+/* Grow a tree built over tree->n_blocks blocks to cache->n_blocks blocks
+ * (decode: a block completes every 512 tokens; [EXPL] "How the hierarchy is
+ * built": the clusters are made as the context grows).  The pairing of a run
+ * of 128 nodes depends on that run alone, and every run but a level's last is
+ * full, so new leaves change only the runs from the first new node on at
+ * each level: those are paired again and everything else is kept.  The
+ * result is bit-identical to lsa_build_tree over the same cache.  A tree
+ * with n_blocks == 0 is built whole; cache->n_blocks < tree->n_blocks, or
+ * more blocks than the tree was bound for, returns LSA_ERR_SHAPE. */
+int lsa_update_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p, void *stream);
 
 /* Steps 3-5 for nq queries ([EXPL] "What one query actually does"; [BLOG]
  * steps 3-5 and read_list).

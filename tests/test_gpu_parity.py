@@ -144,6 +144,51 @@ def test_tree_build_bit_exact(tiny):
     assert np.array_equal(v["centroid_bf16"].view(np.uint16), ot.centroid_bf16)
 
 
+def _assert_tree_levels_equal(tree, ot):
+    """Level by level (the GPU tree is laid out for its capacity, the
+    oracle's compactly): every node array bit-exact, centroids within 1e-6."""
+    assert tree.level_sizes() == ot.level_size.tolist()
+    v = {k: t.cpu().numpy() for k, t in tree.views().items()}
+    for l, n in enumerate(tree.level_sizes()):
+        g0, o0 = tree.t.level_offset[l], int(ot.level_offset[l])
+        for name in ("child", "parent", "weight", "min_block", "max_block"):
+            assert np.array_equal(v[name][g0:g0 + n], getattr(ot, name)[o0:o0 + n]), f"level {l} {name} differs"
+        assert np.array_equal(v["sum"][g0:g0 + n].view(np.uint32), ot.sum[o0:o0 + n].view(np.uint32))
+        assert np.max(np.abs(v["centroid"][g0:g0 + n] - ot.centroid[o0:o0 + n])) <= 1e-6
+        assert np.array_equal(v["centroid_bf16"][g0:g0 + n].view(np.uint16), ot.centroid_bf16[o0:o0 + n])
+
+
+def test_tree_grows_in_place_as_blocks_complete(tiny):
+    """Decode-time growth: the cache takes new keys (ragged steps included),
+    and after each step the tree, extended by lsa_update_tree in a buffer laid
+    out for 8 blocks, equals the oracle's tree over the same prefix and a full
+    rebuild; the index over it matches the oracle's Tree lists."""
+    _need_gpu()
+    keys, q, pos, _ = tiny
+    p = lsa.lsa_default_params(k=256, mode="tree", beam=32)
+    cache, tree, full = lsa.Cache(4096), lsa.Tree(8), lsa.Tree(8)
+    kd = PT.to_dev(keys)
+    t = 0
+    for t_end in (1536, 2048, 2748, 3072, 3584, 4096):
+        lsa.lsa_build_cache(kd, t, t_end, cache, p)
+        lsa.lsa_update_tree(cache, tree, p)
+        t = t_end
+        torch.cuda.synchronize()
+        ot = O.build_tree(O.build_cache(keys[:t_end]))
+        _assert_tree_levels_equal(tree, ot)
+        lsa.lsa_build_tree(cache, full, p)
+        torch.cuda.synchronize()
+        va, vb = tree.views(), full.views()
+        for l, n in enumerate(tree.level_sizes()):  # the nodes in use (the rest of the buffer is never written)
+            g0 = tree.t.level_offset[l]
+            assert all(torch.equal(va[k][g0:g0 + n], vb[k][g0:g0 + n]) for k in va), f"level {l} differs"
+    oc = O.build_cache(keys)
+    sel = np.arange(1000, 4096, 37)
+    gl, gn = _index_gpu(cache, tree, p, q[sel], pos[sel])
+    ol, on = O.index(q[sel], pos[sel], oc, k=256, mode="tree", tree=O.build_tree(oc), beam=32)
+    PT.assert_lists_match(gl, gn, ol, on, q[sel], pos[sel], oc, k=256, tree=O.build_tree(oc), beam=32)
+
+
 @pytest.mark.parametrize("beam", [32, 4, 512])
 def test_tree_index_tiny(tiny, beam):
     keys, q, pos, oc = tiny

@@ -67,7 +67,29 @@ def test_tree_layout_levels():
         assert sizes[0] == nb and sizes[-1] == 1
         assert all(sizes[i + 1] == (sizes[i] + 1) // 2 for i in range(len(sizes) - 1))
         assert t.level_offset[t.n_levels] == sum(sizes)
+        assert t.cap_blocks == nblk and t.n_blocks == 0
     assert lsa.lib().lsa_tree_bytes(2048) > 0
+
+
+def test_update_tree_argument_errors():
+    """Host-side checks of lsa_update_tree (no GPU work is reached)."""
+    L = lsa.lib()
+    p = lsa.lsa_default_params(mode="tree")
+    cache, tree = lsa.lsa_cache(), lsa.lsa_tree()
+    _expect(L.lsa_cache_bind(FAKE, L.lsa_cache_bytes(8192), 8192, C.byref(cache)), 0)
+    _expect(L.lsa_tree_bind(FAKE, L.lsa_tree_bytes(8), 8, C.byref(tree)), 0)
+    _expect(L.lsa_update_tree(None, C.byref(tree), C.byref(p), None), -1)
+    cache.n_blocks = 0
+    _expect(L.lsa_update_tree(C.byref(cache), C.byref(tree), C.byref(p), None), -2)  # no complete block
+    cache.n_blocks = 16
+    _expect(L.lsa_update_tree(C.byref(cache), C.byref(tree), C.byref(p), None), -2)  # more than the tree holds
+    cache.n_blocks, tree.n_blocks = 3, 5
+    _expect(L.lsa_update_tree(C.byref(cache), C.byref(tree), C.byref(p), None), -2)  # cache behind the tree
+    cache.n_blocks = 5
+    _expect(L.lsa_update_tree(C.byref(cache), C.byref(tree), C.byref(p), None), 0)  # nothing new: no work
+    unbound = lsa.lsa_tree()
+    cache.n_blocks = 2
+    _expect(L.lsa_update_tree(C.byref(cache), C.byref(unbound), C.byref(p), None), -1)
 
 
 def _expect(code, want):
