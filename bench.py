@@ -419,10 +419,43 @@ def run_decode(args, dev, workload="flat_1m", mode="flat"):
         graph_us = e0.elapsed_time(e1) * 1e3 / nd
     except Exception as ex:  # report, keep the eager number
         note = f"graph capture failed: {type(ex).__name__}: {ex}"[:200]
+    # a block completes every 512 decode tokens: pool and cluster it and grow
+    # the tree in place (the cache and tree are rewound to T - 512 each time,
+    # re-running a range rewrites identical values); a full tree rebuild for
+    # comparison
+    keys_d = torch.from_numpy(keys_all[:T]).to(dev)
+    nb = T // 512
+    app = []
+    for r in range(6):
+        layer.cache.c.n_blocks = nb - 1
+        if layer.tree is not None:
+            layer.tree.t.n_blocks = nb - 1
+        e0, e1 = ev(), ev()
+        e0.record()
+        layer.append(keys_d, T - 512, T)
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 2:
+            app.append(e0.elapsed_time(e1) * 1e3)
+    rebuild_us = None
+    if layer.tree is not None:
+        reb = []
+        for r in range(4):
+            e0, e1 = ev(), ev()
+            e0.record()
+            lsa.lsa_build_tree(layer.cache, layer.tree, layer.p)
+            e1.record()
+            torch.cuda.synchronize()
+            if r >= 1:
+                reb.append(e0.elapsed_time(e1) * 1e3)
+        rebuild_us = round(float(np.median(reb)), 1)
     out = {"workload": workload, "mode": mode, "T": T, "tokens": nd, "k": wl["k"], "list_len": lens,
            "us_per_token": round(graph_us if graph_us is not None else eager_us, 2),
            "us_per_token_eager": round(eager_us, 2),
-           "note": "batch 1; lsa_index_decode + lsa_sparse_attention per token, replayed from one CUDA graph"}
+           "block_append_us": round(float(np.median(app)), 1), "tree_rebuild_us": rebuild_us,
+           "note": "batch 1; lsa_index_decode + lsa_sparse_attention per token, replayed from one CUDA graph; "
+                   "block_append_us: pool + cluster one completed block and grow the tree in place (every 512 "
+                   "tokens)"}
     if note:
         out["note"] = note
     return out
