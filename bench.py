@@ -189,6 +189,35 @@ def attn_algorithmic_bytes(far_rows: int, nq: int, hq: int, hkv: int) -> int:
     return far_rows * hkv * 2 * 256 + far_rows * 4 + nq * hq * 128 * 2 * 2 + nq * hq * 130 * 4
 
 
+def measure_shrink(K: torch.Tensor, dev, hbm_peak: float):
+    """Step 1 ("Shrink") on its own, outside the timed step: every position's
+    key over all KV heads (D = Hkv x 128, the workload's K as [T, D]) projected
+    by a synthetic bf16 W [64, D] and pooled straight into cache items (the
+    fused tensor-core kernel); HBM-bound on reading K."""
+    T = K.shape[0]
+    V = K.reshape(T, -1)
+    D = V.shape[1]
+    g = torch.Generator(device=dev)
+    g.manual_seed(64)
+    W = (torch.randn((64, D), generator=g, device=dev) / D ** 0.5).to(torch.bfloat16)
+    pooled = torch.empty((T // 4, 64), dtype=torch.float32, device=dev)
+    ts = []
+    for r in range(6):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lsa.lsa_shrink(V, W, 0, T, pooled=pooled)
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 2:
+            ts.append(e0.elapsed_time(e1))
+    ms = float(np.median(ts))
+    nbytes = T * D * 2 + (T // 4) * 64 * 4 + 64 * D * 2
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": "k_shrink", "T": T, "D": D, "ms": round(ms, 3), "bytes": nbytes,
+            "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4), "bound": "hbm",
+            "flop": 2 * T * D * 64}
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -278,6 +307,8 @@ def run_ours(args, world, rank, local):
     if traffic is not None:  # the same launch measured on the DRAM side: bytes that really crossed HBM
         roofline["dram_achieved"] = round(traffic / (attn_ms / 1e3) / 1e9, 1)
         roofline["dram_frac"] = round(traffic / (attn_ms / 1e3) / 1e9 / pk["hbm"], 4)
+
+    roofline["shrink"] = measure_shrink(K, dev, pk["hbm"])
 
     # end to end: same calls, inputs from pinned host memory, output back to host
     e2e = None if args.no_e2e else run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)

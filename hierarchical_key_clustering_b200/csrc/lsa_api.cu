@@ -467,13 +467,13 @@ int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache
     const int64_t i0 = t_begin / LSA_N_POOL, i1 = t_end / LSA_N_POOL;
     const int64_t b0 = t_begin / LSA_BLOCK, b1 = t_end / LSA_BLOCK;
     if (i1 > i0 || b1 > b0) {
-        if (!keys || !aligned16(keys)) return fail(LSA_ERR_ARG, "keys must be non-NULL and 16-byte aligned");
+        if (keys && !aligned16(keys)) return fail(LSA_ERR_ARG, "keys must be 16-byte aligned");
         if (!cache->pooled || !cache->item_bucket || !cache->members || !cache->count || !cache->centroid ||
             !cache->centroid_bf16)
             return fail(LSA_ERR_ARG, "cache arrays are NULL (bind the cache first)");
     }
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = lsa::launch_pool_norm(keys, i0, i1, cache->pooled, st, sm_count());
+    cudaError_t e = keys ? lsa::launch_pool_norm(keys, i0, i1, cache->pooled, st, sm_count()) : cudaSuccess;
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
     e = lsa::launch_ward(cache->pooled, b0, b1, p->cap_items, cache->item_bucket, cache->members, cache->count,
                          cache->centroid, cache->centroid_bf16, st);
@@ -510,6 +510,30 @@ static int tree_grow(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p
                                      size, tree->level_offset, L, (cudaStream_t)stream, sm_count());
     if (e != cudaSuccess) return cuda_fail(e, "tree launch");
     tree->n_blocks = cache->n_blocks;
+    return LSA_OK;
+}
+
+int lsa_shrink(const uint16_t *V, int64_t D, const uint16_t *W, int64_t t_begin, int64_t t_end, float *keys,
+               float *pooled, void *stream)
+{
+    if (!V || !W) return fail(LSA_ERR_ARG, "V and W must be non-NULL");
+    if (!keys && !pooled) return fail(LSA_ERR_ARG, "keys and pooled are both NULL");
+    if (D < 64 || D % 64 != 0 || D > 16384) return fail(LSA_ERR_SHAPE, "D = %lld must be a multiple of 64 <= 16384",
+                                                        (long long)D);
+    if (t_begin < 0 || t_end < t_begin) return fail(LSA_ERR_SHAPE, "need 0 <= t_begin <= t_end");
+    if (pooled && t_begin % LSA_N_POOL != 0) return fail(LSA_ERR_SHAPE, "pooled output needs t_begin %% 4 == 0");
+    if (!aligned16(V) || !aligned16(W) || (keys && !aligned16(keys)) || (pooled && !aligned16(pooled)))
+        return fail(LSA_ERR_ARG, "V, W, keys and pooled must be 16-byte aligned");
+    if (t_end == t_begin) return LSA_OK;
+    lsa::ShrinkArgs a;
+    a.t_begin = t_begin;
+    a.t_end = t_end;
+    a.D = D;
+    a.keys = keys;
+    a.pooled = pooled;
+    a.wait_limit = g_wait_limit;
+    cudaError_t e = lsa::launch_shrink(V, W, a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
     return LSA_OK;
 }
 

@@ -141,6 +141,17 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
                             int n_sm, int *whole_range);
 int read_device_error(int clear);
 
+// Step 1, "Shrink": x_t = W v_t for t in [t_begin, t_end), optional fp32
+// keys [T, 64] and pooled items (t_begin % 4 == 0).
+struct ShrinkArgs {
+    int64_t t_begin, t_end, D;
+    float *keys;
+    float *pooled;
+    uint32_t wait_limit;
+};
+cudaError_t launch_shrink(const uint16_t *V, const uint16_t *W, const ShrinkArgs &a, cudaStream_t st);
+int read_shrink_error(int clear);
+
 cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *tree, cudaStream_t st, int n_sm);
 // Shared memory the expansion kernel needs for `cap` candidates over a cache
 // of n_blocks blocks.

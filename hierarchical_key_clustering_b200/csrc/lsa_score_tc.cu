@@ -473,7 +473,9 @@ int read_device_error(int clear)
         int z = 0;
         cudaMemcpyToSymbol(g_device_error, &z, sizeof(int));
     }
-    return v;
+    const int w = read_shrink_error(clear);  // the projection kernel's own word
+    if (w < 0) return -1;
+    return v | w;
 }
 
 }  // namespace lsa

@@ -37,6 +37,20 @@ class SparseLayer:
         if self.tree is not None:
             lsa.lsa_build_tree(self.cache, self.tree, self.p, stream)
 
+    def build_from_rows(self, V: torch.Tensor, W: torch.Tensor, t_begin: int = 0, t_end: int | None = None,
+                        stream=None):
+        """Build (or grow) the cache from model rows instead of index keys:
+        each row of V (bf16 [T, D], e.g. a position's key over all KV heads)
+        is projected by W (bf16 [64, D]) and pooled straight into the cache
+        (one fused tensor-core kernel), then the completed blocks are
+        clustered and the tree, if any, grown.  t_begin must be a multiple
+        of 4."""
+        t_end = V.shape[0] if t_end is None else t_end
+        lsa.lsa_shrink(V, W, t_begin, t_end, cache=self.cache, stream=stream)
+        lsa.lsa_build_cache(None, t_begin, t_end, self.cache, self.p, stream)
+        if self.tree is not None and self.cache.n_blocks > 0:
+            lsa.lsa_update_tree(self.cache, self.tree, self.p, stream)
+
     def append(self, keys: torch.Tensor, t_begin: int, t_end: int, stream=None):
         """Grow the cache with the index keys of positions t_begin..t_end-1
         (keys holds positions 0..t_end-1): items and blocks that complete are
@@ -92,6 +106,14 @@ class SparseLayer:
         step = -(-nq // max(1, chunks))
         step = -(-step // 128) * 128
         bounds = [(c0, min(nq, c0 + step)) for c0 in range(0, nq, step)]
+        # the last chunk's copy back is the only one nothing overlaps: split it
+        # into quarters (multiples of 128 queries) to shorten that tail, when
+        # each quarter still has the (query, KV head) units that keep its
+        # attention on whole lists (2048)
+        c0, c1 = bounds[-1]
+        q4 = -(-((c1 - c0) // 4) // 128) * 128
+        if len(bounds) > 1 and q4 >= 128 and q4 * h_K.shape[1] >= 2048:
+            bounds = bounds[:-1] + [(a, min(c1, a + q4)) for a in range(c0, c1, q4)]
         # K/V rows each chunk needs: its lists hold positions <= its largest query position
         need = [min(tk, int(h_pos[c0:c1].max()) + 1) for c0, c1 in bounds]
         self._h2d.wait_stream(cs)

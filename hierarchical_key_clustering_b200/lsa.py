@@ -59,7 +59,7 @@ EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "l
            "lsa_debug_wait_test", "lsa_attention_timing", "lsa_attention_timing_read", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
-           "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
+           "lsa_shrink", "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
            "lsa_index_decode_static"]
 
 _lib = None
@@ -99,6 +99,7 @@ def lib():
             "lsa_index_workspace_bytes": (i64, [i64, i64, pp]),
             "lsa_attention_workspace_bytes": (i64, [i64, i32, i32, i32]),
             "lsa_build_cache": (C.c_int, [P, i64, i64, pc, pp, P]),
+            "lsa_shrink": (C.c_int, [P, i64, P, i64, i64, P, P, P]),
             "lsa_build_tree": (C.c_int, [pc, pt, pp, P]),
             "lsa_update_tree": (C.c_int, [pc, pt, pp, P]),
             "lsa_index_prefill": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P, i64, P]),
@@ -274,6 +275,20 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 def lsa_build_cache(keys: torch.Tensor, t_begin: int, t_end: int, cache: Cache, p: lsa_params, stream=None):
     _check(lib().lsa_build_cache(_ptr(keys), t_begin, t_end, C.byref(cache.c), C.byref(p), _stream(stream)))
+
+
+def lsa_shrink(V: torch.Tensor, W: torch.Tensor, t_begin: int, t_end: int, keys=None, pooled=None, cache=None,
+               stream=None):
+    """x_t = W v_t for rows t_begin..t_end-1 of V (bf16 [T, D]) with W (bf16
+    [64, D]); keys: fp32 [T, 64] output (optional); pooled: fp32 [T/4, 64]
+    output, or the cache whose pooled items to write (optional)."""
+    if V.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise ValueError("V and W must be bfloat16")
+    D = V.shape[1]
+    if tuple(W.shape) != (64, D):
+        raise ValueError(f"W must be [64, {D}]")
+    pp_ = C.c_void_p(cache.c.pooled) if cache is not None else _ptr(pooled)
+    _check(lib().lsa_shrink(_ptr(V), D, _ptr(W), t_begin, t_end, _ptr(keys), pp_, _stream(stream)))
 
 
 def lsa_build_tree(cache: Cache, tree: Tree, p: lsa_params, stream=None):

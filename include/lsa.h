@@ -197,6 +197,23 @@ int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, 
 
 /* ---- the five calls of the hot path ---- */
 
+/* Step 1, "Shrink" ([BLOG] "The same steps in general", step 1: each key is
+ * projected to 64 numbers that exist only for choosing; [FORUM] "Key
+ * points": D-LSA learns the projection, a PCA of the keys does nearly as
+ * well).  x_t = W v_t for every row t_begin <= t < t_end of V, fp32
+ * accumulation on the tensor cores.
+ * V bf16 [>= t_end, D] (a position's row, e.g. its key over all KV heads,
+ * D = Hkv x 128); W bf16 [64, D]; D a multiple of 64, <= 16384; V and W
+ * 16-byte aligned.
+ * keys (nullable) fp32 [>= t_end, 64]: x_t written at row t.
+ * pooled (nullable) fp32 [>= t_end / 4, 64]: item j = sum of the normalised
+ * x_4j .. x_4j+3, normalised and summed in the order lsa_build_cache uses,
+ * for every item whose four rows lie in the range (t_begin % 4 == 0 then);
+ * pass cache->pooled and then lsa_build_cache with keys = NULL to cluster
+ * the completed blocks.  At least one of keys, pooled must be non-NULL. */
+int lsa_shrink(const uint16_t *V, int64_t D, const uint16_t *W, int64_t t_begin, int64_t t_end, float *keys,
+               float *pooled, void *stream);
+
 /* Steps 1-2 of the indexer ([EXPL] "How the hierarchy is built"; [FORUM]
  * Key points; [BLOG] step 2).
  * keys: fp32 [>= t_end, 64], the index keys of positions 0..t_end-1.
@@ -209,7 +226,9 @@ int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, 
  * 64 buckets remain.  All fp32 arithmetic of this call follows one fixed
  * order, so results are bit-for-bit reproducible.
  * Re-running over a range rewrites identical values.  Requires
- * t_end <= cache->capacity.  Sets cache->n_blocks = max(n_blocks, t_end/512). */
+ * t_end <= cache->capacity.  Sets cache->n_blocks = max(n_blocks, t_end/512).
+ * keys = NULL skips the pooling: the range's items are already in
+ * cache->pooled (written by lsa_shrink), and only the blocks are clustered. */
 int lsa_build_cache(const float *keys, int64_t t_begin, int64_t t_end, lsa_cache *cache,
                     const lsa_params *p, void *stream);
 

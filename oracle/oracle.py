@@ -125,6 +125,17 @@ def normalize(x: np.ndarray) -> np.ndarray:
 
 # ---- build path -----------------------------------------------------------
 
+def shrink(Vb: np.ndarray, Wb: np.ndarray) -> np.ndarray:
+    """Step 1, "Shrink" (sotaaz blog, "The same steps in general", step 1;
+    zhichai forum post, "Key points"): x_t = W v_t, the product of the bf16
+    inputs in fp64 (each bf16 product is exact there; the sum of D terms
+    carries a relative error below D 2^-53), rounded once to fp32.
+    Vb [T, D], Wb [64, D] bf16 bits."""
+    V = bf16_bits_to_f32(np.asarray(Vb, np.uint16)).astype(np.float64)
+    W = bf16_bits_to_f32(np.asarray(Wb, np.uint16)).astype(np.float64)
+    return (V @ W.T).astype(np.float32)
+
+
 def pool_norm(keys: np.ndarray) -> np.ndarray:
     keys = _c(keys, np.float32)
     n_items = keys.shape[0] // N_POOL

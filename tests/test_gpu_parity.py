@@ -362,3 +362,39 @@ def test_prefill_from_host_matches_device_path(tiny):
                                      pin(torch.from_numpy(pos)), pin(Qd), pin(Kd), pin(Vd), h_O, chunks=chunks)
         torch.cuda.synchronize()
         assert torch.equal(h_O, Od.cpu())
+
+
+@pytest.mark.parametrize("D,t_begin,t_end", [(1024, 0, 4096), (128, 512, 2100), (64, 4, 700)])
+def test_shrink_against_oracle(D, t_begin, t_end):
+    """Step 1 on the tensor cores: keys within the fp32 accumulation bound of
+    the oracle's product, rows outside the range untouched; the fused pooled
+    items match the oracle's pooling of its keys within the bound's effect,
+    and are bit-identical to the cache build pooling the kernel's own keys."""
+    _need_gpu()
+    Vb = I.normal_bf16_bits(21, 901, (t_end, D))
+    Wb = I.normal_bf16_bits(22, 902, (64, D))
+    Vd, Wd = PT.bits_to_bf16(Vb), PT.bits_to_bf16(Wb)
+    keys = torch.full((t_end, 64), float("nan"), dtype=torch.float32, device="cuda")
+    pooled = torch.full((t_end // 4, 64), float("nan"), dtype=torch.float32, device="cuda")
+    lsa.lsa_shrink(Vd, Wd, t_begin, t_end, keys=keys, pooled=pooled)
+    torch.cuda.synchronize()
+    ref = O.shrink(Vb, Wb)
+    g = keys.cpu().numpy()
+    assert np.isnan(g[:t_begin]).all()
+    # fp32 accumulation of D exact products: |err| <= 2 D 2^-24 sum |v w| (+ output rounding)
+    absdot = np.abs(O.bf16_bits_to_f32(Vb)).astype(np.float64) @ np.abs(O.bf16_bits_to_f32(Wb)).astype(np.float64).T
+    bound = 2 * D * 2.0**-24 * absdot + np.abs(ref) * 2.0**-24
+    err = np.abs(g[t_begin:] - ref[t_begin:])
+    assert (err <= bound[t_begin:]).all(), f"max err/bound {np.max(err / bound[t_begin:]):.3g}"
+    i0, i1 = t_begin // 4, t_end // 4
+    gp = pooled.cpu().numpy()
+    assert np.isnan(gp[:i0]).all()
+    rp = O.pool_norm(ref[4 * i0:4 * i1])
+    rel = np.max(bound[t_begin:] / np.maximum(np.linalg.norm(ref[t_begin:], axis=1, keepdims=True), 1e-30))
+    assert np.max(np.abs(gp[i0:i1] - rp)) <= 8 * rel + 1e-6
+    # the cache build's own pooling of the kernel's keys: bit-identical
+    cache = lsa.Cache(-(-t_end // 512) * 512)
+    lsa.lsa_build_cache(keys, t_begin, t_end, cache, lsa.lsa_default_params())
+    torch.cuda.synchronize()
+    cp = cache.views()["pooled"].cpu().numpy()
+    assert np.array_equal(cp[i0:i1].view(np.uint32), gp[i0:i1].view(np.uint32))

@@ -486,3 +486,47 @@ def test_bucket_cache_bytes_per_token():
     centroid + 16 int32 member slots + 1 int32 count)."""
     per_block = 64 * (64 * 2 + 16 * 4 + 4)
     assert per_block / 512 == 24.5
+
+
+# --- step 1, "Shrink": x_t = W v_t ------------------------------------------
+
+BF16_ONE, BF16_MINUS_ONE = 0x3F80, 0xBF80
+
+
+def test_shrink_one_hot_rows_select_dims():
+    """W with one 1.0 per row picks input dims: a dropped term, a transposed
+    operand or a wrong index breaks the equality."""
+    rng = np.random.default_rng(5)
+    D = 256
+    V = I.normal_bf16_bits(5, 701, (37, D))
+    idx = rng.choice(D, 64, replace=False)
+    W = np.zeros((64, D), np.uint16)
+    W[np.arange(64), idx] = BF16_ONE
+    assert np.array_equal(O.shrink(V, W), O.bf16_bits_to_f32(V)[:, idx])
+
+
+def test_shrink_signed_permutation_keeps_norms():
+    """A signed permutation (orthogonal) of 64 dims: each output is plus or
+    minus one input, so the norm of every row is unchanged."""
+    rng = np.random.default_rng(6)
+    V = I.normal_bf16_bits(6, 702, (50, 64))
+    perm, sign = rng.permutation(64), rng.integers(0, 2, 64)
+    W = np.zeros((64, 64), np.uint16)
+    W[np.arange(64), perm] = np.where(sign == 1, BF16_MINUS_ONE, BF16_ONE)
+    x, v = O.shrink(V, W), O.bf16_bits_to_f32(V)
+    assert np.array_equal(x, np.where(sign == 1, -1.0, 1.0).astype(np.float32) * v[:, perm])
+    assert np.allclose(np.linalg.norm(x.astype(np.float64), axis=1), np.linalg.norm(v.astype(np.float64), axis=1),
+                       rtol=1e-12)
+
+
+def test_shrink_small_integers_exact():
+    """Small integers are exact in bf16, fp64 and fp32: the projection must
+    equal the integer contraction sum_d v_td w_ed exactly (D = 1024)."""
+    rng = np.random.default_rng(7)
+    D = 1024
+    vi = rng.integers(-4, 5, (19, D))
+    wi = rng.integers(-3, 4, (64, D))
+    to_bits = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)  # noqa: E731
+    x = O.shrink(to_bits(vi), to_bits(wi))
+    exact = np.einsum("td,ed->te", vi, wi)  # integer arithmetic
+    assert np.array_equal(x, exact.astype(np.float32))
