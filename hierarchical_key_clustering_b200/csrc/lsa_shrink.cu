@@ -1,8 +1,9 @@
-// Step 1 of the indexer, "Shrink": every key is projected to 64 numbers that
-// exist only for choosing (sotaaz blog, "The same steps in general", step 1;
-// zhichai forum post, "Key points": keys projected to a 64-dim latent space,
-// L2-normalised and pooled 4 at a time; D-LSA learns the projection, a PCA
-// of the keys does nearly as well).  x_t = W v_t, with v_t the row of a
+// Step 1 of the indexer, "Shrink" (sotaaz blog, "The same steps in general",
+// step 1; zhichai forum post, "Key points"): before anything is clustered,
+// a position's key is mapped linearly to a 64-dim vector that serves only the
+// selection of keys, never the attention itself.  The D-LSA variant trains
+// that map per layer; the forum post reports that a map taken from principal
+// components works about as well.  x_t = W v_t, with v_t the row of a
 // position (e.g. its key over all KV heads, D = Hkv x 128) and W [64, D].
 //
 // A dense contraction on the tensor cores, bound by reading V from HBM: one

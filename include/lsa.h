@@ -197,11 +197,11 @@ int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, 
 
 /* ---- the five calls of the hot path ---- */
 
-/* Step 1, "Shrink" ([BLOG] "The same steps in general", step 1: each key is
- * projected to 64 numbers that exist only for choosing; [FORUM] "Key
- * points": D-LSA learns the projection, a PCA of the keys does nearly as
- * well).  x_t = W v_t for every row t_begin <= t < t_end of V, fp32
- * accumulation on the tensor cores.
+/* Step 1, "Shrink" ([BLOG] "The same steps in general", step 1; [FORUM] "Key
+ * points"): a linear map of each position's key to a 64-dim vector used only
+ * to choose keys (trained per layer in D-LSA; a principal-component map is
+ * reported to do about as well).  x_t = W v_t for every row
+ * t_begin <= t < t_end of V, fp32 accumulation on the tensor cores.
  * V bf16 [>= t_end, D] (a position's row, e.g. its key over all KV heads,
  * D = Hkv x 128); W bf16 [64, D]; D a multiple of 64, <= 16384; V and W
  * 16-byte aligned.
