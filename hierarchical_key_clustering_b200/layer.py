@@ -76,9 +76,10 @@ class SparseLayer:
         """One prefill step whose inputs and output live in pinned host memory.
 
         Three streams overlap the transfers with the kernels.  The index
-        inputs go first, and the cache build and index start as soon as they
-        land.  Q then arrives in query chunks (multiples of 128 queries, so
-        the near-set tiles of the attention do not change), each preceded by
+        keys go first and the cache build starts as soon as they land, while
+        the index queries follow for the index.  Q then arrives in query
+        chunks (multiples of 128 queries, so the near-set tiles of the
+        attention do not change), each preceded by
         the K and V rows its queries can list (positions up to the chunk's
         largest query position; the rest of K and V follows the last chunk),
         and each chunk's attention starts when its rows are on the device;
@@ -118,8 +119,11 @@ class SparseLayer:
         need = [min(tk, int(h_pos[c0:c1].max()) + 1) for c0, c1 in bounds]
         self._h2d.wait_stream(cs)
         with torch.cuda.stream(self._h2d):
-            for d, h in ((d_keys, h_keys), (d_q, h_qidx), (d_pos, h_pos)):
-                d.copy_(h, non_blocking=True)
+            d_keys.copy_(h_keys, non_blocking=True)  # the build needs only the keys
+            e_keys = torch.cuda.Event()
+            e_keys.record()
+            d_q.copy_(h_qidx, non_blocking=True)
+            d_pos.copy_(h_pos, non_blocking=True)
             e_idx = torch.cuda.Event()
             e_idx.record()
             e_in, have = [], 0
@@ -136,8 +140,9 @@ class SparseLayer:
                 d_V[have:].copy_(h_V[have:], non_blocking=True)
             e_all = torch.cuda.Event()
             e_all.record()
-        cs.wait_event(e_idx)
+        cs.wait_event(e_keys)
         self.build(d_keys, stream=cs)
+        cs.wait_event(e_idx)
         self.index(d_q, d_pos, stream=cs)
         e_o = []
         for (c0, c1), ei in zip(bounds, e_in):
