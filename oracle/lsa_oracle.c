@@ -544,6 +544,44 @@ int orc_index(const float *qidx, const int64_t *pos, int64_t nq, int64_t nblk, i
     return bad ? -1 : 0;
 }
 
+/* Multi-head Flat search (zhichai forum post, "Key points": N-LSA selects
+ * buckets by the best score across heads).  Every query carries n_heads
+ * 64-dim index queries; a bucket's score is the largest of its n_heads
+ * scores (each the exact fp64 sum rounded once to fp32, as orc_score), and
+ * buckets rank by (that score desc, id asc).  Then the same expansion.
+ * qidx [nq, n_heads, 64]. */
+int orc_index_heads(const float *qidx, const int64_t *pos, int64_t nq, int n_heads, int64_t nblk, int n_buckets,
+                    const int32_t *members, const int32_t *count, const uint16_t *centroid_bf16, int k, int sink,
+                    int window, int32_t *lists, int32_t *lens, int Lmax)
+{
+    int64_t nb = nblk * n_buckets;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t i = 0; i < nq; ++i) {
+        uint16_t *qh = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)n_heads * DIM);
+        for (int h = 0; h < n_heads; ++h) orc_qnorm(qidx + (i * n_heads + h) * DIM, 1, qh + h * DIM);
+        int64_t H = pos[i] / BLOCK_KEYS;
+        if (H > nblk) H = nblk;
+        int64_t n = H * n_buckets;
+        scored_t *v = (scored_t *)malloc(sizeof(scored_t) * (size_t)(n > 0 ? n : 1));
+        int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * (size_t)(nb > 0 ? nb : 1));
+        for (int64_t b = 0; b < n; ++b) {
+            float best = orc_score(qh, centroid_bf16 + b * DIM);
+            for (int h = 1; h < n_heads; ++h) {
+                float s = orc_score(qh + h * DIM, centroid_bf16 + b * DIM);
+                if (s > best) best = s;
+            }
+            v[b].s = best;
+            v[b].id = (int32_t)b;
+        }
+        qsort(v, (size_t)n, sizeof(scored_t), cmp_rank);
+        for (int64_t j = 0; j < n; ++j) ids[j] = v[j].id;
+        lens[i] = orc_expand(ids, n, members, count, pos[i], k, sink, window, lists + i * Lmax, Lmax);
+        free(v); free(ids); free(qh);
+    }
+    return bad ? -1 : 0;
+}
+
 /* ---------- step a8: exact softmax attention over each list ---------- */
 
 /* [EXPL] "What one query actually does": plain softmax attention over the

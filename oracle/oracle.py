@@ -68,6 +68,7 @@ def lib():
             "orc_flat_rank": (i64, [P, i64, i32, P, P, P]),
             "orc_tree_rank": (i64, [P, i64, P, P, P, P, P, i32, i32, i64, P, P]),
             "orc_expand": (i32, [P, i64, P, P, i64, i32, i32, i32, P, i32]),
+            "orc_index_heads": (i32, [P, P, i64, i32, i64, i32, P, P, P, i32, i32, i32, P, P, i32]),
             "orc_index": (i32, [P, P, i64, i64, i32, P, P, P, i32, P, P, P, P, P, i32,
                                 i32, i32, i32, i32, P, P, i32]),
             "orc_attention": (None, [P, P, P, i64, i32, i32, i32, P, P, i32, f32, P, P]),
@@ -290,6 +291,25 @@ def index(qidx: np.ndarray, pos: np.ndarray, cache: Cache, k: int, mode: str = "
                         _p(tp) if tp is not None else nul, _p(tmb) if tmb is not None else nul,
                         _p(tcb) if tcb is not None else nul, _p(tls) if tls is not None else nul, tl,
                         k, sink, window, beam, _p(lists), _p(lens), Lmax)
+    if r < 0:
+        raise RuntimeError("oracle index failed")
+    return lists, lens
+
+
+def index_heads(qidx: np.ndarray, pos: np.ndarray, cache: Cache, k: int, sink: int = 4, window: int = 512):
+    """Multi-head Flat search (zhichai forum post, "Key points": N-LSA picks
+    buckets by the best score across heads): qidx [nq, n_heads, 64]; a
+    bucket scores the largest of its per-head scores.  Lists and lens as
+    index()."""
+    qidx = _c(qidx, np.float32)
+    assert qidx.ndim == 3 and qidx.shape[2] == DIM
+    pos = _c(pos, np.int64)
+    nq, nh = qidx.shape[0], qidx.shape[1]
+    Lmax = list_budget(k, sink, window)
+    lists = np.empty((nq, Lmax), np.int32)
+    lens = np.empty(nq, np.int32)
+    r = lib().orc_index_heads(_p(qidx), _p(pos), nq, nh, cache.nblk, N_BUCKETS, _p(cache.members), _p(cache.count),
+                              _p(cache.centroid_bf16), k, sink, window, _p(lists), _p(lens), Lmax)
     if r < 0:
         raise RuntimeError("oracle index failed")
     return lists, lens

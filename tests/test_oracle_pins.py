@@ -405,6 +405,62 @@ def test_expand_skips_near_and_refills():
     assert np.all(out[n:] == -1)
 
 
+# ---------------------------------------------------------------- multi-head Flat search
+
+def test_heads_one_head_is_flat(tiny):
+    _, cache, pos, q = tiny
+    sel = np.arange(0, 4096, 53)
+    lf, nf = O.index(q[sel], pos[sel], cache, k=256)
+    lh, nh = O.index_heads(q[sel][:, None, :], pos[sel], cache, k=256)
+    assert np.array_equal(nf, nh) and np.array_equal(lf, lh)
+
+
+def test_heads_identical_and_rescaled_heads_are_flat(tiny):
+    """Each head is normalised on its own, so copies of one query, each scaled
+    by its own positive factor, select what the single query selects."""
+    _, cache, pos, q = tiny
+    sel = np.arange(7, 4096, 71)
+    lf, nf = O.index(q[sel], pos[sel], cache, k=200)
+    scale = np.array([1.0, 3.0, 0.25, 17.0], np.float32)
+    qh = q[sel][:, None, :] * scale[None, :, None]
+    lh, nh = O.index_heads(qh, pos[sel], cache, k=200)
+    assert np.array_equal(nf, nh) and np.array_equal(lf, lh)
+
+
+def test_heads_max_score_brute_force(tiny):
+    """Buckets ranked by the best per-head score (fp64 products rounded to
+    fp32, score desc then id asc), then the usual expansion."""
+    keys, cache, pos, q = tiny
+    cbf = O.bf16_bits_to_f32(cache.centroid_bf16).astype(np.float64)
+    rng = np.random.default_rng(11)
+    nh = 3
+    for p in (700, 1800, 3333, 4095):
+        qs = np.concatenate([q[p][None], rng.standard_normal((nh - 1, 64)).astype(np.float32)])
+        H = p // 512
+        best = np.full(64 * H, -np.inf, np.float32)
+        for h in range(nh):
+            qb = O.bf16_bits_to_f32(O.qnorm(qs[h])[0]).astype(np.float64)
+            best = np.maximum(best, (cbf[:64 * H] @ qb).astype(np.float32))
+        order = np.array(sorted(range(64 * H), key=lambda b: (-best[b], b)), np.int64)
+        want, n = O.expand(order, cache, p=p, k=300)
+        got, m = O.index_heads(qs[None], np.array([p]), cache, k=300)
+        assert m[0] == n and np.array_equal(got[0, :m[0]], want[:n])
+
+
+def test_heads_centroid_head_opens_its_bucket(tiny):
+    """A head equal to a bucket's centroid scores that bucket near 1, above
+    every other head's score for it, so its keys head the far part."""
+    keys, cache, pos, q = tiny
+    p = 4000
+    b = 3 * 64 + 17
+    c = O.bf16_bits_to_f32(cache.centroid_bf16[b])
+    qs = np.stack([q[p], c, -q[p]])
+    lists, lens = O.index_heads(qs[None], np.array([p]), cache, k=int(cache.count[b]))
+    mem = cache.members[b, :cache.count[b]]
+    far = [t for t in mem if 4 <= t < p - 512]
+    assert set(far) <= set(lists[0, :lens[0]].tolist())
+
+
 # ---------------------------------------------------------------- a6 tree search
 
 def test_wide_beam_tree_equals_flat(tiny):
