@@ -66,6 +66,10 @@ int check_params(const lsa_params *p)
     if (p->k > (1 << 20)) return fail(LSA_ERR_ARG, "k = %d is above the supported 1048576", p->k);
     if (p->mode != LSA_MODE_FLAT && p->mode != LSA_MODE_TREE) return fail(LSA_ERR_ARG, "mode must be 0 or 1");
     if (p->mode == LSA_MODE_TREE && p->beam < 1) return fail(LSA_ERR_ARG, "beam must be >= 1");
+    if (p->index_heads < 1 || p->index_heads > LSA_MAX_INDEX_HEADS)
+        return fail(LSA_ERR_ARG, "index_heads = %d must be in 1..%d", p->index_heads, LSA_MAX_INDEX_HEADS);
+    if (p->mode == LSA_MODE_TREE && p->index_heads != 1)
+        return fail(LSA_ERR_ARG, "Tree search takes one index head (index_heads = %d)", p->index_heads);
     return LSA_OK;
 }
 
@@ -144,26 +148,44 @@ TreeLayout tree_layout(int64_t nblk)
     return T;
 }
 
+// Entries the expansion kernel holds in shared memory per query: the filter
+// keeps about 1.2-1.45 P candidates on the measured workloads; a query with
+// more takes the exact path.
+int64_t expand_slots(int64_t cap, int64_t P)
+{
+    const int64_t kc = lsa::pow2_ceil64((P * 3 + 1) / 2);
+    return cap < kc ? cap : kc;
+}
+
+// The scorer's arrays are per row, a row being one (query, index head); with
+// several index heads the merged candidates of each query follow (one bucket
+// per entry, expand_slots entries per query).
 struct IndexLayout {
-    int64_t off[8];
+    int64_t off[13];
     int64_t bytes;
     int64_t gstride;
     int64_t sstride;
     int64_t cap;
+    int64_t mcap;
 };
 
 IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
 {
     const int64_t N = nblk * LSA_BUCKETS;
+    const int64_t heads = p->index_heads > 1 ? p->index_heads : 1;
+    const int64_t rows = nq * heads;
     IndexLayout L;
-    L.gstride = lsa::HIST_BINS;  // group-maximum histogram per query
+    L.gstride = lsa::HIST_BINS;  // group-maximum histogram per row
     L.cap = cand_cap(p);
+    L.mcap = heads > 1 ? expand_slots(L.cap, top_buckets(p)) : 0;
+    const int64_t mq = heads > 1 ? nq : 0;
     // small batches (decode) keep every score for the filter pass
-    L.sstride = (nq <= lsa::SMALL_NQ && p->mode == LSA_MODE_FLAT) ? N : 0;
-    const int64_t sz[8] = {nq * LSA_DIM * 2, nq * 4,          nq * 4,          nq * 4, nq * L.gstride * 4,
-                           nq * L.cap * 16,  nq * L.cap * 4, nq * L.sstride * 4};
+    L.sstride = (rows <= lsa::SMALL_NQ && p->mode == LSA_MODE_FLAT) ? N : 0;
+    const int64_t sz[13] = {rows * LSA_DIM * 2, rows * 4,        rows * 4, rows * 4, rows * L.gstride * 4,
+                            rows * L.cap * 16,  rows * L.cap * 4, rows * L.sstride * 4,
+                            mq * 4,             mq * 4,          mq * 4,   mq * L.mcap * 16, mq * L.mcap * 4};
     int64_t o = 0;
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 13; ++i) {
         L.off[i] = o;
         o += align256(sz[i]);
     }
@@ -264,6 +286,18 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     iw.scores = L.sstride ? (float *)(w + L.off[7]) : nullptr;
     iw.score_stride = L.sstride;
     iw.cap = (int32_t)L.cap;
+    lsa::IndexWs mw = iw;  // merged candidates of multi-head queries
+    if (p->index_heads > 1) {
+        mw.horizon = (int32_t *)(w + L.off[8]);
+        mw.tau = (float *)(w + L.off[9]);
+        mw.cnt = (int32_t *)(w + L.off[10]);
+        mw.cand4 = (float *)(w + L.off[11]);
+        mw.cand_g = (int32_t *)(w + L.off[12]);
+        mw.ghist = nullptr;
+        mw.scores = nullptr;
+        mw.score_stride = 0;
+        mw.cap = (int32_t)L.mcap;
+    }
     lsa::IndexArgs a;
     a.qidx = qidx;
     a.pos = pos;
@@ -281,6 +315,7 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     a.beam = p->beam;
     a.mode = p->mode;
     a.P = (int32_t)P;
+    a.heads = p->index_heads;
     a.wait_limit = g_wait_limit;
     a.extra_tx = g_extra_tx;
     g_extra_tx = 0;
@@ -296,7 +331,8 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
         for (int l = 0; l < 41; ++l) tv.level_offset[l] = tree->level_offset[l];
         tvp = &tv;
     }
-    cudaError_t e = lsa::launch_index(a, iw, tvp, (cudaStream_t)stream, sm_count());
+    cudaError_t e = lsa::launch_index(a, iw, p->index_heads > 1 ? &mw : nullptr, tvp, (cudaStream_t)stream,
+                                      sm_count());
     if (e != cudaSuccess) return cuda_fail(e, "index launch");
     return LSA_OK;
 }
@@ -366,6 +402,7 @@ void lsa_default_params(lsa_params *p)
     p->beam = 32;
     p->mode = LSA_MODE_FLAT;
     p->cand_cap = 0;
+    p->index_heads = 1;
 }
 
 const char *lsa_last_error_string(void)

@@ -28,8 +28,10 @@ namespace lsa {
 
 
 // ---------------------------------------------------------------------------
+// One warp per row; a row is one index query, `heads` consecutive rows per
+// token (all with that token's horizon).
 __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, const int64_t *__restrict__ pos,
-                                               int64_t nq, int64_t n_blocks, IndexWs ws)
+                                               int64_t nq, int heads, int64_t n_blocks, IndexWs ws)
 {
     pdl_wait();
     pdl_release();
@@ -42,7 +44,7 @@ __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, c
         ws.qhat[q * LSA_D + lane] = f2bf_bits(a);
         ws.qhat[q * LSA_D + lane + 32] = f2bf_bits(b);
         if (lane == 0) {
-            int64_t p = pos[q];
+            int64_t p = pos[q / heads];
             int64_t H = p < 0 ? 0 : p / LSA_BLK;
             if (H > n_blocks) H = n_blocks;
             ws.horizon[q] = (int32_t)H;
@@ -1140,41 +1142,252 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     if (t == 0) lens[q] = len;
 }
 
+// ---------------------------------------------------------------------------
+// Multi-head Flat search (zhichai forum post, "Key points": N-LSA ranks a
+// bucket by its best score across the index heads).  Every (query, head) row
+// went through the Flat passes above on its own.  A bucket among the top P
+// by best score is among the top P of the head that attains that score (a
+// bucket ahead of it for that head is ahead of it overall), so that head
+// listed it, with that very score.  Keeping every listed bucket once, with
+// the largest score any head listed for it, and cutting at the P-th largest
+// of those values keeps exactly the top P: a kept value falls short of a
+// bucket's best only for buckets outside the top P.  The kept buckets go out
+// as one-bucket entries with tau = -inf, for the unchanged expansion.
+// The union is deduplicated in a shared-memory hash table (linear probing,
+// at most 3/4 full).  A query whose rows overflowed their entry slots, whose
+// union does not fit the table, or whose cut keeps more than the expansion's
+// slots (ties) is redone exactly: every visible bucket scored for every head
+// on the CUDA cores, radix select, ties in ascending bucket order.
+constexpr int HM_THREADS = 512;
+constexpr int HM_MAX_SLOTS = 25600;  // 200 KB of table
+
+// Table slots for a launch: about 3 x heads x P (a head lists ~1.2-1.45 P
+// buckets on the measured workloads), a multiple of 512, at most HM_MAX_SLOTS.
+inline int heads_merge_slots(int heads, int P)
+{
+    const int64_t want = ((int64_t)3 * heads * P + 511) / 512 * 512;
+    return (int)(want < HM_MAX_SLOTS ? (want < 512 ? 512 : want) : HM_MAX_SLOTS);
+}
+
+// Insert bucket `id` with ordered score v; returns 1 if the id was new.
+__device__ __forceinline__ int hash_insert(int32_t *hkey, uint32_t *hval, int TS, int32_t id, uint32_t v)
+{
+    uint32_t s = __umulhi((uint32_t)id * 0x9E3779B1u, (uint32_t)TS);
+    for (int n = 0; n < TS; ++n) {  // ends at a free slot: the table has more slots than ids
+        const int32_t prev = atomicCAS(&hkey[s], -1, id);
+        if (prev == -1 || prev == id) {
+            atomicMax(&hval[s], v);
+            return prev == -1;
+        }
+        s = (s + 1 == (uint32_t)TS) ? 0u : s + 1;
+    }
+    return 0;
+}
+
+__global__ void __launch_bounds__(HM_THREADS) k_heads_merge(int heads, int P, int TSMAX,
+                                                           const uint16_t *__restrict__ cbf, IndexWs ws, IndexWs m)
+{
+    pdl_wait();
+    pdl_release();
+    extern __shared__ uint32_t hsm[];
+    int32_t *hkey = reinterpret_cast<int32_t *>(hsm);  // [TS] bucket id, -1 = empty
+    uint32_t *hval = hsm + TSMAX;                      // [TS] f2ord of its best listed score
+    float *qf = reinterpret_cast<float *>(hsm);        // [heads, 64] (exact path only)
+    __shared__ int hist[256];
+    __shared__ int sh[4];
+    __shared__ int wsum[HM_THREADS / 32];
+    __shared__ int s_listed, s_over, s_uniq, s_out, s_exact;
+    const int64_t q = blockIdx.x;
+    const int64_t r0 = q * heads;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const float NEG = __int_as_float(0xff800000);
+    const int KC = m.cap;
+    const int64_t N = (int64_t)ws.horizon[r0] * LSA_NBKT;
+    float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * KC;
+    int32_t *og = m.cand_g + q * KC;
+    if (t == 0) {
+        s_listed = 0;
+        s_over = 0;
+        s_uniq = 0;
+        s_out = 0;
+    }
+    __syncthreads();
+
+    // 1. scores the heads listed
+    int my = 0;
+    for (int h = 0; h < heads; ++h) {
+        const int64_t r = r0 + h;
+        const int ne = ws.cnt[r];
+        if (ne > ws.cap) {  // the row lost entries: exact path
+            s_over = 1;
+            continue;
+        }
+        const float tau = ws.tau[r];
+        const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + r * ws.cap;
+        for (int i = t; i < ne; i += HM_THREADS) {
+            const float4 s4 = c4[i];
+            my += (s4.x >= tau && s4.x > NEG) + (s4.y >= tau && s4.y > NEG) + (s4.z >= tau && s4.z > NEG) +
+                  (s4.w >= tau && s4.w > NEG);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) my += __shfl_xor_sync(LSA_FULL, my, o);
+    if (lane == 0 && my) atomicAdd(&s_listed, my);
+    __syncthreads();
+    const int listed = s_listed;
+    if (t == 0) s_exact = s_over || (int64_t)listed * 4 > (int64_t)TSMAX * 3;
+    __syncthreads();
+
+    // 2. union with the best listed score per bucket, cut at the P-th value
+    if (!s_exact) {
+        const int TS = min(TSMAX, max(2 * listed, 64));
+        for (int i = t; i < TS; i += HM_THREADS) {
+            hkey[i] = -1;
+            hval[i] = 0u;
+        }
+        __syncthreads();
+        int fresh = 0;
+        for (int h = 0; h < heads; ++h) {
+            const int64_t r = r0 + h;
+            const int ne = ws.cnt[r];
+            const float tau = ws.tau[r];
+            const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + r * ws.cap;
+            const int32_t *cg = ws.cand_g + r * ws.cap;
+            for (int i = t; i < ne; i += HM_THREADS) {
+                const float4 s4 = c4[i];
+                const int32_t g = cg[i];
+                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (sv[e] >= tau && sv[e] > NEG) fresh += hash_insert(hkey, hval, TS, g + e, f2ord(sv[e]));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) fresh += __shfl_xor_sync(LSA_FULL, fresh, o);
+        if (lane == 0 && fresh) atomicAdd(&s_uniq, fresh);
+        __syncthreads();
+        // keep everything when it fits the expansion's slots, else the P-th
+        // largest value and every bucket at or above it
+        uint32_t cut = 0u;
+        if (s_uniq > KC) {
+            auto get = [&](int64_t i) { return hkey[i] >= 0 ? ord2f(hval[i]) : NEG; };
+            cut = block_select_kth_largest(TS, P, get, hist, sh);
+        }
+        for (int i = t; i < TS; i += HM_THREADS) {
+            const int32_t id = hkey[i];
+            const uint32_t v = hval[i];
+            if (id >= 0 && v >= cut) {
+                const int j = atomicAdd(&s_out, 1);
+                if (j < KC) {
+                    o4[j] = make_float4(ord2f(v), NEG, NEG, NEG);
+                    og[j] = id;
+                }
+            }
+        }
+        __syncthreads();
+        if (t == 0 && s_out > KC) s_exact = 1;
+        __syncthreads();
+    }
+
+    // 3. exact path
+    if (s_exact) {
+        for (int i = t; i < heads * LSA_D; i += HM_THREADS) qf[i] = bf_bits2f(ws.qhat[r0 * LSA_D + i]);
+        if (t == 0) s_out = 0;
+        __syncthreads();
+        auto best = [&](int64_t b) {
+            const uint16_t *c = cbf + b * LSA_D;
+            float s = dot_bf16_row(qf, c);
+            for (int h = 1; h < heads; ++h) s = fmaxf(s, dot_bf16_row(qf + h * LSA_D, c));
+            return s;
+        };
+        if (N <= P) {
+            for (int64_t b = t; b < N; b += HM_THREADS) {
+                o4[b] = make_float4(best(b), NEG, NEG, NEG);
+                og[b] = (int32_t)b;
+            }
+            if (t == 0) s_out = (int)N;
+        } else {
+            const float ts = ord2f(block_select_kth_largest(N, P, best, hist, sh));
+            for (int64_t b = t; b < N; b += HM_THREADS) {
+                const float s = best(b);
+                if (s > ts) {
+                    const int j = atomicAdd(&s_out, 1);  // fewer than P buckets score above ts
+                    o4[j] = make_float4(s, NEG, NEG, NEG);
+                    og[j] = (int32_t)b;
+                }
+            }
+            __syncthreads();
+            // ties at ts in ascending bucket order, up to P in all
+            for (int64_t base = 0; base < N; base += HM_THREADS) {
+                if (s_out >= P) break;  // block-uniform (read after a barrier)
+                const int64_t b = base + t;
+                const bool tie = (b < N) && (best(b) == ts);
+                const unsigned bal = __ballot_sync(LSA_FULL, tie);
+                if (lane == 0) wsum[warp] = __popc(bal);
+                __syncthreads();
+                int before = s_out;
+                for (int w = 0; w < warp; ++w) before += wsum[w];
+                before += __popc(bal & ((1u << lane) - 1u));
+                if (tie && before < P) {
+                    o4[before] = make_float4(ts, NEG, NEG, NEG);
+                    og[before] = (int32_t)b;
+                }
+                __syncthreads();
+                if (t == 0) {
+                    int tot = 0;
+                    for (int w = 0; w < HM_THREADS / 32; ++w) tot += wsum[w];
+                    s_out = min(P, s_out + tot);
+                }
+                __syncthreads();
+            }
+        }
+    }
+    __syncthreads();
+    if (t == 0) {
+        m.cnt[q] = s_out;
+        m.tau[q] = NEG;
+        m.horizon[q] = ws.horizon[r0];
+    }
+}
+
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks)
 {
     return rank_expand_smem(cap, (int)((n_blocks + 31) / 32) + 1);
 }
 
 // ---------------------------------------------------------------------------
-cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *tree, cudaStream_t st, int n_sm)
+cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *merged, const TreeView *tree,
+                         cudaStream_t st, int n_sm)
 {
     if (a.nq <= 0) return cudaSuccess;
     cudaError_t e;
+    const int heads = a.heads > 1 ? a.heads : 1;
+    const int64_t rows = a.nq * heads;  // one scoring row per (query, index head)
     {
-        int64_t blocks = (a.nq + 7) / 8;
+        int64_t blocks = (rows + 7) / 8;
         if (blocks > (int64_t)n_sm * 32) blocks = (int64_t)n_sm * 32;
-        if ((e = launch_k(a.nq <= SMALL_NQ, k_qnorm, dim3((unsigned)blocks), dim3(256), 0, st, a.qidx, a.pos, a.nq,
-                          a.n_blocks, ws)) != cudaSuccess)
+        if ((e = launch_k(rows <= SMALL_NQ, k_qnorm, dim3((unsigned)blocks), dim3(256), 0, st, a.qidx, a.pos, rows,
+                          heads, a.n_blocks, ws)) != cudaSuccess)
             return e;
         count_launches(1);
     }
     const int64_t nb_total = a.n_blocks * LSA_NBKT;
     const bool small = a.nq <= SMALL_NQ;
     if (a.mode == 0 && nb_total > 0) {
-        if (small) {  // stream every centroid once for the whole batch, keep the scores
+        if (rows <= SMALL_NQ) {  // stream every centroid once for the whole batch, keep the scores
             const int dsm = DS_WARPS * 2 * 32 * DS_ROW;
             cudaFuncSetAttribute(k_dscore, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
             if ((e = launch_k(true, k_dscore, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
-                              (size_t)dsm, st, a.nq, nb_total, a.centroid_bf16, a.P, ws)) != cudaSuccess)
+                              (size_t)dsm, st, rows, nb_total, a.centroid_bf16, a.P, ws)) != cudaSuccess)
                 return e;
             count_launches(1);
-            if ((e = launch_k(true, k_dfilter, dim3((unsigned)((nb_total / 4 + 255) / 256)), dim3(256), 0, st, a.nq, a.P,
+            if ((e = launch_k(true, k_dfilter, dim3((unsigned)((nb_total / 4 + 255) / 256)), dim3(256), 0, st, rows, a.P,
                               ws)) != cudaSuccess)
                 return e;
             count_launches(1);
         } else {  // two passes on the tensor cores: threshold, then filter
             ScoreTcArgs sa;
-            sa.nq = a.nq;
+            sa.nq = rows;
             sa.nb_total = nb_total;
             sa.P = a.P;
             sa.mode = 0;
@@ -1184,7 +1397,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
             int whole = 0;
             if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, &whole)) != cudaSuccess) return e;
             if (!whole) {  // thresholds from the merged histograms
-                k_tau<<<(unsigned)((a.nq + 7) / 8), 256, 0, st>>>(a.nq, a.P, ws);
+                k_tau<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(rows, a.P, ws);
                 count_launches(1);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
@@ -1215,21 +1428,32 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *
         if (e != cudaSuccess) return e;
         count_launches(1);
     }
+    if (merged) {  // several index heads: one candidate set per query
+        const int TSMAX = heads_merge_slots(heads, a.P);
+        const size_t smh = (size_t)TSMAX * 8;
+        cudaFuncSetAttribute(k_heads_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smh);
+        if ((e = launch_k(small, k_heads_merge, dim3((unsigned)a.nq), dim3(HM_THREADS), smh, st, heads, a.P, TSMAX,
+                          a.centroid_bf16, ws, *merged)) != cudaSuccess)
+            return e;
+        count_launches(1);
+    }
+    const IndexWs &ex = merged ? *merged : ws;
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
     // candidates held in shared memory: the filter keeps about 1.2-1.45 P per
     // query on the measured workloads; a query with more takes the exact path
-    const int KC = (int)min((int64_t)ws.cap, pow2_ceil64(((int64_t)a.P * 3 + 1) / 2));
+    // (a merged set never has more than its slots)
+    const int KC = merged ? merged->cap : (int)min((int64_t)ws.cap, pow2_ceil64(((int64_t)a.P * 3 + 1) / 2));
     const size_t smr = rank_expand_smem(KC, TW);
     if (small) {  // one CTA per query, few queries: widest blocks
         cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         const cudaError_t el = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
                                         a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
-                                        a.window, a.P, KC, TW, ws);
+                                        a.window, a.P, KC, TW, ex);
         if (el != cudaSuccess) return el;
     } else {
         cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,
-                                                             a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ws);
+                                                             a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ex);
     }
     count_launches(1);
     return cudaGetLastError();

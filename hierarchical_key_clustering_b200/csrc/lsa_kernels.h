@@ -120,6 +120,7 @@ struct IndexArgs {
     int32_t Lmax;
     int32_t k, sink, window, beam, mode;
     int32_t P;  // top buckets kept
+    int32_t heads;  // index queries per token (Flat: a bucket ranks by its best head score)
     uint32_t wait_limit;  // tries per bounded device-side wait
     uint32_t extra_tx;    // test hook (see lsa_debug_wait_test)
 };
@@ -152,7 +153,10 @@ struct ShrinkArgs {
 cudaError_t launch_shrink(const uint16_t *V, const uint16_t *W, const ShrinkArgs &a, cudaStream_t st);
 int read_shrink_error(int clear);
 
-cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const TreeView *tree, cudaStream_t st, int n_sm);
+// ws holds one row per (query, index head); with several heads `merged`
+// receives each query's merged candidates (nullptr for one head).
+cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *merged, const TreeView *tree,
+                         cudaStream_t st, int n_sm);
 // Shared memory the expansion kernel needs for `cap` candidates over a cache
 // of n_blocks blocks.
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks);

@@ -78,6 +78,20 @@ def index_queries(seed: int, keys: np.ndarray, positions: np.ndarray, sigma: flo
     return np.ascontiguousarray(q, dtype=np.float32)
 
 
+def index_queries_heads(seed: int, keys: np.ndarray, positions: np.ndarray, heads: int) -> np.ndarray:
+    """[nq, heads, 64] fp32 index queries for multi-head search: head 0 is
+    index_queries(seed, ...); head h > 0 is half of it plus the query of
+    another seed for a position spread over the keys, so the heads agree in
+    part and differ in part."""
+    positions = np.asarray(positions, np.int64)
+    q0 = index_queries(seed, keys, positions)
+    out = [q0]
+    for h in range(1, heads):
+        other = (positions * (h + 3) + h) % keys.shape[0]
+        out.append((np.float32(0.5) * q0 + index_queries(seed + 17 * h, keys, other)).astype(np.float32))
+    return np.ascontiguousarray(np.stack(out, axis=1))
+
+
 def normal_bf16_bits(seed: int, stream: int, shape) -> np.ndarray:
     """N(0,1) values rounded to bf16 (round to nearest even), as uint16 bits."""
     x = rng(seed, stream).standard_normal(shape, dtype=np.float32)

@@ -14,8 +14,9 @@ from . import lsa
 class SparseLayer:
     def __init__(self, capacity: int, k: int = 4096, mode: str = "flat", beam: int = 32, sink: int = 4,
                  window: int = 512, max_queries: int = 1, Hq: int = 32, head_dim: int = 128,
-                 cand_cap: int = 0, device="cuda"):
-        self.p = lsa.lsa_default_params(k=k, mode=mode, beam=beam, sink=sink, window=window, cand_cap=cand_cap)
+                 cand_cap: int = 0, index_heads: int = 1, device="cuda"):
+        self.p = lsa.lsa_default_params(k=k, mode=mode, beam=beam, sink=sink, window=window, cand_cap=cand_cap,
+                                        index_heads=index_heads)
         self.mode = mode
         self.cache = lsa.Cache(capacity, device)
         self.tree = lsa.Tree(max(capacity // 512, 1), device) if mode == "tree" else None

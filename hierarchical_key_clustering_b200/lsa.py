@@ -38,7 +38,8 @@ class LsaError(RuntimeError):
 
 class lsa_params(C.Structure):
     _fields_ = [(n, C.c_int32) for n in
-                ("n_pool", "block", "n_buckets", "cap_items", "sink", "window", "k", "beam", "mode", "cand_cap")]
+                ("n_pool", "block", "n_buckets", "cap_items", "sink", "window", "k", "beam", "mode", "cand_cap",
+                 "index_heads")]
 
 
 class lsa_cache(C.Structure):
@@ -301,6 +302,7 @@ def lsa_update_tree(cache: Cache, tree: Tree, p: lsa_params, stream=None):
 
 def _index(fn, qidx, pos, cache, tree, lists, lens, p, ws, stream):
     nq = qidx.shape[0]
+    assert qidx.numel() == nq * max(p.index_heads, 1) * 64, "qidx must be [nq, index_heads, 64]"
     Lmax = lists.shape[1] if lists.dim() == 2 else lsa_list_budget(p)
     _check(fn(_ptr(qidx), _ptr(pos), nq, C.byref(cache.c), C.byref(tree.t) if tree is not None else None,
               _ptr(lists), _ptr(lens), Lmax, C.byref(p), _ptr(ws), ws.numel() if ws is not None else 0,

@@ -50,6 +50,7 @@ extern "C" {
 #define LSA_SLOTS 16         /* member slots per bucket (<= 16 keys, [BLOG] step 2)    */
 #define LSA_HEAD_DIM 128     /* attention head width handled by lsa_sparse_attention   */
 #define LSA_MAX_LEVELS 40    /* tree levels (ceil(log2(buckets)) + 1 <= 40)            */
+#define LSA_MAX_INDEX_HEADS 16 /* index queries per token in multi-head Flat search     */
 
 enum {
     LSA_OK = 0,
@@ -69,7 +70,11 @@ enum { LSA_MODE_FLAT = 0, LSA_MODE_TREE = 1 };
  * beam 32, mode Flat.
  * cand_cap: per-query candidate slots of the Flat search (0 = automatic).
  * A smaller value only routes more queries through the exact fallback
- * selection; results do not change. */
+ * selection; results do not change.
+ * index_heads: index queries per token, 1..LSA_MAX_INDEX_HEADS (default 1).
+ * With more than one, Flat search ranks a bucket by the largest of its
+ * per-head scores (zhichai forum post, "Key points": N-LSA's bucket
+ * selection); qidx is then [nq, index_heads, 64].  Tree mode takes 1 only. */
 typedef struct lsa_params {
     int32_t n_pool;
     int32_t block;
@@ -81,6 +86,7 @@ typedef struct lsa_params {
     int32_t beam;
     int32_t mode;
     int32_t cand_cap;
+    int32_t index_heads;
 } lsa_params;
 
 /* Bucket cache ([EXPL] "How the hierarchy is built": a bucket keeps a
@@ -253,13 +259,15 @@ int lsa_update_tree(const lsa_cache *cache, lsa_tree *tree, const lsa_params *p,
 
 /* Steps 3-5 for nq queries ([EXPL] "What one query actually does"; [BLOG]
  * steps 3-5 and read_list).
- * qidx fp32 [nq, 64] index queries; pos i64 [nq] their positions.  Query i
+ * qidx fp32 [nq, 64] index queries ([nq, p->index_heads, 64] with several
+ * index heads); pos i64 [nq] their positions.  Query i
  * sees the buckets of blocks b < H = min(pos/512, cache->n_blocks).
  *   Flat (p->mode == LSA_MODE_FLAT, tree may be NULL): score every visible
  *   bucket, s = <bf16(q/|q|), centroid_bf16> with fp32 accumulation, rank by
  *   (score desc, bucket id asc).  Supports caches of up to 65535 blocks
  *   (33.5M tokens) and k + sink + window < 32768; larger requests return
- *   LSA_ERR_SHAPE.
+ *   LSA_ERR_SHAPE.  With index_heads > 1 every head is normalised and scored
+ *   on its own and a bucket ranks by its largest head score.
  *   Tree: level-synchronous beam search from the root: candidates at level l
  *   are the children of the nodes kept at level l+1 plus the visible
  *   level-l nodes whose parent is not visible; keep the best

@@ -54,6 +54,19 @@ def assert_cache_equal(g: dict, oc: O.Cache):
     assert np.array_equal(g["centroid_bf16"], oc.centroid_bf16), "bf16 centroids differ"
 
 
+def rank_heads(q_heads: np.ndarray, H: int, oc: O.Cache):
+    """Visible buckets by (best score over the index heads desc, id asc), each
+    head's scores taken from the oracle's Flat ranking."""
+    best = np.full(64 * H, -np.inf, np.float32)
+    for qv in q_heads:
+        ids, sc = O.flat_rank(O.qnorm(qv)[0], H, oc)
+        s = np.empty(64 * H, np.float32)
+        s[ids] = sc
+        best = np.maximum(best, s)
+    order = np.lexsort((np.arange(64 * H), -best.astype(np.float64)))
+    return order, best[order]
+
+
 def _cutoff_buckets(qhat_bits, p, H, oc: O.Cache, k, sink=4, window=512, ranked=None):
     """Scores of the oracle's ranked buckets and the score where k is reached."""
     if ranked is None:
@@ -88,10 +101,13 @@ def assert_lists_match(g_lists, g_lens, o_lists, o_lens, qidx, pos, oc: O.Cache,
             continue
         p = int(pos[i])
         H = min(p // 512, nblk)
-        qh = O.qnorm(qidx[i])[0]
+        qi = np.asarray(qidx[i])
+        qh = O.qnorm(qi.reshape(-1, 64)[0])[0]
         ranked = None
         if tree is not None:
             ranked = O.tree_rank(qh, H, tree, beam, O.top_p(k, sink, window))
+        elif qi.ndim == 2 and qi.shape[0] > 1:
+            ranked = rank_heads(qi, H, oc)
         ids, sc, tau = _cutoff_buckets(qh, p, H, oc, k, sink, window, ranked)
         ok = tau is not None and g_lens[i] == o_lens[i]
         if ok:

@@ -18,11 +18,12 @@ def _need_gpu():
         pytest.fail("a CUDA GPU is required for the -m gpu tests")
 
 
-def _build_gpu(keys: np.ndarray, capacity=None, pieces=None, mode="flat", k=256, beam=32, cand_cap=0):
+def _build_gpu(keys: np.ndarray, capacity=None, pieces=None, mode="flat", k=256, beam=32, cand_cap=0,
+               index_heads=1):
     _need_gpu()
     T = keys.shape[0]
     cache = lsa.Cache(capacity or T)
-    p = lsa.lsa_default_params(k=k, mode=mode, beam=beam, cand_cap=cand_cap)
+    p = lsa.lsa_default_params(k=k, mode=mode, beam=beam, cand_cap=cand_cap, index_heads=index_heads)
     kd = PT.to_dev(keys)
     if pieces is None:
         pieces = [(0, T)]
@@ -129,6 +130,41 @@ def test_decode_positions_past_context(tiny, cand_cap):
         gl, gn = _index_gpu(cache, None, p, qq[:nq], pos[:nq], decode=True)
         ol, on = O.index(qq[:nq], pos[:nq], oc, k=256)
         PT.assert_lists_match(gl, gn, ol, on, qq[:nq], pos[:nq], oc, k=256)
+
+
+@pytest.mark.parametrize("heads,k,cand_cap", [(2, 256, 0), (4, 256, 0), (8, 5000, 0), (3, 7, 0), (4, 256, 193)])
+def test_flat_index_heads_against_oracle(tiny, heads, k, cand_cap):
+    """Multi-head Flat search (a bucket ranks by its best head score), every
+    position class of the edge test, ragged count; cand_cap = P makes rows
+    overflow, so queries take the merge's exact path."""
+    keys, _, _, oc = tiny
+    pos = np.array([0, 3, 4, 511, 512, 513, 1023, 1024, 2047, 2048, 3000, 4095] + list(range(600, 4096, 37)),
+                   np.int64)
+    qq = I.index_queries_heads(5, keys, pos, heads)
+    cache, _, p = _build_gpu(keys, k=k, cand_cap=cand_cap, index_heads=heads)
+    gl, gn = _index_gpu(cache, None, p, qq, pos)
+    ol, on = O.index_heads(qq, pos, oc, k=k)
+    PT.assert_lists_match(gl, gn, ol, on, qq, pos, oc, k=k)
+
+
+def test_flat_index_heads_decode_and_single_head(tiny):
+    """Decode batches (stored-score path) with 4 heads, and identical heads,
+    which must give the single-head lists exactly."""
+    keys, _, _, oc = tiny
+    T = 4096
+    more = I.index_keys(0, T + 8, 32)
+    pos = np.arange(T, T + 8, dtype=np.int64)
+    qq = I.index_queries_heads(9, more, pos, 4)
+    cache, _, p = _build_gpu(keys, k=256, index_heads=4)
+    for nq in (1, 4):
+        gl, gn = _index_gpu(cache, None, p, qq[:nq], pos[:nq], decode=True)
+        ol, on = O.index_heads(qq[:nq], pos[:nq], oc, k=256)
+        PT.assert_lists_match(gl, gn, ol, on, qq[:nq], pos[:nq], oc, k=256)
+    same = np.ascontiguousarray(np.repeat(qq[:, :1], 4, axis=1))
+    p1 = lsa.lsa_default_params(k=256)
+    g4, n4 = _index_gpu(cache, None, p, same, pos)
+    g1, n1 = _index_gpu(cache, None, p1, np.ascontiguousarray(same[:, 0]), pos)
+    assert np.array_equal(n4, n1) and np.array_equal(g4, g1)
 
 
 def test_tree_build_bit_exact(tiny):

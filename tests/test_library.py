@@ -35,8 +35,8 @@ def test_library_builds_and_exports_header_symbols():
 
 def test_default_params_and_budgets():
     p = lsa.lsa_default_params()
-    assert (p.n_pool, p.block, p.n_buckets, p.cap_items, p.sink, p.window, p.k, p.beam, p.mode) == \
-        (4, 512, 64, 4, 4, 512, 4096, 32, 0)
+    assert (p.n_pool, p.block, p.n_buckets, p.cap_items, p.sink, p.window, p.k, p.beam, p.mode, p.index_heads) == \
+        (4, 512, 64, 4, 4, 512, 4096, 32, 0, 1)
     assert lsa.lsa_list_budget(p) == 4096 + 4 + 512 + 1
     assert lsa.lsa_top_buckets(p) == 1153
     assert lsa.lsa_top_buckets(lsa.lsa_default_params(k=2048)) == 641
@@ -121,6 +121,11 @@ def test_argument_errors_return_codes():
     tp = lsa.lsa_default_params(mode="tree")
     _expect(L.lsa_index_prefill(FAKE, FAKE, 10, C.byref(cache), None, FAKE, FAKE, Lmax, C.byref(tp), FAKE,
                                 1 << 40, None), -1)
+    # index heads: 1..16, Flat only
+    for bad_heads in (lsa.lsa_default_params(index_heads=0), lsa.lsa_default_params(index_heads=17),
+                      lsa.lsa_default_params(index_heads=2, mode="tree")):
+        _expect(L.lsa_index_prefill(FAKE, FAKE, 10, C.byref(cache), None, FAKE, FAKE, Lmax, C.byref(bad_heads),
+                                    FAKE, 1 << 40, None), -1)
     # nq = 0 is a no-op
     _expect(L.lsa_index_prefill(None, None, 0, C.byref(cache), None, None, None, Lmax, C.byref(p), None, 0,
                                 None), 0)
@@ -147,6 +152,9 @@ def test_workspace_queries():
     near = lambda nq, hq: sum(-(-x // 256) * 256 for x in (nq * hq * 128 * 4, nq * hq * 2 * 4, nq * 8, nq * 16))
     assert lsa.lsa_attention_workspace_bytes(131072, 32, 128, 2565) == near(131072, 32)
     assert lsa.lsa_attention_workspace_bytes(1, 32, 128, 4613) > 0        # decode: split the list
+    # index heads: the per-row arrays scale with heads, plus one merged set per query
+    p4 = lsa.lsa_default_params(k=2048, index_heads=4)
+    assert lsa.lsa_index_workspace_bytes(1000, 256, p4) > lsa.lsa_index_workspace_bytes(4000, 256, p)
     assert lsa.lsa_attention_workspace_bytes(1, 32, 64, 4613) == -1
 
 
