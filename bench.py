@@ -218,6 +218,42 @@ def measure_shrink(K: torch.Tensor, dev, hbm_peak: float):
             "flop": 2 * T * D * 64}
 
 
+def measure_index_heads(layer, keys_np, pos_np, wl: dict, dev, heads: int = 8, chunk: int = 16384):
+    """Multi-head Flat search (a bucket ranks by its best score over `heads`
+    index heads) for every prefill query of the workload, on the cache the
+    timed step built, outside the timed step: queries [nq, heads, 64] from
+    the seeded generator, indexed in chunks of `chunk` queries (the per-row
+    candidate slots of chunk x heads rows), one event pair around all
+    chunks."""
+    nq = len(pos_np)
+    chunk = min(chunk, nq)
+    qh = torch.from_numpy(I.index_queries_heads(11, keys_np, pos_np, heads)).to(dev)
+    pos = torch.from_numpy(pos_np).to(dev)
+    p = lsa.lsa_default_params(k=wl["k"], index_heads=heads)
+    ws = lsa.workspace(lsa.lsa_index_workspace_bytes(chunk, layer.cache.n_blocks, p), dev)
+    lists, lens = layer.lists, layer.lens
+
+    def run():
+        for a in range(0, nq, chunk):
+            b = min(nq, a + chunk)
+            lsa.lsa_index_prefill(qh[a:b], pos[a:b], layer.cache, None, lists[:b - a], lens[:b - a], p, ws)
+
+    ts = []
+    for r in range(4):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 1:
+            ts.append(e0.elapsed_time(e1))
+    ms = float(np.median(ts))
+    del ws, qh
+    torch.cuda.empty_cache()
+    return {"heads": heads, "queries": nq, "chunk": chunk, "ms": round(ms, 3),
+            "tokens_per_s": round(nq / (ms / 1e3), 1)}
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -309,6 +345,9 @@ def run_ours(args, world, rank, local):
         roofline["dram_frac"] = round(traffic / (attn_ms / 1e3) / 1e9 / pk["hbm"], 4)
 
     roofline["shrink"] = measure_shrink(K, dev, pk["hbm"])
+    index_heads = None
+    if wl["mode"] == "flat" and not args.no_heads:
+        index_heads = measure_index_heads(layer, keys_np, pos_np, wl, dev)
 
     # end to end: same calls, inputs from pinned host memory, output back to host
     e2e = None if args.no_e2e else run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
@@ -340,6 +379,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": int(launches),
         "clocks": clocks,
         "decode": decode,
+        "index_heads": index_heads,
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
@@ -573,6 +613,7 @@ def main():
     ap.add_argument("--mode", default=None, choices=["flat", "tree"], help="override the workload's search mode")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-heads", action="store_true", help="skip the multi-head Flat index measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()

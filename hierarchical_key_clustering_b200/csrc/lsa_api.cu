@@ -11,6 +11,8 @@
 #include "lsa_common.cuh"
 #include "lsa_kernels.h"
 
+static_assert(LSA_MAX_INDEX_HEADS == LSA_MAXHEADS, "index head limit of the header and the kernels");
+
 namespace {
 
 std::atomic<int64_t> g_launches{0};

@@ -21,6 +21,7 @@
 #define LSA_NSLOT 16
 #define LSA_RUN 128
 #define LSA_HEAD 128
+#define LSA_MAXHEADS 16  /* index heads per token (multi-head Flat search) */
 #define LSA_FULL 0xffffffffu
 
 namespace lsa {

@@ -1151,29 +1151,36 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
 // listed it, with that very score.  Keeping every listed bucket once, with
 // the largest score any head listed for it, and cutting at the P-th largest
 // of those values keeps exactly the top P: a kept value falls short of a
-// bucket's best only for buckets outside the top P.  The kept buckets go out
-// as one-bucket entries with tau = -inf, for the unchanged expansion.
-// The union is deduplicated in a shared-memory hash table (linear probing,
-// at most 3/4 full).  A query whose rows overflowed their entry slots, whose
-// union does not fit the table, or whose cut keeps more than the expansion's
-// slots (ties) is redone exactly: every visible bucket scored for every head
-// on the CUDA cores, radix select, ties in ascending bucket order.
+// bucket's best only for buckets outside the top P.  Scores below
+// tau* = max over heads of tau_h are dropped first: every head's top P score
+// at least tau_h, so at least P buckets have a best score >= tau_h for every
+// h, and the P-th best is >= tau*.
+// The kept buckets go out as one-bucket entries with tau = -inf, for the
+// unchanged expansion.  The union is deduplicated in a shared-memory hash
+// table (linear probing, at most 3/4 full).  A query whose rows overflowed
+// their entry slots, whose union does not fit the table, or whose cut keeps
+// more than the expansion's slots (ties) is redone exactly: every visible
+// bucket scored for every head on the CUDA cores, radix select, ties in
+// ascending bucket order.
 constexpr int HM_THREADS = 512;
 constexpr int HM_MAX_SLOTS = 25600;  // 200 KB of table
+constexpr int HM_UNROLL = 4;         // entries a thread loads before using them
 
-// Table slots for a launch: about 3 x heads x P (a head lists ~1.2-1.45 P
-// buckets on the measured workloads), a multiple of 512, at most HM_MAX_SLOTS.
+// Table slots for a launch: about 2 x heads x P (a head lists ~1.2 P
+// buckets at or above tau* on the measured workloads), a multiple of 512, at
+// most HM_MAX_SLOTS.
 inline int heads_merge_slots(int heads, int P)
 {
-    const int64_t want = ((int64_t)3 * heads * P + 511) / 512 * 512;
+    const int64_t want = ((int64_t)2 * heads * P + 511) / 512 * 512;
     return (int)(want < HM_MAX_SLOTS ? (want < 512 ? 512 : want) : HM_MAX_SLOTS);
 }
 
-// Insert bucket `id` with ordered score v; returns 1 if the id was new.
+// Insert bucket `id` with ordered score v: 1 if the id was new, 0 if it was
+// there, -1 if the table is full.
 __device__ __forceinline__ int hash_insert(int32_t *hkey, uint32_t *hval, int TS, int32_t id, uint32_t v)
 {
     uint32_t s = __umulhi((uint32_t)id * 0x9E3779B1u, (uint32_t)TS);
-    for (int n = 0; n < TS; ++n) {  // ends at a free slot: the table has more slots than ids
+    for (int n = 0; n < TS; ++n) {
         const int32_t prev = atomicCAS(&hkey[s], -1, id);
         if (prev == -1 || prev == id) {
             atomicMax(&hval[s], v);
@@ -1181,102 +1188,169 @@ __device__ __forceinline__ int hash_insert(int32_t *hkey, uint32_t *hval, int TS
         }
         s = (s + 1 == (uint32_t)TS) ? 0u : s + 1;
     }
-    return 0;
+    return -1;
 }
 
-__global__ void __launch_bounds__(HM_THREADS) k_heads_merge(int heads, int P, int TSMAX,
-                                                           const uint16_t *__restrict__ cbf, IndexWs ws, IndexWs m)
+// Histogram bin of a merged value over [lo, lo + 256 / scale]; the same
+// rounded operations in the counting and the keeping pass.
+__device__ __forceinline__ int merge_bin(float v, float lo, float scale)
+{
+    return min(255, max(0, __float2int_rz(__fmul_rn(__fsub_rn(v, lo), scale))));
+}
+
+__global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P, int TS,
+                                                              const uint16_t *__restrict__ cbf, IndexWs ws, IndexWs m)
 {
     pdl_wait();
     pdl_release();
     extern __shared__ uint32_t hsm[];
     int32_t *hkey = reinterpret_cast<int32_t *>(hsm);  // [TS] bucket id, -1 = empty
-    uint32_t *hval = hsm + TSMAX;                      // [TS] f2ord of its best listed score
-    float *qf = reinterpret_cast<float *>(hsm);        // [heads, 64] (exact path only)
+    uint32_t *hval = hsm + TS;                         // [TS] f2ord of its best listed score
     __shared__ int hist[256];
     __shared__ int sh[4];
-    __shared__ int wsum[HM_THREADS / 32];
-    __shared__ int s_listed, s_over, s_uniq, s_out, s_exact;
+    __shared__ int s_off[LSA_MAXHEADS + 1];  // entry offsets of the heads' rows, flattened
+    __shared__ float s_tstar;
+    __shared__ int s_over, s_full, s_uniq, s_out, s_exact, s_bstar, s_keep;
+    __shared__ uint32_t s_vmin, s_vmax;
     const int64_t q = blockIdx.x;
     const int64_t r0 = q * heads;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int t = threadIdx.x, lane = t & 31;
     const float NEG = __int_as_float(0xff800000);
     const int KC = m.cap;
-    const int64_t N = (int64_t)ws.horizon[r0] * LSA_NBKT;
     float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * KC;
     int32_t *og = m.cand_g + q * KC;
     if (t == 0) {
-        s_listed = 0;
-        s_over = 0;
+        int o = 0, over = 0;
+        float ts = NEG;
+        for (int h = 0; h < heads; ++h) {
+            const int ne = ws.cnt[r0 + h];
+            over |= ne > ws.cap;  // the row lost entries: exact path
+            s_off[h] = o;
+            o += min(ne, ws.cap);
+            ts = fmaxf(ts, ws.tau[r0 + h]);
+        }
+        s_off[heads] = o;
+        s_tstar = ts;
+        s_over = over;
+        s_full = 0;
         s_uniq = 0;
         s_out = 0;
+        s_vmin = ~0u;
+        s_vmax = 0u;
+    }
+    for (int i = t; i < TS; i += HM_THREADS) {
+        hkey[i] = -1;
+        hval[i] = 0u;
     }
     __syncthreads();
+    const int E = s_off[heads];
+    const float tstar = s_tstar;
 
-    // 1. scores the heads listed
-    int my = 0;
-    for (int h = 0; h < heads; ++h) {
-        const int64_t r = r0 + h;
-        const int ne = ws.cnt[r];
-        if (ne > ws.cap) {  // the row lost entries: exact path
-            s_over = 1;
-            continue;
-        }
-        const float tau = ws.tau[r];
-        const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + r * ws.cap;
-        for (int i = t; i < ne; i += HM_THREADS) {
-            const float4 s4 = c4[i];
-            my += (s4.x >= tau && s4.x > NEG) + (s4.y >= tau && s4.y > NEG) + (s4.z >= tau && s4.z > NEG) +
-                  (s4.w >= tau && s4.w > NEG);
-        }
-    }
+    // 1. union of the scores at or above tau*, best score per bucket
+    int fresh = 0, full = 0;
+    uint32_t vmin = ~0u, vmax = 0u;
+    if (!s_over) {
+        for (int i0 = 0; i0 < E; i0 += HM_THREADS * HM_UNROLL) {
+            float4 sv[HM_UNROLL];
+            int32_t g[HM_UNROLL];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) my += __shfl_xor_sync(LSA_FULL, my, o);
-    if (lane == 0 && my) atomicAdd(&s_listed, my);
-    __syncthreads();
-    const int listed = s_listed;
-    if (t == 0) s_exact = s_over || (int64_t)listed * 4 > (int64_t)TSMAX * 3;
-    __syncthreads();
-
-    // 2. union with the best listed score per bucket, cut at the P-th value
-    if (!s_exact) {
-        const int TS = min(TSMAX, max(2 * listed, 64));
-        for (int i = t; i < TS; i += HM_THREADS) {
-            hkey[i] = -1;
-            hval[i] = 0u;
-        }
-        __syncthreads();
-        int fresh = 0;
-        for (int h = 0; h < heads; ++h) {
-            const int64_t r = r0 + h;
-            const int ne = ws.cnt[r];
-            const float tau = ws.tau[r];
-            const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + r * ws.cap;
-            const int32_t *cg = ws.cand_g + r * ws.cap;
-            for (int i = t; i < ne; i += HM_THREADS) {
-                const float4 s4 = c4[i];
-                const int32_t g = cg[i];
-                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            for (int u = 0; u < HM_UNROLL; ++u) {
+                const int i = i0 + u * HM_THREADS + t;
+                sv[u] = make_float4(NEG, NEG, NEG, NEG);
+                g[u] = 0;
+                if (i < E) {
+                    int h = 0;
+                    while (i >= s_off[h + 1]) ++h;
+                    const int64_t j = (r0 + h) * ws.cap + (i - s_off[h]);
+                    sv[u] = reinterpret_cast<const float4 *>(ws.cand4)[j];
+                    g[u] = ws.cand_g[j];
+                }
+            }
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (sv[e] >= tau && sv[e] > NEG) fresh += hash_insert(hkey, hval, TS, g + e, f2ord(sv[e]));
+            for (int u = 0; u < HM_UNROLL; ++u) {
+                const float x[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (x[e] >= tstar && x[e] > NEG) {
+                        const uint32_t v = f2ord(x[e]);
+                        const int r = hash_insert(hkey, hval, TS, g[u] + e, v);
+                        fresh += r > 0;
+                        full |= r < 0;
+                        vmin = min(vmin, v);
+                        vmax = max(vmax, v);
+                    }
+                }
             }
         }
+    }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) fresh += __shfl_xor_sync(LSA_FULL, fresh, o);
-        if (lane == 0 && fresh) atomicAdd(&s_uniq, fresh);
-        __syncthreads();
-        // keep everything when it fits the expansion's slots, else the P-th
-        // largest value and every bucket at or above it
+    for (int o = 16; o > 0; o >>= 1) {
+        fresh += __shfl_xor_sync(LSA_FULL, fresh, o);
+        full |= __shfl_xor_sync(LSA_FULL, full, o);
+        vmin = min(vmin, __shfl_xor_sync(LSA_FULL, vmin, o));
+        vmax = max(vmax, __shfl_xor_sync(LSA_FULL, vmax, o));
+    }
+    if (lane == 0) {
+        if (fresh) atomicAdd(&s_uniq, fresh);
+        if (full) s_full = 1;
+        atomicMin(&s_vmin, vmin);
+        atomicMax(&s_vmax, vmax);
+    }
+    for (int i = t; i < 256; i += HM_THREADS) hist[i] = 0;
+    __syncthreads();
+    if (t == 0) s_exact = s_over | s_full;
+    const int U = s_uniq;
+    __syncthreads();
+
+    // 2. the cut: all of a small union; else every bucket from the histogram
+    //    bin holding the P-th best value up, which holds the top P; a radix
+    //    select to the P-th value itself when that is more than the slots
+    if (!s_exact) {
+        const float lo = ord2f(s_vmin), hi = ord2f(s_vmax);
+        const float scale = hi > lo ? 256.0f / (hi - lo) : 0.0f;
+        int bstar = 0;
         uint32_t cut = 0u;
-        if (s_uniq > KC) {
-            auto get = [&](int64_t i) { return hkey[i] >= 0 ? ord2f(hval[i]) : NEG; };
-            cut = block_select_kth_largest(TS, P, get, hist, sh);
+        if (U > KC) {
+            for (int i = t; i < TS; i += HM_THREADS)
+                if (hkey[i] >= 0) atomicAdd(&hist[merge_bin(ord2f(hval[i]), lo, scale)], 1);
+            __syncthreads();
+            if (t < 32) {  // warp 0: lane l owns bins 255-8l .. 248-8l
+                int c8 = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) c8 += hist[255 - 8 * lane - e];
+                int incl = c8;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(LSA_FULL, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const int excl = incl - c8;
+                if (excl < P && P <= incl) {
+                    int acc = excl;
+                    for (int e = 0; e < 8; ++e) {
+                        const int d = 255 - 8 * lane - e;
+                        acc += hist[d];
+                        if (acc >= P) {
+                            s_bstar = d;
+                            s_keep = acc;
+                            break;
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+            bstar = s_bstar;
+            if (s_keep > KC) {  // block-uniform: too many at the boundary bin
+                auto get = [&](int64_t i) { return hkey[i] >= 0 ? ord2f(hval[i]) : NEG; };
+                cut = block_select_kth_largest(TS, P, get, hist, sh);
+                bstar = -1;
+            }
         }
         for (int i = t; i < TS; i += HM_THREADS) {
             const int32_t id = hkey[i];
             const uint32_t v = hval[i];
-            if (id >= 0 && v >= cut) {
+            const bool take = id >= 0 && (U <= KC || (bstar >= 0 ? merge_bin(ord2f(v), lo, scale) >= bstar : v >= cut));
+            if (take) {
                 const int j = atomicAdd(&s_out, 1);
                 if (j < KC) {
                     o4[j] = make_float4(ord2f(v), NEG, NEG, NEG);
@@ -1286,68 +1360,88 @@ __global__ void __launch_bounds__(HM_THREADS) k_heads_merge(int heads, int P, in
         }
         __syncthreads();
         if (t == 0 && s_out > KC) s_exact = 1;
-        __syncthreads();
-    }
-
-    // 3. exact path
-    if (s_exact) {
-        for (int i = t; i < heads * LSA_D; i += HM_THREADS) qf[i] = bf_bits2f(ws.qhat[r0 * LSA_D + i]);
-        if (t == 0) s_out = 0;
-        __syncthreads();
-        auto best = [&](int64_t b) {
-            const uint16_t *c = cbf + b * LSA_D;
-            float s = dot_bf16_row(qf, c);
-            for (int h = 1; h < heads; ++h) s = fmaxf(s, dot_bf16_row(qf + h * LSA_D, c));
-            return s;
-        };
-        if (N <= P) {
-            for (int64_t b = t; b < N; b += HM_THREADS) {
-                o4[b] = make_float4(best(b), NEG, NEG, NEG);
-                og[b] = (int32_t)b;
-            }
-            if (t == 0) s_out = (int)N;
-        } else {
-            const float ts = ord2f(block_select_kth_largest(N, P, best, hist, sh));
-            for (int64_t b = t; b < N; b += HM_THREADS) {
-                const float s = best(b);
-                if (s > ts) {
-                    const int j = atomicAdd(&s_out, 1);  // fewer than P buckets score above ts
-                    o4[j] = make_float4(s, NEG, NEG, NEG);
-                    og[j] = (int32_t)b;
-                }
-            }
-            __syncthreads();
-            // ties at ts in ascending bucket order, up to P in all
-            for (int64_t base = 0; base < N; base += HM_THREADS) {
-                if (s_out >= P) break;  // block-uniform (read after a barrier)
-                const int64_t b = base + t;
-                const bool tie = (b < N) && (best(b) == ts);
-                const unsigned bal = __ballot_sync(LSA_FULL, tie);
-                if (lane == 0) wsum[warp] = __popc(bal);
-                __syncthreads();
-                int before = s_out;
-                for (int w = 0; w < warp; ++w) before += wsum[w];
-                before += __popc(bal & ((1u << lane) - 1u));
-                if (tie && before < P) {
-                    o4[before] = make_float4(ts, NEG, NEG, NEG);
-                    og[before] = (int32_t)b;
-                }
-                __syncthreads();
-                if (t == 0) {
-                    int tot = 0;
-                    for (int w = 0; w < HM_THREADS / 32; ++w) tot += wsum[w];
-                    s_out = min(P, s_out + tot);
-                }
-                __syncthreads();
-            }
-        }
     }
     __syncthreads();
     if (t == 0) {
-        m.cnt[q] = s_out;
+        m.cnt[q] = s_exact ? -1 : s_out;  // -1: k_heads_exact redoes the query
         m.tau[q] = NEG;
         m.horizon[q] = ws.horizon[r0];
     }
+}
+
+// The exact path of the merge, for the queries k_heads_merge marked (cnt -1):
+// the top P buckets by best head score, each score recomputed on the CUDA
+// cores, ties at the P-th score in ascending bucket order.
+__global__ void __launch_bounds__(HM_THREADS) k_heads_exact(int heads, int P, const uint16_t *__restrict__ cbf,
+                                                           IndexWs ws, IndexWs m)
+{
+    pdl_wait();
+    pdl_release();
+    const int64_t q = blockIdx.x;
+    if (m.cnt[q] >= 0) return;  // block-uniform
+    __shared__ float qf[LSA_MAXHEADS * LSA_D];
+    __shared__ int hist[256];
+    __shared__ int sh[4];
+    __shared__ int wsum[HM_THREADS / 32];
+    __shared__ int s_out;
+    const int64_t r0 = q * heads;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const float NEG = __int_as_float(0xff800000);
+    const int64_t N = (int64_t)ws.horizon[r0] * LSA_NBKT;
+    float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * m.cap;
+    int32_t *og = m.cand_g + q * m.cap;
+    for (int i = t; i < heads * LSA_D; i += HM_THREADS) qf[i] = bf_bits2f(ws.qhat[r0 * LSA_D + i]);
+    if (t == 0) s_out = 0;
+    __syncthreads();
+    auto best = [&](int64_t b) {
+        const uint16_t *c = cbf + b * LSA_D;
+        float s = dot_bf16_row(qf, c);
+        for (int h = 1; h < heads; ++h) s = fmaxf(s, dot_bf16_row(qf + h * LSA_D, c));
+        return s;
+    };
+    if (N <= P) {
+        for (int64_t b = t; b < N; b += HM_THREADS) {
+            o4[b] = make_float4(best(b), NEG, NEG, NEG);
+            og[b] = (int32_t)b;
+        }
+        if (t == 0) s_out = (int)N;
+    } else {
+        const float ts = ord2f(block_select_kth_largest(N, P, best, hist, sh));
+        for (int64_t b = t; b < N; b += HM_THREADS) {
+            const float s = best(b);
+            if (s > ts) {
+                const int j = atomicAdd(&s_out, 1);  // fewer than P buckets score above ts
+                o4[j] = make_float4(s, NEG, NEG, NEG);
+                og[j] = (int32_t)b;
+            }
+        }
+        __syncthreads();
+        // ties at ts in ascending bucket order, up to P in all
+        for (int64_t base = 0; base < N; base += HM_THREADS) {
+            if (s_out >= P) break;  // block-uniform (read after a barrier)
+            const int64_t b = base + t;
+            const bool tie = (b < N) && (best(b) == ts);
+            const unsigned bal = __ballot_sync(LSA_FULL, tie);
+            if (lane == 0) wsum[warp] = __popc(bal);
+            __syncthreads();
+            int before = s_out;
+            for (int w = 0; w < warp; ++w) before += wsum[w];
+            before += __popc(bal & ((1u << lane) - 1u));
+            if (tie && before < P) {
+                o4[before] = make_float4(ts, NEG, NEG, NEG);
+                og[before] = (int32_t)b;
+            }
+            __syncthreads();
+            if (t == 0) {
+                int tot = 0;
+                for (int w = 0; w < HM_THREADS / 32; ++w) tot += wsum[w];
+                s_out = min(P, s_out + tot);
+            }
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    if (t == 0) m.cnt[q] = s_out;
 }
 
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks)
@@ -1429,13 +1523,16 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
         count_launches(1);
     }
     if (merged) {  // several index heads: one candidate set per query
-        const int TSMAX = heads_merge_slots(heads, a.P);
-        const size_t smh = (size_t)TSMAX * 8;
+        const int TS = heads_merge_slots(heads, a.P);
+        const size_t smh = (size_t)TS * 8;
         cudaFuncSetAttribute(k_heads_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smh);
-        if ((e = launch_k(small, k_heads_merge, dim3((unsigned)a.nq), dim3(HM_THREADS), smh, st, heads, a.P, TSMAX,
+        if ((e = launch_k(small, k_heads_merge, dim3((unsigned)a.nq), dim3(HM_THREADS), smh, st, heads, a.P, TS,
                           a.centroid_bf16, ws, *merged)) != cudaSuccess)
             return e;
-        count_launches(1);
+        if ((e = launch_k(small, k_heads_exact, dim3((unsigned)a.nq), dim3(HM_THREADS), 0, st, heads, a.P,
+                          a.centroid_bf16, ws, *merged)) != cudaSuccess)
+            return e;
+        count_launches(2);
     }
     const IndexWs &ex = merged ? *merged : ws;
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;

@@ -69,7 +69,8 @@ def _check_tree(gtree, otree):
     assert np.array_equal(v["centroid_bf16"].view(np.uint16), otree.centroid_bf16)
 
 
-def test_flat_128k_cache_index_attention():
+@pytest.fixture(scope="module")
+def big128k():
     _need_gpu()
     wl = I.WORKLOADS["flat_128k"]
     T, k = wl["T"], wl["k"]
@@ -79,6 +80,13 @@ def test_flat_128k_cache_index_attention():
     cache = lsa.Cache(T)
     lsa.lsa_build_cache(PT.to_dev(keys), 0, T, cache, p)
     torch.cuda.synchronize()
+    return wl, keys, oc, cache
+
+
+def test_flat_128k_cache_index_attention(big128k):
+    wl, keys, oc, cache = big128k
+    T, k = wl["T"], wl["k"]
+    p = lsa.lsa_default_params(k=k)
     PT.assert_cache_equal(PT.cache_to_numpy(cache, T), oc)
     # all queries through the GPU (the benchmark's launch), 600 sampled for the oracle
     pos = np.arange(T, dtype=np.int64)
@@ -90,6 +98,32 @@ def test_flat_128k_cache_index_attention():
     PT.assert_lists_match(lists_d[torch.from_numpy(sel).cuda()].cpu().numpy(),
                           lens_d[torch.from_numpy(sel).cuda()].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
     _attention_sampled(lists_d, lens_d, sel[::10], T, wl["hq"], wl["hkv"], seed=1)
+
+
+def test_flat_128k_index_heads(big128k):
+    """Multi-head Flat search with 8 index heads over every position, in the
+    benchmark's launches (chunks of 16384 queries); sampled queries against
+    the oracle."""
+    wl, keys, oc, cache = big128k
+    T, k, heads, chunk = wl["T"], wl["k"], 8, 16384
+    p = lsa.lsa_default_params(k=k, index_heads=heads)
+    pos = np.arange(T, dtype=np.int64)
+    q = I.index_queries_heads(11, keys, pos, heads)
+    Lmax = lsa.lsa_list_budget(p)
+    lists = torch.empty((T, Lmax), dtype=torch.int32, device="cuda")
+    lens = torch.empty((T,), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_index_workspace_bytes(chunk, cache.n_blocks, p))
+    qd, pd = PT.to_dev(q), PT.to_dev(pos)
+    for a in range(0, T, chunk):
+        lsa.lsa_index_prefill(qd[a:a + chunk], pd[a:a + chunk], cache, None, lists[a:a + chunk], lens[a:a + chunk],
+                              p, ws)
+    torch.cuda.synchronize()
+    del ws
+    sel = np.unique(np.concatenate([np.linspace(0, T - 1, 190).astype(np.int64),
+                                    [0, 511, 512, 1024, 16383, 16384, 65536, T - 1]]))
+    ol, on = O.index_heads(q[sel], pos[sel], oc, k=k)
+    ix = torch.from_numpy(sel).cuda()
+    PT.assert_lists_match(lists[ix].cpu().numpy(), lens[ix].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
 
 
 @pytest.fixture(scope="module")
