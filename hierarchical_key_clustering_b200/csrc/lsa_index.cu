@@ -1198,103 +1198,142 @@ __device__ __forceinline__ int merge_bin(float v, float lo, float scale)
     return min(255, max(0, __float2int_rz(__fmul_rn(__fsub_rn(v, lo), scale))));
 }
 
-__global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P, int TS,
+__global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P, int TSMAX,
                                                               const uint16_t *__restrict__ cbf, IndexWs ws, IndexWs m)
 {
     pdl_wait();
     pdl_release();
     extern __shared__ uint32_t hsm[];
     int32_t *hkey = reinterpret_cast<int32_t *>(hsm);  // [TS] bucket id, -1 = empty
-    uint32_t *hval = hsm + TS;                         // [TS] f2ord of its best listed score
+    uint32_t *hval = hsm + TSMAX;                      // [TS] f2ord of its best listed score
     __shared__ int hist[256];
     __shared__ int sh[4];
     __shared__ int s_off[LSA_MAXHEADS + 1];  // entry offsets of the heads' rows, flattened
     __shared__ float s_tstar;
     __shared__ int s_over, s_full, s_uniq, s_out, s_exact, s_bstar, s_keep;
     __shared__ uint32_t s_vmin, s_vmax;
+    __shared__ uint2 wq[HM_THREADS / 32][64];  // per warp: kept (bucket, value) pairs waiting to be inserted
     const int64_t q = blockIdx.x;
     const int64_t r0 = q * heads;
-    const int t = threadIdx.x, lane = t & 31;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float NEG = __int_as_float(0xff800000);
     const int KC = m.cap;
     float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * KC;
     int32_t *og = m.cand_g + q * KC;
-    if (t == 0) {
-        int o = 0, over = 0;
-        float ts = NEG;
-        for (int h = 0; h < heads; ++h) {
-            const int ne = ws.cnt[r0 + h];
-            over |= ne > ws.cap;  // the row lost entries: exact path
-            s_off[h] = o;
-            o += min(ne, ws.cap);
-            ts = fmaxf(ts, ws.tau[r0 + h]);
+    if (t < 32) {  // warp 0, lane h: head h's entry count and threshold
+        const int ne = lane < heads ? ws.cnt[r0 + lane] : 0;
+        float ts = lane < heads ? ws.tau[r0 + lane] : NEG;
+        const unsigned over = __ballot_sync(LSA_FULL, ne > ws.cap);  // a row lost entries: exact path
+        int incl = min(ne, ws.cap);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(LSA_FULL, incl, o);
+            if (lane >= o) incl += y;
+            ts = fmaxf(ts, __shfl_xor_sync(LSA_FULL, ts, o));
         }
-        s_off[heads] = o;
-        s_tstar = ts;
-        s_over = over;
-        s_full = 0;
-        s_uniq = 0;
-        s_out = 0;
-        s_vmin = ~0u;
-        s_vmax = 0u;
-    }
-    for (int i = t; i < TS; i += HM_THREADS) {
-        hkey[i] = -1;
-        hval[i] = 0u;
+        if (lane < heads) s_off[lane + 1] = incl;
+        if (lane == 0) {
+            s_off[0] = 0;
+            s_tstar = ts;
+            s_over = over != 0u;
+            s_out = 0;
+        }
     }
     __syncthreads();
     const int E = s_off[heads];
     const float tstar = s_tstar;
+    // a query's table: 1.5 slots per entry (entries hold about one kept score
+    // each); one that fills is redone once with all of the launch's slots,
+    // and a union that fills those takes the exact path
+    int TS = min(TSMAX, max(64, E + E / 2));
+    for (;;) {  // block-uniform, at most two rounds
+        for (int i = t; i < TS; i += HM_THREADS) {
+            hkey[i] = -1;
+            hval[i] = 0u;
+        }
+        if (t == 0) {
+            s_full = 0;
+            s_uniq = 0;
+            s_vmin = ~0u;
+            s_vmax = 0u;
+        }
+        __syncthreads();
 
-    // 1. union of the scores at or above tau*, best score per bucket
-    int fresh = 0, full = 0;
-    uint32_t vmin = ~0u, vmax = 0u;
-    if (!s_over) {
-        for (int i0 = 0; i0 < E; i0 += HM_THREADS * HM_UNROLL) {
-            float4 sv[HM_UNROLL];
-            int32_t g[HM_UNROLL];
+        // 1. union of the scores at or above tau*, best score per bucket
+        int fresh = 0, full = 0, qn = 0;
+        uint32_t vmin = ~0u, vmax = 0u;
+        if (!s_over) {
+            for (int i0 = 0; i0 < E; i0 += HM_THREADS * HM_UNROLL) {
+                float4 sv[HM_UNROLL];
+                int32_t g[HM_UNROLL];
 #pragma unroll
-            for (int u = 0; u < HM_UNROLL; ++u) {
-                const int i = i0 + u * HM_THREADS + t;
-                sv[u] = make_float4(NEG, NEG, NEG, NEG);
-                g[u] = 0;
-                if (i < E) {
-                    int h = 0;
-                    while (i >= s_off[h + 1]) ++h;
-                    const int64_t j = (r0 + h) * ws.cap + (i - s_off[h]);
-                    sv[u] = reinterpret_cast<const float4 *>(ws.cand4)[j];
-                    g[u] = ws.cand_g[j];
+                for (int u = 0; u < HM_UNROLL; ++u) {
+                    const int i = i0 + u * HM_THREADS + t;
+                    sv[u] = make_float4(NEG, NEG, NEG, NEG);
+                    g[u] = 0;
+                    if (i < E) {
+                        int h = 0;
+                        while (i >= s_off[h + 1]) ++h;
+                        const int64_t j = (r0 + h) * ws.cap + (i - s_off[h]);
+                        sv[u] = reinterpret_cast<const float4 *>(ws.cand4)[j];
+                        g[u] = ws.cand_g[j];
+                    }
                 }
-            }
+                // kept scores are queued per warp and inserted 32 at a time, one
+                // per lane (about one score in four is kept)
 #pragma unroll
-            for (int u = 0; u < HM_UNROLL; ++u) {
-                const float x[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+                for (int u = 0; u < HM_UNROLL; ++u) {
+                    const float x[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if (x[e] >= tstar && x[e] > NEG) {
-                        const uint32_t v = f2ord(x[e]);
-                        const int r = hash_insert(hkey, hval, TS, g[u] + e, v);
-                        fresh += r > 0;
-                        full |= r < 0;
-                        vmin = min(vmin, v);
-                        vmax = max(vmax, v);
+                    for (int e = 0; e < 4; ++e) {
+                        const bool k = x[e] >= tstar && x[e] > NEG;
+                        const unsigned bal = __ballot_sync(LSA_FULL, k);
+                        if (k) {
+                            const uint32_t v = f2ord(x[e]);
+                            wq[warp][qn + __popc(bal & ((1u << lane) - 1u))] = make_uint2((uint32_t)(g[u] + e), v);
+                            vmin = min(vmin, v);
+                            vmax = max(vmax, v);
+                        }
+                        qn += __popc(bal);
+                        if (qn >= 32) {  // warp-uniform
+                            __syncwarp();
+                            const uint2 w = wq[warp][lane];
+                            const int r = hash_insert(hkey, hval, TS, (int32_t)w.x, w.y);
+                            fresh += r > 0;
+                            full |= r < 0;
+                            __syncwarp();
+                            if (lane < qn - 32) wq[warp][lane] = wq[warp][32 + lane];
+                            __syncwarp();
+                            qn -= 32;
+                        }
                     }
                 }
             }
+            __syncwarp();
+            if (lane < qn) {
+                const uint2 w = wq[warp][lane];
+                const int r = hash_insert(hkey, hval, TS, (int32_t)w.x, w.y);
+                fresh += r > 0;
+                full |= r < 0;
+            }
         }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        fresh += __shfl_xor_sync(LSA_FULL, fresh, o);
-        full |= __shfl_xor_sync(LSA_FULL, full, o);
-        vmin = min(vmin, __shfl_xor_sync(LSA_FULL, vmin, o));
-        vmax = max(vmax, __shfl_xor_sync(LSA_FULL, vmax, o));
-    }
-    if (lane == 0) {
-        if (fresh) atomicAdd(&s_uniq, fresh);
-        if (full) s_full = 1;
-        atomicMin(&s_vmin, vmin);
-        atomicMax(&s_vmax, vmax);
+        for (int o = 16; o > 0; o >>= 1) {
+            fresh += __shfl_xor_sync(LSA_FULL, fresh, o);
+            full |= __shfl_xor_sync(LSA_FULL, full, o);
+            vmin = min(vmin, __shfl_xor_sync(LSA_FULL, vmin, o));
+            vmax = max(vmax, __shfl_xor_sync(LSA_FULL, vmax, o));
+        }
+        if (lane == 0) {
+            if (fresh) atomicAdd(&s_uniq, fresh);
+            if (full) s_full = 1;
+            atomicMin(&s_vmin, vmin);
+            atomicMax(&s_vmax, vmax);
+        }
+        __syncthreads();
+        if (!s_full || TS == TSMAX) break;
+        TS = TSMAX;
+        __syncthreads();  // s_full read by every thread before the next round resets it
     }
     for (int i = t; i < 256; i += HM_THREADS) hist[i] = 0;
     __syncthreads();
@@ -1369,24 +1408,14 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
     }
 }
 
-// The exact path of the merge, for the queries k_heads_merge marked (cnt -1):
-// the top P buckets by best head score, each score recomputed on the CUDA
-// cores, ties at the P-th score in ascending bucket order.
-__global__ void __launch_bounds__(HM_THREADS) k_heads_exact(int heads, int P, const uint16_t *__restrict__ cbf,
-                                                           IndexWs ws, IndexWs m)
+// One marked query of k_heads_exact, all threads of the block.
+__device__ void heads_exact_query(int64_t q, int heads, int P, const uint16_t *__restrict__ cbf, const IndexWs &ws,
+                                  const IndexWs &m, float *qf, int *hist, int *sh, int *wsum, int &s_out)
 {
-    pdl_wait();
-    pdl_release();
-    const int64_t q = blockIdx.x;
-    if (m.cnt[q] >= 0) return;  // block-uniform
-    __shared__ float qf[LSA_MAXHEADS * LSA_D];
-    __shared__ int hist[256];
-    __shared__ int sh[4];
-    __shared__ int wsum[HM_THREADS / 32];
-    __shared__ int s_out;
     const int64_t r0 = q * heads;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float NEG = __int_as_float(0xff800000);
+
     const int64_t N = (int64_t)ws.horizon[r0] * LSA_NBKT;
     float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * m.cap;
     int32_t *og = m.cand_g + q * m.cap;
@@ -1442,8 +1471,44 @@ __global__ void __launch_bounds__(HM_THREADS) k_heads_exact(int heads, int P, co
     }
     __syncthreads();
     if (t == 0) m.cnt[q] = s_out;
+    __syncthreads();
 }
 
+
+// The exact path of the merge, for the queries k_heads_merge marked (cnt -1):
+// the top P buckets by best head score, each score recomputed on the CUDA
+// cores, ties at the P-th score in ascending bucket order.  Each CTA scans
+// the flags of its share of the queries and redoes the marked ones.
+__global__ void __launch_bounds__(HM_THREADS) k_heads_exact(int64_t nq, int heads, int P,
+                                                           const uint16_t *__restrict__ cbf, IndexWs ws, IndexWs m)
+{
+    pdl_wait();
+    pdl_release();
+    __shared__ float qf[LSA_MAXHEADS * LSA_D];
+    __shared__ int hist[256];
+    __shared__ int sh[4];
+    __shared__ int wsum[HM_THREADS / 32];
+    __shared__ int s_out, s_n;
+    __shared__ int ql[HM_THREADS];  // marked queries of the current range, base-relative
+    const int t = threadIdx.x, lane = t & 31;
+    const int64_t per = (nq + gridDim.x - 1) / gridDim.x;
+    const int64_t qa = (int64_t)blockIdx.x * per, qb = min(nq, qa + per);
+    for (int64_t base = qa; base < qb; base += HM_THREADS) {
+        if (t == 0) s_n = 0;
+        __syncthreads();
+        const bool mark = base + t < qb && m.cnt[base + t] < 0;
+        const unsigned bal = __ballot_sync(LSA_FULL, mark);
+        int at = 0;
+        if (lane == 0 && bal) at = atomicAdd(&s_n, __popc(bal));
+        at = __shfl_sync(LSA_FULL, at, 0);
+        if (mark) ql[at + __popc(bal & ((1u << lane) - 1u))] = t;
+        __syncthreads();
+        const int n = s_n;
+        for (int k = 0; k < n; ++k)  // block-uniform
+            heads_exact_query(base + ql[k], heads, P, cbf, ws, m, qf, hist, sh, wsum, s_out);
+        __syncthreads();
+    }
+}
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks)
 {
     return rank_expand_smem(cap, (int)((n_blocks + 31) / 32) + 1);
@@ -1529,8 +1594,9 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
         if ((e = launch_k(small, k_heads_merge, dim3((unsigned)a.nq), dim3(HM_THREADS), smh, st, heads, a.P, TS,
                           a.centroid_bf16, ws, *merged)) != cudaSuccess)
             return e;
-        if ((e = launch_k(small, k_heads_exact, dim3((unsigned)a.nq), dim3(HM_THREADS), 0, st, heads, a.P,
-                          a.centroid_bf16, ws, *merged)) != cudaSuccess)
+        const unsigned xg = (unsigned)min((int64_t)n_sm, a.nq);
+        if ((e = launch_k(small, k_heads_exact, dim3(xg), dim3(HM_THREADS), 0, st, a.nq, heads, a.P, a.centroid_bf16,
+                          ws, *merged)) != cudaSuccess)
             return e;
         count_launches(2);
     }
