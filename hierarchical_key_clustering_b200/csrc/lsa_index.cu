@@ -21,6 +21,10 @@
 // The expansion kernel keeps the scores >= tau, ranks them by (score desc,
 // id asc) and expands them; a query whose entries or candidates overflow
 // their slots is redone exactly there (radix select on recomputed scores).
+//
+// Several index heads per token (N-LSA's selection by the best head score):
+// the Flat passes run over one row per (query, head), and k_heads_merge
+// turns each query's rows into one candidate set for the same expansion.
 #include "lsa_common.cuh"
 #include "lsa_kernels.h"
 

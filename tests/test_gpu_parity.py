@@ -147,6 +147,22 @@ def test_flat_index_heads_against_oracle(tiny, heads, k, cand_cap):
     PT.assert_lists_match(gl, gn, ol, on, qq, pos, oc, k=k)
 
 
+def test_flat_index_heads_exact_path_many_queries(tiny):
+    """With P entry slots per row most rows past the first blocks overflow, so
+    their queries are redone by the exact kernel, which runs one CTA per SM:
+    1600 queries give each CTA several marked queries to compact and work
+    through."""
+    keys, _, _, oc = tiny
+    P = O.top_p(256)
+    pos = np.concatenate([np.arange(512, 4096, 3), np.arange(2000, 2400)]).astype(np.int64)[:1600]
+    qq = I.index_queries_heads(13, keys, pos, 3)
+    cache, _, p = _build_gpu(keys, k=256, cand_cap=P, index_heads=3)
+    gl, gn = _index_gpu(cache, None, p, qq, pos)
+    sel = np.arange(0, len(pos), 7)
+    ol, on = O.index_heads(qq[sel], pos[sel], oc, k=256)
+    PT.assert_lists_match(gl[sel], gn[sel], ol, on, qq[sel], pos[sel], oc, k=256)
+
+
 def test_flat_index_heads_decode_and_single_head(tiny):
     """Decode batches (stored-score path) with 4 heads, and identical heads,
     which must give the single-head lists exactly."""
