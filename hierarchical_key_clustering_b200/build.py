@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblsa.so")
 SOURCES = ["lsa_api.cu", "lsa_build.cu", "lsa_index.cu", "lsa_score_tc.cu", "lsa_attn.cu", "lsa_noalloc.cu",
-           "lsa_shrink.cu"]
+           "lsa_shrink.cu", "lsa_shard.cu"]
 HEADERS = ["lsa_common.cuh", "lsa_kernels.h", "lsa_tc.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

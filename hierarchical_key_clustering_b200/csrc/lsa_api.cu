@@ -171,16 +171,17 @@ struct IndexLayout {
     int64_t mcap;
 };
 
-IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p)
+IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p, bool shard_local = false)
 {
     const int64_t N = nblk * LSA_BUCKETS;
     const int64_t heads = p->index_heads > 1 ? p->index_heads : 1;
     const int64_t rows = nq * heads;
+    const bool merged = heads > 1 || shard_local;
     IndexLayout L;
     L.gstride = lsa::HIST_BINS;  // group-maximum histogram per row
     L.cap = cand_cap(p);
-    L.mcap = heads > 1 ? expand_slots(L.cap, top_buckets(p)) : 0;
-    const int64_t mq = heads > 1 ? nq : 0;
+    L.mcap = merged ? expand_slots(L.cap, top_buckets(p)) : 0;
+    const int64_t mq = merged ? nq : 0;
     // small batches (decode) keep every score for the filter pass
     L.sstride = (rows <= lsa::SMALL_NQ && p->mode == LSA_MODE_FLAT) ? N : 0;
     const int64_t sz[13] = {rows * LSA_DIM * 2, rows * 4,        rows * 4, rows * 4, rows * L.gstride * 4,
@@ -236,18 +237,34 @@ int64_t near_ws_bytes(int64_t nq, int32_t Hq)
            align256(nq * 16);
 }
 
+// A shard's local step (lsa_index_shard_local): positions shifted to the
+// shard's first token, the merged candidate set packed into `xchg` with
+// global bucket ids instead of an expansion.
+struct ShardLocal {
+    int64_t b_first;
+    void *xchg;
+};
+
 int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache, const lsa_tree *tree,
                int32_t *lists, int32_t *lens, int32_t Lmax, const lsa_params *p, void *ws, int64_t ws_bytes,
-               void *stream)
+               void *stream, const ShardLocal *sl = nullptr)
 {
     int rc = check_params(p);
     if (rc) return rc;
     if (nq < 0) return fail(LSA_ERR_SHAPE, "nq < 0");
     if (!cache) return fail(LSA_ERR_ARG, "cache is NULL");
     if (nq == 0) return LSA_OK;
-    if (!qidx || !pos || !lists || !lens) return fail(LSA_ERR_ARG, "qidx, pos, lists and lens must be non-NULL");
-    if (!aligned16(qidx) || !aligned16(lists)) return fail(LSA_ERR_ARG, "qidx and lists must be 16-byte aligned");
-    if (Lmax < lsa_list_budget(p)) return fail(LSA_ERR_SHAPE, "Lmax %d < list budget %d", Lmax, lsa_list_budget(p));
+    if (sl) {
+        if (!qidx || !pos || !sl->xchg) return fail(LSA_ERR_ARG, "qidx, pos and xchg must be non-NULL");
+        if (!aligned16(qidx) || ((uintptr_t)sl->xchg & 255u)) return fail(LSA_ERR_ARG, "qidx must be 16-byte and xchg 256-byte aligned");
+        if (p->mode != LSA_MODE_FLAT) return fail(LSA_ERR_ARG, "context-parallel search is Flat only");
+        if (sl->b_first < 0) return fail(LSA_ERR_SHAPE, "b_first < 0");
+    } else {
+        if (!qidx || !pos || !lists || !lens) return fail(LSA_ERR_ARG, "qidx, pos, lists and lens must be non-NULL");
+        if (!aligned16(qidx) || !aligned16(lists)) return fail(LSA_ERR_ARG, "qidx and lists must be 16-byte aligned");
+        if (Lmax < lsa_list_budget(p))
+            return fail(LSA_ERR_SHAPE, "Lmax %d < list budget %d", Lmax, lsa_list_budget(p));
+    }
     if (cache->n_blocks < 0 || cache->n_blocks * LSA_BLOCK > cache->capacity)
         return fail(LSA_ERR_SHAPE, "cache n_blocks %lld out of range", (long long)cache->n_blocks);
     if (cache->n_blocks > 0 && (!cache->members || !cache->count || !cache->centroid_bf16))
@@ -267,7 +284,7 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     // (groups of up to 64 buckets, 4P..8P of them)
     if (p->mode == LSA_MODE_FLAT && (cache->n_blocks > 65535 || P >= 8192))
         return fail(LSA_ERR_SHAPE, "Flat search supports up to 65535 blocks and k + sink + window < 32768");
-    IndexLayout L = index_layout(nq, cache->n_blocks, p);
+    IndexLayout L = index_layout(nq, cache->n_blocks, p, sl != nullptr);
     if (L.cap < P) return fail(LSA_ERR_ARG, "cand_cap %lld < top buckets %lld", (long long)L.cap, (long long)P);
     if (L.cap > 8192) return fail(LSA_ERR_ARG, "cand_cap %lld above 8192", (long long)L.cap);
     if (lsa::rank_expand_smem_bytes((int)L.cap, cache->n_blocks) > 227 * 1024)
@@ -288,8 +305,9 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     iw.scores = L.sstride ? (float *)(w + L.off[7]) : nullptr;
     iw.score_stride = L.sstride;
     iw.cap = (int32_t)L.cap;
-    lsa::IndexWs mw = iw;  // merged candidates of multi-head queries
-    if (p->index_heads > 1) {
+    lsa::IndexWs mw = iw;  // merged candidates of multi-head queries or of a shard
+    const bool merged = p->index_heads > 1 || sl;
+    if (merged) {
         mw.horizon = (int32_t *)(w + L.off[8]);
         mw.tau = (float *)(w + L.off[9]);
         mw.cnt = (int32_t *)(w + L.off[10]);
@@ -318,6 +336,8 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     a.mode = p->mode;
     a.P = (int32_t)P;
     a.heads = p->index_heads;
+    a.pos_shift = sl ? sl->b_first * LSA_BLOCK : 0;
+    a.no_expand = sl ? 1 : 0;
     a.wait_limit = g_wait_limit;
     a.extra_tx = g_extra_tx;
     g_extra_tx = 0;
@@ -333,9 +353,12 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
         for (int l = 0; l < 41; ++l) tv.level_offset[l] = tree->level_offset[l];
         tvp = &tv;
     }
-    cudaError_t e = lsa::launch_index(a, iw, p->index_heads > 1 ? &mw : nullptr, tvp, (cudaStream_t)stream,
-                                      sm_count());
+    cudaError_t e = lsa::launch_index(a, iw, merged ? &mw : nullptr, tvp, (cudaStream_t)stream, sm_count());
     if (e != cudaSuccess) return cuda_fail(e, "index launch");
+    if (sl) {
+        e = lsa::launch_shard_pack(mw, nq, sl->b_first * LSA_BUCKETS, sl->xchg, (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail(e, "shard pack launch");
+    }
     return LSA_OK;
 }
 
@@ -667,6 +690,132 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
     }
     cudaError_t e = lsa::launch_attention(a, (cudaStream_t)stream, sm_count());
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return LSA_OK;
+}
+
+// ---- context parallelism (token ranges over ranks) ----
+
+int32_t lsa_shard_slots(const lsa_params *p)
+{
+    if (!p) return -1;
+    return (int32_t)expand_slots(cand_cap(p), top_buckets(p));
+}
+
+int64_t lsa_shard_exchange_bytes(int64_t nq, const lsa_params *p)
+{
+    if (!p || nq < 0) return -1;
+    return align256(nq * 4) + nq * (int64_t)lsa_shard_slots(p) * 8;
+}
+
+int64_t lsa_shard_local_workspace_bytes(int64_t nq, int64_t n_blocks, const lsa_params *p)
+{
+    if (!p || nq < 0 || n_blocks < 0) return -1;
+    return index_layout(nq, n_blocks, p, true).bytes;
+}
+
+int lsa_index_shard_local(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache, int64_t b_first,
+                          void *xchg, const lsa_params *p, void *ws, int64_t ws_bytes, void *stream)
+{
+    ShardLocal sl{b_first, xchg};
+    return index_impl(qidx, pos, nq, cache, nullptr, nullptr, nullptr, 0, p, ws, ws_bytes, stream, &sl);
+}
+
+int64_t lsa_shard_merge_workspace_bytes(int64_t nq, const lsa_params *p)
+{
+    if (!p || nq < 0) return -1;
+    const int64_t KC = lsa_shard_slots(p);
+    return 3 * align256(nq * 4) + align256(nq * KC * 16) + align256(nq * KC * 4);
+}
+
+int lsa_index_shard_merge(const void *xchg_all, int32_t n_shards, const int64_t *pos, int64_t nq,
+                          const int32_t *members, const int32_t *count, int64_t n_blocks, int32_t *lists,
+                          int32_t *lens, int32_t Lmax, const lsa_params *p, void *ws, int64_t ws_bytes, void *stream)
+{
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (p->mode != LSA_MODE_FLAT) return fail(LSA_ERR_ARG, "context-parallel search is Flat only");
+    if (nq < 0 || n_blocks < 0) return fail(LSA_ERR_SHAPE, "nq and n_blocks must be >= 0");
+    if (nq == 0) return LSA_OK;
+    const int64_t KC = lsa_shard_slots(p);
+    if (n_shards < 1 || n_shards > LSA_MAX_INDEX_HEADS || n_shards * KC * 8 > 227 * 1024)
+        return fail(LSA_ERR_ARG, "n_shards = %d: need 1..%d and n_shards x %lld x 8 B <= 227 KB", n_shards,
+                    LSA_MAX_INDEX_HEADS, (long long)KC);
+    if (!xchg_all || !pos || !lists || !lens || (n_blocks > 0 && (!members || !count)))
+        return fail(LSA_ERR_ARG, "xchg_all, pos, members, count, lists and lens must be non-NULL");
+    if (((uintptr_t)xchg_all & 255u) || !aligned16(lists)) return fail(LSA_ERR_ARG, "xchg_all must be 256-byte and lists 16-byte aligned");
+    if (Lmax < lsa_list_budget(p)) return fail(LSA_ERR_SHAPE, "Lmax %d < list budget %d", Lmax, lsa_list_budget(p));
+    if (lsa::rank_expand_smem_bytes((int)KC, n_blocks) > 227 * 1024)
+        return fail(LSA_ERR_ARG, "%lld blocks too many for the expansion kernel", (long long)n_blocks);
+    const int64_t need = lsa_shard_merge_workspace_bytes(nq, p);
+    if (!ws || ws_bytes < need)
+        return fail(LSA_ERR_WORKSPACE, "merge workspace %lld bytes < %lld", (long long)ws_bytes, (long long)need);
+    if (((uintptr_t)ws & 255u) != 0) return fail(LSA_ERR_ARG, "workspace must be 256-byte aligned");
+    char *w = (char *)ws;
+    lsa::IndexWs m{};
+    m.tau = (float *)w;
+    m.cnt = (int32_t *)(w + align256(nq * 4));
+    m.horizon = (int32_t *)(w + 2 * align256(nq * 4));
+    m.cand4 = (float *)(w + 3 * align256(nq * 4));
+    m.cand_g = (int32_t *)(w + 3 * align256(nq * 4) + align256(nq * KC * 16));
+    m.cap = (int32_t)KC;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = lsa::launch_shard_merge(xchg_all, n_shards, nq, (int)KC, (int)top_buckets(p), m, st);
+    if (e != cudaSuccess) return cuda_fail(e, "shard merge launch");
+    lsa::IndexArgs a{};
+    a.pos = pos;
+    a.nq = nq;
+    a.n_blocks = n_blocks;
+    a.members = members;
+    a.count = count;
+    a.centroid_bf16 = nullptr;
+    a.lists = lists;
+    a.lens = lens;
+    a.Lmax = Lmax;
+    a.k = p->k;
+    a.sink = p->sink;
+    a.window = p->window;
+    a.P = (int32_t)top_buckets(p);
+    e = lsa::launch_expand_merged(a, m, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expansion launch");
+    return LSA_OK;
+}
+
+int lsa_shard_publish_members(const lsa_cache *cache, int64_t b_first, int32_t *members_out, int32_t *count_out,
+                              void *stream)
+{
+    if (!cache || !members_out || !count_out) return fail(LSA_ERR_ARG, "cache and tables must be non-NULL");
+    if (b_first < 0) return fail(LSA_ERR_SHAPE, "b_first < 0");
+    if (cache->n_blocks == 0) return LSA_OK;
+    if (!cache->members || !cache->count) return fail(LSA_ERR_ARG, "cache arrays are NULL");
+    cudaError_t e = lsa::launch_publish_members(cache->members, cache->count, cache->n_blocks * LSA_BUCKETS, 0,
+                                                b_first * LSA_BLOCK, members_out, count_out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "publish launch");
+    return LSA_OK;
+}
+
+int lsa_shard_local_lists(const int32_t *lists, const int32_t *lens, int64_t nq, int32_t Lmax, int64_t t_begin,
+                          int64_t t_end, int32_t *out_lists, int32_t *out_lens, void *stream)
+{
+    if (nq < 0 || Lmax < 1 || t_begin < 0 || t_end < t_begin) return fail(LSA_ERR_SHAPE, "bad nq, Lmax or range");
+    if (nq == 0) return LSA_OK;
+    if (!lists || !lens || !out_lists || !out_lens) return fail(LSA_ERR_ARG, "pointers must be non-NULL");
+    if (out_lists == lists) return fail(LSA_ERR_ARG, "out_lists must not alias lists");
+    cudaError_t e = lsa::launch_local_lists(lists, lens, nq, Lmax, t_begin, t_end, out_lists, out_lens,
+                                            (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "local lists launch");
+    return LSA_OK;
+}
+
+int lsa_attention_combine(const uint16_t *O_parts, const float *lse_parts, int32_t n_parts, int64_t nq, int32_t Hq,
+                          int32_t head_dim, uint16_t *O, float *lse, void *stream)
+{
+    if (head_dim != LSA_HEAD_DIM) return fail(LSA_ERR_ARG, "head_dim must be %d", LSA_HEAD_DIM);
+    if (n_parts < 1 || nq < 0 || Hq < 1) return fail(LSA_ERR_SHAPE, "need n_parts >= 1, nq >= 0, Hq >= 1");
+    if (nq == 0) return LSA_OK;
+    if (!O_parts || !lse_parts || !O) return fail(LSA_ERR_ARG, "O_parts, lse_parts and O must be non-NULL");
+    if (((uintptr_t)O_parts & 7u) || ((uintptr_t)O & 7u)) return fail(LSA_ERR_ARG, "O_parts and O must be 8-byte aligned");
+    cudaError_t e = lsa::launch_combine_parts(O_parts, lse_parts, n_parts, nq, Hq, O, lse, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     return LSA_OK;
 }
 

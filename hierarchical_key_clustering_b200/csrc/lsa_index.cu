@@ -35,7 +35,7 @@ namespace lsa {
 // One warp per row; a row is one index query, `heads` consecutive rows per
 // token (all with that token's horizon).
 __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, const int64_t *__restrict__ pos,
-                                               int64_t nq, int heads, int64_t n_blocks, IndexWs ws)
+                                               int64_t nq, int heads, int64_t pos_shift, int64_t n_blocks, IndexWs ws)
 {
     pdl_wait();
     pdl_release();
@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, c
         ws.qhat[q * LSA_D + lane] = f2bf_bits(a);
         ws.qhat[q * LSA_D + lane + 32] = f2bf_bits(b);
         if (lane == 0) {
-            int64_t p = pos[q / heads];
+            int64_t p = pos[q / heads] - pos_shift;  // shift: first position of a shard's cache
             int64_t H = p < 0 ? 0 : p / LSA_BLK;
             if (H > n_blocks) H = n_blocks;
             ws.horizon[q] = (int32_t)H;
@@ -1513,6 +1513,29 @@ __global__ void __launch_bounds__(HM_THREADS) k_heads_exact(int64_t nq, int head
         __syncthreads();
     }
 }
+// Expansion of an already merged candidate set (one-bucket entries, at most
+// m.cap per query, tau = -inf), e.g. the top P of a context-parallel merge.
+cudaError_t launch_expand_merged(const IndexArgs &a, const IndexWs &m, cudaStream_t st)
+{
+    if (a.nq <= 0) return cudaSuccess;
+    const int TW = (int)((a.n_blocks + 31) / 32) + 1;
+    const int KC = m.cap;
+    const size_t smr = rank_expand_smem(KC, TW);
+    if (a.nq <= SMALL_NQ) {
+        cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        const cudaError_t e = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
+                                       a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
+                                       a.window, a.P, KC, TW, m);
+        if (e != cudaSuccess) return e;
+    } else {
+        cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists,
+                                                             a.lens, a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, m);
+    }
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks)
 {
     return rank_expand_smem(cap, (int)((n_blocks + 31) / 32) + 1);
@@ -1530,7 +1553,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
         int64_t blocks = (rows + 7) / 8;
         if (blocks > (int64_t)n_sm * 32) blocks = (int64_t)n_sm * 32;
         if ((e = launch_k(rows <= SMALL_NQ, k_qnorm, dim3((unsigned)blocks), dim3(256), 0, st, a.qidx, a.pos, rows,
-                          heads, a.n_blocks, ws)) != cudaSuccess)
+                          heads, a.pos_shift, a.n_blocks, ws)) != cudaSuccess)
             return e;
         count_launches(1);
     }
@@ -1603,6 +1626,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
                           ws, *merged)) != cudaSuccess)
             return e;
         count_launches(2);
+        if (a.no_expand) return cudaGetLastError();  // a shard's local candidate set stops here
     }
     const IndexWs &ex = merged ? *merged : ws;
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;

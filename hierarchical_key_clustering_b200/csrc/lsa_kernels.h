@@ -121,6 +121,8 @@ struct IndexArgs {
     int32_t k, sink, window, beam, mode;
     int32_t P;  // top buckets kept
     int32_t heads;  // index queries per token (Flat: a bucket ranks by its best head score)
+    int64_t pos_shift;  // subtracted from pos for the horizon (a shard's first position; 0 otherwise)
+    int32_t no_expand;  // stop after the merged candidate set (a shard's local step)
     uint32_t wait_limit;  // tries per bounded device-side wait
     uint32_t extra_tx;    // test hook (see lsa_debug_wait_test)
 };
@@ -157,6 +159,20 @@ int read_shrink_error(int clear);
 // receives each query's merged candidates (nullptr for one head).
 cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *merged, const TreeView *tree,
                          cudaStream_t st, int n_sm);
+cudaError_t launch_expand_merged(const IndexArgs &a, const IndexWs &m, cudaStream_t st);
+
+// Context-parallel pieces (lsa_shard.cu).  Exchange block of one rank:
+// int32 cnt[nq], then {float score, int32 global bucket} [nq][slots].
+cudaError_t launch_shard_pack(const IndexWs &m, int64_t nq, int64_t g0, void *xchg, cudaStream_t st);
+cudaError_t launch_shard_merge(const void *xchg_all, int n_shards, int64_t nq, int slots, int P, const IndexWs &m,
+                               cudaStream_t st);
+cudaError_t launch_local_lists(const int32_t *lists, const int32_t *lens, int64_t nq, int32_t Lmax, int64_t t0,
+                               int64_t t1, int32_t *out_lists, int32_t *out_lens, cudaStream_t st);
+cudaError_t launch_publish_members(const int32_t *members, const int32_t *count, int64_t nb, int64_t g0,
+                                   int64_t pos0, int32_t *members_out, int32_t *count_out, cudaStream_t st);
+cudaError_t launch_combine_parts(const uint16_t *O_parts, const float *lse_parts, int n_parts, int64_t nq, int Hq,
+                                 uint16_t *O, float *lse, cudaStream_t st);
+
 // Shared memory the expansion kernel needs for `cap` candidates over a cache
 // of n_blocks blocks.
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks);

@@ -1,0 +1,295 @@
+// Context-parallel pieces of the LSA path: the KV cache and the bucket cache
+// split by token range over ranks, as the pages' end-to-end runs do with
+// decode context parallelism over 8 GPUs (zhichai forum post, "Reported
+// numbers"; sotaaz blog, "Why 72x in one layer becomes 9x").
+//
+// Rank s holds the complete blocks [b0_s, b1_s) and their K/V rows.  Every
+// query is replicated.  Index: each rank finds a local candidate set that
+// holds its own top P buckets (the Flat passes and merge of lsa_index.cu over
+// its blocks), the sets are exchanged, and every rank takes the same global
+// top P from their union: a bucket among the global top P is among the top P
+// of the rank that owns it, so the union holds it with its exact score.  The
+// same expansion then gives every rank the identical list.  Attention: each
+// rank attends over the list entries it owns and the partial results are
+// combined by log-sum-exp.
+#include "lsa_common.cuh"
+#include "lsa_kernels.h"
+
+namespace lsa {
+
+// Radix select over values produced by get(i), i < n (lsa_index.cu has the
+// same selection for its own callers): the P-th largest ordered key.
+template <typename Get>
+__device__ uint32_t shard_select(int64_t n, int64_t P, Get get, int *hist, int *sh)
+{
+    uint32_t prefix = 0, mask = 0;
+    int64_t rem = P;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint32_t u = get(i);
+            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int64_t acc = 0;
+            int d = 255;
+            for (; d > 0; --d) {
+                if (acc + hist[d] >= rem) break;
+                acc += hist[d];
+            }
+            sh[0] = d;
+            sh[1] = (int)(rem - acc);
+        }
+        __syncthreads();
+        prefix |= ((uint32_t)sh[0]) << shift;
+        mask |= 255u << shift;
+        rem = sh[1];
+        __syncthreads();
+    }
+    return prefix;
+}
+
+// ---------------------------------------------------------------------------
+// A rank's merged local set (one-bucket entries, local bucket ids) into its
+// exchange block with global bucket ids (g0 = 64 x the rank's first block).
+__global__ void k_shard_pack(IndexWs m, int64_t nq, int64_t g0, int32_t *__restrict__ xcnt,
+                             int2 *__restrict__ xent)
+{
+    pdl_wait();
+    pdl_release();
+    const int64_t q = blockIdx.x;
+    const int n = m.cnt[q];
+    if (threadIdx.x == 0) xcnt[q] = n;
+    const float4 *c4 = reinterpret_cast<const float4 *>(m.cand4) + q * m.cap;
+    const int32_t *cg = m.cand_g + q * m.cap;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        xent[q * m.cap + i] = make_int2(__float_as_int(c4[i].x), (int32_t)(cg[i] + g0));
+}
+
+cudaError_t launch_shard_pack(const IndexWs &m, int64_t nq, int64_t g0, void *xchg, cudaStream_t st)
+{
+    if (nq <= 0) return cudaSuccess;
+    int32_t *xcnt = reinterpret_cast<int32_t *>(xchg);
+    int2 *xent = reinterpret_cast<int2 *>(reinterpret_cast<char *>(xchg) + ((nq * 4 + 255) / 256) * 256);
+    k_shard_pack<<<(unsigned)nq, 256, 0, st>>>(m, nq, g0, xcnt, xent);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Global top P of the union of the ranks' sets (disjoint bucket ids, exact
+// scores).  One CTA per query stages the union in shared memory; all of it
+// is kept when it fits the expansion's slots, else the buckets above the
+// P-th score and, at that score, the ties with the lowest ids up to P.
+constexpr int SM_THREADS = 512;
+
+__global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__restrict__ xcnt_all,
+                                                            const int2 *__restrict__ xent_all, int n_shards,
+                                                            int64_t nq, int64_t xstride, int slots, int P, IndexWs m)
+{
+    pdl_wait();
+    pdl_release();
+    extern __shared__ uint2 um[];  // [n_shards * slots] (ordered score, bucket id)
+    __shared__ int hist[256];
+    __shared__ int sh[4];
+    __shared__ int s_off[LSA_MAXHEADS + 1];
+    __shared__ int s_out;
+    const int64_t q = blockIdx.x;
+    const int t = threadIdx.x;
+    const float NEG = __int_as_float(0xff800000);
+    const int KC = m.cap;
+    if (t == 0) {
+        int o = 0;
+        for (int s = 0; s < n_shards; ++s) {
+            s_off[s] = o;
+            o += min(xcnt_all[s * xstride / 4 + q], slots);
+        }
+        s_off[n_shards] = o;
+        s_out = 0;
+    }
+    __syncthreads();
+    const int n = s_off[n_shards];
+    for (int i = t; i < n; i += SM_THREADS) {
+        int s = 0;
+        while (i >= s_off[s + 1]) ++s;
+        const int2 e = *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(xent_all) + s * xstride +
+                                                       (q * slots + (i - s_off[s])) * 8);
+        um[i] = make_uint2(f2ord(__int_as_float(e.x)), (uint32_t)e.y);
+    }
+    __syncthreads();
+    float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * KC;
+    int32_t *og = m.cand_g + q * KC;
+    if (n <= KC) {  // everything fits: the expansion ranks it
+        for (int i = t; i < n; i += SM_THREADS) {
+            o4[i] = make_float4(ord2f(um[i].x), NEG, NEG, NEG);
+            og[i] = (int32_t)um[i].y;
+        }
+        if (t == 0) s_out = n;
+    } else {
+        const uint32_t cut = shard_select(n, P, [&](int64_t i) { return um[i].x; }, hist, sh);
+        int above = 0, ties = 0;
+        for (int i = t; i < n; i += SM_THREADS) {
+            above += um[i].x > cut;
+            ties += um[i].x == cut;
+        }
+        __syncthreads();
+        if (t == 0) sh[2] = 0, sh[3] = 0;
+        __syncthreads();
+        atomicAdd(&sh[2], above);
+        atomicAdd(&sh[3], ties);
+        __syncthreads();
+        const int n_above = sh[2], n_ties = sh[3];
+        // ties at the cut: all of them when they fit, else the lowest ids
+        uint32_t idcut = 0xffffffffu;
+        if (n_above + n_ties > KC) {
+            const int need = P - n_above;
+            // the need-th smallest id among the ties = the need-th largest of ~id
+            idcut = ~shard_select(n, need, [&](int64_t i) { return um[i].x == cut ? ~um[i].y : 0u; }, hist, sh);
+        }
+        for (int i = t; i < n; i += SM_THREADS) {
+            const uint2 u = um[i];
+            if (u.x > cut || (u.x == cut && u.y <= idcut)) {
+                const int j = atomicAdd(&s_out, 1);
+                o4[j] = make_float4(ord2f(u.x), NEG, NEG, NEG);
+                og[j] = (int32_t)u.y;
+            }
+        }
+    }
+    __syncthreads();
+    if (t == 0) {
+        m.cnt[q] = s_out;
+        m.tau[q] = NEG;
+        m.horizon[q] = 0;  // read only by the expansion's exact path, which a merged set never takes
+    }
+}
+
+cudaError_t launch_shard_merge(const void *xchg_all, int n_shards, int64_t nq, int slots, int P, const IndexWs &m,
+                               cudaStream_t st)
+{
+    if (nq <= 0) return cudaSuccess;
+    const int64_t cnt_bytes = ((nq * 4 + 255) / 256) * 256;
+    const int64_t xstride = cnt_bytes + nq * slots * 8;  // one rank's exchange block
+    const int32_t *xcnt = reinterpret_cast<const int32_t *>(xchg_all);
+    const int2 *xent = reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(xchg_all) + cnt_bytes);
+    const size_t smem = (size_t)n_shards * slots * 8;
+    cudaFuncSetAttribute(k_shard_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_shard_merge<<<(unsigned)nq, SM_THREADS, smem, st>>>(xcnt, xent, n_shards, nq, xstride, slots, P, m);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// The entries of each list in [t0, t1), shifted to the rank's K/V rows.  One
+// warp per query; the order is kept, the rest of the row is -1.
+__global__ void __launch_bounds__(256) k_local_lists(const int32_t *__restrict__ lists,
+                                                     const int32_t *__restrict__ lens, int64_t nq, int32_t Lmax,
+                                                     int64_t t0, int64_t t1, int32_t *__restrict__ out_lists,
+                                                     int32_t *__restrict__ out_lens)
+{
+    pdl_wait();
+    pdl_release();
+    const int lane = threadIdx.x & 31;
+    const int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (q >= nq) return;
+    const int32_t *in = lists + q * Lmax;
+    int32_t *out = out_lists + q * Lmax;
+    const int len = min(lens[q], Lmax);
+    int n = 0;
+    for (int i0 = 0; i0 < len; i0 += 32) {
+        const int i = i0 + lane;
+        const int64_t v = i < len ? in[i] : -1;
+        const bool keep = v >= t0 && v < t1;
+        const unsigned bal = __ballot_sync(LSA_FULL, keep);
+        if (keep) out[n + __popc(bal & ((1u << lane) - 1u))] = (int32_t)(v - t0);
+        n += __popc(bal);
+    }
+    for (int i = n + lane; i < Lmax; i += 32) out[i] = -1;
+    if (lane == 0) out_lens[q] = n;
+}
+
+cudaError_t launch_local_lists(const int32_t *lists, const int32_t *lens, int64_t nq, int32_t Lmax, int64_t t0,
+                               int64_t t1, int32_t *out_lists, int32_t *out_lens, cudaStream_t st)
+{
+    if (nq <= 0) return cudaSuccess;
+    k_local_lists<<<(unsigned)((nq + 7) / 8), 256, 0, st>>>(lists, lens, nq, Lmax, t0, t1, out_lists, out_lens);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// A rank's member table and counts into the replicated global tables: bucket
+// g of the rank is global bucket g0 + g, its member positions move by pos0.
+__global__ void k_publish_members(const int32_t *__restrict__ members, const int32_t *__restrict__ count, int64_t nb,
+                                  int64_t g0, int64_t pos0, int32_t *__restrict__ members_out,
+                                  int32_t *__restrict__ count_out)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nb * LSA_NSLOT) return;
+    const int32_t m = members[i];
+    members_out[g0 * LSA_NSLOT + i] = m >= 0 ? (int32_t)(m + pos0) : -1;
+    if (i % LSA_NSLOT == 0) count_out[g0 + i / LSA_NSLOT] = count[i / LSA_NSLOT];
+}
+
+cudaError_t launch_publish_members(const int32_t *members, const int32_t *count, int64_t nb, int64_t g0,
+                                   int64_t pos0, int32_t *members_out, int32_t *count_out, cudaStream_t st)
+{
+    if (nb <= 0) return cudaSuccess;
+    k_publish_members<<<(unsigned)((nb * LSA_NSLOT + 255) / 256), 256, 0, st>>>(members, count, nb, g0, pos0,
+                                                                               members_out, count_out);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp combination of the ranks' attention outputs: O_s normalised
+// over rank s's keys with log-sum-exp lse_s (-inf for a rank with none), so
+// O = sum_s exp(lse_s - M) O_s / sum_s exp(lse_s - M), lse = M + log(that sum).
+// One warp per (query, head), 4 dims per lane.
+__global__ void __launch_bounds__(256) k_combine_parts(const uint16_t *__restrict__ O_parts,
+                                                       const float *__restrict__ lse_parts, int n_parts, int64_t units,
+                                                       uint16_t *__restrict__ O, float *__restrict__ lse)
+{
+    pdl_wait();
+    pdl_release();
+    const int lane = threadIdx.x & 31;
+    const int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (u >= units) return;
+    const float NEG = __int_as_float(0xff800000);
+    float M = NEG;
+    for (int s = 0; s < n_parts; ++s) M = fmaxf(M, lse_parts[s * units + u]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.0f;
+    for (int s = 0; s < n_parts; ++s) {
+        const float ls = lse_parts[s * units + u];
+        if (!(ls > NEG)) continue;  // no keys on this rank
+        const float w = expf(ls - M);
+        L += w;
+        const uint2 v = *reinterpret_cast<const uint2 *>(O_parts + (s * units + u) * LSA_HEAD + lane * 4);
+        acc[0] += w * __uint_as_float(v.x << 16);
+        acc[1] += w * __uint_as_float(v.x & 0xffff0000u);
+        acc[2] += w * __uint_as_float(v.y << 16);
+        acc[3] += w * __uint_as_float(v.y & 0xffff0000u);
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    __nv_bfloat16 b[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) b[e] = __float2bfloat16_rn(acc[e] * inv);
+    uint2 w;
+    w.x = (uint32_t)*reinterpret_cast<uint16_t *>(&b[0]) | ((uint32_t)*reinterpret_cast<uint16_t *>(&b[1]) << 16);
+    w.y = (uint32_t)*reinterpret_cast<uint16_t *>(&b[2]) | ((uint32_t)*reinterpret_cast<uint16_t *>(&b[3]) << 16);
+    *reinterpret_cast<uint2 *>(O + u * LSA_HEAD + lane * 4) = w;
+    if (lane == 0 && lse) lse[u] = L > 0.0f ? M + logf(L) : NEG;
+}
+
+cudaError_t launch_combine_parts(const uint16_t *O_parts, const float *lse_parts, int n_parts, int64_t nq, int Hq,
+                                 uint16_t *O, float *lse, cudaStream_t st)
+{
+    const int64_t units = nq * Hq;
+    if (units <= 0) return cudaSuccess;
+    k_combine_parts<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(O_parts, lse_parts, n_parts, units, O, lse);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace lsa

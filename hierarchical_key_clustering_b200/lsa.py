@@ -61,7 +61,9 @@ EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "l
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
            "lsa_shrink", "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
-           "lsa_index_decode_static"]
+           "lsa_index_decode_static", "lsa_shard_slots", "lsa_shard_exchange_bytes",
+           "lsa_shard_local_workspace_bytes", "lsa_shard_merge_workspace_bytes", "lsa_index_shard_local",
+           "lsa_index_shard_merge", "lsa_shard_publish_members", "lsa_shard_local_lists", "lsa_attention_combine"]
 
 _lib = None
 
@@ -108,6 +110,15 @@ def lib():
             "lsa_index_decode_static": (C.c_int, [P, P, i64, pc, pt, P, P, i32, pp, P]),
             "lsa_sparse_attention": (C.c_int, [P, P, P, i64, i32, i32, i32, i64, P, P, i32, f32, P, P, P,
                                                i64, P]),
+            "lsa_shard_slots": (i32, [pp]),
+            "lsa_shard_exchange_bytes": (i64, [i64, pp]),
+            "lsa_shard_local_workspace_bytes": (i64, [i64, i64, pp]),
+            "lsa_shard_merge_workspace_bytes": (i64, [i64, pp]),
+            "lsa_index_shard_local": (C.c_int, [P, P, i64, pc, i64, P, pp, P, i64, P]),
+            "lsa_index_shard_merge": (C.c_int, [P, i32, P, i64, P, P, i64, P, P, i32, pp, P, i64, P]),
+            "lsa_shard_publish_members": (C.c_int, [pc, i64, P, P, P]),
+            "lsa_shard_local_lists": (C.c_int, [P, P, i64, i32, i64, i64, P, P, P]),
+            "lsa_attention_combine": (C.c_int, [P, P, i32, i64, i32, i32, P, P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -335,3 +346,51 @@ def lsa_sparse_attention(Q, K, V, lists, lens, O, lse=None, scale=None, ws=None,
     _check(lib().lsa_sparse_attention(_ptr(Q), _ptr(K), _ptr(V), nq, Hq, Hkv, dh, Tk, _ptr(lists), _ptr(lens),
                                       lists.shape[1], float(scale), _ptr(O), _ptr(lse), _ptr(ws),
                                       ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+# ---------------------------------------------------------------- context parallelism
+
+def lsa_shard_slots(p: lsa_params) -> int:
+    return int(lib().lsa_shard_slots(C.byref(p)))
+
+
+def lsa_shard_exchange_bytes(nq: int, p: lsa_params) -> int:
+    return int(lib().lsa_shard_exchange_bytes(nq, C.byref(p)))
+
+
+def lsa_shard_local_workspace_bytes(nq: int, n_blocks: int, p: lsa_params) -> int:
+    return int(lib().lsa_shard_local_workspace_bytes(nq, n_blocks, C.byref(p)))
+
+
+def lsa_shard_merge_workspace_bytes(nq: int, p: lsa_params) -> int:
+    return int(lib().lsa_shard_merge_workspace_bytes(nq, C.byref(p)))
+
+
+def lsa_index_shard_local(qidx, pos, cache: Cache, b_first: int, xchg, p: lsa_params, ws, stream=None):
+    nq = qidx.shape[0]
+    assert qidx.numel() == nq * max(p.index_heads, 1) * 64, "qidx must be [nq, index_heads, 64]"
+    _check(lib().lsa_index_shard_local(_ptr(qidx), _ptr(pos), nq, C.byref(cache.c), b_first, _ptr(xchg), C.byref(p),
+                                       _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+def lsa_index_shard_merge(xchg_all, n_shards: int, pos, members, count, n_blocks: int, lists, lens, p: lsa_params, ws,
+                          stream=None):
+    _check(lib().lsa_index_shard_merge(_ptr(xchg_all), n_shards, _ptr(pos), pos.shape[0], _ptr(members),
+                                       _ptr(count), n_blocks, _ptr(lists), _ptr(lens), lists.shape[1], C.byref(p),
+                                       _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+def lsa_shard_publish_members(cache: Cache, b_first: int, members_out, count_out, stream=None):
+    _check(lib().lsa_shard_publish_members(C.byref(cache.c), b_first, _ptr(members_out), _ptr(count_out),
+                                           _stream(stream)))
+
+
+def lsa_shard_local_lists(lists, lens, t_begin: int, t_end: int, out_lists, out_lens, stream=None):
+    _check(lib().lsa_shard_local_lists(_ptr(lists), _ptr(lens), lists.shape[0], lists.shape[1], t_begin, t_end,
+                                       _ptr(out_lists), _ptr(out_lens), _stream(stream)))
+
+
+def lsa_attention_combine(O_parts, lse_parts, O, lse=None, stream=None):
+    n_parts, nq, Hq, D = O_parts.shape
+    _check(lib().lsa_attention_combine(_ptr(O_parts), _ptr(lse_parts), n_parts, nq, Hq, D, _ptr(O), _ptr(lse),
+                                       _stream(stream)))

@@ -344,6 +344,69 @@ int lsa_index_decode_static(const float *qidx, const int64_t *pos, int64_t nq, c
                             const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax,
                             const lsa_params *p, void *stream);
 
+/* ---- context parallelism: the token range split over ranks ----
+ * The pages' end-to-end runs split the KV cache by token range over 8 GPUs
+ * ([FORUM] "Reported numbers"; [BLOG] "Why 72x in one layer becomes 9x").
+ * Rank s holds complete blocks [b_first_s, b_first_s + n_s) of the bucket
+ * cache (a cache built from the keys of positions 512 b_first_s onwards,
+ * member positions relative to that) and the K/V rows of its token range;
+ * queries are replicated.  A bucket among the global top P is among the top
+ * P of the rank that owns it, so each rank sends a set holding its own top P
+ * (lsa_index_shard_local), the sets are all-gathered in rank order, and every
+ * rank computes the same global top P and list (lsa_index_shard_merge),
+ * identical to lsa_index_prefill on the whole cache (Flat, up to ties in the
+ * last bit of a score at the cut).  Each rank attends over its own entries
+ * (lsa_shard_local_lists, then lsa_sparse_attention with lse) and the parts
+ * are combined (lsa_attention_combine).  Flat search only; 1..16 ranks.
+ *
+ * Exchange block of one rank for nq queries, lsa_shard_exchange_bytes(nq, p)
+ * bytes, 256-byte aligned: int32 cnt[nq] padded to 256 bytes, then
+ * {float score; int32 global bucket} [nq][lsa_shard_slots(p)]. */
+int32_t lsa_shard_slots(const lsa_params *p);
+int64_t lsa_shard_exchange_bytes(int64_t nq, const lsa_params *p);
+int64_t lsa_shard_local_workspace_bytes(int64_t nq, int64_t n_blocks, const lsa_params *p);
+int64_t lsa_shard_merge_workspace_bytes(int64_t nq, const lsa_params *p);
+
+/* This rank's candidate set for each query into its exchange block `xchg`:
+ * the Flat passes over `cache` (this rank's blocks, the first being global
+ * block b_first; a query at position p sees the rank's blocks below p/512),
+ * each query's set holding its top P local buckets with their scores, bucket
+ * ids made global (+ 64 b_first).  qidx [nq, index_heads, 64] and pos [nq]
+ * as lsa_index_prefill.  ws: lsa_shard_local_workspace_bytes. */
+int lsa_index_shard_local(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache, int64_t b_first,
+                          void *xchg, const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);
+
+/* The global lists from n_shards exchange blocks stored back to back in rank
+ * order (xchg_all): per query the union's top P by (score desc, bucket id
+ * asc), expanded as lsa_index_prefill does, over the replicated member table
+ * and counts of all n_blocks blocks (members [n_blocks*64, 16] global
+ * positions, count [n_blocks*64]; see lsa_shard_publish_members).  Lists as
+ * lsa_index_prefill.  ws: lsa_shard_merge_workspace_bytes. */
+int lsa_index_shard_merge(const void *xchg_all, int32_t n_shards, const int64_t *pos, int64_t nq,
+                          const int32_t *members, const int32_t *count, int64_t n_blocks, int32_t *lists,
+                          int32_t *lens, int32_t Lmax, const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);
+
+/* This rank's slice of the global member table: members_out [64 n, 16]
+ * (n = cache->n_blocks) gets the cache's member positions moved by
+ * 512 b_first (-1 pads kept), count_out [64 n] its counts.  With slices of
+ * equal size and rank s's first block at s times that size, an all-gather
+ * of the slices in rank order is the global table (68 bytes per bucket,
+ * 8.5 bytes per token). */
+int lsa_shard_publish_members(const lsa_cache *cache, int64_t b_first, int32_t *members_out, int32_t *count_out,
+                              void *stream);
+
+/* The entries of each list inside [t_begin, t_end), in order, minus t_begin
+ * (this rank's K/V rows); out_lists [nq, Lmax] -1 padded, out_lens [nq]. */
+int lsa_shard_local_lists(const int32_t *lists, const int32_t *lens, int64_t nq, int32_t Lmax, int64_t t_begin,
+                          int64_t t_end, int32_t *out_lists, int32_t *out_lens, void *stream);
+
+/* Combine n_parts attention outputs of the same queries over disjoint key
+ * sets: O_parts bf16 [n_parts, nq, Hq, 128] (each normalised over its own
+ * keys), lse_parts fp32 [n_parts, nq, Hq] (-inf for no keys);
+ * O = sum_s e^(lse_s - M) O_s / sum_s e^(lse_s - M), lse = M + log(sum). */
+int lsa_attention_combine(const uint16_t *O_parts, const float *lse_parts, int32_t n_parts, int64_t nq, int32_t Hq,
+                          int32_t head_dim, uint16_t *O, float *lse, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

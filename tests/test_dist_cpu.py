@@ -1,6 +1,8 @@
-"""The bench's multi-process plumbing on CPU (gloo, world size 2, 127.0.0.1):
-max-over-ranks timing and barriers, and a torchrun launch of the reference
-arm, where rank 0 alone works and prints one JSON line."""
+"""Multi-process plumbing on CPU (gloo, world size 2, 127.0.0.1): the bench's
+max-over-ranks timing and barriers, a torchrun launch of the reference arm
+(rank 0 alone works and prints one JSON line), and the context-parallel
+step's exchanges (which rank's tensor lands where; the GPU stages are stood
+in for by CPU ones that record what they receive)."""
 import json
 import os
 import socket
@@ -55,3 +57,79 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+# ---------------------------------------------------------------- context parallelism
+
+def test_shard_ranges_cover_every_block_once():
+    from hierarchical_key_clustering_b200.context_parallel import shard_range
+
+    for T, world in [(4096, 2), (4096, 3), (4096, 5), (4396, 3), (10_000_000, 8), (512, 4), (100, 2)]:
+        nblk = T // 512
+        rs = [shard_range(T, r, world) for r in range(world)]
+        blocks = [b for b0, b1, _, _, _ in rs for b in range(b0, b1)]
+        assert blocks == list(range(nblk))
+        toks = [(t0, t1) for _, _, t0, t1, _ in rs]
+        assert toks[0][0] == 0 and toks[-1][1] == T
+        assert all(toks[i][1] == toks[i + 1][0] for i in range(world - 1))
+        per = rs[0][4]
+        for r, (b0, b1, t0, t1, _) in enumerate(rs):
+            assert b1 == b0 or b0 == r * per  # a rank's table slice sits at rank x slice size
+            assert t0 == 512 * b0
+
+
+class _FakeShard:
+    """A rank's stages with CPU stand-ins that record their inputs."""
+
+    def __init__(self, rank, world):
+        self.rank, self.world, self.seen = rank, world, {}
+
+    def build(self, keys_local):
+        return (torch.full((2, 16), self.rank, dtype=torch.int32), torch.full((2,), 10 + self.rank, dtype=torch.int32))
+
+    def set_members(self, M, C):
+        self.seen["members"], self.seen["count"] = M.clone(), C.clone()
+
+    def index_local(self, qidx, pos):
+        return torch.tensor([self.rank, 100 + self.rank, 200 + self.rank], dtype=torch.uint8)
+
+    def index_merge(self, X, pos):
+        self.seen["xchg"] = X.clone()
+        return X.to(torch.int32).reshape(1, -1), torch.tensor([X.numel()], dtype=torch.int32)
+
+    def attend_local(self, Q, K, V, lists, lens):
+        return torch.full((1, 2, 4), float(self.rank)), torch.full((1, 2), -float(self.rank))
+
+    def combine(self, O_parts, lse_parts):
+        self.seen["O_parts"], self.seen["lse_parts"] = O_parts.clone(), lse_parts.clone()
+        return O_parts.sum(0), lse_parts.max(0).values
+
+
+def _cp_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from hierarchical_key_clustering_b200 import context_parallel as CP
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sh = _FakeShard(rank, world)
+    O, lse, lists, lens = CP.prefill(sh, None, None, None, None, None, None)
+    out[rank] = dict(members=sh.seen["members"][:, 0, 0].tolist(), count=sh.seen["count"][:, 0].tolist(),
+                     xchg=sh.seen["xchg"].tolist(), O=O[0, 0, 0].item(), lse=lse[0, 0].item(),
+                     lists=lists.tolist(), parts=sh.seen["O_parts"][:, 0, 0, 0].tolist())
+    dist.destroy_process_group()
+
+
+def test_context_parallel_exchanges_gloo():
+    """Every rank receives every rank's member slice, exchange block and
+    attention part, in rank order, and computes the same list."""
+    world, port = 2, _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_cp_worker, args=(world, port, out), nprocs=world, join=True)
+    for r in range(world):
+        d = out[r]
+        assert d["members"] == [0, 1] and d["count"] == [10, 11]
+        assert d["xchg"] == [0, 100, 200, 1, 101, 201]
+        assert d["parts"] == [0.0, 1.0] and d["O"] == 1.0 and d["lse"] == 0.0
+        assert d["lists"] == out[0]["lists"]
