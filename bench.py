@@ -254,6 +254,91 @@ def measure_index_heads(layer, keys_np, pos_np, wl: dict, dev, heads: int = 8, c
             "tokens_per_s": round(nq / (ms / 1e3), 1)}
 
 
+def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, ranks: int, chunk: int = 16384):
+    """The context-parallel step of the workload split over `ranks` token
+    ranges, every rank's stages run one after another on this one GPU (the
+    all-gathers become stacking): per stage, the slowest rank's kernel time
+    over all queries (chunks of `chunk`), and the bytes each rank would
+    send and receive.  Communication time is not included."""
+    from hierarchical_key_clustering_b200 import context_parallel as CP
+
+    T, nq, hq, hkv = wl["T"], len(pos_np), wl["hq"], wl["hkv"]
+    chunk = min(chunk, nq)
+    shards = [CP.Shard(r, ranks, T, k=wl["k"], max_queries=chunk, device=dev) for r in range(ranks)]
+    keys = torch.from_numpy(keys_np).to(dev)
+    qidx = torch.from_numpy(q_np).to(dev)
+    pos = torch.from_numpy(pos_np).to(dev)
+    Lmax = shards[0].Lmax
+    ws_attn = lsa.workspace(lsa.lsa_attention_workspace_bytes(chunk, hq, 128, Lmax), dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    t_build = []
+    for s in shards:
+        a, b = ev(), ev()
+        a.record()
+        s.build(keys[s.t0:s.t1])
+        b.record()
+        t_build.append((a, b))
+    M = torch.stack([s.members_slice for s in shards])
+    C = torch.stack([s.count_slice for s in shards])
+    for s in shards:
+        s.set_members(M, C)
+
+    def one_pass(record):
+        t_loc = [[] for _ in shards]
+        t_att = [[] for _ in shards]
+        t_mrg, t_cmb = [], []
+        for c0 in range(0, nq, chunk):
+            c1 = min(nq, c0 + chunk)
+            xs = []
+            for r, s in enumerate(shards):
+                a, b = ev(), ev()
+                a.record()
+                xs.append(s.index_local(qidx[c0:c1], pos[c0:c1]))
+                b.record()
+                t_loc[r].append((a, b))
+            X = torch.stack(xs).reshape(-1)
+            a, b = ev(), ev()
+            a.record()
+            lists, lens = shards[0].index_merge(X, pos[c0:c1])  # every rank does the same
+            b.record()
+            t_mrg.append((a, b))
+            parts = []
+            for r, s in enumerate(shards):
+                a, b = ev(), ev()
+                a.record()
+                parts.append(s.attend_local(Q[c0:c1], K[s.t0:s.t1], V[s.t0:s.t1], lists, lens, ws=ws_attn))
+                b.record()
+                t_att[r].append((a, b))
+            Op, Lp = torch.stack([p_[0] for p_ in parts]), torch.stack([p_[1] for p_ in parts])
+            a, b = ev(), ev()
+            a.record()
+            CP.Shard.combine(Op, Lp)
+            b.record()
+            t_cmb.append((a, b))
+        torch.cuda.synchronize()
+        if not record:
+            return None
+        ms = lambda L: sum(a.elapsed_time(b) for a, b in L)  # noqa: E731
+        return ([ms(L) for L in t_loc], ms(t_mrg), [ms(L) for L in t_att], ms(t_cmb))
+
+    one_pass(False)
+    loc, mrg, att, cmb = one_pass(True)
+    per_rank = [loc[r] + mrg + att[r] + cmb for r in range(ranks)]
+    step = max(per_rank)
+    xbytes = lsa.lsa_shard_exchange_bytes(nq, shards[0].p)
+    part_bytes = nq * hq * (128 * 2 + 4)
+    return {"ranks": ranks, "emulated_on_one_gpu": True, "queries": nq, "chunk": chunk,
+            "build_ms_max_rank": round(max(a.elapsed_time(b) for a, b in t_build), 3),
+            "index_local_ms": {"max_rank": round(max(loc), 3), "min_rank": round(min(loc), 3)},
+            "merge_and_expand_ms": round(mrg, 3),
+            "attention_local_ms": {"max_rank": round(max(att), 3), "min_rank": round(min(att), 3)},
+            "combine_ms": round(cmb, 3), "step_ms_slowest_rank": round(step, 3),
+            "tokens_per_s_without_communication": round(nq / (step / 1e3), 1),
+            "allgather_bytes_sent_per_rank": xbytes + part_bytes,
+            "allgather_bytes_received_per_rank": (ranks - 1) * (xbytes + part_bytes),
+            "note": "kernel time per rank only; the all-gathers of exchange blocks and attention parts are not timed"}
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -348,6 +433,9 @@ def run_ours(args, world, rank, local):
     index_heads = None
     if wl["mode"] == "flat" and not args.no_heads:
         index_heads = measure_index_heads(layer, keys_np, pos_np, wl, dev)
+    context_parallel = None
+    if args.cp > 1 and wl["mode"] == "flat":
+        context_parallel = measure_context_parallel(wl, keys_np, pos_np, q_np, Q, K, V, dev, args.cp)
 
     # end to end: same calls, inputs from pinned host memory, output back to host
     e2e = None if args.no_e2e else run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
@@ -381,6 +469,8 @@ def run_ours(args, world, rank, local):
         "decode": decode,
         "index_heads": index_heads,
     }
+    if context_parallel is not None:
+        line["context_parallel"] = context_parallel
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
@@ -614,6 +704,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-heads", action="store_true", help="skip the multi-head Flat index measurement")
+    ap.add_argument("--cp", type=int, default=0,
+                    help="also run an N-way context-parallel split, its ranks one after another on this GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()

@@ -1246,15 +1246,19 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
     __syncthreads();
     const int E = s_off[heads];
     const float tstar = s_tstar;
-    // a query's table: 1.5 slots per entry (entries hold about one kept score
-    // each); one that fills is redone once with all of the launch's slots,
-    // and a union that fills those takes the exact path
-    int TS = min(TSMAX, max(64, E + E / 2));
+    // a query's table: 2 slots per entry (entries hold one to two kept
+    // scores); one that fills is redone once with all of the launch's
+    // slots, and a union that fills those takes the exact path
+    // one row (a shard's own candidates) holds no bucket twice: its kept
+    // scores are appended as a list instead of hashed
+    const bool direct = heads == 1;
+    int TS = min(TSMAX, max(64, 2 * E));
     for (;;) {  // block-uniform, at most two rounds
-        for (int i = t; i < TS; i += HM_THREADS) {
-            hkey[i] = -1;
-            hval[i] = 0u;
-        }
+        if (!direct)
+            for (int i = t; i < TS; i += HM_THREADS) {
+                hkey[i] = -1;
+                hval[i] = 0u;
+            }
         if (t == 0) {
             s_full = 0;
             s_uniq = 0;
@@ -1302,9 +1306,21 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
                         if (qn >= 32) {  // warp-uniform
                             __syncwarp();
                             const uint2 w = wq[warp][lane];
-                            const int r = hash_insert(hkey, hval, TS, (int32_t)w.x, w.y);
-                            fresh += r > 0;
-                            full |= r < 0;
+                            if (direct) {
+                                int base = 0;
+                                if (lane == 0) base = atomicAdd(&s_uniq, 32);
+                                base = __shfl_sync(LSA_FULL, base, 0);
+                                if (base + lane < TS) {
+                                    hkey[base + lane] = (int32_t)w.x;
+                                    hval[base + lane] = w.y;
+                                } else {
+                                    full = 1;
+                                }
+                            } else {
+                                const int r = hash_insert(hkey, hval, TS, (int32_t)w.x, w.y);
+                                fresh += r > 0;
+                                full |= r < 0;
+                            }
                             __syncwarp();
                             if (lane < qn - 32) wq[warp][lane] = wq[warp][32 + lane];
                             __syncwarp();
@@ -1314,7 +1330,19 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
                 }
             }
             __syncwarp();
-            if (lane < qn) {
+            if (direct) {
+                int base = 0;
+                if (lane == 0 && qn) base = atomicAdd(&s_uniq, qn);
+                base = __shfl_sync(LSA_FULL, base, 0);
+                if (lane < qn) {
+                    if (base + lane < TS) {
+                        hkey[base + lane] = (int32_t)wq[warp][lane].x;
+                        hval[base + lane] = wq[warp][lane].y;
+                    } else {
+                        full = 1;
+                    }
+                }
+            } else if (lane < qn) {
                 const uint2 w = wq[warp][lane];
                 const int r = hash_insert(hkey, hval, TS, (int32_t)w.x, w.y);
                 fresh += r > 0;
@@ -1351,11 +1379,17 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
     if (!s_exact) {
         const float lo = ord2f(s_vmin), hi = ord2f(s_vmax);
         const float scale = hi > lo ? 256.0f / (hi - lo) : 0.0f;
+        const int scan = direct ? min(U, TS) : TS;  // slots that may hold a bucket
         int bstar = 0;
         uint32_t cut = 0u;
         if (U > KC) {
-            for (int i = t; i < TS; i += HM_THREADS)
-                if (hkey[i] >= 0) atomicAdd(&hist[merge_bin(ord2f(hval[i]), lo, scale)], 1);
+            const int n_round = (scan + HM_THREADS - 1) / HM_THREADS * HM_THREADS;
+            for (int i = t; i < n_round; i += HM_THREADS) {
+                const int bin = (i < scan && hkey[i] >= 0) ? merge_bin(ord2f(hval[i]), lo, scale) : -1;
+                // lanes with the same bin add once (values cluster in few bins)
+                const unsigned peers = __match_any_sync(LSA_FULL, bin);
+                if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+            }
             __syncthreads();
             if (t < 32) {  // warp 0: lane l owns bins 255-8l .. 248-8l
                 int c8 = 0;
@@ -1385,11 +1419,11 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
             bstar = s_bstar;
             if (s_keep > KC) {  // block-uniform: too many at the boundary bin
                 auto get = [&](int64_t i) { return hkey[i] >= 0 ? ord2f(hval[i]) : NEG; };
-                cut = block_select_kth_largest(TS, P, get, hist, sh);
+                cut = block_select_kth_largest(scan, P, get, hist, sh);
                 bstar = -1;
             }
         }
-        for (int i = t; i < TS; i += HM_THREADS) {
+        for (int i = t; i < scan; i += HM_THREADS) {
             const int32_t id = hkey[i];
             const uint32_t v = hval[i];
             const bool take = id >= 0 && (U <= KC || (bstar >= 0 ? merge_bin(ord2f(v), lo, scale) >= bstar : v >= cut));

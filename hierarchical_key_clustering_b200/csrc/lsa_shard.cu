@@ -27,9 +27,13 @@ __device__ uint32_t shard_select(int64_t n, int64_t P, Get get, int *hist, int *
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint32_t u = get(i);
-            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1);
+        const int64_t n_round = (n + blockDim.x - 1) / blockDim.x * blockDim.x;
+        for (int64_t i = threadIdx.x; i < n_round; i += blockDim.x) {
+            const uint32_t u = i < n ? get(i) : 0u;
+            const int bin = (i < n && (u & mask) == prefix) ? (int)((u >> shift) & 255) : -1;
+            // lanes with the same bin add once (scores cluster in few bins)
+            const unsigned peers = __match_any_sync(LSA_FULL, bin);
+            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
         }
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -78,11 +82,20 @@ cudaError_t launch_shard_pack(const IndexWs &m, int64_t nq, int64_t g0, void *xc
     return cudaGetLastError();
 }
 
+// Histogram bin of a value over [lo, lo + 256 / scale] (monotone in v): the
+// same rounded operations in the counting and the keeping pass.
+__device__ __forceinline__ int merge_bin_shard(float v, float lo, float scale)
+{
+    return min(255, max(0, __float2int_rz(__fmul_rn(__fsub_rn(v, lo), scale))));
+}
+
 // ---------------------------------------------------------------------------
 // Global top P of the union of the ranks' sets (disjoint bucket ids, exact
 // scores).  One CTA per query stages the union in shared memory; all of it
-// is kept when it fits the expansion's slots, else the buckets above the
-// P-th score and, at that score, the ties with the lowest ids up to P.
+// is kept when it fits the expansion's slots, else every bucket from the
+// histogram bin holding the P-th best value up when those fit, else the
+// buckets above the P-th score and, at that score, the ties with the lowest
+// ids up to P.
 constexpr int SM_THREADS = 512;
 
 __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__restrict__ xcnt_all,
@@ -95,7 +108,8 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
     __shared__ int hist[256];
     __shared__ int sh[4];
     __shared__ int s_off[LSA_MAXHEADS + 1];
-    __shared__ int s_out;
+    __shared__ int s_out, s_bstar, s_keep;
+    __shared__ uint32_t s_vmin, s_vmax;
     const int64_t q = blockIdx.x;
     const int t = threadIdx.x;
     const float NEG = __int_as_float(0xff800000);
@@ -128,6 +142,64 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
         }
         if (t == 0) s_out = n;
     } else {
+        // one 256-bin histogram over the union's [min, max]: every bucket
+        // from the bin holding the P-th best value up holds the top P, and
+        // is kept when it fits the expansion's slots
+        uint32_t vmin = ~0u, vmax = 0u;
+        for (int i = t; i < n; i += SM_THREADS) {
+            vmin = min(vmin, um[i].x);
+            vmax = max(vmax, um[i].x);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            vmin = min(vmin, __shfl_xor_sync(LSA_FULL, vmin, o));
+            vmax = max(vmax, __shfl_xor_sync(LSA_FULL, vmax, o));
+        }
+        if (t == 0) s_vmin = ~0u, s_vmax = 0u;
+        for (int i = t; i < 256; i += SM_THREADS) hist[i] = 0;
+        __syncthreads();
+        if ((t & 31) == 0) {
+            atomicMin(&s_vmin, vmin);
+            atomicMax(&s_vmax, vmax);
+        }
+        __syncthreads();
+        const float lo = ord2f(s_vmin), hi = ord2f(s_vmax);
+        const float scale = hi > lo ? 256.0f / (hi - lo) : 0.0f;
+        const int n_round = (n + SM_THREADS - 1) / SM_THREADS * SM_THREADS;
+        for (int i = t; i < n_round; i += SM_THREADS) {
+            const int bin = i < n ? merge_bin_shard(ord2f(um[i].x), lo, scale) : -1;
+            const unsigned peers = __match_any_sync(LSA_FULL, bin);
+            if (bin >= 0 && (t & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+        __syncthreads();
+        if (t == 0) {
+            int acc = 0, d = 255;
+            for (; d > 0; --d) {
+                if (acc + hist[d] >= P) break;
+                acc += hist[d];
+            }
+            s_bstar = d;
+            s_keep = acc + hist[d];
+        }
+        __syncthreads();
+        if (s_keep <= KC) {  // block-uniform
+            const int bstar = s_bstar;
+            for (int i = t; i < n; i += SM_THREADS) {
+                const uint2 u = um[i];
+                if (merge_bin_shard(ord2f(u.x), lo, scale) >= bstar) {
+                    const int j = atomicAdd(&s_out, 1);
+                    o4[j] = make_float4(ord2f(u.x), NEG, NEG, NEG);
+                    og[j] = (int32_t)u.y;
+                }
+            }
+            __syncthreads();
+            if (t == 0) {
+                m.cnt[q] = s_out;
+                m.tau[q] = NEG;
+                m.horizon[q] = 0;
+            }
+            return;
+        }
         const uint32_t cut = shard_select(n, P, [&](int64_t i) { return um[i].x; }, hist, sh);
         int above = 0, ties = 0;
         for (int i = t; i < n; i += SM_THREADS) {
@@ -182,7 +254,7 @@ cudaError_t launch_shard_merge(const void *xchg_all, int n_shards, int64_t nq, i
 
 // ---------------------------------------------------------------------------
 // The entries of each list in [t0, t1), shifted to the rank's K/V rows.  One
-// warp per query; the order is kept, the rest of the row is -1.
+// warp per query; the order is kept, the rest of the row is not written.
 __global__ void __launch_bounds__(256) k_local_lists(const int32_t *__restrict__ lists,
                                                      const int32_t *__restrict__ lens, int64_t nq, int32_t Lmax,
                                                      int64_t t0, int64_t t1, int32_t *__restrict__ out_lists,
@@ -205,7 +277,6 @@ __global__ void __launch_bounds__(256) k_local_lists(const int32_t *__restrict__
         if (keep) out[n + __popc(bal & ((1u << lane) - 1u))] = (int32_t)(v - t0);
         n += __popc(bal);
     }
-    for (int i = n + lane; i < Lmax; i += 32) out[i] = -1;
     if (lane == 0) out_lens[q] = n;
 }
 

@@ -396,7 +396,8 @@ int lsa_shard_publish_members(const lsa_cache *cache, int64_t b_first, int32_t *
                               void *stream);
 
 /* The entries of each list inside [t_begin, t_end), in order, minus t_begin
- * (this rank's K/V rows); out_lists [nq, Lmax] -1 padded, out_lens [nq]. */
+ * (this rank's K/V rows); out_lists [nq, Lmax] (entries past out_lens[i]
+ * are left unwritten), out_lens [nq]. */
 int lsa_shard_local_lists(const int32_t *lists, const int32_t *lens, int64_t nq, int32_t Lmax, int64_t t_begin,
                           int64_t t_end, int32_t *out_lists, int32_t *out_lens, void *stream);
 
