@@ -1246,13 +1246,14 @@ __global__ void __launch_bounds__(HM_THREADS, 2) k_heads_merge(int heads, int P,
     __syncthreads();
     const int E = s_off[heads];
     const float tstar = s_tstar;
-    // a query's table: 2 slots per entry (entries hold one to two kept
-    // scores); one that fills is redone once with all of the launch's
-    // slots, and a union that fills those takes the exact path
-    // one row (a shard's own candidates) holds no bucket twice: its kept
-    // scores are appended as a list instead of hashed
+    // a query's table: 1.5 slots per entry for several heads (their union
+    // has about 0.7 buckets per entry), 2 for one row (about 1.4 kept
+    // scores per entry when a shard holds few blocks); one that fills is
+    // redone once with all of the launch's slots, and a union that fills
+    // those takes the exact path.  One row (a shard's own candidates) holds
+    // no bucket twice: its kept scores are appended as a list, not hashed.
     const bool direct = heads == 1;
-    int TS = min(TSMAX, max(64, 2 * E));
+    int TS = min(TSMAX, max(64, direct ? 2 * E : E + E / 2));
     for (;;) {  // block-uniform, at most two rounds
         if (!direct)
             for (int i = t; i < TS; i += HM_THREADS) {
