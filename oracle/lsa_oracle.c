@@ -19,8 +19,7 @@
  *           latent, L2-norm, pool 4, 512-key blocks, Ward, <=16 keys,
  *           Flat vs Tree).
  *
- * Readings taken where the pages are silent (each also listed in the
- * design notes):
+ * Readings taken where the pages are silent, labelled R1.. in this file:
  *   R1  64-term sums of squares use one fixed order: t_l = f(x_l) + f(x_{l+32})
  *       for l < 32, then t_l += t_{l+s} for s = 16, 8, 4, 2, 1; result t_0.
  *       No fused multiply-add anywhere on the build path.
