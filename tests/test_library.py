@@ -168,3 +168,48 @@ def test_binding_raises_on_error(name):
         else:
             lsa._check(lsa.lib().lsa_sparse_attention(None, None, None, 1, 0, 0, 128, 1, None, None, 1, 1.0, None,
                                                       None, None, 0, None))
+
+
+def test_shard_sizes_and_argument_errors():
+    """Context-parallel calls: slot count and exchange-block size as the
+    header states them, and the argument checks (no kernel is launched)."""
+    L = lsa.lib()
+    p = lsa.lsa_default_params(k=2048)
+    P = lsa.lsa_top_buckets(p)
+    slots = lsa.lsa_shard_slots(p)
+    assert slots == min(2 ** math.ceil(math.log2(2 * P)), 2 ** math.ceil(math.log2((3 * P + 1) // 2)))
+    assert lsa.lsa_shard_exchange_bytes(1000, p) == 4096 + 1000 * slots * 8
+    assert lsa.lsa_shard_exchange_bytes(1000, p) % 256 == 0
+    assert lsa.lsa_shard_local_workspace_bytes(1000, 32, p) > lsa.lsa_index_workspace_bytes(1000, 32, p)
+    assert lsa.lsa_shard_merge_workspace_bytes(1000, p) > 1000 * slots * 20
+    cache = lsa.lsa_cache()
+    _expect(L.lsa_cache_bind(FAKE, L.lsa_cache_bytes(4096), 4096, C.byref(cache)), 0)
+    cache.n_blocks = 8
+    big = 1 << 40
+    Lmax = L.lsa_list_budget(C.byref(p))
+    # local step: Tree mode, NULL exchange block, unaligned block, negative first block
+    tp = lsa.lsa_default_params(k=2048, mode="tree")
+    _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), 0, FAKE, C.byref(tp), FAKE, big, None), -1)
+    _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), 0, None, C.byref(p), FAKE, big, None), -1)
+    _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), 0, C.c_void_p((1 << 20) + 16), C.byref(p),
+                                    FAKE, big, None), -1)
+    _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), -1, FAKE, C.byref(p), FAKE, big, None), -2)
+    _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), 0, FAKE, C.byref(p), None, 0, None), -5)
+    # merge: rank count, Tree mode, list budget, workspace
+    for n_shards in (0, 17):
+        _expect(L.lsa_index_shard_merge(FAKE, n_shards, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(p), FAKE,
+                                        big, None), -1)
+    _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(tp), FAKE, big,
+                                    None), -1)
+    _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax - 1, C.byref(p), FAKE, big,
+                                    None), -2)
+    _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(p), FAKE, 16, None),
+            -5)
+    _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 0, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(p), None, 0, None), 0)
+    # local lists, member slices, combine
+    _expect(L.lsa_shard_local_lists(FAKE, FAKE, 10, Lmax, 100, 50, FAKE, FAKE, None), -2)
+    _expect(L.lsa_shard_local_lists(FAKE, FAKE, 10, Lmax, 0, 50, FAKE, FAKE, None), -1)  # output aliases input
+    _expect(L.lsa_shard_publish_members(C.byref(cache), -1, FAKE, FAKE, None), -2)
+    _expect(L.lsa_attention_combine(FAKE, FAKE, 2, 10, 32, 64, FAKE, None, None), -1)
+    _expect(L.lsa_attention_combine(FAKE, FAKE, 0, 10, 32, 128, FAKE, None, None), -2)
+    _expect(L.lsa_attention_combine(FAKE, FAKE, 2, 0, 32, 128, FAKE, None, None), 0)
