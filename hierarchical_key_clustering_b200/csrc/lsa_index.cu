@@ -80,61 +80,11 @@ __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *_
 }
 
 // ---------------------------------------------------------------------------
-// Radix select: the P-th largest key (u = f2ord(score)) among values produced
-// by `get(i)` for i in [0, n); all threads of the block call it.
+// Radix select over scores: the P-th largest f2ord(get(i)), i in [0, n).
 template <typename Get>
 __device__ uint32_t block_select_kth_largest(int64_t n, int64_t P, Get get, int *hist, int *sh)
 {
-    uint32_t prefix = 0, mask = 0;
-    int64_t rem = P;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        const int64_t n_round = ((n + blockDim.x - 1) / blockDim.x) * blockDim.x;
-        for (int64_t i = threadIdx.x; i < n_round; i += blockDim.x) {
-            const bool valid = i < n;
-            const uint32_t u = valid ? f2ord(get(i)) : 0u;
-            const int bin = (valid && (u & mask) == prefix) ? (int)((u >> shift) & 255) : -1;
-            // lanes with the same bin add once (scores cluster in few bins)
-            const unsigned peers = __match_any_sync(LSA_FULL, bin);
-            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            // warp 0: lane l owns bins 255-8l .. 248-8l (descending); find the
-            // bin where the count from the top first reaches rem
-            const int lane = threadIdx.x;
-            int c8 = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) c8 += hist[255 - 8 * lane - e];
-            int incl = c8;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(LSA_FULL, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const int excl = incl - c8;
-            if (excl < rem && rem <= incl) {
-                int acc = excl, digit = 255 - 8 * lane;
-                for (int e = 0; e < 8; ++e) {
-                    const int d = 255 - 8 * lane - e;
-                    if (acc + hist[d] >= rem) {
-                        digit = d;
-                        break;
-                    }
-                    acc += hist[d];
-                }
-                sh[0] = digit;
-                sh[1] = (int)(rem - acc);
-            }
-        }
-        __syncthreads();
-        prefix |= ((uint32_t)sh[0]) << shift;
-        mask |= 255u << shift;
-        rem = sh[1];
-        __syncthreads();
-    }
-    return prefix;
+    return block_select_ord(n, P, [&](int64_t i) { return f2ord(get(i)); }, hist, sh);
 }
 
 // ---------------------------------------------------------------------------

@@ -17,44 +17,6 @@
 
 namespace lsa {
 
-// Radix select over values produced by get(i), i < n (lsa_index.cu has the
-// same selection for its own callers): the P-th largest ordered key.
-template <typename Get>
-__device__ uint32_t shard_select(int64_t n, int64_t P, Get get, int *hist, int *sh)
-{
-    uint32_t prefix = 0, mask = 0;
-    int64_t rem = P;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        const int64_t n_round = (n + blockDim.x - 1) / blockDim.x * blockDim.x;
-        for (int64_t i = threadIdx.x; i < n_round; i += blockDim.x) {
-            const uint32_t u = i < n ? get(i) : 0u;
-            const int bin = (i < n && (u & mask) == prefix) ? (int)((u >> shift) & 255) : -1;
-            // lanes with the same bin add once (scores cluster in few bins)
-            const unsigned peers = __match_any_sync(LSA_FULL, bin);
-            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int64_t acc = 0;
-            int d = 255;
-            for (; d > 0; --d) {
-                if (acc + hist[d] >= rem) break;
-                acc += hist[d];
-            }
-            sh[0] = d;
-            sh[1] = (int)(rem - acc);
-        }
-        __syncthreads();
-        prefix |= ((uint32_t)sh[0]) << shift;
-        mask |= 255u << shift;
-        rem = sh[1];
-        __syncthreads();
-    }
-    return prefix;
-}
-
 // ---------------------------------------------------------------------------
 // A rank's merged local set (one-bucket entries, local bucket ids) into its
 // exchange block with global bucket ids (g0 = 64 x the rank's first block).
@@ -200,7 +162,7 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
             }
             return;
         }
-        const uint32_t cut = shard_select(n, P, [&](int64_t i) { return um[i].x; }, hist, sh);
+        const uint32_t cut = block_select_ord(n, P, [&](int64_t i) { return um[i].x; }, hist, sh);
         int above = 0, ties = 0;
         for (int i = t; i < n; i += SM_THREADS) {
             above += um[i].x > cut;
@@ -218,7 +180,7 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
         if (n_above + n_ties > KC) {
             const int need = P - n_above;
             // the need-th smallest id among the ties = the need-th largest of ~id
-            idcut = ~shard_select(n, need, [&](int64_t i) { return um[i].x == cut ? ~um[i].y : 0u; }, hist, sh);
+            idcut = ~block_select_ord(n, need, [&](int64_t i) { return um[i].x == cut ? ~um[i].y : 0u; }, hist, sh);
         }
         for (int i = t; i < n; i += SM_THREADS) {
             const uint2 u = um[i];
