@@ -173,6 +173,67 @@ def test_1m_flat_prefill_and_decode(big1m):
     PT.assert_lists_match(np.stack(gl), np.array(gn), ol, on, dq, dpos, oc, k=k)
 
 
+def test_1m_context_parallel_eight_ranks(big1m):
+    """The 1M Flat prefill split over 8 token ranges (256 blocks each), the
+    ranks run stage by stage in this process in the benchmark's chunks of
+    16384 queries: lists equal the single-GPU lists of every query (the same
+    tensor-core score for every (query, bucket), the same tie order), sampled
+    lists equal the oracle's, sampled combined attention its attention."""
+    from hierarchical_key_clustering_b200 import context_parallel as CP
+
+    wl, keys_all, oc, cache, _ = big1m
+    T, k, npre = wl["T"], wl["k"], wl["n_prefill"]
+    hq, hkv, chunk, ranks = wl["hq"], wl["hkv"], 16384, 8
+    pos = np.arange(T - npre, T, dtype=np.int64)
+    q = I.index_queries(0, keys_all, pos)
+    shards = [CP.Shard(r, ranks, T, k=k, max_queries=chunk) for r in range(ranks)]
+    kd = PT.to_dev(keys_all[:T])
+    built = [s.build(kd[s.t0:s.t1]) for s in shards]
+    M, C = torch.stack([b[0] for b in built]), torch.stack([b[1] for b in built])
+    for s in shards:
+        s.set_members(M, C)
+    del kd
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    Q = torch.randn((npre, hq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    K = torch.randn((T, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((T, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    qd, pd = PT.to_dev(q), PT.to_dev(pos)
+    lists = torch.empty((npre, shards[0].Lmax), dtype=torch.int32, device="cuda")
+    lens = torch.empty((npre,), dtype=torch.int32, device="cuda")
+    O_ = torch.empty_like(Q)
+    lse = torch.empty((npre, hq), dtype=torch.float32, device="cuda")
+    for c0 in range(0, npre, chunk):
+        c1 = min(npre, c0 + chunk)
+        X = torch.stack([s.index_local(qd[c0:c1], pd[c0:c1]) for s in shards]).reshape(-1)
+        l_, n_ = shards[0].index_merge(X, pd[c0:c1])
+        lists[c0:c1].copy_(l_)
+        lens[c0:c1].copy_(n_)
+        parts = [s.attend_local(Q[c0:c1], K[s.t0:s.t1], V[s.t0:s.t1], lists[c0:c1], lens[c0:c1]) for s in shards]
+        o, l2 = CP.Shard.combine(torch.stack([x[0] for x in parts]), torch.stack([x[1] for x in parts]))
+        O_[c0:c1].copy_(o)
+        lse[c0:c1].copy_(l2)
+    torch.cuda.synchronize()
+    single_l, single_n = _gpu_index(cache, None, lsa.lsa_default_params(k=k), q, pos)
+    same = (lens == single_n) & torch.all(lists == single_l, dim=1)
+    assert same.float().mean().item() >= 0.999, f"only {same.float().mean().item():.4f} equal the single-GPU lists"
+    sel = np.linspace(0, npre - 1, 96).astype(np.int64)
+    ix = torch.from_numpy(sel).cuda()
+    ol, on = O.index(q[sel], pos[sel], oc, k=k)
+    PT.assert_lists_match(lists[ix].cpu().numpy(), lens[ix].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
+    sa = sel[::6]
+    ia = torch.from_numpy(sa).cuda()
+    la, na = lists[ia].cpu().numpy(), lens[ia].cpu().numpy()
+    used = np.unique(la[la >= 0])
+    remap = np.full(T, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    ll = np.where(la >= 0, remap[np.maximum(la, 0)], -1).astype(np.int32)
+    ui = torch.from_numpy(used.astype(np.int64)).cuda()
+    bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
+    Oref, lse_ref = O.attention(bits(Q[ia]), bits(K.index_select(0, ui)), bits(V.index_select(0, ui)), ll, na)
+    PT.assert_attention_close(O_[ia], Oref, lse[ia], lse_ref)
+
+
 def test_1m_tree_prefill_and_decode(big1m):
     wl, keys_all, oc, cache, tree = big1m
     T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
