@@ -742,7 +742,8 @@ int lsa_index_shard_merge(const void *xchg_all, int32_t n_shards, const int64_t 
                     LSA_MAX_INDEX_HEADS, (long long)KC);
     if (!xchg_all || !pos || !lists || !lens || (n_blocks > 0 && (!members || !count)))
         return fail(LSA_ERR_ARG, "xchg_all, pos, members, count, lists and lens must be non-NULL");
-    if (((uintptr_t)xchg_all & 255u) || !aligned16(lists)) return fail(LSA_ERR_ARG, "xchg_all must be 256-byte and lists 16-byte aligned");
+    if (((uintptr_t)xchg_all & 255u) || !aligned16(lists) || (members && !aligned16(members)))
+        return fail(LSA_ERR_ARG, "xchg_all must be 256-byte, lists and members 16-byte aligned");
     if (Lmax < lsa_list_budget(p)) return fail(LSA_ERR_SHAPE, "Lmax %d < list budget %d", Lmax, lsa_list_budget(p));
     if (lsa::rank_expand_smem_bytes((int)KC, n_blocks) > 227 * 1024)
         return fail(LSA_ERR_ARG, "%lld blocks too many for the expansion kernel", (long long)n_blocks);

@@ -380,8 +380,9 @@ int lsa_index_shard_local(const float *qidx, const int64_t *pos, int64_t nq, con
  * order (xchg_all): per query the union's top P by (score desc, bucket id
  * asc), expanded as lsa_index_prefill does, over the replicated member table
  * and counts of all n_blocks blocks (members [n_blocks*64, 16] global
- * positions, count [n_blocks*64]; see lsa_shard_publish_members).  Lists as
- * lsa_index_prefill.  ws: lsa_shard_merge_workspace_bytes. */
+ * positions, 16-byte aligned, count [n_blocks*64]; see
+ * lsa_shard_publish_members).  Lists as lsa_index_prefill.
+ * ws: lsa_shard_merge_workspace_bytes. */
 int lsa_index_shard_merge(const void *xchg_all, int32_t n_shards, const int64_t *pos, int64_t nq,
                           const int32_t *members, const int32_t *count, int64_t n_blocks, int32_t *lists,
                           int32_t *lens, int32_t Lmax, const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);

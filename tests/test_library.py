@@ -205,6 +205,8 @@ def test_shard_sizes_and_argument_errors():
                                     None), -2)
     _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(p), FAKE, 16, None),
             -5)
+    _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 10, C.c_void_p((1 << 20) + 4), FAKE, 8, FAKE, FAKE, Lmax,
+                                    C.byref(p), FAKE, big, None), -1)  # member rows are read 16 bytes at a time
     _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 0, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(p), None, 0, None), 0)
     # local lists, member slices, combine
     _expect(L.lsa_shard_local_lists(FAKE, FAKE, 10, Lmax, 100, 50, FAKE, FAKE, None), -2)
