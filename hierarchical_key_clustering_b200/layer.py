@@ -11,6 +11,28 @@ import torch
 from . import lsa
 
 
+def chunk_plan(pos, chunks: int, n_kv_heads: int, tk: int):
+    """Query chunks of prefill_from_host and the K/V rows each one needs.
+
+    The queries are cut into `chunks` pieces rounded up to multiples of 128
+    (so the near-set tiles of the attention do not change).  The last
+    chunk's copy back is the only one nothing overlaps, so it is split into
+    quarters (multiples of 128 queries) when each quarter still has the
+    2048 (query, KV head) units that keep its attention on whole lists.
+    A chunk's lists hold positions up to its largest query position, so it
+    needs K/V rows [0, min(tk, max pos + 1)).  Returns ([(c0, c1)], [rows])."""
+    nq = len(pos)
+    step = -(-nq // max(1, chunks))
+    step = -(-step // 128) * 128
+    bounds = [(c0, min(nq, c0 + step)) for c0 in range(0, nq, step)]
+    c0, c1 = bounds[-1]
+    q4 = -(-((c1 - c0) // 4) // 128) * 128
+    if len(bounds) > 1 and q4 >= 128 and q4 * n_kv_heads >= 2048:
+        bounds = bounds[:-1] + [(a, min(c1, a + q4)) for a in range(c0, c1, q4)]
+    need = [min(tk, int(pos[c0:c1].max()) + 1) for c0, c1 in bounds]
+    return bounds, need
+
+
 class SparseLayer:
     def __init__(self, capacity: int, k: int = 4096, mode: str = "flat", beam: int = 32, sink: int = 4,
                  window: int = 512, max_queries: int = 1, Hq: int = 32, head_dim: int = 128,
@@ -105,19 +127,7 @@ class SparseLayer:
             self._dbuf_key = key
         d_keys, d_q, d_pos, d_Q, d_K, d_V, d_O = self._dbuf
         tk = h_K.shape[0]
-        step = -(-nq // max(1, chunks))
-        step = -(-step // 128) * 128
-        bounds = [(c0, min(nq, c0 + step)) for c0 in range(0, nq, step)]
-        # the last chunk's copy back is the only one nothing overlaps: split it
-        # into quarters (multiples of 128 queries) to shorten that tail, when
-        # each quarter still has the (query, KV head) units that keep its
-        # attention on whole lists (2048)
-        c0, c1 = bounds[-1]
-        q4 = -(-((c1 - c0) // 4) // 128) * 128
-        if len(bounds) > 1 and q4 >= 128 and q4 * h_K.shape[1] >= 2048:
-            bounds = bounds[:-1] + [(a, min(c1, a + q4)) for a in range(c0, c1, q4)]
-        # K/V rows each chunk needs: its lists hold positions <= its largest query position
-        need = [min(tk, int(h_pos[c0:c1].max()) + 1) for c0, c1 in bounds]
+        bounds, need = chunk_plan(h_pos, chunks, h_K.shape[1], tk)
         self._h2d.wait_stream(cs)
         with torch.cuda.stream(self._h2d):
             d_keys.copy_(h_keys, non_blocking=True)  # the build needs only the keys

@@ -215,3 +215,29 @@ def test_shard_sizes_and_argument_errors():
     _expect(L.lsa_attention_combine(FAKE, FAKE, 2, 10, 32, 64, FAKE, None, None), -1)
     _expect(L.lsa_attention_combine(FAKE, FAKE, 0, 10, 32, 128, FAKE, None, None), -2)
     _expect(L.lsa_attention_combine(FAKE, FAKE, 2, 0, 32, 128, FAKE, None, None), 0)
+
+
+@pytest.mark.parametrize("nq,chunks,hkv,T", [(131072, 16, 8, 131072), (32768, 16, 8, 1048576), (1000, 16, 8, 4096),
+                                             (300, 5, 1, 4096), (128, 1, 8, 4096), (5000, 3, 2, 10000)])
+def test_prefill_chunk_plan(nq, chunks, hkv, T):
+    """Host plan of prefill_from_host: contiguous chunks covering every query,
+    starting on multiples of 128; the last chunk quartered only when each
+    quarter keeps 2048 (query, KV head) units; each chunk's K/V rows reach
+    its largest position (ascending positions: non-decreasing)."""
+    import torch
+
+    from hierarchical_key_clustering_b200.layer import chunk_plan
+
+    pos = torch.arange(T - nq, T, dtype=torch.int64)
+    bounds, need = chunk_plan(pos, chunks, hkv, T)
+    assert bounds[0][0] == 0 and bounds[-1][1] == nq
+    assert all(a[1] == b[0] for a, b in zip(bounds, bounds[1:]))
+    assert all(c0 % 128 == 0 and c1 > c0 for c0, c1 in bounds)
+    step = -(-(-(-nq // chunks)) // 128) * 128
+    main = [b for b in bounds if b[1] - b[0] == step]
+    assert len(main) >= len(bounds) - 4
+    tail = bounds[len(main):]
+    if len(tail) > 1:  # quartered: each piece a multiple of 128 (but the last) with >= 2048 units
+        assert all((c1 - c0) * hkv >= 2048 for c0, c1 in tail[:-1])
+    assert need == [min(T, int(pos[c1 - 1]) + 1) for c0, c1 in bounds]
+    assert all(a <= b for a, b in zip(need, need[1:]))
