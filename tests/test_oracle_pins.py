@@ -586,3 +586,44 @@ def test_shrink_small_integers_exact():
     x = O.shrink(to_bits(vi), to_bits(wi))
     exact = np.einsum("td,ed->te", vi, wi)  # integer arithmetic
     assert np.array_equal(x, exact.astype(np.float32))
+
+
+# ---------------------------------------------------------------- selection arguments the merges rely on
+
+@pytest.mark.parametrize("seed", range(6))
+def test_union_of_head_candidates_holds_top_p_by_best_score(seed):
+    """Every head lists every bucket scoring >= tau_h, tau_h <= its P-th
+    score.  Then the buckets listed at or above tau* = max_h tau_h, each with
+    the best score any head listed for it, hold the top P by best score over
+    all heads, with exact values (quantised scores make ties likely)."""
+    rng = np.random.default_rng(seed)
+    H, N, P = int(rng.integers(2, 9)), int(rng.integers(50, 400)), int(rng.integers(5, 40))
+    S = np.round(rng.standard_normal((H, N)) * 8) / 8  # many ties
+    taus = [np.sort(S[h])[::-1][P - 1] - rng.uniform(0, 0.5) for h in range(H)]
+    tstar = max(taus)
+    known = {}
+    for h in range(H):
+        for b in np.nonzero(S[h] >= taus[h])[0]:
+            if S[h, b] >= tstar:
+                known[b] = max(known.get(b, -np.inf), S[h, b])
+    best = S.max(0)
+    top = sorted(range(N), key=lambda b: (-best[b], b))[:P]
+    got = sorted(known, key=lambda b: (-known[b], b))[:P]
+    assert got == top
+    assert all(known[b] == best[b] for b in top)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_union_of_shard_top_p_holds_global_top_p(seed):
+    """Each shard sends its own top P (by score desc, id asc); the top P of
+    the union is the global top P."""
+    rng = np.random.default_rng(100 + seed)
+    N, P, R = int(rng.integers(80, 600)), int(rng.integers(5, 60)), int(rng.integers(2, 9))
+    s = np.round(rng.standard_normal(N) * 6) / 6
+    cuts = np.sort(rng.choice(np.arange(1, N), R - 1, replace=False))
+    parts = np.split(np.arange(N), cuts)
+    union = []
+    for ids in parts:
+        union += sorted(ids.tolist(), key=lambda b: (-s[b], b))[:P]
+    key = lambda b: (-s[b], b)  # noqa: E731
+    assert sorted(union, key=key)[:P] == sorted(range(N), key=key)[:P]
