@@ -1106,16 +1106,17 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
 // the largest score any head listed for it, and cutting at the P-th largest
 // of those values keeps exactly the top P: a kept value falls short of a
 // bucket's best only for buckets outside the top P.  Scores below
-// tau* = max over heads of tau_h are dropped first: every head's top P score
-// at least tau_h, so at least P buckets have a best score >= tau_h for every
-// h, and the P-th best is >= tau*.
+// tau* = max over heads of tau_h are dropped first: every head's top P
+// scores are at least tau_h, so at least P buckets have a best score
+// >= tau_h for every h, and the P-th best is >= tau*.
 // The kept buckets go out as one-bucket entries with tau = -inf, for the
 // unchanged expansion.  The union is deduplicated in a shared-memory hash
-// table (linear probing, at most 3/4 full).  A query whose rows overflowed
-// their entry slots, whose union does not fit the table, or whose cut keeps
-// more than the expansion's slots (ties) is redone exactly: every visible
-// bucket scored for every head on the CUDA cores, radix select, ties in
-// ascending bucket order.
+// table with linear probing, sized from the query's entry count (one retry
+// at the launch's full size).  A query whose rows overflowed their entry
+// slots, whose union does not fit the table, or whose cut keeps more than
+// the expansion's slots (ties) is redone exactly: every visible bucket
+// scored for every head on the CUDA cores, radix select, ties in ascending
+// bucket order.
 constexpr int HM_THREADS = 512;
 constexpr int HM_MAX_SLOTS = 25600;  // 200 KB of table
 constexpr int HM_UNROLL = 4;         // entries a thread loads before using them
