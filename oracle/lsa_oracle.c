@@ -433,10 +433,12 @@ int64_t orc_flat_rank(const uint16_t *qhat, int64_t H, int n_buckets, const uint
  * blocks are < H.  Candidates at level l = children of the nodes kept at
  * level l+1, plus visible level-l nodes whose parent is not visible (or that
  * have no parent).  Keep the best max(W, ceil(P / 2^l)) by (score desc, id
- * asc).  The buckets kept at level 0 are returned ranked (local ids). */
+ * asc).  The buckets kept at level 0 are returned ranked (local ids).
+ * kept_per_level (NULL, or n_levels entries) receives how many nodes each
+ * level kept, a trace for tests; it changes nothing in the search. */
 int64_t orc_tree_rank(const uint16_t *qhat, int64_t H, const int32_t *child, const int32_t *parent,
                       const int32_t *max_block, const uint16_t *cbf, const int64_t *level_size,
-                      int n_levels, int W, int64_t P, int32_t *ids, float *scores)
+                      int n_levels, int W, int64_t P, int32_t *ids, float *scores, int64_t *kept_per_level)
 {
     int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n_levels + 1));
     off[0] = 0;
@@ -465,6 +467,7 @@ int64_t orc_tree_rank(const uint16_t *qhat, int64_t H, const int32_t *child, con
         int64_t B = (P + ((int64_t)1 << l) - 1) >> l;
         if (B < W) B = W;
         n_kept = nc < B ? nc : B;
+        if (kept_per_level) kept_per_level[l] = n_kept;
         for (int64_t i = 0; i < n_kept; ++i) kept[i] = cand[i].id;
         if (l == 0)
             for (int64_t i = 0; i < n_kept; ++i) { ids[i] = cand[i].id; if (scores) scores[i] = cand[i].s; }
@@ -535,7 +538,7 @@ int orc_index(const float *qidx, const int64_t *pos, int64_t nq, int64_t nblk, i
             nr = orc_flat_rank(qh, H, n_buckets, centroid_bf16, ids, NULL);
         else
             nr = orc_tree_rank(qh, H, child, parent, max_block, tree_cbf, level_size, n_levels,
-                               beam, P, ids, NULL);
+                               beam, P, ids, NULL, NULL);
         if (nr < 0) bad = 1;
         lens[i] = orc_expand(ids, nr, members, count, pos[i], k, sink, window, lists + i * Lmax, Lmax);
         free(ids);

@@ -6,10 +6,13 @@ which cites the LSA pages passage by passage.
 
 Parity status per function:
   pool_norm, build_cache (Ward), build_tree, qnorm, flat ranking, expand,
-  attention: pinned by the tests in tests/test_oracle_*.py.
-  tree_rank beyond the invariants (wide beam == Flat, kept nodes visible,
-  beam sizes): parity unpinned -- the pages give no rule mapping a beam of
-  32 to k keys, so the oracle's reading is the specification.
+  attention: pinned by the tests in tests/test_oracle_pins.py.
+  tree_rank: pinned against beam decisions worked out by hand on a
+  hand-built 16-leaf tree (kept set and node count at every level, hidden
+  subtrees included), the narrowest beam still filling k, recall rising
+  with the beam, and a wide beam equal to Flat search.  The beam-size rule
+  itself is a reading (the pages give no rule that maps a beam of 32 to k
+  keys); the pins fix that the oracle carries the reading out exactly.
 """
 from __future__ import annotations
 
@@ -66,7 +69,7 @@ def lib():
             "orc_qnorm": (None, [P, i64, P]),
             "orc_score": (f32, [P, P]),
             "orc_flat_rank": (i64, [P, i64, i32, P, P, P]),
-            "orc_tree_rank": (i64, [P, i64, P, P, P, P, P, i32, i32, i64, P, P]),
+            "orc_tree_rank": (i64, [P, i64, P, P, P, P, P, i32, i32, i64, P, P, P]),
             "orc_expand": (i32, [P, i64, P, P, i64, i32, i32, i32, P, i32]),
             "orc_index_heads": (i32, [P, P, i64, i32, i64, i32, P, P, P, i32, i32, i32, P, P, i32]),
             "orc_index": (i32, [P, P, i64, i64, i32, P, P, P, i32, P, P, P, P, P, i32,
@@ -251,13 +254,18 @@ def flat_rank(qhat_bits: np.ndarray, H: int, cache: Cache, n_buckets: int = N_BU
     return ids[:got], sc[:got]
 
 
-def tree_rank(qhat_bits: np.ndarray, H: int, tree: Tree, beam: int, P: int):
+def tree_rank(qhat_bits: np.ndarray, H: int, tree: Tree, beam: int, P: int, trace: bool = False):
+    """Ranked level-0 ids and scores; with trace=True also the number of
+    nodes the beam kept at each level (index = level)."""
     nb = int(tree.level_size[0])
     ids = np.empty(max(nb, 1), np.int32)
     sc = np.empty(max(nb, 1), np.float32)
+    kept = np.zeros(max(tree.n_levels, 1), np.int64)
     got = lib().orc_tree_rank(_p(_c(qhat_bits, np.uint16)), H, _p(tree.child), _p(tree.parent),
                               _p(tree.max_block), _p(tree.centroid_bf16), _p(tree.level_size),
-                              tree.n_levels, beam, P, _p(ids), _p(sc))
+                              tree.n_levels, beam, P, _p(ids), _p(sc), _p(kept))
+    if trace:
+        return ids[:got], sc[:got], kept[:tree.n_levels]
     return ids[:got], sc[:got]
 
 

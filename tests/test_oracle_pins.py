@@ -482,10 +482,115 @@ def test_tree_beam_keeps_visible_and_sizes(tiny):
         qh = O.qnorm(q[p])[0]
         H = p // 512
         ids, sc = O.tree_rank(qh, H, tree, beam=32, P=P)
-        assert len(ids) == min(P, 64 * H) or len(ids) <= 64 * H
+        assert len(ids) == min(P, 64 * H)  # P kept at level 0 whenever that many buckets are visible
         assert np.all(ids // 64 < H)  # only visible buckets
         assert len(set(ids.tolist())) == len(ids)
         assert np.all(np.diff(sc) <= 0)
+
+
+# A hand-built tree of 16 leaves (levels of 16, 8, 4, 2, 1 nodes; node j of a
+# level has children 2j, 2j + 1 below it).  The query is the unit vector e0
+# and every node's bf16 centroid is (v / 64) e0, so a node scores exactly
+# v / 64: the values below fix every beam decision, and the expected kept
+# sets and per-level counts were worked out by hand from the beam rule
+# (candidates = children of the nodes kept one level up, plus visible nodes
+# whose parent is not visible; keep the best max(W, ceil(P / 2^l))).
+# Leaves 0-7 score highest, so Flat search would take them first; the beam
+# reaches them only through their ancestors.
+_HB_VALUES = {
+    0: [63, 62, 61, 60, 59, 58, 57, 56, 49, 48, 50, 55, 52, 53, 51, 54],
+    1: [44, 39, 47, 46, 40, 43, 41, 42],
+    2: [25, 5, 30, 31],
+    3: [10, 20],
+    4: [1],
+}
+
+
+def _hand_tree(block_of_leaf):
+    t = O.Tree(16)
+    assert t.level_size.tolist() == [16, 8, 4, 2, 1]
+    off = t.level_offset
+    e0 = np.zeros(64, np.float64)
+    for lev, vals in _HB_VALUES.items():
+        for j, v in enumerate(vals):
+            g = off[lev] + j
+            e0[0] = v / 64.0
+            t.centroid_bf16[g] = O.f32_to_bf16_bits(e0.astype(np.float32))
+            t.child[g] = [2 * j, 2 * j + 1] if lev > 0 else [-1, -1]
+            t.parent[g] = j // 2 if lev < 4 else -1
+            leaves = np.arange(j << lev, (j + 1) << lev)
+            t.max_block[g] = max(block_of_leaf(int(x)) for x in leaves)
+            t.min_block[g] = min(block_of_leaf(int(x)) for x in leaves)
+    return t
+
+
+def _e0_query():
+    x = np.zeros(64, np.float32)
+    x[0] = 1.0
+    return O.f32_to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("case", [
+    # (leaf -> block, H, W, P, expected level-0 ids in rank order, kept per level 0..4)
+    ("all", 99, 1, 5, [11, 15, 13, 12, 14], [5, 3, 2, 1, 1]),
+    ("all", 99, 1, 9, [0, 1, 11, 15, 13, 12, 14, 10, 8], [9, 5, 3, 2, 1]),
+    ("all", 99, 3, 5, [0, 1, 11, 15, 14], [5, 3, 3, 2, 1]),
+    ("quarter", 3, 1, 5, [0, 1, 11, 10, 8], [5, 3, 2, 1, 0]),
+    ("half", 3, 1, 5, [0, 1, 2, 3, 4], [5, 3, 1, 0, 0]),
+])
+def test_tree_beam_width_per_level_hand_built(case):
+    """The beam keeps max(W, ceil(P / 2^l)) nodes at level l (capped by the
+    candidates): a floor in place of the ceiling, a min in place of the max,
+    or W alone changes the counts or the kept leaves of at least one case.
+    The 'quarter' and 'half' cases hide the right part of the tree (leaf i in
+    block i // 4 or i // 2, horizon 3 blocks), so the search starts from
+    visible nodes whose parent is not visible."""
+    mapping, H, W, P, want_ids, want_kept = case
+    blk = {"all": lambda i: 0, "quarter": lambda i: i // 4, "half": lambda i: i // 2}[mapping]
+    tree = _hand_tree(blk)
+    ids, sc, kept = O.tree_rank(_e0_query(), H, tree, beam=W, P=P, trace=True)
+    assert kept.tolist() == want_kept
+    assert ids.tolist() == want_ids
+    assert np.array_equal(sc, np.array([_HB_VALUES[0][i] / 64.0 for i in want_ids], np.float32))
+
+
+@pytest.mark.parametrize("k", [16, 64, 256, 1024])
+def test_tree_narrowest_beam_still_fills_k(tiny, k):
+    """With the narrowest beam (W = 1) the buckets kept at level 0 still hold
+    k far keys whenever that many are visible: every list has
+    min(p + 1, |near| + k) entries, as Flat search gives."""
+    _, cache, pos, q = tiny
+    tree = O.build_tree(cache)
+    sel = np.arange(0, 4096, 37)
+    lt, nt = O.index(q[sel], pos[sel], cache, k=k, mode="tree", tree=tree, beam=1)
+    for i, p in enumerate(sel):
+        w0 = max(0, p - 512)
+        near = (p - w0 + 1) + min(4, w0)
+        visible_far = 512 * min(p // 512, 8) - min(4, w0) - max(0, 512 * min(p // 512, 8) - w0)
+        want = near + min(k, visible_far)
+        assert nt[i] == want, (p, nt[i], want)
+
+
+def test_tree_recall_of_flat_top_buckets_grows_with_beam(tiny):
+    """Diagnostic of the beam's width: the share of Flat's top-P buckets that
+    Tree search keeps rises with W, and is 1 once W covers every level."""
+    _, cache, pos, q = tiny
+    tree = O.build_tree(cache)
+    P = O.top_p(64)
+    sel = np.arange(1024, 4096, 29)
+    recall = []
+    for W in (1, 4, 8, 16, 32, 64, 512):
+        r = []
+        for p in sel:
+            qh = O.qnorm(q[p])[0]
+            H = p // 512
+            fids, _ = O.flat_rank(qh, H, cache)
+            tids, _ = O.tree_rank(qh, H, tree, beam=W, P=P)
+            top = set(fids[:P].tolist())
+            r.append(len(top & set(tids[:P].tolist())) / len(top))
+        recall.append(float(np.mean(r)))
+    assert all(b >= a - 1e-12 for a, b in zip(recall, recall[1:])), recall
+    assert recall[-1] == 1.0 and recall[0] < 1.0, recall
 
 
 # ---------------------------------------------------------------- a8 attention
