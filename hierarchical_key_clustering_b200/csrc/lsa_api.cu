@@ -374,6 +374,11 @@ int report_error(int code, const char *msg)
 {
     return fail(code, "%s", msg);
 }
+
+int check_index_params(const lsa_params *p)
+{
+    return check_params(p);
+}
 }  // namespace lsa
 
 extern "C" {
@@ -387,7 +392,8 @@ int lsa_check_device_errors(void)
 {
     int v = lsa::read_device_error(1);
     if (v < 0) return fail(LSA_ERR_CUDA, "could not read the device error word");
-    if (v) fail(LSA_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    if (v & 1) fail(LSA_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    else if (v) fail(LSA_ERR_SHAPE, "a bounds check of the debug build failed (code %d)", v);
     return v;
 }
 

@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     const int64_t q = qg % a.nq;
     const int G = a.Hq / a.Hkv;
     const int len = min(a.lens[q], a.Lmax);
+    if (lane == 0 && split == 0) (void)LSA_IN_BOUNDS(a.lens[q] >= 0 && a.lens[q] <= a.Lmax, BOUNDS_LIST);
     // with a near-set plan the sink prefix and window suffix were done densely
     const int2 plan = a.near_plan ? a.near_plan[q] : make_int2(0, 0);
     const int lend = max(plan.x, len - plan.y);
@@ -171,7 +172,12 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     auto fetch_idx = [&](int ch) {
         const int base = begin + ch * KCH;
         int v = -1;
-        if (lane < KCH && ch < nch && base + lane < end) v = lst[base + lane];
+        if (lane < KCH && ch < nch && base + lane < end) {
+            v = lst[base + lane];
+            // debug build: entries of a list lie in [0, Tk) and strictly increase
+            if (!LSA_IN_BOUNDS(v >= 0 && v < a.Tk && (base + lane == 0 || lst[base + lane - 1] < v), BOUNDS_LIST))
+                v = -1;
+        }
         return v;
     };
     pre = fetch_idx(0);
@@ -465,6 +471,7 @@ __global__ void __launch_bounds__(NEAR_ROWS) k_near_plan(AttnArgs a)
         const int64_t q = q0 + t;
         const int32_t *lst = a.lists + q * (int64_t)a.Lmax;
         const int len = min(a.lens[q], a.Lmax);
+        (void)LSA_IN_BOUNDS(a.lens[q] >= 0 && a.lens[q] <= a.Lmax, BOUNDS_LIST);
         int p = -1, d = 0, s = 0;
         if (len >= 1) {
             p = lst[len - 1];
@@ -782,5 +789,8 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     }
     return e;
 }
+
+// this file's bounds-check word (debug build; always 0 in the release build)
+LSA_BOUNDS_READER(read_bounds_error_attn)
 
 }  // namespace lsa

@@ -211,4 +211,52 @@ __host__ __device__ __forceinline__ int64_t n_groups(int64_t N, int64_t P)
     return (N + g - 1) / g;
 }
 
+// Bounds checks of the debug build (built with -DLSA_BOUNDS_CHECKS=1, the
+// library liblsa_debug.so): the gather indices kernels read from memory --
+// the list entries the attention gathers K/V rows with, the bucket ids and
+// member positions the expansion reads, the child ids the tree search
+// follows -- and every list length are checked before use.  A
+// failed check ORs its code into this translation unit's g_bounds_error and
+// the access is skipped; nothing traps.  lsa_check_device_errors() reads and
+// clears the words of every translation unit.  In the release build
+// LSA_IN_BOUNDS(cond, code) is the constant true and costs nothing.
+#ifndef LSA_BOUNDS_CHECKS
+#define LSA_BOUNDS_CHECKS 0
+#endif
+enum : int {
+    BOUNDS_LIST = 2,    // an index-list entry outside [0, Tk) or not increasing, or a length above Lmax
+    BOUNDS_BUCKET = 4,  // a bucket id outside the query's visible buckets, or a member position out of range
+    BOUNDS_NODE = 8,    // a tree-node id outside its level
+};
+
+static __device__ int g_bounds_error = 0;  // one per translation unit
+
+__device__ __forceinline__ bool bounds_check(bool ok, int code)
+{
+    if (!ok) atomicOr(&g_bounds_error, code);
+    return ok;
+}
+
+#if LSA_BOUNDS_CHECKS
+#define LSA_IN_BOUNDS(cond, code) (::lsa::bounds_check((cond), (code)))
+#else
+#define LSA_IN_BOUNDS(cond, code) (true)
+#endif
+
+// Defines `int name(int clear)`: this translation unit's bounds word (read,
+// and cleared when clear != 0), or -1 if it cannot be read.
+#define LSA_BOUNDS_READER(name)                                                           \
+    int name(int clear)                                                                   \
+    {                                                                                     \
+        int v = 0;                                                                        \
+        if (cudaMemcpyFromSymbol(&v, ::lsa::g_bounds_error, sizeof(int)) != cudaSuccess) \
+            return -1;                                                                    \
+        if (clear && v) {                                                                 \
+            int z = 0;                                                                    \
+            if (cudaMemcpyToSymbol(::lsa::g_bounds_error, &z, sizeof(int)) != cudaSuccess) \
+                return -1;                                                                \
+        }                                                                                 \
+        return v;                                                                         \
+    }
+
 }  // namespace lsa

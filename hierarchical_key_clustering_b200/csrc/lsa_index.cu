@@ -330,7 +330,9 @@ __global__ void __launch_bounds__(TEAM >= 8 ? 32 * TEAM : 256, MINB)
         // children of the kept nodes at fixed slots
         int holes = 0;
         for (int i = tw; i < n_kept; i += TT) {
-            const int2 c = __ldg(child2 + offp + kept[i]);
+            int2 c = __ldg(child2 + offp + kept[i]);
+            if (!LSA_IN_BOUNDS(c.x < (int)tv.level_size[l], BOUNDS_NODE)) c.x = -1;
+            if (!LSA_IN_BOUNDS(c.y < (int)tv.level_size[l], BOUNDS_NODE)) c.y = -1;
             if (2 * i + 1 < CM) {
                 keys[2 * i] = c.x >= 0 ? (uint64_t)(uint32_t)c.x : TB_HOLE;
                 keys[2 * i + 1] = c.y >= 0 ? (uint64_t)(uint32_t)c.y : TB_HOLE;
@@ -855,7 +857,11 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
             }
             int nc = 0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) nc += sv[e] >= tau && sv[e] > NEG;
+            for (int e = 0; e < 4; ++e) {
+                if (sv[e] >= tau && sv[e] > NEG && !LSA_IN_BOUNDS(g + e >= 0 && g + e < N, BOUNDS_BUCKET))
+                    sv[e] = NEG;  // debug build: a bucket the query cannot see is dropped
+                nc += sv[e] >= tau && sv[e] > NEG;
+            }
             // one shared-memory atomic per warp
             int incl = nc;
 #pragma unroll
@@ -931,7 +937,8 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                 const int mm[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int64_t m = mm[e];  // -1 pads are skipped
+                    int64_t m = mm[e];  // -1 pads are skipped
+                    if (m >= 0 && !LSA_IN_BOUNDS(m < N * (LSA_BLK / LSA_NBKT), BOUNDS_BUCKET)) m = -1;
                     nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
                 }
             }
@@ -1047,7 +1054,8 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                 const int mm[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int64_t m = mm[e];
+                    int64_t m = mm[e];
+                    if (m >= 0 && !LSA_IN_BOUNDS(m < N * (LSA_BLK / LSA_NBKT), BOUNDS_BUCKET)) m = -1;
                     if (m >= 0 && !(m < s_end || (m >= w0 && m <= p))) {
                         if (idx < limit) atomicOr(&masks[mword(slot, (int)((m & 511) >> 5))], 1u << (m & 31));
                         ++idx;
@@ -1085,6 +1093,7 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     // take); the list is laid out from what was written either way
     const int nwin = (int)(p - w0 + 1);
     const int len = n_sink + emitted + nwin;
+    if (t == 0) (void)LSA_IN_BOUNDS(len <= Lmax, BOUNDS_LIST);
     for (int i = t; i < Lmax; i += blockDim.x) {
         if (i < n_sink) out[i] = i;
         else if (i < n_sink + emitted) {
@@ -1635,5 +1644,8 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
     count_launches(1);
     return cudaGetLastError();
 }
+
+// this file's bounds-check word (debug build; always 0 in the release build)
+LSA_BOUNDS_READER(read_bounds_error_index)
 
 }  // namespace lsa

@@ -154,6 +154,8 @@ struct ShrinkArgs {
 };
 cudaError_t launch_shrink(const uint16_t *V, const uint16_t *W, const ShrinkArgs &a, cudaStream_t st);
 int read_shrink_error(int clear);
+int read_bounds_error_attn(int clear);   // debug-build bounds words (lsa_common.cuh)
+int read_bounds_error_index(int clear);
 
 // ws holds one row per (query, index head); with several heads `merged`
 // receives each query's merged candidates (nullptr for one head).

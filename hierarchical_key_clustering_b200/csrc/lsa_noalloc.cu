@@ -18,7 +18,19 @@
 // device address: passing it to a kernel would fault, or on a system where the
 // GPU can reach host memory, silently use the wrong memory.  The device
 // address comes from cudaGetSymbolAddress, done once per device (with that
-// device current) on the first call made on it.
+// device current) on the first call made on it, and kept.
+//
+// When the array comes into being: under CUDA's default lazy module loading
+// a module's device memory (this array, and the code of the kernels the call
+// launches) is set up the first time the module is used on a device, not when
+// the library is loaded.  So the first call on each device -- even one with
+// nq = 0, which does the address look-up and launches nothing -- may allocate
+// and synchronise.  Callers should make one call with the sizes they will use
+// before they reserve the rest of device memory and before any stream
+// capture (or run with CUDA_MODULE_LOADING=EAGER); after that, calls allocate
+// nothing.  The kept address assumes the device is never reset
+// (cudaDeviceReset) while the library is in use; a reset also ends every
+// buffer the caller passes in.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -28,6 +40,7 @@
 
 namespace lsa {
 int report_error(int code, const char *msg);  // sets lsa_last_error_string (lsa_api.cu)
+int check_index_params(const lsa_params *p);  // the argument checks of lsa_index_decode (lsa_api.cu)
 }
 
 namespace {
@@ -39,14 +52,15 @@ void *g_scratch_ptr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mu;
 
 // Device address of g_index_scratch on the current device (set up on the
-// first call per device).
+// first call per device).  Returns 0, a cudaError_t, or -1 for a device
+// ordinal this file keeps no slot for.
 int scratch_address(void **out, int *dev_out)
 {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return (int)e;
-    if (dev < 0 || dev >= kMaxDevices) return -1;
     *dev_out = dev;
+    if (dev < 0 || dev >= kMaxDevices) return -1;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
     if (!g_scratch_ptr[dev]) {
         void *ptr = nullptr;
@@ -64,7 +78,11 @@ extern "C" int lsa_index_decode_static(const float *qidx, const int64_t *pos, in
                                        const lsa_tree *tree, int32_t *lists, int32_t *lens, int32_t Lmax,
                                        const lsa_params *p, void *stream)
 {
-    if (!cache || !p) return lsa_index_decode(qidx, pos, nq, cache, tree, lists, lens, Lmax, p, nullptr, 0, stream);
+    // the parameter checks come first, so bad parameters get LSA_ERR_ARG as
+    // they do from lsa_index_decode, never a size computed from them
+    const int pc = lsa::check_index_params(p);
+    if (pc != LSA_OK) return pc;
+    if (!cache) return lsa_index_decode(qidx, pos, nq, cache, tree, lists, lens, Lmax, p, nullptr, 0, stream);
     const int64_t need = lsa_index_workspace_bytes(nq, cache->n_blocks, p);
     if (need > (int64_t)LSA_STATIC_SCRATCH_BYTES) {
         char msg[256];
@@ -79,9 +97,15 @@ extern "C" int lsa_index_decode_static(const float *qidx, const int64_t *pos, in
     int rc = scratch_address(&ws, &dev);
     if (rc != 0) {
         char msg[256];
-        snprintf(msg, sizeof(msg),
-                 "lsa_index_decode_static: cudaGetSymbolAddress of the static scratch failed on device %d (%d)",
-                 dev, rc);
+        if (rc == -1)
+            snprintf(msg, sizeof(msg),
+                     "lsa_index_decode_static: device ordinal %d is above the %d devices the static scratch "
+                     "keeps addresses for",
+                     dev, kMaxDevices - 1);
+        else
+            snprintf(msg, sizeof(msg),
+                     "lsa_index_decode_static: cudaGetSymbolAddress of the static scratch failed on device %d: %s",
+                     dev, cudaGetErrorString((cudaError_t)rc));
         return lsa::report_error(LSA_ERR_CUDA, msg);
     }
     return lsa_index_decode(qidx, pos, nq, cache, tree, lists, lens, Lmax, p, ws, (int64_t)LSA_STATIC_SCRATCH_BYTES,

@@ -388,6 +388,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         volatile int dummy = 0;
         for (int it = max(0, issued - nst); it < issued; ++it)
             wait_bounded(smem_u32(&cs->full[it % nst]), (uint32_t)((it / nst) & 1), a.wait_limit, &dummy);
+        // and the query tile: the wait that ran out may have been the MMA
+        // thread's wait on it, with the copy slow rather than lost
+        if (a.extra_tx == 0) wait_bounded(smem_u32(&cs->a_full), 0, a.wait_limit, &dummy);
     }
     if (warp == 1 && lane == 0) {
         // every MMA this thread issued has finished before its TMEM is freed
@@ -475,7 +478,9 @@ int read_device_error(int clear)
     }
     const int w = read_shrink_error(clear);  // the projection kernel's own word
     if (w < 0) return -1;
-    return v | w;
+    const int ba = read_bounds_error_attn(clear), bi = read_bounds_error_index(clear);  // debug build only
+    if (ba < 0 || bi < 0) return -1;
+    return v | w | ba | bi;
 }
 
 }  // namespace lsa

@@ -68,20 +68,27 @@ EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "l
 _lib = None
 
 
+def debug_build() -> bool:
+    """LSA_BOUNDS_CHECKS=1 in the environment selects liblsa_debug.so, the
+    build with the kernels' bounds checks compiled in."""
+    return os.environ.get("LSA_BOUNDS_CHECKS", "0") not in ("", "0")
+
+
 def library_path() -> str:
-    return _build.LIB
+    return _build.LIB_DEBUG if debug_build() else _build.LIB
 
 
 def lib():
-    """Load liblsa.so (building it if the sources are newer); raise if absent."""
+    """Load liblsa.so, or liblsa_debug.so when debug_build() (building it if
+    the sources are newer); raise if absent."""
     global _lib
     if _lib is None:
         path = library_path()
-        if not os.path.exists(path) or _build._stale():
+        if not os.path.exists(path) or _build._stale(path):
             try:
-                _build.build()
+                _build.build(debug=debug_build())
             except Exception as e:  # no nvcc, no sources: there is no other path
-                raise RuntimeError(f"liblsa.so is missing and could not be built: {e}") from e
+                raise RuntimeError(f"{os.path.basename(path)} is missing and could not be built: {e}") from e
         L = C.CDLL(path)
         P, i64, i32, f32 = C.c_void_p, C.c_int64, C.c_int32, C.c_float
         pp, pc, pt = C.POINTER(lsa_params), C.POINTER(lsa_cache), C.POINTER(lsa_tree)
@@ -335,7 +342,19 @@ def lsa_index_decode_static(qidx, pos, cache: Cache, tree: Tree | None, lists, l
                                          lists.shape[1], C.byref(p), _stream(stream)))
 
 
-STATIC_SCRATCH_BYTES = 16 << 20
+def _static_scratch_bytes() -> int:
+    """LSA_STATIC_SCRATCH_BYTES as include/lsa.h defines it (read from the
+    header, so the binding keeps no second copy of the size)."""
+    import re
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "lsa.h")
+    with open(hdr) as f:
+        m = re.search(r"#define\s+LSA_STATIC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", f.read())
+    if not m:
+        raise RuntimeError("LSA_STATIC_SCRATCH_BYTES not found in include/lsa.h")
+    return int(m.group(1)) << int(m.group(2))
+
+
+STATIC_SCRATCH_BYTES = _static_scratch_bytes()
 
 
 def lsa_sparse_attention(Q, K, V, lists, lens, O, lse=None, scale=None, ws=None, stream=None):

@@ -159,6 +159,16 @@ int64_t lsa_launch_count(void);
  * the current device to go idle, reads and clears that word: 0 = no wait ran
  * out, 1 = one did (outputs of that call are invalid and
  * lsa_last_error_string() says so), < 0 = CUDA error.
+ * The debug build of the library (liblsa_debug.so, built with
+ * -DLSA_BOUNDS_CHECKS=1) also checks, before use, the gather indices that
+ * kernels read from memory -- the list entries the attention gathers K/V rows
+ * with, the bucket ids and member positions the expansion reads, the child
+ * ids the tree search follows -- and every list length; a failed check skips
+ * the access (it never traps) and adds a code to the word:
+ * 2 = an index-list entry outside [0, Tk) or not increasing, or a list length
+ * above Lmax; 4 = a bucket id the query cannot see or a member position past
+ * the cache; 8 = a tree-node id outside its level.  The release build
+ * compiles these checks out.
  * lsa_debug_wait_test(1) is a test hook: in the next lsa_index_* call in
  * Flat mode every score CTA skips its query-tile copy, so the barrier that
  * waits for it never completes, and waits are cut to a short limit; the error
@@ -334,8 +344,15 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
  * fewer keep every bucket score, 5 MB per query at 10M).
  *
  * The first call on a device looks up the array's device address (with that
- * device current) and keeps it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the previous call's
+ * device current) and keeps it.  Under CUDA's default lazy module loading the
+ * array, and the code of the kernels a call launches, are set up on a device
+ * the first time they are used there, so the first call on each device may
+ * allocate device memory and synchronise: make one call with the sizes you
+ * will use (a call with nq = 0 only sets up the array) before reserving the
+ * rest of device memory and before any stream capture, or run with
+ * CUDA_MODULE_LOADING=EAGER.  The kept address assumes the device is not
+ * reset while the library is in use.  Parameters are checked before the size
+ * (bad ones give LSA_ERR_ARG).  All calls share the one array and it keeps the previous call's
  * contents (every value the kernels read is written earlier in the same
  * call); calls whose GPU work overlaps in time -- on different streams, or
  * from several host threads -- race on it and must be serialised by the

@@ -129,6 +129,16 @@ def test_argument_errors_return_codes():
     # nq = 0 is a no-op
     _expect(L.lsa_index_prefill(None, None, 0, C.byref(cache), None, None, None, Lmax, C.byref(p), None, 0,
                                 None), 0)
+    # the static-scratch decode checks its parameters before sizing the request,
+    # with the same code as lsa_index_decode (NULL pointers: nothing can launch)
+    for bad_p in (lsa.lsa_default_params(index_heads=64), lsa.lsa_default_params(k=1 << 21),
+                  lsa.lsa_default_params(n_pool=8), lsa.lsa_default_params(mode="tree", beam=0)):
+        want = L.lsa_index_decode(None, None, 1, C.byref(cache), None, None, None, Lmax, C.byref(bad_p), None, 0,
+                                  None)
+        assert want == -1
+        _expect(L.lsa_index_decode_static(None, None, 1, C.byref(cache), None, None, None, Lmax, C.byref(bad_p),
+                                          None), -1)
+    _expect(L.lsa_index_decode_static(None, None, 1, C.byref(cache), None, None, None, Lmax, None, None), -1)
     # attention shape checks
     _expect(L.lsa_sparse_attention(FAKE, FAKE, FAKE, 4, 32, 8, 64, 100, FAKE, FAKE, 10, 0.1, FAKE, None, None, 0,
                                    None), -1)

@@ -60,14 +60,39 @@ def test_static_scratch_matches_workspace_entry_point(mode):
         assert np.all(na > 0)
 
 
+def test_static_scratch_call_allocates_nothing_after_set_up():
+    """Once a first call has set a device up (module loading under CUDA's lazy
+    loading, the array's address), calls take no device memory: the driver's
+    free-memory count is the same before and after two calls."""
+    keys_all, cache, tree, p = _setup()
+    pos_np = np.array([4096, 4100, 1500], dtype=np.int64)
+    q = torch.from_numpy(I.index_queries(3, keys_all, pos_np)).cuda()
+    pos = torch.from_numpy(pos_np).cuda()
+    Lmax = lsa.lsa_list_budget(p)
+    lists = torch.empty((3, Lmax), dtype=torch.int32, device="cuda")
+    lens = torch.empty((3,), dtype=torch.int32, device="cuda")
+    # a call with no queries sets up the array and launches nothing
+    lsa.lsa_index_decode_static(q[:0], pos[:0], cache, tree, lists[:0], lens[:0], p)
+    lsa.lsa_index_decode_static(q, pos, cache, tree, lists, lens, p)  # first call with work: loads the kernels
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(2):
+        lsa.lsa_index_decode_static(q, pos, cache, tree, lists, lens, p)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert np.all(lens.cpu().numpy() > 0)
+
+
 def test_static_scratch_rejects_requests_above_its_size():
+    """A request above the array's size is refused before anything is enqueued.
+    The pointers are NULL: whichever check runs first, no kernel can start."""
     keys_all, cache, tree, p = _setup()
     nq = 100000
     need = lsa.lsa_index_workspace_bytes(nq, cache.n_blocks, p)
     assert need > lsa.STATIC_SCRATCH_BYTES
     Lmax = lsa.lsa_list_budget(p)
-    fake = C.c_void_p(1 << 20)
-    rc = lsa.lib().lsa_index_decode_static(fake, fake, nq, C.byref(cache.c), None, fake, fake, Lmax, C.byref(p),
+    rc = lsa.lib().lsa_index_decode_static(None, None, nq, C.byref(cache.c), None, None, None, Lmax, C.byref(p),
                                            None)
     assert rc == -5
     msg = lsa.lib().lsa_last_error_string().decode()
