@@ -8,7 +8,9 @@ Rules (stated once, used by every parity test):
     within TIE_TOL = 1e-5 of the score at which the oracle's expansion
     reached k keys (GPU scores are fp32 sums of the same bf16 products);
   * attention: bf16 output within max-abs 2e-2 and mean-abs 2e-3 of the
-    oracle (computed in fp64, rounded to fp32); lse within 2e-3.
+    oracle (computed in fp64, rounded to fp32); lse within 1e-4 (fp32 score
+    sums of 128 bf16 products keep each scaled score within ~1e-5 of the
+    fp64 value at N(0, 1) inputs, and lse moves by at most that).
 """
 from __future__ import annotations
 
@@ -21,7 +23,7 @@ from hierarchical_key_clustering_b200 import lsa
 TIE_TOL = 1e-5
 ATT_MAX = 2e-2
 ATT_MEAN = 2e-3
-LSE_TOL = 2e-3
+LSE_TOL = 1e-4
 
 
 def to_dev(a: np.ndarray, dtype=None):

@@ -149,28 +149,72 @@ def test_1m_cache_and_tree_bit_exact(big1m):
     _check_tree(tree, O.build_tree(oc))
 
 
+def _sample(n: int, count: int = 1024) -> np.ndarray:
+    """Evenly spaced sample of `count` of n prefill queries (all of them when
+    n <= count): the queries the oracle checks one by one."""
+    return np.unique(np.linspace(0, n - 1, min(n, count)).astype(np.int64))
+
+
+def _decode_one_by_one(cache, tree, p, dq, dpos):
+    """lsa_index_decode at batch 1 for every decode token, in order."""
+    gl, gn = [], []
+    for i in range(len(dpos)):
+        l1, n1 = _gpu_index(cache, tree, p, dq[i:i + 1], dpos[i:i + 1], decode=True)
+        gl.append(l1.cpu().numpy()[0])
+        gn.append(int(n1.cpu().numpy()[0]))
+    return np.stack(gl), np.array(gn)
+
+
+def _decode_attention(gl, gn, T_kv, hq, hkv, seed):
+    """Batch-1 attention (the split-list path) for every decode token's list,
+    against the oracle."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    nd = len(gn)
+    Q = torch.randn((nd, hq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    K = torch.randn((T_kv, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((T_kv, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    Lmax = gl.shape[1]
+    O_ = torch.empty_like(Q)
+    lse = torch.empty((nd, hq), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(1, hq, 128, Lmax))
+    ld, nd_ = PT.to_dev(gl), PT.to_dev(gn)
+    for i in range(nd):
+        lsa.lsa_sparse_attention(Q[i:i + 1], K, V, ld[i:i + 1], nd_[i:i + 1], O_[i:i + 1], lse[i:i + 1], ws=ws)
+    torch.cuda.synchronize()
+    used = np.unique(gl[gl >= 0])
+    remap = np.full(T_kv, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    ll = np.where(gl >= 0, remap[np.maximum(gl, 0)], -1).astype(np.int32)
+    ui = torch.from_numpy(used.astype(np.int64)).cuda()
+    bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
+    Oref, lse_ref = O.attention(bits(Q), bits(K.index_select(0, ui)), bits(V.index_select(0, ui)), ll, gn)
+    return PT.assert_attention_close(O_, Oref, lse, lse_ref)
+
+
 def test_1m_flat_prefill_and_decode(big1m):
+    """1M Flat: every prefill query indexed in the benchmark's one launch,
+    1024 evenly spaced of them against the oracle, attention of every query
+    in one launch with 128 sampled; then each of the 64 decode tokens indexed
+    and attended at batch 1, all against the oracle."""
     wl, keys_all, oc, cache, _ = big1m
     T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
     p = lsa.lsa_default_params(k=k)
     pos = np.arange(T - npre, T, dtype=np.int64)
     q = I.index_queries(0, keys_all, pos)
     lists_d, lens_d = _gpu_index(cache, None, p, q, pos)
-    sel = np.linspace(0, npre - 1, 160).astype(np.int64)
+    sel = _sample(npre)
     ol, on = O.index(q[sel], pos[sel], oc, k=k)
-    PT.assert_lists_match(lists_d[torch.from_numpy(sel).cuda()].cpu().numpy(),
-                          lens_d[torch.from_numpy(sel).cuda()].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
+    ix = torch.from_numpy(sel).cuda()
+    PT.assert_lists_match(lists_d[ix].cpu().numpy(), lens_d[ix].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
     _attention_sampled(lists_d, lens_d, sel[::8], T + ndec, wl["hq"], wl["hkv"], seed=2)
-    # decode: one token at a time, every decode position
+    del lists_d, lens_d
     dpos = np.arange(T, T + ndec, dtype=np.int64)
     dq = I.index_queries(1, keys_all, dpos)
-    gl, gn = [], []
-    for i in range(ndec):
-        l1, n1 = _gpu_index(cache, None, p, dq[i:i + 1], dpos[i:i + 1], decode=True)
-        gl.append(l1.cpu().numpy()[0])
-        gn.append(int(n1.cpu().numpy()[0]))
+    gl, gn = _decode_one_by_one(cache, None, p, dq, dpos)
     ol, on = O.index(dq, dpos, oc, k=k)
-    PT.assert_lists_match(np.stack(gl), np.array(gn), ol, on, dq, dpos, oc, k=k)
+    PT.assert_lists_match(gl, gn, ol, on, dq, dpos, oc, k=k)
+    _decode_attention(gl, gn, T + ndec, wl["hq"], wl["hkv"], seed=12)
 
 
 def test_1m_context_parallel_eight_ranks(big1m):
@@ -235,25 +279,40 @@ def test_1m_context_parallel_eight_ranks(big1m):
 
 
 def test_1m_tree_prefill_and_decode(big1m):
+    """1M Tree (beam 32): every prefill query in one launch, 1024 evenly
+    spaced against the oracle; each of the 64 decode tokens at batch 1 (the
+    small-batch beam kernel) against the oracle."""
     wl, keys_all, oc, cache, tree = big1m
     T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
     ot = O.build_tree(oc)
     p = lsa.lsa_default_params(k=k, mode="tree", beam=32)
-    pos = np.concatenate([np.arange(T - npre, T, dtype=np.int64)[np.linspace(0, npre - 1, 96).astype(np.int64)],
-                          np.arange(T, T + ndec, dtype=np.int64)[::4]])
+    pos = np.arange(T - npre, T, dtype=np.int64)
     q = I.index_queries(0, keys_all, pos)
-    gl, gn = _gpu_index(cache, tree, p, q, pos)
-    ol, on = O.index(q, pos, oc, k=k, mode="tree", tree=ot, beam=32)
-    PT.assert_lists_match(gl.cpu().numpy(), gn.cpu().numpy(), ol, on, q, pos, oc, k=k, tree=ot, beam=32)
+    lists_d, lens_d = _gpu_index(cache, tree, p, q, pos)
+    sel = _sample(npre)
+    ix = torch.from_numpy(sel).cuda()
+    ol, on = O.index(q[sel], pos[sel], oc, k=k, mode="tree", tree=ot, beam=32)
+    PT.assert_lists_match(lists_d[ix].cpu().numpy(), lens_d[ix].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k,
+                          tree=ot, beam=32)
+    del lists_d, lens_d
+    dpos = np.arange(T, T + ndec, dtype=np.int64)
+    dq = I.index_queries(1, keys_all, dpos)
+    gl, gn = _decode_one_by_one(cache, tree, p, dq, dpos)
+    ol, on = O.index(dq, dpos, oc, k=k, mode="tree", tree=ot, beam=32)
+    PT.assert_lists_match(gl, gn, ol, on, dq, dpos, oc, k=k, tree=ot, beam=32)
 
 
 def test_10m_flat_and_tree():
-    """10,000,000 tokens: 19531 complete blocks and an unclustered tail of 128;
-    the full cache and tree bit-exact, sampled Flat and Tree lists of the
-    last 65536 positions and of decode tokens, attention over 41 GB of K/V."""
+    """10,000,000 tokens: 19531 complete blocks and an unclustered tail of 128.
+    The full cache and tree bit-exact; Flat and Tree prefill of the last 65536
+    positions, each in one launch as the benchmark runs them, with 1024 evenly
+    spaced queries of each against the oracle; all 128 decode tokens at batch
+    1 in both modes against the oracle; attention over 41 GB of K/V for
+    sampled prefill queries and for every Flat decode token."""
     _need_gpu()
     wl = I.WORKLOADS["flat_tree_10m"]
     T, k, npre, ndec = wl["T"], wl["k"], wl["n_prefill"], wl["n_decode"]
+    hq, hkv = wl["hq"], wl["hkv"]
     keys_all = I.index_keys(0, T + ndec, wl["n_components"])
     keys = keys_all[:T]
     oc = O.build_cache(keys)
@@ -261,21 +320,36 @@ def test_10m_flat_and_tree():
     cache = lsa.Cache(T)
     lsa.lsa_build_cache(PT.to_dev(keys), 0, T, cache, p)
     tree = lsa.Tree(T // 512)
-    lsa.lsa_build_tree(cache, tree, lsa.lsa_default_params(k=k, mode="tree"))
+    pt = lsa.lsa_default_params(k=k, mode="tree", beam=32)
+    lsa.lsa_build_tree(cache, tree, pt)
     torch.cuda.synchronize()
     assert cache.n_blocks == 19531
     PT.assert_cache_equal(PT.cache_to_numpy(cache, T), oc)
     ot = O.build_tree(oc)
     _check_tree(tree, ot)
     del keys
-    pos = np.concatenate([np.arange(T - npre, T, dtype=np.int64)[np.linspace(0, npre - 1, 48).astype(np.int64)],
-                          np.arange(T, T + ndec, dtype=np.int64)[::16]])
+    pos = np.arange(T - npre, T, dtype=np.int64)
     q = I.index_queries(0, keys_all, pos)
-    lists_d, lens_d = _gpu_index(cache, None, p, q, pos)
-    ol, on = O.index(q, pos, oc, k=k)
-    PT.assert_lists_match(lists_d.cpu().numpy(), lens_d.cpu().numpy(), ol, on, q, pos, oc, k=k)
-    pt = lsa.lsa_default_params(k=k, mode="tree", beam=32)
+    sel = _sample(npre)
+    ix = torch.from_numpy(sel).cuda()
+    # Tree first (its lists are dropped before the Flat ones are made)
     tl, tn = _gpu_index(cache, tree, pt, q, pos)
-    otl, otn = O.index(q, pos, oc, k=k, mode="tree", tree=ot, beam=32)
-    PT.assert_lists_match(tl.cpu().numpy(), tn.cpu().numpy(), otl, otn, q, pos, oc, k=k, tree=ot, beam=32)
-    _attention_sampled(lists_d, lens_d, np.arange(0, len(pos), 7), T + ndec, wl["hq"], wl["hkv"], seed=3)
+    otl, otn = O.index(q[sel], pos[sel], oc, k=k, mode="tree", tree=ot, beam=32)
+    PT.assert_lists_match(tl[ix].cpu().numpy(), tn[ix].cpu().numpy(), otl, otn, q[sel], pos[sel], oc, k=k,
+                          tree=ot, beam=32)
+    del tl, tn
+    lists_d, lens_d = _gpu_index(cache, None, p, q, pos)
+    ol, on = O.index(q[sel], pos[sel], oc, k=k)
+    PT.assert_lists_match(lists_d[ix].cpu().numpy(), lens_d[ix].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
+    _attention_sampled(lists_d, lens_d, sel[::16], T + ndec, hq, hkv, seed=3)
+    del lists_d, lens_d
+    torch.cuda.empty_cache()
+    dpos = np.arange(T, T + ndec, dtype=np.int64)
+    dq = I.index_queries(1, keys_all, dpos)
+    gl, gn = _decode_one_by_one(cache, None, p, dq, dpos)
+    ol, on = O.index(dq, dpos, oc, k=k)
+    PT.assert_lists_match(gl, gn, ol, on, dq, dpos, oc, k=k)
+    _decode_attention(gl, gn, T + ndec, hq, hkv, seed=13)
+    tgl, tgn = _decode_one_by_one(cache, tree, pt, dq, dpos)
+    otl, otn = O.index(dq, dpos, oc, k=k, mode="tree", tree=ot, beam=32)
+    PT.assert_lists_match(tgl, tgn, otl, otn, dq, dpos, oc, k=k, tree=ot, beam=32)

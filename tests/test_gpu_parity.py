@@ -255,6 +255,69 @@ def test_tree_index_tiny(tiny, beam):
         PT.assert_lists_match(gl, gn, fl, fn, q[sel], pos[sel], oc, k=256)
 
 
+@pytest.mark.parametrize("beam", [32, 4])
+def test_tree_decode_small_batches(tiny, beam):
+    """Tree search for decode batches of 1, 4 and 16 queries (the small-batch
+    beam kernel: one query per 16-warp team) against the oracle, for tokens
+    past the clustered context and for interior positions."""
+    keys, q, pos, oc = tiny
+    T = 4096
+    ot = O.build_tree(oc)
+    more = I.index_keys(0, T + 16, 32)
+    dpos = np.concatenate([np.arange(T, T + 8, dtype=np.int64), np.array([513, 1024, 2047, 2600, 3000, 3583, 3584,
+                                                                          4095], dtype=np.int64)])
+    dq = I.index_queries(9, more, dpos)
+    cache, tree, p = _build_gpu(keys, mode="tree", k=256, beam=beam)
+    for nq in (1, 4, 16):
+        for a in range(0, 16, nq):
+            gl, gn = _index_gpu(cache, tree, p, dq[a:a + nq], dpos[a:a + nq], decode=True)
+            ol, on = O.index(dq[a:a + nq], dpos[a:a + nq], oc, k=256, mode="tree", tree=ot, beam=beam)
+            PT.assert_lists_match(gl, gn, ol, on, dq[a:a + nq], dpos[a:a + nq], oc, k=256, tree=ot, beam=beam)
+
+
+@pytest.mark.parametrize("nq,consecutive", [(300, False), (1, False), (200, True)])
+def test_attention_peaked_softmax(tiny, nq, consecutive):
+    """Q scaled by 8 (exact in bf16): the softmax of each row is dominated by a
+    few keys, so a dropped, duplicated or misplaced key moves the output by
+    about the size of a value row and fails the tolerance.  The gather path,
+    the split-list path (nq = 1) and the near-set tiles (consecutive
+    queries).  Score rounding grows with the scores, so lse is held to 8x
+    the usual bound."""
+    _need_gpu()
+    keys, q, pos, oc = tiny
+    hq, hkv = 32, 8
+    if consecutive:
+        sel = np.arange(1500, 1500 + nq, dtype=np.int64)
+    else:
+        sel = np.sort(np.random.default_rng(nq).choice(4096, size=nq, replace=False)).astype(np.int64)
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    Qb, Kb, Vb = I.qkv_bf16_bits(21, nq, 4096, hq, hkv)
+    Q8 = PT.bits_to_bf16(Qb) * 8
+    Q8b = Q8.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    Oref, lse_ref = O.attention(Q8b, Kb, Vb, ol, on)
+    Kd, Vd = PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Q8)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, ol.shape[1]))
+    lsa.lsa_sparse_attention(Q8, Kd, Vd, PT.to_dev(ol), PT.to_dev(on), Od, lse, ws=ws)
+    torch.cuda.synchronize()
+    PT.assert_attention_close(Od, Oref)
+    assert np.abs(lse.cpu().numpy() - lse_ref).max() <= 8 * PT.LSE_TOL
+    # the check has teeth: dropping each list's highest-scoring key for head 0
+    # moves the oracle's output far past the tolerance
+    Qf = O.bf16_bits_to_f32(Q8b).astype(np.float64)
+    Kf = O.bf16_bits_to_f32(Kb).astype(np.float64)
+    drop, dn = ol.copy(), on.copy()
+    for i in range(nq):
+        keys_i = ol[i, :on[i]]
+        j = int(np.argmax(Kf[keys_i, 0] @ Qf[i, 0]))
+        drop[i, j:dn[i] - 1] = drop[i, j + 1:dn[i]]
+        drop[i, dn[i] - 1] = -1
+        dn[i] -= 1
+    Odrop, _ = O.attention(Q8b, Kb, Vb, drop, dn)
+    assert np.abs(Odrop[:, 0] - Oref[:, 0]).max(axis=1).min() > PT.ATT_MAX
+
+
 @pytest.mark.parametrize("hq,hkv,nq", [(8, 1, 300), (32, 8, 200), (32, 8, 1), (8, 1, 2), (16, 16, 50)])
 def test_attention_against_oracle(tiny, hq, hkv, nq):
     """Attention over the oracle's own lists (isolates the kernel); nq = 1-2
