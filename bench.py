@@ -2,20 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (default): Flat LSA prefill at T = 131072 -- 64-dim index keys and
-queries from the run-of-8 mixture generator (1024 components), k = 2048,
-sink 4, window 512, attention with 32 query heads over 8 KV heads,
-head_dim 128, bf16.  One step is the whole hot path over that batch:
-bucket-cache build (normalise + pool + Ward for all 256 blocks), Flat index
-of all 131072 queries, and sparse attention for all of them.
-value = prefill tokens (queries) per second, whole job.
+Workload (default): Flat and Tree LSA at T = 10,000,000 tokens -- 64-dim
+index keys and queries from the run-of-8 mixture generator (16384
+components), 19531 complete blocks of 512 keys, k = 4096, sink 4, window
+512, attention with 32 query heads over 8 KV heads, head_dim 128, bf16.
+One step is the whole prefill path over the final 65536 positions:
+bucket-cache build (normalise + pool + Ward for every block), index of the
+65536 queries, and sparse attention for all of them.  `value` is the Flat
+step (prefill tokens per second, whole job); the `tree` object is the same
+step in Tree mode (cache build + tree build + beam-search index +
+attention).  `decode` is batch-1 decode of 128 new tokens in both modes.
 
-Also reported: decode us/token at T = 1,048,576 (index_decode + attention
-for 64 new tokens, batch 1; for the 1M and 10M workloads, at their own T),
-the roofline of the dominant kernel, the
-oracle's CPU time on a bounded sample, and an end-to-end number through the
-same C-ABI calls with inputs copied from pinned host memory every step and
-the output copied back.
+Also reported: per-kernel rooflines (CUDA events around every library
+kernel during the timed steps; algorithmic work per launch over its
+duration, against the measured peaks), the oracle's CPU time on a bounded
+sample, and an end-to-end number through the same calls with the step's
+inputs copied from pinned host memory every step and the output copied
+back.
 
 Multi-GPU: the layer does not shard here (each rank runs its own replica,
 "replicas only"); value = all ranks' tokens / max-over-ranks time.
@@ -42,19 +45,12 @@ from hierarchical_key_clustering_b200.layer import SparseLayer  # noqa: E402
 METRIC = "indexer+sparse-attn prefill tokens/s & decode us/token per layer; % roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes per far (query, KV head, key) row -- a list entry the gather
-# kernel k_attn reads -- that ncu measured for the k_attn launch of each Flat
-# workload (dram__bytes_read.sum + dram__bytes_write.sum of the full launch
-# divided by the launch's far rows x Hkv):
-#   flat_128k      20.21 GB + 1.08 GB over 131072 x 2048 x 8 far rows (the
-#                  near-set tiles take sink and window; k_attn's reads include
-#                  the tiles' partial results);
-#   flat_1m        437.8 GB + 0.28 GB over 32768 x 4613 x 8 rows;
-#   flat_tree_10m  1.09 TB + 0.55 GB over 65536 x 4613 x 8 rows (at 1M and
-#                  10M a KV head does not fit in L2, the library keeps the
-#                  near set in the gather, and every listed row is a far row).
-# Re-measure when k_attn changes.
-ATTN_DRAM_BYTES_PER_FAR_ROW = {"flat_128k": 9.92, "flat_1m": 362.3, "flat_tree_10m": 450.8}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per row gathered by
+# the attention's gather kernel -- a (query, KV head, listed key) the kernel
+# reads -- from one ncu capture of that kernel per workload, divided by the
+# launch's gathered rows.  None: not captured for the kernel as it stands.
+# Keyed by workload name; re-measure whenever k_attn changes.
+ATTN_DRAM_BYTES_PER_ROW = {}
 
 
 def peaks():
@@ -141,21 +137,50 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- workload
 
-def make_prefill_inputs(wl: dict, seed: int = 0):
-    T = wl["T"]
-    keys = I.index_keys(seed, T, wl["n_components"])
-    nq = wl["n_prefill"]
-    pos = np.arange(T - nq, T, dtype=np.int64)
-    q = I.index_queries(seed, keys, pos)
-    return keys, q, pos
+def workload(args) -> dict:
+    wl = dict(I.WORKLOADS[args.workload])
+    if args.queries:
+        wl["n_prefill"] = min(args.queries, wl["n_prefill"])
+    modes = ["flat", "tree"] if wl["mode"] == "both" else [wl["mode"]]
+    if args.mode:
+        modes = [args.mode]
+    wl["modes"] = modes
+    return wl
+
+
+def workload_config(args, wl) -> dict:
+    """The `config` object, identical in both arms."""
+    return {"workload": args.workload if not args.queries else f"{args.workload}[last {wl['n_prefill']} queries]",
+            "T": wl["T"], "queries": wl["n_prefill"], "decode_tokens": wl["n_decode"], "k": wl["k"], "sink": 4,
+            "window": 512, "modes": wl["modes"], "beam": wl.get("beam", 32), "Hq": wl["hq"], "Hkv": wl["hkv"],
+            "head_dim": 128, "index_dim": 64, "mixture_components": wl["n_components"], "parallelism": "replicas",
+            "l2": "256 MiB buffer written between timed steps; K/V exceed L2"}
+
+
+def make_inputs(wl: dict, seed: int = 0):
+    """Index keys for the context and the decode tokens (one prefix-consistent
+    draw), the prefill queries at the last n_prefill positions, and the decode
+    queries."""
+    T, nd = wl["T"], wl["n_decode"]
+    keys_all = I.index_keys(seed, T + nd, wl["n_components"])
+    pos = np.arange(T - wl["n_prefill"], T, dtype=np.int64)
+    q = I.index_queries(seed, keys_all[:T], pos)
+    dpos = np.arange(T, T + nd, dtype=np.int64)
+    dq = I.index_queries(seed + 1, keys_all, dpos) if nd else np.zeros((0, 64), np.float32)
+    return keys_all, q, pos, dq, dpos
 
 
 def device_qkv(nq, n_kv, hq, hkv, seed=0, dev="cuda"):
     g = torch.Generator(device=dev)
     g.manual_seed(seed * 1000 + 5)
     Q = torch.randn((nq, hq, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    K = torch.randn((n_kv, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    V = torch.randn((n_kv, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    K = torch.empty((n_kv, hkv, 128), device=dev, dtype=torch.bfloat16)
+    V = torch.empty((n_kv, hkv, 128), device=dev, dtype=torch.bfloat16)
+    step = 1 << 20  # rows per draw, to bound the fp32 temporaries
+    for a in range(0, n_kv, step):
+        b = min(n_kv, a + step)
+        K[a:b] = torch.randn((b - a, hkv, 128), generator=g, device=dev, dtype=torch.float32)
+        V[a:b] = torch.randn((b - a, hkv, 128), generator=g, device=dev, dtype=torch.float32)
     return Q, K, V
 
 
@@ -182,11 +207,149 @@ def near_split_rows(lists: torch.Tensor, lens: torch.Tensor, chunk: int = 4096):
     return near, far
 
 
-def attn_algorithmic_bytes(far_rows: int, nq: int, hq: int, hkv: int) -> int:
-    """Gather kernel k_attn: K and V rows of every far (query, KV head, key)
-    + their list entries + Q read + O write + the near-set partial results
-    (fp32 O and max/sum per (query, head)) it merges."""
-    return far_rows * hkv * 2 * 256 + far_rows * 4 + nq * hq * 128 * 2 * 2 + nq * hq * 130 * 4
+# --------------------------------------------------------------------------- rooflines
+
+def _rl(kernel, bound, work, ms, launches, peak, unit, note, **extra):
+    """One roofline object: algorithmic work per launch / average launch time."""
+    per_launch = work / max(1, launches)
+    t = ms / max(1, launches) / 1e3
+    scale = 1e9 if unit == "GB/s" else 1e12
+    achieved = per_launch / t / scale if t > 0 else None
+    out = {"kernel": kernel, "bound": bound, "achieved": None if achieved is None else round(achieved, 2),
+           "peak": peak, "unit": unit, "frac": None if achieved is None else round(achieved / peak, 4),
+           "ms_per_launch": round(ms / max(1, launches), 4), "launches": launches,
+           "work_per_launch": int(per_launch), "work_unit": "bytes" if unit == "GB/s" else "flop", "per_unit": note}
+    out.update(extra)
+    return out
+
+
+def kernel_rooflines(kt: dict, wl: dict, pos_np, lens_np, far_rows: int, near_ms_total: float, pk, steps: int):
+    """Per-kernel rooflines of one mode's timed steps from the library's
+    per-kernel events (kt: name -> (ms summed over the steps, launches))."""
+    T, hq, hkv = wl["T"], wl["hq"], wl["hkv"]
+    nblk = T // 512
+    H = np.minimum(pos_np // 512, nblk)
+    out = {}
+    if "k_pool_norm" in kt:
+        ms, n = kt["k_pool_norm"]
+        out["k_pool_norm"] = _rl("k_pool_norm", "hbm", 320.0 * T * steps, ms, n, pk["hbm"], "GB/s",
+                                 "320 B per key: 256 B of fp32 key read, 64 B of pooled item written")
+    s_ms = sum(kt[k][0] for k in ("k_score_tc:threshold", "k_score_tc:filter") if k in kt)
+    if s_ms > 0:
+        flop = 128.0 * float(H.sum()) * 64 * steps
+        n = kt.get("k_score_tc:filter", (0, steps))[1]
+        out["k_score_tc"] = _rl("k_score_tc", "tensor", flop, s_ms, n, pk["bf16_sust"], "TFLOP/s",
+                                "128 flop per (query, visible bucket), one pass; time = both passes (threshold + "
+                                "filter); peak = sustained bf16 (timed inside a long step)",
+                                passes_ms={k: round(kt[k][0] / max(1, kt[k][1]), 4)
+                                           for k in ("k_score_tc:threshold", "k_score_tc:filter") if k in kt})
+    if "k_rank_expand" in kt:
+        ms, n = kt["k_rank_expand"]
+        out["k_rank_expand"] = _rl("k_rank_expand", "hbm", 4.0 * float(lens_np.sum()) * steps, ms, n, pk["hbm"],
+                                   "GB/s", "4 B per list entry written (the list is the kernel's output)")
+    if "k_attn" in kt:
+        ms, n = kt["k_attn"]
+        flop = 512.0 * hq * far_rows * steps
+        o = _rl("k_attn", "tensor", flop, ms, n, pk["bf16_sust"], "TFLOP/s",
+                "512 flop per (query head, gathered key): 2 x 128 for the score, 2 x 128 for P V; peak = "
+                "sustained bf16")
+        gathered = 512.0 * hkv * far_rows
+        o["gathered_bytes_per_launch"] = int(gathered)
+        o["gathered_gbs"] = round(gathered / (ms / n / 1e3) / 1e9, 1)
+        o["gathered_note"] = ("512 B of K + V per (query, KV head, gathered key), served from L2 or HBM: a "
+                              "throughput, not a fraction of the HBM peak")
+        per_row = ATTN_DRAM_BYTES_PER_ROW.get(wl["name"])
+        if per_row is not None:
+            traffic = per_row * hkv * far_rows
+            o["traffic"] = int(traffic)
+            o["dram_gbs"] = round(traffic / (ms / n / 1e3) / 1e9, 1)
+            o["dram_frac"] = round(o["dram_gbs"] / pk["hbm"], 4)
+        else:
+            o["traffic"] = None
+        o["unique_kv_bytes"] = int(T * hkv * 512)
+        if near_ms_total > 0:
+            o["near"] = {"kernels": "k_near_plan + k_attn_near", "ms": round(near_ms_total / steps, 3)}
+        out["k_attn"] = o
+    for name in ("k_ward", "k_tree_leaves", "k_tree_pair", "k_tree_beam", "k_qnorm", "k_tau"):
+        if name in kt:
+            ms, n = kt[name]
+            out[name] = {"kernel": name, "bound": "latency", "ms_per_step": round(ms / steps, 4),
+                         "launches_per_step": n / steps}
+    return out
+
+
+# --------------------------------------------------------------------------- our arm
+
+def time_mode(args, wl, mode, keys, qidx, pos, Q, K, V, flush, world, local):
+    """Warm-up, then the timed steps of one search mode with per-kernel
+    events; returns (layer, per-step ms array, kernel timings, clocks,
+    launches)."""
+    T, nq = wl["T"], wl["n_prefill"]
+    layer = SparseLayer(T, k=wl["k"], mode=mode, beam=wl.get("beam", 32), max_queries=nq, Hq=wl["hq"])
+    st = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    Kp, Vp = K[:T], V[:T]
+    O = torch.empty_like(Q)
+
+    def step(times=None):
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        e0.record(st)
+        layer.build(keys)
+        e1.record(st)
+        layer.index(qidx, pos)
+        e2.record(st)
+        layer.attend(Q, Kp, Vp, O)
+        e3.record(st)
+        if times is not None:
+            times.append((e0, e1, e2, e3))
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    launches0 = lsa.lsa_launch_count()
+    lsa.lsa_kernel_timing_read()  # drop anything recorded before
+    lsa.lsa_kernel_timing(True)
+    clk = Clocks(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.start()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        step(times)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    barrier(world)
+    lsa.lsa_kernel_timing(False)
+    kt = lsa.lsa_kernel_timing_read()
+    launches = lsa.lsa_launch_count() - launches0
+    per = np.array([[a.elapsed_time(b), b.elapsed_time(c), c.elapsed_time(d), a.elapsed_time(d)]
+                    for a, b, c, d in times])
+    del O
+    return layer, per, kt, clocks, launches
+
+
+def mode_summary(args, wl, mode, layer, per, kt, world, pk):
+    nq = wl["n_prefill"]
+    total_ms = max_over_ranks(float(per[:, 3].sum()), world)
+    lens_np = layer.lens[:nq].cpu().numpy()
+    near_ms = sum(kt[k][0] for k in ("k_near_plan", "k_attn_near") if k in kt)
+    if near_ms > 0:
+        _, far_rows = near_split_rows(layer.lists[:nq], layer.lens[:nq])
+    else:
+        far_rows = int(lens_np.astype(np.int64).sum())
+    pos_np = np.arange(wl["T"] - nq, wl["T"], dtype=np.int64)
+    kr = kernel_rooflines(kt, wl, pos_np, lens_np, far_rows, near_ms, pk, args.steps)
+    return {
+        "mode": mode, "value": round(world * nq * args.steps / (total_ms / 1e3), 1), "unit": UNIT,
+        "ms_per_step": round(total_ms / args.steps, 3),
+        "breakdown_ms": {"build": round(float(per[:, 0].mean()), 3), "index": round(float(per[:, 1].mean()), 3),
+                         "attention": round(float(per[:, 2].mean()), 3)},
+        "mean_list_len": round(float(lens_np.mean()), 1),
+        "kernels": kr,
+        "kernel_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in kt.items()},
+    }
 
 
 def measure_shrink(K: torch.Tensor, dev, hbm_peak: float):
@@ -194,8 +357,8 @@ def measure_shrink(K: torch.Tensor, dev, hbm_peak: float):
     key over all KV heads (D = Hkv x 128, the workload's K as [T, D]) projected
     by a synthetic bf16 W [64, D] and pooled straight into cache items (the
     fused tensor-core kernel); HBM-bound on reading K."""
-    T = K.shape[0]
-    V = K.reshape(T, -1)
+    T = K.shape[0] - K.shape[0] % 4
+    V = K[:T].reshape(T, -1)
     D = V.shape[1]
     g = torch.Generator(device=dev)
     g.manual_seed(64)
@@ -213,8 +376,8 @@ def measure_shrink(K: torch.Tensor, dev, hbm_peak: float):
     ms = float(np.median(ts))
     nbytes = T * D * 2 + (T // 4) * 64 * 4 + 64 * D * 2
     gbs = nbytes / (ms / 1e3) / 1e9
-    return {"kernel": "k_shrink", "T": T, "D": D, "ms": round(ms, 3), "bytes": nbytes,
-            "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4), "bound": "hbm",
+    return {"kernel": "k_shrink", "T": T, "D": D, "ms": round(ms, 3), "bytes": nbytes, "bound": "hbm",
+            "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
             "flop": 2 * T * D * 64}
 
 
@@ -239,7 +402,7 @@ def measure_index_heads(layer, keys_np, pos_np, wl: dict, dev, heads: int = 8, c
             lsa.lsa_index_prefill(qh[a:b], pos[a:b], layer.cache, None, lists[:b - a], lens[:b - a], p, ws)
 
     ts = []
-    for r in range(4):
+    for r in range(3):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         run()
@@ -262,7 +425,7 @@ def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, rank
     send and receive.  Communication time is not included."""
     from hierarchical_key_clustering_b200 import context_parallel as CP
 
-    T, nq, hq, hkv = wl["T"], len(pos_np), wl["hq"], wl["hkv"]
+    T, nq, hq = wl["T"], len(pos_np), wl["hq"]
     chunk = min(chunk, nq)
     shards = [CP.Shard(r, ranks, T, k=wl["k"], max_queries=chunk, device=dev) for r in range(ranks)]
     keys = torch.from_numpy(keys_np).to(dev)
@@ -333,6 +496,7 @@ def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, rank
             "merge_and_expand_ms": round(mrg, 3),
             "attention_local_ms": {"max_rank": round(max(att), 3), "min_rank": round(min(att), 3)},
             "combine_ms": round(cmb, 3), "step_ms_slowest_rank": round(step, 3),
+            "step_ms_mean_rank": round(float(np.mean(per_rank)), 3),
             "tokens_per_s_without_communication": round(nq / (step / 1e3), 1),
             "allgather_bytes_sent_per_rank": xbytes + part_bytes,
             "allgather_bytes_received_per_rank": (ranks - 1) * (xbytes + part_bytes),
@@ -342,133 +506,78 @@ def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, rank
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = dict(I.WORKLOADS[args.workload])
-    if args.queries:
-        wl["n_prefill"] = min(args.queries, wl["n_prefill"])
-    if args.mode:
-        wl["mode"] = args.mode
-    if wl["mode"] == "both":
-        wl["mode"] = "flat"
-    T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
-    keys_np, q_np, pos_np = make_prefill_inputs(wl)
-    layer = SparseLayer(T, k=wl["k"], mode=wl["mode"], beam=wl.get("beam", 32), max_queries=nq, Hq=hq)
+    wl = workload(args)
+    wl["name"] = args.workload
+    T, nq, nd, hq, hkv = wl["T"], wl["n_prefill"], wl["n_decode"], wl["hq"], wl["hkv"]
+    keys_all, q_np, pos_np, dq_np, dpos_np = make_inputs(wl)
+    keys_np = keys_all[:T]
     keys = torch.from_numpy(keys_np).to(dev)
     qidx = torch.from_numpy(q_np).to(dev)
     pos = torch.from_numpy(pos_np).to(dev)
-    Q, K, V = device_qkv(nq, T, hq, hkv)
-    O = torch.empty_like(Q)
+    Q, K, V = device_qkv(nq, T + nd, hq, hkv)  # K/V also hold the decode tokens' rows
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    st = torch.cuda.current_stream()
-
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-
-    def step(times=None):
-        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
-        e0.record(st)
-        layer.build(keys)
-        e1.record(st)
-        layer.index(qidx, pos)
-        e2.record(st)
-        layer.attend(Q, K, V, O)
-        e3.record(st)
-        if times is not None:
-            times.append((e0, e1, e2, e3))
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    lens_np = layer.lens[:nq].cpu().numpy()
-
-    launches0 = lsa.lsa_launch_count()
-    lsa.lsa_attention_timing_read()  # drop the warm-up calls' events
-    lsa.lsa_attention_timing(True)
-    clk = Clocks(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    clk.start()
-    times = []
-    for _ in range(args.steps):
-        flush.zero_()
-        step(times)
-    torch.cuda.synchronize()
-    clocks = clk.stop()
-    barrier(world)
-    launches = lsa.lsa_launch_count() - launches0
-    lsa.lsa_attention_timing(False)
-    near_ms, gather_ms, n_calls = lsa.lsa_attention_timing_read()
-    per = np.array([[a.elapsed_time(b), b.elapsed_time(c), c.elapsed_time(d), a.elapsed_time(d)]
-                    for a, b, c, d in times])
-    total_ms = float(per[:, 3].sum())
-    total_ms = max_over_ranks(total_ms, world)
-    ms_step = total_ms / args.steps
-    value = world * nq * args.steps / (total_ms / 1e3)
-
-    # roofline of the dominant kernel: k_attn, the far-key gather (one launch
-    # per step), timed by the library's events around it on the step's stream
     pk = peaks()
-    if near_ms > 0.0:  # the near-set tiles ran
-        near_rows, far_rows = near_split_rows(layer.lists[:nq], layer.lens[:nq])
-    else:
-        near_rows, far_rows = 0, int(lens_np.astype(np.int64).sum())
-    attn_ms = gather_ms / max(1, n_calls)
-    abytes = attn_algorithmic_bytes(far_rows, nq, hq, hkv)
-    achieved = abytes / (attn_ms / 1e3) / 1e9
-    traffic = None
-    per_row = ATTN_DRAM_BYTES_PER_FAR_ROW.get(args.workload) if wl["mode"] == "flat" else None
-    if per_row is not None:
-        traffic = int(per_row * far_rows * hkv)
-    roofline = {"kernel": "k_attn", "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
-                "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
-                "peak_source": pk["src"], "algorithmic_bytes": abytes, "launch_ms": round(attn_ms, 3),
-                "traffic_note": "ncu DRAM bytes per far row of this workload's launch, times its far rows",
-                "near": {"kernels": "k_near_plan + k_attn_near", "ms": round(near_ms / max(1, n_calls), 3),
-                         "rows_per_query": round(near_rows / nq, 1),
-                         "far_rows_per_query": round(far_rows / nq, 1)}}
-    if traffic is not None:  # the same launch measured on the DRAM side: bytes that really crossed HBM
-        roofline["dram_achieved"] = round(traffic / (attn_ms / 1e3) / 1e9, 1)
-        roofline["dram_frac"] = round(traffic / (attn_ms / 1e3) / 1e9 / pk["hbm"], 4)
 
-    roofline["shrink"] = measure_shrink(K, dev, pk["hbm"])
+    modes = {}
+    primary = wl["modes"][0]
+    keep = None
+    clocks_all, launches_primary = {}, 0
+    for mode in wl["modes"]:
+        layer, per, kt, clocks, launches = time_mode(args, wl, mode, keys, qidx, pos, Q, K, V, flush, world, local)
+        modes[mode] = mode_summary(args, wl, mode, layer, per, kt, world, pk)
+        modes[mode]["clocks"] = clocks
+        modes[mode]["gpu_launches"] = int(launches)
+        if mode == primary:
+            keep = layer
+            clocks_all, launches_primary = clocks, launches
+        else:
+            del layer
+            torch.cuda.empty_cache()
+    main = modes[primary]
+
+    shrink = measure_shrink(K[:T], dev, pk["hbm"])
     index_heads = None
-    if wl["mode"] == "flat" and not args.no_heads:
-        index_heads = measure_index_heads(layer, keys_np, pos_np, wl, dev)
+    if primary == "flat" and not args.no_heads:
+        index_heads = measure_index_heads(keep, keys_np, pos_np, wl, dev)
     context_parallel = None
-    if args.cp > 1 and wl["mode"] == "flat":
-        context_parallel = measure_context_parallel(wl, keys_np, pos_np, q_np, Q, K, V, dev, args.cp)
+    if args.cp > 1 and primary == "flat":
+        context_parallel = measure_context_parallel(wl, keys_np, pos_np, q_np, Q, K[:T], V[:T], dev, args.cp)
 
-    # end to end: same calls, inputs from pinned host memory, output back to host
-    e2e = None if args.no_e2e else run_e2e(args, layer, keys_np, q_np, pos_np, Q, K, V, dev, world)
+    # end to end: same calls, the step's inputs from pinned host memory, O back
+    e2e = None if args.no_e2e else run_e2e(args, keep, keys_np, q_np, pos_np, Q, K, V, wl, dev, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=args.cpu_budget)
+        cpu = cpu_baseline(wl, primary, keys_np, q_np, pos_np, budget_s=args.cpu_budget,
+                           kv_rows=lambda rows: (K.index_select(0, rows.to(dev)).cpu(),
+                                                 V.index_select(0, rows.to(dev)).cpu()))
 
     decode = None
-    if not args.no_decode:
-        del Q, K, V, O, flush, layer
+    if not args.no_decode and nd > 0:
+        del keep
         torch.cuda.empty_cache()
-        dwl = "flat_1m" if args.workload == "flat_128k" else args.workload
-        decode = run_decode(args, dev, dwl, wl["mode"])
+        decode = {m: run_decode(args, dev, wl, m, keys, dq_np, dpos_np, K, V, pk) for m in wl["modes"]}
 
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload if not args.queries else f"{args.workload}[last {nq} queries]",
-                   "T": T, "queries": nq, "k": wl["k"], "sink": 4, "window": 512,
-                   "mode": wl["mode"], "Hq": hq, "Hkv": hkv, "head_dim": 128, "index_dim": 64,
-                   "mixture_components": wl["n_components"], "parallelism": "replicas",
-                   "l2": "256 MiB buffer written between timed steps; K/V exceed L2"},
-        "breakdown_ms": {"build": round(float(per[:, 0].mean()), 3), "index": round(float(per[:, 1].mean()), 3),
-                         "attention": round(float(per[:, 2].mean()), 3)},
-        "roofline": roofline,
+        "config": workload_config(args, wl),
+        "mode": primary,
+        "breakdown_ms": main["breakdown_ms"],
+        "roofline": dict(main["kernels"].get("k_attn", {}), peak_source=pk["src"]),
+        "kernels": main["kernels"],
         "e2e": e2e,
-        "gpu_launches": int(launches),
-        "clocks": clocks,
+        "gpu_launches": int(launches_primary),
+        "clocks": clocks_all,
         "decode": decode,
-        "index_heads": index_heads,
     }
+    for m in wl["modes"]:
+        if m != primary:
+            line[m] = modes[m]
+    line["shrink"] = shrink
+    if index_heads is not None:
+        line["index_heads"] = index_heads
     if context_parallel is not None:
         line["context_parallel"] = context_parallel
     if cpu is not None:
@@ -477,21 +586,28 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, dev, world):
-    """The step through SparseLayer.prefill_from_host: inputs from pinned host
-    memory, O back to pinned host memory, every step (transfers overlapped
-    with the kernels on copy streams, the step still ends after its last
-    copy back)."""
+def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, wl, dev, world):
+    """The step through SparseLayer.prefill_from_host: the step's inputs from
+    pinned host memory -- every index key (the cache is rebuilt), the index
+    queries and positions, Q, and the K/V rows of the positions being
+    prefilled -- and O back to pinned host memory, every step.  K/V rows of
+    the earlier context are the resident KV cache of the earlier chunks.
+    Transfers overlap the kernels on copy streams; the step still ends after
+    its last copy back."""
     st = torch.cuda.current_stream()
+    T, nq = wl["T"], len(pos_np)
+    t0 = T - nq  # first prefilled position: rows [t0, T) of K/V arrive with the step
     pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
     h_keys, h_q, h_pos = pin(keys_np), pin(q_np), pin(pos_np)
-    h_Q, h_K, h_V = Qd.cpu().pin_memory(), Kd.cpu().pin_memory(), Vd.cpu().pin_memory()
+    h_Q = Qd.cpu().pin_memory()
+    h_K, h_V = Kd[t0:T].cpu().pin_memory(), Vd[t0:T].cpu().pin_memory()
     h_O = torch.empty(Qd.shape, dtype=Qd.dtype).pin_memory()
+    Kc, Vc = Kd[:T], Vd[:T]
     h2d = sum(t.numel() * t.element_size() for t in (h_keys, h_q, h_pos, h_Q, h_K, h_V))
     d2h = h_O.numel() * h_O.element_size()
 
     def step():
-        layer.prefill_from_host(h_keys, h_q, h_pos, h_Q, h_K, h_V, h_O)
+        layer.prefill_from_host(h_keys, h_q, h_pos, h_Q, h_K, h_V, h_O, kv_cache=(Kc, Vc), kv_first=t0)
 
     for _ in range(max(1, args.warmup)):
         step()
@@ -504,37 +620,35 @@ def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, dev, world):
     e1.record(st)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    nq = q_np.shape[0]
     return {"value": round(world * nq * args.steps / (ms / 1e3), 1), "unit": UNIT,
-            "ms_per_step": round(ms / args.steps, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "ms_per_step": round(ms / args.steps, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "note": "index keys, queries, Q and the prefilled positions' K/V rows copied in every step, O copied "
+                    "back; the earlier context's K/V rows stay resident as the KV cache"}
 
 
-def run_decode(args, dev, workload="flat_1m", mode="flat"):
-    """Decode at T = 1M (Flat, k = 4096): per new token, batch 1, the index of
-    that token (lsa_index_decode) and its sparse attention.  The two calls are
-    captured once in a CUDA graph; each token copies its query into the
-    graph's input buffers and replays it (both inside the timed region).
-    Mean us/token over 64 tokens; the eager (uncaptured) figure is kept too."""
-    wl = I.WORKLOADS[workload]
-    T, nd, hq, hkv = wl["T"], wl["n_decode"], wl["hq"], wl["hkv"]
-    keys_all = I.index_keys(0, T + nd, wl["n_components"])
-    pos_np = np.arange(T, T + nd, dtype=np.int64)
-    q_np = I.index_queries(0, keys_all, pos_np)
+def run_decode(args, dev, wl, mode, keys, dq_np, dpos_np, K, V, pk):
+    """Batch-1 decode after the context: per new token, its index
+    (lsa_index_decode) and its sparse attention.  The two calls are captured
+    once in a CUDA graph; each token copies its query into the graph's input
+    buffers and replays it (both inside the timed region).  Mean us/token
+    over the decode tokens; the eager figure is kept too, and one more eager
+    pass with per-kernel events gives the kernels' rooflines."""
+    T, hq, hkv = wl["T"], wl["hq"], wl["hkv"]
+    nd = len(dpos_np)
     layer = SparseLayer(T, k=wl["k"], mode=mode, beam=wl.get("beam", 32), max_queries=1, Hq=hq)
-    layer.build(torch.from_numpy(keys_all[:T]).to(dev))
+    layer.build(keys)
     g = torch.Generator(device=dev)
     g.manual_seed(77)
-    K = torch.randn((T + nd, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    V = torch.randn((T + nd, hkv, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
     Qd = torch.randn((nd, 1, hq, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    qd = torch.from_numpy(q_np).to(dev)
-    pd = torch.from_numpy(pos_np).to(dev)
+    qd = torch.from_numpy(dq_np).to(dev)
+    pd = torch.from_numpy(dpos_np).to(dev)
     q_in, p_in, Q_in = qd[:1].clone(), pd[:1].clone(), Qd[0].clone()
     O = torch.empty((1, hq, 128), dtype=torch.bfloat16, device=dev)
+    Kd, Vd = K[:T + nd], V[:T + nd]
 
     def token():
         layer.index(q_in, p_in, decode=True)
-        layer.attend(Q_in, K, V, O)
+        layer.attend(Q_in, Kd, Vd, O)
 
     def feed(i):
         q_in.copy_(qd[i:i + 1])
@@ -555,6 +669,15 @@ def run_decode(args, dev, workload="flat_1m", mode="flat"):
     torch.cuda.synchronize()
     eager_us = e0.elapsed_time(e1) * 1e3 / nd
     lens = int(layer.lens[:1].item())
+    # per-kernel events over one more eager pass (outside the timed region)
+    lsa.lsa_kernel_timing_read()
+    lsa.lsa_kernel_timing(True)
+    for i in range(nd):
+        feed(i)
+        token()
+    torch.cuda.synchronize()
+    lsa.lsa_kernel_timing(False)
+    kt = lsa.lsa_kernel_timing_read()
     graph_us, note = None, None
     try:
         graph = torch.cuda.CUDAGraph()
@@ -578,22 +701,47 @@ def run_decode(args, dev, workload="flat_1m", mode="flat"):
         e1.record()
         torch.cuda.synchronize()
         graph_us = e0.elapsed_time(e1) * 1e3 / nd
+        del graph
     except Exception as ex:  # report, keep the eager number
         note = f"graph capture failed: {type(ex).__name__}: {ex}"[:200]
+    per_tok = {k: round(v[0] * 1e3 / nd, 2) for k, v in kt.items()}
+    nb = (T // 512) * 64
+    index_us = sum(v for k, v in per_tok.items() if k in ("k_qnorm", "k_dscore", "k_dfilter", "k_tree_beam",
+                                                          "k_rank_expand"))
+    attn_us = sum(v for k, v in per_tok.items() if k in ("k_attn", "k_attn_combine"))
+    kernels = {}
+    if mode == "flat" and index_us > 0:
+        b = 128.0 * nb
+        kernels["decode_index"] = {"kernels": "k_qnorm + k_dscore + k_dfilter + k_rank_expand", "bound": "hbm",
+                                   "achieved": round(b / (index_us / 1e6) / 1e9, 1), "peak": pk["hbm"],
+                                   "unit": "GB/s", "frac": round(b / (index_us / 1e6) / 1e9 / pk["hbm"], 4),
+                                   "us_per_token": round(index_us, 2), "bytes_per_token": int(b),
+                                   "per_unit": "128 B of bf16 centroid read per bucket"}
+        if "k_dscore" in per_tok:
+            ds = per_tok["k_dscore"]
+            kernels["k_dscore"] = {"bound": "hbm", "achieved": round(b / (ds / 1e6) / 1e9, 1), "peak": pk["hbm"],
+                                   "unit": "GB/s", "frac": round(b / (ds / 1e6) / 1e9 / pk["hbm"], 4),
+                                   "us_per_token": ds}
+    if attn_us > 0:
+        b = 512.0 * hkv * lens
+        kernels["decode_attention"] = {"kernels": "k_attn + k_attn_combine", "bound": "hbm",
+                                       "achieved": round(b / (attn_us / 1e6) / 1e9, 1), "peak": pk["hbm"],
+                                       "unit": "GB/s", "frac": round(b / (attn_us / 1e6) / 1e9 / pk["hbm"], 4),
+                                       "us_per_token": round(attn_us, 2), "bytes_per_token": int(b),
+                                       "per_unit": "512 B of K + V per (listed key, KV head)"}
     # a block completes every 512 decode tokens: pool and cluster it and grow
     # the tree in place (the cache and tree are rewound to T - 512 each time,
     # re-running a range rewrites identical values); a full tree rebuild for
     # comparison
-    keys_d = torch.from_numpy(keys_all[:T]).to(dev)
-    nb = T // 512
+    nblk = T // 512
     app = []
     for r in range(6):
-        layer.cache.c.n_blocks = nb - 1
+        layer.cache.c.n_blocks = nblk - 1
         if layer.tree is not None:
-            layer.tree.t.n_blocks = nb - 1
+            layer.tree.t.n_blocks = nblk - 1
         e0, e1 = ev(), ev()
         e0.record()
-        layer.append(keys_d, T - 512, T)
+        layer.append(keys, nblk * 512 - 512, nblk * 512)
         e1.record()
         torch.cuda.synchronize()
         if r >= 2:
@@ -610,80 +758,110 @@ def run_decode(args, dev, workload="flat_1m", mode="flat"):
             if r >= 1:
                 reb.append(e0.elapsed_time(e1) * 1e3)
         rebuild_us = round(float(np.median(reb)), 1)
-    out = {"workload": workload, "mode": mode, "T": T, "tokens": nd, "k": wl["k"], "list_len": lens,
+    out = {"mode": mode, "T": T, "tokens": nd, "k": wl["k"], "list_len": lens,
            "us_per_token": round(graph_us if graph_us is not None else eager_us, 2),
-           "us_per_token_eager": round(eager_us, 2),
+           "us_per_token_eager": round(eager_us, 2), "kernel_us_per_token": per_tok, "kernels": kernels,
            "block_append_us": round(float(np.median(app)), 1), "tree_rebuild_us": rebuild_us,
            "note": "batch 1; lsa_index_decode + lsa_sparse_attention per token, replayed from one CUDA graph; "
-                   "block_append_us: pool + cluster one completed block and grow the tree in place (every 512 "
-                   "tokens)"}
+                   "kernel times from an eager pass with per-kernel events; block_append_us: pool + cluster one "
+                   "completed block and grow the tree in place (every 512 tokens)"}
     if note:
         out["note"] = note
+    del layer
+    torch.cuda.empty_cache()
     return out
 
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(wl, keys_np, q_np, pos_np, K, V, hq, budget_s=20.0, sample=None):
-    """The oracle as it stands on this host's cores: full cache build + index and
-    attention of evenly spaced sample queries, extrapolated to all queries."""
+def _oracle_attention(O, lists, lens, Qb, kv_rows, hq):
+    """The oracle's attention over sampled lists, with the K/V rows fetched
+    for exactly the listed positions (kv_rows(rows) -> bf16 K, V rows)."""
+    used = np.unique(lists[lists >= 0])
+    remap = np.full(int(used.max()) + 1 if len(used) else 1, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    ll = np.where(lists >= 0, remap[np.maximum(lists, 0)], -1).astype(np.int32)
+    Kr, Vr = kv_rows(torch.from_numpy(used.astype(np.int64)))
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    O.attention(Qb, bits(Kr), bits(Vr), ll, lens)
+
+
+def cpu_baseline(wl, mode, keys_np, q_np, pos_np, budget_s=20.0, sample=None, kv_rows=None):
+    """The oracle as it stands on this host's cores, on a bounded sample of
+    the workload: the cache build (and the tree in Tree mode) over a sample
+    of whole blocks, then index + attention of evenly spaced sample queries
+    over the full cache; extrapolated to the full build and all queries."""
     import oracle as O
     cores = len(os.sched_getaffinity(0))
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
     O.build()
-    nq = len(pos_np)
+    T, nq, hq, hkv = wl["T"], len(pos_np), wl["hq"], wl["hkv"]
+    nblk = T // 512
+    # build: time the first b_s blocks, scale to all; the full cache is needed
+    # for the index anyway, so it is built in full but only the sample is timed
+    b_s = min(nblk, 1024)
     t0 = time.perf_counter()
+    O.build_cache(keys_np[:b_s * 512])
+    t_build_s = time.perf_counter() - t0
     oc = O.build_cache(keys_np)
-    ot = O.build_tree(oc) if wl["mode"] == "tree" else None
-    t_build = time.perf_counter() - t0
-    Kb = K.view(torch.int16).cpu().numpy().view(np.uint16)
-    Vb = V.view(torch.int16).cpu().numpy().view(np.uint16)
-    hkv = Kb.shape[1]
-    S = sample or 64
-    done, t_q = 0, 0.0
-    rng_idx = np.linspace(0, nq - 1, 4096).astype(np.int64)
+    ot = O.build_tree(oc) if mode == "tree" else None
+    t_build = t_build_s * nblk / b_s
+    if mode == "tree":
+        t0 = time.perf_counter()
+        O.build_tree(oc)
+        t_build += time.perf_counter() - t0
+    if kv_rows is None:
+        def kv_rows(rows):
+            n = len(rows)
+            f = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)  # noqa: E731
+            return (f(I.normal_bf16_bits(0, I.STREAM_K, (n, hkv, 128))),
+                    f(I.normal_bf16_bits(0, I.STREAM_V, (n, hkv, 128))))
+    S = sample or 16
+    grid = np.linspace(0, nq - 1, 4096).astype(np.int64)
     while True:
-        sel = rng_idx[(np.arange(S) * 4096 // S)]
+        sel = grid[(np.arange(S) * 4096 // S)]
         Qb = I.normal_bf16_bits(1, I.STREAM_Q, (S, hq, 128))
         t0 = time.perf_counter()
-        lists, lens = O.index(q_np[sel], pos_np[sel], oc, k=wl["k"], mode=wl["mode"], tree=ot,
+        lists, lens = O.index(q_np[sel], pos_np[sel], oc, k=wl["k"], mode=mode, tree=ot,
                               beam=wl.get("beam", 32))
-        O.attention(Qb, Kb, Vb, lists, lens)
+        _oracle_attention(O, lists, lens, Qb, kv_rows, hq)
         t_q = time.perf_counter() - t0
-        done = S
-        if t_q * 2 > budget_s or S >= 1024:
+        if sample or t_q * 2 > budget_s or S >= 1024:
             break
         S *= 2
-    per_q = t_q / done
+    per_q = t_q / S
     total = t_build + per_q * nq
-    return {"value": round(nq / total, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"full cache build ({t_build:.2f} s) + index and attention of {done} evenly spaced of "
-                      f"{nq} queries ({t_q:.2f} s), extrapolated to all queries",
-            "hkv": hkv}
+    return {"value": round(nq / total, 2), "unit": UNIT, "cores": cores, "kind": "oracle", "mode": mode,
+            "sample": f"cache build of {b_s} of {nblk} blocks timed ({t_build_s:.2f} s){' + tree' if ot else ''}, "
+                      f"index and attention of {S} evenly spaced of {nq} queries ({t_q:.2f} s); extrapolated to "
+                      f"the full build and all queries",
+            "sampled_seconds": round(t_build_s + t_q, 2)}
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the CPU oracle on this host, same metric and workload."""
+    """The reference arm: the CPU oracle on this host, same metric and
+    workload; each step is one timed bounded sample (its wall time is
+    ms_per_step) and the value is extrapolated from it."""
     if rank != 0:
         return
-    wl = dict(I.WORKLOADS[args.workload])
-    wl["mode"] = args.mode or ("flat" if wl["mode"] == "both" else wl["mode"])
-    keys_np, q_np, pos_np = make_prefill_inputs(wl)
-    T, nq, hq, hkv = wl["T"], wl["n_prefill"], wl["hq"], wl["hkv"]
-    Kb = torch.from_numpy(I.normal_bf16_bits(0, I.STREAM_K, (T, hkv, 128)).view(np.int16)).view(torch.bfloat16)
-    Vb = torch.from_numpy(I.normal_bf16_bits(0, I.STREAM_V, (T, hkv, 128)).view(np.int16)).view(torch.bfloat16)
-    vals = []
+    wl = workload(args)
+    wl["name"] = args.workload
+    keys_all, q_np, pos_np, _, _ = make_inputs(wl)
+    keys_np = keys_all[:wl["T"]]
+    mode = wl["modes"][0]
+    vals, walls = [], []
     for _ in range(args.warmup + args.steps):
-        vals.append(cpu_baseline(wl, keys_np, q_np, pos_np, Kb, Vb, hq, budget_s=args.cpu_budget, sample=32))
-    vals = vals[args.warmup:]
+        t0 = time.perf_counter()
+        vals.append(cpu_baseline(wl, mode, keys_np, q_np, pos_np, budget_s=args.cpu_budget, sample=16))
+        walls.append(time.perf_counter() - t0)
+    vals, walls = vals[args.warmup:], walls[args.warmup:]
     v = float(np.mean([x["value"] for x in vals]))
     line = {"metric": METRIC, "value": round(v, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(nq / v * 1e3, 1), "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(walls)), 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": args.workload if not args.queries else f"{args.workload}[last {nq} queries]",
-                   "T": T, "queries": nq, "k": wl["k"], "mode": wl["mode"],
-                       "Hq": hq, "Hkv": hkv, "head_dim": 128, "parallelism": "host cores"},
+            "impl": "reference", "config": workload_config(args, wl), "mode": mode,
+            "extrapolated": True,
+            "step": "one bounded sample per step (its wall time is ms_per_step): " + vals[-1]["sample"],
             "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": vals[-1]["cores"], "kind": "oracle",
                              "sample": vals[-1]["sample"]},
             "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -697,10 +875,10 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="flat_128k", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="flat_tree_10m", choices=sorted(I.WORKLOADS))
     ap.add_argument("--queries", type=int, default=0,
                     help="time only the last N prefill queries of the workload (profiling slices)")
-    ap.add_argument("--mode", default=None, choices=["flat", "tree"], help="override the workload's search mode")
+    ap.add_argument("--mode", default=None, choices=["flat", "tree"], help="run only this search mode")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-heads", action="store_true", help="skip the multi-head Flat index measurement")

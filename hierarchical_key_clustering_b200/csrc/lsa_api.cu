@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <vector>
 
 #include "lsa.h"
 #include "lsa_common.cuh"
@@ -370,6 +371,50 @@ void count_launches(int n)
     g_launches.fetch_add(n, std::memory_order_relaxed);
 }
 
+// Per-kernel timing: one record (name, start event, end event) per launch
+// while timing is on; events come from a pool and go back to it on read.
+namespace {
+struct KtRec {
+    const char *name;
+    cudaEvent_t a, b;
+    bool ended;
+};
+bool g_kt_on = false;
+std::vector<KtRec> g_kt;
+std::vector<cudaEvent_t> g_kt_pool;
+
+cudaEvent_t kt_event()
+{
+    cudaEvent_t e = nullptr;
+    if (!g_kt_pool.empty()) {
+        e = g_kt_pool.back();
+        g_kt_pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+        e = nullptr;
+    }
+    return e;
+}
+}  // namespace
+
+int kt_begin(const char *name, cudaStream_t st)
+{
+    if (!g_kt_on) return -1;
+    cudaEvent_t a = kt_event(), b = kt_event();
+    if (!a || !b || cudaEventRecord(a, st) != cudaSuccess) {
+        if (a) g_kt_pool.push_back(a);
+        if (b) g_kt_pool.push_back(b);
+        return -1;
+    }
+    g_kt.push_back(KtRec{name, a, b, false});
+    return (int)g_kt.size() - 1;
+}
+
+void kt_end(int handle, cudaStream_t st)
+{
+    if (handle < 0 || handle >= (int)g_kt.size()) return;
+    g_kt[handle].ended = cudaEventRecord(g_kt[handle].b, st) == cudaSuccess;
+}
+
 int report_error(int code, const char *msg)
 {
     return fail(code, "%s", msg);
@@ -397,21 +442,43 @@ int lsa_check_device_errors(void)
     return v;
 }
 
-void lsa_attention_timing(int32_t enable)
+void lsa_kernel_timing(int32_t enable)
 {
-    lsa::attention_timing(enable != 0);
+    lsa::g_kt_on = enable != 0;
 }
 
-int lsa_attention_timing_read(double *near_ms, double *gather_ms, int32_t *calls)
+int lsa_kernel_timing_read(char *names, int32_t name_len, double *ms, int64_t *launches, int32_t max_kernels)
 {
-    double a = 0.0, b = 0.0;
     int n = 0;
-    cudaError_t e = lsa::attention_timing_read(a, b, n);
-    if (near_ms) *near_ms = a;
-    if (gather_ms) *gather_ms = b;
-    if (calls) *calls = n;
-    if (e != cudaSuccess) return cuda_fail(e, "attention timing events");
-    return LSA_OK;
+    cudaError_t err = cudaSuccess;
+    std::vector<const char *> seen;
+    for (auto &r : lsa::g_kt) {
+        float x = 0.0f;
+        cudaError_t e = r.ended ? cudaEventSynchronize(r.b) : cudaErrorNotReady;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&x, r.a, r.b);
+        if (e != cudaSuccess && r.ended) err = e;
+        lsa::g_kt_pool.push_back(r.a);
+        lsa::g_kt_pool.push_back(r.b);
+        if (e != cudaSuccess) continue;
+        int i = 0;
+        while (i < (int)seen.size() && strcmp(seen[i], r.name) != 0) ++i;
+        if (i == (int)seen.size()) {
+            seen.push_back(r.name);
+            if (i < max_kernels) {
+                if (names && name_len > 0) snprintf(names + (int64_t)i * name_len, (size_t)name_len, "%s", r.name);
+                if (ms) ms[i] = 0.0;
+                if (launches) launches[i] = 0;
+            }
+        }
+        if (i < max_kernels) {
+            if (ms) ms[i] += x;
+            if (launches) launches[i] += 1;
+        }
+    }
+    lsa::g_kt.clear();
+    n = (int)seen.size();
+    if (err != cudaSuccess) return cuda_fail(err, "kernel timing events");
+    return n;
 }
 
 void lsa_debug_wait_test(int32_t enable)

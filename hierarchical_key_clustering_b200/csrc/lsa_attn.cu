@@ -699,60 +699,10 @@ int attention_list_cap()
     return 1 << 30;  // the list is streamed, not staged: any length
 }
 
-// Per-kernel timing (lsa_attention_timing): three events per call.
-namespace {
-bool g_time_on = false;
-struct TimedCall {
-    std::array<cudaEvent_t, 3> ev;
-    bool near;  // the near-set kernels ran
-};
-std::vector<TimedCall> g_time_calls;
-std::vector<cudaEvent_t> g_time_pool;
-cudaEvent_t time_event()
-{
-    cudaEvent_t e = nullptr;
-    if (!g_time_pool.empty()) {
-        e = g_time_pool.back();
-        g_time_pool.pop_back();
-    } else if (cudaEventCreate(&e) != cudaSuccess) {
-        e = nullptr;
-    }
-    return e;
-}
-}  // namespace
-
-void attention_timing(bool on) { g_time_on = on; }
-
-cudaError_t attention_timing_read(double &near_ms, double &gather_ms, int &calls)
-{
-    near_ms = gather_ms = 0.0;
-    calls = 0;
-    cudaError_t err = cudaSuccess;
-    for (auto &c : g_time_calls) {
-        float x = 0.0f, y = 0.0f;
-        cudaError_t e = cudaEventSynchronize(c.ev[2]);
-        if (e == cudaSuccess && c.near) e = cudaEventElapsedTime(&x, c.ev[0], c.ev[1]);
-        if (e == cudaSuccess) e = cudaEventElapsedTime(&y, c.ev[1], c.ev[2]);
-        if (e != cudaSuccess) err = e;
-        near_ms += x;
-        gather_ms += y;
-        ++calls;
-        for (cudaEvent_t ev : c.ev) g_time_pool.push_back(ev);
-    }
-    g_time_calls.clear();
-    return err;
-}
-
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
 {
     (void)n_sm;
     if (a.nq <= 0) return cudaSuccess;
-    std::array<cudaEvent_t, 3> tev = {nullptr, nullptr, nullptr};
-    if (g_time_on) {
-        for (auto &e : tev) e = time_event();
-        if (tev[0] && tev[1] && tev[2]) cudaEventRecord(tev[0], st);
-        else g_time_on = false;
-    }
     const int smem = AWARPS * WARP_BYTES;
     const int G = a.Hq / a.Hkv;
     auto kern = G <= 8 ? k_attn<1> : k_attn<2>;
@@ -763,29 +713,31 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     if (a.near_plan) {  // near sets of consecutive queries first (plans + partials)
         const int QT = near_tile_queries(G);
         const unsigned tiles = (unsigned)((a.nq + QT - 1) / QT);
+        int kt = kt_begin("k_near_plan", st);
         k_near_plan<<<tiles, NEAR_ROWS, 0, st>>>(a);
+        kt_end(kt, st);
         if ((e = cudaFuncSetAttribute(k_attn_near, cudaFuncAttributeMaxDynamicSharedMemorySize, NEAR_SMEM)) !=
             cudaSuccess)
             return e;
+        kt = kt_begin("k_attn_near", st);
         k_attn_near<<<dim3(tiles, (unsigned)a.Hkv), NEAR_WARPS * 32, NEAR_SMEM, st>>>(a);
+        kt_end(kt, st);
         count_launches(2);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (g_time_on) cudaEventRecord(tev[1], st);
     const int64_t units = a.nq * a.Hkv * a.nsplit;
     const int64_t blocks = (units + AWARPS - 1) / AWARPS;
     // split lists (few queries, decode): short kernels, launched back to back
-    if ((e = launch_k(a.nsplit > 1, kern, dim3((unsigned)blocks), dim3(AWARPS * 32), (size_t)smem, st, a, kps)) !=
-        cudaSuccess)
-        return e;
+    int kt = kt_begin("k_attn", st);
+    e = launch_k(a.nsplit > 1, kern, dim3((unsigned)blocks), dim3(AWARPS * 32), (size_t)smem, st, a, kps);
+    kt_end(kt, st);
+    if (e != cudaSuccess) return e;
     count_launches(1);
     if (a.nsplit > 1) {
+        kt = kt_begin("k_attn_combine", st);
         e = launch_k(true, k_attn_combine, dim3((unsigned)(a.nq * a.Hq)), dim3(512), 0, st, a);
+        kt_end(kt, st);
         count_launches(1);
-    }
-    if (g_time_on && e == cudaSuccess) {
-        cudaEventRecord(tev[2], st);
-        g_time_calls.push_back(TimedCall{tev, a.near_plan != nullptr});
     }
     return e;
 }

@@ -504,7 +504,9 @@ cudaError_t launch_pool_norm(const float *keys, int64_t item_begin, int64_t item
     int64_t blocks = (warps + 7) / 8;
     int64_t cap = (int64_t)n_sm * 16;
     if (blocks > cap) blocks = cap;
+    const int kt = kt_begin("k_pool_norm", st);
     k_pool_norm<<<(unsigned)blocks, 256, 0, st>>>(keys, item_begin, item_end, pooled);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -521,8 +523,10 @@ cudaError_t launch_ward(const float *pooled, int64_t blk_begin, int64_t blk_end,
     int64_t n = blk_end - blk_begin;
     for (int64_t s = 0; s < n; s += 2147483647LL) {
         int64_t cnt = (n - s) < 2147483647LL ? (n - s) : 2147483647LL;
+        const int kt = kt_begin("k_ward", st);
         k_ward<<<(unsigned)cnt, 128, WARD_SMEM, st>>>(pooled, blk_begin + s, cap, item_bucket, members, count,
                                                       centroid, centroid_bf16);
+        kt_end(kt, st);
         count_launches(1);
     }
     return cudaGetLastError();
@@ -537,7 +541,9 @@ cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32
     int64_t blocks = (nb - g_first + 7) / 8;
     if (blocks > (int64_t)n_sm * 16) blocks = (int64_t)n_sm * 16;
     if (blocks < 1) blocks = 1;
+    const int kt = kt_begin("k_tree_leaves", st);
     k_tree_leaves<<<(unsigned)blocks, 256, 0, st>>>(pooled, members, count, g_first, nb, tr);
+    kt_end(kt, st);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -550,8 +556,10 @@ cudaError_t launch_tree(const float *pooled, const int32_t *members, const int32
         const int64_t runs = (n_prev + LSA_RUN - 1) / LSA_RUN;
         const int64_t run0 = changed / LSA_RUN;
         if (runs > run0) {
+            const int ktp = kt_begin("k_tree_pair", st);
             k_tree_pair<<<(unsigned)(runs - run0), 128, WARD_SMEM, st>>>(tr, run0, level_offset[l - 1], n_prev,
                                                                         level_offset[l]);
+            kt_end(ktp, st);
             count_launches(1);
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;

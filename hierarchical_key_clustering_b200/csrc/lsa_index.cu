@@ -1516,16 +1516,19 @@ cudaError_t launch_expand_merged(const IndexArgs &a, const IndexWs &m, cudaStrea
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
     const int KC = m.cap;
     const size_t smr = rank_expand_smem(KC, TW);
+    const int kt = kt_begin("k_rank_expand", st);
     if (a.nq <= SMALL_NQ) {
         cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         const cudaError_t e = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
                                        a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
                                        a.window, a.P, KC, TW, m);
+        kt_end(kt, st);
         if (e != cudaSuccess) return e;
     } else {
         cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists,
                                                              a.lens, a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, m);
+        kt_end(kt, st);
     }
     count_launches(1);
     return cudaGetLastError();
@@ -1547,9 +1550,11 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
     {
         int64_t blocks = (rows + 7) / 8;
         if (blocks > (int64_t)n_sm * 32) blocks = (int64_t)n_sm * 32;
-        if ((e = launch_k(rows <= SMALL_NQ, k_qnorm, dim3((unsigned)blocks), dim3(256), 0, st, a.qidx, a.pos, rows,
-                          heads, a.pos_shift, a.n_blocks, ws)) != cudaSuccess)
-            return e;
+        const int kt = kt_begin("k_qnorm", st);
+        e = launch_k(rows <= SMALL_NQ, k_qnorm, dim3((unsigned)blocks), dim3(256), 0, st, a.qidx, a.pos, rows, heads,
+                     a.pos_shift, a.n_blocks, ws);
+        kt_end(kt, st);
+        if (e != cudaSuccess) return e;
         count_launches(1);
     }
     const int64_t nb_total = a.n_blocks * LSA_NBKT;
@@ -1558,13 +1563,17 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
         if (rows <= SMALL_NQ) {  // stream every centroid once for the whole batch, keep the scores
             const int dsm = DS_WARPS * 2 * 32 * DS_ROW;
             cudaFuncSetAttribute(k_dscore, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-            if ((e = launch_k(true, k_dscore, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
-                              (size_t)dsm, st, rows, nb_total, a.centroid_bf16, a.P, ws)) != cudaSuccess)
-                return e;
+            int kt = kt_begin("k_dscore", st);
+            e = launch_k(true, k_dscore, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
+                         (size_t)dsm, st, rows, nb_total, a.centroid_bf16, a.P, ws);
+            kt_end(kt, st);
+            if (e != cudaSuccess) return e;
             count_launches(1);
-            if ((e = launch_k(true, k_dfilter, dim3((unsigned)((nb_total / 4 + 255) / 256)), dim3(256), 0, st, rows, a.P,
-                              ws)) != cudaSuccess)
-                return e;
+            kt = kt_begin("k_dfilter", st);
+            e = launch_k(true, k_dfilter, dim3((unsigned)((nb_total / 4 + 255) / 256)), dim3(256), 0, st, rows, a.P,
+                         ws);
+            kt_end(kt, st);
+            if (e != cudaSuccess) return e;
             count_launches(1);
         } else {  // two passes on the tensor cores: threshold, then filter
             ScoreTcArgs sa;
@@ -1578,7 +1587,9 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
             int whole = 0;
             if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, &whole)) != cudaSuccess) return e;
             if (!whole) {  // thresholds from the merged histograms
+                const int kt = kt_begin("k_tau", st);
                 k_tau<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(rows, a.P, ws);
+                kt_end(kt, st);
                 count_launches(1);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
@@ -1592,6 +1603,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
         // candidates per level: the children of at most B1 kept nodes plus one run
         const int CM = (int)(2 * B1 + LSA_RUN + 2);
         const int KM = (int)B1;
+        const int kt = kt_begin("k_tree_beam", st);
         if (small) {  // one query per CTA of 16 warps
             auto kern = k_tree_beam<16, 1>;
             const size_t tb = tree_beam_team_bytes(CM, KM, 16);
@@ -1606,6 +1618,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
             e = launch_k(false, kern, dim3((unsigned)((a.nq + qpb - 1) / qpb)), dim3(32 * BEAM_TEAM * qpb), qpb * tb,
                          st, a.nq, *tree, a.beam, a.P, CM, KM, ws);
         }
+        kt_end(kt, st);
         if (e != cudaSuccess) return e;
         count_launches(1);
     }
@@ -1613,13 +1626,17 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
         const int TS = heads_merge_slots(heads, a.P);
         const size_t smh = (size_t)TS * 8;
         cudaFuncSetAttribute(k_heads_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smh);
-        if ((e = launch_k(small, k_heads_merge, dim3((unsigned)a.nq), dim3(HM_THREADS), smh, st, heads, a.P, TS,
-                          a.centroid_bf16, ws, *merged)) != cudaSuccess)
-            return e;
+        int kt = kt_begin("k_heads_merge", st);
+        e = launch_k(small, k_heads_merge, dim3((unsigned)a.nq), dim3(HM_THREADS), smh, st, heads, a.P, TS,
+                     a.centroid_bf16, ws, *merged);
+        kt_end(kt, st);
+        if (e != cudaSuccess) return e;
         const unsigned xg = (unsigned)min((int64_t)n_sm, a.nq);
-        if ((e = launch_k(small, k_heads_exact, dim3(xg), dim3(HM_THREADS), 0, st, a.nq, heads, a.P, a.centroid_bf16,
-                          ws, *merged)) != cudaSuccess)
-            return e;
+        kt = kt_begin("k_heads_exact", st);
+        e = launch_k(small, k_heads_exact, dim3(xg), dim3(HM_THREADS), 0, st, a.nq, heads, a.P, a.centroid_bf16, ws,
+                     *merged);
+        kt_end(kt, st);
+        if (e != cudaSuccess) return e;
         count_launches(2);
         if (a.no_expand) return cudaGetLastError();  // a shard's local candidate set stops here
     }
@@ -1630,16 +1647,19 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
     // (a merged set never has more than its slots)
     const int KC = merged ? merged->cap : (int)min((int64_t)ws.cap, pow2_ceil64(((int64_t)a.P * 3 + 1) / 2));
     const size_t smr = rank_expand_smem(KC, TW);
+    const int kt = kt_begin("k_rank_expand", st);
     if (small) {  // one CTA per query, few queries: widest blocks
         cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         const cudaError_t el = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
                                         a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
                                         a.window, a.P, KC, TW, ex);
+        kt_end(kt, st);
         if (el != cudaSuccess) return el;
     } else {
         cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
         k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,
                                                              a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ex);
+        kt_end(kt, st);
     }
     count_launches(1);
     return cudaGetLastError();

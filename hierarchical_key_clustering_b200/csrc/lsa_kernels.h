@@ -9,6 +9,13 @@ namespace lsa {
 // Kernels enqueued since load (see lsa_launch_count in lsa.h).
 void count_launches(int n);
 
+// Per-kernel timing (lsa_kernel_timing in lsa.h): while it is on, every
+// launch site brackets its kernel with two events on the launch's stream,
+// tagged with the kernel's name.  kt_begin returns the record's handle (-1
+// when timing is off); kt_end records the closing event.
+int kt_begin(const char *name, cudaStream_t st);
+void kt_end(int handle, cudaStream_t st);
+
 struct TreeDev {
     int32_t *child;
     int32_t *parent;
@@ -206,8 +213,6 @@ constexpr int NEAR_ROWS = 128;
 __host__ __device__ inline int near_tile_queries(int G) { return (G >= 1 && NEAR_ROWS % G == 0) ? NEAR_ROWS / G : 0; }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm);
-void attention_timing(bool on);
-cudaError_t attention_timing_read(double &near_ms, double &gather_ms, int &calls);
 int attention_list_cap();
 
 }  // namespace lsa

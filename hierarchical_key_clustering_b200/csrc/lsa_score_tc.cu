@@ -463,7 +463,9 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
                         (a.mode == 0 ? HIST_BYTES : ROWCNT_BYTES) + sizeof(TcSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    const int kt = kt_begin(a.mode == 0 ? "k_score_tc:threshold" : "k_score_tc:filter", st);
     k_score_tc<<<dim3((unsigned)qpairs, (unsigned)chunks), THREADS, smem, st>>>(tmA, tmB, b, ws);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }

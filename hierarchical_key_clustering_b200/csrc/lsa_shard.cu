@@ -39,7 +39,9 @@ cudaError_t launch_shard_pack(const IndexWs &m, int64_t nq, int64_t g0, void *xc
     if (nq <= 0) return cudaSuccess;
     int32_t *xcnt = reinterpret_cast<int32_t *>(xchg);
     int2 *xent = reinterpret_cast<int2 *>(reinterpret_cast<char *>(xchg) + ((nq * 4 + 255) / 256) * 256);
+    const int kt = kt_begin("k_shard_pack", st);
     k_shard_pack<<<(unsigned)nq, 256, 0, st>>>(m, nq, g0, xcnt, xent);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -209,7 +211,9 @@ cudaError_t launch_shard_merge(const void *xchg_all, int n_shards, int64_t nq, i
     const int2 *xent = reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(xchg_all) + cnt_bytes);
     const size_t smem = (size_t)n_shards * slots * 8;
     cudaFuncSetAttribute(k_shard_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int kt = kt_begin("k_shard_merge", st);
     k_shard_merge<<<(unsigned)nq, SM_THREADS, smem, st>>>(xcnt, xent, n_shards, nq, xstride, slots, P, m);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -246,7 +250,9 @@ cudaError_t launch_local_lists(const int32_t *lists, const int32_t *lens, int64_
                                int64_t t1, int32_t *out_lists, int32_t *out_lens, cudaStream_t st)
 {
     if (nq <= 0) return cudaSuccess;
+    const int kt = kt_begin("k_local_lists", st);
     k_local_lists<<<(unsigned)((nq + 7) / 8), 256, 0, st>>>(lists, lens, nq, Lmax, t0, t1, out_lists, out_lens);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -269,8 +275,10 @@ cudaError_t launch_publish_members(const int32_t *members, const int32_t *count,
                                    int64_t pos0, int32_t *members_out, int32_t *count_out, cudaStream_t st)
 {
     if (nb <= 0) return cudaSuccess;
+    const int kt = kt_begin("k_publish_members", st);
     k_publish_members<<<(unsigned)((nb * LSA_NSLOT + 255) / 256), 256, 0, st>>>(members, count, nb, g0, pos0,
                                                                                members_out, count_out);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -320,7 +328,9 @@ cudaError_t launch_combine_parts(const uint16_t *O_parts, const float *lse_parts
 {
     const int64_t units = nq * Hq;
     if (units <= 0) return cudaSuccess;
+    const int kt = kt_begin("k_combine_parts", st);
     k_combine_parts<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(O_parts, lse_parts, n_parts, units, O, lse);
+    kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -202,7 +202,9 @@ cudaError_t launch_shrink(const uint16_t *V, const uint16_t *W, const ShrinkArgs
         ShrinkArgs b = a;
         b.t_begin = a.t_begin + s * SH_M;
         const int64_t n = min(tiles - s, (int64_t)2147483647LL);
+        const int kt = kt_begin("k_shrink", st);
         k_shrink<<<(unsigned)n, SH_THREADS, SH_SMEM, st>>>(tmV, tmW, b);
+        kt_end(kt, st);
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

@@ -95,7 +95,8 @@ class SparseLayer:
                                  stream=stream)
         return O
 
-    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int = 16):
+    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int = 16,
+                          kv_cache=None, kv_first: int = 0):
         """One prefill step whose inputs and output live in pinned host memory.
 
         Three streams overlap the transfers with the kernels.  The index
@@ -113,6 +114,11 @@ class SparseLayer:
         those of build + index + attend on device copies of the inputs, up to
         the attention's summation order when a chunk holds so few (query, KV
         head) units that the attention splits lists over warps.
+
+        kv_cache=(K, V): device tensors [Tk, Hkv, 128] that already hold the
+        K/V rows of positions < kv_first (the KV cache of the earlier
+        context); h_K/h_V then hold only rows kv_first..Tk-1, which are copied
+        into them before the attention that can read them.
         """
         nq = h_Q.shape[0]
         assert nq <= self.max_queries
@@ -120,13 +126,19 @@ class SparseLayer:
         cs = torch.cuda.current_stream(dev)
         if self._h2d is None:
             self._h2d, self._d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        hs = (h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O)
+        hs = (h_keys, h_qidx, h_pos, h_Q, h_O) + (() if kv_cache is not None else (h_K, h_V))
         key = tuple((tuple(t.shape), t.dtype) for t in hs)
         if self._dbuf_key != key:
             self._dbuf = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hs]
             self._dbuf_key = key
-        d_keys, d_q, d_pos, d_Q, d_K, d_V, d_O = self._dbuf
-        tk = h_K.shape[0]
+        d_keys, d_q, d_pos, d_Q, d_O = self._dbuf[:5]
+        if kv_cache is not None:
+            d_K, d_V = kv_cache
+            assert d_K.shape[0] == kv_first + h_K.shape[0] and d_V.shape == d_K.shape
+        else:
+            d_K, d_V = self._dbuf[5:]
+            kv_first = 0
+        tk = d_K.shape[0]
         bounds, need = chunk_plan(h_pos, chunks, h_K.shape[1], tk)
         self._h2d.wait_stream(cs)
         with torch.cuda.stream(self._h2d):
@@ -137,18 +149,18 @@ class SparseLayer:
             d_pos.copy_(h_pos, non_blocking=True)
             e_idx = torch.cuda.Event()
             e_idx.record()
-            e_in, have = [], 0
+            e_in, have = [], kv_first
             for (c0, c1), n in zip(bounds, need):
                 if n > have:
-                    d_K[have:n].copy_(h_K[have:n], non_blocking=True)
-                    d_V[have:n].copy_(h_V[have:n], non_blocking=True)
+                    d_K[have:n].copy_(h_K[have - kv_first:n - kv_first], non_blocking=True)
+                    d_V[have:n].copy_(h_V[have - kv_first:n - kv_first], non_blocking=True)
                     have = n
                 d_Q[c0:c1].copy_(h_Q[c0:c1], non_blocking=True)
                 e_in.append(torch.cuda.Event())
                 e_in[-1].record()
             if have < tk:
-                d_K[have:].copy_(h_K[have:], non_blocking=True)
-                d_V[have:].copy_(h_V[have:], non_blocking=True)
+                d_K[have:].copy_(h_K[have - kv_first:], non_blocking=True)
+                d_V[have:].copy_(h_V[have - kv_first:], non_blocking=True)
             e_all = torch.cuda.Event()
             e_all.record()
         cs.wait_event(e_keys)

@@ -57,7 +57,7 @@ class lsa_tree(C.Structure):
 
 
 EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_check_device_errors",
-           "lsa_debug_wait_test", "lsa_attention_timing", "lsa_attention_timing_read", "lsa_list_budget", "lsa_top_buckets",
+           "lsa_debug_wait_test", "lsa_kernel_timing", "lsa_kernel_timing_read", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
            "lsa_shrink", "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
@@ -98,8 +98,8 @@ def lib():
             "lsa_launch_count": (i64, []),
             "lsa_check_device_errors": (C.c_int, []),
             "lsa_debug_wait_test": (None, [i32]),
-            "lsa_attention_timing": (None, [i32]),
-            "lsa_attention_timing_read": (C.c_int, [C.POINTER(C.c_double), C.POINTER(C.c_double), C.POINTER(i32)]),
+            "lsa_kernel_timing": (None, [i32]),
+            "lsa_kernel_timing_read": (C.c_int, [C.c_char_p, i32, C.POINTER(C.c_double), C.POINTER(i64), i32]),
             "lsa_list_budget": (i32, [pp]),
             "lsa_top_buckets": (i32, [pp]),
             "lsa_cache_bytes": (i64, [i64]),
@@ -173,16 +173,26 @@ def lsa_launch_count() -> int:
     return lib().lsa_launch_count()
 
 
-def lsa_attention_timing(enable: bool) -> None:
-    """Record per-kernel CUDA events in every lsa_sparse_attention call (profiling aid)."""
-    lib().lsa_attention_timing(1 if enable else 0)
+def lsa_kernel_timing(enable: bool) -> None:
+    """Bracket every kernel the library launches with CUDA events on its
+    stream (profiling aid; not while a stream is being captured)."""
+    lib().lsa_kernel_timing(1 if enable else 0)
 
 
-def lsa_attention_timing_read():
-    """(near-set ms, gather ms, calls) summed since the last read; waits for the events."""
-    a, b, n = C.c_double(), C.c_double(), C.c_int32()
-    _check(lib().lsa_attention_timing_read(C.byref(a), C.byref(b), C.byref(n)))
-    return a.value, b.value, n.value
+def lsa_kernel_timing_read(max_kernels: int = 64) -> dict:
+    """{kernel name: (milliseconds, launches)} summed since the last read, in
+    first-launch order; waits for the recorded events."""
+    name_len = 64
+    names = C.create_string_buffer(name_len * max_kernels)
+    ms = (C.c_double * max_kernels)()
+    launches = (C.c_int64 * max_kernels)()
+    n = lib().lsa_kernel_timing_read(names, name_len, ms, launches, max_kernels)
+    _check(n if n < 0 else 0)
+    out = {}
+    for i in range(min(n, max_kernels)):
+        nm = names.raw[i * name_len:(i + 1) * name_len].split(b"\0", 1)[0].decode()
+        out[nm] = (ms[i], int(launches[i]))
+    return out
 
 
 def lsa_check_device_errors() -> int:

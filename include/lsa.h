@@ -177,16 +177,19 @@ int64_t lsa_launch_count(void);
 int lsa_check_device_errors(void);
 void lsa_debug_wait_test(int32_t enable);
 
-/* Per-kernel timing of lsa_sparse_attention, a profiling aid.  While enabled
- * (lsa_attention_timing(1)), every call records three CUDA events on its own
- * stream: before its near-set kernels (plan + dense tiles), between them and
- * the gather kernel (with its split merge), and after; nothing else changes.
- * lsa_attention_timing_read waits for the recorded events and returns the
- * milliseconds summed over the calls since the last read (near set, 0 for a
- * call that did not take it; gather) and their count, then forgets them.  Returns LSA_OK or LSA_ERR_CUDA.  Not
- * thread-safe: enable, call and read from one host thread. */
-void lsa_attention_timing(int32_t enable);
-int lsa_attention_timing_read(double *near_ms, double *gather_ms, int32_t *calls);
+/* Per-kernel timing, a profiling aid.  While enabled (lsa_kernel_timing(1)),
+ * every kernel the library launches is bracketed by two CUDA events recorded
+ * on the stream it is launched on, tagged with the kernel's name (the
+ * tensor-core score passes as "k_score_tc:threshold" and
+ * "k_score_tc:filter"); nothing else changes.  lsa_kernel_timing_read waits
+ * for the recorded events, sums milliseconds and launches per kernel name
+ * since the last read, writes up to max_kernels of them (names as
+ * NUL-terminated strings of name_len bytes each, in first-launch order) and
+ * forgets the records.  Returns the number of distinct kernels (which may
+ * exceed max_kernels), or LSA_ERR_CUDA.  Not thread-safe: enable, call and
+ * read from one host thread; do not enable it around a stream capture. */
+void lsa_kernel_timing(int32_t enable);
+int lsa_kernel_timing_read(char *names, int32_t name_len, double *ms, int64_t *launches, int32_t max_kernels);
 
 
 /* Longest index list: sink + window + 1 (the query itself) + k. */
