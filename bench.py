@@ -417,9 +417,10 @@ def measure_index_heads(layer, keys_np, pos_np, wl: dict, dev, heads: int = 8, c
             "tokens_per_s": round(nq / (ms / 1e3), 1)}
 
 
-def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, ranks: int, chunk: int = 16384):
-    """The context-parallel step of the workload split over `ranks` token
-    ranges, every rank's stages run one after another on this one GPU (the
+def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, ranks: int, chunk: int = 16384,
+                             layout: str = "zigzag"):
+    """The context-parallel step of the workload split over `ranks` ranks in
+    `layout`, every rank's stages run one after another on this one GPU (the
     all-gathers become stacking): per stage, the slowest rank's kernel time
     over all queries (chunks of `chunk`), and the bytes each rank would
     send and receive.  Communication time is not included."""
@@ -427,22 +428,23 @@ def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, rank
 
     T, nq, hq = wl["T"], len(pos_np), wl["hq"]
     chunk = min(chunk, nq)
-    shards = [CP.Shard(r, ranks, T, k=wl["k"], max_queries=chunk, device=dev) for r in range(ranks)]
+    shards = [CP.Shard(r, ranks, T, k=wl["k"], max_queries=chunk, layout=layout, device=dev) for r in range(ranks)]
     keys = torch.from_numpy(keys_np).to(dev)
     qidx = torch.from_numpy(q_np).to(dev)
     pos = torch.from_numpy(pos_np).to(dev)
     Lmax = shards[0].Lmax
-    ws_attn = lsa.workspace(lsa.lsa_attention_workspace_bytes(chunk, hq, 128, Lmax), dev)
+    span = max(t1 - t0 for s in shards for t0, t1 in s.spans)
+    ws_attn = lsa.workspace(lsa.lsa_attention_workspace_bytes(chunk, hq, 128, Lmax, span), dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    t_build = []
+    t_build, built = [], []
     for s in shards:
         a, b = ev(), ev()
         a.record()
-        s.build(keys[s.t0:s.t1])
+        built.append(s.build(keys))
         b.record()
         t_build.append((a, b))
-    M = torch.stack([s.members_slice for s in shards])
-    C = torch.stack([s.count_slice for s in shards])
+    M = torch.stack([x[0] for x in built])
+    C = torch.stack([x[1] for x in built])
     for s in shards:
         s.set_members(M, C)
 
@@ -469,7 +471,7 @@ def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, rank
             for r, s in enumerate(shards):
                 a, b = ev(), ev()
                 a.record()
-                parts.append(s.attend_local(Q[c0:c1], K[s.t0:s.t1], V[s.t0:s.t1], lists, lens, ws=ws_attn))
+                parts.append(s.attend_local(Q[c0:c1], K, V, lists, lens, ws=ws_attn))
                 b.record()
                 t_att[r].append((a, b))
             Op, Lp = torch.stack([p_[0] for p_ in parts]), torch.stack([p_[1] for p_ in parts])
@@ -488,14 +490,17 @@ def measure_context_parallel(wl: dict, keys_np, pos_np, q_np, Q, K, V, dev, rank
     loc, mrg, att, cmb = one_pass(True)
     per_rank = [loc[r] + mrg + att[r] + cmb for r in range(ranks)]
     step = max(per_rank)
-    xbytes = lsa.lsa_shard_exchange_bytes(nq, shards[0].p)
-    part_bytes = nq * hq * (128 * 2 + 4)
-    return {"ranks": ranks, "emulated_on_one_gpu": True, "queries": nq, "chunk": chunk,
+    n_parts = len(shards[0].parts)
+    xbytes = lsa.lsa_shard_exchange_bytes(nq, shards[0].p) * n_parts
+    part_bytes = nq * hq * (128 * 2 + 4) * n_parts
+    return {"ranks": ranks, "layout": layout, "emulated_on_one_gpu": True, "queries": nq, "chunk": chunk,
             "build_ms_max_rank": round(max(a.elapsed_time(b) for a, b in t_build), 3),
             "index_local_ms": {"max_rank": round(max(loc), 3), "min_rank": round(min(loc), 3)},
             "merge_and_expand_ms": round(mrg, 3),
             "attention_local_ms": {"max_rank": round(max(att), 3), "min_rank": round(min(att), 3)},
             "combine_ms": round(cmb, 3), "step_ms_slowest_rank": round(step, 3),
+            "attention_slowest_over_mean": round(max(att) / float(np.mean(att)), 3),
+            "step_slowest_over_mean": round(step / float(np.mean(per_rank)), 3),
             "step_ms_mean_rank": round(float(np.mean(per_rank)), 3),
             "tokens_per_s_without_communication": round(nq / (step / 1e3), 1),
             "allgather_bytes_sent_per_rank": xbytes + part_bytes,
@@ -541,7 +546,8 @@ def run_ours(args, world, rank, local):
         index_heads = measure_index_heads(keep, keys_np, pos_np, wl, dev)
     context_parallel = None
     if args.cp > 1 and primary == "flat":
-        context_parallel = measure_context_parallel(wl, keys_np, pos_np, q_np, Q, K[:T], V[:T], dev, args.cp)
+        context_parallel = {lay: measure_context_parallel(wl, keys_np, pos_np, q_np, Q, K[:T], V[:T], dev, args.cp,
+                                                          layout=lay) for lay in ("zigzag", "contiguous")}
 
     # end to end: same calls, the step's inputs from pinned host memory, O back
     e2e = None if args.no_e2e else run_e2e(args, keep, keys_np, q_np, pos_np, Q, K, V, wl, dev, world)

@@ -88,6 +88,37 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int by
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes));
 }
 
+__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void *src, int bytes, uint64_t pol)
+{
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
+                 "r"(bytes), "l"(pol));
+}
+
+__device__ __forceinline__ float ld_f_hint(const float *p, uint64_t pol)
+{
+    float v;
+    asm volatile("ld.global.L2::cache_hint.f32 %0, [%1], %2;\n" : "=f"(v) : "l"(p), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ float2 ld_f2_hint(const float *p, uint64_t pol)
+{
+    float2 v;
+    asm volatile("ld.global.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;\n" : "=f"(v.x), "=f"(v.y) : "l"(p), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ void st_f_hint(float *p, float v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_f2_hint(float *p, float2 v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;\n" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_commit()
 {
     asm volatile("cp.async.commit_group;\n" ::);
@@ -126,7 +157,17 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x)
 // heads 2c, 2c + 1 of each column tile, and keeps the running max / sum of
 // those two heads; P^T turns into the B operand of the PV product by one
 // movmatrix transpose per 8 x 8 block.
-template <int NT>
+//
+// PH (position-range phases, AttnArgs::state_o set): the launch runs one KV
+// head phase_g and one key range phase_r for every query (one warp per
+// query): the query's list entries in that range, starting from the running
+// result the earlier ranges left in state_o / state_ml (nothing yet when the
+// running max is -inf).  The warp whose range holds the query's last entry
+// writes the normalised output and lse; the others write the running result
+// back.  K/V rows are fetched with an L2 evict-last policy and the
+// per-query data with evict-first, so the range's rows stay in L2 while
+// every query reads them.
+template <int NT, bool PH>
 __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_split)
 {
     pdl_wait();
@@ -134,23 +175,39 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     extern __shared__ __align__(128) uint8_t asmem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t unit = (int64_t)blockIdx.x * AWARPS + warp;
-    const int64_t total = a.nq * a.Hkv * a.nsplit;
+    const int64_t total = PH ? a.nq : a.nq * a.Hkv * a.nsplit;
     if (unit >= total) return;
     // head-major order: the warps in flight all read one KV head, whose rows
     // (Tk x 512 B of K+V) stay resident in L2 while its queries run
-    const int split = (int)(unit % a.nsplit);
-    const int64_t qg = unit / a.nsplit;
-    const int g = (int)(qg / a.nq);
-    const int64_t q = qg % a.nq;
+    const int split = PH ? 0 : (int)(unit % a.nsplit);
+    const int64_t qg = PH ? unit : unit / a.nsplit;
+    const int g = PH ? a.phase_g : (int)(qg / a.nq);
+    const int64_t q = PH ? unit : qg % a.nq;
     const int G = a.Hq / a.Hkv;
     const int len = min(a.lens[q], a.Lmax);
-    if (lane == 0 && split == 0) (void)LSA_IN_BOUNDS(a.lens[q] >= 0 && a.lens[q] <= a.Lmax, BOUNDS_LIST);
+    if (lane == 0 && split == 0 && (!PH || (a.phase_g == 0 && a.phase_r == 0)))
+        (void)LSA_IN_BOUNDS(a.lens[q] >= 0 && a.lens[q] <= a.Lmax, BOUNDS_LIST);
     // with a near-set plan the sink prefix and window suffix were done densely
-    const int2 plan = a.near_plan ? a.near_plan[q] : make_int2(0, 0);
+    const int2 plan = (!PH && a.near_plan) ? a.near_plan[q] : make_int2(0, 0);
     const int lend = max(plan.x, len - plan.y);
-    const int begin = plan.x + split * keys_per_split;
-    const int end = min(lend, begin + keys_per_split);
+    int begin, end;
+    bool last = true;  // this warp writes the query's output
+    if (PH) {
+        const int32_t *ro = a.range_off + q * (int64_t)(a.n_ranges + 1) + a.phase_r;
+        begin = ro[0];
+        end = min(ro[1], len);
+        last = (begin < end && end == len) || (len <= 0 && a.phase_r == 0);
+        if (begin >= end && !last) return;  // nothing of this query in the range
+    } else {
+        begin = plan.x + split * keys_per_split;
+        end = min(lend, begin + keys_per_split);
+    }
     const int nch = end > begin ? (end - begin + KCH - 1) / KCH : 0;
+    uint64_t pol_kv = 0, pol_q = 0;
+    if (PH) {
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol_kv));
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol_q));
+    }
     const uint32_t sbase = smem_u32(asmem + warp * WARP_BYTES);
     const int32_t *lst = a.lists + q * (int64_t)a.Lmax;
 
@@ -195,8 +252,13 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
             const int64_t off = ((int64_t)(idx < 0 ? 0 : idx) * a.Hkv + g) * LSA_HEAD + seg * 8;
             const int bytes = idx < 0 ? 0 : 16;
             const uint32_t so = tile_off(row, seg);
-            cp_async16(sK + so, a.K + off, bytes);
-            cp_async16(sV + so, a.V + off, bytes);
+            if (PH) {
+                cp_async16_hint(sK + so, a.K + off, bytes, pol_kv);
+                cp_async16_hint(sV + so, a.V + off, bytes, pol_kv);
+            } else {
+                cp_async16(sK + so, a.K + off, bytes);
+                cp_async16(sV + so, a.V + off, bytes);
+            }
         }
         cp_commit();
     };
@@ -213,12 +275,32 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = NEG, l[nt][0] = l[nt][1] = 0.0f;
     const float sl2 = a.scale * LOG2E;
-
 #pragma unroll
     for (int s = 0; s < NST - 1; ++s) {
         if (s < nch) load(s, s);
         else cp_commit();
     }
+    if (PH) {  // the running result of the earlier ranges, if any (read while the first rows are in flight)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int h = nt * 8 + 2 * c + e;
+                if (h >= G) continue;
+                const int64_t row = (q * a.Hq) + (int64_t)g * G + h;
+                const float2 ml = ld_f2_hint(a.state_ml + row * 2, pol_q);
+                if (ml.x == NEG) continue;
+                m[nt][e] = ml.x;
+                l[nt][e] = ml.y;
+                const float *so = a.state_o + row * LSA_HEAD;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[nt][mt][e] = ld_f_hint(so + mt * 16 + r0, pol_q);
+                    o[nt][mt][2 + e] = ld_f_hint(so + mt * 16 + 8 + r0, pol_q);
+                }
+            }
+    }
+
     for (int ch = 0; ch < nch; ++ch) {
         const int nxt = ch + NST - 1;
         if (nxt < nch) load(nxt, nxt % NST);
@@ -307,7 +389,23 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     }
     cp_wait<0>();
 
-    if (a.nsplit == 1) {
+    if (PH && !last) {  // the running result goes back for the next range
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int h = nt * 8 + 2 * c + e;
+                if (h >= G) continue;
+                const int64_t row = (q * a.Hq) + (int64_t)g * G + h;
+                float *so = a.state_o + row * LSA_HEAD;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    st_f_hint(so + mt * 16 + r0, o[nt][mt][e], pol_q);
+                    st_f_hint(so + mt * 16 + 8 + r0, o[nt][mt][2 + e], pol_q);
+                }
+                if (r0 == 0) st_f2_hint(a.state_ml + row * 2, make_float2(m[nt][e], l[nt][e]), pol_q);
+            }
+    } else if (a.nsplit == 1) {
         if (plan.x | plan.y) {  // merge the near-set partial results
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -699,14 +797,75 @@ int attention_list_cap()
     return 1 << 30;  // the list is streamed, not staged: any length
 }
 
+// Plan of the phased gather: per query, the index of its first list entry at
+// or past each range start (a lower bound in the ascending list; the last
+// bound is the list length), and its running results set to "nothing yet".
+// One warp per query, one lane per range bound.
+__global__ void __launch_bounds__(256) k_range_plan(AttnArgs a)
+{
+    pdl_wait();
+    pdl_release();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t q = (int64_t)blockIdx.x * 8 + warp;
+    if (q >= a.nq) return;
+    const int len = max(0, min(a.lens[q], a.Lmax));
+    const int32_t *lst = a.lists + q * (int64_t)a.Lmax;
+    int32_t *ro = a.range_off + q * (int64_t)(a.n_ranges + 1);
+    for (int r = lane; r <= a.n_ranges; r += 32) {
+        int lo = len;
+        if (r < a.n_ranges) {
+            const int64_t b = (int64_t)r * a.range_rows;
+            int hi = len;
+            lo = 0;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if ((int64_t)lst[mid] < b) lo = mid + 1;
+                else hi = mid;
+            }
+        }
+        ro[r] = lo;
+    }
+    float2 *ml = reinterpret_cast<float2 *>(a.state_ml) + q * a.Hq;
+    for (int h = lane; h < a.Hq; h += 32) ml[h] = make_float2(__int_as_float(0xff800000), 0.0f);
+}
+
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
 {
     (void)n_sm;
     if (a.nq <= 0) return cudaSuccess;
     const int smem = AWARPS * WARP_BYTES;
     const int G = a.Hq / a.Hkv;
-    auto kern = G <= 8 ? k_attn<1> : k_attn<2>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e;
+    if (a.state_o) {  // position-range phases: one launch per (KV head, range)
+        auto kph = G <= 8 ? k_attn<1, true> : k_attn<2, true>;
+        if ((e = cudaFuncSetAttribute(kph, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+            return e;
+        int kt = kt_begin("k_range_plan", st);
+        k_range_plan<<<(unsigned)((a.nq + 7) / 8), 256, 0, st>>>(a);
+        kt_end(kt, st);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        kt = kt_begin("k_attn", st);
+        AttnArgs b = a;
+        const unsigned blocks = (unsigned)((a.nq + AWARPS - 1) / AWARPS);
+        for (int g = 0; g < a.Hkv; ++g)
+            for (int r = 0; r < a.n_ranges; ++r) {
+                b.phase_g = g;
+                b.phase_r = r;
+                // each launch waits for the previous one's results (griddepcontrol.wait) but its launch
+                // overlaps the previous one's tail
+                e = launch_k(true, kph, dim3(blocks), dim3(AWARPS * 32), (size_t)smem, st, b, 0);
+                if (e != cudaSuccess) {
+                    kt_end(kt, st);
+                    return e;
+                }
+            }
+        kt_end(kt, st);
+        count_launches(a.Hkv * a.n_ranges);
+        return cudaSuccess;
+    }
+    auto kern = G <= 8 ? k_attn<1, false> : k_attn<2, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int kps = (a.Lmax + a.nsplit - 1) / a.nsplit;
     kps = ((kps + KCH - 1) / KCH) * KCH;

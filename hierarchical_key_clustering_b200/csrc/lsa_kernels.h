@@ -206,6 +206,18 @@ struct AttnArgs {
     int4 *near_tile;  // per tile: {usable, first position, lowest near key, longest sink prefix}
     float *near_o;
     float *near_ml;
+    // position-range phases (nsplit == 1 and no near plan; NULL = off): the
+    // keys are cut into n_ranges ranges of range_rows positions, and one
+    // launch per (KV head phase_g, range phase_r) runs every query's list
+    // entries in that range, carrying a running result per (query, head)
+    // from launch to launch, so that the K/V rows the launch gathers (one
+    // head's rows of one range) stay in L2 while every query reads them
+    int32_t *range_off;  // [nq, n_ranges + 1]: index of the first list entry at or past each range start
+    float *state_o;      // [nq, Hq, 128] unnormalised O, relative to the running max
+    float *state_ml;     // [nq, Hq, 2] running max (log2 units; -inf = nothing yet), running sum
+    int32_t n_ranges;
+    int64_t range_rows;
+    int32_t phase_g, phase_r;
 };
 
 // Queries per near-set tile for G query heads per KV head, 0 = no near path.

@@ -54,24 +54,28 @@ __device__ __forceinline__ int merge_bin_shard(float v, float lo, float scale)
 }
 
 // ---------------------------------------------------------------------------
-// Global top P of the union of the ranks' sets (disjoint bucket ids, exact
-// scores).  One CTA per query stages the union in shared memory; all of it
-// is kept when it fits the expansion's slots, else every bucket from the
-// histogram bin holding the P-th best value up when those fit, else the
-// buckets above the P-th score and, at that score, the ties with the lowest
-// ids up to P.
+// Global top P of the union of the shards' sets (disjoint bucket ids, exact
+// scores).  One CTA per query stages the union in shared memory when it fits
+// (up to cap_smem entries; every access otherwise goes to the exchange
+// blocks in global memory); all of it is kept when it fits the expansion's
+// slots, else every bucket from the histogram bin holding the P-th best
+// value up when those fit, else the buckets above the P-th score and, at
+// that score, the ties with the lowest ids up to P.
 constexpr int SM_THREADS = 512;
+constexpr int SM_MAX_SHARDS = 32;
+constexpr int64_t SM_SMEM_MAX = 200 * 1024;  // staged union, bytes
 
 __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__restrict__ xcnt_all,
                                                             const int2 *__restrict__ xent_all, int n_shards,
-                                                            int64_t nq, int64_t xstride, int slots, int P, IndexWs m)
+                                                            int64_t nq, int64_t xstride, int slots, int P,
+                                                            int cap_smem, IndexWs m)
 {
     pdl_wait();
     pdl_release();
-    extern __shared__ uint2 um[];  // [n_shards * slots] (ordered score, bucket id)
+    extern __shared__ uint2 um[];  // [cap_smem] (ordered score, bucket id)
     __shared__ int hist[256];
     __shared__ int sh[4];
-    __shared__ int s_off[LSA_MAXHEADS + 1];
+    __shared__ int s_off[SM_MAX_SHARDS + 1];
     __shared__ int s_out, s_bstar, s_keep;
     __shared__ uint32_t s_vmin, s_vmax;
     const int64_t q = blockIdx.x;
@@ -89,20 +93,26 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
     }
     __syncthreads();
     const int n = s_off[n_shards];
-    for (int i = t; i < n; i += SM_THREADS) {
+    const bool staged = n <= cap_smem;  // block-uniform
+    auto from_global = [&](int i) {
         int s = 0;
         while (i >= s_off[s + 1]) ++s;
         const int2 e = *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(xent_all) + s * xstride +
                                                        (q * slots + (i - s_off[s])) * 8);
-        um[i] = make_uint2(f2ord(__int_as_float(e.x)), (uint32_t)e.y);
+        return make_uint2(f2ord(__int_as_float(e.x)), (uint32_t)e.y);
+    };
+    auto entry = [&](int i) { return staged ? um[i] : from_global(i); };
+    if (staged) {
+        for (int i = t; i < n; i += SM_THREADS) um[i] = from_global(i);
+        __syncthreads();
     }
-    __syncthreads();
     float4 *o4 = reinterpret_cast<float4 *>(m.cand4) + q * KC;
     int32_t *og = m.cand_g + q * KC;
     if (n <= KC) {  // everything fits: the expansion ranks it
         for (int i = t; i < n; i += SM_THREADS) {
-            o4[i] = make_float4(ord2f(um[i].x), NEG, NEG, NEG);
-            og[i] = (int32_t)um[i].y;
+            const uint2 u = entry(i);
+            o4[i] = make_float4(ord2f(u.x), NEG, NEG, NEG);
+            og[i] = (int32_t)u.y;
         }
         if (t == 0) s_out = n;
     } else {
@@ -111,8 +121,9 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
         // is kept when it fits the expansion's slots
         uint32_t vmin = ~0u, vmax = 0u;
         for (int i = t; i < n; i += SM_THREADS) {
-            vmin = min(vmin, um[i].x);
-            vmax = max(vmax, um[i].x);
+            const uint32_t v = entry(i).x;
+            vmin = min(vmin, v);
+            vmax = max(vmax, v);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
         const float scale = hi > lo ? 256.0f / (hi - lo) : 0.0f;
         const int n_round = (n + SM_THREADS - 1) / SM_THREADS * SM_THREADS;
         for (int i = t; i < n_round; i += SM_THREADS) {
-            const int bin = i < n ? merge_bin_shard(ord2f(um[i].x), lo, scale) : -1;
+            const int bin = i < n ? merge_bin_shard(ord2f(entry(i).x), lo, scale) : -1;
             const unsigned peers = __match_any_sync(LSA_FULL, bin);
             if (bin >= 0 && (t & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
         }
@@ -149,7 +160,7 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
         if (s_keep <= KC) {  // block-uniform
             const int bstar = s_bstar;
             for (int i = t; i < n; i += SM_THREADS) {
-                const uint2 u = um[i];
+                const uint2 u = entry(i);
                 if (merge_bin_shard(ord2f(u.x), lo, scale) >= bstar) {
                     const int j = atomicAdd(&s_out, 1);
                     o4[j] = make_float4(ord2f(u.x), NEG, NEG, NEG);
@@ -164,11 +175,12 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
             }
             return;
         }
-        const uint32_t cut = block_select_ord(n, P, [&](int64_t i) { return um[i].x; }, hist, sh);
+        const uint32_t cut = block_select_ord(n, P, [&](int64_t i) { return entry((int)i).x; }, hist, sh);
         int above = 0, ties = 0;
         for (int i = t; i < n; i += SM_THREADS) {
-            above += um[i].x > cut;
-            ties += um[i].x == cut;
+            const uint32_t v = entry(i).x;
+            above += v > cut;
+            ties += v == cut;
         }
         __syncthreads();
         if (t == 0) sh[2] = 0, sh[3] = 0;
@@ -182,10 +194,13 @@ __global__ void __launch_bounds__(SM_THREADS) k_shard_merge(const int32_t *__res
         if (n_above + n_ties > KC) {
             const int need = P - n_above;
             // the need-th smallest id among the ties = the need-th largest of ~id
-            idcut = ~block_select_ord(n, need, [&](int64_t i) { return um[i].x == cut ? ~um[i].y : 0u; }, hist, sh);
+            idcut = ~block_select_ord(n, need, [&](int64_t i) {
+                const uint2 u = entry((int)i);
+                return u.x == cut ? ~u.y : 0u;
+            }, hist, sh);
         }
         for (int i = t; i < n; i += SM_THREADS) {
-            const uint2 u = um[i];
+            const uint2 u = entry(i);
             if (u.x > cut || (u.x == cut && u.y <= idcut)) {
                 const int j = atomicAdd(&s_out, 1);
                 o4[j] = make_float4(ord2f(u.x), NEG, NEG, NEG);
@@ -209,10 +224,13 @@ cudaError_t launch_shard_merge(const void *xchg_all, int n_shards, int64_t nq, i
     const int64_t xstride = cnt_bytes + nq * slots * 8;  // one rank's exchange block
     const int32_t *xcnt = reinterpret_cast<const int32_t *>(xchg_all);
     const int2 *xent = reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(xchg_all) + cnt_bytes);
-    const size_t smem = (size_t)n_shards * slots * 8;
+    // the union staged in shared memory when it fits (each shard lists about
+    // 1.1 P of its slots), else read from the exchange blocks
+    const int cap_smem = (int)min((int64_t)n_shards * slots, (int64_t)(SM_SMEM_MAX / 8));
+    const size_t smem = (size_t)cap_smem * 8;
     cudaFuncSetAttribute(k_shard_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int kt = kt_begin("k_shard_merge", st);
-    k_shard_merge<<<(unsigned)nq, SM_THREADS, smem, st>>>(xcnt, xent, n_shards, nq, xstride, slots, P, m);
+    k_shard_merge<<<(unsigned)nq, SM_THREADS, smem, st>>>(xcnt, xent, n_shards, nq, xstride, slots, P, cap_smem, m);
     kt_end(kt, st);
     count_launches(1);
     return cudaGetLastError();

@@ -47,8 +47,8 @@ class SparseLayer:
         self.Hq = Hq
         nblk = capacity // 512
         self.ws_index = lsa.workspace(lsa.lsa_index_workspace_bytes(max_queries, nblk, self.p), device)
-        self.ws_attn = lsa.workspace(lsa.lsa_attention_workspace_bytes(max_queries, Hq, head_dim, self.Lmax),
-                                     device)
+        self.ws_attn = lsa.workspace(lsa.lsa_attention_workspace_bytes(max_queries, Hq, head_dim, self.Lmax,
+                                                                       capacity), device)
         self.lists = torch.empty((max_queries, self.Lmax), dtype=torch.int32, device=device)
         self.lens = torch.empty((max_queries,), dtype=torch.int32, device=device)
         self._h2d = self._d2h = None  # copy streams of prefill_from_host
@@ -95,7 +95,7 @@ class SparseLayer:
                                  stream=stream)
         return O
 
-    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int = 16,
+    def prefill_from_host(self, h_keys, h_qidx, h_pos, h_Q, h_K, h_V, h_O, lse=None, chunks: int | None = None,
                           kv_cache=None, kv_first: int = 0):
         """One prefill step whose inputs and output live in pinned host memory.
 
@@ -114,6 +114,11 @@ class SparseLayer:
         those of build + index + attend on device copies of the inputs, up to
         the attention's summation order when a chunk holds so few (query, KV
         head) units that the attention splits lists over warps.
+
+        chunks (None: automatic) -- 16, or 2 when the attention takes its keys
+        in position ranges (long contexts, see lsa_sparse_attention): every
+        range's rows are then reused by all queries of a call, so fewer and
+        larger calls pay more than finer copy overlap.
 
         kv_cache=(K, V): device tensors [Tk, Hkv, 128] that already hold the
         K/V rows of positions < kv_first (the KV cache of the earlier
@@ -139,6 +144,11 @@ class SparseLayer:
             d_K, d_V = self._dbuf[5:]
             kv_first = 0
         tk = d_K.shape[0]
+        if chunks is None:
+            hq = h_Q.shape[1]
+            ranged = (lsa.lsa_attention_workspace_bytes(nq, hq, 128, self.Lmax, tk) >
+                      lsa.lsa_attention_workspace_bytes(nq, hq, 128, self.Lmax, 0))
+            chunks = 2 if ranged else 16
         bounds, need = chunk_plan(h_pos, chunks, h_K.shape[1], tk)
         self._h2d.wait_stream(cs)
         with torch.cuda.stream(self._h2d):

@@ -57,7 +57,7 @@ class lsa_tree(C.Structure):
 
 
 EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_check_device_errors",
-           "lsa_debug_wait_test", "lsa_kernel_timing", "lsa_kernel_timing_read", "lsa_list_budget", "lsa_top_buckets",
+           "lsa_debug_wait_test", "lsa_debug_attention_ranges", "lsa_kernel_timing", "lsa_kernel_timing_read", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
            "lsa_shrink", "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
@@ -98,6 +98,7 @@ def lib():
             "lsa_launch_count": (i64, []),
             "lsa_check_device_errors": (C.c_int, []),
             "lsa_debug_wait_test": (None, [i32]),
+            "lsa_debug_attention_ranges": (None, [i64]),
             "lsa_kernel_timing": (None, [i32]),
             "lsa_kernel_timing_read": (C.c_int, [C.c_char_p, i32, C.POINTER(C.c_double), C.POINTER(i64), i32]),
             "lsa_list_budget": (i32, [pp]),
@@ -107,7 +108,7 @@ def lib():
             "lsa_tree_bytes": (i64, [i64]),
             "lsa_tree_bind": (C.c_int, [P, i64, i64, pt]),
             "lsa_index_workspace_bytes": (i64, [i64, i64, pp]),
-            "lsa_attention_workspace_bytes": (i64, [i64, i32, i32, i32]),
+            "lsa_attention_workspace_bytes": (i64, [i64, i32, i32, i32, i64]),
             "lsa_build_cache": (C.c_int, [P, i64, i64, pc, pp, P]),
             "lsa_shrink": (C.c_int, [P, i64, P, i64, i64, P, P, P]),
             "lsa_build_tree": (C.c_int, [pc, pt, pp, P]),
@@ -204,6 +205,12 @@ def lsa_debug_wait_test(enable: bool):
     lib().lsa_debug_wait_test(1 if enable else 0)
 
 
+def lsa_debug_attention_ranges(range_rows: int):
+    """Test hook: force the attention's position-range phases with ranges of
+    range_rows positions (0: automatic)."""
+    lib().lsa_debug_attention_ranges(int(range_rows))
+
+
 def lsa_list_budget(p: lsa_params) -> int:
     return lib().lsa_list_budget(C.byref(p))
 
@@ -216,8 +223,10 @@ def lsa_index_workspace_bytes(nq: int, n_blocks: int, p: lsa_params) -> int:
     return lib().lsa_index_workspace_bytes(nq, n_blocks, C.byref(p))
 
 
-def lsa_attention_workspace_bytes(nq: int, Hq: int, head_dim: int, Lmax: int) -> int:
-    return lib().lsa_attention_workspace_bytes(nq, Hq, head_dim, Lmax)
+def lsa_attention_workspace_bytes(nq: int, Hq: int, head_dim: int, Lmax: int, Tk: int = 0) -> int:
+    """Workspace of lsa_sparse_attention for nq queries over Tk keys (Tk = 0:
+    without the position-range phases)."""
+    return lib().lsa_attention_workspace_bytes(nq, Hq, head_dim, Lmax, Tk)
 
 
 # ---------------------------------------------------------------- buffers

@@ -177,6 +177,13 @@ int64_t lsa_launch_count(void);
 int lsa_check_device_errors(void);
 void lsa_debug_wait_test(int32_t enable);
 
+/* Test hook of lsa_sparse_attention: range_rows > 0 makes every batch with a
+ * large enough workspace (sized after the hook is set) take the
+ * position-range phases with ranges of range_rows positions, so that small
+ * inputs exercise that path; range_rows < 0 turns the phases off; 0
+ * restores the automatic choice. */
+void lsa_debug_attention_ranges(int64_t range_rows);
+
 /* Per-kernel timing, a profiling aid.  While enabled (lsa_kernel_timing(1)),
  * every kernel the library launches is bracketed by two CUDA events recorded
  * on the stream it is launched on, tagged with the kernel's name (the
@@ -210,9 +217,10 @@ int64_t lsa_tree_bytes(int64_t n_blocks);
 int lsa_tree_bind(void *base, int64_t bytes, int64_t n_blocks, lsa_tree *out);
 
 /* Workspace of lsa_index_prefill / lsa_index_decode for nq queries against a
- * cache of n_blocks blocks, and of lsa_sparse_attention. */
+ * cache of n_blocks blocks, and of lsa_sparse_attention for nq queries over
+ * Tk keys (Tk = 0: size without the position-range phases). */
 int64_t lsa_index_workspace_bytes(int64_t nq, int64_t n_blocks, const lsa_params *p);
-int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, int32_t Lmax);
+int64_t lsa_attention_workspace_bytes(int64_t nq, int32_t Hq, int32_t head_dim, int32_t Lmax, int64_t Tk);
 
 /* ---- the five calls of the hot path ---- */
 
@@ -311,15 +319,20 @@ int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const ls
  * O[i,h] = sum_j softmax_j(scale * Q[i,h] . K[j]) V[j] over j in list(i),
  * fp32 softmax and accumulation; O bf16 [nq, Hq, 128]; lse fp32 [nq, Hq]
  * (natural-log log-sum-exp of the scaled scores; may be NULL).
- * ws: >= lsa_attention_workspace_bytes(nq, Hq, 128, Lmax) bytes.  It holds
- * the partial results when few queries split their lists over many warps
- * (decode), or, for batches of at least 64 queries whose KV head fits in
- * three quarters of L2 (Tk x 512 B), the near-set results of tiles of
+ * ws: >= lsa_attention_workspace_bytes(nq, Hq, 128, Lmax, Tk) bytes.  It
+ * holds the partial results when few queries split their lists over many
+ * warps (decode), or, for batches of at least 64 queries whose KV head fits
+ * in three quarters of L2 (Tk x 512 B), the near-set results of tiles of
  * consecutive queries: the run of consecutive positions that ends a list and
  * the run 0, 1, .. that starts it are read once per tile and merged with the
- * rest of each list by log-sum-exp.  With a smaller workspace (or none) fewer
- * splits, or no tiles, are used; results are the same up to fp32 summation
- * order. */
+ * rest of each list by log-sum-exp.  For batches of at least 512 queries
+ * whose KV head does not fit in L2, and lists long enough for at least 256
+ * entries per range (Lmax >= 256 x ranges), it holds one running result per
+ * (query, head) and the keys are taken in position ranges of about half of
+ * L2 per head, one kernel launch per (KV head, range), so that the rows of a
+ * range stay in L2 while every query reads them.  With a smaller workspace (or
+ * none) fewer splits, no tiles or no ranges are used; results are the same
+ * up to fp32 summation order. */
 int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t nq,
                          int32_t Hq, int32_t Hkv, int32_t head_dim, int64_t Tk, const int32_t *lists,
                          const int32_t *lens, int32_t Lmax, float scale, uint16_t *O, float *lse,
@@ -396,9 +409,11 @@ int64_t lsa_shard_merge_workspace_bytes(int64_t nq, const lsa_params *p);
 int lsa_index_shard_local(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cache *cache, int64_t b_first,
                           void *xchg, const lsa_params *p, void *ws, int64_t ws_bytes, void *stream);
 
-/* The global lists from n_shards exchange blocks stored back to back in rank
- * order (xchg_all): per query the union's top P by (score desc, bucket id
- * asc), expanded as lsa_index_prefill does, over the replicated member table
+/* The global lists from n_shards (1..32) exchange blocks stored back to back
+ * (xchg_all; one per shard, in any order -- a rank holding several chunks of
+ * the context gives one block per chunk): per query the union's top P by
+ * (score desc, bucket id asc), expanded as lsa_index_prefill does, over the
+ * replicated member table
  * and counts of all n_blocks blocks (members [n_blocks*64, 16] global
  * positions, 16-byte aligned, count [n_blocks*64]; see
  * lsa_shard_publish_members).  Lists as lsa_index_prefill.

@@ -78,6 +78,48 @@ def test_shard_ranges_cover_every_block_once():
             assert t0 == 512 * b0
 
 
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_zigzag_chunks_cover_every_block_once_and_balance(world):
+    """Zig-zag: 2 x world chunks, rank r holds chunks r and 2 world - 1 - r;
+    together they cover every block once, the tail goes with the last chunk,
+    chunk_order lists each chunk's (rank, part), and for a causal prefill of
+    the last positions every rank's share of the listed positions (each
+    query reads all blocks before it: an early block is read by more
+    queries) is close to the mean."""
+    from hierarchical_key_clustering_b200 import context_parallel as CP
+
+    for T in (4096, 4396, 1 << 20, 10_000_000):
+        nblk = T // 512
+        C = CP.n_chunks(world, "zigzag")
+        blocks, toks = [], []
+        for r in range(world):
+            for c in CP.rank_chunks(r, world, "zigzag"):
+                b0, b1, t0, t1, _ = CP.chunk_range(T, c, C)
+                blocks += list(range(b0, b1))
+                toks.append((c, t0, t1))
+        assert sorted(blocks) == list(range(nblk))
+        toks.sort()
+        assert toks[0][1] == 0 and toks[-1][2] == T
+        assert all(toks[i][2] == toks[i + 1][1] for i in range(len(toks) - 1))
+        order = CP.chunk_order(world, "zigzag")
+        assert [CP.rank_chunks(r, world, "zigzag")[i] for r, i in order] == list(range(C))
+    # attention work per rank of a causal prefill of every position of a 1M context: keys before each query
+    T = 1 << 20
+    for layout, bound in (("zigzag", 1.3), ("contiguous", None)):
+        C = CP.n_chunks(world, layout)
+        work = []
+        for r in range(world):
+            w = 0
+            for c in CP.rank_chunks(r, world, layout):
+                _, _, t0, t1, _ = CP.chunk_range(T, c, C)
+                # sum over queries p of |[t0, t1) n [0, p]| = sum_{t in [t0, t1)} (T - t)
+                w += (t1 - t0) * T - (t1 * (t1 - 1) - t0 * (t0 - 1)) // 2
+            work.append(w)
+        mean = sum(work) / world
+        if bound is not None:
+            assert max(work) <= bound * mean, (layout, world, max(work) / mean)
+
+
 class _FakeShard:
     """A rank's stages with CPU stand-ins that record their inputs."""
 

@@ -44,7 +44,7 @@ def _attention_sampled(lists_d, lens_d, sel, T_kv, hq, hkv, seed):
     V = torch.randn((T_kv, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
     O_ = torch.empty_like(Q)
     lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
-    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, lists_d.shape[1]))
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, lists_d.shape[1], T_kv))
     lsa.lsa_sparse_attention(Q, K, V, lists_d, lens_d, O_, lse, ws=ws)
     torch.cuda.synchronize()
     lists = lists_d[sel].cpu().numpy()
@@ -218,7 +218,8 @@ def test_1m_flat_prefill_and_decode(big1m):
 
 
 def test_1m_context_parallel_eight_ranks(big1m):
-    """The 1M Flat prefill split over 8 token ranges (256 blocks each), the
+    """The 1M Flat prefill split over 8 ranks in the zig-zag layout (16 chunks
+    of 128 blocks, rank r holding chunks r and 15 - r), the
     ranks run stage by stage in this process in the benchmark's chunks of
     16384 queries: lists equal the single-GPU lists of every query (the same
     tensor-core score for every (query, bucket), the same tie order), sampled
@@ -230,9 +231,9 @@ def test_1m_context_parallel_eight_ranks(big1m):
     hq, hkv, chunk, ranks = wl["hq"], wl["hkv"], 16384, 8
     pos = np.arange(T - npre, T, dtype=np.int64)
     q = I.index_queries(0, keys_all, pos)
-    shards = [CP.Shard(r, ranks, T, k=k, max_queries=chunk) for r in range(ranks)]
+    shards = [CP.Shard(r, ranks, T, k=k, max_queries=chunk, layout="zigzag") for r in range(ranks)]
     kd = PT.to_dev(keys_all[:T])
-    built = [s.build(kd[s.t0:s.t1]) for s in shards]
+    built = [s.build(kd) for s in shards]
     M, C = torch.stack([b[0] for b in built]), torch.stack([b[1] for b in built])
     for s in shards:
         s.set_members(M, C)
@@ -253,7 +254,7 @@ def test_1m_context_parallel_eight_ranks(big1m):
         l_, n_ = shards[0].index_merge(X, pd[c0:c1])
         lists[c0:c1].copy_(l_)
         lens[c0:c1].copy_(n_)
-        parts = [s.attend_local(Q[c0:c1], K[s.t0:s.t1], V[s.t0:s.t1], lists[c0:c1], lens[c0:c1]) for s in shards]
+        parts = [s.attend_local(Q[c0:c1], K, V, lists[c0:c1], lens[c0:c1]) for s in shards]
         o, l2 = CP.Shard.combine(torch.stack([x[0] for x in parts]), torch.stack([x[1] for x in parts]))
         O_[c0:c1].copy_(o)
         lse[c0:c1].copy_(l2)
@@ -276,6 +277,43 @@ def test_1m_context_parallel_eight_ranks(big1m):
     bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
     Oref, lse_ref = O.attention(bits(Q[ia]), bits(K.index_select(0, ui)), bits(V.index_select(0, ui)), ll, na)
     PT.assert_attention_close(O_[ia], Oref, lse[ia], lse_ref)
+
+
+def test_1m_context_parallel_merge_past_shared_memory(big1m):
+    """16 ranks in the zig-zag layout (32 chunks of 64 blocks) over the 1M
+    workload: the union of the chunks' candidate sets (~32 x 1.1 P entries)
+    no longer fits the merge kernel's shared memory, so the merge reads it
+    from the exchange blocks; lists equal the single-GPU lists, sampled ones
+    the oracle's."""
+    from hierarchical_key_clustering_b200 import context_parallel as CP
+
+    wl, keys_all, oc, cache, _ = big1m
+    T, k, npre = wl["T"], wl["k"], wl["n_prefill"]
+    ranks, nq = 16, 2048
+    pos = np.arange(T - npre, T, dtype=np.int64)[np.linspace(0, npre - 1, nq).astype(np.int64)]
+    q = I.index_queries(0, keys_all, pos)
+    shards = [CP.Shard(r, ranks, T, k=k, max_queries=nq, layout="zigzag") for r in range(ranks)]
+    kd = PT.to_dev(keys_all[:T])
+    built = [s.build(kd) for s in shards]
+    M, C = torch.stack([b[0] for b in built]), torch.stack([b[1] for b in built])
+    for s in shards:
+        s.set_members(M, C)
+    del kd
+    qd, pd = PT.to_dev(q), PT.to_dev(pos)
+    X = torch.stack([s.index_local(qd, pd) for s in shards]).reshape(-1)
+    cnt = lsa.lsa_shard_exchange_bytes(nq, shards[0].p)
+    slots = lsa.lsa_shard_slots(shards[0].p)
+    counts = torch.stack([X[i * cnt:i * cnt + nq * 4].view(torch.int32).clamp(max=slots)
+                          for i in range(2 * ranks)]).sum(0)
+    assert int(counts.min()) * 8 > 200 * 1024  # every query's union is read from global memory
+    lists, lens = shards[0].index_merge(X, pd)
+    single_l, single_n = _gpu_index(cache, None, lsa.lsa_default_params(k=k), q, pos)
+    same = (lens == single_n) & torch.all(lists == single_l, dim=1)
+    assert same.float().mean().item() >= 0.999, f"only {same.float().mean().item():.4f} equal the single-GPU lists"
+    sel = np.linspace(0, nq - 1, 64).astype(np.int64)
+    ix = torch.from_numpy(sel).cuda()
+    ol, on = O.index(q[sel], pos[sel], oc, k=k)
+    PT.assert_lists_match(lists[ix].cpu().numpy(), lens[ix].cpu().numpy(), ol, on, q[sel], pos[sel], oc, k=k)
 
 
 def test_1m_tree_prefill_and_decode(big1m):

@@ -318,6 +318,50 @@ def test_attention_peaked_softmax(tiny, nq, consecutive):
     assert np.abs(Odrop[:, 0] - Oref[:, 0]).max(axis=1).min() > PT.ATT_MAX
 
 
+@pytest.mark.parametrize("rows,hq,hkv,consecutive", [(300, 32, 8, False), (1000, 8, 1, True), (4096, 32, 8, False),
+                                                    (97, 16, 16, False), (513, 32, 8, True)])
+def test_attention_position_ranges_against_oracle(tiny, rows, hq, hkv, consecutive):
+    """The gather taken in position ranges (one launch per KV head and range,
+    a running result per (query, head) carried between launches), forced on
+    the small workload with ranges of `rows` positions: ragged last ranges,
+    queries with nothing in some ranges, an empty list and a one-key list,
+    against the oracle (output and lse)."""
+    _need_gpu()
+    keys, q, pos, oc = tiny
+    nq = max(300, -(-2048 // hkv))  # enough (query, KV head) units to keep whole lists (no key splits)
+    if consecutive:
+        sel = np.arange(4096 - nq, 4096, dtype=np.int64)
+    else:
+        sel = np.sort(np.random.default_rng(rows).choice(4096, size=nq, replace=False)).astype(np.int64)
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    ol[5] = -1
+    on[5] = 0  # an empty list
+    ol[6, 1:] = -1
+    on[6] = 1  # one key
+    Qb, Kb, Vb = I.qkv_bf16_bits(rows, nq, 4096, hq, hkv)
+    Oref, lse_ref = O.attention(Qb, Kb, Vb, ol, on)
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    lsa.lsa_debug_attention_ranges(rows)
+    try:
+        ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, ol.shape[1], 4096))
+        lsa.lsa_kernel_timing(True)
+        lsa.lsa_sparse_attention(Qd, Kd, Vd, PT.to_dev(ol), PT.to_dev(on), Od, lse, ws=ws)
+        torch.cuda.synchronize()
+        lsa.lsa_kernel_timing(False)
+        kt = lsa.lsa_kernel_timing_read()
+    finally:
+        lsa.lsa_debug_attention_ranges(0)
+    assert "k_range_plan" in kt and kt["k_attn"][1] == 1  # the phased path ran (one timed record)
+    og = Od.float().cpu().numpy()
+    assert np.all(og[5] == 0) and np.all(np.isneginf(lse.cpu().numpy()[5]))
+    keep = np.ones(nq, bool)
+    keep[5] = False
+    PT.assert_attention_close(Od[torch.from_numpy(np.nonzero(keep)[0]).cuda()], Oref[keep],
+                              lse[torch.from_numpy(np.nonzero(keep)[0]).cuda()], lse_ref[keep])
+
+
 @pytest.mark.parametrize("hq,hkv,nq", [(8, 1, 300), (32, 8, 200), (32, 8, 1), (8, 1, 2), (16, 16, 50)])
 def test_attention_against_oracle(tiny, hq, hkv, nq):
     """Attention over the oracle's own lists (isolates the kernel); nq = 1-2

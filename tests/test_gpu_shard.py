@@ -17,14 +17,14 @@ from . import parity as PT
 pytestmark = pytest.mark.gpu
 
 
-def _run(keys, qidx, pos, world, k, heads=1, hq=8, hkv=2, seed=3):
+def _run(keys, qidx, pos, world, k, heads=1, hq=8, hkv=2, seed=3, layout="contiguous"):
     if not torch.cuda.is_available():
         pytest.fail("a CUDA GPU is required for the -m gpu tests")
     T = keys.shape[0]
     nq = len(pos)
-    shards = [CP.Shard(r, world, T, k=k, index_heads=heads, max_queries=nq) for r in range(world)]
+    shards = [CP.Shard(r, world, T, k=k, index_heads=heads, max_queries=nq, layout=layout) for r in range(world)]
     kd = PT.to_dev(keys)
-    built = [s.build(kd[s.t0:s.t1]) for s in shards]
+    built = [s.build(kd) for s in shards]
     M = torch.stack([b[0] for b in built])
     C = torch.stack([b[1] for b in built])
     for s in shards:
@@ -38,10 +38,10 @@ def _run(keys, qidx, pos, world, k, heads=1, hq=8, hkv=2, seed=3):
     Qb, Kb, Vb = I.qkv_bf16_bits(seed, nq, T, hq, hkv)
     f = lambda a: PT.bits_to_bf16(a)  # noqa: E731
     Qd, Kd, Vd = f(Qb), f(Kb), f(Vb)
-    parts = [s.attend_local(Qd, Kd[s.t0:s.t1], Vd[s.t0:s.t1], res[0][0], res[0][1]) for s in shards]
+    parts = [s.attend_local(Qd, Kd, Vd, res[0][0], res[0][1]) for s in shards]
     Oc, lse = CP.Shard.combine(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
     torch.cuda.synchronize()
-    return shards, M, lists, lens, (Qb, Kb, Vb), Oc, lse
+    return shards, shards[0].members, lists, lens, (Qb, Kb, Vb), Oc, lse
 
 
 @pytest.fixture(scope="module")
@@ -52,19 +52,22 @@ def tiny():
     return keys, oc
 
 
-@pytest.mark.parametrize("world", [2, 3, 4, 5])
-def test_shards_lists_and_attention_match_unsharded_oracle(tiny, world):
+@pytest.mark.parametrize("world,layout", [(2, "contiguous"), (3, "contiguous"), (4, "contiguous"),
+                                          (5, "contiguous"), (2, "zigzag"), (3, "zigzag"), (4, "zigzag")])
+def test_shards_lists_and_attention_match_unsharded_oracle(tiny, world, layout):
     """2-5 ranks over 8 blocks (3 ranks: 3 + 3 + 2 blocks; 5 ranks: the last
-    holds nothing): member table bit-exact, every rank the same lists, lists
-    as the oracle's unsharded Flat search, combined attention as its
-    unsharded attention."""
+    holds nothing), and the zig-zag layout (rank r holds chunks r and
+    2 world - 1 - r; 4 ranks: 8 one-block chunks; 3 ranks: two chunks
+    empty): member table bit-exact, every rank the same lists, lists as the
+    oracle's unsharded Flat search, combined attention as its unsharded
+    attention."""
     keys, oc = tiny
     pos = np.array([0, 3, 4, 511, 512, 1023, 1024, 1535, 2047, 2048, 3071, 3072, 4095] + list(range(700, 4096, 29)),
                    np.int64)
     q = I.index_queries(4, keys, pos)
-    shards, M, lists, lens, (Qb, Kb, Vb), Oc, lse = _run(keys, q, pos, world, k=256)
+    shards, M, lists, lens, (Qb, Kb, Vb), Oc, lse = _run(keys, q, pos, world, k=256, layout=layout)
     nb = 8 * 64
-    assert np.array_equal(M.reshape(-1, 16)[:nb].cpu().numpy(), oc.members)
+    assert np.array_equal(M[:nb].cpu().numpy(), oc.members)
     for r in range(1, world):
         assert np.array_equal(lists[r], lists[0]) and np.array_equal(lens[r], lens[0])
     ol, on = O.index(q, pos, oc, k=256)
@@ -81,7 +84,7 @@ def test_shards_ragged_tail_heads_and_decode():
     oc = O.build_cache(keys)
     pos = np.array([600, 2000, 4095, 4096, 4200, T - 1] + list(range(900, T, 97)), np.int64)
     q = I.index_queries_heads(6, keys, pos, 2)
-    _, _, lists, lens, (Qb, Kb, Vb), Oc, lse = _run(keys, q, pos, 3, k=200, heads=2)
+    _, _, lists, lens, (Qb, Kb, Vb), Oc, lse = _run(keys, q, pos, 3, k=200, heads=2, layout="zigzag")
     ol, on = O.index_heads(q, pos, oc, k=200)
     PT.assert_lists_match(lists[0], lens[0], ol, on, q, pos, oc, k=200)
     Oref, lse_ref = O.attention(Qb, Kb, Vb, lists[0], lens[0])

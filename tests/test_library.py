@@ -162,6 +162,15 @@ def test_workspace_queries():
     near = lambda nq, hq: sum(-(-x // 256) * 256 for x in (nq * hq * 128 * 4, nq * hq * 2 * 4, nq * 8, nq * 16))
     assert lsa.lsa_attention_workspace_bytes(131072, 32, 128, 2565) == near(131072, 32)
     assert lsa.lsa_attention_workspace_bytes(1, 32, 128, 4613) > 0        # decode: split the list
+    # position-range phases (no GPU here: L2 taken as 126 MiB, ranges of 129024 positions): at 1M keys, 9
+    # ranges and 4613-entry lists (>= 256 per range) add the range bounds and one fp32 running result per
+    # (query, head); at 10M keys (78 ranges) the lists are too short per range and nothing is added
+    a256 = lambda x: -(-x // 256) * 256  # noqa: E731
+    phase = a256(32768 * 10 * 4) + a256(32768 * 32 * 128 * 4) + a256(32768 * 32 * 2 * 4)
+    assert lsa.lsa_attention_workspace_bytes(32768, 32, 128, 4613, 1 << 20) == max(phase, near(32768, 32))
+    assert lsa.lsa_attention_workspace_bytes(65536, 32, 128, 4613, 10_000_000) == near(65536, 32)
+    assert lsa.lsa_attention_workspace_bytes(32768, 32, 128, 4613, 0) == near(32768, 32)
+    assert lsa.lsa_attention_workspace_bytes(32768, 32, 128, 4613, -1) == -1
     # index heads: the per-row arrays scale with heads, plus one merged set per query
     p4 = lsa.lsa_default_params(k=2048, index_heads=4)
     assert lsa.lsa_index_workspace_bytes(1000, 256, p4) > lsa.lsa_index_workspace_bytes(4000, 256, p)
@@ -206,7 +215,7 @@ def test_shard_sizes_and_argument_errors():
     _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), -1, FAKE, C.byref(p), FAKE, big, None), -2)
     _expect(L.lsa_index_shard_local(FAKE, FAKE, 10, C.byref(cache), 0, FAKE, C.byref(p), None, 0, None), -5)
     # merge: rank count, Tree mode, list budget, workspace
-    for n_shards in (0, 17):
+    for n_shards in (0, 33):
         _expect(L.lsa_index_shard_merge(FAKE, n_shards, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(p), FAKE,
                                         big, None), -1)
     _expect(L.lsa_index_shard_merge(FAKE, 2, FAKE, 10, FAKE, FAKE, 8, FAKE, FAKE, Lmax, C.byref(tp), FAKE, big,
