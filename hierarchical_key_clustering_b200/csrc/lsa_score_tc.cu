@@ -446,28 +446,13 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
         return cudaErrorInvalidValue;
     const int64_t qpairs = (a.nq + QT * TQ - 1) / (QT * TQ);
     const int64_t tiles = (a.nb_total + TB - 1) / TB;
-    // One CTA per SM (shared memory).  A CTA covers a pair of query tiles
-    // over its whole bucket range (no atomics, threshold set in place) unless
-    // splitting the range into `chunks` parts evens out the waves: the time
-    // goes as ceil(qpairs x chunks / SMs) / chunks (e.g. 256 pairs on 148 SMs:
-    // 2 waves of whole ranges, or 7 waves of quarter ranges = 1.75); chunks
-    // of at least 16 tiles, the fewest chunks within 2 % of the best.
+    // One CTA per pair of query tiles over its whole bucket range when that
+    // fills most SMs (no atomics, threshold set in place); otherwise split the
+    // range so that about four waves of CTAs balance the SMs.  (Splitting to
+    // even out the waves of 256 pairs on 148 SMs measured slower: the filter
+    // pass then counts every row's entries with global atomics.)
     int64_t chunks = 1;
-    {
-        const int64_t cmax = min((int64_t)16, max((int64_t)1, (tiles + 15) / 16));
-        auto waves = [&](int64_t c) { return (double)((qpairs * c + n_sm - 1) / n_sm) / (double)c; };
-        double best = 1e30;
-        for (int64_t c = 1; c <= cmax; ++c) best = fmin(best, waves(c));
-        for (int64_t c = 1; c <= cmax; ++c)
-            if (waves(c) <= best * 1.02) {
-                chunks = c;
-                break;
-            }
-    }
-    if (qpairs * 4 < (int64_t)n_sm * 3) {  // very few query pairs: about four waves of range pieces
-        const int64_t c4 = (4LL * n_sm + qpairs - 1) / qpairs;
-        if (c4 > chunks) chunks = c4;
-    }
+    if (qpairs * 4 < (int64_t)n_sm * 3) chunks = (4LL * n_sm + qpairs - 1) / qpairs;
     if (chunks > tiles) chunks = tiles;
     if (chunks < 1) chunks = 1;
     if (chunks > 65535) chunks = 65535;
