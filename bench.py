@@ -47,10 +47,12 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per row gathered by
 # the attention's gather kernel -- a (query, KV head, listed key) the kernel
-# reads -- from one ncu capture of that kernel per workload, divided by the
-# launch's gathered rows.  None: not captured for the kernel as it stands.
-# Keyed by workload name; re-measure whenever k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = {}
+# reads -- from one ncu capture of that kernel's launch in the timed step,
+# divided by the launch's gathered rows (profiles/launches_flat_tree_10m.md:
+# 1.0889e12 B over 65536 x 4613 x 8 rows).  Keyed by (workload, mode); a
+# workload or mode without a capture of the kernel as it stands reports
+# traffic null.  Re-measure whenever k_attn changes.
+ATTN_DRAM_BYTES_PER_ROW = {("flat_tree_10m", "flat"): 450.2}
 
 
 def peaks():
@@ -223,7 +225,8 @@ def _rl(kernel, bound, work, ms, launches, peak, unit, note, **extra):
     return out
 
 
-def kernel_rooflines(kt: dict, wl: dict, pos_np, lens_np, far_rows: int, near_ms_total: float, pk, steps: int):
+def kernel_rooflines(kt: dict, wl: dict, mode: str, pos_np, lens_np, far_rows: int, near_ms_total: float, pk,
+                     steps: int):
     """Per-kernel rooflines of one mode's timed steps from the library's
     per-kernel events (kt: name -> (ms summed over the steps, launches))."""
     T, hq, hkv = wl["T"], wl["hq"], wl["hkv"]
@@ -258,7 +261,7 @@ def kernel_rooflines(kt: dict, wl: dict, pos_np, lens_np, far_rows: int, near_ms
         o["gathered_gbs"] = round(gathered / (ms / n / 1e3) / 1e9, 1)
         o["gathered_note"] = ("512 B of K + V per (query, KV head, gathered key), served from L2 or HBM: a "
                               "throughput, not a fraction of the HBM peak")
-        per_row = ATTN_DRAM_BYTES_PER_ROW.get(wl["name"])
+        per_row = ATTN_DRAM_BYTES_PER_ROW.get((wl["name"], mode))
         if per_row is not None:
             traffic = per_row * hkv * far_rows
             o["traffic"] = int(traffic)
@@ -340,7 +343,7 @@ def mode_summary(args, wl, mode, layer, per, kt, world, pk):
     else:
         far_rows = int(lens_np.astype(np.int64).sum())
     pos_np = np.arange(wl["T"] - nq, wl["T"], dtype=np.int64)
-    kr = kernel_rooflines(kt, wl, pos_np, lens_np, far_rows, near_ms, pk, args.steps)
+    kr = kernel_rooflines(kt, wl, mode, pos_np, lens_np, far_rows, near_ms, pk, args.steps)
     return {
         "mode": mode, "value": round(world * nq * args.steps / (total_ms / 1e3), 1), "unit": UNIT,
         "ms_per_step": round(total_ms / args.steps, 3),
