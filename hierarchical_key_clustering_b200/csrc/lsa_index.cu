@@ -528,7 +528,8 @@ __global__ void __launch_bounds__(TEAM >= 8 ? 32 * TEAM : 256, MINB)
 // Block-wide inclusive scan of a[0..n) in shared memory.  Warp w scans the
 // contiguous segment [w * seg, (w + 1) * seg) 32 elements at a time, lane i
 // on element i (no bank conflicts), carrying the running total; then the
-// segment totals are added in.  Any block size up to 1024 threads.
+// segment totals are added in (each warp sums the totals of the warps before
+// it with one shuffle reduction).  Any block size up to 1024 threads.
 template <typename T>
 __device__ void block_inclusive_scan(T *a, int n, T *wsum)
 {
@@ -549,8 +550,9 @@ __device__ void block_inclusive_scan(T *a, int n, T *wsum)
     }
     if (lane == 0) wsum[w] = carry;
     __syncthreads();
-    T before = 0;
-    for (int k = 0; k < w; ++k) before += wsum[k];
+    T before = lane < w ? wsum[lane] : T(0);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) before += __shfl_xor_sync(LSA_FULL, before, o);
     if (before != T(0))
         for (int i = lo + lane; i < hi; i += 32) a[i] += before;
     __syncthreads();

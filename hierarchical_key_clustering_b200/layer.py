@@ -33,6 +33,18 @@ def chunk_plan(pos, chunks: int, n_kv_heads: int, tk: int):
     return bounds, need
 
 
+def key_chunks(T: int, pieces: int = 8):
+    """[(a, b)] cutting positions 0..T into about `pieces` ranges at block
+    (512-key) boundaries, the last one ending at T: building the cache range
+    by range gives the same cache as one build (items and blocks are pooled
+    and clustered on their own), so each range can be built as soon as its
+    keys are on the device."""
+    nblk = T // 512
+    cuts = sorted({min(nblk, (nblk * i) // pieces) * 512 for i in range(1, pieces)} - {0})
+    edges = [0] + [c for c in cuts if 0 < c < T] + [T]
+    return [(a, b) for a, b in zip(edges, edges[1:]) if b > a]
+
+
 class SparseLayer:
     def __init__(self, capacity: int, k: int = 4096, mode: str = "flat", beam: int = 32, sink: int = 4,
                  window: int = 512, max_queries: int = 1, Hq: int = 32, head_dim: int = 128,
@@ -100,8 +112,9 @@ class SparseLayer:
         """One prefill step whose inputs and output live in pinned host memory.
 
         Three streams overlap the transfers with the kernels.  The index
-        keys go first and the cache build starts as soon as they land, while
-        the index queries follow for the index.  Q then arrives in query
+        keys go first, in whole-block pieces, and each piece is pooled and
+        clustered as soon as it lands, while the index queries follow for the
+        index.  Q then arrives in query
         chunks (multiples of 128 queries, so the near-set tiles of the
         attention do not change), each preceded by
         the K and V rows its queries can list (positions up to the chunk's
@@ -150,11 +163,14 @@ class SparseLayer:
                       lsa.lsa_attention_workspace_bytes(nq, hq, 128, self.Lmax, 0))
             chunks = 2 if ranged else 16
         bounds, need = chunk_plan(h_pos, chunks, h_K.shape[1], tk)
+        kb = key_chunks(h_keys.shape[0])
         self._h2d.wait_stream(cs)
         with torch.cuda.stream(self._h2d):
-            d_keys.copy_(h_keys, non_blocking=True)  # the build needs only the keys
-            e_keys = torch.cuda.Event()
-            e_keys.record()
+            e_keys = []  # the keys in whole-block pieces: each piece is pooled and clustered once it lands
+            for a, b in kb:
+                d_keys[a:b].copy_(h_keys[a:b], non_blocking=True)
+                e_keys.append(torch.cuda.Event())
+                e_keys[-1].record()
             d_q.copy_(h_qidx, non_blocking=True)
             d_pos.copy_(h_pos, non_blocking=True)
             e_idx = torch.cuda.Event()
@@ -173,8 +189,11 @@ class SparseLayer:
                 d_V[have:].copy_(h_V[have - kv_first:], non_blocking=True)
             e_all = torch.cuda.Event()
             e_all.record()
-        cs.wait_event(e_keys)
-        self.build(d_keys, stream=cs)
+        for (a, b), ek in zip(kb, e_keys):
+            cs.wait_event(ek)
+            lsa.lsa_build_cache(d_keys, a, b, self.cache, self.p, cs)
+        if self.tree is not None:
+            lsa.lsa_build_tree(self.cache, self.tree, self.p, cs)
         cs.wait_event(e_idx)
         self.index(d_q, d_pos, stream=cs)
         e_o = []

@@ -260,3 +260,16 @@ def test_prefill_chunk_plan(nq, chunks, hkv, T):
         assert all((c1 - c0) * hkv >= 2048 for c0, c1 in tail[:-1])
     assert need == [min(T, int(pos[c1 - 1]) + 1) for c0, c1 in bounds]
     assert all(a <= b for a, b in zip(need, need[1:]))
+
+
+@pytest.mark.parametrize("T", [100, 512, 4096, 4396, 131072, 1 << 20, 10_000_000])
+def test_key_chunks_cover_the_keys_at_block_boundaries(T):
+    """The pieces prefill_from_host copies and builds the cache from: they
+    cover 0..T in order, every cut on a 512-key block boundary (so a block is
+    always clustered from one piece), at most 8 of them."""
+    from hierarchical_key_clustering_b200.layer import key_chunks
+
+    k = key_chunks(T)
+    assert k[0][0] == 0 and k[-1][1] == T and len(k) <= 8
+    assert all(a[1] == b[0] for a, b in zip(k, k[1:]))
+    assert all(a % 512 == 0 and b > a for a, b in k)
