@@ -472,56 +472,80 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
 }
 
 // Merge the partial results of the key splits of one (query, head): one
-// 512-thread CTA.  The split weights 2^(m_s - M) are computed once in shared
-// memory; then 4 groups of 128 threads (one per output dim) each sum a
-// quarter of the splits and the groups are added.
+// 128-thread CTA.  Each thread loads the (max, sum) records of its splits
+// t, t + 128, .. at once; the split weights 2^(m_s - M) go to shared memory;
+// then warp w sums the splits w, w + 4, .. of the unnormalised outputs, lane
+// i owning dims 4i .. 4i + 3 (16-byte loads, several in flight), and warp 0
+// adds the four parts.
 constexpr int MAX_SPLIT = 1024;
-__global__ void __launch_bounds__(512) k_attn_combine(AttnArgs a)
+constexpr int CB_THREADS = 128;
+__global__ void __launch_bounds__(CB_THREADS) k_attn_combine(AttnArgs a)
 {
     pdl_wait();
     pdl_release();
     __shared__ float wts[MAX_SPLIT];
-    __shared__ float red[16];
-    __shared__ float part[3][LSA_HEAD];
+    __shared__ float red[2][CB_THREADS / 32];
+    __shared__ float4 part[CB_THREADS / 32 - 1][32];
     const int64_t unit = blockIdx.x;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const float *ml = a.part_ml + unit * a.nsplit * 2;
-    float M = __int_as_float(0xff800000);
-    for (int s = t; s < a.nsplit; s += blockDim.x)
-        if (ml[2 * s + 1] > 0.0f) M = fmaxf(M, ml[2 * s]);
+    const float NEG = __int_as_float(0xff800000);
+    const float2 *ml = reinterpret_cast<const float2 *>(a.part_ml + unit * a.nsplit * 2);
+    float2 v[MAX_SPLIT / CB_THREADS];
+    float M = NEG;
+#pragma unroll
+    for (int k = 0; k < MAX_SPLIT / CB_THREADS; ++k) {
+        const int s = t + k * CB_THREADS;
+        v[k] = s < a.nsplit ? ml[s] : make_float2(NEG, 0.0f);
+        if (v[k].y > 0.0f) M = fmaxf(M, v[k].x);
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(LSA_FULL, M, o));
-    if (lane == 0) red[warp] = M;
+    if (lane == 0) red[0][warp] = M;
     __syncthreads();
-    M = red[0];
-    for (int w = 1; w < 16; ++w) M = fmaxf(M, red[w]);
-    __syncthreads();
+    M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
     float L = 0.0f;
-    for (int s = t; s < a.nsplit; s += blockDim.x) {
-        const float l = ml[2 * s + 1];
-        const float w = (l > 0.0f) ? exp2f(ml[2 * s] - M) : 0.0f;
-        wts[s] = w;
-        L += l * w;
+#pragma unroll
+    for (int k = 0; k < MAX_SPLIT / CB_THREADS; ++k) {
+        const int s = t + k * CB_THREADS;
+        if (s < a.nsplit) {
+            const float w = (v[k].y > 0.0f) ? exp2f(v[k].x - M) : 0.0f;
+            wts[s] = w;
+            L += v[k].y * w;
+        }
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(LSA_FULL, L, o);
-    if (lane == 0) red[warp] = L;
+    if (lane == 0) red[1][warp] = L;
     __syncthreads();
-    L = 0.0f;
-    for (int w = 0; w < 16; ++w) L += red[w];
-    const int d = t & (LSA_HEAD - 1), grp = t >> 7;
-    const float *po = a.part_o + unit * a.nsplit * LSA_HEAD + d;
-    float acc = 0.0f;
+    L = (red[1][0] + red[1][1]) + (red[1][2] + red[1][3]);
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + unit * a.nsplit * LSA_HEAD) + lane;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll 4
-    for (int s = grp; s < a.nsplit; s += 4) acc += (wts[s] > 0.0f) ? po[(int64_t)s * LSA_HEAD] * wts[s] : 0.0f;
-    if (grp > 0) part[grp - 1][d] = acc;
+    for (int s = warp; s < a.nsplit; s += CB_THREADS / 32) {
+        const float w = wts[s];
+        if (w > 0.0f) {
+            const float4 x = po[(int64_t)s * (LSA_HEAD / 4)];
+            acc.x += x.x * w;
+            acc.y += x.y * w;
+            acc.z += x.z * w;
+            acc.w += x.w * w;
+        }
+    }
+    if (warp > 0) part[warp - 1][lane] = acc;
     __syncthreads();
-    if (grp == 0) {
-        acc += part[0][d] + part[1][d] + part[2][d];
+    if (warp == 0) {
+#pragma unroll
+        for (int g = 0; g < CB_THREADS / 32 - 1; ++g) {
+            const float4 x = part[g][lane];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        __nv_bfloat16 v = __float2bfloat16_rn(acc * inv);
-        a.O[unit * LSA_HEAD + d] = *reinterpret_cast<uint16_t *>(&v);
-        if (d == 0 && a.lse) a.lse[unit] = M * LN2 + logf(L);
+        const uint32_t lo = pack_bf16(acc.x * inv, acc.y * inv), hi = pack_bf16(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2 *>(a.O + unit * LSA_HEAD + lane * 4) = make_uint2(lo, hi);
+        if (lane == 0 && a.lse) a.lse[unit] = M * LN2 + logf(L);
     }
 }
 
@@ -894,7 +918,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     count_launches(1);
     if (a.nsplit > 1) {
         kt = kt_begin("k_attn_combine", st);
-        e = launch_k(true, k_attn_combine, dim3((unsigned)(a.nq * a.Hq)), dim3(512), 0, st, a);
+        e = launch_k(true, k_attn_combine, dim3((unsigned)(a.nq * a.Hq)), dim3(CB_THREADS), 0, st, a);
         kt_end(kt, st);
         count_launches(1);
     }

@@ -845,17 +845,25 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
         const float tau = ws.tau[q];
         const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + q * ws.cap;
         const int32_t *cg = ws.cand_g + q * ws.cap;
+        // each thread's next entry is loaded before this one's shuffles and
+        // shared-memory atomic, so the loads of consecutive rounds overlap
+        float4 nx4 = make_float4(NEG, NEG, NEG, NEG);
+        int32_t nxg = 0;
+        if (t < ne) {
+            nx4 = c4[t];
+            nxg = cg[t];
+        }
         for (int i0 = 0; i0 < ne; i0 += blockDim.x) {  // block-uniform trip count
-            const int i = i0 + t;
-            float sv[4] = {NEG, NEG, NEG, NEG};
-            int32_t g = 0;
-            if (i < ne) {
-                const float4 s4 = c4[i];
-                g = cg[i];
-                sv[0] = s4.x;
-                sv[1] = s4.y;
-                sv[2] = s4.z;
-                sv[3] = s4.w;
+            float sv[4] = {nx4.x, nx4.y, nx4.z, nx4.w};
+            const int32_t g = nxg;
+            {
+                const int in = i0 + (int)blockDim.x + t;
+                nx4 = make_float4(NEG, NEG, NEG, NEG);
+                nxg = 0;
+                if (in < ne) {
+                    nx4 = c4[in];
+                    nxg = cg[in];
+                }
             }
             int nc = 0;
 #pragma unroll
@@ -925,12 +933,16 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     //    a bucket of any other block weighs its member count.
     int my_tot = 0;
     unsigned long long my_lo = ~0ull, my_hi = 0ull;
+    // the next candidate's member count is loaded before this one is used
+    int nx_cnt = t < n ? __ldg(count + rank_key_id(keys[t])) : 0;
     for (int i = t; i < n; i += blockDim.x) {
         const int32_t b = rank_key_id(keys[i]);
         const int64_t blo = (int64_t)(b / LSA_NBKT) * LSA_BLK;
+        const int cnt_b = nx_cnt;
+        if (i + (int)blockDim.x < n) nx_cnt = __ldg(count + rank_key_id(keys[i + blockDim.x]));
         int nn = 0;
         if (blo >= s_end && blo + LSA_BLK <= w0) {
-            nn = __ldg(count + b);
+            nn = cnt_b;
         } else {
             const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
 #pragma unroll
@@ -1039,20 +1051,54 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
         const int nb = min(RX_SLOTS, nslots - b0);
         for (int i = t; i < nb * RX_MW; i += blockDim.x) masks[i] = 0u;
         __syncthreads();
-        for (int i = t; i < n; i += blockDim.x) {
-            if (!(any && wt[i] > 0 && keys[i] <= cut)) continue;
+        // the member row of this thread's next marked candidate is loaded
+        // before the current one's atomics
+        auto marked = [&](int i) { return i < n && any && wt[i] > 0 && keys[i] <= cut; };
+        auto row_of = [&](int i) {
+            return reinterpret_cast<const int4 *>(members + (int64_t)rank_key_id(keys[i]) * LSA_NSLOT);
+        };
+        int nxi = t;
+        while (nxi < n && !marked(nxi)) nxi += blockDim.x;
+        int4 nxm[4];
+        if (nxi < n) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) nxm[v] = __ldg(row_of(nxi) + v);
+        }
+        while (nxi < n) {
+            const int i = nxi;
+            int4 mrow[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) mrow[v] = nxm[v];
+            nxi = i + blockDim.x;
+            while (nxi < n && !marked(nxi)) nxi += blockDim.x;
+            if (nxi < n) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) nxm[v] = __ldg(row_of(nxi) + v);
+            }
             const int32_t b = rank_key_id(keys[i]);
             const int blk = b / LSA_NBKT;
             const uint32_t word = touched[blk >> 5];
             const int slot = wrank[blk >> 5] - __popc(word) + __popc(word & ((1u << (blk & 31)) - 1u)) - b0;
             if (slot < 0 || slot >= nb) continue;
             slot_blk[slot] = blk;
+            const int64_t blo = (int64_t)blk * LSA_BLK;
+            if (keys[i] != cut && blo >= s_end && blo + LSA_BLK <= w0) {
+                // a bucket taken whole in a block clear of sink and window: its
+                // members are whole pooled items (slots 4v .. 4v + 3 hold the 4
+                // consecutive positions of item v), marked 4 bits at a time
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    int m = mrow[v].x;
+                    if (m >= 0 && !LSA_IN_BOUNDS(m < N * (LSA_BLK / LSA_NBKT), BOUNDS_BUCKET)) m = -1;
+                    if (m >= 0) atomicOr(&masks[mword(slot, (m & 511) >> 5)], 0xFu << (m & 31));
+                }
+                continue;
+            }
             const int limit = (keys[i] == cut) ? take : 16;
-            const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
             int idx = 0;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-                const int4 w = __ldg(m4 + v);
+                const int4 w = mrow[v];
                 const int mm[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
