@@ -537,16 +537,26 @@ __device__ void block_inclusive_scan(T *a, int n, T *wsum)
     const int seg = (((n + nw - 1) / nw) + 31) & ~31;
     const int lo = min(n, w * seg), hi = min(n, lo + seg);
     T carry = 0;
-    for (int base = lo; base < hi; base += 32) {  // warp-uniform
-        const int i = base + lane;
-        T x = i < hi ? a[i] : T(0);
+    for (int base = lo; base < hi; base += 128) {  // warp-uniform; 4 independent 32-element scans per round
+        T x[4];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const T y = __shfl_up_sync(LSA_FULL, x, o);
-            if (lane >= o) x += y;
+        for (int k = 0; k < 4; ++k) {
+            const int i = base + 32 * k + lane;
+            x[k] = i < hi ? a[i] : T(0);
         }
-        if (i < hi) a[i] = x + carry;
-        carry += __shfl_sync(LSA_FULL, x, 31);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const T y = __shfl_up_sync(LSA_FULL, x[k], o);
+                if (lane >= o) x[k] += y;
+            }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = base + 32 * k + lane;
+            if (i < hi) a[i] = x[k] + carry;
+            carry += __shfl_sync(LSA_FULL, x[k], 31);
+        }
     }
     if (lane == 0) wsum[w] = carry;
     __syncthreads();
@@ -1129,8 +1139,19 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
             for (int w = 0; w < 16; ++w) {
                 uint32_t bits = masks[mword(sl, w)];
                 while (bits) {
-                    dst[o++] = base + 32 * w + __ffs(bits) - 1;
-                    bits &= bits - 1;
+                    const int b = __ffs(bits) - 1;
+                    const int32_t pos0 = base + 32 * w + b;
+                    if ((b & 3) == 0 && ((bits >> b) & 0xFu) == 0xFu) {  // a whole item: 4 positions at once
+                        dst[o] = pos0;
+                        dst[o + 1] = pos0 + 1;
+                        dst[o + 2] = pos0 + 2;
+                        dst[o + 3] = pos0 + 3;
+                        o += 4;
+                        bits &= ~(0xFu << b);
+                    } else {
+                        dst[o++] = pos0;
+                        bits &= bits - 1;
+                    }
                 }
             }
         }
