@@ -237,15 +237,15 @@ def kernel_rooflines(kt: dict, wl: dict, mode: str, pos_np, lens_np, far_rows: i
         ms, n = kt["k_pool_norm"]
         out["k_pool_norm"] = _rl("k_pool_norm", "hbm", 320.0 * T * steps, ms, n, pk["hbm"], "GB/s",
                                  "320 B per key: 256 B of fp32 key read, 64 B of pooled item written")
-    s_ms = sum(kt[k][0] for k in ("k_score_tc:threshold", "k_score_tc:filter") if k in kt)
+    passes = ("k_score_tc:sampled", "k_score_tc:threshold", "k_score_tc:filter")
+    s_ms = sum(kt[k][0] for k in passes if k in kt)
     if s_ms > 0:
         flop = 128.0 * float(H.sum()) * 64 * steps
         n = kt.get("k_score_tc:filter", (0, steps))[1]
         out["k_score_tc"] = _rl("k_score_tc", "tensor", flop, s_ms, n, pk["bf16_sust"], "TFLOP/s",
-                                "128 flop per (query, visible bucket), one pass; time = both passes (threshold + "
-                                "filter); peak = sustained bf16 (timed inside a long step)",
-                                passes_ms={k: round(kt[k][0] / max(1, kt[k][1]), 4)
-                                           for k in ("k_score_tc:threshold", "k_score_tc:filter") if k in kt})
+                                "128 flop per (query, visible bucket), one pass; time = both passes (threshold, "
+                                "sampled or full, + filter); peak = sustained bf16 (timed inside a long step)",
+                                passes_ms={k: round(kt[k][0] / max(1, kt[k][1]), 4) for k in passes if k in kt})
     if "k_rank_expand" in kt:
         ms, n = kt["k_rank_expand"]
         out["k_rank_expand"] = _rl("k_rank_expand", "hbm", 4.0 * float(lens_np.sum()) * steps, ms, n, pk["hbm"],

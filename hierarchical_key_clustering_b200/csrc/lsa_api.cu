@@ -197,13 +197,19 @@ IndexLayout index_layout(int64_t nq, int64_t nblk, const lsa_params *p, bool sha
     return L;
 }
 
-// Key splits per query: about 2048 warps in flight for small batches (one
-// warp per (query, KV head, split)), at least 32 keys per split.
 // Bounded device-side waits: tries per wait, and the test hook that makes one
 // wait run out (lsa_debug_wait_test).
 uint32_t g_wait_limit = 1u << 20;
 uint32_t g_extra_tx = 0;
+// Sampled threshold pass of Flat search (lsa_debug_score_sample): every 16th
+// centroid tile, tau set so that about 0.9 P buckets lie above it, for
+// queries that see at least 16 x 128 x 32 buckets.
+int32_t g_sample = 16;
+float g_sample_margin = 0.9f;
+constexpr int64_t SAMPLE_MIN_TILES = 32;
 
+// Key splits per query for small batches (one warp per (query, KV head,
+// split)), at least 32 keys per split.
 int attention_nsplit(int64_t nq, int32_t Hkv, int32_t Lmax)
 {
     // few queries: split each list so that about 512 warps run (measured at
@@ -374,6 +380,9 @@ int index_impl(const float *qidx, const int64_t *pos, int64_t nq, const lsa_cach
     a.wait_limit = g_wait_limit;
     a.extra_tx = g_extra_tx;
     g_extra_tx = 0;
+    a.sample = g_sample;
+    a.sample_margin = g_sample_margin;
+    a.sample_min_n = (int64_t)(g_sample > 1 ? g_sample : 1) * 128 * SAMPLE_MIN_TILES;
     lsa::TreeView tv;
     const lsa::TreeView *tvp = nullptr;
     if (p->mode == LSA_MODE_TREE && cache->n_blocks > 0) {
@@ -511,6 +520,12 @@ int lsa_kernel_timing_read(char *names, int32_t name_len, double *ms, int64_t *l
     n = (int)seen.size();
     if (err != cudaSuccess) return cuda_fail(err, "kernel timing events");
     return n;
+}
+
+void lsa_debug_score_sample(int32_t stride, float margin)
+{
+    g_sample = stride;
+    g_sample_margin = margin > 0.0f ? margin : 0.9f;
 }
 
 void lsa_debug_attention_ranges(int64_t range_rows)

@@ -39,8 +39,8 @@ namespace lsa {
 constexpr int KCH = 16;                          // keys per chunk
 constexpr int ROWB = 128;                        // bf16 per smem row (256 B, 16-byte segments XOR-swizzled)
 constexpr int NST = 2;                           // pipeline stages (2 x 8 KB per warp: 3 CTAs of 4 warps per SM)
+constexpr int NST_SPLIT = 4;                     // stages of split lists (few warps: one CTA per SM, deeper rings)
 constexpr int STAGE_BYTES = 2 * KCH * ROWB * 2;  // K + V
-constexpr int WARP_BYTES = NST * STAGE_BYTES;
 constexpr int AWARPS = 4;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -167,11 +167,9 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x)
 // back.  K/V rows are fetched with an L2 evict-last policy and the
 // per-query data with evict-first, so the range's rows stay in L2 while
 // every query reads them.
-template <int NT, bool PH>
+template <int NT, bool PH, int NS>
 __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_split)
 {
-    pdl_wait();
-    pdl_release();
     extern __shared__ __align__(128) uint8_t asmem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t unit = (int64_t)blockIdx.x * AWARPS + warp;
@@ -184,6 +182,23 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     const int g = PH ? a.phase_g : (int)(qg / a.nq);
     const int64_t q = PH ? unit : qg % a.nq;
     const int G = a.Hq / a.Hkv;
+    const int r0 = lane >> 2, c = lane & 3;
+    // B operand Q^T: dims 2c, 2c + 1 (and + 8) of dim block kk, head 8 nt + r0.
+    // Q is not written by the kernels this one waits for (the index lists),
+    // so it is loaded before the wait.
+    const uint16_t *Qb = a.Q + ((q * a.Hq) + (int64_t)g * G) * LSA_HEAD;
+    uint32_t qb[NT][8][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = nt * 8 + r0;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            qb[nt][kk][0] = h < G ? ld_u32(Qb + h * LSA_HEAD + kk * 16 + 2 * c) : 0u;
+            qb[nt][kk][1] = h < G ? ld_u32(Qb + h * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
+        }
+    }
+    pdl_wait();
+    pdl_release();
     const int len = min(a.lens[q], a.Lmax);
     if (lane == 0 && split == 0 && (!PH || (a.phase_g == 0 && a.phase_r == 0)))
         (void)LSA_IN_BOUNDS(a.lens[q] >= 0 && a.lens[q] <= a.Lmax, BOUNDS_LIST);
@@ -208,24 +223,9 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
         asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol_kv));
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol_q));
     }
-    const uint32_t sbase = smem_u32(asmem + warp * WARP_BYTES);
+    const uint32_t sbase = smem_u32(asmem + warp * NS * STAGE_BYTES);
     const int32_t *lst = a.lists + q * (int64_t)a.Lmax;
 
-    const int r0 = lane >> 2, c = lane & 3;
-    const uint16_t *Qb = a.Q + ((q * a.Hq) + (int64_t)g * G) * LSA_HEAD;
-    // B operand Q^T: dims 2c, 2c + 1 (and + 8) of dim block kk, head 8 nt + r0
-    uint32_t qb[NT][8][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int h = nt * 8 + r0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            qb[nt][kk][0] = h < G ? ld_u32(Qb + h * LSA_HEAD + kk * 16 + 2 * c) : 0u;
-            qb[nt][kk][1] = h < G ? ld_u32(Qb + h * LSA_HEAD + kk * 16 + 8 + 2 * c) : 0u;
-        }
-    }
-
-    int pre = -1;  // index of lane's row in the chunk issued next
     auto fetch_idx = [&](int ch) {
         const int base = begin + ch * KCH;
         int v = -1;
@@ -237,10 +237,16 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
         }
         return v;
     };
-    pre = fetch_idx(0);
+    // lane's list entry in each of the next NS - 1 chunks to issue: the
+    // entries of a chunk are loaded NS - 1 issues ahead of its rows
+    int pre[NS - 1];
+#pragma unroll
+    for (int j = 0; j < NS - 1; ++j) pre[j] = fetch_idx(j);
     auto load = [&](int ch, int st) {
-        int my = pre;
-        pre = fetch_idx(ch + 1);
+        int my = pre[0];
+#pragma unroll
+        for (int j = 0; j < NS - 2; ++j) pre[j] = pre[j + 1];
+        pre[NS - 2] = fetch_idx(ch + NS - 1);
         if (my >= a.Tk) my = -1;  // out-of-range entries are read as zeros, never fetched
         const uint32_t sK = sbase + st * STAGE_BYTES;
         const uint32_t sV = sK + KCH * ROWB * 2;
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = NEG, l[nt][0] = l[nt][1] = 0.0f;
     const float sl2 = a.scale * LOG2E;
 #pragma unroll
-    for (int s = 0; s < NST - 1; ++s) {
+    for (int s = 0; s < NS - 1; ++s) {
         if (s < nch) load(s, s);
         else cp_commit();
     }
@@ -302,12 +308,12 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
     }
 
     for (int ch = 0; ch < nch; ++ch) {
-        const int nxt = ch + NST - 1;
-        if (nxt < nch) load(nxt, nxt % NST);
+        const int nxt = ch + NS - 1;
+        if (nxt < nch) load(nxt, nxt % NS);
         else cp_commit();
-        cp_wait<NST - 1>();
+        cp_wait<NS - 1>();
         __syncwarp();
-        const uint32_t sK = sbase + (ch % NST) * STAGE_BYTES;
+        const uint32_t sK = sbase + (ch % NS) * STAGE_BYTES;
         const uint32_t sV = sK + KCH * ROWB * 2;
         float s[NT][4];
 #pragma unroll
@@ -472,75 +478,87 @@ __global__ void __launch_bounds__(AWARPS * 32) k_attn(AttnArgs a, int keys_per_s
 }
 
 // Merge the partial results of the key splits of one (query, head): one
-// 128-thread CTA.  Each thread loads the (max, sum) records of its splits
-// t, t + 128, .. at once; the split weights 2^(m_s - M) go to shared memory;
-// then warp w sums the splits w, w + 4, .. of the unnormalised outputs, lane
-// i owning dims 4i .. 4i + 3 (16-byte loads, several in flight), and warp 0
-// adds the four parts.
-constexpr int MAX_SPLIT = 1024;
-constexpr int CB_THREADS = 128;
+// 256-thread CTA.  Warp w takes the splits w, w + 8, .. in batches of
+// CB_BATCH; lane i loads dims 4i .. 4i + 3 of each of its splits'
+// unnormalised outputs (16-byte loads) and the splits' (max, sum) records
+// before the maximum M over all splits is known, so the partials arrive in
+// one round trip; the weights 2^(m_s - M) then scale them (a split with no
+// key weighs 0), and the warps' sums are added in shared memory.
+constexpr int CB_THREADS = 256;
+constexpr int CB_WARPS = CB_THREADS / 32;
+constexpr int CB_BATCH = 8;
 __global__ void __launch_bounds__(CB_THREADS) k_attn_combine(AttnArgs a)
 {
     pdl_wait();
     pdl_release();
-    __shared__ float wts[MAX_SPLIT];
-    __shared__ float red[2][CB_THREADS / 32];
-    __shared__ float4 part[CB_THREADS / 32 - 1][32];
+    __shared__ float red[2][CB_WARPS];
+    __shared__ float4 part[CB_WARPS][32];
     const int64_t unit = blockIdx.x;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float NEG = __int_as_float(0xff800000);
-    const float2 *ml = reinterpret_cast<const float2 *>(a.part_ml + unit * a.nsplit * 2);
-    float2 v[MAX_SPLIT / CB_THREADS];
-    float M = NEG;
+    const int ns = a.nsplit;
+    const float2 *ml = reinterpret_cast<const float2 *>(a.part_ml + unit * ns * 2);
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + unit * ns * LSA_HEAD) + lane;
+    float4 x[CB_BATCH];
+    float2 r[CB_BATCH];
+    auto fetch = [&](int b0) {
 #pragma unroll
-    for (int k = 0; k < MAX_SPLIT / CB_THREADS; ++k) {
-        const int s = t + k * CB_THREADS;
-        v[k] = s < a.nsplit ? ml[s] : make_float2(NEG, 0.0f);
-        if (v[k].y > 0.0f) M = fmaxf(M, v[k].x);
+        for (int j = 0; j < CB_BATCH; ++j) {
+            const int sp = b0 + warp + j * CB_WARPS;
+            r[j] = sp < ns ? ml[sp] : make_float2(NEG, 0.0f);
+            x[j] = sp < ns ? po[(int64_t)sp * (LSA_HEAD / 4)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+    };
+    fetch(0);
+    float M = NEG;
+    for (int sp = t; sp < ns; sp += CB_THREADS) {
+        const float2 v = ml[sp];
+        if (v.y > 0.0f) M = fmaxf(M, v.x);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(LSA_FULL, M, o));
     if (lane == 0) red[0][warp] = M;
     __syncthreads();
-    M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
-    float L = 0.0f;
+    M = red[0][0];
 #pragma unroll
-    for (int k = 0; k < MAX_SPLIT / CB_THREADS; ++k) {
-        const int s = t + k * CB_THREADS;
-        if (s < a.nsplit) {
-            const float w = (v[k].y > 0.0f) ? exp2f(v[k].x - M) : 0.0f;
-            wts[s] = w;
-            L += v[k].y * w;
-        }
+    for (int w = 1; w < CB_WARPS; ++w) M = fmaxf(M, red[0][w]);
+    float L = 0.0f;
+    for (int sp = t; sp < ns; sp += CB_THREADS) {
+        const float2 v = ml[sp];
+        if (v.y > 0.0f) L += v.y * exp2f(v.x - M);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(LSA_FULL, L, o);
     if (lane == 0) red[1][warp] = L;
-    __syncthreads();
-    L = (red[1][0] + red[1][1]) + (red[1][2] + red[1][3]);
-    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + unit * a.nsplit * LSA_HEAD) + lane;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 4
-    for (int s = warp; s < a.nsplit; s += CB_THREADS / 32) {
-        const float w = wts[s];
-        if (w > 0.0f) {
-            const float4 x = po[(int64_t)s * (LSA_HEAD / 4)];
-            acc.x += x.x * w;
-            acc.y += x.y * w;
-            acc.z += x.z * w;
-            acc.w += x.w * w;
+    for (int b0 = 0;;) {  // warp-uniform
+#pragma unroll
+        for (int j = 0; j < CB_BATCH; ++j) {
+            if (r[j].y > 0.0f) {
+                const float w = exp2f(r[j].x - M);
+                acc.x += x[j].x * w;
+                acc.y += x[j].y * w;
+                acc.z += x[j].z * w;
+                acc.w += x[j].w * w;
+            }
         }
+        b0 += CB_BATCH * CB_WARPS;
+        if (b0 >= ns) break;
+        fetch(b0);
     }
-    if (warp > 0) part[warp - 1][lane] = acc;
+    part[warp][lane] = acc;
     __syncthreads();
     if (warp == 0) {
+        acc = part[0][lane];
+        L = red[1][0];
 #pragma unroll
-        for (int g = 0; g < CB_THREADS / 32 - 1; ++g) {
-            const float4 x = part[g][lane];
-            acc.x += x.x;
-            acc.y += x.y;
-            acc.z += x.z;
-            acc.w += x.w;
+        for (int w = 1; w < CB_WARPS; ++w) {
+            const float4 y = part[w][lane];
+            acc.x += y.x;
+            acc.y += y.y;
+            acc.z += y.z;
+            acc.w += y.w;
+            L += red[1][w];
         }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
         const uint32_t lo = pack_bf16(acc.x * inv, acc.y * inv), hi = pack_bf16(acc.z * inv, acc.w * inv);
@@ -857,11 +875,11 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
 {
     (void)n_sm;
     if (a.nq <= 0) return cudaSuccess;
-    const int smem = AWARPS * WARP_BYTES;
+    const int smem = AWARPS * NST * STAGE_BYTES;
     const int G = a.Hq / a.Hkv;
     cudaError_t e;
     if (a.state_o) {  // position-range phases: one launch per (KV head, range)
-        auto kph = G <= 8 ? k_attn<1, true> : k_attn<2, true>;
+        auto kph = G <= 8 ? k_attn<1, true, NST> : k_attn<2, true, NST>;
         if ((e = cudaFuncSetAttribute(kph, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
             return e;
         int kt = kt_begin("k_range_plan", st);
@@ -888,8 +906,12 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
         count_launches(a.Hkv * a.n_ranges);
         return cudaSuccess;
     }
-    auto kern = G <= 8 ? k_attn<1, false> : k_attn<2, false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // split lists (few queries): few warps, so deeper rings (one CTA per SM)
+    const bool split = a.nsplit > 1;
+    auto kern = split ? (G <= 8 ? k_attn<1, false, NST_SPLIT> : k_attn<2, false, NST_SPLIT>)
+                      : (G <= 8 ? k_attn<1, false, NST> : k_attn<2, false, NST>);
+    const int smem_g = AWARPS * (split ? NST_SPLIT : NST) * STAGE_BYTES;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_g);
     if (e != cudaSuccess) return e;
     int kps = (a.Lmax + a.nsplit - 1) / a.nsplit;
     kps = ((kps + KCH - 1) / KCH) * KCH;
@@ -912,7 +934,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
     const int64_t blocks = (units + AWARPS - 1) / AWARPS;
     // split lists (few queries, decode): short kernels, launched back to back
     int kt = kt_begin("k_attn", st);
-    e = launch_k(a.nsplit > 1, kern, dim3((unsigned)blocks), dim3(AWARPS * 32), (size_t)smem, st, a, kps);
+    e = launch_k(split, kern, dim3((unsigned)blocks), dim3(AWARPS * 32), (size_t)smem_g, st, a, kps);
     kt_end(kt, st);
     if (e != cudaSuccess) return e;
     count_launches(1);

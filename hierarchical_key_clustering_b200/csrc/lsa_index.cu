@@ -640,20 +640,13 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb_total,
                                                           const uint16_t *__restrict__ cbf, int P, IndexWs ws)
 {
-    pdl_wait();
-    pdl_release();
-    __shared__ __align__(16) float qf[SMALL_NQ][LSA_D];
-    __shared__ uint32_t hs[SMALL_NQ][HIST_BINS];
-    extern __shared__ __align__(16) uint8_t ds_dyn[];  // [DS_WARPS][2][32 * DS_ROW] staged rows
+    // dynamic shared memory: [DS_WARPS][2][32 * DS_ROW] staged rows, then the
+    // batch's histograms [nq][HIST_BINS] and queries [nq][LSA_D]
+    extern __shared__ __align__(16) uint8_t ds_dyn[];
+    uint32_t *hs = reinterpret_cast<uint32_t *>(ds_dyn + DS_WARPS * 2 * 32 * DS_ROW);
+    float *qf = reinterpret_cast<float *>(hs + nq * HIST_BINS);
     __shared__ int Nq[SMALL_NQ], gq[SMALL_NQ];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    for (int i = t; i < nq * LSA_D; i += blockDim.x) qf[i / LSA_D][i % LSA_D] = bf_bits2f(ws.qhat[i]);
-    for (int i = t; i < nq * HIST_BINS; i += blockDim.x) hs[i / HIST_BINS][i % HIST_BINS] = 0u;
-    if (t < nq) {
-        const int N = ws.horizon[t] * LSA_NBKT;
-        Nq[t] = N;
-        gq[t] = group_width(N, P);
-    }
     const float NEG = __int_as_float(0xff800000);
     const int64_t wbase = (int64_t)blockIdx.x * DS_SPAN + warp * 128;
     // copy the 32 rows of round r into stage[warp][r & 1]: instruction v moves
@@ -671,18 +664,27 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
     };
+    // the centroid rows are not written by the kernel this one waits for (the
+    // query normalisation), so the first two rounds are in flight before the wait
     issue(0);
+    issue(1);
+    pdl_wait();
+    pdl_release();
+    for (int i = t; i < nq * LSA_D; i += blockDim.x) qf[i] = bf_bits2f(ws.qhat[i]);
+    for (int i = t; i < nq * HIST_BINS; i += blockDim.x) hs[i] = 0u;
+    if (t < nq) {
+        const int N = ws.horizon[t] * LSA_NBKT;
+        Nq[t] = N;
+        gq[t] = group_width(N, P);
+    }
     __syncthreads();
     float run[SMALL_NQ];
 #pragma unroll
     for (int i = 0; i < SMALL_NQ; ++i) run[i] = NEG;
     for (int r = 0; r < 4; ++r) {
-        if (r + 1 < 4) {
-            issue(r + 1);
-            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-        }
+        if (r >= 1 && r + 1 < 4) issue(r + 1);  // rounds 0 and 1 were issued above
+        if (r + 1 < 4) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
         __syncwarp();
         const int64_t b = wbase + r * 32 + lane;
         uint32_t cw[32];
@@ -699,7 +701,7 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
 #pragma unroll
         for (int qi = 0; qi < SMALL_NQ; ++qi) {
             if (qi >= nq) break;  // uniform
-            const float4 *qv = reinterpret_cast<const float4 *>(qf[qi]);
+            const float4 *qv = reinterpret_cast<const float4 *>(qf + qi * LSA_D);
             float acc = 0.0f;
 #pragma unroll
             for (int v = 0; v < 16; ++v) {
@@ -715,7 +717,7 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
             float m = valid ? acc : NEG;
             if (g <= 32) {
                 for (int o = 1; o < g; o <<= 1) m = fmaxf(m, __shfl_xor_sync(LSA_FULL, m, o));
-                if (valid && (lane & (g - 1)) == 0) atomicAdd(&hs[qi][hist_bin(m)], 1u);
+                if (valid && (lane & (g - 1)) == 0) atomicAdd(&hs[qi * HIST_BINS + hist_bin(m)], 1u);
             } else {
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(LSA_FULL, m, o));
@@ -723,7 +725,7 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
                 const int per = g >> 5;  // 2 or 4 rounds per group
                 if ((r & (per - 1)) == per - 1) {
                     const int64_t gstart = wbase + (int64_t)(r - per + 1) * 32;
-                    if (lane == 0 && gstart < Nq[qi]) atomicAdd(&hs[qi][hist_bin(run[qi])], 1u);
+                    if (lane == 0 && gstart < Nq[qi]) atomicAdd(&hs[qi * HIST_BINS + hist_bin(run[qi])], 1u);
                     run[qi] = NEG;
                 }
             }
@@ -731,7 +733,7 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
     }
     __syncthreads();
     for (int i = t; i < nq * HIST_BINS; i += blockDim.x) {
-        const uint32_t c = hs[i / HIST_BINS][i % HIST_BINS];
+        const uint32_t c = hs[i];
         if (c) atomicAdd(ws.ghist + i, c);
     }
 }
@@ -773,26 +775,30 @@ __global__ void __launch_bounds__(256) k_dfilter(int64_t nq, int P, IndexWs ws)
 
 // ---------------------------------------------------------------------------
 // Rank the candidates of one query and expand them into its index list.
-//   1. candidates: every listed score >= tau (a Flat query whose entries or
-//      candidates overflow is redone exactly here: radix select of the P-th
-//      largest score recomputed on the CUDA cores, then every bucket above it
-//      and the lowest-id buckets equal to it, P in all);
-//   2. each candidate's weight: its members outside near;
+//   1. candidates: every listed score >= tau, each with its weight (its
+//      members outside near), in one pass (a Flat query whose entries or
+//      candidates overflow, or whose sampled tau keeps fewer than k far keys,
+//      is redone exactly here: radix select of the P-th largest score
+//      recomputed on the CUDA cores, then every bucket above it and the
+//      lowest-id buckets equal to it, P in all; 2. weighs those);
 //   3. the walk over buckets in (score desc, id asc) order stops at the
 //      bucket where the weights reach k: found by histogramming the weights
-//      over the candidates' rank keys (4096 bins over the remaining key range)
-//      and narrowing to the bin where k is reached until it holds one key --
-//      buckets ranked before it are taken whole, their order does not matter;
+//      over the candidates' rank keys (1024 or 4096 bins over the remaining
+//      key range) and narrowing to the bin where k is reached until it holds
+//      at most 32 keys, which one warp ranks -- buckets ranked before the cut
+//      are taken whole, their order does not matter;
 //   4. the chosen positions are marked in one 512-bit mask per touched block
 //      (blocks found through a bitmap over all visible blocks, RX_SLOTS
 //      blocks at a time) and emitted block by block in ascending order -- the
-//      far keys come out sorted without sorting them;
+//      far keys come out sorted without sorting them; with few queries (1024
+//      threads per query) k_rx_emit does this for all touched blocks at once;
 //   5. sink, far keys and window are written.
 // Every bucket has >= 4 keys and at most sink + window clustered keys are
 // near, so the best P buckets already hold k far keys: the cut never falls
 // outside the top P.
 constexpr int RX_SLOTS = 512;  // touched blocks per emit batch
-constexpr int RX_BINS = 4096;  // bins of the cut search (aliases the masks)
+constexpr int RX_BINS = 4096;  // bins of the cut search at most (aliases the masks)
+constexpr int RX_SPLIT = 2048; // touched blocks handed to k_rx_emit at most (16 B of shared memory each)
 
 constexpr int RX_MW = 16;      // words per touched block's mask row; word w sits at w ^ (slot & 15), so
                                // one thread per slot reading word w hits at most 2-way bank conflicts
@@ -829,7 +835,7 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     __shared__ int hist[256];
     __shared__ int sh[4];
     __shared__ float qf[LSA_D];
-    __shared__ int nk_s, fb_s, tot_s, cnt_s, excl_s;
+    __shared__ int nk_s, fb_s, tot_s, cnt_s, excl_s, ng_s;
     __shared__ unsigned long long lo_s, hi_s, cut_s;
 
     const int64_t q = blockIdx.x;
@@ -850,9 +856,35 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     for (int i = t; i < TW; i += blockDim.x) touched[i] = 0u;
     __syncthreads();
 
-    // 1. candidates
+    const float tau = ws.tau[q];
+    // Weights: only a block that overlaps the sink or the window can hold near
+    // keys; a bucket of any other block weighs its member count.
+    auto clear_of_near = [&](int32_t b) {
+        const int64_t blo = (int64_t)(b / LSA_NBKT) * LSA_BLK;
+        return blo >= s_end && blo + LSA_BLK <= w0;
+    };
+    auto far_members = [&](int32_t b) {  // members of b outside sink and window
+        const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
+        int nn = 0;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int4 w = __ldg(m4 + v);
+            const int mm[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                int64_t m = mm[e];  // -1 pads are skipped
+                if (m >= 0 && !LSA_IN_BOUNDS(m < N * (LSA_BLK / LSA_NBKT), BOUNDS_BUCKET)) m = -1;
+                nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
+            }
+        }
+        return nn;
+    };
+    int n = 0;
+    int my_tot = 0;  // this thread's weights and weighted key range
+    unsigned long long my_lo = ~0ull, my_hi = 0ull;
+    for (;;) {  // at most twice: a sampled threshold that keeps too little is redone exactly
+    // 1. candidates with their weights (2. below for the exact path)
     if (!fb_s) {
-        const float tau = ws.tau[q];
         const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + q * ws.cap;
         const int32_t *cg = ws.cand_g + q * ws.cap;
         // each thread's next entry is loaded before this one's shuffles and
@@ -876,11 +908,14 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                 }
             }
             int nc = 0;
+            int cb[4];  // member counts of kept buckets clear of near, loaded before the slot search
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 if (sv[e] >= tau && sv[e] > NEG && !LSA_IN_BOUNDS(g + e >= 0 && g + e < N, BOUNDS_BUCKET))
                     sv[e] = NEG;  // debug build: a bucket the query cannot see is dropped
-                nc += sv[e] >= tau && sv[e] > NEG;
+                const bool kept = sv[e] >= tau && sv[e] > NEG;
+                nc += kept;
+                cb[e] = kept && clear_of_near(g + e) ? __ldg(count + g + e) : -1;
             }
             // one shared-memory atomic per warp
             int incl = nc;
@@ -895,8 +930,18 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 if (sv[e] >= tau && sv[e] > NEG) {
-                    if (slot < KC) keys[slot] = rank_key(sv[e], g + e);
+                    const int nn = cb[e] >= 0 ? cb[e] : far_members(g + e);
+                    const uint64_t key = rank_key(sv[e], g + e);
+                    if (slot < KC) {
+                        keys[slot] = key;
+                        wt[slot] = (uint8_t)nn;
+                    }
                     ++slot;
+                    my_tot += nn;
+                    if (nn > 0) {
+                        my_lo = min(my_lo, (unsigned long long)key);
+                        my_hi = max(my_hi, (unsigned long long)key);
+                    }
                 }
             }
         }
@@ -936,42 +981,26 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
             __syncthreads();
         }
     }
-    const int n = nk_s;
+    n = nk_s;
 
-    // 2. weights (members outside near) and the key range of weighted candidates.
-    //    Only a block that overlaps the sink or the window can hold near keys;
-    //    a bucket of any other block weighs its member count.
-    int my_tot = 0;
-    unsigned long long my_lo = ~0ull, my_hi = 0ull;
-    // the next candidate's member count is loaded before this one is used
-    int nx_cnt = t < n ? __ldg(count + rank_key_id(keys[t])) : 0;
-    for (int i = t; i < n; i += blockDim.x) {
-        const int32_t b = rank_key_id(keys[i]);
-        const int64_t blo = (int64_t)(b / LSA_NBKT) * LSA_BLK;
-        const int cnt_b = nx_cnt;
-        if (i + (int)blockDim.x < n) nx_cnt = __ldg(count + rank_key_id(keys[i + blockDim.x]));
-        int nn = 0;
-        if (blo >= s_end && blo + LSA_BLK <= w0) {
-            nn = cnt_b;
-        } else {
-            const int4 *m4 = reinterpret_cast<const int4 *>(members + (int64_t)b * LSA_NSLOT);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const int4 w = __ldg(m4 + v);
-                const int mm[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    int64_t m = mm[e];  // -1 pads are skipped
-                    if (m >= 0 && !LSA_IN_BOUNDS(m < N * (LSA_BLK / LSA_NBKT), BOUNDS_BUCKET)) m = -1;
-                    nn += (m >= 0) && !(m < s_end || (m >= w0 && m <= p));
-                }
+    // 2. (exact path) weights of the selected buckets and their key range
+    if (fb_s) {
+        my_tot = 0;  // whatever the candidate pass added before it overflowed
+        my_lo = ~0ull;
+        my_hi = 0ull;
+        // the next candidate's member count is loaded before this one is used
+        int nx_cnt = t < n ? __ldg(count + rank_key_id(keys[t])) : 0;
+        for (int i = t; i < n; i += blockDim.x) {
+            const int32_t b = rank_key_id(keys[i]);
+            const int cnt_b = nx_cnt;
+            if (i + (int)blockDim.x < n) nx_cnt = __ldg(count + rank_key_id(keys[i + blockDim.x]));
+            const int nn = clear_of_near(b) ? cnt_b : far_members(b);
+            wt[i] = (uint8_t)nn;
+            my_tot += nn;
+            if (nn > 0) {
+                my_lo = min(my_lo, (unsigned long long)keys[i]);
+                my_hi = max(my_hi, (unsigned long long)keys[i]);
             }
-        }
-        wt[i] = (uint8_t)nn;
-        my_tot += nn;
-        if (nn > 0) {
-            my_lo = min(my_lo, (unsigned long long)keys[i]);
-            my_hi = max(my_hi, (unsigned long long)keys[i]);
         }
     }
 #pragma unroll
@@ -986,6 +1015,20 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
         atomicMax(&hi_s, my_hi);
     }
     __syncthreads();
+    // An exact tau sits at or below the P-th best score, and the best P
+    // buckets hold k far keys, so fewer than k above it means tau = -inf.
+    // A sampled tau can land above the cut: then the query is redone by the
+    // exact selection (block-uniform: read after the barrier).
+    if (fb_s || tot_s >= k || !(tau > NEG)) break;
+    __syncthreads();
+    if (t == 0) {
+        fb_s = 1;
+        tot_s = 0;
+        lo_s = ~0ull;
+        hi_s = 0ull;
+    }
+    __syncthreads();
+    }
     const int nfar = min(k, tot_s);
 
     // 3. the cut: smallest key K with (weight of keys <= K) >= nfar, and the
@@ -995,10 +1038,13 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     if (nfar > 0) {
         uint64_t lo = lo_s, hi = hi_s;
         int rem = nfar;
+        // 1024 bins for up to 2048 candidates (a cut bin then holds a few keys,
+        // ranked by one warp below), 4096 for more
+        const int nbins = n <= 2048 ? 1024 : RX_BINS, lb = 31 - __clz(nbins);
         for (int round = 0;; ++round) {  // block-uniform
             const uint64_t span = hi - lo;
-            const int shift = (span >> 12) == 0 ? 0 : (64 - __clzll((long long)span)) - 12;
-            for (int i = t; i < RX_BINS; i += blockDim.x) bins[i] = 0u;
+            const int shift = (span >> lb) == 0 ? 0 : (64 - __clzll((long long)span)) - lb;
+            for (int i = t; i < nbins; i += blockDim.x) bins[i] = 0u;
             if (t == 0) cut_s = ~0ull;
             __syncthreads();
             for (int i = t; i < n; i += blockDim.x) {
@@ -1007,8 +1053,8 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                     atomicAdd(&bins[(key - lo) >> shift], (1u << 18) | (uint32_t)wt[i]);
             }
             __syncthreads();
-            block_inclusive_scan(bins, RX_BINS, reinterpret_cast<uint32_t *>(wsum));  // count << 18 | weight
-            for (int c = t; c < RX_BINS; c += blockDim.x) {
+            block_inclusive_scan(bins, nbins, reinterpret_cast<uint32_t *>(wsum));  // count << 18 | weight
+            for (int c = t; c < nbins; c += blockDim.x) {
                 const uint32_t inc = bins[c], exc = c > 0 ? bins[c - 1] : 0u;
                 if ((int)(exc & 0x3ffffu) < rem && rem <= (int)(inc & 0x3ffffu)) {
                     sh[0] = c;
@@ -1029,6 +1075,40 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                 __syncthreads();
                 cut = cut_s;
                 take = rem;
+                break;
+            }
+            if (cnt_s <= 32) {
+                // a few weighted keys left in [blo, bhi]: one warp ranks them
+                // by pairwise comparison, each key's weight before it gives the cut
+                uint64_t *gk = reinterpret_cast<uint64_t *>(bins);  // [32] (the bins are read by now)
+                uint32_t *gw = bins + 64;                            // [32]
+                if (t == 0) ng_s = 0;
+                __syncthreads();
+                for (int i = t; i < n; i += blockDim.x)
+                    if (wt[i] > 0 && keys[i] >= blo && keys[i] <= bhi) {
+                        const int g = atomicAdd(&ng_s, 1);
+                        gk[g] = keys[i];
+                        gw[g] = wt[i];
+                    }
+                __syncthreads();
+                if (warp == 0) {
+                    const int m = ng_s;
+                    const uint64_t mk = lane < m ? gk[lane] : ~0ull;
+                    const int mw = lane < m ? (int)gw[lane] : 0;
+                    int before = 0;
+                    for (int j = 0; j < m; ++j) {
+                        const uint64_t kj = __shfl_sync(LSA_FULL, mk, j);
+                        const int wj = __shfl_sync(LSA_FULL, mw, j);
+                        if (kj < mk) before += wj;
+                    }
+                    if (lane < m && before < rem && rem <= before + mw) {
+                        cut_s = mk;
+                        excl_s = before;
+                    }
+                }
+                __syncthreads();
+                cut = cut_s;
+                take = rem - excl_s;
                 break;
             }
             lo = blo;
@@ -1053,11 +1133,51 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     const int n_sink = (int)min(s_end, w0);
     int32_t *out = lists + q * (int64_t)Lmax;
     int emitted = 0;
+    // Wide blocks (few queries): each touched block's chosen buckets (a 64-bit
+    // mask) and the list offset of its far keys go to the candidate space
+    // (read whole by now), and k_rx_emit emits the blocks in parallel.
+    const bool split = NT >= 1024 && any && nslots <= RX_SPLIT && ws.cap >= 3;
+    if (split) {
+        uint64_t *smask = reinterpret_cast<uint64_t *>(masks);  // [RX_SPLIT]
+        int32_t *scnt = reinterpret_cast<int32_t *>(smask + RX_SPLIT);
+        int32_t *sblk = scnt + RX_SPLIT;
+        for (int i = t; i < nslots; i += blockDim.x) {
+            smask[i] = 0ull;
+            scnt[i] = 0;
+        }
+        __syncthreads();
+        for (int i = t; i < n; i += blockDim.x) {
+            if (wt[i] > 0 && keys[i] <= cut) {
+                const int32_t b = rank_key_id(keys[i]);
+                const int blk = b / LSA_NBKT;
+                const uint32_t word = touched[blk >> 5];
+                const int slot = wrank[blk >> 5] - __popc(word) + __popc(word & ((1u << (blk & 31)) - 1u));
+                atomicOr(reinterpret_cast<unsigned long long *>(smask + slot), 1ull << (b % LSA_NBKT));
+                atomicAdd(scnt + slot, keys[i] == cut ? take : (int)wt[i]);
+                sblk[slot] = blk;  // every writer of a slot writes the same block
+            }
+        }
+        __syncthreads();
+        block_inclusive_scan(scnt, nslots, wsum);
+        int4 *rec = reinterpret_cast<int4 *>(ws.cand4) + q * ws.cap;
+        for (int i = t; i < nslots; i += blockDim.x)
+            rec[i] = make_int4(sblk[i], i > 0 ? scnt[i - 1] : 0, (int)(uint32_t)smask[i],
+                               (int)(uint32_t)(smask[i] >> 32));
+        if (t == 0) {
+            int32_t *hd = ws.cand_g + q * ws.cap;
+            hd[0] = nslots;
+            hd[1] = rank_key_id(cut);
+            hd[2] = take;
+        }
+        emitted = scnt[nslots - 1];
+    } else if (NT >= 1024 && t == 0 && ws.cap >= 1) {
+        ws.cand_g[q * ws.cap] = -1;  // nothing left for k_rx_emit
+    }
     // one batch whose far keys fit in the candidate keys' space (free once the
     // marks are set): stage them there and copy the whole list out coalesced
-    const bool stage = nslots <= RX_SLOTS && nfar <= 2 * KC;
+    const bool stage = !split && nslots <= RX_SLOTS && nfar <= 2 * KC;
     int32_t *stg = reinterpret_cast<int32_t *>(keys);
-    for (int b0 = 0; b0 < nslots; b0 += RX_SLOTS) {
+    for (int b0 = 0; b0 < (split ? 0 : nslots); b0 += RX_SLOTS) {
         const int nb = min(RX_SLOTS, nslots - b0);
         for (int i = t; i < nb * RX_MW; i += blockDim.x) masks[i] = 0u;
         __syncthreads();
@@ -1172,6 +1292,75 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
         else out[i] = -1;
     }
     if (t == 0) lens[q] = len;
+}
+
+// ---------------------------------------------------------------------------
+// The far keys of one query's touched blocks, for the wide (few-query)
+// expansion: one warp per touched block.  Its chosen buckets (a 64-bit mask)
+// are read two at a time, 16 member slots each; far members (not sink, not
+// window) are marked in the warp's 512-bit mask -- of the cut bucket only the
+// first `take` in slot order -- and lane w < 16 writes the positions of word
+// w in ascending order at the block's offset.
+__global__ void __launch_bounds__(256) k_rx_emit(const int64_t *__restrict__ pos,
+                                                 const int32_t *__restrict__ members, int32_t *__restrict__ lists,
+                                                 int Lmax, int sink, int window, IndexWs ws)
+{
+    pdl_wait();
+    pdl_release();
+    __shared__ uint32_t words[8][16];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t q = blockIdx.y;
+    const int32_t *hd = ws.cand_g + q * ws.cap;
+    const int nslots = hd[0];  // -1: the expansion wrote the list itself
+    const int slot = blockIdx.x * 8 + warp;
+    if (slot >= nslots) return;
+    const int32_t cutb = hd[1];
+    const int take = hd[2];
+    const int64_t p = pos[q];
+    const int64_t w0 = p - window > 0 ? p - window : 0;
+    const int64_t s_end = (int64_t)sink < p + 1 ? (int64_t)sink : p + 1;
+    const int n_sink = (int)min(s_end, w0);
+    const int64_t N = (int64_t)ws.horizon[q] * LSA_NBKT;
+    (void)N;  // read by the debug build's bounds checks only
+    const int4 r = reinterpret_cast<const int4 *>(ws.cand4)[q * ws.cap + slot];
+    const int blk = r.x;
+    if (!LSA_IN_BOUNDS(blk >= 0 && (int64_t)blk * LSA_NBKT < N, BOUNDS_BUCKET)) return;
+    uint64_t mm = ((uint64_t)(uint32_t)r.w << 32) | (uint32_t)r.z;
+    if (lane < 16) words[warp][lane] = 0u;
+    __syncwarp();
+    const int half = lane >> 4, li = lane & 15;
+    while (mm) {  // warp-uniform
+        const int j0 = __ffsll((long long)mm) - 1;
+        mm &= mm - 1;
+        const int j1 = mm ? __ffsll((long long)mm) - 1 : -1;
+        if (mm) mm &= mm - 1;
+        const int j = half ? j1 : j0;
+        const int32_t b = blk * LSA_NBKT + j;
+        int m = j >= 0 ? __ldg(members + (int64_t)b * LSA_NSLOT + li) : -1;
+        if (m >= 0 && !LSA_IN_BOUNDS(m < N * (LSA_BLK / LSA_NBKT), BOUNDS_BUCKET)) m = -1;
+        bool far = m >= 0 && !(m < s_end || (m >= w0 && m <= p));
+        const unsigned bal = __ballot_sync(LSA_FULL, far);
+        if (far && b == cutb) far = __popc((bal >> (16 * half)) & ((1u << li) - 1u)) < take;
+        if (far) atomicOr(&words[warp][(m & (LSA_BLK - 1)) >> 5], 1u << (m & 31));
+    }
+    __syncwarp();
+    uint32_t bits = lane < 16 ? words[warp][lane] : 0u;
+    const int c = __popc(bits);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+        const int y = __shfl_up_sync(LSA_FULL, incl, o);
+        if (lane >= o) incl += y;
+    }
+    int o = n_sink + r.y + incl - c;
+    if (!LSA_IN_BOUNDS(o + c <= Lmax, BOUNDS_LIST)) return;
+    int32_t *out = lists + q * (int64_t)Lmax;
+    const int32_t base = blk * LSA_BLK + 32 * lane;
+    while (bits) {
+        const int b = __ffs(bits) - 1;
+        out[o++] = base + b;
+        bits &= bits - 1;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1579,33 +1768,55 @@ __global__ void __launch_bounds__(HM_THREADS) k_heads_exact(int64_t nq, int head
 }
 // Expansion of an already merged candidate set (one-bucket entries, at most
 // m.cap per query, tau = -inf), e.g. the top P of a context-parallel merge.
+static cudaError_t launch_rank_expand(const IndexArgs &a, const IndexWs &ex, int KC, int TW, bool small,
+                                      cudaStream_t st);
+
 cudaError_t launch_expand_merged(const IndexArgs &a, const IndexWs &m, cudaStream_t st)
 {
     if (a.nq <= 0) return cudaSuccess;
     const int TW = (int)((a.n_blocks + 31) / 32) + 1;
-    const int KC = m.cap;
-    const size_t smr = rank_expand_smem(KC, TW);
-    const int kt = kt_begin("k_rank_expand", st);
-    if (a.nq <= SMALL_NQ) {
-        cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        const cudaError_t e = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
-                                       a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
-                                       a.window, a.P, KC, TW, m);
-        kt_end(kt, st);
-        if (e != cudaSuccess) return e;
-    } else {
-        cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists,
-                                                             a.lens, a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, m);
-        kt_end(kt, st);
-    }
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_rank_expand(a, m, m.cap, TW, a.nq <= SMALL_NQ, st);
 }
 
 size_t rank_expand_smem_bytes(int cap, int64_t n_blocks)
 {
     return rank_expand_smem(cap, (int)((n_blocks + 31) / 32) + 1);
+}
+
+// ---------------------------------------------------------------------------
+// Expansion of every query's candidates into its list.  Many queries: one
+// 256-thread CTA per query does everything.  Few: one 1024-thread CTA per
+// query ranks and cuts, and k_rx_emit writes the far keys block by block.
+static cudaError_t launch_rank_expand(const IndexArgs &a, const IndexWs &ex, int KC, int TW, bool small,
+                                      cudaStream_t st)
+{
+    const size_t smr = rank_expand_smem(KC, TW);
+    int kt = kt_begin("k_rank_expand", st);
+    if (small) {
+        cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        cudaError_t e = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
+                                 a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink, a.window,
+                                 a.P, KC, TW, ex);
+        kt_end(kt, st);
+        if (e != cudaSuccess) return e;
+        count_launches(1);
+        if (ex.cap >= 3) {
+            kt = kt_begin("k_rx_emit", st);
+            const unsigned gx = (unsigned)((min(KC, RX_SPLIT) + 7) / 8);
+            e = launch_k(true, k_rx_emit, dim3(gx, (unsigned)a.nq), dim3(256), 0, st, a.pos, a.members, a.lists,
+                         a.Lmax, a.sink, a.window, ex);
+            kt_end(kt, st);
+            if (e != cudaSuccess) return e;
+            count_launches(1);
+        }
+    } else {
+        cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists,
+                                                             a.lens, a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ex);
+        kt_end(kt, st);
+        count_launches(1);
+    }
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -1630,7 +1841,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
     const bool small = a.nq <= SMALL_NQ;
     if (a.mode == 0 && nb_total > 0) {
         if (rows <= SMALL_NQ) {  // stream every centroid once for the whole batch, keep the scores
-            const int dsm = DS_WARPS * 2 * 32 * DS_ROW;
+            const int dsm = DS_WARPS * 2 * 32 * DS_ROW + (int)rows * (HIST_BINS + LSA_D) * 4;
             cudaFuncSetAttribute(k_dscore, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
             int kt = kt_begin("k_dscore", st);
             e = launch_k(true, k_dscore, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
@@ -1653,6 +1864,11 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
             sa.chunk_tiles = 0;
             sa.wait_limit = a.wait_limit;
             sa.extra_tx = a.extra_tx;
+            // sampled threshold: single-head Flat search that expands its own
+            // candidates (the multi-head and shard merges rely on an exact tau)
+            sa.sample = (heads == 1 && !a.no_expand) ? a.sample : 0;
+            sa.sample_margin = a.sample_margin;
+            sa.sample_min_n = a.sample_min_n;
             int whole = 0;
             if ((e = launch_score_tc(sa, ws, a.centroid_bf16, st, n_sm, &whole)) != cudaSuccess) return e;
             if (!whole) {  // thresholds from the merged histograms
@@ -1715,23 +1931,7 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
     // query on the measured workloads; a query with more takes the exact path
     // (a merged set never has more than its slots)
     const int KC = merged ? merged->cap : (int)min((int64_t)ws.cap, pow2_ceil64(((int64_t)a.P * 3 + 1) / 2));
-    const size_t smr = rank_expand_smem(KC, TW);
-    const int kt = kt_begin("k_rank_expand", st);
-    if (small) {  // one CTA per query, few queries: widest blocks
-        cudaFuncSetAttribute(k_rank_expand<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        const cudaError_t el = launch_k(true, k_rank_expand<1024>, dim3((unsigned)a.nq), dim3(1024), smr, st, a.pos,
-                                        a.members, a.count, a.centroid_bf16, a.lists, a.lens, a.Lmax, a.k, a.sink,
-                                        a.window, a.P, KC, TW, ex);
-        kt_end(kt, st);
-        if (el != cudaSuccess) return el;
-    } else {
-        cudaFuncSetAttribute(k_rank_expand<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
-        k_rank_expand<256><<<(unsigned)a.nq, 256, smr, st>>>(a.pos, a.members, a.count, a.centroid_bf16, a.lists, a.lens,
-                                                             a.Lmax, a.k, a.sink, a.window, a.P, KC, TW, ex);
-        kt_end(kt, st);
-    }
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_rank_expand(a, ex, KC, TW, small, st);
 }
 
 // this file's bounds-check word (debug build; always 0 in the release build)

@@ -132,6 +132,9 @@ struct IndexArgs {
     int32_t no_expand;  // stop after the merged candidate set (a shard's local step)
     uint32_t wait_limit;  // tries per bounded device-side wait
     uint32_t extra_tx;    // test hook (see lsa_debug_wait_test)
+    int32_t sample;       // sampled threshold pass (see ScoreTcArgs; <= 1: off)
+    float sample_margin;
+    int64_t sample_min_n;
 };
 
 // Flat scoring on the tensor cores (lsa_score_tc.cu).  mode 0: threshold
@@ -146,6 +149,15 @@ struct ScoreTcArgs {
     int64_t chunk_tiles;
     uint32_t wait_limit;  // tries per bounded mbarrier wait
     uint32_t extra_tx;    // test hook: non-zero skips the query-tile copy, so its barrier never completes
+    // threshold pass (mode 0) from a sample: a CTA whose rows all see at least
+    // sample_min_n buckets, and that covers their whole range, scores only
+    // every sample-th centroid tile and sets tau at the score above which
+    // sample_margin x P x (sampled / visible buckets) of its sampled scores lie
+    // (sample <= 1: off; the expansion redoes a query exactly if its
+    // candidates then hold fewer than k far keys)
+    int32_t sample;
+    float sample_margin;
+    int64_t sample_min_n;
 };
 cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint16_t *centroid_bf16, cudaStream_t st,
                             int n_sm, int *whole_range);

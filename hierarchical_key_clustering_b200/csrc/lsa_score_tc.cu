@@ -42,6 +42,8 @@
 // copies it issued, frees its TMEM and exits.
 #include <cuda.h>
 
+#include <climits>
+
 #include "lsa_common.cuh"
 #include "lsa_kernels.h"
 #include "lsa_tc.cuh"
@@ -61,6 +63,7 @@ constexpr int NST_MAX = 8;
 constexpr uint32_t A_BYTES = QT * TQ * LSA_D * 2;  // 32 KB
 constexpr uint32_t B_BYTES = TB * LSA_D * 2;       // 16 KB
 constexpr int TMEM_COLS = 512;      // [query tile][buffer] x 128 fp32 columns
+constexpr int SAMPLE_G = 8;         // group width of the sampled threshold pass
 constexpr int EPI_WARPS = 8 * QT;   // 16: TMEM lane quadrant x query tile x column half
 constexpr int THREADS = 64 + 32 * EPI_WARPS;  // 576
 constexpr int HSTRIDE = HIST_BINS / 2 + 1;   // 32-bit words per row histogram (2 x u16 bins per word, +1 pad)
@@ -121,6 +124,7 @@ struct TcSmem {
     uint32_t tmem_base;
     int abort;
     int nmax;
+    int nmin;
 };
 
 }  // namespace
@@ -155,6 +159,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (threadIdx.x == 0) {
         cs->nmax = 0;
+        cs->nmin = INT_MAX;
         cs->abort = 0;
         for (int s = 0; s < nst; ++s) {
             mbar_init(smem_u32(&cs->full[s]), 1);
@@ -173,12 +178,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int64_t q = q0 + threadIdx.x;
         const int N = (q < a.nq) ? ws.horizon[q] * LSA_NBKT : 0;
         atomicMax(&cs->nmax, N);
+        if (q < a.nq) atomicMin(&cs->nmin, N);
     }
     __syncthreads();
+    // the sampled threshold pass (block-uniform): every S-th centroid tile,
+    // while a query's sampled groups of 8 stay below 2^16 (the bin counters)
+    const bool sampled = a.mode == 0 && a.sample > 1 && a.whole_range && (int64_t)cs->nmin >= a.sample_min_n &&
+                         (int64_t)cs->nmax <= (int64_t)a.sample * 500000;
+    const int S = sampled ? a.sample : 1;
     const int64_t tiles_all = ((int64_t)cs->nmax + TB - 1) / TB;
     const int64_t j0 = (int64_t)blockIdx.y * a.chunk_tiles;
     const int64_t j1 = min(j0 + a.chunk_tiles, tiles_all);
-    const int ntiles = j1 > j0 ? (int)(j1 - j0) : 0;
+    const int ntiles = j1 > j0 ? (int)((j1 - j0 + S - 1) / S) : 0;
     if (ntiles == 0) return;  // uniform: nothing allocated yet
     // CTAs start their walk at evenly spread tiles of the range (and wrap), so
     // that at any moment they read different centroid tiles instead of all
@@ -186,7 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int rot = (int)(((int64_t)blockIdx.x * ntiles) / gridDim.x);
     auto tile_of = [&](int it) {
         const int r = it + rot;
-        return j0 + (r >= ntiles ? r - ntiles : r);
+        return j0 + (int64_t)(r >= ntiles ? r - ntiles : r) * S;
     };
 
     volatile int *abort = &cs->abort;
@@ -255,7 +266,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         // tile qt) and one 64-column half of each 128-column accumulator, 32
         // columns at a time; the row's two halves go to two warps
         const float NEG = __int_as_float(0xff800000);
-        const int g = ep_N > 0 ? group_width(ep_N, a.P) : 1;  // <= 64: a group never spans two halves
+        // <= 64: a group never spans two halves; a sampled pass counts the
+        // maxima of groups of 8 (its targets lie far in the tail, where a
+        // group rarely holds two buckets above them)
+        const int g = sampled ? SAMPLE_G : (ep_N > 0 ? group_width(ep_N, a.P) : 1);
         const float tau = (a.mode == 1 && ep_q < a.nq) ? ws.tau[ep_q] : 0.0f;
         uint32_t *hrow = hist + (ep_qt * TQ + ep_r) * HSTRIDE;
         auto count = [&](float m) {  // counts per bin stay below 2^16 (at most 2^16 - 1 groups per query)
@@ -359,14 +373,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (a.mode == 1) {
             if (a.whole_range) ws.cnt[ep_q] = rowcnt[ep_qt * TQ + ep_r];
         } else if (a.whole_range) {
-            // this CTA saw every bucket of the query: threshold from the histogram
-            const int64_t G = n_groups(ep_N, a.P);
+            // this CTA saw every bucket of the query (or every S-th tile of
+            // them): threshold from the histogram.  Exact pass: the P-th
+            // largest group maximum, so >= P buckets score >= tau.  Sampled
+            // pass: the score above which margin x P x (sampled / visible)
+            // sampled scores lie -- about margin x P buckets in all, checked
+            // by the expansion
+            int64_t count = n_groups(ep_N, a.P), target = a.P;
+            if (sampled) {
+                const int64_t full = ep_N / TB;  // N is a multiple of 64: at most one half tile
+                const int64_t ns = ((full + S - 1) / S) * TB + ((ep_N % TB) != 0 && full % S == 0 ? ep_N % TB : 0);
+                count = ns / SAMPLE_G;
+                target = (int64_t)ceilf(a.sample_margin * (float)a.P * (float)ns / (float)ep_N);
+            }
             float t = __int_as_float(0xff800000);
-            if (G > a.P) {
-                int acc = 0;
+            if (count > target) {
+                int64_t acc = 0;
                 for (int bin = HIST_BINS - 1; bin > 0; --bin) {
                     acc += (hrow[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
-                    if (acc >= a.P) {
+                    if (acc >= target) {
                         t = hist_edge(bin);
                         break;
                     }
@@ -465,7 +490,9 @@ cudaError_t launch_score_tc(const ScoreTcArgs &a, const IndexWs &ws, const uint1
                         (a.mode == 0 ? HIST_BYTES : ROWCNT_BYTES) + sizeof(TcSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int kt = kt_begin(a.mode == 0 ? "k_score_tc:threshold" : "k_score_tc:filter", st);
+    const int kt = kt_begin(a.mode == 0 ? (a.sample > 1 && b.whole_range ? "k_score_tc:sampled" : "k_score_tc:threshold")
+                                        : "k_score_tc:filter",
+                            st);
     k_score_tc<<<dim3((unsigned)qpairs, (unsigned)chunks), THREADS, smem, st>>>(tmA, tmB, b, ws);
     kt_end(kt, st);
     count_launches(1);

@@ -57,7 +57,7 @@ class lsa_tree(C.Structure):
 
 
 EXPORTS = ["lsa_default_params", "lsa_last_error_string", "lsa_launch_count", "lsa_check_device_errors",
-           "lsa_debug_wait_test", "lsa_debug_attention_ranges", "lsa_kernel_timing", "lsa_kernel_timing_read", "lsa_list_budget", "lsa_top_buckets",
+           "lsa_debug_wait_test", "lsa_debug_attention_ranges", "lsa_debug_score_sample", "lsa_kernel_timing", "lsa_kernel_timing_read", "lsa_list_budget", "lsa_top_buckets",
            "lsa_cache_bytes", "lsa_cache_bind", "lsa_tree_bytes", "lsa_tree_bind",
            "lsa_index_workspace_bytes", "lsa_attention_workspace_bytes", "lsa_build_cache",
            "lsa_shrink", "lsa_build_tree", "lsa_update_tree", "lsa_index_prefill", "lsa_index_decode", "lsa_sparse_attention",
@@ -99,6 +99,7 @@ def lib():
             "lsa_check_device_errors": (C.c_int, []),
             "lsa_debug_wait_test": (None, [i32]),
             "lsa_debug_attention_ranges": (None, [i64]),
+            "lsa_debug_score_sample": (None, [i32, C.c_float]),
             "lsa_kernel_timing": (None, [i32]),
             "lsa_kernel_timing_read": (C.c_int, [C.c_char_p, i32, C.POINTER(C.c_double), C.POINTER(i64), i32]),
             "lsa_list_budget": (i32, [pp]),
@@ -209,6 +210,12 @@ def lsa_debug_attention_ranges(range_rows: int):
     """Test hook: force the attention's position-range phases with ranges of
     range_rows positions (0: automatic)."""
     lib().lsa_debug_attention_ranges(int(range_rows))
+
+
+def lsa_debug_score_sample(stride: int = 16, margin: float = 0.9):
+    """Flat search's sampled threshold: every stride-th centroid tile, tau
+    with about margin x P buckets above it (stride <= 1: exact histogram)."""
+    lib().lsa_debug_score_sample(int(stride), float(margin))
 
 
 def lsa_list_budget(p: lsa_params) -> int:

@@ -184,6 +184,17 @@ void lsa_debug_wait_test(int32_t enable);
  * restores the automatic choice. */
 void lsa_debug_attention_ranges(int64_t range_rows);
 
+/* Tuning and test hook of Flat search.  A single-head Flat query that sees
+ * at least stride x 4096 buckets takes its threshold tau from every
+ * stride-th tile of 128 centroids (stride 16 and margin 0.9 by default):
+ * tau is set so that about margin x P of the visible buckets lie above it.
+ * Every bucket at or above tau is still ranked, so the result is the exact
+ * one; a query whose buckets above tau hold fewer than k far keys is redone
+ * by the exact selection.  stride <= 1 turns the sampling off (the exact
+ * histogram of all buckets); a small margin (e.g. 0.01) makes the exact
+ * redo happen, which tests exercise. */
+void lsa_debug_score_sample(int32_t stride, float margin);
+
 /* Per-kernel timing, a profiling aid.  While enabled (lsa_kernel_timing(1)),
  * every kernel the library launches is bracketed by two CUDA events recorded
  * on the stream it is launched on, tagged with the kernel's name (the

@@ -115,6 +115,54 @@ def test_flat_exact_fallback_selection(tiny):
     PT.assert_lists_match(gl, gn, ol, on, q[sel], pos[sel], oc, k=256)
 
 
+@pytest.fixture(scope="module")
+def ctx96k():
+    """192 full blocks (12288 buckets) and a ragged tail of 300 keys."""
+    T = 98304 + 300
+    keys = I.index_keys(5, T, 32)
+    pos = np.arange(T, dtype=np.int64)
+    q = I.index_queries(5, keys, pos)
+    return keys, q, O.build_cache(keys)
+
+
+@pytest.mark.parametrize("stride,margin", [(2, 1.25), (4, 1.25), (4, 0.9), (2, 0.5), (2, 0.01)])
+def test_flat_sampled_threshold(ctx96k, stride, margin):
+    """Flat search's threshold taken from every stride-th centroid tile (a
+    batch of > 28K queries, each seeing >= 128 blocks, so that one CTA scans a
+    query tile's whole bucket range): the lists are the exact ones.  With
+    margin 1.25 about 1.25 P buckets (~10 k far keys) lie above tau, so no
+    query is redone and the lists equal the full histogram's bit for bit.
+    Smaller margins (the default 0.9 among them) may put tau above the cut
+    for some queries (0.5) or every one (0.01), which is then redone by the
+    exact selection: its scores come from the CUDA cores instead of the
+    tensor cores, so near-ties may order differently, and those lists are
+    held to the oracle's near-tie rule on a denser sample."""
+    keys, q, oc = ctx96k
+    T = keys.shape[0]
+    sel = np.arange(66000, T, dtype=np.int64)
+    qq = q[sel]
+    cache, _, p = _build_gpu(keys, k=256)
+    try:
+        lsa.lsa_debug_score_sample(1)
+        el, en = _index_gpu(cache, None, p, qq, sel)
+        lsa.lsa_debug_score_sample(stride, margin)
+        lsa.lsa_kernel_timing(1)
+        gl, gn = _index_gpu(cache, None, p, qq, sel)
+        names = list(lsa.lsa_kernel_timing_read())
+    finally:
+        lsa.lsa_kernel_timing(0)
+        lsa.lsa_debug_score_sample()
+    assert "k_score_tc:sampled" in names
+    assert np.array_equal(gn, en)
+    if margin >= 1.0:
+        L = int(en.max())
+        mask = np.arange(L)[None, :] < en[:, None]
+        assert np.array_equal(np.where(mask, gl[:, :L], -1), np.where(mask, el[:, :L], -1))
+    sub = np.arange(0, len(sel), 41 if margin >= 1.0 else 7)
+    ol, on = O.index(qq[sub], sel[sub], oc, k=256)
+    PT.assert_lists_match(gl[sub], gn[sub], ol, on, qq[sub], sel[sub], oc, k=256)
+
+
 @pytest.mark.parametrize("cand_cap", [0, 193])
 def test_decode_positions_past_context(tiny, cand_cap):
     """Decode: new tokens at or past the clustered context see every block
@@ -130,6 +178,24 @@ def test_decode_positions_past_context(tiny, cand_cap):
         gl, gn = _index_gpu(cache, None, p, qq[:nq], pos[:nq], decode=True)
         ol, on = O.index(qq[:nq], pos[:nq], oc, k=256)
         PT.assert_lists_match(gl, gn, ol, on, qq[:nq], pos[:nq], oc, k=256)
+
+
+@pytest.mark.parametrize("k", [1, 7, 256, 5000])
+def test_small_batches_edge_positions(tiny, k):
+    """Batches of <= 16 queries (one wide CTA per query ranks and cuts, the
+    far keys are written block by block by a second kernel) at the edge
+    positions: before the first block, in the sink, at block edges, with the
+    window over clustered blocks, k from 1 to dense."""
+    keys, q, _, oc = tiny
+    pos = np.array([0, 1, 4, 5, 511, 512, 513, 515, 516, 1023, 1024, 1025, 1535, 2047, 2048, 2049, 3000, 4095,
+                    4094, 600, 661, 3999, 1500, 2600], np.int64)
+    cache, _, p = _build_gpu(keys, k=k)
+    for a in range(0, len(pos), 16):
+        pp = pos[a:a + 16]
+        qq = q[pp]
+        gl, gn = _index_gpu(cache, None, p, qq, pp)
+        ol, on = O.index(qq, pp, oc, k=k)
+        PT.assert_lists_match(gl, gn, ol, on, qq, pp, oc, k=k)
 
 
 @pytest.mark.parametrize("heads,k,cand_cap", [(2, 256, 0), (4, 256, 0), (8, 5000, 0), (3, 7, 0), (4, 256, 193)])
