@@ -48,11 +48,12 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per row gathered by
 # the attention's gather kernel -- a (query, KV head, listed key) the kernel
 # reads -- from one ncu capture of that kernel's launch in the timed step,
-# divided by the launch's gathered rows (profiles/launches_flat_tree_10m.md:
-# 1.0889e12 B over 65536 x 4613 x 8 rows).  Keyed by (workload, mode); a
-# workload or mode without a capture of the kernel as it stands reports
-# traffic null.  Re-measure whenever k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = {("flat_tree_10m", "flat"): 450.2}
+# divided by the launch's gathered rows (profiles/launches_flat_tree_10m.md for
+# 10M; profiles/k_attn_ranges_flat_1m.md for 1M, summed over the 72 range
+# launches of the call: 39.83e9 B over 32768 x 4613 x 8 rows).  Keyed by
+# (workload, mode); a workload or mode without a capture of the kernel as it
+# stands reports traffic null.  Re-measure whenever k_attn changes.
+ATTN_DRAM_BYTES_PER_ROW = {("flat_1m", "flat"): 32.9}
 
 
 def peaks():

@@ -775,12 +775,12 @@ __global__ void __launch_bounds__(256) k_dfilter(int64_t nq, int P, IndexWs ws)
 
 // ---------------------------------------------------------------------------
 // Rank the candidates of one query and expand them into its index list.
-//   1. candidates: every listed score >= tau, each with its weight (its
-//      members outside near), in one pass (a Flat query whose entries or
+//   1. candidates: every listed score >= tau (a Flat query whose entries or
 //      candidates overflow, or whose sampled tau keeps fewer than k far keys,
 //      is redone exactly here: radix select of the P-th largest score
 //      recomputed on the CUDA cores, then every bucket above it and the
-//      lowest-id buckets equal to it, P in all; 2. weighs those);
+//      lowest-id buckets equal to it, P in all);
+//   2. each candidate's weight: its members outside near;
 //   3. the walk over buckets in (score desc, id asc) order stops at the
 //      bucket where the weights reach k: found by histogramming the weights
 //      over the candidates' rank keys (1024 or 4096 bins over the remaining
@@ -883,7 +883,7 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     int my_tot = 0;  // this thread's weights and weighted key range
     unsigned long long my_lo = ~0ull, my_hi = 0ull;
     for (;;) {  // at most twice: a sampled threshold that keeps too little is redone exactly
-    // 1. candidates with their weights (2. below for the exact path)
+    // 1. candidates
     if (!fb_s) {
         const float4 *c4 = reinterpret_cast<const float4 *>(ws.cand4) + q * ws.cap;
         const int32_t *cg = ws.cand_g + q * ws.cap;
@@ -908,14 +908,11 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
                 }
             }
             int nc = 0;
-            int cb[4];  // member counts of kept buckets clear of near, loaded before the slot search
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 if (sv[e] >= tau && sv[e] > NEG && !LSA_IN_BOUNDS(g + e >= 0 && g + e < N, BOUNDS_BUCKET))
                     sv[e] = NEG;  // debug build: a bucket the query cannot see is dropped
-                const bool kept = sv[e] >= tau && sv[e] > NEG;
-                nc += kept;
-                cb[e] = kept && clear_of_near(g + e) ? __ldg(count + g + e) : -1;
+                nc += sv[e] >= tau && sv[e] > NEG;
             }
             // one shared-memory atomic per warp
             int incl = nc;
@@ -930,18 +927,8 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 if (sv[e] >= tau && sv[e] > NEG) {
-                    const int nn = cb[e] >= 0 ? cb[e] : far_members(g + e);
-                    const uint64_t key = rank_key(sv[e], g + e);
-                    if (slot < KC) {
-                        keys[slot] = key;
-                        wt[slot] = (uint8_t)nn;
-                    }
+                    if (slot < KC) keys[slot] = rank_key(sv[e], g + e);
                     ++slot;
-                    my_tot += nn;
-                    if (nn > 0) {
-                        my_lo = min(my_lo, (unsigned long long)key);
-                        my_hi = max(my_hi, (unsigned long long)key);
-                    }
                 }
             }
         }
@@ -983,9 +970,9 @@ __global__ void __launch_bounds__(NT) k_rank_expand(const int64_t *__restrict__ 
     }
     n = nk_s;
 
-    // 2. (exact path) weights of the selected buckets and their key range
-    if (fb_s) {
-        my_tot = 0;  // whatever the candidate pass added before it overflowed
+    // 2. weights of the candidates and the range of their weighted keys
+    {
+        my_tot = 0;
         my_lo = ~0ull;
         my_hi = 0ull;
         // the next candidate's member count is loaded before this one is used

@@ -385,7 +385,7 @@ def test_attention_peaked_softmax(tiny, nq, consecutive):
 
 
 @pytest.mark.parametrize("rows,hq,hkv,consecutive", [(300, 32, 8, False), (1000, 8, 1, True), (4096, 32, 8, False),
-                                                    (97, 16, 16, False), (513, 32, 8, True)])
+                                                    (97, 16, 16, False), (513, 32, 8, True), (700, 16, 1, False)])
 def test_attention_position_ranges_against_oracle(tiny, rows, hq, hkv, consecutive):
     """The gather taken in position ranges (one launch per KV head and range,
     a running result per (query, head) carried between launches), forced on
