@@ -639,8 +639,9 @@ def run_e2e(args, layer, keys_np, q_np, pos_np, Qd, Kd, Vd, wl, dev, world):
 def run_decode(args, dev, wl, mode, keys, dq_np, dpos_np, K, V, pk):
     """Batch-1 decode after the context: per new token, its index
     (lsa_index_decode) and its sparse attention.  The two calls are captured
-    once in a CUDA graph; each token copies its query into the graph's input
-    buffers and replays it (both inside the timed region).  Mean us/token
+    once in a CUDA graph; each token copies its inputs (index query, position,
+    Q, packed in one row) into the graph's input row and replays it (both
+    inside the timed region).  Mean us/token
     over the decode tokens; the eager figure is kept too, and one more eager
     pass with per-kernel events gives the kernels' rooflines."""
     T, hq, hkv = wl["T"], wl["hq"], wl["hkv"]
@@ -650,9 +651,19 @@ def run_decode(args, dev, wl, mode, keys, dq_np, dpos_np, K, V, pk):
     g = torch.Generator(device=dev)
     g.manual_seed(77)
     Qd = torch.randn((nd, 1, hq, 128), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    qd = torch.from_numpy(dq_np).to(dev)
-    pd = torch.from_numpy(dpos_np).to(dev)
-    q_in, p_in, Q_in = qd[:1].clone(), pd[:1].clone(), Qd[0].clone()
+    # each token's inputs packed in one row -- index query (64 fp32), position
+    # (int64, padded to 16 B), Q (hq x 128 bf16) -- so that a token is fed by
+    # one copy into the graph's input row, whose views are the call arguments
+    qbytes, qoff = 64 * 4, 64 * 4 + 16
+    row = qoff + hq * 128 * 2
+    packed = torch.empty((nd, row), dtype=torch.uint8, device=dev)
+    packed[:, :qbytes].view(torch.float32).copy_(torch.from_numpy(dq_np).to(dev))
+    packed[:, qbytes:qbytes + 8].view(torch.int64).copy_(torch.from_numpy(dpos_np).to(dev)[:, None])
+    packed[:, qoff:].view(torch.bfloat16).copy_(Qd.reshape(nd, hq * 128))
+    inp = packed[0].clone()
+    q_in = inp[:qbytes].view(torch.float32).view(1, 64)
+    p_in = inp[qbytes:qbytes + 8].view(torch.int64)
+    Q_in = inp[qoff:].view(torch.bfloat16).view(1, hq, 128)
     O = torch.empty((1, hq, 128), dtype=torch.bfloat16, device=dev)
     Kd, Vd = K[:T + nd], V[:T + nd]
 
@@ -661,9 +672,7 @@ def run_decode(args, dev, wl, mode, keys, dq_np, dpos_np, K, V, pk):
         layer.attend(Q_in, Kd, Vd, O)
 
     def feed(i):
-        q_in.copy_(qd[i:i + 1])
-        p_in.copy_(pd[i:i + 1])
-        Q_in.copy_(Qd[i])
+        inp.copy_(packed[i])
 
     for i in range(4):
         feed(i)

@@ -637,6 +637,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
+// NQ: the batch rounded up to a power of two (the per-query loops are
+// unrolled over it, so a batch of one keeps few registers and many CTAs).
+template <int NQ>
 __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb_total,
                                                           const uint16_t *__restrict__ cbf, int P, IndexWs ws)
 {
@@ -645,7 +648,7 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
     extern __shared__ __align__(16) uint8_t ds_dyn[];
     uint32_t *hs = reinterpret_cast<uint32_t *>(ds_dyn + DS_WARPS * 2 * 32 * DS_ROW);
     float *qf = reinterpret_cast<float *>(hs + nq * HIST_BINS);
-    __shared__ int Nq[SMALL_NQ], gq[SMALL_NQ];
+    __shared__ int Nq[NQ], gq[NQ];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float NEG = __int_as_float(0xff800000);
     const int64_t wbase = (int64_t)blockIdx.x * DS_SPAN + warp * 128;
@@ -678,9 +681,9 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
         gq[t] = group_width(N, P);
     }
     __syncthreads();
-    float run[SMALL_NQ];
+    float run[NQ];
 #pragma unroll
-    for (int i = 0; i < SMALL_NQ; ++i) run[i] = NEG;
+    for (int i = 0; i < NQ; ++i) run[i] = NEG;
     for (int r = 0; r < 4; ++r) {
         if (r >= 1 && r + 1 < 4) issue(r + 1);  // rounds 0 and 1 were issued above
         if (r + 1 < 4) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
@@ -699,7 +702,7 @@ __global__ void __launch_bounds__(DS_WARPS * 32) k_dscore(int64_t nq, int64_t nb
         }
         __syncwarp();  // this buffer is refilled two rounds later
 #pragma unroll
-        for (int qi = 0; qi < SMALL_NQ; ++qi) {
+        for (int qi = 0; qi < NQ; ++qi) {
             if (qi >= nq) break;  // uniform
             const float4 *qv = reinterpret_cast<const float4 *>(qf + qi * LSA_D);
             float acc = 0.0f;
@@ -1829,9 +1832,11 @@ cudaError_t launch_index(const IndexArgs &a, const IndexWs &ws, const IndexWs *m
     if (a.mode == 0 && nb_total > 0) {
         if (rows <= SMALL_NQ) {  // stream every centroid once for the whole batch, keep the scores
             const int dsm = DS_WARPS * 2 * 32 * DS_ROW + (int)rows * (HIST_BINS + LSA_D) * 4;
-            cudaFuncSetAttribute(k_dscore, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+            auto ds = rows <= 1 ? k_dscore<1> : rows <= 2 ? k_dscore<2> : rows <= 4 ? k_dscore<4>
+                    : rows <= 8 ? k_dscore<8> : k_dscore<SMALL_NQ>;
+            cudaFuncSetAttribute(ds, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
             int kt = kt_begin("k_dscore", st);
-            e = launch_k(true, k_dscore, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
+            e = launch_k(true, ds, dim3((unsigned)((nb_total + DS_SPAN - 1) / DS_SPAN)), dim3(DS_WARPS * 32),
                          (size_t)dsm, st, rows, nb_total, a.centroid_bf16, a.P, ws);
             kt_end(kt, st);
             if (e != cudaSuccess) return e;
