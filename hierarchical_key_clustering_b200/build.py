@@ -14,8 +14,8 @@ LIB = os.path.join(PKG, "liblsa.so")
 # (-DLSA_BOUNDS_CHECKS=1); a failed check is reported through
 # lsa_check_device_errors(), never a trap
 LIB_DEBUG = os.path.join(PKG, "liblsa_debug.so")
-SOURCES = ["lsa_api.cu", "lsa_build.cu", "lsa_index.cu", "lsa_score_tc.cu", "lsa_attn.cu", "lsa_noalloc.cu",
-           "lsa_shrink.cu", "lsa_shard.cu"]
+SOURCES = ["lsa_api.cu", "lsa_build.cu", "lsa_index.cu", "lsa_score_tc.cu", "lsa_attn.cu", "lsa_near_tc.cu",
+           "lsa_noalloc.cu", "lsa_shrink.cu", "lsa_shard.cu"]
 HEADERS = ["lsa_common.cuh", "lsa_kernels.h", "lsa_tc.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

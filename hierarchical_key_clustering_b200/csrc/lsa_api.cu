@@ -799,6 +799,7 @@ int lsa_sparse_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V
     a.range_off = nullptr;
     a.state_o = nullptr;
     a.state_ml = nullptr;
+    a.wait_limit = g_wait_limit;
     a.n_ranges = 0;
     a.range_rows = 0;
     a.phase_g = a.phase_r = 0;

@@ -571,26 +571,22 @@ __global__ void __launch_bounds__(CB_THREADS) k_attn_combine(AttnArgs a)
 // Near set, shared by consecutive queries.  A list written by the indexer
 // ends with the window [p - window, p] and starts with the sink keys
 // 0 .. sink - 1; consecutive queries (positions p, p + 1, ...) read almost
-// the same window rows.  k_attn_near takes, per query, the longest run of
+// the same window rows.  The near-set kernel takes, per query, the longest run of
 // consecutive positions that ends the list (at most NEAR_DMAX keys, the last
 // being p) and the run 0, 1, .. that starts it (at most NEAR_SMAX keys,
 // disjoint from the first), read from the list itself, so any strictly
 // increasing list is handled.  A CTA takes a tile of NEAR_ROWS / G
 // consecutive queries and one KV head: the union of the tile's near keys
 // streams through shared memory once, 64 keys at a time, and every query
-// head of the tile is a row of a 128 x 64 score tile (8 warps x 16 rows,
-// mma.sync m16n8k16, fp32 online softmax masked per row to the query's own
-// keys).  The partial results (unnormalised O, running max, sum) go to the
-// workspace; k_attn then reads only the rest of each list and merges.  A tile
+// head of the tile is a row of a 128 x 64 score tile on the tensor cores
+// (k_attn_near_tc, lsa_near_tc.cu: tcgen05 with TMEM accumulators, fp32
+// online softmax masked per row to the query's own keys).  The partial
+// results (unnormalised O, reference max, sum) go to the workspace; k_attn
+// then reads only the rest of each list and merges.  A tile
 // whose queries do not sit at consecutive positions gets an empty plan and
 // k_attn reads those lists whole.
 constexpr int NEAR_DMAX = 1024;  // longest window suffix taken densely
 constexpr int NEAR_SMAX = 16;    // longest sink prefix taken densely
-constexpr int NKC = 64;          // keys per chunk
-constexpr int NEAR_WARPS = NEAR_ROWS / 16;
-constexpr int NEAR_NST = 4;      // chunk ring stages
-constexpr int NEAR_STAGE = 2 * NKC * ROWB * 2;  // K + V of one chunk
-constexpr int NEAR_SMEM = NEAR_NST * NEAR_STAGE;
 
 // Plan of one tile (one CTA of NEAR_ROWS threads): per query p = its last
 // listed position, d = the run of consecutive positions that ends the list,
@@ -650,189 +646,6 @@ __global__ void __launch_bounds__(NEAR_ROWS) k_near_plan(AttnArgs a)
     }
 }
 
-__global__ void __launch_bounds__(NEAR_WARPS * 32, 1) k_attn_near(AttnArgs a)
-{
-    extern __shared__ __align__(128) uint8_t nsmem[];
-    const int4 tile = a.near_tile[blockIdx.x];
-    if (!tile.x) return;
-    const int G = a.Hq / a.Hkv;
-    const int QT = near_tile_queries(G);
-    const int g = blockIdx.y;
-    const int64_t q0 = (int64_t)blockIdx.x * QT;
-    const int nt_q = (int)min((int64_t)QT, a.nq - q0);
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int lo = tile.z, smax = tile.w, hi = tile.y + nt_q - 1;
-    const int n_band = (hi - lo + NKC) / NKC;
-    const int nch = (smax > 0 ? 1 : 0) + n_band;  // the sink chunk first, then the band
-    auto chunk_first = [&](int ch) { return smax > 0 ? (ch == 0 ? 0 : lo + (ch - 1) * NKC) : lo + ch * NKC; };
-    auto chunk_last = [&](int ch) { return (smax > 0 && ch == 0) ? smax - 1 : min(hi, chunk_first(ch) + NKC - 1); };
-
-    // this warp's 16 rows: row r = query r / G, head r % G of KV head g
-    const int r0 = lane >> 2, c = lane & 3;
-    const int rA = warp * 16 + r0, rB = rA + 8;
-    const int qa = rA / G, qb = rB / G;
-    const bool va = qa < nt_q, vb = qb < nt_q;
-    const int2 pla = va ? a.near_plan[q0 + qa] : make_int2(0, 0), plb = vb ? a.near_plan[q0 + qb] : make_int2(0, 0);
-    const int pa = tile.y + qa, pb = tile.y + qb;
-    const int la = pa - pla.y + 1, lb = pb - plb.y + 1;
-    const int sa = pla.x, sb = plb.x;
-    const uint16_t *QA = a.Q + (((q0 + (va ? qa : 0)) * a.Hq) + (int64_t)g * G + rA % G) * LSA_HEAD;
-    const uint16_t *QB = a.Q + (((q0 + (vb ? qb : 0)) * a.Hq) + (int64_t)g * G + rB % G) * LSA_HEAD;
-    uint32_t qf[8][4];
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        qf[kk][0] = va ? ld_u32(QA + kk * 16 + 2 * c) : 0u;
-        qf[kk][1] = vb ? ld_u32(QB + kk * 16 + 2 * c) : 0u;
-        qf[kk][2] = va ? ld_u32(QA + kk * 16 + 8 + 2 * c) : 0u;
-        qf[kk][3] = vb ? ld_u32(QB + kk * 16 + 8 + 2 * c) : 0u;
-    }
-
-    const uint32_t sbase = smem_u32(nsmem);
-    auto load = [&](int ch, int st) {
-        const int k0 = chunk_first(ch), k1 = chunk_last(ch);
-        const uint32_t sK = sbase + st * NEAR_STAGE, sV = sK + NKC * ROWB * 2;
-#pragma unroll
-        for (int it = 0; it < (NKC * 16) / (NEAR_WARPS * 32); ++it) {
-            const int lin = it * NEAR_WARPS * 32 + t;
-            const int row = lin >> 4, seg = lin & 15;
-            const int key = k0 + row;
-            const bool in = key <= k1;
-            const int64_t off = ((int64_t)(in ? key : 0) * a.Hkv + g) * LSA_HEAD + seg * 8;
-            const uint32_t so = tile_off(row, seg);
-            cp_async16(sK + so, a.K + off, in ? 16 : 0);
-            cp_async16(sV + so, a.V + off, in ? 16 : 0);
-        }
-        cp_commit();
-    };
-
-    const float NEG = __int_as_float(0xff800000);
-    const float sl2 = a.scale * LOG2E;
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) o[n][j] = 0.0f;
-    float mA = NEG, mB = NEG, lA = 0.0f, lB = 0.0f;
-
-#pragma unroll
-    for (int st = 0; st < NEAR_NST - 1; ++st) {
-        if (st < nch) load(st, st);
-        else cp_commit();
-    }
-    for (int ch = 0; ch < nch; ++ch) {
-        const int nxt = ch + NEAR_NST - 1;
-        if (nxt < nch) load(nxt, nxt % NEAR_NST);
-        else cp_commit();
-        cp_wait<NEAR_NST - 1>();
-        __syncthreads();
-        const uint32_t sK = sbase + (ch % NEAR_NST) * NEAR_STAGE, sV = sK + NKC * ROWB * 2;
-        const bool sink = smax > 0 && ch == 0;
-        const int k0 = chunk_first(ch);
-        // S = Q K^T over the chunk's 64 keys: 8 tiles of 8 keys
-        float s[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) s[n][j] = 0.0f;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-            for (int jp = 0; jp < 4; ++jp) {  // key tiles 2 jp, 2 jp + 1
-                uint32_t kb[4];
-                const int mi = lane >> 3;
-                ldsm_x4(kb, sK + tile_off(16 * jp + (lane & 7) + ((mi >> 1) << 3), 2 * kk + (mi & 1)));
-                mma16816(s[2 * jp], qf[kk], kb[0], kb[1]);
-                mma16816(s[2 * jp + 1], qf[kk], kb[2], kb[3]);
-            }
-        }
-        // mask each row to its own keys, then the online softmax
-        float mxA = NEG, mxB = NEG;
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int key = k0 + 8 * n + 2 * c + e;
-                const bool inA = sink ? key < sa : (key >= la && key <= pa);
-                const bool inB = sink ? key < sb : (key >= lb && key <= pb);
-                s[n][e] = (va && inA) ? s[n][e] * sl2 : NEG;
-                s[n][2 + e] = (vb && inB) ? s[n][2 + e] * sl2 : NEG;
-                mxA = fmaxf(mxA, s[n][e]);
-                mxB = fmaxf(mxB, s[n][2 + e]);
-            }
-        }
-#pragma unroll
-        for (int o2 = 1; o2 < 4; o2 <<= 1) {
-            mxA = fmaxf(mxA, __shfl_xor_sync(LSA_FULL, mxA, o2));
-            mxB = fmaxf(mxB, __shfl_xor_sync(LSA_FULL, mxB, o2));
-        }
-        const float mnA = fmaxf(mA, mxA), mnB = fmaxf(mB, mxB);
-        // rows with no key yet keep max -inf; exp2 of (-inf) - (-inf) is avoided
-        const float alA = mnA == NEG ? 1.0f : exp2f(mA - mnA), alB = mnB == NEG ? 1.0f : exp2f(mB - mnB);
-        float rsA = 0.0f, rsB = 0.0f;
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                s[n][e] = mnA == NEG ? 0.0f : exp2f(s[n][e] - mnA);
-                s[n][2 + e] = mnB == NEG ? 0.0f : exp2f(s[n][2 + e] - mnB);
-                rsA += s[n][e];
-                rsB += s[n][2 + e];
-            }
-        }
-#pragma unroll
-        for (int o2 = 1; o2 < 4; o2 <<= 1) {
-            rsA += __shfl_xor_sync(LSA_FULL, rsA, o2);
-            rsB += __shfl_xor_sync(LSA_FULL, rsB, o2);
-        }
-        lA = lA * alA + rsA;
-        lB = lB * alB + rsB;
-        mA = mnA;
-        mB = mnB;
-        if (alA != 1.0f || alB != 1.0f) {
-#pragma unroll
-            for (int n = 0; n < 16; ++n) {
-                o[n][0] *= alA;
-                o[n][1] *= alA;
-                o[n][2] *= alB;
-                o[n][3] *= alB;
-            }
-        }
-        // O += P V: P (16 rows x 64 keys) as 4 A tiles, V^T via transposing loads
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t pa4[4];
-            pa4[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-            pa4[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-            pa4[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-            pa4[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-            for (int dp = 0; dp < 8; ++dp) {  // dim tiles 2 dp, 2 dp + 1
-                uint32_t vb4[4];
-                const int mi = lane >> 3;
-                ldsm_x4_t(vb4, sV + tile_off(16 * kk + (lane & 7) + ((mi & 1) << 3), 2 * dp + (mi >> 1)));
-                mma16816(o[2 * dp], pa4, vb4[0], vb4[1]);
-                mma16816(o[2 * dp + 1], pa4, vb4[2], vb4[3]);
-            }
-        }
-        __syncthreads();  // this stage is refilled NEAR_NST - 1 chunks later
-    }
-    cp_wait<0>();
-    // partial results of rows rA, rB
-    if (va) {
-        const int64_t row = (q0 + qa) * a.Hq + (int64_t)g * G + rA % G;
-        float *po = a.near_o + row * LSA_HEAD;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) *reinterpret_cast<float2 *>(po + 8 * n + 2 * c) = make_float2(o[n][0], o[n][1]);
-        if (c == 0) *reinterpret_cast<float2 *>(a.near_ml + row * 2) = make_float2(mA, lA);
-    }
-    if (vb) {
-        const int64_t row = (q0 + qb) * a.Hq + (int64_t)g * G + rB % G;
-        float *po = a.near_o + row * LSA_HEAD;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) *reinterpret_cast<float2 *>(po + 8 * n + 2 * c) = make_float2(o[n][2], o[n][3]);
-        if (c == 0) *reinterpret_cast<float2 *>(a.near_ml + row * 2) = make_float2(mB, lB);
-    }
-}
 
 int attention_list_cap()
 {
@@ -921,12 +734,10 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
         int kt = kt_begin("k_near_plan", st);
         k_near_plan<<<tiles, NEAR_ROWS, 0, st>>>(a);
         kt_end(kt, st);
-        if ((e = cudaFuncSetAttribute(k_attn_near, cudaFuncAttributeMaxDynamicSharedMemorySize, NEAR_SMEM)) !=
-            cudaSuccess)
-            return e;
         kt = kt_begin("k_attn_near", st);
-        k_attn_near<<<dim3(tiles, (unsigned)a.Hkv), NEAR_WARPS * 32, NEAR_SMEM, st>>>(a);
+        e = launch_attention_near_tc(a, (int)tiles, st);
         kt_end(kt, st);
+        if (e != cudaSuccess) return e;
         count_launches(2);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

@@ -230,6 +230,7 @@ struct AttnArgs {
     int32_t n_ranges;
     int64_t range_rows;
     int32_t phase_g, phase_r;
+    uint32_t wait_limit;  // tries per bounded device-side wait (tensor-core near tiles)
 };
 
 // Queries per near-set tile for G query heads per KV head, 0 = no near path.
@@ -237,6 +238,8 @@ constexpr int NEAR_ROWS = 128;
 __host__ __device__ inline int near_tile_queries(int G) { return (G >= 1 && NEAR_ROWS % G == 0) ? NEAR_ROWS / G : 0; }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm);
+cudaError_t launch_attention_near_tc(const AttnArgs &a, int tiles, cudaStream_t st);
+int read_near_error(int clear);
 int attention_list_cap();
 
 }  // namespace lsa

@@ -509,9 +509,11 @@ int read_device_error(int clear)
     }
     const int w = read_shrink_error(clear);  // the projection kernel's own word
     if (w < 0) return -1;
+    const int wn = read_near_error(clear);  // the near-set tensor-core attention's word
+    if (wn < 0) return -1;
     const int ba = read_bounds_error_attn(clear), bi = read_bounds_error_index(clear);  // debug build only
     if (ba < 0 || bi < 0) return -1;
-    return v | w | ba | bi;
+    return v | w | wn | ba | bi;
 }
 
 }  // namespace lsa
