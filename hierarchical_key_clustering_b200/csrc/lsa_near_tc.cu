@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
         // chunk j once the P V of chunk j - 2 has read its stage
         auto load_k = [&](int j) {
             const int s = j % NT_KST;
-            if (j >= NT_KST && !tc::wait_bounded(bar(cs->k_empty[s]), (uint32_t)(((j / NT_KST) - 1) & 1), wl, abort, err))
+            if (j >= NT_KST && !tc::wait_bounded_sleep(bar(cs->k_empty[s]), (uint32_t)(((j / NT_KST) - 1) & 1), wl, abort, err))
                 return false;
             const uint32_t dk = tc::smem_u32(sK + s * NT_K_BYTES);
             tc::mbar_expect_tx(bar(cs->k_full[s]), NT_K_BYTES);
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
         };
         auto load_v = [&](int j) {
             const int s = j % NT_KST;
-            if (j >= NT_KST && !tc::wait_bounded(bar(cs->v_empty[s]), (uint32_t)(((j / NT_KST) - 1) & 1), wl, abort, err))
+            if (j >= NT_KST && !tc::wait_bounded_sleep(bar(cs->v_empty[s]), (uint32_t)(((j / NT_KST) - 1) & 1), wl, abort, err))
                 return false;
             const uint32_t dv = tc::smem_u32(sV + s * NT_V_BYTES);
             tc::mbar_expect_tx(bar(cs->v_full[s]), NT_V_BYTES);
@@ -158,8 +158,8 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
     } else if (warp == 1 && lane == 0) {
         auto issue_pv = [&](int c) {
             const int s = c % NT_KST, b = c & 1;
-            if (!tc::wait_bounded(bar(cs->pv_ready), (uint32_t)(c & 1), wl, abort, err)) return false;
-            if (!tc::wait_bounded(bar(cs->v_full[s]), (uint32_t)((c / NT_KST) & 1), wl, abort, err)) return false;
+            if (!tc::wait_bounded_sleep(bar(cs->pv_ready), (uint32_t)(c & 1), wl, abort, err)) return false;
+            if (!tc::wait_bounded_sleep(bar(cs->v_full[s]), (uint32_t)((c / NT_KST) & 1), wl, abort, err)) return false;
             tc::fence_after();
             // P from the first 32 columns of score buffer b (16 keys = 8 columns per
             // instruction); the V chunk as the MN-major B operand: 64-dim halves
@@ -174,14 +174,14 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
             tc::mma_commit(bar(cs->pv_done));
             return true;
         };
-        bool ok = tc::wait_bounded(bar(cs->q_full), 0, wl, abort, err);
+        bool ok = tc::wait_bounded_sleep(bar(cs->q_full), 0, wl, abort, err);
         for (int i = 0; ok && i < nch; ++i) {
             const int s = i % NT_KST, b = i & 1;
-            if (!tc::wait_bounded(bar(cs->k_full[s]), (uint32_t)((i / NT_KST) & 1), wl, abort, err)) {
+            if (!tc::wait_bounded_sleep(bar(cs->k_full[s]), (uint32_t)((i / NT_KST) & 1), wl, abort, err)) {
                 ok = false;
                 break;
             }
-            if (i >= 2 && !tc::wait_bounded(bar(cs->s_empty[b]), (uint32_t)(((i >> 1) - 1) & 1), wl, abort, err)) {
+            if (i >= 2 && !tc::wait_bounded_sleep(bar(cs->s_empty[b]), (uint32_t)(((i >> 1) - 1) & 1), wl, abort, err)) {
                 ok = false;
                 break;
             }
@@ -215,23 +215,38 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
         bool ok = true;
         for (int i = 0; i < nch; ++i) {
             const int b = i & 1;
-            ok = __all_sync(LSA_FULL, tc::wait_bounded(bar(cs->s_full[b]), (uint32_t)((i >> 1) & 1), wl, abort, err));
+            ok = __all_sync(LSA_FULL, tc::wait_bounded_sleep(bar(cs->s_full[b]), (uint32_t)((i >> 1) & 1), wl, abort, err));
             if (!ok) break;
             tc::fence_after();
             float v[NT_KC];
             tc::tmem_ld32_nowait(trow + b * NT_KC, v);
             tc::tmem_ld32_nowait(trow + b * NT_KC + 32, v + 32);
             tc::tmem_wait_ld();
-            const bool sink = smax > 0 && i == 0;
+            // the row's keys in this chunk as a column range [ca, cb]
             const int k0 = chunk_first(i), k1 = chunk_last(i);
-            float mx = NEG;
-#pragma unroll
-            for (int j = 0; j < NT_KC; ++j) {
-                const int key = k0 + j;
-                const bool in = valid && key <= k1 && (sink ? key < sr : (key >= lr && key <= pr));
-                v[j] = in ? v[j] * sl2 : NEG;
-                mx = fmaxf(mx, v[j]);
+            int ca = 1, cb = 0;  // empty
+            if (valid) {
+                if (smax > 0 && i == 0) {
+                    ca = 0;
+                    cb = min(sr - 1, k1) - k0;
+                } else {
+                    ca = max(lr, k0) - k0;
+                    cb = min(pr, k1) - k0;
+                }
             }
+            if (!__all_sync(LSA_FULL, ca == 0 && cb >= NT_KC - 1)) {  // some row has masked columns
+#pragma unroll
+                for (int j = 0; j < NT_KC; ++j) v[j] = (j >= ca && j <= cb) ? v[j] : NEG;
+            }
+            // row maximum of the raw scores by a tree (the scale is positive)
+            float t[NT_KC / 2];
+#pragma unroll
+            for (int j = 0; j < NT_KC / 2; ++j) t[j] = fmaxf(v[j], v[j + NT_KC / 2]);
+#pragma unroll
+            for (int w = NT_KC / 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+            const float mx = t[0] > NEG ? t[0] * sl2 : NEG;
             // the reference moves to a new maximum only when the row had none
             // yet or it rose more than NT_RESCALE; then O and l are scaled
             float alpha = 1.0f;
@@ -240,21 +255,24 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
                 m = mx;
             }
             float pk[NT_KC / 2];  // bf16 pairs, as 32-bit columns
-            float rs = 0.0f;
+            float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const float mneg = m > NEG ? -m : 0.0f;
 #pragma unroll
             for (int j = 0; j < NT_KC; j += 2) {
-                const float p0 = v[j] > NEG ? exp2f(v[j] - m) : 0.0f;
-                const float p1 = v[j + 1] > NEG ? exp2f(v[j + 1] - m) : 0.0f;
-                rs += p0 + p1;
+                // masked columns hold -inf, so exp2 gives 0 there
+                const float p0 = exp2f(fmaf(v[j], sl2, mneg));
+                const float p1 = exp2f(fmaf(v[j + 1], sl2, mneg));
+                rs4[(j >> 1) & 3] += p0 + p1;
                 pk[j >> 1] = __uint_as_float(pack_bf16x2(p0, p1));
             }
+            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
             l = l * alpha + rs;
             // the previous P V is waited for at every chunk, not only before a
             // rescale: a waiter that skipped phases could no longer tell them
             // apart by parity.  Rare: a row's reference maximum moved, and this
             // warp's O rows are rescaled in TMEM.
             if (i >= 1) {
-                ok = __all_sync(LSA_FULL, tc::wait_bounded(bar(cs->pv_done), (uint32_t)((i - 1) & 1), wl, abort, err));
+                ok = __all_sync(LSA_FULL, tc::wait_bounded_sleep(bar(cs->pv_done), (uint32_t)((i - 1) & 1), wl, abort, err));
                 if (!ok) break;
                 tc::fence_after();
             }
@@ -275,7 +293,7 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(cs->pv_ready));
         }
-        if (ok) ok = __all_sync(LSA_FULL, tc::wait_bounded(bar(cs->o_full), 0, wl, abort, err));
+        if (ok) ok = __all_sync(LSA_FULL, tc::wait_bounded_sleep(bar(cs->o_full), 0, wl, abort, err));
         if (ok) {
             tc::fence_after();
             const int64_t row = (q0 + qi) * a.Hq + (int64_t)g * G + h;

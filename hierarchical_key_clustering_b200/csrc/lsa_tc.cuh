@@ -41,6 +41,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// One try with a suspend-time hint (ns): a thread whose phase is not yet
+// complete sleeps until it completes or the hint runs out, instead of
+// spinning on the issue slots its neighbours need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with sleeping tries (at most limit tries of up to 1 us each).
+__device__ __forceinline__ bool wait_bounded_sleep(uint32_t bar, uint32_t parity, uint32_t limit, volatile int *abort,
+                                                   int *err)
+{
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+        if ((i & 15u) == 15u && *abort) return false;
+    }
+    atomicExch(err, 1);
+    *abort = 1;
+    return false;
+}
+
 // Bounded wait; on expiry sets *err and the CTA abort flag.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit, volatile int *abort,
                                              int *err)
