@@ -81,9 +81,11 @@ using tc::tmem_wait_ld;
 using tc::mma_commit;
 
 // Bounded wait; on expiry sets the device error word and the CTA abort flag.
+// Waiting threads sleep on the barrier instead of spinning, so that the
+// epilogue warps' spins do not take the issue slots of the working ones.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit, volatile int *abort)
 {
-    return tc::wait_bounded(bar, parity, limit, abort, &g_device_error);
+    return tc::wait_bounded_sleep(bar, parity, limit, abort, &g_device_error);
 }
 
 // kind::f16: D fp32, A and B bf16, both K-major, N = 128, M = 128.

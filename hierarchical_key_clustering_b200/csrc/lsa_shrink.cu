@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(SH_THREADS, 3)
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmW) : "memory");
         for (int k = 0; k < nk && !*abort; ++k) {
             const int s = k % SH_NST;
-            if (k >= SH_NST && !tc::wait_bounded(bar(cs->empty[s]), (uint32_t)(((k / SH_NST) - 1) & 1), wl, abort, err))
+            if (k >= SH_NST && !tc::wait_bounded_sleep(bar(cs->empty[s]), (uint32_t)(((k / SH_NST) - 1) & 1), wl, abort, err))
                 break;
             tc::mbar_expect_tx(bar(cs->full[s]), SH_A_BYTES + SH_B_BYTES);
             tc::tma_load_2d(tc::smem_u32(sA + s * SH_A_BYTES), &tmV, k * SH_KB, (int)t0, bar(cs->full[s]));
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(SH_THREADS, 3)
         bool ok = true;
         for (int k = 0; k < nk; ++k) {
             const int s = k % SH_NST;
-            if (!tc::wait_bounded(bar(cs->full[s]), (uint32_t)((k / SH_NST) & 1), wl, abort, err)) {
+            if (!tc::wait_bounded_sleep(bar(cs->full[s]), (uint32_t)((k / SH_NST) & 1), wl, abort, err)) {
                 ok = false;
                 break;
             }
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(SH_THREADS, 3)
     } else if (warp >= 2) {
         const int quad = warp & 3, r = quad * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        const bool ok = __all_sync(LSA_FULL, tc::wait_bounded(bar(cs->acc), 0, wl, abort, err));
+        const bool ok = __all_sync(LSA_FULL, tc::wait_bounded_sleep(bar(cs->acc), 0, wl, abort, err));
         if (ok) {
             tc::fence_after();
             float x[64];
