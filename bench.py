@@ -53,7 +53,7 @@ L2_FLUSH_BYTES = 256 << 20
 # launches of the call: 39.83e9 B over 32768 x 4613 x 8 rows).  Keyed by
 # (workload, mode); a workload or mode without a capture of the kernel as it
 # stands reports traffic null.  Re-measure whenever k_attn changes.
-ATTN_DRAM_BYTES_PER_ROW = {("flat_1m", "flat"): 32.9}
+ATTN_DRAM_BYTES_PER_ROW = {("flat_tree_10m", "flat"): 450.2, ("flat_1m", "flat"): 32.9}
 
 
 def peaks():

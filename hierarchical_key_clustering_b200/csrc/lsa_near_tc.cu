@@ -12,6 +12,8 @@
 // head r % G) are the MMA M, so one pass reads each key once for all of them:
 //   warp 0     TMA producer: the Q rows once (two 64-dim boxes, 128-byte
 //              swizzle), then per 64-key chunk K and V (2-stage rings each);
+//              in a chunk with fewer than 64 keys it zeroes the V rows past
+//              them once they land (they are not the tile's keys);
 //   warp 1     allocates 256 TMEM columns (two 64-column score buffers, 128
 //              columns of O); one thread issues S = Q K^T (M 128, N 64, K 128)
 //              per chunk and, one chunk behind, O += P V (M 128, N 128, K 64)
@@ -51,7 +53,7 @@ constexpr float NT_LOG2E = 1.4426950408889634f;
 
 struct NearTcCtl {
     uint64_t q_full, pv_ready, pv_done, o_full, mma_done;
-    uint64_t k_full[NT_KST], k_empty[NT_KST], v_full[NT_KST], v_empty[NT_KST], s_full[2], s_empty[2];
+    uint64_t k_full[NT_KST], k_empty[NT_KST], v_full[NT_KST], v_ready[NT_KST], v_empty[NT_KST], s_full[2], s_empty[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
             tc::mbar_init(bar(cs->k_full[s]), 1);
             tc::mbar_init(bar(cs->k_empty[s]), 1);
             tc::mbar_init(bar(cs->v_full[s]), 1);
+            tc::mbar_init(bar(cs->v_ready[s]), 1);
             tc::mbar_init(bar(cs->v_empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -122,13 +125,15 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
     const float NEG = __int_as_float(0xff800000);
 
     int k_issued = 0, v_issued = 0;  // the producer's copies, for the abort drain
-    if (warp == 0 && lane == 0) {
-        asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmQ) : "memory");
-        asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmK) : "memory");
-        asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmV) : "memory");
-        tc::mbar_expect_tx(bar(cs->q_full), NT_Q_BYTES);
-        tc::tma_load_3d(tc::smem_u32(sQ), &tmQ, 0, g * G, (int)q0, bar(cs->q_full));
-        tc::tma_load_3d(tc::smem_u32(sQ + NT_Q_BYTES / 2), &tmQ, 64, g * G, (int)q0, bar(cs->q_full));
+    if (warp == 0) {  // lane 0 issues the copies; the warp zeroes V rows past a chunk's keys
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmQ) : "memory");
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmK) : "memory");
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&tmV) : "memory");
+            tc::mbar_expect_tx(bar(cs->q_full), NT_Q_BYTES);
+            tc::tma_load_3d(tc::smem_u32(sQ), &tmQ, 0, g * G, (int)q0, bar(cs->q_full));
+            tc::tma_load_3d(tc::smem_u32(sQ + NT_Q_BYTES / 2), &tmQ, 64, g * G, (int)q0, bar(cs->q_full));
+        }
         // K of chunk j once the S of chunk j - 2 has read its stage, V of
         // chunk j once the P V of chunk j - 2 has read its stage
         auto load_k = [&](int j) {
@@ -153,13 +158,44 @@ __global__ void __launch_bounds__(NT_THREADS, 2)
             ++v_issued;
             return true;
         };
-        bool ok = true;
-        for (int j = 0; ok && j < nch; ++j) ok = load_k(j) && load_v(j);
+        // chunk j's copies are issued before chunk j - 1's tail is handled, so
+        // that the wait for those rows to land does not hold back the next copies
+        for (int j = 0; j <= nch; ++j) {
+            if (j < nch) {
+                int okl = 1;
+                if (lane == 0) okl = load_k(j) && load_v(j);
+                if (!__shfl_sync(LSA_FULL, okl, 0)) break;
+            }
+            if (j == 0) continue;
+            const int c = j - 1, s = c % NT_KST, nvalid = chunk_last(c) - chunk_first(c) + 1;
+            if (nvalid < NT_KC) {
+                // The box also brought the rows past the chunk's last key: not
+                // the tile's keys, possibly rows nothing has written yet.  Their
+                // scores are masked, but P = 0 times a NaN row is still NaN, so
+                // the V rows are zeroed once they land (the stage's next copy is
+                // not issued yet, so the phase waited for is unambiguous).
+                int okw = 1;
+                if (lane == 0)
+                    okw = tc::wait_bounded_sleep(bar(cs->v_full[s]), (uint32_t)((c / NT_KST) & 1), wl, abort, err);
+                if (!__shfl_sync(LSA_FULL, okw, 0)) break;
+                uint8_t *dv = sV + s * NT_V_BYTES;
+                const int n16 = (NT_KC - nvalid) * 8;  // 16-byte pieces of the tail rows per 64-dim box
+                for (int t = lane; t < 2 * n16; t += 32) {
+                    const int box = t / n16, piece = t - box * n16;
+                    *reinterpret_cast<uint4 *>(dv + box * (NT_V_BYTES / 2) + nvalid * 128 + piece * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+            }
+            if (lane == 0) tc::mbar_arrive(bar(cs->v_ready[s]));
+        }
     } else if (warp == 1 && lane == 0) {
         auto issue_pv = [&](int c) {
             const int s = c % NT_KST, b = c & 1;
             if (!tc::wait_bounded_sleep(bar(cs->pv_ready), (uint32_t)(c & 1), wl, abort, err)) return false;
             if (!tc::wait_bounded_sleep(bar(cs->v_full[s]), (uint32_t)((c / NT_KST) & 1), wl, abort, err)) return false;
+            if (!tc::wait_bounded_sleep(bar(cs->v_ready[s]), (uint32_t)((c / NT_KST) & 1), wl, abort, err)) return false;
             tc::fence_after();
             // P from the first 32 columns of score buffer b (16 keys = 8 columns per
             // instruction); the V chunk as the MN-major B operand: 64-dim halves

@@ -470,6 +470,30 @@ def test_attention_near_tiles_against_oracle(tiny, hq, hkv, p0, nq):
     PT.assert_attention_close(Od, Oref, lse, lse_ref)
 
 
+@pytest.mark.parametrize("hq,hkv,p0,nq", [(32, 8, 1000, 300), (16, 16, 0, 130)])
+def test_attention_near_tiles_ignore_rows_past_the_queries(tiny, hq, hkv, p0, nq):
+    """K and V rows past the last query position (not in any list) hold NaN,
+    as an unwritten cache tail may: the near-set tiles load whole 64-key
+    boxes, so their partial last chunk must keep those rows out of O."""
+    _need_gpu()
+    keys, q, pos, oc = tiny
+    sel = np.arange(p0, p0 + nq, dtype=np.int64)
+    ol, on = O.index(q[sel], pos[sel], oc, k=256)
+    Qb, Kb, Vb = I.qkv_bf16_bits(11, nq, 4096, hq, hkv)
+    Oref, lse_ref = O.attention(Qb, Kb, Vb, ol, on)
+    Kb, Vb = Kb.copy(), Vb.copy()
+    Kb[p0 + nq:] = 0x7FC0  # bf16 NaN
+    Vb[p0 + nq:] = 0x7FC0
+    Qd, Kd, Vd = PT.bits_to_bf16(Qb), PT.bits_to_bf16(Kb), PT.bits_to_bf16(Vb)
+    Od = torch.empty_like(Qd)
+    lse = torch.empty((nq, hq), dtype=torch.float32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_attention_workspace_bytes(nq, hq, 128, ol.shape[1]))
+    lsa.lsa_sparse_attention(Qd, Kd, Vd, PT.to_dev(ol), PT.to_dev(on), Od, lse, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(Od.float()).all()
+    PT.assert_attention_close(Od, Oref, lse, lse_ref)
+
+
 def test_attention_near_tiles_irregular_lists(tiny):
     """Lists without a window (random subsets ending at the query's position),
     and a batch whose positions jump inside a tile: the near-set plan must
