@@ -227,7 +227,7 @@ def _rl(kernel, bound, work, ms, launches, peak, unit, note, **extra):
 
 
 def kernel_rooflines(kt: dict, wl: dict, mode: str, pos_np, lens_np, far_rows: int, near_ms_total: float, pk,
-                     steps: int):
+                     steps: int, near_rows: int = 0):
     """Per-kernel rooflines of one mode's timed steps from the library's
     per-kernel events (kt: name -> (ms summed over the steps, launches))."""
     T, hq, hkv = wl["T"], wl["hq"], wl["hkv"]
@@ -272,8 +272,14 @@ def kernel_rooflines(kt: dict, wl: dict, mode: str, pos_np, lens_np, far_rows: i
             o["traffic"] = None
         o["unique_kv_bytes"] = int(T * hkv * 512)
         if near_ms_total > 0:
-            o["near"] = {"kernels": "k_near_plan + k_attn_near", "ms": round(near_ms_total / steps, 3)}
+            o["near"] = {"kernels": "k_near_plan + k_attn_near_tc", "ms": round(near_ms_total / steps, 3)}
         out["k_attn"] = o
+    if "k_attn_near_tc" in kt and near_rows > 0:
+        ms, n = kt["k_attn_near_tc"]
+        out["k_attn_near_tc"] = _rl("k_attn_near_tc", "tensor", 512.0 * hq * near_rows * steps, ms, n, pk["bf16_sust"],
+                                    "TFLOP/s", "512 flop per (query head, near key) the tiles take (score + P V); a "
+                                    "tile computes its rows over the union of its queries' near keys, masked, so "
+                                    "the tensor pipe does more than this; peak = sustained bf16")
     for name in ("k_ward", "k_tree_leaves", "k_tree_pair", "k_tree_beam", "k_qnorm", "k_tau"):
         if name in kt:
             ms, n = kt[name]
@@ -338,13 +344,14 @@ def mode_summary(args, wl, mode, layer, per, kt, world, pk):
     nq = wl["n_prefill"]
     total_ms = max_over_ranks(float(per[:, 3].sum()), world)
     lens_np = layer.lens[:nq].cpu().numpy()
-    near_ms = sum(kt[k][0] for k in ("k_near_plan", "k_attn_near") if k in kt)
+    near_ms = sum(kt[k][0] for k in ("k_near_plan", "k_attn_near_tc") if k in kt)
+    near_rows = 0
     if near_ms > 0:
-        _, far_rows = near_split_rows(layer.lists[:nq], layer.lens[:nq])
+        near_rows, far_rows = near_split_rows(layer.lists[:nq], layer.lens[:nq])
     else:
         far_rows = int(lens_np.astype(np.int64).sum())
     pos_np = np.arange(wl["T"] - nq, wl["T"], dtype=np.int64)
-    kr = kernel_rooflines(kt, wl, mode, pos_np, lens_np, far_rows, near_ms, pk, args.steps)
+    kr = kernel_rooflines(kt, wl, mode, pos_np, lens_np, far_rows, near_ms, pk, args.steps, near_rows)
     return {
         "mode": mode, "value": round(world * nq * args.steps / (total_ms / 1e3), 1), "unit": UNIT,
         "ms_per_step": round(total_ms / args.steps, 3),

@@ -734,7 +734,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st, int n_sm)
         int kt = kt_begin("k_near_plan", st);
         k_near_plan<<<tiles, NEAR_ROWS, 0, st>>>(a);
         kt_end(kt, st);
-        kt = kt_begin("k_attn_near", st);
+        kt = kt_begin("k_attn_near_tc", st);
         e = launch_attention_near_tc(a, (int)tiles, st);
         kt_end(kt, st);
         if (e != cudaSuccess) return e;
