@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_and_barrier_gloo():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of a threaded process
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert dict(out) == {0: 11.0, 1: 11.0}
 
@@ -167,7 +167,7 @@ def test_context_parallel_exchanges_gloo():
     """Every rank receives every rank's member slice, exchange block and
     attention part, in rank order, and computes the same list."""
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of a threaded process
     mp.spawn(_cp_worker, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
         d = out[r]
