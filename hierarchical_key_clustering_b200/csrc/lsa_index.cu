@@ -59,9 +59,10 @@ __global__ void __launch_bounds__(256) k_qnorm(const float *__restrict__ qidx, c
 }
 
 // Score of one bucket on the CUDA cores: fp32 FMA chain over d = 0..63 of the
-// bf16 operands (k_fallback).  It can differ from the tensor cores' sum of
-// the same products in the last bit, which only matters for scores within
-// ~1e-6 of each other, at the one cut a Flat search makes.
+// bf16 operands (the exact selections of a query whose candidates overflowed
+// or whose sampled threshold kept too little).  It can differ from the tensor
+// cores' sum of the same products in the last bit, which only matters for
+// scores within ~1e-6 of each other, at the one cut a Flat search makes.
 __device__ __forceinline__ float dot_bf16_row(const float *qf, const uint16_t *__restrict__ c)
 {
     const uint4 *c4 = reinterpret_cast<const uint4 *>(c);
