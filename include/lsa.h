@@ -326,7 +326,9 @@ int lsa_index_decode(const float *qidx, const int64_t *pos, int64_t nq, const ls
  * Q bf16 [nq, Hq, 128]; K, V bf16 [Tk, Hkv, 128]; query head h reads KV head
  * h / (Hq / Hkv) (Hq a multiple of Hkv, Hq / Hkv <= 16).  lists/lens as
  * written by lsa_index_*: each list strictly increasing, every listed
- * position < Tk.
+ * position < Tk.  Rows of K and V that no list holds may hold anything
+ * (an unwritten cache tail, NaN included): the results depend on listed
+ * rows only.
  * O[i,h] = sum_j softmax_j(scale * Q[i,h] . K[j]) V[j] over j in list(i),
  * fp32 softmax and accumulation; O bf16 [nq, Hq, 128]; lse fp32 [nq, Hq]
  * (natural-log log-sum-exp of the scaled scores; may be NULL).
